@@ -1,0 +1,306 @@
+"""Python binding of libgpt2.so: one GPT-2 pretraining step on one B200.
+
+Argument marshalling only.  Every step of the path runs in the library's
+CUDA kernels; PyTorch provides device memory and streams.  The library is
+loaded on first use; a RuntimeError is raised if it has not been built (``python -m decoder_only_transformer_step_b200.build_lib``):
+there is no CPU fallback.
+
+Functions named like the C entry points take torch tensors (device memory)
+and ints/floats; ``GPT2`` bundles the buffers a context needs.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgpt2.so")
+
+GPT2_OK = 0
+ERRORS = {
+    -1: "GPT2_ERR_INVALID_ARG", -2: "GPT2_ERR_UNSUPPORTED_SHAPE", -3: "GPT2_ERR_CUDA",
+    -4: "GPT2_ERR_BAD_STATE", -5: "GPT2_ERR_TOKEN_RANGE", -6: "GPT2_ERR_NONFINITE",
+    -7: "GPT2_ERR_TIMEOUT", -8: "GPT2_ERR_WORKSPACE",
+}
+
+
+class Gpt2Error(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {ERRORS.get(code, code)} ({_lib().gpt2_strerror(code).decode()})")
+        self.code = code
+
+
+class gpt2_config(ctypes.Structure):
+    _fields_ = [("n_layer", ctypes.c_int), ("d_model", ctypes.c_int), ("n_head", ctypes.c_int),
+                ("n_ctx", ctypes.c_int), ("vocab_real", ctypes.c_int), ("vocab_padded", ctypes.c_int),
+                ("max_batch", ctypes.c_int), ("mode", ctypes.c_int)]
+
+
+class gpt2_buffers(ctypes.Structure):
+    _fields_ = [("master", ctypes.c_void_p), ("shadow", ctypes.c_void_p), ("grad", ctypes.c_void_p),
+                ("m", ctypes.c_void_p), ("v", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+EXPORTS = [
+    "gpt2_param_count", "gpt2_workspace_bytes", "gpt2_tensor_info", "gpt2_create", "gpt2_destroy",
+    "gpt2_init_params", "gpt2_refresh_shadow", "gpt2_forward_loss", "gpt2_backward",
+    "gpt2_adamw_step", "gpt2_zero_grad", "gpt2_get_status", "gpt2_step_host", "gpt2_strerror",
+    "gpt2_op_gemm_bf16", "gpt2_op_attention_fwd_bf16", "gpt2_op_attention_bwd_bf16",
+]
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m decoder_only_transformer_step_b200.build_lib`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, F, S, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
+    cfgp = ctypes.POINTER(gpt2_config)
+    sig = {
+        "gpt2_param_count": (S, [cfgp]),
+        "gpt2_workspace_bytes": (S, [cfgp, I]),
+        "gpt2_tensor_info": (I, [cfgp, I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(S),
+                                 ctypes.POINTER(S), ctypes.POINTER(S)]),
+        "gpt2_create": (I, [cfgp, ctypes.POINTER(gpt2_buffers), ctypes.POINTER(P)]),
+        "gpt2_destroy": (I, [P]),
+        "gpt2_init_params": (I, [P, U64, P]),
+        "gpt2_refresh_shadow": (I, [P, P]),
+        "gpt2_forward_loss": (I, [P, P, P, I, P, P]),
+        "gpt2_backward": (I, [P, F, I, P]),
+        "gpt2_adamw_step": (I, [P, F, F, F, F, F, I, P]),
+        "gpt2_zero_grad": (I, [P, P]),
+        "gpt2_get_status": (I, [P, P]),
+        "gpt2_step_host": (I, [P, P, P, I, P, F, F, F, F, F, I, P]),
+        "gpt2_strerror": (ctypes.c_char_p, [I]),
+        "gpt2_op_gemm_bf16": (I, [P, I, I, P, I, I, P, I, I, I, I, I, F, F, P, S, I, I, P]),
+        "gpt2_op_attention_fwd_bf16": (I, [P, P, P, I, I, I, I, P]),
+        "gpt2_op_attention_bwd_bf16": (I, [P, P, P, P, P, P, I, I, I, I, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _LIB = L
+    return L
+
+
+def _check(rc: int, where: str):
+    if rc != GPT2_OK:
+        raise Gpt2Error(rc, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# --------------------------------------------------------------- C names ---
+
+def make_config(n_layer, d_model, n_head, n_ctx, vocab_real, vocab_padded, max_batch, mode=0):
+    return gpt2_config(n_layer, d_model, n_head, n_ctx, vocab_real, vocab_padded, max_batch, mode)
+
+
+def gpt2_param_count(cfg: gpt2_config) -> int:
+    return int(_lib().gpt2_param_count(ctypes.byref(cfg)))
+
+
+def gpt2_workspace_bytes(cfg: gpt2_config, batch: int) -> int:
+    return int(_lib().gpt2_workspace_bytes(ctypes.byref(cfg), batch))
+
+
+def gpt2_tensor_info(cfg: gpt2_config, index: int):
+    """(name, offset, rows, cols) or None past the last tensor."""
+    name = ctypes.c_char_p()
+    off, r, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    rc = _lib().gpt2_tensor_info(ctypes.byref(cfg), index, ctypes.byref(name), ctypes.byref(off),
+                                 ctypes.byref(r), ctypes.byref(c))
+    if rc != GPT2_OK:
+        return None
+    return name.value.decode(), off.value, r.value, c.value
+
+
+def gpt2_tensors(cfg: gpt2_config):
+    out, i = [], 0
+    while True:
+        t = gpt2_tensor_info(cfg, i)
+        if t is None:
+            return out
+        out.append(t)
+        i += 1
+
+
+def gpt2_create(cfg, master, shadow, grad, m, v, workspace):
+    bufs = gpt2_buffers(master.data_ptr(), shadow.data_ptr() if shadow is not None else None,
+                        grad.data_ptr(), m.data_ptr(), v.data_ptr(), workspace.data_ptr(),
+                        workspace.numel() * workspace.element_size())
+    ctx = ctypes.c_void_p()
+    _check(_lib().gpt2_create(ctypes.byref(cfg), ctypes.byref(bufs), ctypes.byref(ctx)), "gpt2_create")
+    return ctx
+
+
+def gpt2_destroy(ctx):
+    _check(_lib().gpt2_destroy(ctx), "gpt2_destroy")
+
+
+def gpt2_init_params(ctx, seed: int, stream=None):
+    _check(_lib().gpt2_init_params(ctx, seed, _stream(stream)), "gpt2_init_params")
+
+
+def gpt2_refresh_shadow(ctx, stream=None):
+    _check(_lib().gpt2_refresh_shadow(ctx, _stream(stream)), "gpt2_refresh_shadow")
+
+
+def gpt2_forward_loss(ctx, tokens, targets, batch: int, loss_dev, stream=None):
+    _check(_lib().gpt2_forward_loss(ctx, _ptr(tokens), _ptr(targets), batch, _ptr(loss_dev),
+                                    _stream(stream)), "gpt2_forward_loss")
+
+
+def gpt2_backward(ctx, grad_scale: float = 1.0, accumulate: int = 0, stream=None):
+    _check(_lib().gpt2_backward(ctx, grad_scale, accumulate, _stream(stream)), "gpt2_backward")
+
+
+def gpt2_adamw_step(ctx, lr, beta1, beta2, eps, weight_decay, step, stream=None):
+    _check(_lib().gpt2_adamw_step(ctx, lr, beta1, beta2, eps, weight_decay, step, _stream(stream)),
+           "gpt2_adamw_step")
+
+
+def gpt2_zero_grad(ctx, stream=None):
+    _check(_lib().gpt2_zero_grad(ctx, _stream(stream)), "gpt2_zero_grad")
+
+
+def gpt2_get_status(ctx, stream=None) -> int:
+    return int(_lib().gpt2_get_status(ctx, _stream(stream)))
+
+
+def gpt2_step_host(ctx, tokens_host, targets_host, batch, loss_host, lr, beta1, beta2, eps,
+                   weight_decay, step, stream=None):
+    """tokens_host/targets_host/loss_host: CPU (ideally pinned) torch tensors."""
+    _check(_lib().gpt2_step_host(ctx, _ptr(tokens_host), _ptr(targets_host), batch, _ptr(loss_host),
+                                 lr, beta1, beta2, eps, weight_decay, step, _stream(stream)),
+           "gpt2_step_host")
+
+
+def gpt2_op_gemm_bf16(A, a_mn_major, lda, B, b_mn_major, ldb, C, c_fp32, ldc, M, N, K,
+                      alpha=1.0, beta=0.0, workspace=None, bn=0, splits=0, stream=None):
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib().gpt2_op_gemm_bf16(_ptr(A), a_mn_major, lda, _ptr(B), b_mn_major, ldb, _ptr(C), c_fp32,
+                                    ldc, M, N, K, alpha, beta, _ptr(workspace), wsb, bn, splits,
+                                    _stream(stream)), "gpt2_op_gemm_bf16")
+
+
+def gpt2_op_attention_fwd_bf16(qkv, o, lse, B, T, H, hd, stream=None):
+    _check(_lib().gpt2_op_attention_fwd_bf16(_ptr(qkv), _ptr(o), _ptr(lse), B, T, H, hd,
+                                             _stream(stream)), "gpt2_op_attention_fwd_bf16")
+
+
+def gpt2_op_attention_bwd_bf16(qkv, o, lse, dout, dqkv, scratch, B, T, H, hd, stream=None):
+    _check(_lib().gpt2_op_attention_bwd_bf16(_ptr(qkv), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dqkv),
+                                             _ptr(scratch), B, T, H, hd, _stream(stream)),
+           "gpt2_op_attention_bwd_bf16")
+
+
+# ------------------------------------------------------------ convenience ---
+
+@dataclass(frozen=True)
+class ModelConfig:
+    n_layer: int
+    d_model: int
+    n_head: int
+    n_ctx: int
+    vocab_real: int
+    vocab_padded: int
+    max_batch: int
+    mode: int = 0  # 0 bf16 tensor cores, 1 fp32 correctness mode
+
+    def c(self) -> gpt2_config:
+        return make_config(self.n_layer, self.d_model, self.n_head, self.n_ctx, self.vocab_real,
+                           self.vocab_padded, self.max_batch, self.mode)
+
+
+GPT2_124M = ModelConfig(12, 768, 12, 1024, 50257, 50304, 16)
+GPT2_350M = ModelConfig(24, 1024, 16, 1024, 50257, 50304, 16)
+GPT2_1558M = ModelConfig(48, 1600, 25, 1024, 50257, 50304, 8)
+GPT2_124M_T4096 = ModelConfig(12, 768, 12, 4096, 50257, 50304, 4)
+GPT2_TINY = ModelConfig(2, 64, 4, 64, 512, 512, 4, mode=1)
+
+
+class GPT2:
+    """A context plus the torch-owned device buffers it runs on."""
+
+    def __init__(self, mc: ModelConfig, device="cuda"):
+        import torch
+        self.mc = mc
+        self.cfg = mc.c()
+        n = gpt2_param_count(self.cfg)
+        if n == 0:
+            raise ValueError(f"invalid config {mc}")
+        self.n_params = n
+        f32 = dict(dtype=torch.float32, device=device)
+        self.master = torch.zeros(n, **f32)
+        self.grad = torch.zeros(n, **f32)
+        self.m = torch.zeros(n, **f32)
+        self.v = torch.zeros(n, **f32)
+        self.shadow = torch.zeros(n, dtype=torch.bfloat16, device=device)
+        wsb = gpt2_workspace_bytes(self.cfg, mc.max_batch)
+        self.workspace = torch.empty(wsb, dtype=torch.uint8, device=device)
+        self.loss = torch.zeros(1, **f32)
+        self.ctx = gpt2_create(self.cfg, self.master, self.shadow, self.grad, self.m, self.v, self.workspace)
+        self.layout = gpt2_tensors(self.cfg)
+
+    def close(self):
+        if self.ctx is not None:
+            gpt2_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def view(self, flat, name):
+        """View of one named tensor inside a flat buffer (master, grad, m, v)."""
+        for nm, off, r, c in self.layout:
+            if nm == name:
+                t = flat[off:off + r * c]
+                return t.view(r, c) if c > 1 else t
+        raise KeyError(name)
+
+    def init_params(self, seed=0):
+        gpt2_init_params(self.ctx, seed)
+
+    def refresh_shadow(self):
+        gpt2_refresh_shadow(self.ctx)
+
+    def forward_loss(self, tokens, targets):
+        gpt2_forward_loss(self.ctx, tokens, targets, tokens.shape[0], self.loss)
+        return self.loss
+
+    def backward(self, grad_scale=1.0, accumulate=0):
+        gpt2_backward(self.ctx, grad_scale, accumulate)
+
+    def adamw_step(self, step, lr=6e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1):
+        gpt2_adamw_step(self.ctx, lr, beta1, beta2, eps, weight_decay, step)
+
+    def zero_grad(self):
+        gpt2_zero_grad(self.ctx)
+
+    def status(self) -> int:
+        return gpt2_get_status(self.ctx)
+
+    def step_host(self, tokens_host, targets_host, loss_host, step, lr=6e-4, beta1=0.9, beta2=0.95,
+                  eps=1e-8, weight_decay=0.1):
+        gpt2_step_host(self.ctx, tokens_host, targets_host, tokens_host.shape[0], loss_host, lr, beta1,
+                       beta2, eps, weight_decay, step)

@@ -1,0 +1,223 @@
+// Shared device helpers: types, conversions, warp reductions, bounded waits,
+// and thin inline-PTX wrappers for the sm_100a asynchronous machinery
+// (mbarrier, TMA bulk tensor copies, tcgen05 tensor-memory MMA).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/gpt2.h"
+
+typedef __nv_bfloat16 bf16;
+
+// Bits of the device status word (latched until gpt2_get_status reads it).
+enum : int {
+  DEV_ERR_TOKEN = 1,
+  DEV_ERR_NONFINITE = 2,
+  DEV_ERR_TIMEOUT = 4,
+};
+
+// A pipeline wait that has not completed after this long is treated as a
+// hang: the kernel records DEV_ERR_TIMEOUT and leaves the wait.
+#define WAIT_TIMEOUT_NS 2000000000ull
+
+#define DEVI __device__ __forceinline__
+
+// ------------------------------------------------------------ conversions --
+
+template <typename T> DEVI float to_f(T x);
+template <> DEVI float to_f<float>(float x) { return x; }
+template <> DEVI float to_f<bf16>(bf16 x) { return __bfloat162float(x); }
+
+template <typename T> DEVI T from_f(float x);
+template <> DEVI float from_f<float>(float x) { return x; }
+template <> DEVI bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
+
+DEVI uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+DEVI float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+DEVI float bf16hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// ------------------------------------------------------------- reductions --
+
+DEVI float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+DEVI float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// ------------------------------------------------------------------ GELU --
+// tanh form: 0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))).
+#define GELU_K0 0.7978845608028654f
+#define GELU_K1 0.044715f
+
+DEVI float tanh_fast(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+template <bool FAST> DEVI float gelu_f(float u) {
+  float t = GELU_K0 * (u + GELU_K1 * u * u * u);
+  float th = FAST ? tanh_fast(t) : tanhf(t);
+  return 0.5f * u * (1.f + th);
+}
+template <bool FAST> DEVI float dgelu_f(float u) {
+  float t = GELU_K0 * (u + GELU_K1 * u * u * u);
+  float th = FAST ? tanh_fast(t) : tanhf(t);
+  return 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * GELU_K0 * (1.f + 3.f * GELU_K1 * u * u);
+}
+
+// ------------------------------------------------------------ shared mem --
+
+DEVI uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+DEVI uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// --------------------------------------------------------------- mbarrier --
+
+DEVI void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+DEVI void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+DEVI void mbar_arrive(uint32_t bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
+               : "memory");
+}
+DEVI void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+                   bar),
+               "r"(bytes)
+               : "memory");
+}
+DEVI bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false (after raising the
+// shared abort flag and the device timeout bit) if the phase did not complete
+// within WAIT_TIMEOUT_NS, or if another role of the CTA already aborted.
+DEVI bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                            int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = globaltimer();
+  uint32_t spins = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if ((++spins & 63u) == 0 && globaltimer() - t0 > WAIT_TIMEOUT_NS) {
+      *abort_flag = 1;
+      if (err) atomicOr(err, DEV_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Wait that ignores the abort flag (used only while draining in-flight async
+// copies before exit); still bounded in time.
+DEVI void mbar_drain_bounded(uint32_t bar, uint32_t parity) {
+  uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > WAIT_TIMEOUT_NS) return;
+  }
+}
+
+// -------------------------------------------------------------------- TMA --
+
+DEVI void tma_prefetch_desc(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+// 2-D tiled bulk tensor load global -> shared, completing on an mbarrier.
+// c0 is the innermost (contiguous) coordinate in elements.
+DEVI void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// ---------------------------------------------------------------- tcgen05 --
+
+DEVI void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+DEVI void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Whole-warp collective: allocate `ncols` TMEM columns, address written to smem.
+DEVI void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+DEVI void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 inputs, fp32 accum).
+DEVI void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                      uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on an mbarrier once all previously issued tcgen05.mma of this thread complete.
+DEVI void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// 32 lanes x 32 columns of fp32 from TMEM: thread i of the warp gets lane
+// (base lane + i), columns [col, col+32).
+DEVI void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+DEVI void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ------------------------------------------------------------ host checks --
+
+#define CUDA_TRY(expr)                                   \
+  do {                                                   \
+    cudaError_t e_ = (expr);                             \
+    if (e_ != cudaSuccess) return GPT2_ERR_CUDA;         \
+  } while (0)
+
+#define LAUNCH_CHECK() CUDA_TRY(cudaGetLastError())

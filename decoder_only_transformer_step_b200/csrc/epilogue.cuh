@@ -1,0 +1,137 @@
+// GEMM epilogues: the bias, residual, GELU and GELU' steps of a decoder block
+// fused into the store of the matmul result, plus the fp32 weight-gradient
+// store (beta * old + alpha * acc).
+#pragma once
+
+#include "common.cuh"
+#include "internal.h"
+
+// One element (used by the CUDA-core GEMM and by ragged tile edges).
+template <typename T>
+DEVI void epi_one(const EpiArgs& e, float* partial, int split, int M, int N, int row, int col,
+                  float v) {
+  constexpr bool FAST = sizeof(T) == 2;
+  const long idx = (long)row * e.ldo + col;
+  switch (e.kind) {
+    case EPI_STORE:
+      ((T*)e.out)[idx] = from_f<T>(e.alpha * v);
+      break;
+    case EPI_BIAS:
+      ((T*)e.out)[idx] = from_f<T>(v + to_f(((const T*)e.bias)[col]));
+      break;
+    case EPI_BIAS_RESID:
+      ((T*)e.out)[idx] =
+          from_f<T>(v + to_f(((const T*)e.bias)[col]) + to_f(((const T*)e.resid)[idx]));
+      break;
+    case EPI_BIAS_GELU: {
+      float u = v + to_f(((const T*)e.bias)[col]);
+      ((T*)e.out)[idx] = from_f<T>(u);
+      ((T*)e.out2)[idx] = from_f<T>(gelu_f<FAST>(u));
+      break;
+    }
+    case EPI_DGELU:
+      ((T*)e.out)[idx] = from_f<T>(v * dgelu_f<FAST>(to_f(((const T*)e.aux)[idx])));
+      break;
+    case EPI_F32: {
+      float* o = (float*)e.out;
+      o[idx] = (e.beta != 0.f ? e.beta * o[idx] : 0.f) + e.alpha * v;
+      break;
+    }
+    case EPI_F32_PARTIAL:
+      partial[((long)split * M + row) * N + col] = v;
+      break;
+  }
+}
+
+// ---- 32 consecutive bf16 columns of one row, 16-byte vector accesses ----
+
+DEVI void ld_bf16x32(const bf16* p, float (&f)[32]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 u = q[i];
+    f[8 * i + 0] = bf16lo(u.x); f[8 * i + 1] = bf16hi(u.x);
+    f[8 * i + 2] = bf16lo(u.y); f[8 * i + 3] = bf16hi(u.y);
+    f[8 * i + 4] = bf16lo(u.z); f[8 * i + 5] = bf16hi(u.z);
+    f[8 * i + 6] = bf16lo(u.w); f[8 * i + 7] = bf16hi(u.w);
+  }
+}
+DEVI void st_bf16x32(bf16* p, const float (&f)[32]) {
+  uint4* q = reinterpret_cast<uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 u;
+    u.x = pack_bf16x2(f[8 * i + 0], f[8 * i + 1]);
+    u.y = pack_bf16x2(f[8 * i + 2], f[8 * i + 3]);
+    u.z = pack_bf16x2(f[8 * i + 4], f[8 * i + 5]);
+    u.w = pack_bf16x2(f[8 * i + 6], f[8 * i + 7]);
+    q[i] = u;
+  }
+}
+
+// Full chunk: row < M and col0 + 32 <= N, all row pitches multiples of 8.
+DEVI void epi_row32_bf16(const EpiArgs& e, float* partial, int split, int M, int N, int row,
+                         int col0, float (&v)[32]) {
+  const long idx = (long)row * e.ldo + col0;
+  float t[32];
+  switch (e.kind) {
+    case EPI_STORE:
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= e.alpha;
+      st_bf16x32((bf16*)e.out + idx, v);
+      break;
+    case EPI_BIAS:
+      ld_bf16x32((const bf16*)e.bias + col0, t);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += t[j];
+      st_bf16x32((bf16*)e.out + idx, v);
+      break;
+    case EPI_BIAS_RESID:
+      ld_bf16x32((const bf16*)e.bias + col0, t);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += t[j];
+      ld_bf16x32((const bf16*)e.resid + idx, t);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += t[j];
+      st_bf16x32((bf16*)e.out + idx, v);
+      break;
+    case EPI_BIAS_GELU:
+      ld_bf16x32((const bf16*)e.bias + col0, t);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += t[j];
+      st_bf16x32((bf16*)e.out + idx, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = gelu_f<true>(v[j]);
+      st_bf16x32((bf16*)e.out2 + idx, v);
+      break;
+    case EPI_DGELU:
+      ld_bf16x32((const bf16*)e.aux + idx, t);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= dgelu_f<true>(t[j]);
+      st_bf16x32((bf16*)e.out + idx, v);
+      break;
+    case EPI_F32: {
+      float4* o = reinterpret_cast<float4*>((float*)e.out + idx);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (e.beta != 0.f) {
+          r = o[i];
+          r.x *= e.beta; r.y *= e.beta; r.z *= e.beta; r.w *= e.beta;
+        }
+        r.x += e.alpha * v[4 * i + 0];
+        r.y += e.alpha * v[4 * i + 1];
+        r.z += e.alpha * v[4 * i + 2];
+        r.w += e.alpha * v[4 * i + 3];
+        o[i] = r;
+      }
+      break;
+    }
+    case EPI_F32_PARTIAL: {
+      float4* o = reinterpret_cast<float4*>(partial + ((long)split * M + row) * N + col0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      break;
+    }
+  }
+}

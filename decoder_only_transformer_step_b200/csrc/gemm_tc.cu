@@ -1,0 +1,421 @@
+// tcgen05 GEMM for sm_100a: the linear layers of the decoder (QKV, attention
+// output, MLP fc / proj, tied LM head) and their input- and weight-gradient
+// products.  "Pré-treinar um LLM" (compute section) counts each of these as one
+// matmul of the forward and two of the same size in the backward; all of them
+// are C = A B^T with A and B either K-major or MN-major, which is what this
+// kernel takes, so no operand is ever transposed in memory.
+//
+// Design (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: 128B-swizzled tiles of A (128 x 64) and B
+//               (BN x 64) into a STAGES-deep shared-memory ring (mbarriers).
+//   warp 1      allocates TMEM and issues tcgen05.mma (M=128, N=BN, K=16)
+//               from one thread; tcgen05.commit frees each ring slot and
+//               signals a finished accumulator.
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (each warp owns
+//               the 32 TMEM lanes = tile rows its warp index allows), fused
+//               bias / residual / GELU / GELU' / fp32-gradient stores.
+// The accumulator is double-buffered in TMEM (2 x BN columns), so the
+// epilogue of tile i overlaps the main loop of tile i+1.  Weight gradients
+// with few output tiles are split along K; partial sums go to a workspace and
+// a deterministic reduction adds them in split order.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "internal.h"
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;               // one 128-byte swizzle row of bf16
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t MN_ATOM_BYTES = 64 * BK * 2;  // one {64 MN x 64 K} TMA box
+
+template <int BN>
+struct TcCfg {
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int NUM_BARS = 2 * STAGES + 5;  // full, empty, acc_full[2], acc_empty[2], drain
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
+};
+
+struct TcParams {
+  int M, N, K;
+  int a_mn, b_mn;
+  int m_tiles, n_tiles, splits, kb_total;
+  uint32_t idesc;
+  EpiArgs epi;
+  float* partial;
+  int* err;
+};
+
+// Shared-memory matrix descriptor (tcgen05), 128-byte swizzle, sm_100 version 1.
+DEVI uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// K-major tile (rows of 64 k = 128 B, 8-row groups 1024 B apart): the k-th
+// 16-wide slice starts 32 B further inside the swizzle row.
+// MN-major tile ({64 mn x 64 k} boxes 8 KB apart, k rows 128 B apart): the
+// k-th 16-row slice starts 2 KB further.
+DEVI uint64_t operand_desc(uint32_t tile, int mn_major, int k) {
+  return mn_major ? sdesc(tile + k * 2048, MN_ATOM_BYTES, 1024) : sdesc(tile + k * 32, 16, 1024);
+}
+
+// Work unit u -> (m tile origin, n tile index, split index, k-block range).
+// m varies fastest, so consecutive CTAs share the B tile (weights) in L2.
+DEVI void decode_unit(const TcParams& p, int u, int& m0, int& nt, int& s, int& kb0, int& kb1) {
+  const int mt = u % p.m_tiles;
+  const int rest = u / p.m_tiles;
+  nt = rest % p.n_tiles;
+  s = rest / p.n_tiles;
+  m0 = mt * BM;
+  kb0 = (int)((long long)s * p.kb_total / p.splits);
+  kb1 = (int)((long long)(s + 1) * p.kb_total / p.splits);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const TcParams p) {
+  using C = TcCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t tiles = (raw + 1023u) & ~1023u;
+  uint8_t* tiles_ptr = smem_raw + (tiles - raw);
+  const uint32_t bars = tiles + C::STAGES * C::STAGE_BYTES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tiles_ptr + C::STAGES * C::STAGE_BYTES + C::NUM_BARS * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (C::STAGES + s); };
+  auto accf_bar = [&](int b) { return bars + 8u * (2 * C::STAGES + b); };
+  auto acce_bar = [&](int b) { return bars + 8u * (2 * C::STAGES + 2 + b); };
+  const uint32_t drain_bar = bars + 8u * (2 * C::STAGES + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int units = p.m_tiles * p.n_tiles * p.splits;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer ----
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int m0, nt, s, kb0, kb1;
+        decode_unit(p, u, m0, nt, s, kb0, kb1);
+        const int n0 = nt * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full_bar(stage);
+          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          const uint32_t sa = tiles + stage * C::STAGE_BYTES;
+          const uint32_t sb = sa + C::A_BYTES;
+          if (!p.a_mn) {
+            tma_load_2d(sa, &tmA, fb, kb * BK, m0);
+          } else {
+            tma_load_2d(sa, &tmA, fb, m0, kb * BK);
+            tma_load_2d(sa + MN_ATOM_BYTES, &tmA, fb, m0 + 64, kb * BK);
+          }
+          if (!p.b_mn) {
+            tma_load_2d(sb, &tmB, fb, kb * BK, n0);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * MN_ATOM_BYTES, &tmB, fb, n0 + 64 * j, kb * BK);
+          }
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the copies already in flight land before the CTA exits.
+        int n = issued < C::STAGES ? issued : C::STAGES;
+        for (int i = 1; i <= n; ++i) {
+          int s2 = (stage - i + C::STAGES) % C::STAGES;
+          uint32_t par = s2 < stage ? phase : (phase ^ 1u);
+          mbar_drain_bounded(full_bar(s2), par);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------- MMA issuer ----
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++it) {
+        int m0, nt, s, kb0, kb1;
+        decode_unit(p, u, m0, nt, s, kb0, kb1);
+        const int buf = it & 1;
+        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait_bounded(acce_bar(buf), aph ^ 1u, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = tiles + stage * C::STAGE_BYTES;
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            tc_mma_bf16(d_tmem, operand_desc(sa, p.a_mn, k), operand_desc(sb, p.b_mn, k), p.idesc,
+                        (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          issued_any = true;
+          tc_commit(empty_bar(stage));
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(accf_bar(buf));
+      }
+      if (!ok && issued_any) {
+        // Wait (bounded) for the MMAs already issued before TMEM is freed.
+        tc_commit(drain_bar);
+        mbar_drain_bounded(drain_bar, 0);
+      }
+    }
+  } else {
+    // ---------------------------------------------------- epilogue ----
+    const int q = warp & 3;  // TMEM lanes [32q, 32q+32) are this warp's
+    int it = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+      int m0, nt, s, kb0, kb1;
+      decode_unit(p, u, m0, nt, s, kb0, kb1);
+      const int n0 = nt * BN;
+      const int buf = it & 1;
+      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      if (!mbar_wait_bounded(accf_bar(buf), aph, abort_flag, p.err)) break;
+      tc_fence_after();
+      const int row = m0 + q * 32 + lane;
+      for (int c = 0; c < BN; c += 32) {
+        if (n0 + c >= p.N) break;  // warp-uniform
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c), r);
+        tmem_ld_wait();
+        if (row < p.M) {
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          const int col0 = n0 + c;
+          if (col0 + 32 <= p.N) {
+            epi_row32_bf16(p.epi, p.partial, s, p.M, p.N, row, col0, v);
+          } else {
+            for (int j = 0; j < 32 && col0 + j < p.N; ++j)
+              epi_one<bf16>(p.epi, p.partial, s, p.M, p.N, row, col0 + j, v[j]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acce_bar(buf));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// out = beta*out + alpha * sum_s part[s]   (fixed order over s)
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, long mn,
+                                     float* __restrict__ out, float alpha, float beta) {
+  long i = (blockIdx.x * (long)blockDim.x + threadIdx.x) * 4;
+  if (i >= mn) return;
+  if (i + 4 <= mn) {
+    float4 acc = reinterpret_cast<const float4*>(part + i)[0];
+    for (int s = 1; s < splits; ++s) {
+      float4 t = reinterpret_cast<const float4*>(part + (long)s * mn + i)[0];
+      acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
+    }
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (beta != 0.f) {
+      o = reinterpret_cast<float4*>(out + i)[0];
+      o.x *= beta; o.y *= beta; o.z *= beta; o.w *= beta;
+    }
+    o.x += alpha * acc.x; o.y += alpha * acc.y; o.z += alpha * acc.z; o.w += alpha * acc.w;
+    reinterpret_cast<float4*>(out + i)[0] = o;
+  } else {
+    for (long j = i; j < mn; ++j) {
+      float acc = 0.f;
+      for (int s = 0; s < splits; ++s) acc += part[(long)s * mn + j];
+      out[j] = (beta != 0.f ? beta * out[j] : 0.f) + alpha * acc;
+    }
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] with row pitch `pitch` elements.
+bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
+               uint32_t box_inner, uint32_t box_outer) {
+  auto enc = tmap_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN>
+int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int grid, cudaStream_t st) {
+  using C = TcCfg<BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  C::SMEM_BYTES));
+    attr_set = true;
+  }
+  gemm_tc_kernel<BN><<<grid, NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, p);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int auto_splits(int M, int N, int K) {
+  const int tiles = ((M + BM - 1) / BM) * ((N + 255) / 256);
+  const int kb = K / BK;
+  const int sms = num_sms();
+  if (tiles >= sms) return 1;
+  int s = (2 * sms + tiles - 1) / tiles;
+  if (s > kb / 4) s = kb / 4;
+  return s < 1 ? 1 : s;
+}
+
+}  // namespace
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
+size_t gemm_tc_split_bytes(int M, int N, int K) {
+  int s = auto_splits(M, N, K);
+  return s > 1 ? (size_t)s * M * N * sizeof(float) : 0;
+}
+
+int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int splits, int* err,
+                 cudaStream_t st) {
+  if (g.M <= 0 || g.N <= 0) return GPT2_OK;
+  if (g.K <= 0 || g.K % BK) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (g.lda % 8 || g.ldb % 8 || g.epi.ldo % 8) return GPT2_ERR_INVALID_ARG;
+  if (((uintptr_t)g.A | (uintptr_t)g.B | (uintptr_t)g.epi.out) & 15) return GPT2_ERR_INVALID_ARG;
+  if (bn == 0) bn = g.N <= 128 ? 128 : 256;
+  if (bn != 128 && bn != 256) return GPT2_ERR_INVALID_ARG;
+  const int kb_total = g.K / BK;
+  if (splits == 0) splits = g.epi.kind == EPI_F32 ? auto_splits(g.M, g.N, g.K) : 1;
+  if (splits > kb_total) splits = kb_total;
+  if (splits > 1) {
+    if (g.epi.kind != EPI_F32 || g.N % 4 || g.epi.ldo != g.N) return GPT2_ERR_INVALID_ARG;
+    size_t need = (size_t)splits * g.M * g.N * sizeof(float);
+    if (!ws || ws_bytes < need) splits = 1;
+  }
+
+  CUtensorMap ta, tb;
+  bool ok_a = g.a_mn ? make_tmap(&ta, g.A, g.M, g.K, g.lda, 64, 64)
+                     : make_tmap(&ta, g.A, g.K, g.M, g.lda, 64, BM);
+  bool ok_b = g.b_mn ? make_tmap(&tb, g.B, g.N, g.K, g.ldb, 64, 64)
+                     : make_tmap(&tb, g.B, g.K, g.N, g.ldb, 64, bn);
+  if (!ok_a || !ok_b) return GPT2_ERR_CUDA;
+
+  TcParams p;
+  p.M = g.M; p.N = g.N; p.K = g.K;
+  p.a_mn = g.a_mn; p.b_mn = g.b_mn;
+  p.m_tiles = (g.M + BM - 1) / BM;
+  p.n_tiles = (g.N + bn - 1) / bn;
+  p.splits = splits;
+  p.kb_total = kb_total;
+  // instruction descriptor, kind::f16: D fp32 (bit 4), A and B bf16 (bits 7, 10),
+  // operand majorness (bits 15, 16), N >> 3 at bit 17, M >> 4 at bit 24.
+  p.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)g.a_mn << 15) | ((uint32_t)g.b_mn << 16) |
+            ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  p.epi = g.epi;
+  p.partial = (float*)ws;
+  p.err = err;
+  if (splits > 1) p.epi.kind = EPI_F32_PARTIAL;
+
+  const int units = p.m_tiles * p.n_tiles * splits;
+  const int grid = units < num_sms() ? units : num_sms();
+  int rc = bn == 256 ? launch_tc<256>(ta, tb, p, grid, st) : launch_tc<128>(ta, tb, p, grid, st);
+  if (rc) return rc;
+  if (splits > 1) {
+    long mn = (long)g.M * g.N;
+    long threads = (mn + 3) / 4;
+    splitk_reduce_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+        (const float*)ws, splits, mn, (float*)g.epi.out, g.epi.alpha, g.epi.beta);
+    LAUNCH_CHECK();
+  }
+  return GPT2_OK;
+}

@@ -1,0 +1,556 @@
+// C ABI of libgpt2.so: parameter layout, workspace carving, and the sequence
+// of kernels that makes one GPT-2 training step (forward + loss, backward,
+// AdamW).  Everything here runs on the host and only enqueues work.
+#include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+enum LayerTensor { LN1_G, LN1_B, W_QKV, B_QKV, W_O, B_O, LN2_G, LN2_B, W_FC, B_FC, W_MP, B_MP, N_LT };
+const char* const kLayerNames[N_LT] = {"ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
+                                       "ln2_g", "ln2_b", "w_fc", "b_fc", "w_mp", "b_mp"};
+
+struct Shape {
+  long L, d, H, T, V, Vr, hd;
+  int mode;
+};
+
+void lt_dims(long d, int t, long* rows, long* cols) {
+  switch (t) {
+    case W_QKV: *rows = 3 * d; *cols = d; return;
+    case B_QKV: *rows = 3 * d; *cols = 1; return;
+    case W_O: *rows = d; *cols = d; return;
+    case W_FC: *rows = 4 * d; *cols = d; return;
+    case B_FC: *rows = 4 * d; *cols = 1; return;
+    case W_MP: *rows = d; *cols = 4 * d; return;
+    default: *rows = d; *cols = 1; return;
+  }
+}
+long lt_offset(long d, int t) {
+  long off = 0;
+  for (int i = 0; i < t; ++i) {
+    long r, c;
+    lt_dims(d, i, &r, &c);
+    off += r * c;
+  }
+  return off;
+}
+long layer_size(long d) { return lt_offset(d, N_LT); }
+
+struct Offsets {
+  Shape s;
+  size_t wte() const { return 0; }
+  size_t wpe() const { return (size_t)(s.V * s.d); }
+  size_t layer(int l, int t) const {
+    return (size_t)((s.V + s.T) * s.d + l * layer_size(s.d) + lt_offset(s.d, t));
+  }
+  size_t lnf_g() const { return (size_t)((s.V + s.T) * s.d + s.L * layer_size(s.d)); }
+  size_t lnf_b() const { return lnf_g() + s.d; }
+  size_t total() const { return lnf_b() + s.d; }
+};
+
+bool shape_from_cfg(const gpt2_config* c, Shape* s) {
+  if (!c) return false;
+  if (c->n_layer < 1 || c->d_model < 1 || c->n_head < 1 || c->n_ctx < 1 || c->vocab_real < 1 ||
+      c->vocab_padded < c->vocab_real || c->max_batch < 1 || (c->mode != 0 && c->mode != 1))
+    return false;
+  if (c->d_model % c->n_head) return false;
+  s->L = c->n_layer; s->d = c->d_model; s->H = c->n_head; s->T = c->n_ctx;
+  s->V = c->vocab_padded; s->Vr = c->vocab_real; s->hd = c->d_model / c->n_head; s->mode = c->mode;
+  return true;
+}
+
+int check_supported(const Shape& s, int max_batch) {
+  if (s.d % 64) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (s.V % 128) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (s.hd != 16 && s.hd != 64) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (s.d > 2048) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (s.mode == 1 && s.T > 4096) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if ((long)max_batch * s.T > (1L << 30)) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  return GPT2_OK;
+}
+
+// Bump allocator over the workspace (base may be NULL to only measure).
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  template <typename P>
+  P* take(size_t bytes) {
+    off = (off + 255) & ~(size_t)255;
+    P* p = base ? reinterpret_cast<P*>(base + off) : nullptr;
+    off += bytes;
+    return p;
+  }
+};
+
+struct LayerActs {
+  void *x_in, *x_mid, *y1, *qkv, *o, *y2, *u, *g;
+  float *mean1, *rstd1, *mean2, *rstd2, *lse;
+};
+
+struct Work {
+  int* err;
+  float* loss;
+  int32_t *tok, *tgt, *tok_stage, *tgt_stage;
+  std::vector<LayerActs> layers;
+  void *x_final, *yf, *logits;
+  float *meanf, *rstdf, *loss_rows;
+  void *dres, *dy, *du, *dqkv, *dout;
+  float *dq_acc, *dvec, *ln_part, *cs_part;
+  void* split_ws;
+  size_t split_bytes;
+  long long* emb_acc;
+  uint8_t* touched;
+};
+
+size_t split_ws_need(const Shape& s, long M) {
+  if (s.mode != 0) return 0;
+  size_t need = 0;
+  const long d = s.d;
+  const long shapes[5][2] = {{3 * d, d}, {d, d}, {4 * d, d}, {d, 4 * d}, {s.V, d}};
+  for (auto& sh : shapes) {
+    size_t b = gemm_tc_split_bytes((int)sh[0], (int)sh[1], (int)M);
+    if (b > need) need = b;
+  }
+  return need;
+}
+
+size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
+  Carver c{base};
+  const long M = (long)batch * s.T, d = s.d;
+  const size_t act = s.mode ? 4 : 2;
+  w->err = c.take<int>(sizeof(int));
+  w->loss = c.take<float>(sizeof(float));
+  w->tok = c.take<int32_t>(M * 4);
+  w->tgt = c.take<int32_t>(M * 4);
+  w->tok_stage = c.take<int32_t>(M * 4);
+  w->tgt_stage = c.take<int32_t>(M * 4);
+  w->layers.assign(s.L, LayerActs{});
+  void* x_prev = c.take<void>(M * d * act);  // x_0: the embedding output
+  for (long l = 0; l < s.L; ++l) {
+    LayerActs& a = w->layers[l];
+    a.x_in = x_prev;
+    a.y1 = c.take<void>(M * d * act);
+    a.mean1 = c.take<float>(M * 4);
+    a.rstd1 = c.take<float>(M * 4);
+    a.qkv = c.take<void>(M * 3 * d * act);
+    a.o = c.take<void>(M * d * act);
+    a.lse = c.take<float>(M * s.H * 4);
+    a.x_mid = c.take<void>(M * d * act);
+    a.y2 = c.take<void>(M * d * act);
+    a.mean2 = c.take<float>(M * 4);
+    a.rstd2 = c.take<float>(M * 4);
+    a.u = c.take<void>(M * 4 * d * act);
+    a.g = c.take<void>(M * 4 * d * act);
+    x_prev = c.take<void>(M * d * act);
+  }
+  w->x_final = x_prev;
+  w->yf = c.take<void>(M * d * act);
+  w->meanf = c.take<float>(M * 4);
+  w->rstdf = c.take<float>(M * 4);
+  w->logits = c.take<void>(M * s.V * act);
+  w->loss_rows = c.take<float>(M * 4);
+  w->dres = c.take<void>(M * d * act);
+  w->dy = c.take<void>(M * d * act);
+  w->du = c.take<void>(M * 4 * d * act);
+  w->dqkv = c.take<void>(M * 3 * d * act);
+  w->dout = c.take<void>(M * d * act);
+  w->dq_acc = c.take<float>(M * d * 4);
+  w->dvec = c.take<float>(M * s.H * 4);
+  w->ln_part = c.take<float>(layernorm_bwd_part_floats((int)M, (int)d) * 4);
+  w->cs_part = c.take<float>(colsum_part_floats((int)M, (int)(4 * d)) * 4);
+  w->split_bytes = split_ws_need(s, M);
+  w->split_ws = c.take<void>(w->split_bytes);
+  w->emb_acc = c.take<long long>((size_t)s.V * d * 8);
+  w->touched = c.take<uint8_t>((size_t)s.V);
+  return (c.off + 255) & ~(size_t)255;
+}
+
+}  // namespace
+
+struct gpt2_ctx {
+  gpt2_config cfg;
+  Shape s;
+  Offsets off;
+  gpt2_buffers buf;
+  Work w;
+  int have_fwd = 0;
+  int fwd_batch = 0;
+};
+
+namespace {
+
+cudaStream_t S(void* st) { return reinterpret_cast<cudaStream_t>(st); }
+
+// Parameter pointers in the compute dtype: bf16 shadow (mode 0) or fp32 master.
+const void* Wp(const gpt2_ctx* c, size_t off) {
+  return c->s.mode ? (const void*)(c->buf.master + off) : (const void*)(c->buf.shadow + off);
+}
+size_t act_bytes(const gpt2_ctx* c) { return c->s.mode ? 4 : 2; }
+
+int run_gemm(gpt2_ctx* c, const GemmArgs& g, cudaStream_t st) {
+  if (c->s.mode) return gemm_simt_f32(g, st);
+  return gemm_tc_bf16(g, c->w.split_ws, c->w.split_bytes, 0, 0, c->w.err, st);
+}
+
+GemmArgs make_gemm(int M, int N, int K, const void* A, int a_mn, long lda, const void* B, int b_mn, long ldb,
+                   int kind, void* out, long ldo) {
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.M = M; g.N = N; g.K = K;
+  g.A = A; g.a_mn = a_mn; g.lda = lda;
+  g.B = B; g.b_mn = b_mn; g.ldb = ldb;
+  g.epi.kind = kind;
+  g.epi.out = out;
+  g.epi.ldo = ldo;
+  g.epi.alpha = 1.f;
+  g.epi.beta = 0.f;
+  return g;
+}
+
+#define TRY(x)              \
+  do {                      \
+    int rc_ = (x);          \
+    if (rc_) return rc_;    \
+  } while (0)
+
+// param grads of one (gamma, beta) pair / bias from block partials
+int ln_param_grads(gpt2_ctx* c, int nblk, size_t goff, float beta, cudaStream_t st) {
+  return reduce_rows_f32(c->w.ln_part, nblk, (int)(2 * c->s.d), c->buf.grad + goff, beta, st);
+}
+int bias_grad(gpt2_ctx* c, const void* x, int M, int N, size_t goff, float beta, cudaStream_t st) {
+  int nblk = 0;
+  TRY(colsum_partial(c->s.mode, x, M, N, c->w.cs_part, &nblk, st));
+  return reduce_rows_f32(c->w.cs_part, nblk, N, c->buf.grad + goff, beta, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gpt2_param_count(const gpt2_config* cfg) {
+  Shape s;
+  if (!shape_from_cfg(cfg, &s)) return 0;
+  Offsets o{s};
+  return o.total();
+}
+
+size_t gpt2_workspace_bytes(const gpt2_config* cfg, int batch) {
+  Shape s;
+  if (!shape_from_cfg(cfg, &s) || batch < 1) return 0;
+  Work w;
+  return carve(s, batch, nullptr, &w);
+}
+
+int gpt2_tensor_info(const gpt2_config* cfg, int index, const char** name, size_t* offset, size_t* rows,
+                     size_t* cols) {
+  static char namebuf[64];
+  Shape s;
+  if (!shape_from_cfg(cfg, &s) || index < 0) return GPT2_ERR_INVALID_ARG;
+  Offsets o{s};
+  long r = 0, cc = 1;
+  size_t off = 0;
+  const int nl = (int)s.L * N_LT;
+  if (index == 0) {
+    snprintf(namebuf, sizeof(namebuf), "wte"); off = o.wte(); r = s.V; cc = s.d;
+  } else if (index == 1) {
+    snprintf(namebuf, sizeof(namebuf), "wpe"); off = o.wpe(); r = s.T; cc = s.d;
+  } else if (index < 2 + nl) {
+    int l = (index - 2) / N_LT, t = (index - 2) % N_LT;
+    snprintf(namebuf, sizeof(namebuf), "h%d.%s", l, kLayerNames[t]);
+    off = o.layer(l, t);
+    lt_dims(s.d, t, &r, &cc);
+  } else if (index == 2 + nl) {
+    snprintf(namebuf, sizeof(namebuf), "lnf_g"); off = o.lnf_g(); r = s.d;
+  } else if (index == 3 + nl) {
+    snprintf(namebuf, sizeof(namebuf), "lnf_b"); off = o.lnf_b(); r = s.d;
+  } else {
+    return GPT2_ERR_INVALID_ARG;
+  }
+  if (name) *name = namebuf;
+  if (offset) *offset = off;
+  if (rows) *rows = (size_t)r;
+  if (cols) *cols = (size_t)cc;
+  return GPT2_OK;
+}
+
+int gpt2_create(const gpt2_config* cfg, const gpt2_buffers* bufs, gpt2_ctx** out) {
+  if (!cfg || !bufs || !out) return GPT2_ERR_INVALID_ARG;
+  *out = nullptr;
+  Shape s;
+  if (!shape_from_cfg(cfg, &s)) return GPT2_ERR_INVALID_ARG;
+  TRY(check_supported(s, cfg->max_batch));
+  if (s.mode == 0 && ((long)cfg->max_batch * s.T) % 64) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (!bufs->master || !bufs->grad || !bufs->m || !bufs->v || !bufs->workspace) return GPT2_ERR_INVALID_ARG;
+  if (s.mode == 0 && !bufs->shadow) return GPT2_ERR_INVALID_ARG;
+  const uintptr_t align = (uintptr_t)bufs->master | (uintptr_t)bufs->grad | (uintptr_t)bufs->m |
+                          (uintptr_t)bufs->v | (uintptr_t)bufs->workspace | (uintptr_t)bufs->shadow;
+  if (align & 15) return GPT2_ERR_INVALID_ARG;
+  gpt2_ctx* c = new gpt2_ctx();
+  c->cfg = *cfg;
+  c->s = s;
+  c->off = Offsets{s};
+  c->buf = *bufs;
+  const size_t need = carve(s, cfg->max_batch, (uint8_t*)bufs->workspace, &c->w);
+  if (bufs->workspace_bytes < need) {
+    delete c;
+    return GPT2_ERR_WORKSPACE;
+  }
+  if (cudaMemset(c->w.err, 0, sizeof(int)) != cudaSuccess ||
+      cudaMemset(c->w.emb_acc, 0, (size_t)s.V * s.d * 8) != cudaSuccess ||
+      cudaMemset(c->w.touched, 0, (size_t)s.V) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    delete c;
+    return GPT2_ERR_CUDA;
+  }
+  *out = c;
+  return GPT2_OK;
+}
+
+int gpt2_destroy(gpt2_ctx* ctx) {
+  delete ctx;
+  return GPT2_OK;
+}
+
+int gpt2_refresh_shadow(gpt2_ctx* c, void* stream) {
+  if (!c) return GPT2_ERR_INVALID_ARG;
+  if (!c->buf.shadow) return GPT2_OK;
+  return cast_shadow(c->buf.master, c->buf.shadow, c->off.total(), S(stream));
+}
+
+int gpt2_init_params(gpt2_ctx* c, uint64_t seed, void* stream) {
+  if (!c) return GPT2_ERR_INVALID_ARG;
+  const size_t n = c->off.total();
+  LayoutDims ld{c->s.V, c->s.T, c->s.d, c->s.L};
+  TRY(init_params(c->buf.master, n, ld, seed, S(stream)));
+  TRY(fill_zero(c->buf.grad, n * 4, S(stream)));
+  TRY(fill_zero(c->buf.m, n * 4, S(stream)));
+  TRY(fill_zero(c->buf.v, n * 4, S(stream)));
+  return gpt2_refresh_shadow(c, stream);
+}
+
+int gpt2_zero_grad(gpt2_ctx* c, void* stream) {
+  if (!c) return GPT2_ERR_INVALID_ARG;
+  return fill_zero(c->buf.grad, c->off.total() * 4, S(stream));
+}
+
+int gpt2_forward_loss(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets, int batch, float* loss_dev,
+                      void* stream) {
+  if (!c || !tokens || !targets) return GPT2_ERR_INVALID_ARG;
+  if (batch < 1 || batch > c->cfg.max_batch) return GPT2_ERR_INVALID_ARG;
+  const Shape& s = c->s;
+  const int M = batch * (int)s.T, d = (int)s.d, V = (int)s.V;
+  if (s.mode == 0 && M % 64) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = S(stream);
+  Work& w = c->w;
+  const Offsets& o = c->off;
+  const int f32 = s.mode;
+  CUDA_TRY(cudaMemcpyAsync(w.tok, tokens, (size_t)M * 4, cudaMemcpyDeviceToDevice, st));
+  CUDA_TRY(cudaMemcpyAsync(w.tgt, targets, (size_t)M * 4, cudaMemcpyDeviceToDevice, st));
+  c->have_fwd = 0;
+
+  TRY(embed_fwd(f32, w.tok, Wp(c, o.wte()), Wp(c, o.wpe()), w.layers[0].x_in, M, (int)s.T, d, (int)s.Vr, w.err,
+                st));
+  for (int l = 0; l < (int)s.L; ++l) {
+    LayerActs& a = w.layers[l];
+    TRY(layernorm_fwd(f32, a.x_in, Wp(c, o.layer(l, LN1_G)), Wp(c, o.layer(l, LN1_B)), a.y1, a.mean1, a.rstd1, M,
+                      d, st));
+    GemmArgs g = make_gemm(M, 3 * d, d, a.y1, 0, d, Wp(c, o.layer(l, W_QKV)), 0, d, EPI_BIAS, a.qkv, 3 * d);
+    g.epi.bias = Wp(c, o.layer(l, B_QKV));
+    TRY(run_gemm(c, g, st));
+    if (f32)
+      TRY(attn_fwd_f32((const float*)a.qkv, (float*)a.o, a.lse, batch, (int)s.T, (int)s.H, (int)s.hd, st));
+    else
+      TRY(attn_fwd_bf16(a.qkv, a.o, a.lse, batch, (int)s.T, (int)s.H, (int)s.hd, st));
+    g = make_gemm(M, d, d, a.o, 0, d, Wp(c, o.layer(l, W_O)), 0, d, EPI_BIAS_RESID, a.x_mid, d);
+    g.epi.bias = Wp(c, o.layer(l, B_O));
+    g.epi.resid = a.x_in;
+    TRY(run_gemm(c, g, st));
+    TRY(layernorm_fwd(f32, a.x_mid, Wp(c, o.layer(l, LN2_G)), Wp(c, o.layer(l, LN2_B)), a.y2, a.mean2, a.rstd2,
+                      M, d, st));
+    g = make_gemm(M, 4 * d, d, a.y2, 0, d, Wp(c, o.layer(l, W_FC)), 0, d, EPI_BIAS_GELU, a.u, 4 * d);
+    g.epi.bias = Wp(c, o.layer(l, B_FC));
+    g.epi.out2 = a.g;
+    TRY(run_gemm(c, g, st));
+    void* x_out = (l + 1 < (int)s.L) ? w.layers[l + 1].x_in : w.x_final;
+    g = make_gemm(M, d, 4 * d, a.g, 0, 4 * d, Wp(c, o.layer(l, W_MP)), 0, 4 * d, EPI_BIAS_RESID, x_out, d);
+    g.epi.bias = Wp(c, o.layer(l, B_MP));
+    g.epi.resid = a.x_mid;
+    TRY(run_gemm(c, g, st));
+  }
+  TRY(layernorm_fwd(f32, w.x_final, Wp(c, o.lnf_g()), Wp(c, o.lnf_b()), w.yf, w.meanf, w.rstdf, M, d, st));
+  GemmArgs g = make_gemm(M, V, d, w.yf, 0, d, Wp(c, o.wte()), 0, d, EPI_STORE, w.logits, V);
+  TRY(run_gemm(c, g, st));
+  TRY(ce_fwd(f32, w.logits, w.tgt, w.loss_rows, M, V, (int)s.Vr, w.err, st));
+  TRY(loss_mean(w.loss_rows, M, loss_dev ? loss_dev : w.loss, w.err, st));
+  c->have_fwd = 1;
+  c->fwd_batch = batch;
+  return GPT2_OK;
+}
+
+int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
+  if (!c) return GPT2_ERR_INVALID_ARG;
+  if (!c->have_fwd) return GPT2_ERR_BAD_STATE;
+  const Shape& s = c->s;
+  const int batch = c->fwd_batch;
+  const int M = batch * (int)s.T, d = (int)s.d, V = (int)s.V;
+  cudaStream_t st = S(stream);
+  Work& w = c->w;
+  const Offsets& o = c->off;
+  const int f32 = s.mode;
+  const float beta = accumulate ? 1.f : 0.f;
+  const float sc = grad_scale / (float)M;
+  float* G = c->buf.grad;
+
+  // LM head (tied): dX_f = s * dz wte ; dwte (=/+=) s * dz^T X_f
+  GemmArgs g = make_gemm(M, d, V, w.logits, 0, V, Wp(c, o.wte()), 1, d, EPI_STORE, w.dy, d);
+  g.epi.alpha = sc;
+  TRY(run_gemm(c, g, st));
+  g = make_gemm(V, d, M, w.logits, 1, V, w.yf, 1, d, EPI_F32, G + o.wte(), d);
+  g.epi.alpha = sc;
+  g.epi.beta = beta;
+  TRY(run_gemm(c, g, st));
+  int nblk = 0;
+  TRY(layernorm_bwd(f32, w.dy, w.x_final, w.meanf, w.rstdf, Wp(c, o.lnf_g()), w.dres, 1, w.ln_part, &nblk, M, d,
+                    st));
+  TRY(ln_param_grads(c, nblk, o.lnf_g(), beta, st));
+
+  for (int l = (int)s.L - 1; l >= 0; --l) {
+    LayerActs& a = w.layers[l];
+    // MLP projection: x_out = x_mid + g W_mp^T + b_mp
+    g = make_gemm(M, 4 * d, d, w.dres, 0, d, Wp(c, o.layer(l, W_MP)), 1, 4 * d, EPI_DGELU, w.du, 4 * d);
+    g.epi.aux = a.u;
+    TRY(run_gemm(c, g, st));
+    g = make_gemm(d, 4 * d, M, w.dres, 1, d, a.g, 1, 4 * d, EPI_F32, G + o.layer(l, W_MP), 4 * d);
+    g.epi.beta = beta;
+    TRY(run_gemm(c, g, st));
+    TRY(bias_grad(c, w.dres, M, d, o.layer(l, B_MP), beta, st));
+    // MLP fc: u = y2 W_fc^T + b_fc
+    g = make_gemm(M, d, 4 * d, w.du, 0, 4 * d, Wp(c, o.layer(l, W_FC)), 1, d, EPI_STORE, w.dy, d);
+    TRY(run_gemm(c, g, st));
+    g = make_gemm(4 * d, d, M, w.du, 1, 4 * d, a.y2, 1, d, EPI_F32, G + o.layer(l, W_FC), d);
+    g.epi.beta = beta;
+    TRY(run_gemm(c, g, st));
+    TRY(bias_grad(c, w.du, M, 4 * d, o.layer(l, B_FC), beta, st));
+    TRY(layernorm_bwd(f32, w.dy, a.x_mid, a.mean2, a.rstd2, Wp(c, o.layer(l, LN2_G)), w.dres, 0, w.ln_part, &nblk,
+                      M, d, st));
+    TRY(ln_param_grads(c, nblk, o.layer(l, LN2_G), beta, st));
+    // attention projection: x_mid = x_in + o W_o^T + b_o
+    g = make_gemm(M, d, d, w.dres, 0, d, Wp(c, o.layer(l, W_O)), 1, d, EPI_STORE, w.dout, d);
+    TRY(run_gemm(c, g, st));
+    g = make_gemm(d, d, M, w.dres, 1, d, a.o, 1, d, EPI_F32, G + o.layer(l, W_O), d);
+    g.epi.beta = beta;
+    TRY(run_gemm(c, g, st));
+    TRY(bias_grad(c, w.dres, M, d, o.layer(l, B_O), beta, st));
+    // attention
+    if (f32)
+      TRY(attn_bwd_f32((const float*)a.qkv, (const float*)a.o, a.lse, (const float*)w.dout, (float*)w.dqkv, w.dvec,
+                       batch, (int)s.T, (int)s.H, (int)s.hd, st));
+    else
+      TRY(attn_bwd_bf16(a.qkv, a.o, a.lse, w.dout, w.dqkv, w.dq_acc, w.dvec, batch, (int)s.T, (int)s.H, (int)s.hd,
+                        st));
+    // QKV: qkv = y1 W_qkv^T + b_qkv
+    g = make_gemm(M, d, 3 * d, w.dqkv, 0, 3 * d, Wp(c, o.layer(l, W_QKV)), 1, d, EPI_STORE, w.dy, d);
+    TRY(run_gemm(c, g, st));
+    g = make_gemm(3 * d, d, M, w.dqkv, 1, 3 * d, a.y1, 1, d, EPI_F32, G + o.layer(l, W_QKV), d);
+    g.epi.beta = beta;
+    TRY(run_gemm(c, g, st));
+    TRY(bias_grad(c, w.dqkv, M, 3 * d, o.layer(l, B_QKV), beta, st));
+    TRY(layernorm_bwd(f32, w.dy, a.x_in, a.mean1, a.rstd1, Wp(c, o.layer(l, LN1_G)), w.dres, 0, w.ln_part, &nblk,
+                      M, d, st));
+    TRY(ln_param_grads(c, nblk, o.layer(l, LN1_G), beta, st));
+  }
+  // x_0 = wte[tok] + wpe[t]
+  TRY(embed_bwd(f32, w.tok, w.dres, G + o.wte(), G + o.wpe(), w.emb_acc, w.touched, M, (int)s.T, d, V, accumulate,
+                st));
+  return GPT2_OK;
+}
+
+int gpt2_adamw_step(gpt2_ctx* c, float lr, float beta1, float beta2, float eps, float weight_decay, int step,
+                    void* stream) {
+  if (!c || step < 1) return GPT2_ERR_INVALID_ARG;
+  AdamArgs a;
+  a.lr = lr; a.beta1 = beta1; a.beta2 = beta2; a.eps = eps; a.wd = weight_decay;
+  a.bc1 = (float)(1.0 - pow((double)beta1, (double)step));
+  a.bc2 = (float)(1.0 - pow((double)beta2, (double)step));
+  LayoutDims ld{c->s.V, c->s.T, c->s.d, c->s.L};
+  return adamw(c->buf.master, c->buf.grad, c->buf.m, c->buf.v, c->s.mode ? nullptr : c->buf.shadow,
+               c->off.total(), ld, a, S(stream));
+}
+
+int gpt2_get_status(gpt2_ctx* c, void* stream) {
+  if (!c) return GPT2_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return GPT2_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpy(&h, c->w.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GPT2_ERR_CUDA;
+  if (h && cudaMemset(c->w.err, 0, sizeof(int)) != cudaSuccess) return GPT2_ERR_CUDA;
+  if (h & DEV_ERR_TIMEOUT) return GPT2_ERR_TIMEOUT;
+  if (h & DEV_ERR_NONFINITE) return GPT2_ERR_NONFINITE;
+  if (h & DEV_ERR_TOKEN) return GPT2_ERR_TOKEN_RANGE;
+  return GPT2_OK;
+}
+
+int gpt2_step_host(gpt2_ctx* c, const int32_t* tokens_host, const int32_t* targets_host, int batch,
+                   float* loss_host, float lr, float beta1, float beta2, float eps, float weight_decay, int step,
+                   void* stream) {
+  if (!c || !tokens_host || !targets_host || !loss_host) return GPT2_ERR_INVALID_ARG;
+  if (batch < 1 || batch > c->cfg.max_batch) return GPT2_ERR_INVALID_ARG;
+  cudaStream_t st = S(stream);
+  const size_t bytes = (size_t)batch * c->s.T * 4;
+  CUDA_TRY(cudaMemcpyAsync(c->w.tok_stage, tokens_host, bytes, cudaMemcpyHostToDevice, st));
+  CUDA_TRY(cudaMemcpyAsync(c->w.tgt_stage, targets_host, bytes, cudaMemcpyHostToDevice, st));
+  TRY(gpt2_forward_loss(c, c->w.tok_stage, c->w.tgt_stage, batch, c->w.loss, stream));
+  TRY(gpt2_backward(c, 1.f, 0, stream));
+  TRY(gpt2_adamw_step(c, lr, beta1, beta2, eps, weight_decay, step, stream));
+  CUDA_TRY(cudaMemcpyAsync(loss_host, c->w.loss, sizeof(float), cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  return GPT2_OK;
+}
+
+const char* gpt2_strerror(int code) {
+  switch (code) {
+    case GPT2_OK: return "ok";
+    case GPT2_ERR_INVALID_ARG: return "invalid argument";
+    case GPT2_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case GPT2_ERR_CUDA: return "CUDA error";
+    case GPT2_ERR_BAD_STATE: return "bad state (backward without forward?)";
+    case GPT2_ERR_TOKEN_RANGE: return "token or target id out of range";
+    case GPT2_ERR_NONFINITE: return "non-finite loss";
+    case GPT2_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case GPT2_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown error";
+  }
+}
+
+int gpt2_op_gemm_bf16(const uint16_t* A, int a_mn_major, int lda, const uint16_t* B, int b_mn_major, int ldb,
+                      void* C, int c_fp32, int ldc, int M, int N, int K, float alpha, float beta, void* workspace,
+                      size_t workspace_bytes, int bn, int splits, void* stream) {
+  if (!A || !B || !C || M < 0 || N < 0 || K < 0) return GPT2_ERR_INVALID_ARG;
+  GemmArgs g = make_gemm(M, N, K, A, a_mn_major ? 1 : 0, lda, B, b_mn_major ? 1 : 0, ldb,
+                         c_fp32 ? EPI_F32 : EPI_STORE, C, ldc);
+  g.epi.alpha = alpha;
+  g.epi.beta = c_fp32 ? beta : 0.f;
+  return gemm_tc_bf16(g, workspace, workspace_bytes, bn, splits, nullptr, S(stream));
+}
+
+int gpt2_op_attention_fwd_bf16(const uint16_t* qkv, uint16_t* o, float* lse, int B, int T, int H, int hd,
+                               void* stream) {
+  if (!qkv || !o || !lse || B < 0 || T < 0 || H < 1) return GPT2_ERR_INVALID_ARG;
+  return attn_fwd_bf16(qkv, o, lse, B, T, H, hd, S(stream));
+}
+
+int gpt2_op_attention_bwd_bf16(const uint16_t* qkv, const uint16_t* o, const float* lse, const uint16_t* dout,
+                               uint16_t* dqkv, float* scratch, int B, int T, int H, int hd, void* stream) {
+  if (!qkv || !o || !lse || !dout || !dqkv || !scratch || B < 0 || T < 0 || H < 1) return GPT2_ERR_INVALID_ARG;
+  float* dq_acc = scratch;
+  float* dvec = scratch + (size_t)B * T * H * hd;
+  return attn_bwd_bf16(qkv, o, lse, dout, dqkv, dq_acc, dvec, B, T, H, hd, S(stream));
+}
+
+}  // extern "C"

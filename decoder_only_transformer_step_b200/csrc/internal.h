@@ -1,0 +1,101 @@
+// Host-side interface between the library's compilation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+// Epilogue applied to each GEMM output element (row m, column n, fp32 acc).
+// "act" is the activation type of the mode (bf16 or fp32).
+enum EpiKind : int {
+  EPI_STORE = 0,    // out(act)  = alpha * acc
+  EPI_BIAS,         // out(act)  = acc + bias[n]
+  EPI_BIAS_RESID,   // out(act)  = acc + bias[n] + resid[m,n]
+  EPI_BIAS_GELU,    // out(act)  = u = acc + bias[n];  out2(act) = gelu(u)
+  EPI_DGELU,        // out(act)  = acc * gelu'(aux[m,n])
+  EPI_F32,          // out(fp32) = beta * out + alpha * acc
+  EPI_F32_PARTIAL,  // partial[split][m,n] = acc (split-K, internal)
+};
+
+struct EpiArgs {
+  int kind;
+  void* out;          // [M, ldo]
+  void* out2;         // [M, ldo] (EPI_BIAS_GELU)
+  const void* bias;   // [N] act
+  const void* resid;  // [M, ldo] act
+  const void* aux;    // [M, ldo] act
+  long ldo;
+  float alpha, beta;
+};
+
+// C[m,n] = sum_k A(m,k) B(n,k), then the epilogue.
+// a_mn = 0: A(m,k) = A[m*lda + k]; a_mn = 1: A(m,k) = A[k*lda + m].
+// b_mn = 0: B(n,k) = B[n*ldb + k]; b_mn = 1: B(n,k) = B[k*ldb + n].
+struct GemmArgs {
+  int M, N, K;
+  const void* A; int a_mn; long lda;
+  const void* B; int b_mn; long ldb;
+  EpiArgs epi;
+};
+
+// tcgen05 bf16 GEMM (sm_100a).  ws (may be NULL) holds split-K partials for
+// EPI_F32.  bn: 0 auto / 128 / 256; splits: 0 auto.
+int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int splits, int* err,
+                 cudaStream_t st);
+// Workspace bytes the automatic split-K choice wants for this problem.
+size_t gemm_tc_split_bytes(int M, int N, int K);
+
+// fp32 CUDA-core GEMM for the correctness mode.
+int gemm_simt_f32(const GemmArgs& g, cudaStream_t st);
+
+int num_sms();
+
+// ---- attention ----------------------------------------------------------
+// qkv [B*T, 3*H*hd] (act), o [B*T, H*hd] (act), lse [B,H,T] fp32.
+int attn_fwd_bf16(const void* qkv, void* o, float* lse, int B, int T, int H, int hd,
+                  cudaStream_t st);
+int attn_fwd_f32(const float* qkv, float* o, float* lse, int B, int T, int H, int hd,
+                 cudaStream_t st);
+// dq_acc: fp32 [B*T, H*hd] scratch; dvec: fp32 [B,H,T] scratch.
+int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* dout, void* dqkv,
+                  float* dq_acc, float* dvec, int B, int T, int H, int hd, cudaStream_t st);
+int attn_bwd_f32(const float* qkv, const float* o, const float* lse, const float* dout,
+                 float* dqkv, float* dvec, int B, int T, int H, int hd, cudaStream_t st);
+
+// ---- elementwise / reductions (templated on bf16 = 0 / fp32 = 1) -------
+int embed_fwd(int f32, const int32_t* tok, const void* wte, const void* wpe, void* x, int M, int T,
+              int d, int vocab_real, int* err, cudaStream_t st);
+int layernorm_fwd(int f32, const void* x, const void* g, const void* b, void* y, float* mean,
+                  float* rstd, int M, int d, cudaStream_t st);
+// dres = (dres_init ? 0 : dres) + LN'(dy); writes per-block partials of
+// dgamma, dbeta into part [nblk, 2, d]; returns nblk via *nblk.
+int layernorm_bwd(int f32, const void* dy, const void* x, const float* mean, const float* rstd,
+                  const void* g, void* dres, int dres_init, float* part, int* nblk, int M, int d,
+                  cudaStream_t st);
+size_t layernorm_bwd_part_floats(int M, int d);
+// grad[j] = beta*grad[j] + sum_b part[b, j]  for j < n  (part row pitch n)
+int reduce_rows_f32(const float* part, int nrows, int n, float* grad, float beta, cudaStream_t st);
+// per-block column sums of x [M, N] (act) into part [nblk, N]
+int colsum_partial(int f32, const void* x, int M, int N, float* part, int* nblk, cudaStream_t st);
+size_t colsum_part_floats(int M, int N);
+// cross-entropy: logits [M, V] (act) -> in place dz = softmax - onehot; loss_rows [M]
+int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, int V,
+           int vocab_real, int* err, cudaStream_t st);
+int loss_mean(const float* loss_rows, int M, float* loss, int* err, cudaStream_t st);
+// dwte[tok[m]] += dx[m] (deterministic fixed-point scatter), dwpe (=/+=) sum_b dx
+int embed_bwd(int f32, const int32_t* tok, const void* dx, float* dwte, float* dwpe,
+              long long* acc, uint8_t* touched, int M, int T, int d, int V, int wpe_accumulate,
+              cudaStream_t st);
+// AdamW over the flat buffer with the decay mask derived from the layout.
+struct AdamArgs {
+  float lr, beta1, beta2, eps, wd, bc1, bc2;
+};
+struct LayoutDims {
+  long V, T, d, L;
+};
+int adamw(float* p, const float* g, float* m, float* v, uint16_t* shadow, size_t n,
+          const LayoutDims& ld, const AdamArgs& a, cudaStream_t st);
+int init_params(float* p, size_t n, const LayoutDims& ld, uint64_t seed, cudaStream_t st);
+int cast_shadow(const float* p, uint16_t* shadow, size_t n, cudaStream_t st);
+int fill_zero(void* p, size_t bytes, cudaStream_t st);
+int f32_to_act(int f32, const float* src, void* dst, long n, float scale, cudaStream_t st);

@@ -1,0 +1,698 @@
+// Bandwidth-bound kernels of the GPT-2 step: token + position embedding and
+// its (tied, deterministic) backward scatter, LayerNorm forward/backward,
+// bias-gradient column sums, the cross-entropy over the padded vocabulary,
+// the loss mean, AdamW, and the initialisation.
+//
+// All accesses are 16-byte vectors along the feature dimension; row
+// reductions use warp shuffles; every cross-row reduction is a fixed-order
+// two-level sum (per-block partials, then a column reduction), so repeated
+// runs give bitwise-identical results.
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+template <typename T>
+struct Vec;  // one 16-byte chunk
+template <>
+struct Vec<bf16> {
+  static constexpr int N = 8;
+  DEVI static void load(const bf16* p, float (&f)[8]) {
+    uint4 u = *reinterpret_cast<const uint4*>(p);
+    f[0] = bf16lo(u.x); f[1] = bf16hi(u.x); f[2] = bf16lo(u.y); f[3] = bf16hi(u.y);
+    f[4] = bf16lo(u.z); f[5] = bf16hi(u.z); f[6] = bf16lo(u.w); f[7] = bf16hi(u.w);
+  }
+  DEVI static void store(bf16* p, const float (&f)[8]) {
+    uint4 u;
+    u.x = pack_bf16x2(f[0], f[1]); u.y = pack_bf16x2(f[2], f[3]);
+    u.z = pack_bf16x2(f[4], f[5]); u.w = pack_bf16x2(f[6], f[7]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  DEVI static void load(const float* p, float (&f)[4]) {
+    float4 u = *reinterpret_cast<const float4*>(p);
+    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+  }
+  DEVI static void store(float* p, const float (&f)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+  }
+};
+
+// ------------------------------------------------------------- embedding --
+
+// x[m] = wte[tok[m]] + wpe[m mod T]; one warp per row.
+template <typename T>
+__global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const T* __restrict__ wte,
+                                 const T* __restrict__ wpe, T* __restrict__ x, int M, int Tn, int d,
+                                 int vocab_real, int* err) {
+  constexpr int VN = Vec<T>::N;
+  const int m = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (m >= M) return;
+  int id = tok[m];
+  if (id < 0 || id >= vocab_real) {
+    if (lane == 0) atomicOr(err, DEV_ERR_TOKEN);
+    id = 0;
+  }
+  const T* a = wte + (long)id * d;
+  const T* p = wpe + (long)(m % Tn) * d;
+  T* o = x + (long)m * d;
+  for (int c = lane * VN; c < d; c += 32 * VN) {
+    float fa[VN], fb[VN];
+    Vec<T>::load(a + c, fa);
+    Vec<T>::load(p + c, fb);
+#pragma unroll
+    for (int j = 0; j < VN; ++j) fa[j] += fb[j];
+    Vec<T>::store(o + c, fa);
+  }
+}
+
+// Deterministic scatter-add of dx rows into the tied wte gradient: each value
+// is rounded once to a 2^-32 fixed-point integer and added with 64-bit
+// integer atomics, which are order-independent; then the touched rows are
+// converted back and added to dwte (and the accumulator is re-zeroed).
+#define FIX_SCALE 4294967296.0
+
+template <typename T>
+__global__ void embed_scatter_kernel(const int32_t* __restrict__ tok, const T* __restrict__ dx,
+                                     unsigned long long* __restrict__ acc, uint8_t* __restrict__ touched,
+                                     int M, int d, int V) {
+  long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
+  if (i >= (long)M * d) return;
+  const int m = (int)(i / d), c = (int)(i % d);
+  int id = tok[m];
+  if (id < 0 || id >= V) id = 0;
+  double v = (double)to_f(dx[i]) * FIX_SCALE;
+  v = fmin(fmax(v, -9.2e18), 9.2e18);
+  atomicAdd(acc + (long)id * d + c, (unsigned long long)__double2ll_rn(v));
+  if (c == 0) touched[id] = 1;
+}
+
+__global__ void embed_convert_kernel(unsigned long long* __restrict__ acc, uint8_t* __restrict__ touched,
+                                     float* __restrict__ dwte, int V, int d) {
+  const int v = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (v >= V || !touched[v]) return;
+  unsigned long long* a = acc + (long)v * d;
+  float* g = dwte + (long)v * d;
+  for (int c = lane; c < d; c += 32) {
+    long long q = (long long)a[c];
+    g[c] += (float)((double)q / FIX_SCALE);
+    a[c] = 0ull;
+  }
+  __syncwarp();
+  if (lane == 0) touched[v] = 0;
+}
+
+// dwpe[t] = (accumulate ? dwpe[t] : 0) + sum_b dx[b, t]   (fixed order in b)
+template <typename T>
+__global__ void wpe_grad_kernel(const T* __restrict__ dx, float* __restrict__ dwpe, int B, int Tn, int d,
+                                int accumulate) {
+  long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
+  if (i >= (long)Tn * d) return;
+  float s = 0.f;
+  for (int b = 0; b < B; ++b) s += to_f(dx[(long)b * Tn * d + i]);
+  dwpe[i] = (accumulate ? dwpe[i] : 0.f) + s;
+}
+
+// ------------------------------------------------------------- LayerNorm --
+// y = (x - mean) * rstd * g + b, mean/var over the row, var biased, eps 1e-5.
+// One warp per row; NC = 16-byte chunks per lane (row cached in registers).
+
+template <typename T, int NC>
+__global__ void ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ g, const T* __restrict__ b,
+                              T* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd, int M,
+                              int d) {
+  constexpr int VN = Vec<T>::N;
+  const int m = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (m >= M) return;
+  const T* xr = x + (long)m * d;
+  float v[NC][VN];
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    const int c = (lane + 32 * k) * VN;
+    if (c < d) {
+      Vec<T>::load(xr + c, v[k]);
+#pragma unroll
+      for (int j = 0; j < VN; ++j) s += v[k][j];
+    }
+  }
+  const float mu = warp_sum(s) / d;
+  float q = 0.f;
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    const int c = (lane + 32 * k) * VN;
+    if (c < d) {
+#pragma unroll
+      for (int j = 0; j < VN; ++j) {
+        float t = v[k][j] - mu;
+        q += t * t;
+      }
+    }
+  }
+  const float rs = rsqrtf(warp_sum(q) / d + 1e-5f);
+  T* yr = y + (long)m * d;
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    const int c = (lane + 32 * k) * VN;
+    if (c < d) {
+      float gg[VN], bb[VN], o[VN];
+      Vec<T>::load(g + c, gg);
+      Vec<T>::load(b + c, bb);
+#pragma unroll
+      for (int j = 0; j < VN; ++j) o[j] = (v[k][j] - mu) * rs * gg[j] + bb[j];
+      Vec<T>::store(yr + c, o);
+    }
+  }
+  if (lane == 0) {
+    mean[m] = mu;
+    rstd[m] = rs;
+  }
+}
+
+// dx = rstd * (dxhat - mean(dxhat) - xhat * mean(dxhat * xhat)), dxhat = dy * g;
+// dres = (init ? 0 : dres) + dx.  dgamma += dy * xhat, dbeta += dy, reduced in a
+// fixed order over the CTA's rows into part[blockIdx.x][0:d] and [d:2d].
+constexpr int LNB_WARPS = 8;
+constexpr int LNB_ROWS_PER_WARP = 16;
+constexpr int LNB_ROWS = LNB_WARPS * LNB_ROWS_PER_WARP;
+
+template <typename T, int NC>
+__global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x,
+                                                     const float* __restrict__ mean,
+                                                     const float* __restrict__ rstd, const T* __restrict__ g,
+                                                     T* __restrict__ dres, int dres_init,
+                                                     float* __restrict__ part, int M, int d) {
+  constexpr int VN = Vec<T>::N;
+  extern __shared__ float red[];  // [2d]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float gg[NC][VN], dg[NC][VN], db[NC][VN];
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    const int c = (lane + 32 * k) * VN;
+#pragma unroll
+    for (int j = 0; j < VN; ++j) dg[k][j] = db[k][j] = 0.f;
+    if (c < d) Vec<T>::load(g + c, gg[k]);
+  }
+  const int row0 = blockIdx.x * LNB_ROWS + warp * LNB_ROWS_PER_WARP;
+  for (int r = 0; r < LNB_ROWS_PER_WARP; ++r) {
+    const int m = row0 + r;
+    if (m >= M) break;
+    const float mu = mean[m], rs = rstd[m];
+    float xv[NC][VN], dv[NC][VN];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = (lane + 32 * k) * VN;
+      if (c < d) {
+        Vec<T>::load(x + (long)m * d + c, xv[k]);
+        Vec<T>::load(dy + (long)m * d + c, dv[k]);
+#pragma unroll
+        for (int j = 0; j < VN; ++j) {
+          const float xh = (xv[k][j] - mu) * rs;
+          xv[k][j] = xh;
+          const float gh = dv[k][j] * gg[k][j];
+          s1 += gh;
+          s2 += gh * xh;
+          dg[k][j] += dv[k][j] * xh;
+          db[k][j] += dv[k][j];
+        }
+      }
+    }
+    s1 = warp_sum(s1) / d;
+    s2 = warp_sum(s2) / d;
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = (lane + 32 * k) * VN;
+      if (c < d) {
+        float o[VN];
+        if (!dres_init) {
+          Vec<T>::load(dres + (long)m * d + c, o);
+        } else {
+#pragma unroll
+          for (int j = 0; j < VN; ++j) o[j] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < VN; ++j) o[j] += rs * (dv[k][j] * gg[k][j] - s1 - xv[k][j] * s2);
+        Vec<T>::store(dres + (long)m * d + c, o);
+      }
+    }
+  }
+  // fixed-order reduction over the CTA's warps
+  for (int w = 0; w < LNB_WARPS; ++w) {
+    if (warp == w) {
+#pragma unroll
+      for (int k = 0; k < NC; ++k) {
+        const int c = (lane + 32 * k) * VN;
+        if (c < d) {
+#pragma unroll
+          for (int j = 0; j < VN; ++j) {
+            if (w == 0) {
+              red[c + j] = dg[k][j];
+              red[d + c + j] = db[k][j];
+            } else {
+              red[c + j] += dg[k][j];
+              red[d + c + j] += db[k][j];
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+  for (int i = threadIdx.x; i < 2 * d; i += blockDim.x) part[(long)blockIdx.x * 2 * d + i] = red[i];
+}
+
+// grad[j] = beta * grad[j] + sum_r part[r, j] (r ascending); 8 row slices per
+// column reduced in a fixed order.
+__global__ void reduce_rows_kernel(const float* __restrict__ part, int nrows, int n, float* __restrict__ grad,
+                                   float beta) {
+  __shared__ float sm[8][33];
+  const int cx = threadIdx.x & 31, ry = threadIdx.x >> 5;
+  const int j = blockIdx.x * 32 + cx;
+  float s = 0.f;
+  if (j < n)
+    for (int r = ry; r < nrows; r += 8) s += part[(long)r * n + j];
+  sm[ry][cx] = s;
+  __syncthreads();
+  if (ry == 0 && j < n) {
+    float t = sm[0][cx];
+    for (int k = 1; k < 8; ++k) t += sm[k][cx];
+    grad[j] = (beta != 0.f ? beta * grad[j] : 0.f) + t;
+  }
+}
+
+// Column sums of x[M, N] over blocks of 128 rows -> part[rowblock, N].
+constexpr int CS_ROWS = 128;
+
+template <typename T>
+__global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ x, int M, int N,
+                                                     float* __restrict__ part) {
+  constexpr int VN = Vec<T>::N;
+  __shared__ float red[8][32 * VN];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = (blockIdx.x * 32 + lane) * VN;
+  const int r0 = blockIdx.y * CS_ROWS;
+  float s[VN];
+#pragma unroll
+  for (int j = 0; j < VN; ++j) s[j] = 0.f;
+  if (c < N) {
+    for (int r = r0 + warp; r < min(r0 + CS_ROWS, M); r += 8) {
+      float f[VN];
+      Vec<T>::load(x + (long)r * N + c, f);
+#pragma unroll
+      for (int j = 0; j < VN; ++j) s[j] += f[j];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < VN; ++j) red[warp][lane * VN + j] = s[j];
+  __syncthreads();
+  for (int i = threadIdx.x; i < 32 * VN; i += 256) {
+    const int col = blockIdx.x * 32 * VN + i;
+    if (col < N) {
+      float t = red[0][i];
+      for (int w = 1; w < 8; ++w) t += red[w][i];
+      part[(long)blockIdx.y * N + col] = t;
+    }
+  }
+}
+
+// ---------------------------------------------------------- cross-entropy --
+// Row m: lse = log sum_v exp(z_v) over all V (padded) ids; loss = lse - z[y];
+// then, in place, dz_v = exp(z_v - lse) - [v == y] (unscaled; the backward
+// GEMMs apply grad_scale / M).
+template <typename T>
+__global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const int32_t* __restrict__ tgt,
+                                                 float* __restrict__ loss_rows, int V, int vocab_real,
+                                                 int* err) {
+  constexpr int VN = Vec<T>::N;
+  __shared__ float sm_m[256], sm_s[256];
+  const int m = blockIdx.x;
+  T* z = logits + (long)m * V;
+  float mx = -INFINITY, sum = 0.f;
+  for (int c = threadIdx.x * VN; c < V; c += 256 * VN) {
+    float f[VN];
+    Vec<T>::load(z + c, f);
+    float lm = f[0];
+#pragma unroll
+    for (int j = 1; j < VN; ++j) lm = fmaxf(lm, f[j]);
+    if (lm > mx) {
+      sum *= exp2f((mx - lm) * 1.4426950408889634f);
+      mx = lm;
+    }
+#pragma unroll
+    for (int j = 0; j < VN; ++j) sum += exp2f((f[j] - mx) * 1.4426950408889634f);
+  }
+  sm_m[threadIdx.x] = mx;
+  sm_s[threadIdx.x] = sum;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) {
+      float m1 = sm_m[threadIdx.x], m2 = sm_m[threadIdx.x + o];
+      float s1 = sm_s[threadIdx.x], s2 = sm_s[threadIdx.x + o];
+      float mm = fmaxf(m1, m2);
+      float ss = (m1 == -INFINITY ? 0.f : s1 * expf(m1 - mm)) + (m2 == -INFINITY ? 0.f : s2 * expf(m2 - mm));
+      sm_m[threadIdx.x] = mm;
+      sm_s[threadIdx.x] = ss;
+    }
+    __syncthreads();
+  }
+  const float lse = sm_m[0] + logf(sm_s[0]);
+  int y = tgt[m];
+  if (y < 0 || y >= vocab_real) {
+    if (threadIdx.x == 0) atomicOr(err, DEV_ERR_TOKEN);
+    y = 0;
+  }
+  const float zy = to_f(z[y]);
+  __syncthreads();  // every thread has read z[y] before it is overwritten
+  if (threadIdx.x == 0) loss_rows[m] = lse - zy;
+  for (int c = threadIdx.x * VN; c < V; c += 256 * VN) {
+    float f[VN];
+    Vec<T>::load(z + c, f);
+#pragma unroll
+    for (int j = 0; j < VN; ++j) f[j] = __expf(f[j] - lse) - (c + j == y ? 1.f : 0.f);
+    Vec<T>::store(z + c, f);
+  }
+}
+
+// loss = mean(loss_rows), fixed-order tree; flags a non-finite result.
+__global__ void loss_mean_kernel(const float* __restrict__ rows, int M, float* __restrict__ loss, int* err) {
+  __shared__ float sm[1024];
+  float s = 0.f;
+  for (int i = threadIdx.x; i < M; i += 1024) s += rows[i];
+  sm[threadIdx.x] = s;
+  __syncthreads();
+  for (int o = 512; o > 0; o >>= 1) {
+    if (threadIdx.x < o) sm[threadIdx.x] += sm[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    float v = sm[0] / M;
+    *loss = v;
+    if (!isfinite(v)) atomicOr(err, DEV_ERR_NONFINITE);
+  }
+}
+
+// ---------------------------------------------------------------- AdamW --
+
+// Which flat-layout elements are 2-D weights (wte, wpe, w_qkv, w_o, w_fc,
+// w_mp): those get weight decay and, at init, N(0, std) draws.
+// Returns 0 = 1-D tensor, 1 = 2-D weight, 2 = residual projection (w_o, w_mp);
+// *one = 1 for LayerNorm gains.
+DEVI int tensor_kind(long i, const LayoutDims& L, int* one) {
+  const long d = L.d;
+  *one = 0;
+  const long emb = (L.V + L.T) * d;
+  if (i < emb) return 1;
+  const long per = 12 * d * d + 13 * d;
+  const long j = i - emb;
+  if (j >= L.L * per) {  // lnf_g, lnf_b
+    *one = (j - L.L * per) < d;
+    return 0;
+  }
+  const long r = j % per;
+  long o = d;
+  if (r < o) { *one = 1; return 0; }  // ln1_g
+  o += d;
+  if (r < o) return 0;                // ln1_b
+  o += 3 * d * d;
+  if (r < o) return 1;                // w_qkv
+  o += 3 * d;
+  if (r < o) return 0;                // b_qkv
+  o += d * d;
+  if (r < o) return 2;                // w_o
+  o += d;
+  if (r < o) return 0;                // b_o
+  o += d;
+  if (r < o) { *one = 1; return 0; }  // ln2_g
+  o += d;
+  if (r < o) return 0;                // ln2_b
+  o += 4 * d * d;
+  if (r < o) return 1;                // w_fc
+  o += 4 * d;
+  if (r < o) return 0;                // b_fc
+  o += 4 * d * d;
+  if (r < o) return 2;                // w_mp
+  return 0;                           // b_mp
+}
+
+__global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
+                             float* __restrict__ v, uint16_t* __restrict__ shadow, long n4, LayoutDims L,
+                             AdamArgs a) {
+  for (long i4 = blockIdx.x * (long)blockDim.x + threadIdx.x; i4 < n4; i4 += (long)gridDim.x * blockDim.x) {
+    const long i = i4 * 4;
+    int one;
+    const bool decay = tensor_kind(i, L, &one) != 0;
+    float4 pp = reinterpret_cast<float4*>(p)[i4];
+    const float4 gg = reinterpret_cast<const float4*>(g)[i4];
+    float4 mm = reinterpret_cast<float4*>(m)[i4];
+    float4 vv = reinterpret_cast<float4*>(v)[i4];
+    const float dec = decay ? 1.f - a.lr * a.wd : 1.f;
+    float* P = &pp.x;
+    const float* G = &gg.x;
+    float* Mm = &mm.x;
+    float* Vv = &vv.x;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      Mm[j] = a.beta1 * Mm[j] + (1.f - a.beta1) * G[j];
+      Vv[j] = a.beta2 * Vv[j] + (1.f - a.beta2) * G[j] * G[j];
+      const float mh = Mm[j] / a.bc1;
+      const float vh = Vv[j] / a.bc2;
+      P[j] = P[j] * dec - a.lr * mh / (sqrtf(vh) + a.eps);
+    }
+    reinterpret_cast<float4*>(p)[i4] = pp;
+    reinterpret_cast<float4*>(m)[i4] = mm;
+    reinterpret_cast<float4*>(v)[i4] = vv;
+    if (shadow) {
+      uint2 u = make_uint2(pack_bf16x2(pp.x, pp.y), pack_bf16x2(pp.z, pp.w));
+      reinterpret_cast<uint2*>(shadow)[i4] = u;
+    }
+  }
+}
+
+// --------------------------------------------------------- initialisation --
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw: "Parallel random numbers: as easy
+// as 1, 2, 3", SC'11): 10 rounds of two 32x32->64 multiplies with a Weyl key
+// schedule; counter = element index, key = seed.
+DEVI void philox4x32_10(uint32_t (&c)[4], uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t lo0 = 0xD2511F53u * c[0], hi0 = __umulhi(0xD2511F53u, c[0]);
+    const uint32_t lo1 = 0xCD9E8D57u * c[2], hi1 = __umulhi(0xCD9E8D57u, c[2]);
+    const uint32_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+    c[0] = n0; c[1] = lo1; c[2] = n2; c[3] = lo0;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+}
+
+__global__ void init_kernel(float* __restrict__ p, long n, LayoutDims L, uint64_t seed) {
+  const float std_w = 0.02f;
+  const float std_proj = 0.02f / sqrtf(2.f * (float)L.L);
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+    int one;
+    const int kind = tensor_kind(i, L, &one);
+    float val;
+    if (kind == 0) {
+      val = one ? 1.f : 0.f;
+    } else {
+      uint32_t c[4] = {(uint32_t)i, (uint32_t)((uint64_t)i >> 32), 0u, 0u};
+      philox4x32_10(c, (uint32_t)seed, (uint32_t)(seed >> 32));
+      // Box-Muller on two uniforms in (0, 1]
+      const float u1 = ((float)c[0] + 1.f) * 2.3283064365386963e-10f;
+      const float u2 = (float)c[1] * 2.3283064365386963e-10f;
+      const float z = sqrtf(-2.f * logf(fminf(u1, 1.f))) * cospif(2.f * u2);
+      val = z * (kind == 2 ? std_proj : std_w);
+    }
+    p[i] = val;
+  }
+}
+
+__global__ void cast_shadow_kernel(const float* __restrict__ p, uint16_t* __restrict__ s, long n4) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+    float4 v = reinterpret_cast<const float4*>(p)[i];
+    reinterpret_cast<uint2*>(s)[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
+}
+
+int grid_for(long n, int threads) {
+  long b = (n + threads - 1) / threads;
+  long cap = (long)num_sms() * 16;
+  return (int)(b < cap ? (b < 1 ? 1 : b) : cap);
+}
+
+template <typename T, int NC>
+void ln_fwd_launch(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int M,
+                   int d, cudaStream_t st) {
+  ln_fwd_kernel<T, NC><<<(M + 7) / 8, 256, 0, st>>>((const T*)x, (const T*)g, (const T*)b, (T*)y, mean, rstd,
+                                                    M, d);
+}
+
+template <typename T>
+int ln_fwd_dispatch(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int M,
+                    int d, cudaStream_t st) {
+  const int nc = (d / Vec<T>::N + 31) / 32;
+  switch (nc) {
+    case 1: ln_fwd_launch<T, 1>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 2: ln_fwd_launch<T, 2>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 3: ln_fwd_launch<T, 3>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 4: ln_fwd_launch<T, 4>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 5: ln_fwd_launch<T, 5>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 6: ln_fwd_launch<T, 6>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 7: ln_fwd_launch<T, 7>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 8: ln_fwd_launch<T, 8>(x, g, b, y, mean, rstd, M, d, st); break;
+    default: return GPT2_ERR_UNSUPPORTED_SHAPE;
+  }
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+template <typename T, int NC>
+void ln_bwd_launch(const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
+                   void* dres, int init, float* part, int M, int d, cudaStream_t st) {
+  ln_bwd_kernel<T, NC><<<(M + LNB_ROWS - 1) / LNB_ROWS, 256, 2 * d * sizeof(float), st>>>(
+      (const T*)dy, (const T*)x, mean, rstd, (const T*)g, (T*)dres, init, part, M, d);
+}
+
+template <typename T>
+int ln_bwd_dispatch(const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
+                    void* dres, int init, float* part, int M, int d, cudaStream_t st) {
+  const int nc = (d / Vec<T>::N + 31) / 32;
+  switch (nc) {
+    case 1: ln_bwd_launch<T, 1>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
+    case 2: ln_bwd_launch<T, 2>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
+    case 3: ln_bwd_launch<T, 3>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
+    case 4: ln_bwd_launch<T, 4>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
+    case 5: ln_bwd_launch<T, 5>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
+    case 6: ln_bwd_launch<T, 6>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
+    case 7: ln_bwd_launch<T, 7>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
+    case 8: ln_bwd_launch<T, 8>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
+    default: return GPT2_ERR_UNSUPPORTED_SHAPE;
+  }
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------ launchers --
+
+int embed_fwd(int f32, const int32_t* tok, const void* wte, const void* wpe, void* x, int M, int T, int d,
+              int vocab_real, int* err, cudaStream_t st) {
+  const int blocks = (M + 7) / 8;
+  if (f32)
+    embed_fwd_kernel<float><<<blocks, 256, 0, st>>>(tok, (const float*)wte, (const float*)wpe, (float*)x, M, T,
+                                                    d, vocab_real, err);
+  else
+    embed_fwd_kernel<bf16><<<blocks, 256, 0, st>>>(tok, (const bf16*)wte, (const bf16*)wpe, (bf16*)x, M, T, d,
+                                                   vocab_real, err);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int layernorm_fwd(int f32, const void* x, const void* g, const void* b, void* y, float* mean, float* rstd,
+                  int M, int d, cudaStream_t st) {
+  return f32 ? ln_fwd_dispatch<float>(x, g, b, y, mean, rstd, M, d, st)
+             : ln_fwd_dispatch<bf16>(x, g, b, y, mean, rstd, M, d, st);
+}
+
+size_t layernorm_bwd_part_floats(int M, int d) { return (size_t)((M + LNB_ROWS - 1) / LNB_ROWS) * 2 * d; }
+
+int layernorm_bwd(int f32, const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
+                  void* dres, int dres_init, float* part, int* nblk, int M, int d, cudaStream_t st) {
+  *nblk = (M + LNB_ROWS - 1) / LNB_ROWS;
+  return f32 ? ln_bwd_dispatch<float>(dy, x, mean, rstd, g, dres, dres_init, part, M, d, st)
+             : ln_bwd_dispatch<bf16>(dy, x, mean, rstd, g, dres, dres_init, part, M, d, st);
+}
+
+int reduce_rows_f32(const float* part, int nrows, int n, float* grad, float beta, cudaStream_t st) {
+  reduce_rows_kernel<<<(n + 31) / 32, 256, 0, st>>>(part, nrows, n, grad, beta);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+size_t colsum_part_floats(int M, int N) { return (size_t)((M + CS_ROWS - 1) / CS_ROWS) * N; }
+
+int colsum_partial(int f32, const void* x, int M, int N, float* part, int* nblk, cudaStream_t st) {
+  *nblk = (M + CS_ROWS - 1) / CS_ROWS;
+  const int vn = f32 ? 4 : 8;
+  dim3 grid((N + 32 * vn - 1) / (32 * vn), *nblk);
+  if (f32)
+    colsum_kernel<float><<<grid, 256, 0, st>>>((const float*)x, M, N, part);
+  else
+    colsum_kernel<bf16><<<grid, 256, 0, st>>>((const bf16*)x, M, N, part);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, int V, int vocab_real, int* err,
+           cudaStream_t st) {
+  if (f32)
+    ce_kernel<float><<<M, 256, 0, st>>>((float*)logits, tgt, loss_rows, V, vocab_real, err);
+  else
+    ce_kernel<bf16><<<M, 256, 0, st>>>((bf16*)logits, tgt, loss_rows, V, vocab_real, err);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int loss_mean(const float* loss_rows, int M, float* loss, int* err, cudaStream_t st) {
+  loss_mean_kernel<<<1, 1024, 0, st>>>(loss_rows, M, loss, err);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int embed_bwd(int f32, const int32_t* tok, const void* dx, float* dwte, float* dwpe, long long* acc,
+              uint8_t* touched, int M, int T, int d, int V, int wpe_accumulate, cudaStream_t st) {
+  const long n = (long)M * d;
+  unsigned long long* a = reinterpret_cast<unsigned long long*>(acc);
+  if (f32)
+    embed_scatter_kernel<float><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(tok, (const float*)dx, a, touched,
+                                                                             M, d, V);
+  else
+    embed_scatter_kernel<bf16><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(tok, (const bf16*)dx, a, touched, M,
+                                                                            d, V);
+  LAUNCH_CHECK();
+  embed_convert_kernel<<<(V + 7) / 8, 256, 0, st>>>(a, touched, dwte, V, d);
+  LAUNCH_CHECK();
+  const long tn = (long)T * d;
+  const int B = M / T;
+  if (f32)
+    wpe_grad_kernel<float><<<(unsigned)((tn + 255) / 256), 256, 0, st>>>((const float*)dx, dwpe, B, T, d,
+                                                                         wpe_accumulate);
+  else
+    wpe_grad_kernel<bf16><<<(unsigned)((tn + 255) / 256), 256, 0, st>>>((const bf16*)dx, dwpe, B, T, d,
+                                                                        wpe_accumulate);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int adamw(float* p, const float* g, float* m, float* v, uint16_t* shadow, size_t n, const LayoutDims& ld,
+          const AdamArgs& a, cudaStream_t st) {
+  const long n4 = (long)(n / 4);
+  adamw_kernel<<<grid_for(n4, 256), 256, 0, st>>>(p, g, m, v, shadow, n4, ld, a);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int init_params(float* p, size_t n, const LayoutDims& ld, uint64_t seed, cudaStream_t st) {
+  init_kernel<<<grid_for((long)n, 256), 256, 0, st>>>(p, (long)n, ld, seed);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int cast_shadow(const float* p, uint16_t* shadow, size_t n, cudaStream_t st) {
+  const long n4 = (long)(n / 4);
+  cast_shadow_kernel<<<grid_for(n4, 256), 256, 0, st>>>(p, shadow, n4);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int fill_zero(void* p, size_t bytes, cudaStream_t st) {
+  CUDA_TRY(cudaMemsetAsync(p, 0, bytes, st));
+  return GPT2_OK;
+}

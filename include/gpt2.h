@@ -1,0 +1,201 @@
+/*
+ * gpt2.h -- C ABI of libgpt2.so: one GPT-2 pretraining step on one B200.
+ *
+ * The step is the one the GPT-2 pages describe: "Criei GPT-2 do zero com uma
+ * RTX 4090" (section "Configuração do treinamento": GPT-2 small, micro-batch
+ * 16x1024, 32x gradient accumulation, vocabulary padded 50257 -> 50304) and
+ * "Pré-treinar um LLM: dados, compute, leis de escala e custo" (opening
+ * section: next-token cross-entropy optimised by AdamW; compute section:
+ * forward 2N, backward two matmul-sized gradients per layer; memory section:
+ * fp32 weight, gradient, m and v).  Model: pre-LayerNorm decoder blocks with
+ * learned positions, causal multi-head attention, GELU(tanh) MLP, LM head
+ * tied to the token embedding; mean cross-entropy over all B*T positions;
+ * decoupled-weight-decay AdamW with fp32 master weights.
+ *
+ * Conventions for every function below
+ * - Ownership: the caller allocates and owns every device buffer (the
+ *   parameters, gradients, AdamW moments and one workspace).  The library
+ *   allocates only its small host-side context in gpt2_create.
+ * - Pointers: device pointers unless a parameter says "host".  Buffers must be
+ *   16-byte aligned.  Token / target ids are int32, row-major [batch, n_ctx].
+ * - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).  Every
+ *   call except gpt2_get_status, gpt2_step_host and gpt2_create/destroy is
+ *   asynchronous on that stream and returns after enqueueing its kernels.
+ * - Errors: 0 on success, a negative GPT2_ERR_* code otherwise.  Argument and
+ *   shape errors are detected on the host before anything is enqueued.
+ *   Conditions only the device can see (an id outside [0, vocab_real), a
+ *   non-finite loss, a bounded device wait that ran out) are latched in a
+ *   device word and returned by the next gpt2_get_status.  No kernel traps or
+ *   asserts.
+ * - Precision: mode 0 computes in bf16 on tensor cores with fp32 accumulation
+ *   (activations bf16; master weights, gradients and AdamW state fp32); mode 1
+ *   is a correctness mode that computes everything in fp32 on CUDA cores.
+ *
+ * Flat parameter layout (fp32 master, fp32 grad, m, v and the bf16 shadow all
+ * share it; offsets in elements):
+ *   wte[V,d], wpe[n_ctx,d], then for each layer
+ *   ln1_g[d], ln1_b[d], w_qkv[3d,d], b_qkv[3d], w_o[d,d], b_o[d],
+ *   ln2_g[d], ln2_b[d], w_fc[4d,d], b_fc[4d], w_mp[d,4d], b_mp[d],
+ *   and finally lnf_g[d], lnf_b[d].
+ * Weights are [out, in] row-major (y = x W^T + b).  q, k, v are consecutive
+ * d-column blocks of the QKV output; head h owns columns [h*hd, (h+1)*hd) of
+ * each block, hd = d / n_head.
+ */
+#ifndef GPT2_B200_H
+#define GPT2_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct gpt2_ctx gpt2_ctx;
+
+enum {
+  GPT2_OK = 0,
+  GPT2_ERR_INVALID_ARG = -1,      /* NULL pointer, bad value, misaligned buffer */
+  GPT2_ERR_UNSUPPORTED_SHAPE = -2,/* d % 64, vocab_padded % 128, hd not in {16, 64}, ... */
+  GPT2_ERR_CUDA = -3,             /* a CUDA runtime/driver call failed */
+  GPT2_ERR_BAD_STATE = -4,        /* e.g. gpt2_backward without a preceding forward */
+  GPT2_ERR_TOKEN_RANGE = -5,      /* device: an id outside [0, vocab_real) (clamped to 0) */
+  GPT2_ERR_NONFINITE = -6,        /* device: loss is NaN or Inf */
+  GPT2_ERR_TIMEOUT = -7,          /* device: a bounded pipeline wait ran out */
+  GPT2_ERR_WORKSPACE = -8         /* workspace smaller than gpt2_workspace_bytes */
+};
+
+typedef struct {
+  int n_layer;      /* L */
+  int d_model;      /* d, a multiple of 64 */
+  int n_head;       /* H; head_dim = d / H must be 16 or 64 */
+  int n_ctx;        /* T: sequence length of every batch row; wpe has n_ctx rows */
+  int vocab_real;   /* ids must lie in [0, vocab_real) (50257 for GPT-2) */
+  int vocab_padded; /* V >= vocab_real, a multiple of 128 (50304); the softmax spans all V */
+  int max_batch;    /* largest batch any call will pass */
+  int mode;         /* 0 = bf16 tensor-core compute, 1 = fp32 correctness mode */
+} gpt2_config;
+
+typedef struct {
+  float* master;          /* fp32 [param_count] */
+  uint16_t* shadow;       /* bf16 copy of master [param_count]; may be NULL in mode 1 */
+  float* grad;            /* fp32 [param_count] */
+  float* m;               /* fp32 [param_count], AdamW first moment */
+  float* v;               /* fp32 [param_count], AdamW second moment */
+  void* workspace;        /* device scratch of workspace_bytes bytes */
+  size_t workspace_bytes; /* >= gpt2_workspace_bytes(cfg, cfg->max_batch) */
+} gpt2_buffers;
+
+/* Number of parameters (elements) in the flat layout; 0 for an invalid cfg. */
+size_t gpt2_param_count(const gpt2_config* cfg);
+
+/* Bytes of workspace needed for micro-batches up to `batch` rows: saved
+ * activations of every layer, the bf16 (mode 0) logits/dlogits buffer
+ * [batch*n_ctx, V] and backward scratch.  0 for an invalid cfg. */
+size_t gpt2_workspace_bytes(const gpt2_config* cfg, int batch);
+
+/* Describe tensor `index` (0-based, in layout order) of the flat layout:
+ * its name ("wte", "wpe", "h<l>.<name>", "lnf_g", "lnf_b"), element offset,
+ * rows and cols (cols = 1 for vectors).  *name points to static storage
+ * valid until the next call.  GPT2_ERR_INVALID_ARG past the last tensor. */
+int gpt2_tensor_info(const gpt2_config* cfg, int index, const char** name,
+                     size_t* offset, size_t* rows, size_t* cols);
+
+/* Validate cfg and buffers and create a context bound to them.  Zeroes the
+ * internal scatter accumulator inside the workspace (synchronously).  The
+ * buffers must outlive the context. */
+int gpt2_create(const gpt2_config* cfg, const gpt2_buffers* bufs, gpt2_ctx** out);
+int gpt2_destroy(gpt2_ctx* ctx);
+
+/* GPT-2 initialisation: every 2-D weight (wte, wpe, w_qkv, w_fc) ~ N(0, 0.02^2)
+ * except the two projections into the residual stream (w_o, w_mp) ~
+ * N(0, (0.02/sqrt(2L))^2); biases and LayerNorm shifts 0, LayerNorm gains 1.
+ * Normal draws: Box-Muller on Philox4x32-10 (Salmon et al., SC'11) keyed by
+ * `seed`, counter = element index.  Also zeroes grad, m, v and refreshes
+ * the bf16 shadow. */
+int gpt2_init_params(gpt2_ctx* ctx, uint64_t seed, void* stream);
+
+/* Re-derive the bf16 shadow from the fp32 master (after the caller wrote the
+ * master directly, e.g. when restoring a checkpoint). */
+int gpt2_refresh_shadow(gpt2_ctx* ctx, void* stream);
+
+/* Forward pass and loss.  tokens, targets: device int32 [batch, n_ctx]
+ * (targets[b,t] is the id at t+1 of the stream).  Writes the mean
+ * cross-entropy over batch*n_ctx positions to *loss_dev (device fp32) and
+ * keeps the activations (and the dlogits of this batch) in the workspace for
+ * gpt2_backward.  The ids are copied into the workspace, so the caller's
+ * arrays may be reused as soon as this call's work has run. */
+int gpt2_forward_loss(gpt2_ctx* ctx, const int32_t* tokens, const int32_t* targets,
+                      int batch, float* loss_dev, void* stream);
+
+/* Backward pass of the last forward: grad = (accumulate ? grad : 0)
+ * + grad_scale * d(loss)/d(params).  With k-step gradient accumulation pass
+ * grad_scale = 1/k and accumulate = 0 on the first micro-batch, 1 after.
+ * GPT2_ERR_BAD_STATE if no forward preceded it. */
+int gpt2_backward(gpt2_ctx* ctx, float grad_scale, int accumulate, void* stream);
+
+/* One AdamW step over the whole flat buffer (decoupled weight decay on the
+ * 2-D tensors only; bias-corrected with step counter `step` >= 1):
+ *   p <- p (1 - lr wd);  m <- b1 m + (1-b1) g;  v <- b2 v + (1-b2) g^2
+ *   p <- p - lr (m / (1-b1^step)) / (sqrt(v / (1-b2^step)) + eps)
+ * and refreshes the bf16 shadow. */
+int gpt2_adamw_step(gpt2_ctx* ctx, float lr, float beta1, float beta2, float eps,
+                    float weight_decay, int step, void* stream);
+
+/* grad <- 0. */
+int gpt2_zero_grad(gpt2_ctx* ctx, void* stream);
+
+/* Synchronises `stream`, returns and clears the latched device status
+ * (GPT2_OK, GPT2_ERR_TOKEN_RANGE, GPT2_ERR_NONFINITE or GPT2_ERR_TIMEOUT),
+ * or GPT2_ERR_CUDA if the stream reports an error. */
+int gpt2_get_status(gpt2_ctx* ctx, void* stream);
+
+/* One whole training step from HOST memory: copies tokens/targets (host,
+ * int32 [batch, n_ctx], preferably pinned) to the device, runs forward,
+ * backward (grad_scale 1, accumulate 0) and AdamW, copies the loss back into
+ * *loss_host and synchronises the stream before returning. */
+int gpt2_step_host(gpt2_ctx* ctx, const int32_t* tokens_host, const int32_t* targets_host,
+                   int batch, float* loss_host, float lr, float beta1, float beta2,
+                   float eps, float weight_decay, int step, void* stream);
+
+/* Static text for an error code. */
+const char* gpt2_strerror(int code);
+
+/* ------------------------------------------------------------------------
+ * Single-operation entry points used by the kernel unit tests.  They run the
+ * same kernels the step runs, on caller buffers.
+ * ---------------------------------------------------------------------- */
+
+/* C[M,N] = alpha * sum_k A(m,k) B(n,k)  (+ beta * C when C is fp32).
+ * The linear layers' forward, input-gradient and weight-gradient products of
+ * the compute section are all of this form with different operand majorness.
+ * A: bf16; a_mn_major = 0 -> stored [M, lda] (k contiguous),
+ *                         1 -> stored [K, lda] (m contiguous).
+ * B: bf16; b_mn_major = 0 -> stored [N, ldb], 1 -> stored [K, ldb].
+ * C: c_fp32 = 0 -> bf16 [M, ldc] (beta ignored); 1 -> fp32 [M, ldc].
+ * K must be a multiple of 64; lda, ldb, ldc multiples of 8.
+ * workspace (device, may be NULL) holds split-K partial sums for fp32 C;
+ * bn (0 = auto, 128 or 256) and splits (0 = auto) override the tiling. */
+int gpt2_op_gemm_bf16(const uint16_t* A, int a_mn_major, int lda,
+                      const uint16_t* B, int b_mn_major, int ldb,
+                      void* C, int c_fp32, int ldc, int M, int N, int K,
+                      float alpha, float beta, void* workspace, size_t workspace_bytes,
+                      int bn, int splits, void* stream);
+
+/* Causal attention forward on a packed QKV activation: qkv bf16 [B*T, 3*H*hd]
+ * -> o bf16 [B*T, H*hd], lse fp32 [B, H, T] (natural-log log-sum-exp of the
+ * scaled scores).  hd in {16, 64}. */
+int gpt2_op_attention_fwd_bf16(const uint16_t* qkv, uint16_t* o, float* lse,
+                               int B, int T, int H, int hd, void* stream);
+
+/* Its backward: given do (bf16 [B*T, H*hd]) writes dqkv (bf16 [B*T, 3*H*hd]).
+ * scratch: device fp32, at least B*T*H*hd + B*H*T floats. */
+int gpt2_op_attention_bwd_bf16(const uint16_t* qkv, const uint16_t* o, const float* lse,
+                               const uint16_t* dout, uint16_t* dqkv, float* scratch,
+                               int B, int T, int H, int hd, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPT2_B200_H */

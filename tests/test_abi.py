@@ -1,0 +1,98 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point include/gpt2.h declares, and its host-side logic (parameter layout,
+workspace sizing, argument validation) agrees with the specification the
+oracle implements independently."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decoder_only_transformer_step_b200 as gp
+from decoder_only_transformer_step_b200 import build_lib
+import oracle
+from oracle import flops as FL
+from oracle_fixtures import TINY, GPT2_124M
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build_lib.build()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "gpt2.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gpt2_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    lib = ctypes.CDLL(gp.LIB_PATH)
+    declared = header_functions()
+    assert len(declared) >= 17
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(gp.EXPORTS) == declared
+
+
+def _cfg(oc, max_batch=4, vocab_real=None, mode=0):
+    return gp.make_config(oc.n_layer, oc.d_model, oc.n_head, oc.n_ctx,
+                          vocab_real or oc.vocab, oc.vocab, max_batch, mode)
+
+
+@pytest.mark.parametrize("oc", [TINY, GPT2_124M])
+def test_layout_matches_oracle_spec(oc):
+    cfg = _cfg(oc)
+    assert gp.gpt2_param_count(cfg) == oracle.param_count(oc)
+    lib_tensors = gp.gpt2_tensors(cfg)
+    off = 0
+    shapes = oracle.param_shapes(oc)
+    assert len(lib_tensors) == len(shapes)
+    for (name, o, r, c), (oname, oshape) in zip(lib_tensors, shapes):
+        assert name == oname
+        assert o == off
+        assert (r, c) == (oshape + (1,) if len(oshape) == 1 else oshape)
+        off += r * c
+        assert o % 8 == 0  # every tensor starts 16-byte aligned in the bf16 shadow
+
+
+def test_param_counts_of_named_configs():
+    for mc, n in [(gp.GPT2_124M, 124_475_904), (gp.GPT2_1558M, 1_557_686_400)]:
+        assert gp.gpt2_param_count(mc.c()) == n
+        assert n == FL.n_params_total(mc.n_layer, mc.d_model, mc.vocab_padded, mc.n_ctx)
+
+
+def test_workspace_fits_b200():
+    for mc in (gp.GPT2_124M, gp.GPT2_350M, gp.GPT2_1558M, gp.GPT2_124M_T4096):
+        ws = gp.gpt2_workspace_bytes(mc.c(), mc.max_batch)
+        n = gp.gpt2_param_count(mc.c())
+        total = ws + n * (4 * 4 + 2)
+        assert 0 < total < 170e9, (mc, total / 1e9)
+    assert gp.gpt2_workspace_bytes(gp.GPT2_124M.c(), 2) < gp.gpt2_workspace_bytes(gp.GPT2_124M.c(), 16)
+
+
+def test_invalid_configs_are_rejected_on_host():
+    bad = gp.make_config(2, 64, 3, 64, 512, 512, 4, 0)      # d % heads
+    assert gp.gpt2_param_count(bad) == 0
+    assert gp.gpt2_workspace_bytes(bad, 4) == 0
+    lib = gp._lib()
+    ctx = ctypes.c_void_p()
+    bufs = gp.gpt2_buffers()
+    cfg = gp.make_config(2, 64, 4, 64, 512, 512, 4, 0)
+    # NULL buffers
+    assert lib.gpt2_create(ctypes.byref(cfg), ctypes.byref(bufs), ctypes.byref(ctx)) == -1
+    # d not a multiple of 64 / head_dim unsupported / vocab not a multiple of 128
+    for c in (gp.make_config(2, 96, 4, 64, 512, 512, 4, 0), gp.make_config(2, 128, 4, 64, 512, 512, 4, 0),
+              gp.make_config(2, 64, 4, 64, 500, 500, 4, 0)):
+        fake = gp.gpt2_buffers(16, 16, 16, 16, 16, 16, 1 << 40)
+        assert lib.gpt2_create(ctypes.byref(c), ctypes.byref(fake), ctypes.byref(ctx)) == -2
+    # misaligned pointer
+    fake = gp.gpt2_buffers(16, 16, 24, 16, 16, 16, 1 << 40)
+    assert lib.gpt2_create(ctypes.byref(cfg), ctypes.byref(fake), ctypes.byref(ctx)) == -1
+    # workspace too small
+    fake = gp.gpt2_buffers(16, 16, 16, 16, 16, 16, 1024)
+    assert lib.gpt2_create(ctypes.byref(cfg), ctypes.byref(fake), ctypes.byref(ctx)) == -8
+    assert lib.gpt2_backward(None, ctypes.c_float(1.0), 0, None) == -1
+    assert lib.gpt2_strerror(-5) == b"token or target id out of range"

@@ -1,0 +1,213 @@
+"""Whole-step parity: the CUDA path through the C ABI against the fp64 oracle
+on the same seeded inputs.  Tolerances: loss within 1e-2 relative in bf16
+(1e-4 in the fp32 mode); every parameter gradient with cosine similarity
+>= 0.999 and max|delta| / max|g_ref| <= 2e-2 (a per-element relative error is
+meaningless where g_ref ~ 0); parameters after 10 AdamW steps within 1e-2
+(relative L2 per tensor)."""
+import numpy as np
+import pytest
+import torch
+
+import decoder_only_transformer_step_b200 as gp
+from decoder_only_transformer_step_b200 import inputs
+import oracle
+from oracle import Config, forward, backward, adamw_step, param_shapes
+from oracle_fixtures import TINY, SMALL_124M_L2, params_for
+
+pytestmark = pytest.mark.gpu
+
+
+def make_model(oc: Config, vocab_real, batch, mode):
+    mc = gp.ModelConfig(oc.n_layer, oc.d_model, oc.n_head, oc.n_ctx, vocab_real, oc.vocab, batch, mode)
+    return gp.GPT2(mc)
+
+
+def load_params(model, params, oc):
+    flat32 = oracle.flatten(params, oc).astype(np.float32)
+    model.master.copy_(torch.from_numpy(flat32))
+    model.refresh_shadow()
+    # the oracle sees exactly the fp32 values the GPU holds
+    return oracle.unflatten(flat32.astype(np.float64), oc)
+
+
+def gpu_grads(model, oc):
+    g = model.grad.double().cpu().numpy()
+    return oracle.unflatten(g, oc)
+
+
+def compare_grads(g_gpu, g_ref, cos_min, rel_max):
+    worst = []
+    for n in g_ref:
+        a, r = g_gpu[n].ravel(), g_ref[n].ravel()
+        nr = np.linalg.norm(r)
+        if nr == 0:
+            assert np.abs(a).max() <= 1e-6, n
+            continue
+        cos = float(a @ r / (np.linalg.norm(a) * nr + 1e-300))
+        rel = float(np.abs(a - r).max() / np.abs(r).max())
+        worst.append((n, cos, rel))
+        assert cos >= cos_min and rel <= rel_max, (n, cos, rel)
+    return worst
+
+
+def run_step(model, tok, tgt):
+    tok_d = torch.from_numpy(tok).cuda()
+    tgt_d = torch.from_numpy(tgt).cuda()
+    loss = model.forward_loss(tok_d, tgt_d)
+    model.backward(1.0, 0)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    return float(loss.item())
+
+
+@pytest.mark.parametrize("mode", [1, 0])
+def test_tiny_loss_and_grads(mode):
+    params = params_for(TINY, seed=21)
+    tok, tgt = inputs.uniform_tokens(4, 64, TINY.vocab, seed=22)
+    model = make_model(TINY, TINY.vocab, 4, mode)
+    p32 = load_params(model, params, TINY)
+    loss = run_step(model, tok, tgt)
+    ref_loss, cache = forward(p32, TINY, tok, tgt)
+    ref_g = backward(p32, TINY, cache)
+    tol_loss = 1e-4 if mode == 1 else 1e-2
+    assert abs(loss - ref_loss) <= tol_loss * abs(ref_loss), (loss, ref_loss)
+    if mode == 1:
+        compare_grads(gpu_grads(model, TINY), ref_g, 0.99999, 1e-3)
+    else:
+        compare_grads(gpu_grads(model, TINY), ref_g, 0.999, 2e-2)
+
+
+def test_tiny_ten_adamw_steps():
+    params = params_for(TINY, seed=31)
+    model = make_model(TINY, TINY.vocab, 4, 0)
+    p = load_params(model, params, TINY)
+    m = {n: np.zeros(s) for n, s in param_shapes(TINY)}
+    v = {n: np.zeros(s) for n, s in param_shapes(TINY)}
+    for step in range(1, 11):
+        tok, tgt = inputs.uniform_tokens(4, 64, TINY.vocab, seed=300 + step)
+        loss = run_step(model, tok, tgt)
+        model.adamw_step(step)
+        ref_loss, cache = forward(p, TINY, tok, tgt)
+        g = backward(p, TINY, cache)
+        p, m, v = adamw_step(p, g, m, v, step, TINY)
+        assert abs(loss - ref_loss) <= 1e-2 * abs(ref_loss)
+    torch.cuda.synchronize()
+    got = oracle.unflatten(model.master.double().cpu().numpy(), TINY)
+    for n in p:
+        rel = np.linalg.norm(got[n] - p[n]) / np.linalg.norm(p[n])
+        assert rel <= 1e-2, (n, rel)
+
+
+@pytest.mark.slow
+def test_124m_shaped_two_layers():
+    """d=768, 12 heads, T=1024, V=50304 (production tile paths, padded vocab),
+    two layers, batch 1, Zipf ids."""
+    oc = SMALL_124M_L2
+    params = params_for(oc, seed=41)
+    tok, tgt = inputs.zipf_tokens(1, 1024, seed=42)
+    model = make_model(oc, 50257, 1, 0)
+    p32 = load_params(model, params, oc)
+    loss = run_step(model, tok, tgt)
+    ref_loss, cache = forward(p32, oc, tok, tgt)
+    ref_g = backward(p32, oc, cache)
+    assert abs(loss - ref_loss) <= 1e-2 * abs(ref_loss), (loss, ref_loss)
+    compare_grads(gpu_grads(model, oc), ref_g, 0.999, 2e-2)
+
+
+def test_gradient_accumulation_and_scale():
+    """Two micro-batches with grad_scale 1/2 and accumulate: the sum of the
+    two scaled gradients (fp32 mode, tight)."""
+    params = params_for(TINY, seed=51)
+    model = make_model(TINY, TINY.vocab, 4, 1)
+    p32 = load_params(model, params, TINY)
+    ref = None
+    for k in range(2):
+        tok, tgt = inputs.uniform_tokens(4, 64, TINY.vocab, seed=500 + k)
+        model.forward_loss(torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda())
+        model.backward(0.5, k)
+        _, cache = forward(p32, TINY, tok, tgt)
+        g = backward(p32, TINY, cache, grad_scale=0.5)
+        ref = g if ref is None else {n: ref[n] + g[n] for n in g}
+    torch.cuda.synchronize()
+    compare_grads(gpu_grads(model, TINY), ref, 0.99999, 1e-3)
+
+
+def test_init_params_statistics():
+    model = gp.GPT2(gp.ModelConfig(4, 256, 4, 128, 1000, 1024, 1, 0))
+    model.init_params(seed=7)
+    torch.cuda.synchronize()
+    L = 4
+    for name, off, r, c in model.layout:
+        t = model.master[off:off + r * c].double()
+        short = name.split(".")[-1]
+        if short in ("w_o", "w_mp"):
+            assert abs(t.std().item() - 0.02 / np.sqrt(2 * L)) < 0.0005, name
+        elif c > 1:
+            assert abs(t.std().item() - 0.02) < 0.0005 and abs(t.mean().item()) < 5e-4, name
+        elif short.endswith("_g"):
+            assert torch.all(t == 1.0), name
+        else:
+            assert torch.all(t == 0.0), name
+    assert torch.all(model.grad == 0) and torch.all(model.m == 0) and torch.all(model.v == 0)
+    assert torch.equal(model.shadow, model.master.to(torch.bfloat16))
+    # same seed -> identical; other seed -> different
+    a = model.master.clone()
+    model.init_params(seed=7)
+    assert torch.equal(a, model.master)
+    model.init_params(seed=8)
+    assert not torch.equal(a, model.master)
+
+
+def test_init_loss_near_log_vocab():
+    model = gp.GPT2(gp.ModelConfig(2, 768, 12, 1024, 50257, 50304, 1, 0))
+    model.init_params(seed=0)
+    tok, tgt = inputs.zipf_tokens(1, 1024, seed=1000)
+    loss = model.forward_loss(torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda()).item()
+    assert abs(loss - (np.log(50304) + 0.5 * 0.02 ** 2 * 768)) < 0.15, loss
+
+
+def test_device_errors_are_reported():
+    model = make_model(TINY, 500, 4, 0)
+    model.init_params(seed=1)
+    tok, tgt = inputs.uniform_tokens(4, 64, 500, seed=60)
+    tok[1, 5] = 505                       # >= vocab_real: clamped, flagged
+    model.forward_loss(torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda())
+    assert model.status() == -5
+    assert model.status() == 0            # reading clears it
+    model.master[3] = float("nan")
+    model.refresh_shadow()
+    tok[1, 5] = 3
+    model.forward_loss(torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda())
+    assert model.status() == -6
+    with pytest.raises(gp.Gpt2Error):
+        gp.GPT2(gp.ModelConfig(2, 64, 4, 64, 512, 512, 4, 0)).backward()
+
+
+def test_fp32_mode_is_deterministic():
+    params = params_for(TINY, seed=71)
+    tok, tgt = inputs.uniform_tokens(4, 64, TINY.vocab, seed=72)
+    outs = []
+    for _ in range(2):
+        model = make_model(TINY, TINY.vocab, 4, 1)
+        load_params(model, params, TINY)
+        run_step(model, tok, tgt)
+        outs.append(model.grad.clone())
+    assert torch.equal(outs[0], outs[1])
+
+
+def test_step_host_matches_device_path():
+    params = params_for(TINY, seed=81)
+    tok, tgt = inputs.uniform_tokens(4, 64, TINY.vocab, seed=82)
+    a = make_model(TINY, TINY.vocab, 4, 1)
+    b = make_model(TINY, TINY.vocab, 4, 1)
+    load_params(a, params, TINY)
+    load_params(b, params, TINY)
+    loss_a = run_step(a, tok, tgt)
+    a.adamw_step(1)
+    th = torch.from_numpy(tok).pin_memory()
+    gh = torch.from_numpy(tgt).pin_memory()
+    lh = torch.zeros(1).pin_memory()
+    b.step_host(th, gh, lh, 1)
+    assert abs(lh.item() - loss_a) <= 1e-6 * abs(loss_a)
+    torch.cuda.synchronize()
+    assert (a.master - b.master).abs().max().item() <= 1e-6
