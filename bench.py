@@ -1,0 +1,441 @@
+#!/usr/bin/env python
+"""Throughput of the GPT-2 pretraining step on B200 (tokens/s and MFU).
+
+One step = forward + next-token cross-entropy + backward + AdamW over one
+micro-batch of synthetic Zipf(1.1) token ids (stand-in for FineWeb-Edu, which
+is not available offline), the workload of "Criei GPT-2 do zero com uma RTX
+4090" (section "Configuração do treinamento": GPT-2 small, micro-batch
+16 x 1024, vocabulary 50304).  MFU follows "Pré-treinar um LLM" (compute
+section): (6 N + 12 L T d) FLOPs per token over the dense bf16 peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 124m|350m|1.5b|lc4096]
+    python bench.py --impl reference ...   (the CPU oracle, timed on host cores)
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank trains its
+own micro-batch and gradients are averaged with an NCCL all-reduce before
+AdamW (data parallel, weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "train tokens/s, GPT-2 124M T=1024 bf16 on 1 B200; MFU (6N+attn FLOPs)"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+CONFIGS = {
+    # name: (n_layer, d, heads, T, vocab_real, vocab_padded, micro_batch)
+    "124m": (12, 768, 12, 1024, 50257, 50304, 16),
+    "350m": (24, 1024, 16, 1024, 50257, 50304, 16),
+    "1.5b": (48, 1600, 25, 1024, 50257, 50304, 8),
+    "lc4096": (12, 768, 12, 4096, 50257, 50304, 4),
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def workload_name(name, c):
+    L, d, H, T, Vr, V, B = c
+    return f"GPT-2 {name} (L{L} d{d} H{H}) T={T} micro-batch {B}, vocab {V}, Zipf(1.1) ids"
+
+
+# ------------------------------------------------------------ clock sampler --
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid):
+        self.gpu = gpu_uuid
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- our arm --
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import decoder_only_transformer_step_b200 as gp
+    from decoder_only_transformer_step_b200 import inputs, flops
+    from decoder_only_transformer_step_b200.dp import average_gradients
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    L, d, H, T, Vr, V, B = CONFIGS[args.config]
+    mc = gp.ModelConfig(L, d, H, T, Vr, V, B, 0)
+    model = gp.GPT2(mc)
+    model.init_params(seed=0)
+    M = B * T
+
+    # synthetic inputs, uploaded before timing; a small pool cycled over steps
+    pool = []
+    for s in range(min(4, args.steps + args.warmup)):
+        tok, tgt = inputs.zipf_tokens(B, T, n_ids=Vr, seed=1000 + s + 7919 * rank)
+        pool.append((torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda()))
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        tok, tgt = pool[i % len(pool)]
+        model.forward_loss(tok, tgt)
+        model.backward(1.0, 0)
+        if world > 1:
+            average_gradients(model.grad)
+        model.adamw_step(i + 1)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if model.status() != 0:
+        raise RuntimeError("device status after warm-up: %d" % model.status())
+
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(local_rank).uuid)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = gp.gpt2_kernel_launches()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(uuid) as clocks:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = gp.gpt2_kernel_launches() - launches0
+    ms = e0.elapsed_time(e1)
+    status = model.status()
+    loss = float(model.loss.item())
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    tokens_per_s = world * M * args.steps / (ms / 1e3)
+
+    # end to end through the public API with host buffers (copies inside)
+    tok_h = [torch.from_numpy(inputs.zipf_tokens(B, T, n_ids=Vr, seed=5000 + s + 7919 * rank)[0]).pin_memory()
+             for s in range(2)]
+    tgt_h = [torch.from_numpy(inputs.zipf_tokens(B, T, n_ids=Vr, seed=5000 + s + 7919 * rank)[1]).pin_memory()
+             for s in range(2)]
+    loss_h = torch.zeros(1).pin_memory()
+    e_steps = max(3, args.steps // 2)
+
+    def e2e_step(i):
+        if world == 1:
+            model.step_host(tok_h[i % 2], tgt_h[i % 2], loss_h, args.warmup + args.steps + i + 1)
+        else:
+            tok = tok_h[i % 2].cuda(non_blocking=True)
+            tgt = tgt_h[i % 2].cuda(non_blocking=True)
+            model.forward_loss(tok, tgt)
+            model.backward(1.0, 0)
+            average_gradients(model.grad)
+            model.adamw_step(args.warmup + args.steps + i + 1)
+            loss_h.copy_(model.loss)
+            torch.cuda.synchronize()
+
+    e2e_step(0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(e_steps):
+        e2e_step(i + 1)
+    torch.cuda.synchronize()
+    e2e_s = time.perf_counter() - t0
+    if world > 1:
+        t = torch.tensor([e2e_s], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    e2e_tps = world * M * e_steps / e2e_s
+
+    # dominant kernel: the tied LM-head GEMM [M x V x d], timed alone
+    roof = lm_head_roofline(gp, model, M, V, d, stream)
+
+    peaks, peak_kind = load_peaks()
+    fpt = flops.train_flops_per_token(L, d, V, T, T)
+    result = {
+        "metric": METRIC,
+        "value": round(tokens_per_s, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic Zipf(1.1) token ids over [0, 50257), random-init GPT-2 weights",
+        "config": {"workload": workload_name(args.config, CONFIGS[args.config]), "batch_per_gpu": B,
+                   "seq_len": T, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2: the step's working set (>5 GB) exceeds the 126 MB L2"},
+        "mfu": round(flops.mfu(tokens_per_s / world, fpt, peaks["bf16_tflops"] * 1e12), 4),
+        "mfu_vs_sustained": round(flops.mfu(tokens_per_s / world, fpt, peaks["bf16_tflops_sustained"] * 1e12), 4),
+        "flops_per_token": fpt,
+        "peak_source": peak_kind,
+        "final_loss": round(loss, 4),
+        "device_status": status,
+        "gpu_launches": int(launches),
+        "e2e": {"value": round(e2e_tps, 1), "unit": "tokens/s", "h2d_bytes_per_step": 2 * M * 4,
+                "d2h_bytes_per_step": 4},
+        "roofline": roof,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args.config)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def lm_head_roofline(gp, model, M, V, d, stream):
+    import torch
+    peaks, kind = load_peaks()
+    A = torch.randn(M, d, device="cuda").to(torch.bfloat16)
+    wte = model.view(model.shadow, "wte")
+    C = torch.empty(M, V, dtype=torch.bfloat16, device="cuda")
+    reps = 10
+    for _ in range(3):
+        gp.gpt2_op_gemm_bf16(A, 0, d, wte, 0, d, C, 0, V, M, V, d)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        gp.gpt2_op_gemm_bf16(A, 0, d, wte, 0, d, C, 0, V, M, V, d)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    sec = e0.elapsed_time(e1) / 1e3 / reps
+    flop = 2.0 * M * V * d
+    achieved = flop / sec / 1e12
+    peak = peaks["bf16_tflops"]
+    del A, C
+    return {"kernel": "gemm_tc_kernel<256> (tied LM head, forward: logits = LN_f(x) wte^T)",
+            "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "peak_source": f"{kind} bf16_tflops (burst)",
+            "launch_ms": round(sec * 1e3, 4), "flop_per_launch": flop,
+            "traffic": recorded_traffic("lm_head_gemm")}
+
+
+def recorded_traffic(key):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(key)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["bytes_per_launch"] if sha == rec["source_sha256_16"] else None
+
+
+# ------------------------------------------------------ CPU oracle timing --
+
+def oracle_one_step(config, seed=1000, tokens=None):
+    """One fwd + bwd + AdamW step of the CPU oracle on one sequence of the
+    workload (batch 1, full depth, width and vocabulary; the first `tokens`
+    positions of a T-token stream, all T by default); returns seconds."""
+    import numpy as np
+    import oracle
+    from decoder_only_transformer_step_b200 import inputs
+    L, d, H, T, Vr, V, B = CONFIGS[config]
+    cfg = oracle.Config(L, d, H, T, V)
+    rng = np.random.default_rng(seed)
+    params = {}
+    for n, s in oracle.param_shapes(cfg):
+        params[n] = np.ones(s) if n.endswith("_g") else (0.02 * rng.standard_normal(s) if len(s) == 2 else np.zeros(s))
+    m = {n: np.zeros(s) for n, s in oracle.param_shapes(cfg)}
+    v = {n: np.zeros(s) for n, s in oracle.param_shapes(cfg)}
+    tok, tgt = inputs.zipf_tokens(1, T, n_ids=Vr, seed=seed)
+    if tokens is not None:
+        tok, tgt = tok[:, :tokens], tgt[:, :tokens]
+    t0 = time.perf_counter()
+    oracle.train_step(params, m, v, 1, cfg, tok, tgt)
+    return time.perf_counter() - t0, tok.size
+
+
+def host_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        if info:
+            return int(info[0].get("num_threads") or os.cpu_count())
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_baseline(config):
+    sec, tokens = oracle_one_step(config)
+    return {"value": round(tokens / sec, 2), "unit": "tokens/s", "cores": host_threads(), "kind": "oracle",
+            "sample": f"one full training step (fwd+bwd+AdamW, fp64 numpy) on 1 sequence of {tokens} tokens "
+                      f"of the same model: {sec:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    L, d, H, T, Vr, V, B = CONFIGS[args.config]
+    # warm-up steps of a CPU program only warm caches: at most one is run
+    sample = 256
+    for _ in range(min(args.warmup, 1)):
+        oracle_one_step(args.config, tokens=sample)
+    total, tokens = 0.0, 0
+    for i in range(args.steps):
+        s, t = oracle_one_step(args.config, seed=1000 + i, tokens=sample)
+        total += s
+        tokens += t
+    tps = tokens / total
+    cores = host_threads()
+    sample = (f"each step: one fwd+bwd+AdamW of the fp64 oracle on the first {sample} tokens of one "
+              f"{T}-token sequence (full depth, width and vocabulary)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(tps, 2), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic Zipf(1.1) token ids", "config": {
+            "workload": workload_name(args.config, CONFIGS[args.config]), "batch_per_gpu": B, "seq_len": T,
+            "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(tps, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(tps, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def run_kernel(args):
+    """One kernel of the step on its own, at a chosen token count (small cases
+    for profiler captures): the LM-head GEMM, the attention forward or backward."""
+    import torch
+    import decoder_only_transformer_step_b200 as gp
+    L, d, H, T, Vr, V, B = CONFIGS[args.config]
+    M = args.tokens
+    g = torch.Generator(device="cuda").manual_seed(0)
+    torch.cuda.synchronize()
+    if args.kernel == "lm_head":
+        A = torch.randn(M, d, device="cuda", generator=g).to(torch.bfloat16)
+        W = (0.02 * torch.randn(V, d, device="cuda", generator=g)).to(torch.bfloat16)
+        C = torch.empty(M, V, dtype=torch.bfloat16, device="cuda")
+        fn = lambda: gp.gpt2_op_gemm_bf16(A, 0, d, W, 0, d, C, 0, V, M, V, d)  # noqa: E731
+        flop = 2.0 * M * V * d
+    else:
+        Bn = max(1, M // T)
+        qkv = torch.randn(Bn * T, 3 * d, device="cuda", generator=g).to(torch.bfloat16)
+        o = torch.empty(Bn * T, d, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(Bn, H, T, device="cuda")
+        gp.gpt2_op_attention_fwd_bf16(qkv, o, lse, Bn, T, H, d // H)
+        flop = 2.0 * 2 * Bn * H * T * T * (d // H) / 2
+        if args.kernel == "attn_fwd":
+            fn = lambda: gp.gpt2_op_attention_fwd_bf16(qkv, o, lse, Bn, T, H, d // H)  # noqa: E731
+        else:
+            do = torch.randn(Bn * T, d, device="cuda", generator=g).to(torch.bfloat16)
+            dqkv = torch.empty(Bn * T, 3 * d, dtype=torch.bfloat16, device="cuda")
+            scr = torch.empty(Bn * T * d + Bn * H * T, device="cuda")
+            fn = lambda: gp.gpt2_op_attention_bwd_bf16(qkv, o, lse, do, dqkv, scr, Bn, T, H, d // H)  # noqa: E731
+            flop *= 2.5
+    for _ in range(2):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.reps
+    print(json.dumps({"kernel": args.kernel, "tokens": M, "ms": round(ms, 4),
+                      "tflops": round(flop / ms / 1e9, 1)}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--kernel", choices=["lm_head", "attn_fwd", "attn_bwd"], default=None,
+                    help="time one kernel alone instead of the step (profiler captures)")
+    ap.add_argument("--tokens", type=int, default=4096)
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="124m", choices=sorted(CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.kernel:
+        run_kernel(args)
+    elif args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

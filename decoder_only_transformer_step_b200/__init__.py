@@ -47,6 +47,7 @@ EXPORTS = [
     "gpt2_param_count", "gpt2_workspace_bytes", "gpt2_tensor_info", "gpt2_create", "gpt2_destroy",
     "gpt2_init_params", "gpt2_refresh_shadow", "gpt2_forward_loss", "gpt2_backward",
     "gpt2_adamw_step", "gpt2_zero_grad", "gpt2_get_status", "gpt2_step_host", "gpt2_strerror",
+    "gpt2_kernel_launches",
     "gpt2_op_gemm_bf16", "gpt2_op_attention_fwd_bf16", "gpt2_op_attention_bwd_bf16",
 ]
 
@@ -79,6 +80,7 @@ def _lib():
         "gpt2_get_status": (I, [P, P]),
         "gpt2_step_host": (I, [P, P, P, I, P, F, F, F, F, F, I, P]),
         "gpt2_strerror": (ctypes.c_char_p, [I]),
+        "gpt2_kernel_launches": (ctypes.c_uint64, []),
         "gpt2_op_gemm_bf16": (I, [P, I, I, P, I, I, P, I, I, I, I, I, F, F, P, S, I, I, P]),
         "gpt2_op_attention_fwd_bf16": (I, [P, P, P, I, I, I, I, P]),
         "gpt2_op_attention_bwd_bf16": (I, [P, P, P, P, P, P, I, I, I, I, P]),
@@ -190,6 +192,10 @@ def gpt2_step_host(ctx, tokens_host, targets_host, batch, loss_host, lr, beta1, 
     _check(_lib().gpt2_step_host(ctx, _ptr(tokens_host), _ptr(targets_host), batch, _ptr(loss_host),
                                  lr, beta1, beta2, eps, weight_decay, step, _stream(stream)),
            "gpt2_step_host")
+
+
+def gpt2_kernel_launches() -> int:
+    return int(_lib().gpt2_kernel_launches())
 
 
 def gpt2_op_gemm_bf16(A, a_mn_major, lda, B, b_mn_major, ldb, C, c_fp32, ldc, M, N, K,

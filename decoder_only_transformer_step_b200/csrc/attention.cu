@@ -238,6 +238,36 @@ __global__ void attn_bwd_prep_kernel(const T_* __restrict__ o, const T_* __restr
     for (int c = 0; c < hd; ++c) dq_acc[m * d + h * hd + c] = 0.f;
 }
 
+// bf16 version: one warp per token row, 16-byte loads; the lanes holding one
+// head's chunks reduce with shuffles.  Also zeroes the dQ accumulator row.
+template <int HD>
+__global__ void attn_bwd_prep_bf16_kernel(const bf16* __restrict__ o, const bf16* __restrict__ dout,
+                                          float* __restrict__ dvec, float* __restrict__ dq_acc, long M, int T,
+                                          int H) {
+  constexpr int CPH = HD / 8;  // 16-byte chunks per head
+  const long m = blockIdx.x * (long)(blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (m >= M) return;
+  const int d = H * HD, nch = d / 8;
+  const long b = m / T, t = m % T;
+  for (int c0 = 0; c0 < nch; c0 += 32) {
+    const int c = c0 + lane;
+    float acc = 0.f;
+    if (c < nch) {
+      uint4 a = *reinterpret_cast<const uint4*>(o + m * d + c * 8);
+      uint4 g = *reinterpret_cast<const uint4*>(dout + m * d + c * 8);
+      acc = bf16lo(a.x) * bf16lo(g.x) + bf16hi(a.x) * bf16hi(g.x) + bf16lo(a.y) * bf16lo(g.y) +
+            bf16hi(a.y) * bf16hi(g.y) + bf16lo(a.z) * bf16lo(g.z) + bf16hi(a.z) * bf16hi(g.z) +
+            bf16lo(a.w) * bf16lo(g.w) + bf16hi(a.w) * bf16hi(g.w);
+    }
+#pragma unroll
+    for (int off = 1; off < CPH; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (c < nch && (lane % CPH) == 0) dvec[(b * H + c / CPH) * T + t] = acc;
+  }
+  float4* z = reinterpret_cast<float4*>(dq_acc + m * d);
+  for (int i = lane; i < d / 4; i += 32) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 template <int HD>
 __global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ qkv,
                                                        const bf16* __restrict__ dout,
@@ -628,14 +658,17 @@ int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* 
                   float* dq_acc, float* dvec, int B, int T, int H, int hd, cudaStream_t st) {
   if (B <= 0 || T <= 0) return GPT2_OK;
   if (hd != 64 && hd != 16) return GPT2_ERR_UNSUPPORTED_SHAPE;
-  long rows = (long)B * T * H;
-  attn_bwd_prep_kernel<bf16><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(
-      (const bf16*)o, (const bf16*)dout, dvec, dq_acc, B, T, H, hd);
+  const long M = (long)B * T;
+  if (hd == 64)
+    attn_bwd_prep_bf16_kernel<64><<<(unsigned)((M + 7) / 8), 256, 0, st>>>((const bf16*)o, (const bf16*)dout,
+                                                                           dvec, dq_acc, M, T, H);
+  else
+    attn_bwd_prep_bf16_kernel<16><<<(unsigned)((M + 7) / 8), 256, 0, st>>>((const bf16*)o, (const bf16*)dout,
+                                                                           dvec, dq_acc, M, T, H);
   LAUNCH_CHECK();
   int rc = hd == 64 ? launch_bwd<64>(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st)
                     : launch_bwd<16>(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st);
   if (rc) return rc;
-  const long M = (long)B * T;
   const int d = H * hd;
   long n4 = (M * d) / 4;
   dq_to_bf16_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dq_acc, (bf16*)dqkv, M, d);

@@ -20,6 +20,7 @@
 // a deterministic reduction adds them in split order.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "epilogue.cuh"
@@ -29,7 +30,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;               // one 128-byte swizzle row of bf16
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_EPI_WARPS = 8;  // two per TMEM lane quarter, each owning half the columns
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t MN_ATOM_BYTES = 64 * BK * 2;  // one {64 MN x 64 K} TMA box
 
 template <int BN>
@@ -40,7 +42,19 @@ struct TcCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int NUM_BARS = 2 * STAGES + 5;  // full, empty, acc_full[2], acc_empty[2], drain
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
+  // one 4 KB staging box per epilogue warp (TMA store source)
+  static constexpr int EPI_BYTES = NUM_EPI_WARPS * 4096;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + NUM_BARS * 8 + 16;
+};
+
+// How the epilogue writes its result.
+enum StoreMode : int {
+  ST_REG = 0,       // per-thread global stores (general fallback)
+  ST_BF16 = 1,      // one bf16 output, staged and stored coalesced
+  ST_BF16_X2 = 2,   // two bf16 outputs (u and GELU(u)), staged and stored coalesced
+  ST_F32 = 3,       // fp32 output, TMA store (beta = 0)
+  ST_F32_ADD = 4,   // fp32 output, TMA reduce-add (beta = 1)
+  ST_F32_PART = 5,  // fp32 split-K partial [split][M][N], 3-D TMA store
 };
 
 struct TcParams {
@@ -48,6 +62,7 @@ struct TcParams {
   int a_mn, b_mn;
   int m_tiles, n_tiles, splits, kb_total;
   uint32_t idesc;
+  int store;
   EpiArgs epi;
   float* partial;
   int* err;
@@ -87,14 +102,17 @@ DEVI void decode_unit(const TcParams& p, int u, int& m0, int& nt, int& s, int& k
 template <int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
                    const TcParams p) {
   using C = TcCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t tiles = (raw + 1023u) & ~1023u;
   uint8_t* tiles_ptr = smem_raw + (tiles - raw);
-  const uint32_t bars = tiles + C::STAGES * C::STAGE_BYTES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tiles_ptr + C::STAGES * C::STAGE_BYTES + C::NUM_BARS * 8);
+  const uint32_t epi_smem = tiles + C::STAGES * C::STAGE_BYTES;
+  const uint32_t bars = epi_smem + C::EPI_BYTES;
+  uint32_t* tmem_slot =
+      reinterpret_cast<uint32_t*>(tiles_ptr + C::STAGES * C::STAGE_BYTES + C::EPI_BYTES + C::NUM_BARS * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   auto full_bar = [&](int s) { return bars + 8u * s; };
@@ -113,7 +131,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(accf_bar(b), 1);
-      mbar_init(acce_bar(b), 128);
+      mbar_init(acce_bar(b), 32 * NUM_EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -228,7 +246,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ---------------------------------------------------- epilogue ----
-    const int q = warp & 3;  // TMEM lanes [32q, 32q+32) are this warp's
+    const int e = warp - 2;
+    const int q = warp & 3;              // TMEM lanes [32q, 32q+32) are this warp's
+    const int c_begin = (e >> 2) * (BN / 2);
+    const uint32_t box = epi_smem + (uint32_t)e * 4096u;
+    const bool has_operand = p.epi.kind == EPI_BIAS_RESID || p.epi.kind == EPI_DGELU;
+    const bf16* operand = (const bf16*)(p.epi.kind == EPI_DGELU ? p.epi.aux : p.epi.resid);
     int it = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
       int m0, nt, s, kb0, kb1;
@@ -236,30 +259,86 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int n0 = nt * BN;
       const int buf = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      const int row0 = m0 + q * 32;
+      const int row = row0 + lane;
+      // the first chunk's residual / GELU' operand does not depend on the
+      // accumulator: fetch it while the MMAs run
+      uint4 pre[4];
+      if (has_operand) prefetch_bf16x32(operand, p.epi.ldo, p.M, p.N, row, n0 + c_begin, pre);
       if (!mbar_wait_bounded(accf_bar(buf), aph, abort_flag, p.err)) break;
       tc_fence_after();
-      const int row = m0 + q * 32 + lane;
-      for (int c = 0; c < BN; c += 32) {
-        if (n0 + c >= p.N) break;  // warp-uniform
+      for (int c = c_begin; c < c_begin + BN / 2; c += 32) {
+        const int col0 = n0 + c;
+        if (col0 >= p.N) break;  // warp-uniform
+        uint4 cur[4];
+        if (has_operand) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cur[i] = pre[i];
+          if (c + 32 < c_begin + BN / 2 && col0 + 32 < p.N)
+            prefetch_bf16x32(operand, p.epi.ldo, p.M, p.N, row, col0 + 32, pre);
+        }
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c), r);
         tmem_ld_wait();
-        if (row < p.M) {
-          float v[32];
+        float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          const int col0 = n0 + c;
-          if (col0 + 32 <= p.N) {
-            epi_row32_bf16(p.epi, p.partial, s, p.M, p.N, row, col0, v);
-          } else {
-            for (int j = 0; j < 32 && col0 + j < p.N; ++j)
-              epi_one<bf16>(p.epi, p.partial, s, p.M, p.N, row, col0 + j, v[j]);
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (p.store == ST_REG) {
+          if (row < p.M) {
+            if (col0 + 32 <= p.N) {
+              epi_row32_bf16(p.epi, p.partial, s, p.M, p.N, row, col0, v);
+            } else {
+              // fully unrolled: a runtime-bounded loop would put v in local memory
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < p.N) epi_one<bf16>(p.epi, p.partial, s, p.M, p.N, row, col0 + j, v[j]);
+            }
           }
+          continue;
+        }
+        epi_apply_row32(p.epi, p.N, col0, v, cur);
+        if (p.store == ST_BF16 || p.store == ST_BF16_X2) {
+          // bf16 outputs: transpose through the box, coalesced direct stores
+          stage_bf16_row(box, lane, v);
+          if (p.store == ST_BF16_X2) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = gelu_f<true>(v[j]);
+            stage_bf16_row(box + 2048u, lane, v);
+          }
+          __syncwarp();
+          unstage_bf16_box(box, lane, (bf16*)p.epi.out, p.epi.ldo, p.M, p.N, row0, col0);
+          if (p.store == ST_BF16_X2)
+            unstage_bf16_box(box + 2048u, lane, (bf16*)p.epi.out2, p.epi.ldo, p.M, p.N, row0, col0);
+          __syncwarp();
+          continue;
+        }
+        // fp32 outputs: TMA store / reduce-add; the previous store from this
+        // box must have read it
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        stage_f32_row(box, lane, v);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          switch (p.store) {
+            case ST_F32:
+              tma_store_2d(&tmC, box, col0, row0);
+              break;
+            case ST_F32_ADD:
+              tma_reduce_add_2d(&tmC, box, col0, row0);
+              break;
+            case ST_F32_PART:
+              tma_store_3d(&tmC, box, col0, row0, s);
+              break;
+          }
+          bulk_commit();
         }
       }
       tc_fence_before();
       mbar_arrive(acce_bar(buf));
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -310,23 +389,45 @@ PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
   return fn;
 }
 
-// 2-D bf16 tensor [outer, inner] with row pitch `pitch` elements.
-bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
-               uint32_t box_inner, uint32_t box_outer) {
+// Tensor map over a row-major tensor: dims[0] is the contiguous (innermost)
+// extent in elements, strides are in bytes for dims 1..rank-1.
+bool encode_tmap(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, int rank, const uint64_t* dims,
+                 const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw) {
   auto enc = tmap_encoder();
   if (!enc) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {pitch * 2};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  cuuint64_t d[3], st[2];
+  cuuint32_t b[3], e[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides[i];
+  CUresult r = enc(tm, dt, rank, const_cast<void*>(base), d, st, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
+// 2-D bf16 operand [outer, inner] with row pitch `pitch` elements, 128-byte swizzle.
+bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
+               uint32_t box_inner, uint32_t box_outer) {
+  const uint64_t dims[2] = {inner, outer}, strides[1] = {pitch * 2};
+  const uint32_t box[2] = {box_inner, box_outer};
+  return encode_tmap(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 2, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Output [M, N] with pitch ldo, stored in 32 x 32 boxes: bf16 with the 64-byte
+// swizzle, fp32 with the 128-byte swizzle (matching stage_*_row).
+bool make_out_tmap(CUtensorMap* tm, const void* base, int M, int N, long ldo, bool f32) {
+  const uint64_t dims[2] = {(uint64_t)N, (uint64_t)M}, strides[1] = {(uint64_t)ldo * (f32 ? 4 : 2)};
+  const uint32_t box[2] = {32, 32};
+  return encode_tmap(tm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 2,
+                     dims, strides, box, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 template <int BN>
-int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, int grid, cudaStream_t st) {
+int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tc2,
+              const TcParams& p, int grid, cudaStream_t st) {
   using C = TcCfg<BN>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -334,7 +435,7 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const TcParams& p, i
                                   C::SMEM_BYTES));
     attr_set = true;
   }
-  gemm_tc_kernel<BN><<<grid, NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, p);
+  gemm_tc_kernel<BN><<<grid, NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, tc, tc2, p);
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -406,9 +507,47 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   p.err = err;
   if (splits > 1) p.epi.kind = EPI_F32_PARTIAL;
 
+  // output path: TMA stores of 32 x 32 boxes staged in shared memory
+  CUtensorMap tc, tc2;
+  memset(&tc, 0, sizeof(tc));
+  memset(&tc2, 0, sizeof(tc2));
+  bool ok_c = true;
+  switch (p.epi.kind) {
+    case EPI_STORE:
+    case EPI_BIAS:
+    case EPI_BIAS_RESID:
+    case EPI_DGELU:
+      p.store = ST_BF16;
+      break;
+    case EPI_BIAS_GELU:
+      p.store = ST_BF16_X2;
+      break;
+    case EPI_F32:
+      if (g.epi.beta == 0.f || g.epi.beta == 1.f) {
+        p.store = g.epi.beta == 0.f ? ST_F32 : ST_F32_ADD;
+        ok_c = g.epi.ldo % 4 == 0 && make_out_tmap(&tc, g.epi.out, g.M, g.N, g.epi.ldo, true);
+      } else {
+        p.store = ST_REG;
+      }
+      break;
+    case EPI_F32_PARTIAL: {
+      p.store = ST_F32_PART;
+      const uint64_t dims[3] = {(uint64_t)g.N, (uint64_t)g.M, (uint64_t)splits};
+      const uint64_t strides[2] = {(uint64_t)g.N * 4, (uint64_t)g.M * g.N * 4};
+      const uint32_t box[3] = {32, 32, 1};
+      ok_c = encode_tmap(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ws, 3, dims, strides, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+      break;
+    }
+    default:
+      p.store = ST_REG;
+  }
+  if (!ok_c) return GPT2_ERR_CUDA;
+  if (p.store == ST_BF16_X2 && ((uintptr_t)g.epi.out2 & 15)) return GPT2_ERR_INVALID_ARG;
+
   const int units = p.m_tiles * p.n_tiles * splits;
   const int grid = units < num_sms() ? units : num_sms();
-  int rc = bn == 256 ? launch_tc<256>(ta, tb, p, grid, st) : launch_tc<128>(ta, tb, p, grid, st);
+  int rc = bn == 256 ? launch_tc<256>(ta, tb, tc, tc2, p, grid, st) : launch_tc<128>(ta, tb, tc, tc2, p, grid, st);
   if (rc) return rc;
   if (splits > 1) {
     long mn = (long)g.M * g.N;

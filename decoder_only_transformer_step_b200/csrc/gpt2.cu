@@ -6,6 +6,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <vector>
 
 #include "common.cuh"
@@ -174,6 +175,9 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
 }
 
 }  // namespace
+
+static std::atomic<unsigned long long> g_launches{0};
+void gpt2_count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 struct gpt2_ctx {
   gpt2_config cfg;
@@ -512,6 +516,8 @@ int gpt2_step_host(gpt2_ctx* c, const int32_t* tokens_host, const int32_t* targe
   CUDA_TRY(cudaStreamSynchronize(st));
   return GPT2_OK;
 }
+
+uint64_t gpt2_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* gpt2_strerror(int code) {
   switch (code) {

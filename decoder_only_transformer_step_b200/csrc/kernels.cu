@@ -178,9 +178,24 @@ __global__ void ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ g, 
 // dx = rstd * (dxhat - mean(dxhat) - xhat * mean(dxhat * xhat)), dxhat = dy * g;
 // dres = (init ? 0 : dres) + dx.  dgamma += dy * xhat, dbeta += dy, reduced in a
 // fixed order over the CTA's rows into part[blockIdx.x][0:d] and [d:2d].
+// A fixed grid (at most LNB_MAX_CTAS) of 8-warp CTAs; each warp strides over
+// rows and fetches the next row's x, dy, dres while it computes the current.
 constexpr int LNB_WARPS = 8;
-constexpr int LNB_ROWS_PER_WARP = 16;
-constexpr int LNB_ROWS = LNB_WARPS * LNB_ROWS_PER_WARP;
+constexpr int LNB_MAX_CTAS = 512;
+
+DEVI uint4 ld16(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+template <typename T>
+DEVI void unpack16(const uint4& u, float (&f)[Vec<T>::N]);
+template <>
+DEVI void unpack16<bf16>(const uint4& u, float (&f)[8]) {
+  f[0] = bf16lo(u.x); f[1] = bf16hi(u.x); f[2] = bf16lo(u.y); f[3] = bf16hi(u.y);
+  f[4] = bf16lo(u.z); f[5] = bf16hi(u.z); f[6] = bf16lo(u.w); f[7] = bf16hi(u.w);
+}
+template <>
+DEVI void unpack16<float>(const uint4& u, float (&f)[4]) {
+  f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+}
 
 template <typename T, int NC>
 __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x,
@@ -199,19 +214,42 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
     for (int j = 0; j < VN; ++j) dg[k][j] = db[k][j] = 0.f;
     if (c < d) Vec<T>::load(g + c, gg[k]);
   }
-  const int row0 = blockIdx.x * LNB_ROWS + warp * LNB_ROWS_PER_WARP;
-  for (int r = 0; r < LNB_ROWS_PER_WARP; ++r) {
-    const int m = row0 + r;
-    if (m >= M) break;
-    const float mu = mean[m], rs = rstd[m];
+  const int nwarps = gridDim.x * LNB_WARPS;
+  uint4 px[NC], pd[NC], pr[NC];
+  float pmu = 0.f, prs = 0.f;
+#define LNB_FETCH(mm)                                              \
+  do {                                                             \
+    _Pragma("unroll") for (int k = 0; k < NC; ++k) {               \
+      const int c = (lane + 32 * k) * VN;                          \
+      if (c < d) {                                                 \
+        px[k] = ld16(x + (long)(mm) * d + c);                      \
+        pd[k] = ld16(dy + (long)(mm) * d + c);                     \
+        if (!dres_init) pr[k] = ld16(dres + (long)(mm) * d + c);   \
+      }                                                            \
+    }                                                              \
+    pmu = mean[mm];                                                \
+    prs = rstd[mm];                                                \
+  } while (0)
+  int m = blockIdx.x * LNB_WARPS + warp;
+  if (m < M) LNB_FETCH(m);
+  for (; m < M; m += nwarps) {
+    uint4 cx[NC], cd[NC], cr[NC];
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      cx[k] = px[k];
+      cd[k] = pd[k];
+      cr[k] = pr[k];
+    }
+    const float mu = pmu, rs = prs;
+    if (m + nwarps < M) LNB_FETCH(m + nwarps);
     float xv[NC][VN], dv[NC][VN];
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
     for (int k = 0; k < NC; ++k) {
       const int c = (lane + 32 * k) * VN;
       if (c < d) {
-        Vec<T>::load(x + (long)m * d + c, xv[k]);
-        Vec<T>::load(dy + (long)m * d + c, dv[k]);
+        unpack16<T>(cx[k], xv[k]);
+        unpack16<T>(cd[k], dv[k]);
 #pragma unroll
         for (int j = 0; j < VN; ++j) {
           const float xh = (xv[k][j] - mu) * rs;
@@ -232,7 +270,7 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
       if (c < d) {
         float o[VN];
         if (!dres_init) {
-          Vec<T>::load(dres + (long)m * d + c, o);
+          unpack16<T>(cr[k], o);
         } else {
 #pragma unroll
           for (int j = 0; j < VN; ++j) o[j] = 0.f;
@@ -267,6 +305,7 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, c
   }
   for (int i = threadIdx.x; i < 2 * d; i += blockDim.x) part[(long)blockIdx.x * 2 * d + i] = red[i];
 }
+#undef LNB_FETCH
 
 // grad[j] = beta * grad[j] + sum_r part[r, j] (r ascending); 8 row slices per
 // column reduced in a fixed order.
@@ -552,10 +591,15 @@ int ln_fwd_dispatch(const void* x, const void* g, const void* b, void* y, float*
   return GPT2_OK;
 }
 
+int ln_bwd_blocks(int M) {
+  const int b = (M + LNB_WARPS - 1) / LNB_WARPS;
+  return b < LNB_MAX_CTAS ? b : LNB_MAX_CTAS;
+}
+
 template <typename T, int NC>
 void ln_bwd_launch(const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
                    void* dres, int init, float* part, int M, int d, cudaStream_t st) {
-  ln_bwd_kernel<T, NC><<<(M + LNB_ROWS - 1) / LNB_ROWS, 256, 2 * d * sizeof(float), st>>>(
+  ln_bwd_kernel<T, NC><<<ln_bwd_blocks(M), 256, 2 * d * sizeof(float), st>>>(
       (const T*)dy, (const T*)x, mean, rstd, (const T*)g, (T*)dres, init, part, M, d);
 }
 
@@ -601,11 +645,11 @@ int layernorm_fwd(int f32, const void* x, const void* g, const void* b, void* y,
              : ln_fwd_dispatch<bf16>(x, g, b, y, mean, rstd, M, d, st);
 }
 
-size_t layernorm_bwd_part_floats(int M, int d) { return (size_t)((M + LNB_ROWS - 1) / LNB_ROWS) * 2 * d; }
+size_t layernorm_bwd_part_floats(int M, int d) { return (size_t)ln_bwd_blocks(M) * 2 * d; }
 
 int layernorm_bwd(int f32, const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
                   void* dres, int dres_init, float* part, int* nblk, int M, int d, cudaStream_t st) {
-  *nblk = (M + LNB_ROWS - 1) / LNB_ROWS;
+  *nblk = ln_bwd_blocks(M);
   return f32 ? ln_bwd_dispatch<float>(dy, x, mean, rstd, g, dres, dres_init, part, M, d, st)
              : ln_bwd_dispatch<bf16>(dy, x, mean, rstd, g, dres, dres_init, part, M, d, st);
 }

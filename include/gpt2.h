@@ -161,6 +161,10 @@ int gpt2_step_host(gpt2_ctx* ctx, const int32_t* tokens_host, const int32_t* tar
 /* Static text for an error code. */
 const char* gpt2_strerror(int code);
 
+/* Number of CUDA kernels this library has launched in this process so far
+ * (all contexts and entry points); a diagnostic for launch accounting. */
+uint64_t gpt2_kernel_launches(void);
+
 /* ------------------------------------------------------------------------
  * Single-operation entry points used by the kernel unit tests.  They run the
  * same kernels the step runs, on caller buffers.

@@ -37,12 +37,16 @@ def test_gemm_layouts(a_mn, b_mn, bn, c_fp32):
     ref = A_log.double() @ B_log.double().t()
     alpha = 0.75
     dev = "cuda"
-    C = torch.zeros((M, N), dtype=torch.float32 if c_fp32 else torch.bfloat16, device=dev)
+    # fp32 output accumulates onto existing values (beta = 1, the gradient
+    # accumulation path); bf16 output overwrites
+    C0 = torch.randn((M, N), generator=torch.Generator().manual_seed(9)) if c_fp32 else torch.zeros((M, N))
+    C = C0.to(torch.float32 if c_fp32 else torch.bfloat16).to(dev)
     gp.gpt2_op_gemm_bf16(A_st.to(dev), a_mn, lda, B_st.to(dev), b_mn, ldb, C, c_fp32, N, M, N, K,
-                         alpha=alpha, bn=bn, splits=1)
+                         alpha=alpha, beta=1.0 if c_fp32 else 0.0, bn=bn, splits=1)
     torch.cuda.synchronize()
     out = C.double().cpu()
-    err = (out - alpha * ref).abs().max().item()
+    expect = alpha * ref + (C0.double() if c_fp32 else 0.0)
+    err = (out - expect).abs().max().item()
     scale = (alpha * ref).abs().max().item()
     assert err <= (1e-5 if c_fp32 else 8e-3) * scale, (err, scale)
 

@@ -93,8 +93,20 @@ def test_tiny_ten_adamw_steps():
         assert abs(loss - ref_loss) <= 1e-2 * abs(ref_loss)
     torch.cuda.synchronize()
     got = oracle.unflatten(model.master.double().cpu().numpy(), TINY)
+    d = TINY.d_model
     for n in p:
-        rel = np.linalg.norm(got[n] - p[n]) / np.linalg.norm(p[n])
+        a, r = got[n], p[n]
+        if n.endswith("b_qkv"):
+            # The key-bias gradient is exactly zero in exact arithmetic (a shift
+            # of every key leaves the softmax unchanged; pinned in the oracle
+            # tests), so Adam's normalised step turns each side's rounding noise
+            # into updates of either sign.  That block is held to Adam's
+            # per-step bound instead: |m_hat| / sqrt(v_hat) <= 1/sqrt(1-beta2).
+            kb = slice(d, 2 * d)
+            assert np.abs(a[kb] - r[kb]).max() <= 2 * 10 * 6e-4 / np.sqrt(1 - 0.95)
+            a = np.concatenate([a[:d], a[2 * d:]])
+            r = np.concatenate([r[:d], r[2 * d:]])
+        rel = np.linalg.norm(a - r) / np.linalg.norm(r)
         assert rel <= 1e-2, (n, rel)
 
 
