@@ -21,7 +21,7 @@ GPT2_OK = 0
 ERRORS = {
     -1: "GPT2_ERR_INVALID_ARG", -2: "GPT2_ERR_UNSUPPORTED_SHAPE", -3: "GPT2_ERR_CUDA",
     -4: "GPT2_ERR_BAD_STATE", -5: "GPT2_ERR_TOKEN_RANGE", -6: "GPT2_ERR_NONFINITE",
-    -7: "GPT2_ERR_TIMEOUT", -8: "GPT2_ERR_WORKSPACE",
+    -7: "GPT2_ERR_TIMEOUT", -8: "GPT2_ERR_WORKSPACE", -9: "GPT2_ERR_TOO_LARGE",
 }
 
 
@@ -49,6 +49,7 @@ EXPORTS = [
     "gpt2_adamw_step", "gpt2_zero_grad", "gpt2_get_status", "gpt2_step_host", "gpt2_strerror",
     "gpt2_kernel_launches",
     "gpt2_op_gemm_bf16", "gpt2_op_attention_fwd_bf16", "gpt2_op_attention_bwd_bf16",
+    "gpt2_op_attention_bwd_bf16_noalloc",
 ]
 
 _LIB = None
@@ -84,6 +85,7 @@ def _lib():
         "gpt2_op_gemm_bf16": (I, [P, I, I, P, I, I, P, I, I, I, I, I, F, F, P, S, I, I, P]),
         "gpt2_op_attention_fwd_bf16": (I, [P, P, P, I, I, I, I, P]),
         "gpt2_op_attention_bwd_bf16": (I, [P, P, P, P, P, P, I, I, I, I, P]),
+        "gpt2_op_attention_bwd_bf16_noalloc": (I, [P, P, P, P, P, I, I, I, I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -215,6 +217,14 @@ def gpt2_op_attention_bwd_bf16(qkv, o, lse, dout, dqkv, scratch, B, T, H, hd, st
     _check(_lib().gpt2_op_attention_bwd_bf16(_ptr(qkv), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dqkv),
                                              _ptr(scratch), B, T, H, hd, _stream(stream)),
            "gpt2_op_attention_bwd_bf16")
+
+
+def gpt2_op_attention_bwd_bf16_noalloc(qkv, o, lse, dout, dqkv, B, T, H, hd, stream=None):
+    """Allocation-free attention backward: scratch lives in the library (see
+    include/gpt2.h); for callers that cannot allocate device memory."""
+    _check(_lib().gpt2_op_attention_bwd_bf16_noalloc(_ptr(qkv), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dqkv),
+                                                     B, T, H, hd, _stream(stream)),
+           "gpt2_op_attention_bwd_bf16_noalloc")
 
 
 # ------------------------------------------------------------ convenience ---

@@ -530,6 +530,7 @@ const char* gpt2_strerror(int code) {
     case GPT2_ERR_NONFINITE: return "non-finite loss";
     case GPT2_ERR_TIMEOUT: return "device pipeline wait timed out";
     case GPT2_ERR_WORKSPACE: return "workspace too small";
+    case GPT2_ERR_TOO_LARGE: return "problem exceeds the built-in scratch of the allocation-free entry point";
     default: return "unknown error";
   }
 }

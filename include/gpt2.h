@@ -62,7 +62,8 @@ enum {
   GPT2_ERR_TOKEN_RANGE = -5,      /* device: an id outside [0, vocab_real) (clamped to 0) */
   GPT2_ERR_NONFINITE = -6,        /* device: loss is NaN or Inf */
   GPT2_ERR_TIMEOUT = -7,          /* device: a bounded pipeline wait ran out */
-  GPT2_ERR_WORKSPACE = -8         /* workspace smaller than gpt2_workspace_bytes */
+  GPT2_ERR_WORKSPACE = -8,        /* workspace smaller than gpt2_workspace_bytes */
+  GPT2_ERR_TOO_LARGE = -9         /* problem exceeds the built-in scratch of an allocation-free entry point */
 };
 
 typedef struct {
@@ -197,6 +198,23 @@ int gpt2_op_attention_fwd_bf16(const uint16_t* qkv, uint16_t* o, float* lse,
 int gpt2_op_attention_bwd_bf16(const uint16_t* qkv, const uint16_t* o, const float* lse,
                                const uint16_t* dout, uint16_t* dqkv, float* scratch,
                                int B, int T, int H, int hd, void* stream);
+
+/* Allocation-free variant of gpt2_op_attention_bwd_bf16 (same inputs, same
+ * output dqkv, no scratch argument).  The paper has no counterpart: this entry
+ * point exists for callers that cannot call cudaMalloc -- a host that gives a
+ * plug-in only its input and output buffers, a runtime whose caching
+ * allocator already holds the device memory, or a loop that cannot afford
+ * cudaMalloc's device synchronisation.  Its scratch (fp32 dQ accumulator and
+ * D vector, B*T*H*hd + B*H*T floats) lives in a 16 MiB array compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  Larger problems return GPT2_ERR_TOO_LARGE.  The first call on a
+ * device looks up that device's address of the array (cudaGetSymbolAddress);
+ * make that first call before any stream capture.  All calls share the one
+ * array: calls that may overlap on the GPU (unordered streams) race and must
+ * not be issued.  It calls no allocator. */
+int gpt2_op_attention_bwd_bf16_noalloc(const uint16_t* qkv, const uint16_t* o, const float* lse,
+                                       const uint16_t* dout, uint16_t* dqkv,
+                                       int B, int T, int H, int hd, void* stream);
 
 #ifdef __cplusplus
 }
