@@ -12,6 +12,8 @@
 // accumulates dK, dV in registers over the query blocks at or below the
 // diagonal; dQ contributions go to an fp32 buffer with vector reductions.
 // fp32 path (correctness mode): plain CUDA-core kernels.
+#include <stdlib.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -647,8 +649,20 @@ int launch_bwd(const void* qkv, const void* dout, const float* lse, const float*
 
 }  // namespace
 
+// head_dim 64 runs on the tcgen05 kernel (attention_tc.cu); GPT2_ATTN_FWD=mma
+// selects the warp-level mma.sync kernel instead (a diagnostic switch).
+static bool use_mma_fwd() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("GPT2_ATTN_FWD");
+    v = (e && e[0] == 'm') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 int attn_fwd_bf16(const void* qkv, void* o, float* lse, int B, int T, int H, int hd, cudaStream_t st) {
   if (B <= 0 || T <= 0) return GPT2_OK;
+  if (hd == 64 && !use_mma_fwd()) return attn_fwd_tc(qkv, o, lse, B, T, H, st);
   if (hd == 64) return launch_fwd<64>(qkv, o, lse, B, T, H, st);
   if (hd == 16) return launch_fwd<16>(qkv, o, lse, B, T, H, st);
   return GPT2_ERR_UNSUPPORTED_SHAPE;

@@ -1,0 +1,334 @@
+// Causal self-attention forward on the 5th-generation tensor cores (tcgen05),
+// head_dim 64: softmax(q k^T / sqrt(64), keys j <= query i) v per (batch, head).
+// The O(T^2) scores of the Kaplan Eq. (2.2) term ("Pré-treinar um LLM") live
+// only in tensor memory and registers: per 128-key tile the scores S = Q K^T
+// are accumulated in TMEM, one softmax thread per query row turns its row of S
+// into probabilities P (bf16, written to shared memory as the next MMA's A
+// operand), and O_tile = P V goes back to TMEM; the row's output accumulates in
+// registers with the running-max correction (online softmax), and only O and
+// the per-row log-sum-exp reach HBM.
+//
+// One CTA per (batch, head, 128-query block), 192 threads:
+//   warp 0      TMA: Q once, K/V tiles into a 2-stage ring (a 3-D tensor map
+//               over the packed QKV activation; rows past T read as zeros)
+//   warp 1      TMEM allocation; tcgen05.mma S(j) = Q K_j^T (M128 N128 K64) into
+//               a double-buffered S, then O_tile(j-1) = P(j-1) V(j-1) (M128 N64
+//               K128, V as an MN-major operand) into a double-buffered O_tile
+//   warps 2..5  softmax of S(j) (row per thread, no shuffles), P(j) to shared
+//               memory, then fold O_tile(j-1) into the register accumulator
+// so S(j+1) is computed while the softmax of tile j runs.  Every mbarrier wait
+// is bounded; a timeout sets the device status and the CTA drains and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+// 3-D bf16 tensor map, 128-byte swizzle, box {64, 128, 1}.
+bool tmap_3d(CUtensorMap* tm, const void* base, const uint64_t* dims, const uint64_t* strides) {
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  if (!enc) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  cuuint64_t d[3] = {dims[0], dims[1], dims[2]}, s[2] = {strides[0], strides[1]};
+  cuuint32_t box[3] = {64, 128, 1}, e[3] = {1, 1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), d, s, box, e,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int HD = 64, BQ = 128, BKV = 128;
+constexpr int TILE = 128 * 128;  // one 128-row x 64-col bf16 tile, 128B-swizzled
+constexpr int SM_Q = 0;
+constexpr int SM_K = SM_Q + TILE;       // 2 stages
+constexpr int SM_V = SM_K + 2 * TILE;   // 2 stages
+constexpr int SM_P = SM_V + 2 * TILE;   // 2 buffers x (keys 0-63 | keys 64-127)
+constexpr int SM_TILES = SM_P + 4 * TILE;
+// q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full[2], o_full[2], drain
+constexpr int NUM_BARS = 14;
+constexpr int SMEM_BYTES = SM_TILES + 1024 + NUM_BARS * 8 + 16;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t S_COL = 0, O_COL = 256;
+constexpr int NUM_THREADS = 192;
+
+#define LN2_F 0.6931471805599453f
+#define LOG2E_F 1.4426950408889634f
+
+DEVI uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// kind::f16 instruction descriptors: fp32 accumulate, bf16 operands, M = 128.
+constexpr uint32_t IDESC_S = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t IDESC_O =
+    (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+
+DEVI void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+DEVI float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmO,
+                       float* __restrict__ lse, int T, int H, float scale_log2, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t bars = base + SM_TILES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + SM_TILES + NUM_BARS * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t q_full = bars;
+  auto kv_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto kv_empty = [&](int s) { return bars + 8u * (3 + s); };
+  auto s_full = [&](int s) { return bars + 8u * (5 + s); };
+  auto s_free = [&](int s) { return bars + 8u * (7 + s); };
+  auto p_full = [&](int s) { return bars + 8u * (9 + s); };
+  auto o_full = [&](int s) { return bars + 8u * (11 + s); };
+  const uint32_t drain_bar = bars + 8u * 13;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = (T + BQ - 1) / BQ;
+  const int qb = nqb - 1 - (int)blockIdx.x;  // longest causal blocks first
+  const int b = blockIdx.y / H, h = blockIdx.y % H;
+  const int d = H * HD;
+  const int q0 = qb * BQ;
+  const int nkv = qb + 1;  // key tiles 0..qb (BKV == BQ)
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+      mbar_init(s_full(s), 1);
+      mbar_init(s_free(s), 128);
+      mbar_init(p_full(s), 128);
+      mbar_init(o_full(s), 1);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tmQKV);
+    tma_prefetch_desc(&tmO);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- TMA ----
+      int issued = 0;
+      bool ok = true;
+      mbar_arrive_expect_tx(q_full, TILE);
+      tma_load_3d(base + SM_Q, &tmQKV, q_full, h * HD, q0, b);
+      for (int j = 0; j < nkv; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !mbar_wait_bounded(kv_empty(st), ((j - 2) >> 1) & 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(kv_full(st), 2 * TILE);
+        tma_load_3d(base + SM_K + st * TILE, &tmQKV, kv_full(st), d + h * HD, j * BKV, b);
+        tma_load_3d(base + SM_V + st * TILE, &tmQKV, kv_full(st), 2 * d + h * HD, j * BKV, b);
+        ++issued;
+      }
+      if (!ok) {
+        mbar_drain_bounded(q_full, 0);
+        for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) mbar_drain_bounded(kv_full(j & 1), (j >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- MMA ----
+      bool ok = mbar_wait_bounded(q_full, 0, abort_flag, err);
+      bool issued_any = false;
+      auto issue_pv = [&](int t) -> bool {
+        const int pb = t & 1;
+        if (!mbar_wait_bounded(p_full(pb), (t >> 1) & 1, abort_flag, err)) return false;
+        tc_fence_after();
+        const uint32_t pbase = base + SM_P + pb * 2 * TILE;
+        const uint32_t vbase = base + SM_V + (t & 1) * TILE;
+#pragma unroll
+        for (int k = 0; k < BKV / 16; ++k)
+          tc_mma_bf16(tmem + O_COL + pb * HD, sdesc(pbase + (k >> 2) * TILE + (k & 3) * 32, 16, 1024),
+                      sdesc(vbase + k * 2048, 8192, 1024), IDESC_O, k > 0 ? 1u : 0u);
+        tc_commit(o_full(pb));
+        tc_commit(kv_empty(t & 1));
+        return true;
+      };
+      if (ok) tc_fence_after();
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait_bounded(kv_full(st), (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (j >= 2 && !mbar_wait_bounded(s_free(st), ((j - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kbase = base + SM_K + st * TILE;
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k)
+          tc_mma_bf16(tmem + S_COL + st * BKV, sdesc(base + SM_Q + k * 32, 16, 1024), sdesc(kbase + k * 32, 16, 1024),
+                      IDESC_S, k > 0 ? 1u : 0u);
+        issued_any = true;
+        tc_commit(s_full(st));
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok) ok = issue_pv(nkv - 1);
+      if (!ok && issued_any) {
+        tc_commit(drain_bar);
+        mbar_drain_bounded(drain_bar, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------- softmax ----
+    const int q = warp & 3;  // TMEM lanes [32q, 32q+32)
+    const int row = q * 32 + lane;
+    const int grow = q0 + row;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
+    float acc[HD];
+#pragma unroll
+    for (int i = 0; i < HD; ++i) acc[i] = 0.f;
+    bool ok = true;
+    auto fold = [&](int t, float a) -> bool {
+      const int ob = t & 1;
+      if (!mbar_wait_bounded(o_full(ob), (t >> 1) & 1, abort_flag, err)) return false;
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      tmem_ld_32x32b_x32(tmem + lane_off + O_COL + ob * HD, r0);
+      tmem_ld_32x32b_x32(tmem + lane_off + O_COL + ob * HD + 32, r1);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        acc[i] = acc[i] * a + __uint_as_float(r0[i]);
+        acc[32 + i] = acc[32 + i] * a + __uint_as_float(r1[i]);
+      }
+      tc_fence_before();
+      return true;
+    };
+    for (int j = 0; j < nkv; ++j) {
+      const int sb = j & 1;
+      if (!mbar_wait_bounded(s_full(sb), (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem + lane_off + S_COL + sb * BKV + 32 * c, r[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(s_free(sb));
+      const bool diag = (j == nkv - 1);
+      const int kv0 = j * BKV;
+      float mx = m;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          float v = __uint_as_float(r[c][i]) * scale_log2;
+          if (diag && kv0 + 32 * c + i > grow) v = -INFINITY;
+          r[c][i] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      const float alpha = ex2(m - mx);
+      m = mx;
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p = ex2(__uint_as_float(r[c][i]) - m);
+          r[c][i] = __float_as_uint(p);
+          sum += p;
+        }
+      l = l * alpha + sum;
+      // P row -> shared memory, 128B-swizzled K-major (keys 0-63 | 64-127)
+      const uint32_t pb = base + SM_P + sb * 2 * TILE + (uint32_t)row * 128u;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int g = c >> 2, o8 = (c & 3) * 8;
+        st_shared_v4(pb + (uint32_t)(c >> 3) * TILE + 16u * (uint32_t)((c & 7) ^ (row & 7)),
+                     pack_bf16x2(__uint_as_float(r[g][o8 + 0]), __uint_as_float(r[g][o8 + 1])),
+                     pack_bf16x2(__uint_as_float(r[g][o8 + 2]), __uint_as_float(r[g][o8 + 3])),
+                     pack_bf16x2(__uint_as_float(r[g][o8 + 4]), __uint_as_float(r[g][o8 + 5])),
+                     pack_bf16x2(__uint_as_float(r[g][o8 + 6]), __uint_as_float(r[g][o8 + 7])));
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(p_full(sb));
+      if (j >= 1 && !fold(j - 1, alpha_prev)) { ok = false; break; }
+      alpha_prev = alpha;
+    }
+    if (ok) ok = fold(nkv - 1, alpha_prev);
+    if (ok) {
+      // O / l -> shared memory (the Q tile is no longer read) -> one TMA store
+      const float inv = 1.f / l;
+      const uint32_t ob = base + SM_Q + (uint32_t)row * 128u;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(ob + 16u * (uint32_t)(c ^ (row & 7)), pack_bf16x2(acc[8 * c] * inv, acc[8 * c + 1] * inv),
+                     pack_bf16x2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv),
+                     pack_bf16x2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv),
+                     pack_bf16x2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv));
+      if (grow < T) lse[((long)b * H + h) * T + grow] = (m + __log2f(l)) * LN2_F;
+      fence_proxy_async_smem();
+    }
+    // all four softmax warps arrive here (an abort makes every wait return)
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (warp == 2 && lane == 0 && !*abort_flag) {
+      tma_store_3d(&tmO, base + SM_Q, h * HD, q0, b);
+      bulk_commit();
+      bulk_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+int attn_fwd_tc(const void* qkv, void* o, float* lse, int B, int T, int H, cudaStream_t st) {
+  if (B <= 0 || T <= 0) return GPT2_OK;
+  const uint64_t d = (uint64_t)H * HD;
+  CUtensorMap tq, to;
+  const uint64_t dq[3] = {3 * d, (uint64_t)T, (uint64_t)B};
+  const uint64_t sq[2] = {3 * d * 2, (uint64_t)T * 3 * d * 2};
+  const uint64_t dout[3] = {d, (uint64_t)T, (uint64_t)B};
+  const uint64_t sout[2] = {d * 2, (uint64_t)T * d * 2};
+  if (!tmap_3d(&tq, qkv, dq, sq) || !tmap_3d(&to, o, dout, sout)) return GPT2_ERR_CUDA;
+  static bool attr = false;
+  if (!attr) {
+    CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    attr = true;
+  }
+  dim3 grid((T + BQ - 1) / BQ, B * H);
+  attn_fwd_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tq, to, lse, T, H, LOG2E_F / 8.f, nullptr);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}

@@ -50,6 +50,9 @@ int gemm_simt_f32(const GemmArgs& g, cudaStream_t st);
 
 int num_sms();
 
+// tcgen05 causal attention forward, head_dim 64 (bf16).
+int attn_fwd_tc(const void* qkv, void* o, float* lse, int B, int T, int H, cudaStream_t st);
+
 // ---- attention ----------------------------------------------------------
 // qkv [B*T, 3*H*hd] (act), o [B*T, H*hd] (act), lse [B,H,T] fp32.
 int attn_fwd_bf16(const void* qkv, void* o, float* lse, int B, int T, int H, int hd,
