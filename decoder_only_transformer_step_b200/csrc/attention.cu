@@ -649,15 +649,23 @@ int launch_bwd(const void* qkv, const void* dout, const float* lse, const float*
 
 }  // namespace
 
-// head_dim 64 runs on the tcgen05 kernel (attention_tc.cu); GPT2_ATTN_FWD=mma
-// selects the warp-level mma.sync kernel instead (a diagnostic switch).
+// head_dim 64 runs on the tcgen05 kernels (attention_tc.cu); GPT2_ATTN_FWD=mma
+// / GPT2_ATTN_BWD=mma select the warp-level mma.sync kernels instead (a
+// diagnostic switch).
+static bool env_is_mma(const char* name, int* cache) {
+  if (*cache < 0) {
+    const char* e = getenv(name);
+    *cache = (e && e[0] == 'm') ? 1 : 0;
+  }
+  return *cache == 1;
+}
 static bool use_mma_fwd() {
   static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("GPT2_ATTN_FWD");
-    v = (e && e[0] == 'm') ? 1 : 0;
-  }
-  return v == 1;
+  return env_is_mma("GPT2_ATTN_FWD", &v);
+}
+static bool use_mma_bwd() {
+  static int v = -1;
+  return env_is_mma("GPT2_ATTN_BWD", &v);
 }
 
 int attn_fwd_bf16(const void* qkv, void* o, float* lse, int B, int T, int H, int hd, cudaStream_t st) {
@@ -680,8 +688,10 @@ int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* 
     attn_bwd_prep_bf16_kernel<16><<<(unsigned)((M + 7) / 8), 256, 0, st>>>((const bf16*)o, (const bf16*)dout,
                                                                            dvec, dq_acc, M, T, H);
   LAUNCH_CHECK();
-  int rc = hd == 64 ? launch_bwd<64>(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st)
-                    : launch_bwd<16>(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st);
+  int rc = (hd == 64 && !use_mma_bwd())
+               ? attn_bwd_tc(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st)
+               : (hd == 64 ? launch_bwd<64>(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st)
+                           : launch_bwd<16>(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st));
   if (rc) return rc;
   const int d = H * hd;
   long n4 = (M * d) / 4;

@@ -311,7 +311,301 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// ----------------------------------------------------------------- backward --
+// One CTA per (batch, head, 128-key block), looping over the query blocks at or
+// below the diagonal.  Per query block t:
+//   S^T = K Q^T and dP^T = V dO^T          (M128 N128 K64, into TMEM)
+//   P^T = exp(scale S^T - LSE), dS^T = P^T (dP^T - D)   (elementwise warps)
+//   dV += P^T dO, dK += dS^T Q              (M128 N64 K128, TMEM accumulators)
+//   dQ  = dS K                              (A = the dS^T buffer read MN-major)
+// and dQ is reduced into an fp32 buffer.  Eight elementwise warps (two per TMEM
+// lane quarter, 64 of the 128 query columns each) need no row reductions here,
+// so they split the columns with no communication; the next block's S^T/dP^T
+// MMAs run while they work.
+constexpr int BS_K = 0, BS_V = TILE, BS_Q = 2 * TILE, BS_DO = 4 * TILE, BS_P = 6 * TILE, BS_DS = 8 * TILE;
+constexpr int BS_LD = 10 * TILE;                   // [2][LSE x128 | D x128] floats
+constexpr int BS_TILES = 10 * TILE + 2 * 256 * 4;
+// kv_full, qdo_full[2], qdo_empty[2], st_full, st_free, ps_full, mma2_done, drain
+constexpr int B_NUM_BARS = 10;
+constexpr int B_SMEM_BYTES = BS_TILES + 1024 + B_NUM_BARS * 8 + 16;
+constexpr int B_NUM_THREADS = 320;
+constexpr uint32_t C_ST = 0, C_DPT = 128, C_DV = 256, C_DK = 320, C_DQ = 384;
+// dQ = dS K: both operands read MN-major
+constexpr uint32_t IDESC_DQ =
+    (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+
+DEVI void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(B_NUM_THREADS, 1)
+    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
+                       const float* __restrict__ lse, const float* __restrict__ dvec, float* __restrict__ dq_acc,
+                       bf16* __restrict__ dqkv, int T, int H, float scale, float scale_log2, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  float* sLD = reinterpret_cast<float*>(base_ptr + BS_LD);
+  const uint32_t bars = base + BS_TILES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + BS_TILES + B_NUM_BARS * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t kv_full = bars;
+  auto qdo_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto qdo_empty = [&](int s) { return bars + 8u * (3 + s); };
+  const uint32_t st_full = bars + 8u * 5, st_free = bars + 8u * 6, ps_full = bars + 8u * 7;
+  const uint32_t mma2_done = bars + 8u * 8, drain_bar = bars + 8u * 9;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nq = (T + BQ - 1) / BQ;
+  const int kvb = blockIdx.x;  // low key blocks have the most query blocks: first
+  const int b = blockIdx.y / H, h = blockIdx.y % H;
+  const int d = H * HD;
+  const int kv0 = kvb * BKV;
+  const int nblk = nq - kvb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(qdo_full(s), 1);
+      mbar_init(qdo_empty(s), 1);
+    }
+    mbar_init(st_full, 1);
+    mbar_init(st_free, 256);
+    mbar_init(ps_full, 256);
+    mbar_init(mma2_done, 1);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tmQKV);
+    tma_prefetch_desc(&tmDO);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- TMA ----
+      int issued = 0;
+      bool ok = true;
+      mbar_arrive_expect_tx(kv_full, 2 * TILE);
+      tma_load_3d(base + BS_K, &tmQKV, kv_full, d + h * HD, kv0, b);
+      tma_load_3d(base + BS_V, &tmQKV, kv_full, 2 * d + h * HD, kv0, b);
+      for (int t = 0; t < nblk; ++t) {
+        const int buf = t & 1;
+        if (t >= 2 && !mbar_wait_bounded(qdo_empty(buf), ((t - 2) >> 1) & 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        const int q0 = (kvb + t) * BQ;
+        mbar_arrive_expect_tx(qdo_full(buf), 2 * TILE);
+        tma_load_3d(base + BS_Q + buf * TILE, &tmQKV, qdo_full(buf), h * HD, q0, b);
+        tma_load_3d(base + BS_DO + buf * TILE, &tmDO, qdo_full(buf), h * HD, q0, b);
+        ++issued;
+      }
+      if (!ok) {
+        mbar_drain_bounded(kv_full, 0);
+        for (int t = issued - 2 < 0 ? 0 : issued - 2; t < issued; ++t)
+          mbar_drain_bounded(qdo_full(t & 1), (t >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- MMA ----
+      bool ok = mbar_wait_bounded(kv_full, 0, abort_flag, err);
+      bool issued_any = false;
+      auto issue_s = [&](int t) -> bool {
+        const int buf = t & 1;
+        if (!mbar_wait_bounded(qdo_full(buf), (t >> 1) & 1, abort_flag, err)) return false;
+        if (t >= 1 && !mbar_wait_bounded(st_free, (t - 1) & 1, abort_flag, err)) return false;
+        tc_fence_after();
+        const uint32_t qb = base + BS_Q + buf * TILE, ob = base + BS_DO + buf * TILE;
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k)
+          tc_mma_bf16(tmem + C_ST, sdesc(base + BS_K + k * 32, 16, 1024), sdesc(qb + k * 32, 16, 1024), IDESC_S,
+                      k > 0 ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k)
+          tc_mma_bf16(tmem + C_DPT, sdesc(base + BS_V + k * 32, 16, 1024), sdesc(ob + k * 32, 16, 1024), IDESC_S,
+                      k > 0 ? 1u : 0u);
+        issued_any = true;
+        tc_commit(st_full);
+        return true;
+      };
+      auto issue_mma2 = [&](int t) -> bool {
+        const int buf = t & 1;
+        if (!mbar_wait_bounded(ps_full, t & 1, abort_flag, err)) return false;
+        tc_fence_after();
+        const uint32_t qb = base + BS_Q + buf * TILE, ob = base + BS_DO + buf * TILE;
+#pragma unroll
+        for (int k = 0; k < BQ / 16; ++k)
+          tc_mma_bf16(tmem + C_DV, sdesc(base + BS_P + (k >> 2) * TILE + (k & 3) * 32, 16, 1024),
+                      sdesc(ob + k * 2048, 8192, 1024), IDESC_O, (t > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < BQ / 16; ++k)
+          tc_mma_bf16(tmem + C_DK, sdesc(base + BS_DS + (k >> 2) * TILE + (k & 3) * 32, 16, 1024),
+                      sdesc(qb + k * 2048, 8192, 1024), IDESC_O, (t > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < BKV / 16; ++k)
+          tc_mma_bf16(tmem + C_DQ, sdesc(base + BS_DS + k * 2048, TILE, 1024),
+                      sdesc(base + BS_K + k * 2048, 8192, 1024), IDESC_DQ, k > 0 ? 1u : 0u);
+        tc_commit(mma2_done);
+        tc_commit(qdo_empty(buf));
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int t = 0; t < nblk && ok; ++t) {
+        if (t + 1 < nblk && !issue_s(t + 1)) { ok = false; break; }
+        if (!issue_mma2(t)) { ok = false; break; }
+      }
+      if (!ok && issued_any) {
+        tc_commit(drain_bar);
+        mbar_drain_bounded(drain_bar, 0);
+      }
+    }
+  } else {
+    // -------------------------------------------- elementwise + dQ drain ----
+    const int e = warp - 2;
+    const int q = warp & 3;    // TMEM lanes [32q, 32q+32)
+    const int half = e >> 2;   // query columns [64*half, 64*half+64)
+    const int row = q * 32 + lane;
+    const int kv = kv0 + row;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const int tid = threadIdx.x - 64;
+    bool ok = true;
+    auto drain_dq = [&](int t) {
+      // dQ rows are queries of block t; this warp takes 32 of the 64 columns
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tmem + lane_off + C_DQ + 32 * half, r);
+      tmem_ld_wait();
+      const int gq = (kvb + t) * BQ + row;
+      if (gq < T) {
+        float* dst = dq_acc + ((long)b * T + gq) * d + h * HD + 32 * half;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          red_add_v4(dst + 4 * j, __uint_as_float(r[4 * j]) * scale, __uint_as_float(r[4 * j + 1]) * scale,
+                     __uint_as_float(r[4 * j + 2]) * scale, __uint_as_float(r[4 * j + 3]) * scale);
+      }
+    };
+    for (int t = 0; t < nblk; ++t) {
+      const int q0 = (kvb + t) * BQ;
+      float* ld = sLD + (t & 1) * 256;
+      if (tid < 128) {
+        const int qq = q0 + tid;
+        ld[tid] = qq < T ? lse[((long)b * H + h) * T + qq] * LOG2E_F : INFINITY;
+      } else {
+        const int qq = q0 + tid - 128;
+        ld[tid] = qq < T ? dvec[((long)b * H + h) * T + qq] : 0.f;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (!mbar_wait_bounded(st_full, t & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t ppk[32], dpk[32];
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub) {
+        const int c0 = 64 * half + 32 * sub;
+        uint32_t s[32], dp[32];
+        tmem_ld_32x32b_x32(tmem + lane_off + C_ST + c0, s);
+        tmem_ld_32x32b_x32(tmem + lane_off + C_DPT + c0, dp);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int c = c0 + i + u;
+            const int qq = q0 + c;
+            float p = ex2(__uint_as_float(s[i + u]) * scale_log2 - ld[c]);
+            if (qq < kv || qq >= T || kv >= T) p = 0.f;
+            pv[u] = p;
+            dv[u] = p * (__uint_as_float(dp[i + u]) - ld[128 + c]);
+          }
+          ppk[sub * 16 + i / 2] = pack_bf16x2(pv[0], pv[1]);
+          dpk[sub * 16 + i / 2] = pack_bf16x2(dv[0], dv[1]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(st_free);
+      if (t >= 1) {
+        // block t-1's dV/dK/dQ MMAs are done: P/dS buffers and dQ are free
+        if (!mbar_wait_bounded(mma2_done, (t - 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        drain_dq(t - 1);
+      }
+      const uint32_t prow = base + BS_P + half * TILE + (uint32_t)row * 128u;
+      const uint32_t drow = base + BS_DS + half * TILE + (uint32_t)row * 128u;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t off = 16u * (uint32_t)(c ^ (row & 7));
+        st_shared_v4(prow + off, ppk[4 * c], ppk[4 * c + 1], ppk[4 * c + 2], ppk[4 * c + 3]);
+        st_shared_v4(drow + off, dpk[4 * c], dpk[4 * c + 1], dpk[4 * c + 2], dpk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(ps_full);
+    }
+    if (ok && mbar_wait_bounded(mma2_done, (nblk - 1) & 1, abort_flag, err)) {
+      tc_fence_after();
+      drain_dq(nblk - 1);
+      uint32_t rk[32], rv[32];
+      tmem_ld_32x32b_x32(tmem + lane_off + C_DK + 32 * half, rk);
+      tmem_ld_32x32b_x32(tmem + lane_off + C_DV + 32 * half, rv);
+      tmem_ld_wait();
+      if (kv < T) {
+        bf16* dst = dqkv + ((long)b * T + kv) * 3 * d + h * HD + 32 * half;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int o = 8 * j;
+          *reinterpret_cast<uint4*>(dst + d + o) = make_uint4(
+              pack_bf16x2(__uint_as_float(rk[o]) * scale, __uint_as_float(rk[o + 1]) * scale),
+              pack_bf16x2(__uint_as_float(rk[o + 2]) * scale, __uint_as_float(rk[o + 3]) * scale),
+              pack_bf16x2(__uint_as_float(rk[o + 4]) * scale, __uint_as_float(rk[o + 5]) * scale),
+              pack_bf16x2(__uint_as_float(rk[o + 6]) * scale, __uint_as_float(rk[o + 7]) * scale));
+          *reinterpret_cast<uint4*>(dst + 2 * d + o) = make_uint4(
+              pack_bf16x2(__uint_as_float(rv[o]), __uint_as_float(rv[o + 1])),
+              pack_bf16x2(__uint_as_float(rv[o + 2]), __uint_as_float(rv[o + 3])),
+              pack_bf16x2(__uint_as_float(rv[o + 4]), __uint_as_float(rv[o + 5])),
+              pack_bf16x2(__uint_as_float(rv[o + 6]), __uint_as_float(rv[o + 7])));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 }  // namespace
+
+int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float* dvec, void* dqkv, float* dq_acc,
+                int B, int T, int H, cudaStream_t st) {
+  if (B <= 0 || T <= 0) return GPT2_OK;
+  const uint64_t d = (uint64_t)H * HD;
+  CUtensorMap tq, tdo;
+  const uint64_t dq[3] = {3 * d, (uint64_t)T, (uint64_t)B};
+  const uint64_t sq[2] = {3 * d * 2, (uint64_t)T * 3 * d * 2};
+  const uint64_t dd[3] = {d, (uint64_t)T, (uint64_t)B};
+  const uint64_t sd[2] = {d * 2, (uint64_t)T * d * 2};
+  if (!tmap_3d(&tq, qkv, dq, sq) || !tmap_3d(&tdo, dout, dd, sd)) return GPT2_ERR_CUDA;
+  static bool attr = false;
+  if (!attr) {
+    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B_SMEM_BYTES));
+    attr = true;
+  }
+  dim3 grid((T + BKV - 1) / BKV, B * H);
+  attn_bwd_tc_kernel<<<grid, B_NUM_THREADS, B_SMEM_BYTES, st>>>(tq, tdo, lse, dvec, dq_acc, (bf16*)dqkv, T, H,
+                                                                 0.125f, LOG2E_F / 8.f, nullptr);
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
 
 int attn_fwd_tc(const void* qkv, void* o, float* lse, int B, int T, int H, cudaStream_t st) {
   if (B <= 0 || T <= 0) return GPT2_OK;

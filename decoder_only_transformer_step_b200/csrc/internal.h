@@ -50,8 +50,12 @@ int gemm_simt_f32(const GemmArgs& g, cudaStream_t st);
 
 int num_sms();
 
-// tcgen05 causal attention forward, head_dim 64 (bf16).
+// tcgen05 causal attention forward / backward, head_dim 64 (bf16).  The
+// backward expects dvec = rowsum(dO * O) and a zeroed fp32 dq_acc; it writes dK,
+// dV into dqkv and reduces scale * dQ into dq_acc.
 int attn_fwd_tc(const void* qkv, void* o, float* lse, int B, int T, int H, cudaStream_t st);
+int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float* dvec, void* dqkv, float* dq_acc,
+                int B, int T, int H, cudaStream_t st);
 
 // ---- attention ----------------------------------------------------------
 // qkv [B*T, 3*H*hd] (act), o [B*T, H*hd] (act), lse [B,H,T] fp32.
