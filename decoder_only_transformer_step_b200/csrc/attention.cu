@@ -688,7 +688,7 @@ int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* 
     attn_bwd_prep_bf16_kernel<16><<<(unsigned)((M + 7) / 8), 256, 0, st>>>((const bf16*)o, (const bf16*)dout,
                                                                            dvec, dq_acc, M, T, H);
   LAUNCH_CHECK();
-  int rc = (hd == 64 && !use_mma_bwd())
+  int rc = (hd == 64 && !use_mma_bwd() && T <= 4096)
                ? attn_bwd_tc(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st)
                : (hd == 64 ? launch_bwd<64>(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st)
                            : launch_bwd<16>(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st));

@@ -8,14 +8,14 @@
 // registers with the running-max correction (online softmax), and only O and
 // the per-row log-sum-exp reach HBM.
 //
-// One CTA per (batch, head, 128-query block), 192 threads:
+// One CTA per (batch, head, 128-query block), 320 threads:
 //   warp 0      TMA: Q once, K/V tiles into a 2-stage ring (a 3-D tensor map
 //               over the packed QKV activation; rows past T read as zeros)
 //   warp 1      TMEM allocation; tcgen05.mma S(j) = Q K_j^T (M128 N128 K64) into
 //               a double-buffered S, then O_tile(j-1) = P(j-1) V(j-1) (M128 N64
 //               K128, V as an MN-major operand) into a double-buffered O_tile
-//   warps 2..5  softmax of S(j) (row per thread, no shuffles), P(j) to shared
-//               memory, then fold O_tile(j-1) into the register accumulator
+//   warps 2..9  softmax of S(j) (two warps per row group, 64 keys each), P(j)
+//               to shared memory, then fold O_tile(j-1) into the registers
 // so S(j+1) is computed while the softmax of tile j runs.  Every mbarrier wait
 // is bounded; a timeout sets the device status and the CTA drains and exits.
 #include <cuda.h>
@@ -48,16 +48,18 @@ bool tmap_3d(CUtensorMap* tm, const void* base, const uint64_t* dims, const uint
 constexpr int HD = 64, BQ = 128, BKV = 128;
 constexpr int TILE = 128 * 128;  // one 128-row x 64-col bf16 tile, 128B-swizzled
 constexpr int SM_Q = 0;
-constexpr int SM_K = SM_Q + TILE;       // 2 stages
-constexpr int SM_V = SM_K + 2 * TILE;   // 2 stages
-constexpr int SM_P = SM_V + 2 * TILE;   // 2 buffers x (keys 0-63 | keys 64-127)
-constexpr int SM_TILES = SM_P + 4 * TILE;
-// q_full, kv_full[2], kv_empty[2], s_full[2], s_free[2], p_full[2], o_full[2], drain
-constexpr int NUM_BARS = 14;
+constexpr int KVS = 4;                    // K/V ring depth: loads run KVS-1 tiles ahead
+constexpr int SM_K = SM_Q + TILE;         // KVS stages
+constexpr int SM_V = SM_K + KVS * TILE;   // KVS stages
+constexpr int SM_P = SM_V + KVS * TILE;   // 2 buffers x (keys 0-63 | keys 64-127)
+constexpr int SM_XCHG = SM_P + 4 * TILE;  // [2][2][128] floats: row max / sum exchange
+constexpr int SM_TILES = SM_XCHG + 2 * 2 * 128 * 4;
+// q_full, kv_full[KVS], kv_empty[KVS], s_full[2], s_free[2], p_full[2], o_full[2], drain
+constexpr int NUM_BARS = 2 * KVS + 10;
 constexpr int SMEM_BYTES = SM_TILES + 1024 + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t S_COL = 0, O_COL = 256;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;  // TMA warp, MMA warp, 8 softmax warps
 
 #define LN2_F 0.6931471805599453f
 #define LOG2E_F 1.4426950408889634f
@@ -103,12 +105,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t q_full = bars;
   auto kv_full = [&](int s) { return bars + 8u * (1 + s); };
-  auto kv_empty = [&](int s) { return bars + 8u * (3 + s); };
-  auto s_full = [&](int s) { return bars + 8u * (5 + s); };
-  auto s_free = [&](int s) { return bars + 8u * (7 + s); };
-  auto p_full = [&](int s) { return bars + 8u * (9 + s); };
-  auto o_full = [&](int s) { return bars + 8u * (11 + s); };
-  const uint32_t drain_bar = bars + 8u * 13;
+  auto kv_empty = [&](int s) { return bars + 8u * (1 + KVS + s); };
+  auto s_full = [&](int s) { return bars + 8u * (1 + 2 * KVS + s); };
+  auto s_free = [&](int s) { return bars + 8u * (3 + 2 * KVS + s); };
+  auto p_full = [&](int s) { return bars + 8u * (5 + 2 * KVS + s); };
+  auto o_full = [&](int s) { return bars + 8u * (7 + 2 * KVS + s); };
+  const uint32_t drain_bar = bars + 8u * (9 + 2 * KVS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (T + BQ - 1) / BQ;
@@ -120,12 +122,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < KVS; ++s) {
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(s_full(s), 1);
-      mbar_init(s_free(s), 128);
-      mbar_init(p_full(s), 128);
+      mbar_init(s_free(s), 256);
+      mbar_init(p_full(s), 256);
       mbar_init(o_full(s), 1);
     }
     mbar_init(drain_bar, 1);
@@ -148,8 +152,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_arrive_expect_tx(q_full, TILE);
       tma_load_3d(base + SM_Q, &tmQKV, q_full, h * HD, q0, b);
       for (int j = 0; j < nkv; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait_bounded(kv_empty(st), ((j - 2) >> 1) & 1, abort_flag, err)) {
+        const int st = j % KVS;
+        if (j >= KVS && !mbar_wait_bounded(kv_empty(st), ((j - KVS) / KVS) & 1, abort_flag, err)) {
           ok = false;
           break;
         }
@@ -160,7 +164,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok) {
         mbar_drain_bounded(q_full, 0);
-        for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) mbar_drain_bounded(kv_full(j & 1), (j >> 1) & 1);
+        for (int j = issued - KVS < 0 ? 0 : issued - KVS; j < issued; ++j)
+          mbar_drain_bounded(kv_full(j % KVS), (j / KVS) & 1);
       }
     }
   } else if (warp == 1) {
@@ -173,28 +178,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait_bounded(p_full(pb), (t >> 1) & 1, abort_flag, err)) return false;
         tc_fence_after();
         const uint32_t pbase = base + SM_P + pb * 2 * TILE;
-        const uint32_t vbase = base + SM_V + (t & 1) * TILE;
+        const uint32_t vbase = base + SM_V + (t % KVS) * TILE;
 #pragma unroll
         for (int k = 0; k < BKV / 16; ++k)
           tc_mma_bf16(tmem + O_COL + pb * HD, sdesc(pbase + (k >> 2) * TILE + (k & 3) * 32, 16, 1024),
                       sdesc(vbase + k * 2048, 8192, 1024), IDESC_O, k > 0 ? 1u : 0u);
         tc_commit(o_full(pb));
-        tc_commit(kv_empty(t & 1));
+        tc_commit(kv_empty(t % KVS));
         return true;
       };
       if (ok) tc_fence_after();
       for (int j = 0; j < nkv && ok; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait_bounded(kv_full(st), (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait_bounded(s_free(st), ((j - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        const int st = j % KVS, sb = j & 1;
+        if (!mbar_wait_bounded(kv_full(st), (j / KVS) & 1, abort_flag, err)) { ok = false; break; }
+        if (j >= 2 && !mbar_wait_bounded(s_free(sb), ((j - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t kbase = base + SM_K + st * TILE;
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k)
-          tc_mma_bf16(tmem + S_COL + st * BKV, sdesc(base + SM_Q + k * 32, 16, 1024), sdesc(kbase + k * 32, 16, 1024),
+          tc_mma_bf16(tmem + S_COL + sb * BKV, sdesc(base + SM_Q + k * 32, 16, 1024), sdesc(kbase + k * 32, 16, 1024),
                       IDESC_S, k > 0 ? 1u : 0u);
         issued_any = true;
-        tc_commit(s_full(st));
+        tc_commit(s_full(sb));
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok) ok = issue_pv(nkv - 1);
@@ -205,28 +210,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------- softmax ----
+    // Eight warps: two per TMEM lane quarter, each owning 64 of the 128 key
+    // columns of its rows and 32 of the 64 output columns; the two halves of
+    // a row exchange partial maxima (per tile) and sums (at the end) through
+    // shared memory.
+    const int e = warp - 2;
     const int q = warp & 3;  // TMEM lanes [32q, 32q+32)
+    const int half = e >> 2;
     const int row = q * 32 + lane;
     const int grow = q0 + row;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    float* xchg = reinterpret_cast<float*>(base_ptr + SM_XCHG);  // [parity][half][128 rows]
     float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
-    float acc[HD];
+    float acc[32];
 #pragma unroll
-    for (int i = 0; i < HD; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
     bool ok = true;
     auto fold = [&](int t, float a) -> bool {
       const int ob = t & 1;
       if (!mbar_wait_bounded(o_full(ob), (t >> 1) & 1, abort_flag, err)) return false;
       tc_fence_after();
-      uint32_t r0[32], r1[32];
-      tmem_ld_32x32b_x32(tmem + lane_off + O_COL + ob * HD, r0);
-      tmem_ld_32x32b_x32(tmem + lane_off + O_COL + ob * HD + 32, r1);
+      uint32_t r0[32];
+      tmem_ld_32x32b_x32(tmem + lane_off + O_COL + ob * HD + 32 * half, r0);
       tmem_ld_wait();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        acc[i] = acc[i] * a + __uint_as_float(r0[i]);
-        acc[32 + i] = acc[32 + i] * a + __uint_as_float(r1[i]);
-      }
+      for (int i = 0; i < 32; ++i) acc[i] = acc[i] * a + __uint_as_float(r0[i]);
       tc_fence_before();
       return true;
     };
@@ -234,29 +242,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int sb = j & 1;
       if (!mbar_wait_bounded(s_full(sb), (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
-      uint32_t r[4][32];
+      uint32_t r[2][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem + lane_off + S_COL + sb * BKV + 32 * c, r[c]);
+      for (int c = 0; c < 2; ++c)
+        tmem_ld_32x32b_x32(tmem + lane_off + S_COL + sb * BKV + 64 * half + 32 * c, r[c]);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(s_free(sb));
       const bool diag = (j == nkv - 1);
-      const int kv0 = j * BKV;
-      float mx = m;
+      const int kc0 = j * BKV + 64 * half;
+      float pmax = m;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           float v = __uint_as_float(r[c][i]) * scale_log2;
-          if (diag && kv0 + 32 * c + i > grow) v = -INFINITY;
+          if (diag && kc0 + 32 * c + i > grow) v = -INFINITY;
           r[c][i] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          pmax = fmaxf(pmax, v);
         }
+      float* xp = xchg + (j & 1) * 256;
+      xp[half * 128 + row] = pmax;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const float mx = fmaxf(pmax, xp[(1 - half) * 128 + row]);
       const float alpha = ex2(m - mx);
       m = mx;
       float sum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float p = ex2(__uint_as_float(r[c][i]) - m);
@@ -264,12 +277,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           sum += p;
         }
       l = l * alpha + sum;
-      // P row -> shared memory, 128B-swizzled K-major (keys 0-63 | 64-127)
-      const uint32_t pb = base + SM_P + sb * 2 * TILE + (uint32_t)row * 128u;
+      // this half's 64 keys of the P row -> its 128B-swizzled K-major block
+      const uint32_t pb = base + SM_P + sb * 2 * TILE + half * TILE + (uint32_t)row * 128u;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
+      for (int c = 0; c < 8; ++c) {
         const int g = c >> 2, o8 = (c & 3) * 8;
-        st_shared_v4(pb + (uint32_t)(c >> 3) * TILE + 16u * (uint32_t)((c & 7) ^ (row & 7)),
+        st_shared_v4(pb + 16u * (uint32_t)(c ^ (row & 7)),
                      pack_bf16x2(__uint_as_float(r[g][o8 + 0]), __uint_as_float(r[g][o8 + 1])),
                      pack_bf16x2(__uint_as_float(r[g][o8 + 2]), __uint_as_float(r[g][o8 + 3])),
                      pack_bf16x2(__uint_as_float(r[g][o8 + 4]), __uint_as_float(r[g][o8 + 5])),
@@ -281,21 +294,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       alpha_prev = alpha;
     }
     if (ok) ok = fold(nkv - 1, alpha_prev);
+    // row sum = both halves' partial sums (both were kept relative to the same m)
+    float* xs = xchg + (nkv & 1) * 256;
+    xs[half * 128 + row] = l;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    l += xs[(1 - half) * 128 + row];
     if (ok) {
       // O / l -> shared memory (the Q tile is no longer read) -> one TMA store
       const float inv = 1.f / l;
       const uint32_t ob = base + SM_Q + (uint32_t)row * 128u;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_shared_v4(ob + 16u * (uint32_t)(c ^ (row & 7)), pack_bf16x2(acc[8 * c] * inv, acc[8 * c + 1] * inv),
+      for (int c = 0; c < 4; ++c)
+        st_shared_v4(ob + 16u * (uint32_t)((4 * half + c) ^ (row & 7)),
+                     pack_bf16x2(acc[8 * c] * inv, acc[8 * c + 1] * inv),
                      pack_bf16x2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv),
                      pack_bf16x2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv),
                      pack_bf16x2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv));
-      if (grow < T) lse[((long)b * H + h) * T + grow] = (m + __log2f(l)) * LN2_F;
+      if (half == 0 && grow < T) lse[((long)b * H + h) * T + grow] = (m + __log2f(l)) * LN2_F;
       fence_proxy_async_smem();
     }
-    // all four softmax warps arrive here (an abort makes every wait return)
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    // all eight softmax warps arrive here (an abort makes every wait return)
+    asm volatile("bar.sync 1, 256;" ::: "memory");
     if (warp == 2 && lane == 0 && !*abort_flag) {
       tma_store_3d(&tmO, base + SM_Q, h * HD, q0, b);
       bulk_commit();
@@ -322,11 +341,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // lane quarter, 64 of the 128 query columns each) need no row reductions here,
 // so they split the columns with no communication; the next block's S^T/dP^T
 // MMAs run while they work.
-constexpr int BS_K = 0, BS_V = TILE, BS_Q = 2 * TILE, BS_DO = 4 * TILE, BS_P = 6 * TILE, BS_DS = 8 * TILE;
-constexpr int BS_LD = 10 * TILE;                   // [2][LSE x128 | D x128] floats
-constexpr int BS_TILES = 10 * TILE + 2 * 256 * 4;
-// kv_full, qdo_full[2], qdo_empty[2], st_full, st_free, ps_full, mma2_done, drain
-constexpr int B_NUM_BARS = 10;
+constexpr int QS = 3;  // Q/dO ring depth: loads run QS-1 query blocks ahead
+constexpr int BS_K = 0, BS_V = TILE, BS_Q = 2 * TILE, BS_DO = BS_Q + QS * TILE, BS_P = BS_DO + QS * TILE;
+constexpr int BS_DS = BS_P + 2 * TILE;
+constexpr int BS_MAX_QBLOCKS = 32;  // T <= 4096
+constexpr int BS_LD = BS_DS + 2 * TILE;  // [query block][LSE x128 | D x128] floats
+constexpr int BS_TILES = BS_LD + BS_MAX_QBLOCKS * 256 * 4;
+// kv_full, qdo_full[QS], qdo_empty[QS], st_full, st_free, ps_full, mma2_done, drain
+constexpr int B_NUM_BARS = 2 * QS + 6;
 constexpr int B_SMEM_BYTES = BS_TILES + 1024 + B_NUM_BARS * 8 + 16;
 constexpr int B_NUM_THREADS = 320;
 constexpr uint32_t C_ST = 0, C_DPT = 128, C_DV = 256, C_DK = 320, C_DQ = 384;
@@ -353,9 +375,10 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t kv_full = bars;
   auto qdo_full = [&](int s) { return bars + 8u * (1 + s); };
-  auto qdo_empty = [&](int s) { return bars + 8u * (3 + s); };
-  const uint32_t st_full = bars + 8u * 5, st_free = bars + 8u * 6, ps_full = bars + 8u * 7;
-  const uint32_t mma2_done = bars + 8u * 8, drain_bar = bars + 8u * 9;
+  auto qdo_empty = [&](int s) { return bars + 8u * (1 + QS + s); };
+  const uint32_t st_full = bars + 8u * (1 + 2 * QS), st_free = bars + 8u * (2 + 2 * QS);
+  const uint32_t ps_full = bars + 8u * (3 + 2 * QS);
+  const uint32_t mma2_done = bars + 8u * (4 + 2 * QS), drain_bar = bars + 8u * (5 + 2 * QS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nq = (T + BQ - 1) / BQ;
@@ -367,7 +390,7 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < QS; ++s) {
       mbar_init(qdo_full(s), 1);
       mbar_init(qdo_empty(s), 1);
     }
@@ -396,8 +419,8 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
       tma_load_3d(base + BS_K, &tmQKV, kv_full, d + h * HD, kv0, b);
       tma_load_3d(base + BS_V, &tmQKV, kv_full, 2 * d + h * HD, kv0, b);
       for (int t = 0; t < nblk; ++t) {
-        const int buf = t & 1;
-        if (t >= 2 && !mbar_wait_bounded(qdo_empty(buf), ((t - 2) >> 1) & 1, abort_flag, err)) {
+        const int buf = t % QS;
+        if (t >= QS && !mbar_wait_bounded(qdo_empty(buf), ((t - QS) / QS) & 1, abort_flag, err)) {
           ok = false;
           break;
         }
@@ -409,8 +432,8 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
       }
       if (!ok) {
         mbar_drain_bounded(kv_full, 0);
-        for (int t = issued - 2 < 0 ? 0 : issued - 2; t < issued; ++t)
-          mbar_drain_bounded(qdo_full(t & 1), (t >> 1) & 1);
+        for (int t = issued - QS < 0 ? 0 : issued - QS; t < issued; ++t)
+          mbar_drain_bounded(qdo_full(t % QS), (t / QS) & 1);
       }
     }
   } else if (warp == 1) {
@@ -419,8 +442,8 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
       bool ok = mbar_wait_bounded(kv_full, 0, abort_flag, err);
       bool issued_any = false;
       auto issue_s = [&](int t) -> bool {
-        const int buf = t & 1;
-        if (!mbar_wait_bounded(qdo_full(buf), (t >> 1) & 1, abort_flag, err)) return false;
+        const int buf = t % QS;
+        if (!mbar_wait_bounded(qdo_full(buf), (t / QS) & 1, abort_flag, err)) return false;
         if (t >= 1 && !mbar_wait_bounded(st_free, (t - 1) & 1, abort_flag, err)) return false;
         tc_fence_after();
         const uint32_t qb = base + BS_Q + buf * TILE, ob = base + BS_DO + buf * TILE;
@@ -437,7 +460,7 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
         return true;
       };
       auto issue_mma2 = [&](int t) -> bool {
-        const int buf = t & 1;
+        const int buf = t % QS;
         if (!mbar_wait_bounded(ps_full, t & 1, abort_flag, err)) return false;
         tc_fence_after();
         const uint32_t qb = base + BS_Q + buf * TILE, ob = base + BS_DO + buf * TILE;
@@ -491,17 +514,20 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
                      __uint_as_float(r[4 * j + 2]) * scale, __uint_as_float(r[4 * j + 3]) * scale);
       }
     };
+    // LSE (log2 domain) and D of every query block this CTA visits, once:
+    // [block][LSE x128 | D x128]; queries past T get LSE = +inf (P = 0).
+    for (int i = tid; i < nblk * 256; i += 256) {
+      const int blk = i >> 8, k = i & 255;
+      const int qq = (kvb + blk) * BQ + (k & 127);
+      const long gi = ((long)b * H + h) * T + qq;
+      sLD[i] = k < 128 ? (qq < T ? lse[gi] * LOG2E_F : INFINITY) : (qq < T ? dvec[gi] : 0.f);
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
     for (int t = 0; t < nblk; ++t) {
       const int q0 = (kvb + t) * BQ;
-      float* ld = sLD + (t & 1) * 256;
-      if (tid < 128) {
-        const int qq = q0 + tid;
-        ld[tid] = qq < T ? lse[((long)b * H + h) * T + qq] * LOG2E_F : INFINITY;
-      } else {
-        const int qq = q0 + tid - 128;
-        ld[tid] = qq < T ? dvec[((long)b * H + h) * T + qq] : 0.f;
-      }
-      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const float* ld = sLD + t * 256;
+      // masking only on the diagonal block, past T, or for keys past T
+      const bool need_mask = (t == 0) || (q0 + BQ > T) || (kv >= T);
       if (!mbar_wait_bounded(st_full, t & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
       uint32_t ppk[32], dpk[32];
@@ -513,19 +539,26 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
         tmem_ld_32x32b_x32(tmem + lane_off + C_DPT + c0, dp);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float pv[2], dv[2];
+        for (int i = 0; i < 32; i += 4) {
+          // broadcast reads: every lane needs the same four columns
+          const float4 l4 = *reinterpret_cast<const float4*>(ld + c0 + i);
+          const float4 d4 = *reinterpret_cast<const float4*>(ld + 128 + c0 + i);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], dv[4];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = c0 + i + u;
-            const int qq = q0 + c;
-            float p = ex2(__uint_as_float(s[i + u]) * scale_log2 - ld[c]);
-            if (qq < kv || qq >= T || kv >= T) p = 0.f;
+          for (int u = 0; u < 4; ++u) {
+            float p = ex2(fmaf(__uint_as_float(s[i + u]), scale_log2, -lv[u]));
+            if (need_mask) {
+              const int qq = q0 + c0 + i + u;
+              if (qq < kv || qq >= T || kv >= T) p = 0.f;
+            }
             pv[u] = p;
-            dv[u] = p * (__uint_as_float(dp[i + u]) - ld[128 + c]);
+            dv[u] = p * (__uint_as_float(dp[i + u]) - dd[u]);
           }
           ppk[sub * 16 + i / 2] = pack_bf16x2(pv[0], pv[1]);
+          ppk[sub * 16 + i / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
           dpk[sub * 16 + i / 2] = pack_bf16x2(dv[0], dv[1]);
+          dpk[sub * 16 + i / 2 + 1] = pack_bf16x2(dv[2], dv[3]);
         }
       }
       tc_fence_before();
@@ -588,6 +621,7 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
 int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float* dvec, void* dqkv, float* dq_acc,
                 int B, int T, int H, cudaStream_t st) {
   if (B <= 0 || T <= 0) return GPT2_OK;
+  if ((T + BQ - 1) / BQ > BS_MAX_QBLOCKS) return GPT2_ERR_UNSUPPORTED_SHAPE;
   const uint64_t d = (uint64_t)H * HD;
   CUtensorMap tq, tdo;
   const uint64_t dq[3] = {3 * d, (uint64_t)T, (uint64_t)B};

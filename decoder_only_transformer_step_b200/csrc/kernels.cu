@@ -176,136 +176,104 @@ __global__ void ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ g, 
 }
 
 // dx = rstd * (dxhat - mean(dxhat) - xhat * mean(dxhat * xhat)), dxhat = dy * g;
-// dres = (init ? 0 : dres) + dx.  dgamma += dy * xhat, dbeta += dy, reduced in a
-// fixed order over the CTA's rows into part[blockIdx.x][0:d] and [d:2d].
-// A fixed grid (at most LNB_MAX_CTAS) of 8-warp CTAs; each warp strides over
-// rows and fetches the next row's x, dy, dres while it computes the current.
-constexpr int LNB_WARPS = 8;
-constexpr int LNB_MAX_CTAS = 512;
-
-DEVI uint4 ld16(const void* p) { return *reinterpret_cast<const uint4*>(p); }
-template <typename T>
-DEVI void unpack16(const uint4& u, float (&f)[Vec<T>::N]);
-template <>
-DEVI void unpack16<bf16>(const uint4& u, float (&f)[8]) {
-  f[0] = bf16lo(u.x); f[1] = bf16hi(u.x); f[2] = bf16lo(u.y); f[3] = bf16hi(u.y);
-  f[4] = bf16lo(u.z); f[5] = bf16hi(u.z); f[6] = bf16lo(u.w); f[7] = bf16hi(u.w);
-}
-template <>
-DEVI void unpack16<float>(const uint4& u, float (&f)[4]) {
-  f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
-  f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
-}
-
+// dres = (init ? 0 : dres) + dx.  One warp per row with the row in registers;
+// no per-thread accumulators, so many warps are resident to cover HBM latency.
 template <typename T, int NC>
-__global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ x,
-                                                     const float* __restrict__ mean,
-                                                     const float* __restrict__ rstd, const T* __restrict__ g,
-                                                     T* __restrict__ dres, int dres_init,
-                                                     float* __restrict__ part, int M, int d) {
+__global__ void __launch_bounds__(256) ln_bwd_dx_kernel(const T* __restrict__ dy, const T* __restrict__ x,
+                                                        const float* __restrict__ mean,
+                                                        const float* __restrict__ rstd,
+                                                        const T* __restrict__ g, T* __restrict__ dres,
+                                                        int dres_init, int M, int d) {
   constexpr int VN = Vec<T>::N;
-  extern __shared__ float red[];  // [2d]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float gg[NC][VN], dg[NC][VN], db[NC][VN];
+  const int m = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (m >= M) return;
+  const float mu = mean[m], rs = rstd[m];
+  float xh[NC][VN], gd[NC][VN];
+  float s1 = 0.f, s2 = 0.f;
 #pragma unroll
   for (int k = 0; k < NC; ++k) {
     const int c = (lane + 32 * k) * VN;
+    if (c < d) {
+      float xv[VN], dv[VN], gv[VN];
+      Vec<T>::load(x + (long)m * d + c, xv);
+      Vec<T>::load(dy + (long)m * d + c, dv);
+      Vec<T>::load(g + c, gv);
 #pragma unroll
-    for (int j = 0; j < VN; ++j) dg[k][j] = db[k][j] = 0.f;
-    if (c < d) Vec<T>::load(g + c, gg[k]);
-  }
-  const int nwarps = gridDim.x * LNB_WARPS;
-  uint4 px[NC], pd[NC], pr[NC];
-  float pmu = 0.f, prs = 0.f;
-#define LNB_FETCH(mm)                                              \
-  do {                                                             \
-    _Pragma("unroll") for (int k = 0; k < NC; ++k) {               \
-      const int c = (lane + 32 * k) * VN;                          \
-      if (c < d) {                                                 \
-        px[k] = ld16(x + (long)(mm) * d + c);                      \
-        pd[k] = ld16(dy + (long)(mm) * d + c);                     \
-        if (!dres_init) pr[k] = ld16(dres + (long)(mm) * d + c);   \
-      }                                                            \
-    }                                                              \
-    pmu = mean[mm];                                                \
-    prs = rstd[mm];                                                \
-  } while (0)
-  int m = blockIdx.x * LNB_WARPS + warp;
-  if (m < M) LNB_FETCH(m);
-  for (; m < M; m += nwarps) {
-    uint4 cx[NC], cd[NC], cr[NC];
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-      cx[k] = px[k];
-      cd[k] = pd[k];
-      cr[k] = pr[k];
-    }
-    const float mu = pmu, rs = prs;
-    if (m + nwarps < M) LNB_FETCH(m + nwarps);
-    float xv[NC][VN], dv[NC][VN];
-    float s1 = 0.f, s2 = 0.f;
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-      const int c = (lane + 32 * k) * VN;
-      if (c < d) {
-        unpack16<T>(cx[k], xv[k]);
-        unpack16<T>(cd[k], dv[k]);
-#pragma unroll
-        for (int j = 0; j < VN; ++j) {
-          const float xh = (xv[k][j] - mu) * rs;
-          xv[k][j] = xh;
-          const float gh = dv[k][j] * gg[k][j];
-          s1 += gh;
-          s2 += gh * xh;
-          dg[k][j] += dv[k][j] * xh;
-          db[k][j] += dv[k][j];
-        }
-      }
-    }
-    s1 = warp_sum(s1) / d;
-    s2 = warp_sum(s2) / d;
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-      const int c = (lane + 32 * k) * VN;
-      if (c < d) {
-        float o[VN];
-        if (!dres_init) {
-          unpack16<T>(cr[k], o);
-        } else {
-#pragma unroll
-          for (int j = 0; j < VN; ++j) o[j] = 0.f;
-        }
-#pragma unroll
-        for (int j = 0; j < VN; ++j) o[j] += rs * (dv[k][j] * gg[k][j] - s1 - xv[k][j] * s2);
-        Vec<T>::store(dres + (long)m * d + c, o);
+      for (int j = 0; j < VN; ++j) {
+        xh[k][j] = (xv[j] - mu) * rs;
+        gd[k][j] = dv[j] * gv[j];
+        s1 += gd[k][j];
+        s2 += gd[k][j] * xh[k][j];
       }
     }
   }
-  // fixed-order reduction over the CTA's warps
-  for (int w = 0; w < LNB_WARPS; ++w) {
-    if (warp == w) {
+  s1 = warp_sum(s1) / d;
+  s2 = warp_sum(s2) / d;
 #pragma unroll
-      for (int k = 0; k < NC; ++k) {
-        const int c = (lane + 32 * k) * VN;
-        if (c < d) {
+  for (int k = 0; k < NC; ++k) {
+    const int c = (lane + 32 * k) * VN;
+    if (c < d) {
+      float o[VN];
+      if (!dres_init) {
+        Vec<T>::load(dres + (long)m * d + c, o);
+      } else {
 #pragma unroll
-          for (int j = 0; j < VN; ++j) {
-            if (w == 0) {
-              red[c + j] = dg[k][j];
-              red[d + c + j] = db[k][j];
-            } else {
-              red[c + j] += dg[k][j];
-              red[d + c + j] += db[k][j];
-            }
-          }
-        }
+        for (int j = 0; j < VN; ++j) o[j] = 0.f;
       }
+#pragma unroll
+      for (int j = 0; j < VN; ++j) o[j] += rs * (gd[k][j] - s1 - xh[k][j] * s2);
+      Vec<T>::store(dres + (long)m * d + c, o);
     }
-    __syncthreads();
   }
-  for (int i = threadIdx.x; i < 2 * d; i += blockDim.x) part[(long)blockIdx.x * 2 * d + i] = red[i];
 }
-#undef LNB_FETCH
+
+// LayerNorm parameter gradients: dgamma = sum_m dy * xhat, dbeta = sum_m dy,
+// per block of LNP_ROWS rows (fixed order) into part[rowblock][0:d | d:2d].
+constexpr int LNP_ROWS = 128;
+
+template <typename T>
+__global__ void __launch_bounds__(256) ln_param_colsum_kernel(const T* __restrict__ dy, const T* __restrict__ x,
+                                                              const float* __restrict__ mean,
+                                                              const float* __restrict__ rstd, int M, int d,
+                                                              float* __restrict__ part) {
+  constexpr int VN = Vec<T>::N;
+  __shared__ float red[8][2][32 * VN];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = (blockIdx.x * 32 + lane) * VN;
+  const int r0 = blockIdx.y * LNP_ROWS;
+  float sg[VN], sb[VN];
+#pragma unroll
+  for (int j = 0; j < VN; ++j) sg[j] = sb[j] = 0.f;
+  if (c < d) {
+    for (int r = r0 + warp; r < min(r0 + LNP_ROWS, M); r += 8) {
+      const float mu = mean[r], rs = rstd[r];
+      float xv[VN], dv[VN];
+      Vec<T>::load(x + (long)r * d + c, xv);
+      Vec<T>::load(dy + (long)r * d + c, dv);
+#pragma unroll
+      for (int j = 0; j < VN; ++j) {
+        sg[j] += dv[j] * (xv[j] - mu) * rs;
+        sb[j] += dv[j];
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < VN; ++j) {
+    red[warp][0][lane * VN + j] = sg[j];
+    red[warp][1][lane * VN + j] = sb[j];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 2 * 32 * VN; i += 256) {
+    const int which = i / (32 * VN), k = i % (32 * VN);
+    const int col = blockIdx.x * 32 * VN + k;
+    if (col < d) {
+      float t = red[0][which][k];
+      for (int w = 1; w < 8; ++w) t += red[w][which][k];
+      part[(long)blockIdx.y * 2 * d + which * d + col] = t;
+    }
+  }
+}
 
 // grad[j] = beta * grad[j] + sum_r part[r, j] (r ascending); 8 row slices per
 // column reduced in a fixed order.
@@ -591,16 +559,15 @@ int ln_fwd_dispatch(const void* x, const void* g, const void* b, void* y, float*
   return GPT2_OK;
 }
 
-int ln_bwd_blocks(int M) {
-  const int b = (M + LNB_WARPS - 1) / LNB_WARPS;
-  return b < LNB_MAX_CTAS ? b : LNB_MAX_CTAS;
-}
-
 template <typename T, int NC>
 void ln_bwd_launch(const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
                    void* dres, int init, float* part, int M, int d, cudaStream_t st) {
-  ln_bwd_kernel<T, NC><<<ln_bwd_blocks(M), 256, 2 * d * sizeof(float), st>>>(
-      (const T*)dy, (const T*)x, mean, rstd, (const T*)g, (T*)dres, init, part, M, d);
+  ln_bwd_dx_kernel<T, NC><<<(M + 7) / 8, 256, 0, st>>>((const T*)dy, (const T*)x, mean, rstd, (const T*)g,
+                                                       (T*)dres, init, M, d);
+  gpt2_count_launch();
+  constexpr int VN = Vec<T>::N;
+  dim3 grid((d + 32 * VN - 1) / (32 * VN), (M + LNP_ROWS - 1) / LNP_ROWS);
+  ln_param_colsum_kernel<T><<<grid, 256, 0, st>>>((const T*)dy, (const T*)x, mean, rstd, M, d, part);
 }
 
 template <typename T>
@@ -645,11 +612,11 @@ int layernorm_fwd(int f32, const void* x, const void* g, const void* b, void* y,
              : ln_fwd_dispatch<bf16>(x, g, b, y, mean, rstd, M, d, st);
 }
 
-size_t layernorm_bwd_part_floats(int M, int d) { return (size_t)ln_bwd_blocks(M) * 2 * d; }
+size_t layernorm_bwd_part_floats(int M, int d) { return (size_t)((M + LNP_ROWS - 1) / LNP_ROWS) * 2 * d; }
 
 int layernorm_bwd(int f32, const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
                   void* dres, int dres_init, float* part, int* nblk, int M, int d, cudaStream_t st) {
-  *nblk = ln_bwd_blocks(M);
+  *nblk = (M + LNP_ROWS - 1) / LNP_ROWS;
   return f32 ? ln_bwd_dispatch<float>(dy, x, mean, rstd, g, dres, dres_init, part, M, d, st)
              : ln_bwd_dispatch<bf16>(dy, x, mean, rstd, g, dres, dres_init, part, M, d, st);
 }
