@@ -351,6 +351,8 @@ constexpr int BS_TILES = BS_LD + BS_MAX_QBLOCKS * 256 * 4;
 constexpr int B_NUM_BARS = 2 * QS + 6;
 constexpr int B_SMEM_BYTES = BS_TILES + 1024 + B_NUM_BARS * 8 + 16;
 constexpr int B_NUM_THREADS = 320;
+// dQ is double-buffered (C_DQ + 64 * (t & 1)) so block t's MMAs never wait for
+// block t-1's dQ to be drained.
 constexpr uint32_t C_ST = 0, C_DPT = 128, C_DV = 256, C_DK = 320, C_DQ = 384;
 // dQ = dS K: both operands read MN-major
 constexpr uint32_t IDESC_DQ =
@@ -474,7 +476,7 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
                       sdesc(qb + k * 2048, 8192, 1024), IDESC_O, (t > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
         for (int k = 0; k < BKV / 16; ++k)
-          tc_mma_bf16(tmem + C_DQ, sdesc(base + BS_DS + k * 2048, TILE, 1024),
+          tc_mma_bf16(tmem + C_DQ + 64 * (t & 1), sdesc(base + BS_DS + k * 2048, TILE, 1024),
                       sdesc(base + BS_K + k * 2048, 8192, 1024), IDESC_DQ, k > 0 ? 1u : 0u);
         tc_commit(mma2_done);
         tc_commit(qdo_empty(buf));
@@ -503,7 +505,7 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
     auto drain_dq = [&](int t) {
       // dQ rows are queries of block t; this warp takes 32 of the 64 columns
       uint32_t r[32];
-      tmem_ld_32x32b_x32(tmem + lane_off + C_DQ + 32 * half, r);
+      tmem_ld_32x32b_x32(tmem + lane_off + C_DQ + 64 * (t & 1) + 32 * half, r);
       tmem_ld_wait();
       const int gq = (kvb + t) * BQ + row;
       if (gq < T) {
@@ -530,14 +532,24 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
       const bool need_mask = (t == 0) || (q0 + BQ > T) || (kv >= T);
       if (!mbar_wait_bounded(st_full, t & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
+      // this warp's S^T / dP^T columns in two batches: the second batch is in
+      // flight while the first is processed, and TMEM is released as soon as
+      // it has landed so block t+1's S^T/dP^T MMAs overlap the math below
+      uint32_t s[2][32], dp[2][32];
+      tmem_ld_32x32b_x32(tmem + lane_off + C_ST + 64 * half, s[0]);
+      tmem_ld_32x32b_x32(tmem + lane_off + C_DPT + 64 * half, dp[0]);
+      tmem_ld_wait();
+      tmem_ld_32x32b_x32(tmem + lane_off + C_ST + 64 * half + 32, s[1]);
+      tmem_ld_32x32b_x32(tmem + lane_off + C_DPT + 64 * half + 32, dp[1]);
       uint32_t ppk[32], dpk[32];
 #pragma unroll
       for (int sub = 0; sub < 2; ++sub) {
+        if (sub == 1) {
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(st_free);
+        }
         const int c0 = 64 * half + 32 * sub;
-        uint32_t s[32], dp[32];
-        tmem_ld_32x32b_x32(tmem + lane_off + C_ST + c0, s);
-        tmem_ld_32x32b_x32(tmem + lane_off + C_DPT + c0, dp);
-        tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           // broadcast reads: every lane needs the same four columns
@@ -547,13 +559,13 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
           float pv[4], dv[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            float p = ex2(fmaf(__uint_as_float(s[i + u]), scale_log2, -lv[u]));
+            float p = ex2(fmaf(__uint_as_float(s[sub][i + u]), scale_log2, -lv[u]));
             if (need_mask) {
               const int qq = q0 + c0 + i + u;
               if (qq < kv || qq >= T || kv >= T) p = 0.f;
             }
             pv[u] = p;
-            dv[u] = p * (__uint_as_float(dp[i + u]) - dd[u]);
+            dv[u] = p * (__uint_as_float(dp[sub][i + u]) - dd[u]);
           }
           ppk[sub * 16 + i / 2] = pack_bf16x2(pv[0], pv[1]);
           ppk[sub * 16 + i / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
@@ -561,14 +573,10 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
           dpk[sub * 16 + i / 2 + 1] = pack_bf16x2(dv[2], dv[3]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(st_free);
-      if (t >= 1) {
-        // block t-1's dV/dK/dQ MMAs are done: P/dS buffers and dQ are free
-        if (!mbar_wait_bounded(mma2_done, (t - 1) & 1, abort_flag, err)) { ok = false; break; }
-        tc_fence_after();
-        drain_dq(t - 1);
-      }
+      // block t-1's dV/dK/dQ MMAs read P/dS: they must be done before the
+      // buffers are overwritten (and before dQ(t-1) is drained below)
+      if (t >= 1 && !mbar_wait_bounded(mma2_done, (t - 1) & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after();
       const uint32_t prow = base + BS_P + half * TILE + (uint32_t)row * 128u;
       const uint32_t drow = base + BS_DS + half * TILE + (uint32_t)row * 128u;
 #pragma unroll
@@ -580,6 +588,11 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(ps_full);
+      // dQ of block t-1 sits in the other TMEM buffer; reducing it into global
+      // memory only after the release keeps these reductions off the MMA path.
+      // Block t+1's dQ MMAs reuse that buffer only after this thread's next
+      // ps_full arrival, which follows the completed loads below.
+      if (t >= 1) drain_dq(t - 1);
     }
     if (ok && mbar_wait_bounded(mma2_done, (nblk - 1) & 1, abort_flag, err)) {
       tc_fence_after();
