@@ -47,16 +47,21 @@ bool tmap_3d(CUtensorMap* tm, const void* base, const uint64_t* dims, const uint
 
 constexpr int HD = 64, BQ = 128, BKV = 128;
 constexpr int TILE = 128 * 128;  // one 128-row x 64-col bf16 tile, 128B-swizzled
+// forward shared memory: Q (2 buffers: the next work item's Q loads while the
+// current one runs; a finished item's O is staged in its Q buffer), a KVS-deep
+// K/V ring, P (2 buffers x keys 0-63 | keys 64-127), row max / sum exchange
 constexpr int SM_Q = 0;
-constexpr int KVS = 4;                    // K/V ring depth: loads run KVS-1 tiles ahead
-constexpr int SM_K = SM_Q + TILE;         // KVS stages
+constexpr int KVS = 3;                    // K/V ring depth: loads run KVS-1 tiles ahead
+constexpr int SM_K = SM_Q + 2 * TILE;     // KVS stages
 constexpr int SM_V = SM_K + KVS * TILE;   // KVS stages
-constexpr int SM_P = SM_V + KVS * TILE;   // 2 buffers x (keys 0-63 | keys 64-127)
-constexpr int SM_XCHG = SM_P + 4 * TILE;  // [2][2][128] floats: row max / sum exchange
-constexpr int SM_TILES = SM_XCHG + 2 * 2 * 128 * 4;
-// q_full, kv_full[KVS], kv_empty[KVS], s_full[2], s_free[2], p_full[2], o_full[2], drain
-constexpr int NUM_BARS = 2 * KVS + 10;
+constexpr int SM_P = SM_V + KVS * TILE;
+constexpr int SM_XCHG = SM_P + 4 * TILE;  // [2][2][128] row maxima + [2][128] row sums (floats)
+constexpr int SM_TILES = SM_XCHG + 3 * 2 * 128 * 4;
+// q_full[2], q_empty[2], kv_full[KVS], kv_empty[KVS], s_full[2], s_free[2], p_full[2], o_full[2], drain,
+// xch[2] (row-max exchange), row_sync (per-item exchanges of the softmax warps)
+constexpr int NUM_BARS = 2 * KVS + 16;
 constexpr int SMEM_BYTES = SM_TILES + 1024 + NUM_BARS * 8 + 16;
+static_assert(SMEM_BYTES <= 232448, "forward shared memory");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t S_COL = 0, O_COL = 256;
 constexpr int NUM_THREADS = 320;  // TMA warp, MMA warp, 8 softmax warps
@@ -93,9 +98,14 @@ DEVI float ex2(float x) {
   return y;
 }
 
+// Persistent: each CTA takes work items (query block, batch, head) w =
+// blockIdx.x, blockIdx.x + gridDim.x, ...; items are numbered longest causal
+// row first.  Key/value blocks are counted globally across a CTA's items (g),
+// so the K/V ring, the S / P / O double buffers and their barrier phases run
+// on without a break between items.
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmO,
-                       float* __restrict__ lse, int T, int H, float scale_log2, int* err) {
+                       float* __restrict__ lse, int T, int H, int n_items, float scale_log2, int* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -103,36 +113,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t bars = base + SM_TILES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + SM_TILES + NUM_BARS * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const uint32_t q_full = bars;
-  auto kv_full = [&](int s) { return bars + 8u * (1 + s); };
-  auto kv_empty = [&](int s) { return bars + 8u * (1 + KVS + s); };
-  auto s_full = [&](int s) { return bars + 8u * (1 + 2 * KVS + s); };
-  auto s_free = [&](int s) { return bars + 8u * (3 + 2 * KVS + s); };
-  auto p_full = [&](int s) { return bars + 8u * (5 + 2 * KVS + s); };
-  auto o_full = [&](int s) { return bars + 8u * (7 + 2 * KVS + s); };
-  const uint32_t drain_bar = bars + 8u * (9 + 2 * KVS);
+  auto q_full = [&](int s) { return bars + 8u * s; };
+  auto q_empty = [&](int s) { return bars + 8u * (2 + s); };
+  auto kv_full = [&](int s) { return bars + 8u * (4 + s); };
+  auto kv_empty = [&](int s) { return bars + 8u * (4 + KVS + s); };
+  auto s_full = [&](int s) { return bars + 8u * (4 + 2 * KVS + s); };
+  auto s_free = [&](int s) { return bars + 8u * (6 + 2 * KVS + s); };
+  auto p_full = [&](int s) { return bars + 8u * (8 + 2 * KVS + s); };
+  auto o_full = [&](int s) { return bars + 8u * (10 + 2 * KVS + s); };
+  const uint32_t drain_bar = bars + 8u * (12 + 2 * KVS);
+  auto xch_bar = [&](int s) { return bars + 8u * (13 + 2 * KVS + s); };
+  const uint32_t row_sync = bars + 8u * (15 + 2 * KVS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (T + BQ - 1) / BQ;
-  const int qb = nqb - 1 - (int)blockIdx.x;  // longest causal blocks first
-  const int b = blockIdx.y / H, h = blockIdx.y % H;
+  const int BH = n_items / nqb;
   const int d = H * HD;
-  const int q0 = qb * BQ;
-  const int nkv = qb + 1;  // key tiles 0..qb (BKV == BQ)
+  // work item -> (query block, batch, head); the key blocks are 0..qb
+  auto item = [&](int w, int& qb, int& b, int& h) {
+    qb = nqb - 1 - w / BH;
+    const int bh = w % BH;
+    b = bh / H;
+    h = bh % H;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < KVS; ++s) {
-      mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
-    }
     for (int s = 0; s < 2; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), 1);
       mbar_init(s_full(s), 1);
       mbar_init(s_free(s), 256);
       mbar_init(p_full(s), 256);
       mbar_init(o_full(s), 1);
     }
+    for (int s = 0; s < KVS; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
     mbar_init(drain_bar, 1);
+    mbar_init(xch_bar(0), 256);
+    mbar_init(xch_bar(1), 256);
+    mbar_init(row_sync, 256);
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmQKV);
@@ -147,62 +168,87 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ----------------------------------------------------------- TMA ----
-      int issued = 0;
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, TILE);
-      tma_load_3d(base + SM_Q, &tmQKV, q_full, h * HD, q0, b);
-      for (int j = 0; j < nkv; ++j) {
-        const int st = j % KVS;
-        if (j >= KVS && !mbar_wait_bounded(kv_empty(st), ((j - KVS) / KVS) & 1, abort_flag, err)) {
+      int g = 0, it = 0;
+      int q_issued = 0, kv_issued = 0;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+        int qb, b, h;
+        item(w, qb, b, h);
+        const int qs = it & 1;
+        // the Q buffer was last used by item it-2, whose O store has read it
+        if (it >= 2 && !mbar_wait_bounded(q_empty(qs), ((it - 2) >> 1) & 1, abort_flag, err)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(kv_full(st), 2 * TILE);
-        tma_load_3d(base + SM_K + st * TILE, &tmQKV, kv_full(st), d + h * HD, j * BKV, b);
-        tma_load_3d(base + SM_V + st * TILE, &tmQKV, kv_full(st), 2 * d + h * HD, j * BKV, b);
-        ++issued;
+        mbar_arrive_expect_tx(q_full(qs), TILE);
+        tma_load_3d(base + SM_Q + qs * TILE, &tmQKV, q_full(qs), h * HD, qb * BQ, b);
+        ++q_issued;
+        for (int j = 0; j <= qb; ++j, ++g) {
+          const int st = g % KVS;
+          if (g >= KVS && !mbar_wait_bounded(kv_empty(st), ((g - KVS) / KVS) & 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(kv_full(st), 2 * TILE);
+          tma_load_3d(base + SM_K + st * TILE, &tmQKV, kv_full(st), d + h * HD, j * BKV, b);
+          tma_load_3d(base + SM_V + st * TILE, &tmQKV, kv_full(st), 2 * d + h * HD, j * BKV, b);
+          ++kv_issued;
+        }
       }
       if (!ok) {
-        mbar_drain_bounded(q_full, 0);
-        for (int j = issued - KVS < 0 ? 0 : issued - KVS; j < issued; ++j)
-          mbar_drain_bounded(kv_full(j % KVS), (j / KVS) & 1);
+        // let the copies in flight land before the CTA exits
+        for (int i = q_issued - 2 < 0 ? 0 : q_issued - 2; i < q_issued; ++i)
+          mbar_drain_bounded(q_full(i & 1), (i >> 1) & 1);
+        for (int i = kv_issued - KVS < 0 ? 0 : kv_issued - KVS; i < kv_issued; ++i)
+          mbar_drain_bounded(kv_full(i % KVS), (i / KVS) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ----------------------------------------------------------- MMA ----
-      bool ok = mbar_wait_bounded(q_full, 0, abort_flag, err);
+      bool ok = true;
       bool issued_any = false;
-      auto issue_pv = [&](int t) -> bool {
-        const int pb = t & 1;
-        if (!mbar_wait_bounded(p_full(pb), (t >> 1) & 1, abort_flag, err)) return false;
+      // O_tile(g) = P(g) V(g) into the O buffer of block g
+      auto issue_pv = [&](int gg) -> bool {
+        const int pb = gg & 1;
+        if (!mbar_wait_bounded(p_full(pb), (gg >> 1) & 1, abort_flag, err)) return false;
         tc_fence_after();
         const uint32_t pbase = base + SM_P + pb * 2 * TILE;
-        const uint32_t vbase = base + SM_V + (t % KVS) * TILE;
+        const uint32_t vbase = base + SM_V + (gg % KVS) * TILE;
 #pragma unroll
         for (int k = 0; k < BKV / 16; ++k)
           tc_mma_bf16(tmem + O_COL + pb * HD, sdesc(pbase + (k >> 2) * TILE + (k & 3) * 32, 16, 1024),
                       sdesc(vbase + k * 2048, 8192, 1024), IDESC_O, k > 0 ? 1u : 0u);
         tc_commit(o_full(pb));
-        tc_commit(kv_empty(t % KVS));
+        tc_commit(kv_empty(gg % KVS));
         return true;
       };
-      if (ok) tc_fence_after();
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int st = j % KVS, sb = j & 1;
-        if (!mbar_wait_bounded(kv_full(st), (j / KVS) & 1, abort_flag, err)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait_bounded(s_free(sb), ((j - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      int g = 0, it = 0;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+        int qb, b, h;
+        item(w, qb, b, h);
+        const int qs = it & 1;
+        if (!mbar_wait_bounded(q_full(qs), (it >> 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t kbase = base + SM_K + st * TILE;
+        const uint32_t qbase = base + SM_Q + qs * TILE;
+        for (int j = 0; j <= qb; ++j, ++g) {
+          const int st = g % KVS, sb = g & 1;
+          if (!mbar_wait_bounded(kv_full(st), (g / KVS) & 1, abort_flag, err)) { ok = false; break; }
+          if (g >= 2 && !mbar_wait_bounded(s_free(sb), ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kbase = base + SM_K + st * TILE;
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k)
-          tc_mma_bf16(tmem + S_COL + sb * BKV, sdesc(base + SM_Q + k * 32, 16, 1024), sdesc(kbase + k * 32, 16, 1024),
-                      IDESC_S, k > 0 ? 1u : 0u);
-        issued_any = true;
-        tc_commit(s_full(sb));
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+          for (int k = 0; k < HD / 16; ++k)
+            tc_mma_bf16(tmem + S_COL + sb * BKV, sdesc(qbase + k * 32, 16, 1024), sdesc(kbase + k * 32, 16, 1024),
+                        IDESC_S, k > 0 ? 1u : 0u);
+          issued_any = true;
+          tc_commit(s_full(sb));
+          // the previous block's PV (possibly of the previous item) follows
+          // this block's S, so softmax of block g overlaps P(g-1) V(g-1)
+          if (g >= 1 && !issue_pv(g - 1)) { ok = false; break; }
+        }
       }
-      if (ok) ok = issue_pv(nkv - 1);
+      if (ok && g >= 1) ok = issue_pv(g - 1);
       if (!ok && issued_any) {
         tc_commit(drain_bar);
         mbar_drain_bounded(drain_bar, 0);
@@ -212,114 +258,132 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------- softmax ----
     // Eight warps: two per TMEM lane quarter, each owning 64 of the 128 key
     // columns of its rows and 32 of the 64 output columns; the two halves of
-    // a row exchange partial maxima (per tile) and sums (at the end) through
-    // shared memory.
+    // a row exchange partial maxima (per block) and sums (per item) through
+    // shared memory.  The exchanges synchronise the 256 threads on mbarriers
+    // (bounded waits), so an abort in one warp cannot strand the others.
     const int e = warp - 2;
     const int q = warp & 3;  // TMEM lanes [32q, 32q+32)
     const int half = e >> 2;
     const int row = q * 32 + lane;
-    const int grow = q0 + row;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    float* xchg = reinterpret_cast<float*>(base_ptr + SM_XCHG);  // [parity][half][128 rows]
-    float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
-    float acc[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+    float* xchg = reinterpret_cast<float*>(base_ptr + SM_XCHG);  // [parity][half][128 rows] maxima
+    float* xsum = xchg + 2 * 256;                                 // [half][128 rows] sums
     bool ok = true;
-    auto fold = [&](int t, float a) -> bool {
-      const int ob = t & 1;
-      if (!mbar_wait_bounded(o_full(ob), (t >> 1) & 1, abort_flag, err)) return false;
-      tc_fence_after();
-      uint32_t r0[32];
-      tmem_ld_32x32b_x32(tmem + lane_off + O_COL + ob * HD + 32 * half, r0);
-      tmem_ld_wait();
+    int g = 0, it = 0;
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+      int qb, b, h;
+      item(w, qb, b, h);
+      const int q0 = qb * BQ, grow = q0 + row;
+      float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
+      float acc[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = acc[i] * a + __uint_as_float(r0[i]);
-      tc_fence_before();
-      return true;
-    };
-    for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1;
-      if (!mbar_wait_bounded(s_full(sb), (j >> 1) & 1, abort_flag, err)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t r[2][32];
+      for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+      auto fold = [&](int gg, float a) -> bool {
+        const int ob = gg & 1;
+        if (!mbar_wait_bounded(o_full(ob), (gg >> 1) & 1, abort_flag, err)) return false;
+        tc_fence_after();
+        uint32_t r0[32];
+        tmem_ld_32x32b_x32(tmem + lane_off + O_COL + ob * HD + 32 * half, r0);
+        tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
-        tmem_ld_32x32b_x32(tmem + lane_off + S_COL + sb * BKV + 64 * half + 32 * c, r[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(s_free(sb));
-      const bool diag = (j == nkv - 1);
-      const int kc0 = j * BKV + 64 * half;
-      float pmax = m;
+        for (int i = 0; i < 32; ++i) acc[i] = acc[i] * a + __uint_as_float(r0[i]);
+        tc_fence_before();
+        return true;
+      };
+      for (int j = 0; j <= qb; ++j, ++g) {
+        const int sb = g & 1;
+        if (!mbar_wait_bounded(s_full(sb), (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r[2][32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < 2; ++c)
+          tmem_ld_32x32b_x32(tmem + lane_off + S_COL + sb * BKV + 64 * half + 32 * c, r[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(s_free(sb));
+        const bool diag = (j == qb);
+        const int kc0 = j * BKV + 64 * half;
+        float pmax = m;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float v = __uint_as_float(r[c][i]) * scale_log2;
-          if (diag && kc0 + 32 * c + i > grow) v = -INFINITY;
-          r[c][i] = __float_as_uint(v);
-          pmax = fmaxf(pmax, v);
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float v = __uint_as_float(r[c][i]) * scale_log2;
+            if (diag && kc0 + 32 * c + i > grow) v = -INFINITY;
+            r[c][i] = __float_as_uint(v);
+            pmax = fmaxf(pmax, v);
+          }
+        float* xp = xchg + sb * 256;
+        xp[half * 128 + row] = pmax;
+        mbar_arrive(xch_bar(sb));
+        if (!mbar_wait_bounded(xch_bar(sb), (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        const float mx = fmaxf(pmax, xp[(1 - half) * 128 + row]);
+        const float alpha = ex2(m - mx);
+        m = mx;
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p = ex2(__uint_as_float(r[c][i]) - m);
+            r[c][i] = __float_as_uint(p);
+            sum += p;
+          }
+        l = l * alpha + sum;
+        // this half's 64 keys of the P row -> its 128B-swizzled K-major block
+        const uint32_t pb = base + SM_P + sb * 2 * TILE + half * TILE + (uint32_t)row * 128u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int gq = c >> 2, o8 = (c & 3) * 8;
+          st_shared_v4(pb + 16u * (uint32_t)(c ^ (row & 7)),
+                       pack_bf16x2(__uint_as_float(r[gq][o8 + 0]), __uint_as_float(r[gq][o8 + 1])),
+                       pack_bf16x2(__uint_as_float(r[gq][o8 + 2]), __uint_as_float(r[gq][o8 + 3])),
+                       pack_bf16x2(__uint_as_float(r[gq][o8 + 4]), __uint_as_float(r[gq][o8 + 5])),
+                       pack_bf16x2(__uint_as_float(r[gq][o8 + 6]), __uint_as_float(r[gq][o8 + 7])));
         }
-      float* xp = xchg + (j & 1) * 256;
-      xp[half * 128 + row] = pmax;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      const float mx = fmaxf(pmax, xp[(1 - half) * 128 + row]);
-      const float alpha = ex2(m - mx);
-      m = mx;
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p = ex2(__uint_as_float(r[c][i]) - m);
-          r[c][i] = __float_as_uint(p);
-          sum += p;
-        }
-      l = l * alpha + sum;
-      // this half's 64 keys of the P row -> its 128B-swizzled K-major block
-      const uint32_t pb = base + SM_P + sb * 2 * TILE + half * TILE + (uint32_t)row * 128u;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int g = c >> 2, o8 = (c & 3) * 8;
-        st_shared_v4(pb + 16u * (uint32_t)(c ^ (row & 7)),
-                     pack_bf16x2(__uint_as_float(r[g][o8 + 0]), __uint_as_float(r[g][o8 + 1])),
-                     pack_bf16x2(__uint_as_float(r[g][o8 + 2]), __uint_as_float(r[g][o8 + 3])),
-                     pack_bf16x2(__uint_as_float(r[g][o8 + 4]), __uint_as_float(r[g][o8 + 5])),
-                     pack_bf16x2(__uint_as_float(r[g][o8 + 6]), __uint_as_float(r[g][o8 + 7])));
+        fence_proxy_async_smem();
+        mbar_arrive(p_full(sb));
+        if (j >= 1 && !fold(g - 1, alpha_prev)) { ok = false; break; }
+        alpha_prev = alpha;
       }
-      fence_proxy_async_smem();
-      mbar_arrive(p_full(sb));
-      if (j >= 1 && !fold(j - 1, alpha_prev)) { ok = false; break; }
-      alpha_prev = alpha;
-    }
-    if (ok) ok = fold(nkv - 1, alpha_prev);
-    // row sum = both halves' partial sums (both were kept relative to the same m)
-    float* xs = xchg + (nkv & 1) * 256;
-    xs[half * 128 + row] = l;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    l += xs[(1 - half) * 128 + row];
-    if (ok) {
-      // O / l -> shared memory (the Q tile is no longer read) -> one TMA store
-      const float inv = 1.f / l;
-      const uint32_t ob = base + SM_Q + (uint32_t)row * 128u;
+      if (ok) ok = fold(g - 1, alpha_prev);
+      // row sum = both halves' partial sums (both kept relative to the same m)
+      xsum[half * 128 + row] = l;
+      mbar_arrive(row_sync);
+      if (!mbar_wait_bounded(row_sync, 0, abort_flag, err)) ok = false;
+      l += xsum[(1 - half) * 128 + row];
+      const int qs = it & 1;
+      if (ok) {
+        // O / l -> this item's Q buffer (its S MMAs are complete: the last
+        // PV, committed after them, has been waited on) -> one TMA store
+        const float inv = 1.f / l;
+        const uint32_t ob = base + SM_Q + qs * TILE + (uint32_t)row * 128u;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        st_shared_v4(ob + 16u * (uint32_t)((4 * half + c) ^ (row & 7)),
-                     pack_bf16x2(acc[8 * c] * inv, acc[8 * c + 1] * inv),
-                     pack_bf16x2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv),
-                     pack_bf16x2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv),
-                     pack_bf16x2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv));
-      if (half == 0 && grow < T) lse[((long)b * H + h) * T + grow] = (m + __log2f(l)) * LN2_F;
-      fence_proxy_async_smem();
+        for (int c = 0; c < 4; ++c)
+          st_shared_v4(ob + 16u * (uint32_t)((4 * half + c) ^ (row & 7)),
+                       pack_bf16x2(acc[8 * c] * inv, acc[8 * c + 1] * inv),
+                       pack_bf16x2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv),
+                       pack_bf16x2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv),
+                       pack_bf16x2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv));
+        if (half == 0 && grow < T) lse[((long)b * H + h) * T + grow] = (m + __log2f(l)) * LN2_F;
+        fence_proxy_async_smem();
+      }
+      // all eight softmax warps have staged O (an abort makes every wait
+      // return); it also keeps the row-sum exchange of the next item from
+      // overwriting a slot before its partner has read it
+      mbar_arrive(row_sync);
+      if (!mbar_wait_bounded(row_sync, 1, abort_flag, err)) ok = false;
+      if (warp == 2 && lane == 0) {
+        if (ok && !*abort_flag) {
+          tma_store_3d(&tmO, base + SM_Q + qs * TILE, h * HD, q0, b);
+          bulk_commit();
+          bulk_wait_read<0>();
+        }
+        mbar_arrive(q_empty(qs));
+      }
+      __syncwarp();
     }
-    // all eight softmax warps arrive here (an abort makes every wait return)
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (warp == 2 && lane == 0 && !*abort_flag) {
-      tma_store_3d(&tmO, base + SM_Q, h * HD, q0, b);
-      bulk_commit();
-      bulk_wait_all();
-    }
+    if (warp == 2 && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -668,8 +732,9 @@ int attn_fwd_tc(const void* qkv, void* o, float* lse, int B, int T, int H, cudaS
     CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
     attr = true;
   }
-  dim3 grid((T + BQ - 1) / BQ, B * H);
-  attn_fwd_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tq, to, lse, T, H, LOG2E_F / 8.f, nullptr);
+  const int n_items = ((T + BQ - 1) / BQ) * B * H;
+  const int grid = n_items < num_sms() ? n_items : num_sms();
+  attn_fwd_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tq, to, lse, T, H, n_items, LOG2E_F / 8.f, nullptr);
   LAUNCH_CHECK();
   return GPT2_OK;
 }

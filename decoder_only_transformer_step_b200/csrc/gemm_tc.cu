@@ -5,19 +5,27 @@
 // are C = A B^T with A and B either K-major or MN-major, which is what this
 // kernel takes, so no operand is ever transposed in memory.
 //
-// Design (one CTA per SM, persistent over output tiles):
+// Design (persistent over output tiles, one CTA per SM):
 //   warp 0      TMA producer: 128B-swizzled tiles of A (128 x 64) and B
-//               (BN x 64) into a STAGES-deep shared-memory ring (mbarriers).
-//   warp 1      allocates TMEM and issues tcgen05.mma (M=128, N=BN, K=16)
-//               from one thread; tcgen05.commit frees each ring slot and
-//               signals a finished accumulator.
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (each warp owns
-//               the 32 TMEM lanes = tile rows its warp index allows), fused
-//               bias / residual / GELU / GELU' / fp32-gradient stores.
+//               into a STAGES-deep shared-memory ring (mbarriers).
+//   warp 1      allocates TMEM and issues tcgen05.mma (K=16 steps) from one
+//               thread; tcgen05.commit frees each ring slot and signals a
+//               finished accumulator.
+//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator (each warp owns
+//               the 32 TMEM lanes = tile rows its warp index allows, and half
+//               of the columns), fused bias / residual / GELU / GELU' /
+//               fp32-gradient stores.
 // The accumulator is double-buffered in TMEM (2 x BN columns), so the
-// epilogue of tile i overlaps the main loop of tile i+1.  Weight gradients
-// with few output tiles are split along K; partial sums go to a workspace and
-// a deterministic reduction adds them in split order.
+// epilogue of tile i overlaps the main loop of tile i+1.
+//
+// Two tile shapes: a single CTA computing 128 x BN (BN 128 or 256), and a CTA
+// pair (cluster of two SMs) computing 256 x 256 with tcgen05.mma.cta_group::2:
+// each CTA loads its 128 rows of A and 128 of the 256 rows of B, so per
+// multiply-add each SM moves two thirds of the operand bytes the single-CTA
+// 128 x 256 tile needs.  The even CTA issues the MMAs; both run the epilogue
+// on their own 128 accumulator rows.  Weight gradients with few output tiles
+// are split along K; partial sums go to a workspace and a deterministic
+// reduction adds them in split order.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <string.h>
@@ -34,17 +42,22 @@ constexpr int NUM_EPI_WARPS = 8;  // two per TMEM lane quarter, each owning half
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t MN_ATOM_BYTES = 64 * BK * 2;  // one {64 MN x 64 K} TMA box
 
-template <int BN>
+template <int BN, bool PAIR>
 struct TcCfg {
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int TILE_M = PAIR ? 2 * BM : BM;   // output rows per work unit
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;   // rows of B this CTA loads per stage
+  static constexpr int STAGES = PAIR ? 6 : (BN == 256 ? 4 : 6);
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int NUM_BARS = 2 * STAGES + 5;  // full, empty, acc_full[2], acc_empty[2], drain
+  // accumulator-empty arrivals: one per epilogue warp of every CTA of the unit
+  static constexpr uint32_t ACCE_COUNT = (PAIR ? 2 : 1) * NUM_EPI_WARPS;
   // one 4 KB staging box per epilogue warp (TMA store source)
   static constexpr int EPI_BYTES = NUM_EPI_WARPS * 4096;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + NUM_BARS * 8 + 16;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
 // How the epilogue writes its result.
@@ -61,6 +74,7 @@ struct TcParams {
   int M, N, K;
   int a_mn, b_mn;
   int m_tiles, n_tiles, splits, kb_total;
+  int tile_m;  // output rows per work unit (128, or 256 for a CTA pair)
   uint32_t idesc;
   int store;
   EpiArgs epi;
@@ -94,17 +108,17 @@ DEVI void decode_unit(const TcParams& p, int u, int& m0, int& nt, int& s, int& k
   const int rest = u / p.m_tiles;
   nt = rest % p.n_tiles;
   s = rest / p.n_tiles;
-  m0 = mt * BM;
+  m0 = mt * p.tile_m;
   kb0 = (int)((long long)s * p.kb_total / p.splits);
   kb1 = (int)((long long)(s + 1) * p.kb_total / p.splits);
 }
 
-template <int BN>
+template <int BN, bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
                    const TcParams p) {
-  using C = TcCfg<BN>;
+  using C = TcCfg<BN, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t tiles = (raw + 1023u) & ~1023u;
@@ -123,6 +137,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // CTA pairs: consecutive blocks form a cluster; rank 0 issues the MMAs
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int unit0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int unit_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -131,7 +149,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(accf_bar(b), 1);
-      mbar_init(acce_bar(b), 32 * NUM_EPI_WARPS);
+      mbar_init(acce_bar(b), C::ACCE_COUNT);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -139,9 +157,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  if (warp == 1) {
+    if constexpr (PAIR)
+      tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
+    else
+      tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  }
   tc_fence_before();
   __syncthreads();
+  // the peer's barriers must be initialised before anything signals them
+  if constexpr (PAIR) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -154,30 +179,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int u = unit0; u < units && ok; u += unit_step) {
         int m0, nt, s, kb0, kb1;
         decode_unit(p, u, m0, nt, s, kb0, kb1);
-        const int n0 = nt * BN;
+        const int ma = m0 + (int)rank * BM;             // this CTA's rows of A
+        const int nb = nt * BN + (int)rank * C::B_ROWS;  // this CTA's rows of B
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.err)) {
             ok = false;
             break;
           }
-          const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
           const uint32_t sa = tiles + stage * C::STAGE_BYTES;
           const uint32_t sb = sa + C::A_BYTES;
-          if (!p.a_mn) {
-            tma_load_2d(sa, &tmA, fb, kb * BK, m0);
-          } else {
-            tma_load_2d(sa, &tmA, fb, m0, kb * BK);
-            tma_load_2d(sa + MN_ATOM_BYTES, &tmA, fb, m0 + 64, kb * BK);
-          }
-          if (!p.b_mn) {
-            tma_load_2d(sb, &tmB, fb, kb * BK, n0);
-          } else {
+          if constexpr (PAIR) {
+            // both CTAs' bytes are counted on the even CTA's full barrier
+            const uint32_t fb = mapa_shared(full_bar(stage), 0);
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
+            if (!p.a_mn) {
+              tma_load_2d_pair(sa, &tmA, fb, kb * BK, ma);
+            } else {
+              tma_load_2d_pair(sa, &tmA, fb, ma, kb * BK);
+              tma_load_2d_pair(sa + MN_ATOM_BYTES, &tmA, fb, ma + 64, kb * BK);
+            }
+            if (!p.b_mn) {
+              tma_load_2d_pair(sb, &tmB, fb, kb * BK, nb);
+            } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * MN_ATOM_BYTES, &tmB, fb, n0 + 64 * j, kb * BK);
+              for (int j = 0; j < C::B_ROWS / 64; ++j)
+                tma_load_2d_pair(sb + j * MN_ATOM_BYTES, &tmB, fb, nb + 64 * j, kb * BK);
+            }
+          } else {
+            const uint32_t fb = full_bar(stage);
+            mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+            if (!p.a_mn) {
+              tma_load_2d(sa, &tmA, fb, kb * BK, ma);
+            } else {
+              tma_load_2d(sa, &tmA, fb, ma, kb * BK);
+              tma_load_2d(sa + MN_ATOM_BYTES, &tmA, fb, ma + 64, kb * BK);
+            }
+            if (!p.b_mn) {
+              tma_load_2d(sb, &tmB, fb, kb * BK, nb);
+            } else {
+#pragma unroll
+              for (int j = 0; j < C::B_ROWS / 64; ++j)
+                tma_load_2d(sb + j * MN_ATOM_BYTES, &tmB, fb, nb + 64 * j, kb * BK);
+            }
           }
           ++issued;
           if (++stage == C::STAGES) {
@@ -186,8 +232,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (!ok) {
-        // Let the copies already in flight land before the CTA exits.
+      if (!ok && rank == 0) {
+        // Let the copies already in flight land before the CTA exits (for a
+        // pair, the even CTA's full barriers count both CTAs' copies).
         int n = issued < C::STAGES ? issued : C::STAGES;
         for (int i = 1; i <= n; ++i) {
           int s2 = (stage - i + C::STAGES) % C::STAGES;
@@ -197,19 +244,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ---------------------------------------------- MMA issuer ----
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
       bool issued_any = false;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++it) {
+      for (int u = unit0; u < units && ok; u += unit_step, ++it) {
         int m0, nt, s, kb0, kb1;
         decode_unit(p, u, m0, nt, s, kb0, kb1);
         const int buf = it & 1;
         const uint32_t aph = (uint32_t)(it >> 1) & 1u;
-        if (!mbar_wait_bounded(acce_bar(buf), aph ^ 1u, abort_flag, p.err)) {
+        const bool acc_free = PAIR ? mbar_wait_bounded_cluster(acce_bar(buf), aph ^ 1u, abort_flag, p.err)
+                                   : mbar_wait_bounded(acce_bar(buf), aph ^ 1u, abort_flag, p.err);
+        if (!acc_free) {
           ok = false;
           break;
         }
@@ -225,22 +274,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            tc_mma_bf16(d_tmem, operand_desc(sa, p.a_mn, k), operand_desc(sb, p.b_mn, k), p.idesc,
-                        (kb > kb0 || k > 0) ? 1u : 0u);
+            const uint64_t ad = operand_desc(sa, p.a_mn, k), bd = operand_desc(sb, p.b_mn, k);
+            const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
+            if constexpr (PAIR)
+              tc_mma_bf16_pair(d_tmem, ad, bd, p.idesc, acc);
+            else
+              tc_mma_bf16(d_tmem, ad, bd, p.idesc, acc);
           }
           issued_any = true;
-          tc_commit(empty_bar(stage));
+          if constexpr (PAIR)
+            tc_commit_pair_mask(empty_bar(stage), 3);  // both CTAs' ring slots
+          else
+            tc_commit(empty_bar(stage));
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(accf_bar(buf));
+        if constexpr (PAIR)
+          tc_commit_pair_mask(accf_bar(buf), 3);
+        else
+          tc_commit(accf_bar(buf));
       }
       if (!ok && issued_any) {
         // Wait (bounded) for the MMAs already issued before TMEM is freed.
-        tc_commit(drain_bar);
+        if constexpr (PAIR)
+          tc_commit_pair(drain_bar);
+        else
+          tc_commit(drain_bar);
         mbar_drain_bounded(drain_bar, 0);
       }
     }
@@ -253,13 +315,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const bool has_operand = p.epi.kind == EPI_BIAS_RESID || p.epi.kind == EPI_DGELU;
     const bf16* operand = (const bf16*)(p.epi.kind == EPI_DGELU ? p.epi.aux : p.epi.resid);
     int it = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+    for (int u = unit0; u < units; u += unit_step, ++it) {
       int m0, nt, s, kb0, kb1;
       decode_unit(p, u, m0, nt, s, kb0, kb1);
       const int n0 = nt * BN;
       const int buf = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
-      const int row0 = m0 + q * 32;
+      const int row0 = m0 + (int)rank * BM + q * 32;
       const int row = row0 + lane;
       // the first chunk's residual / GELU' operand does not depend on the
       // accumulator: fetch it while the MMAs run
@@ -334,8 +396,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           bulk_commit();
         }
       }
+      // every lane's TMEM loads have completed (tcgen05.wait::ld above)
       tc_fence_before();
-      mbar_arrive(acce_bar(buf));
+      __syncwarp();
+      if (lane == 0) {
+        // accumulator-empty barrier of the CTA that issues the MMAs
+        if constexpr (PAIR)
+          mbar_arrive_cluster(mapa_shared(acce_bar(buf), 0));
+        else
+          mbar_arrive(acce_bar(buf));
+      }
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
@@ -343,9 +413,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  // neither CTA of a pair leaves while the other may still signal its barriers
+  if constexpr (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -425,27 +500,63 @@ bool make_out_tmap(CUtensorMap* tm, const void* base, int M, int N, long ldo, bo
                      dims, strides, box, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-template <int BN>
+template <int BN, bool PAIR>
 int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tc2,
-              const TcParams& p, int grid, cudaStream_t st) {
-  using C = TcCfg<BN>;
+              const TcParams& p, int units, cudaStream_t st) {
+  using C = TcCfg<BN, PAIR>;
   static bool attr_set = false;
+  static int max_slots = 0;  // co-resident CTAs (single) or clusters (pairs)
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
   if (!attr_set) {
-    CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   C::SMEM_BYTES));
+    if (PAIR) {
+      cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<BN, PAIR>, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = num_sms() / 2;
+      }
+      max_slots = n;
+    } else {
+      max_slots = num_sms();
+    }
     attr_set = true;
   }
-  gemm_tc_kernel<BN><<<grid, NUM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, tc, tc2, p);
+  const int slots = units < max_slots ? units : max_slots;
+  cfg.gridDim = dim3((PAIR ? 2 : 1) * slots, 1, 1);
+  CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, PAIR>, ta, tb, tc, tc2, p));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
 
-int auto_splits(int M, int N, int K) {
-  const int tiles = ((M + BM - 1) / BM) * ((N + 255) / 256);
+// Tile choice: bn 0 = automatic (the CTA-pair 256 x 256 tile unless N <= 128),
+// 128 / 256 = single-CTA 128 x bn tiles, 512 = the CTA-pair tile.
+int resolve_bn(int bn, int N) {
+  if (bn == 0) return N <= 128 ? 128 : 512;
+  return bn;
+}
+
+int auto_splits(int M, int N, int K, int bn) {
+  const bool pair = bn == 512;
+  const int tile_m = pair ? 2 * BM : BM, tile_n = pair ? 256 : bn;
+  const int tiles = ((M + tile_m - 1) / tile_m) * ((N + tile_n - 1) / tile_n);
   const int kb = K / BK;
-  const int sms = num_sms();
-  if (tiles >= sms) return 1;
-  int s = (2 * sms + tiles - 1) / tiles;
+  const int slots = pair ? num_sms() / 2 : num_sms();
+  if (tiles >= slots) return 1;
+  int s = (2 * slots + tiles - 1) / tiles;
   if (s > kb / 4) s = kb / 4;
   return s < 1 ? 1 : s;
 }
@@ -463,7 +574,7 @@ int num_sms() {
 }
 
 size_t gemm_tc_split_bytes(int M, int N, int K) {
-  int s = auto_splits(M, N, K);
+  int s = auto_splits(M, N, K, resolve_bn(0, N));
   return s > 1 ? (size_t)s * M * N * sizeof(float) : 0;
 }
 
@@ -473,10 +584,12 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   if (g.K <= 0 || g.K % BK) return GPT2_ERR_UNSUPPORTED_SHAPE;
   if (g.lda % 8 || g.ldb % 8 || g.epi.ldo % 8) return GPT2_ERR_INVALID_ARG;
   if (((uintptr_t)g.A | (uintptr_t)g.B | (uintptr_t)g.epi.out) & 15) return GPT2_ERR_INVALID_ARG;
-  if (bn == 0) bn = g.N <= 128 ? 128 : 256;
-  if (bn != 128 && bn != 256) return GPT2_ERR_INVALID_ARG;
+  bn = resolve_bn(bn, g.N);
+  if (bn != 128 && bn != 256 && bn != 512) return GPT2_ERR_INVALID_ARG;
+  const bool pair = bn == 512;
+  const int n_mma = pair ? 256 : bn;  // N of one MMA instruction and of the tile
   const int kb_total = g.K / BK;
-  if (splits == 0) splits = g.epi.kind == EPI_F32 ? auto_splits(g.M, g.N, g.K) : 1;
+  if (splits == 0) splits = g.epi.kind == EPI_F32 ? auto_splits(g.M, g.N, g.K, bn) : 1;
   if (splits > kb_total) splits = kb_total;
   if (splits > 1) {
     if (g.epi.kind != EPI_F32 || g.N % 4 || g.epi.ldo != g.N) return GPT2_ERR_INVALID_ARG;
@@ -488,20 +601,22 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   bool ok_a = g.a_mn ? make_tmap(&ta, g.A, g.M, g.K, g.lda, 64, 64)
                      : make_tmap(&ta, g.A, g.K, g.M, g.lda, 64, BM);
   bool ok_b = g.b_mn ? make_tmap(&tb, g.B, g.N, g.K, g.ldb, 64, 64)
-                     : make_tmap(&tb, g.B, g.K, g.N, g.ldb, 64, bn);
+                     : make_tmap(&tb, g.B, g.K, g.N, g.ldb, 64, pair ? n_mma / 2 : n_mma);
   if (!ok_a || !ok_b) return GPT2_ERR_CUDA;
 
   TcParams p;
   p.M = g.M; p.N = g.N; p.K = g.K;
   p.a_mn = g.a_mn; p.b_mn = g.b_mn;
-  p.m_tiles = (g.M + BM - 1) / BM;
-  p.n_tiles = (g.N + bn - 1) / bn;
+  p.tile_m = pair ? 2 * BM : BM;
+  p.m_tiles = (g.M + p.tile_m - 1) / p.tile_m;
+  p.n_tiles = (g.N + n_mma - 1) / n_mma;
   p.splits = splits;
   p.kb_total = kb_total;
   // instruction descriptor, kind::f16: D fp32 (bit 4), A and B bf16 (bits 7, 10),
-  // operand majorness (bits 15, 16), N >> 3 at bit 17, M >> 4 at bit 24.
+  // operand majorness (bits 15, 16), N >> 3 at bit 17, M >> 4 at bit 24 (M = 256
+  // for a CTA pair: 128 rows in each CTA).
   p.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)g.a_mn << 15) | ((uint32_t)g.b_mn << 16) |
-            ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+            ((uint32_t)(n_mma >> 3) << 17) | ((uint32_t)(p.tile_m >> 4) << 24);
   p.epi = g.epi;
   p.partial = (float*)ws;
   p.err = err;
@@ -546,8 +661,9 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   if (p.store == ST_BF16_X2 && ((uintptr_t)g.epi.out2 & 15)) return GPT2_ERR_INVALID_ARG;
 
   const int units = p.m_tiles * p.n_tiles * splits;
-  const int grid = units < num_sms() ? units : num_sms();
-  int rc = bn == 256 ? launch_tc<256>(ta, tb, tc, tc2, p, grid, st) : launch_tc<128>(ta, tb, tc, tc2, p, grid, st);
+  int rc = pair        ? launch_tc<256, true>(ta, tb, tc, tc2, p, units, st)
+           : bn == 256 ? launch_tc<256, false>(ta, tb, tc, tc2, p, units, st)
+                       : launch_tc<128, false>(ta, tb, tc, tc2, p, units, st);
   if (rc) return rc;
   if (splits > 1) {
     long mn = (long)g.M * g.N;

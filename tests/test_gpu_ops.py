@@ -20,9 +20,10 @@ def bf16_rand(shape, seed, scale=1.0):
 
 @pytest.mark.parametrize("a_mn", [0, 1])
 @pytest.mark.parametrize("b_mn", [0, 1])
-@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("bn", [128, 256, 512])
 @pytest.mark.parametrize("c_fp32", [0, 1])
 def test_gemm_layouts(a_mn, b_mn, bn, c_fp32):
+    """bn 128 / 256: single-CTA 128 x bn tiles; 512: the CTA-pair 256 x 256 tile."""
     M, N, K = 300, 520, 192
     lda = 304 if a_mn else K
     A_log = bf16_rand((M, K), 1)                       # logical A(m, k)
@@ -51,8 +52,9 @@ def test_gemm_layouts(a_mn, b_mn, bn, c_fp32):
     assert err <= (1e-5 if c_fp32 else 8e-3) * scale, (err, scale)
 
 
+@pytest.mark.parametrize("bn", [128, 512])
 @pytest.mark.parametrize("splits", [2, 3, 5])
-def test_gemm_split_k_accumulate(splits):
+def test_gemm_split_k_accumulate(splits, bn):
     """Weight-gradient shape: MN-major operands, fp32 out, split along K with
     the deterministic partial-sum reduction, beta = 1 accumulation."""
     M, N, K = 200, 136, 640
@@ -65,15 +67,36 @@ def test_gemm_split_k_accumulate(splits):
     C = C0.clone().cuda()
     ws = torch.empty(splits * M * N * 4, dtype=torch.uint8, device="cuda")
     gp.gpt2_op_gemm_bf16(A_st.cuda(), 1, 200, B_st.cuda(), 1, N, C, 1, N, M, N, K, alpha=0.5, beta=1.0,
-                         workspace=ws, bn=128, splits=splits)
+                         workspace=ws, bn=bn, splits=splits)
     ref = C0.double() + 0.5 * (A_log.double() @ B_log.double().t())
     err = (C.double().cpu() - ref).abs().max().item()
     assert err <= 1e-5 * ref.abs().max().item()
     # deterministic: the same call twice gives bitwise-identical output
     C2 = C0.clone().cuda()
     gp.gpt2_op_gemm_bf16(A_st.cuda(), 1, 200, B_st.cuda(), 1, N, C2, 1, N, M, N, K, alpha=0.5, beta=1.0,
-                         workspace=ws, bn=128, splits=splits)
+                         workspace=ws, bn=bn, splits=splits)
     assert torch.equal(C, C2)
+
+
+@pytest.mark.parametrize("M,N", [(100, 136), (257, 600), (384, 256)])
+@pytest.mark.parametrize("a_mn", [0, 1])
+def test_gemm_pair_ragged(M, N, a_mn):
+    """CTA-pair tiles whose second CTA holds no valid row (M = 100), a single
+    valid row (M = 257), or whose B half lies past N (N = 136, 600)."""
+    K = 128
+    A_log = bf16_rand((M, K), 11)
+    B_log = bf16_rand((N, K), 12)
+    lda = (M + 7) // 8 * 8 + 8 if a_mn else K
+    if a_mn:
+        A_st = torch.zeros((K, lda), dtype=torch.bfloat16)
+        A_st[:, :M] = A_log.t()
+    else:
+        A_st = A_log.contiguous()
+    C = torch.full((M, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    gp.gpt2_op_gemm_bf16(A_st.cuda(), a_mn, lda, B_log.cuda(), 0, K, C, 0, N, M, N, K, bn=512, splits=1)
+    ref = A_log.double() @ B_log.double().t()
+    err = (C.double().cpu() - ref).abs().max().item()
+    assert err <= 8e-3 * ref.abs().max().item(), err
 
 
 def test_gemm_large_k_many_tiles():
@@ -105,6 +128,26 @@ def test_attention_forward(hd, T):
     B, H = 2, 3
     d = H * hd
     qkv = _attn_inputs(B, T, H, hd, 10 + T)
+    o = torch.empty((B * T, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    gp.gpt2_op_attention_fwd_bf16(qkv.cuda(), o, lse, B, T, H, hd)
+    q, k, v = _split(qkv, B, T, H, hd)
+    o_ref, p = G.attention_fwd(q, k, v, None)
+    s = np.einsum("bhid,bhjd->bhij", q, k) / math.sqrt(hd)
+    s = np.where(np.triu(np.ones((T, T), bool), 1), -np.inf, s)
+    lse_ref = np.log(np.exp(s - s.max(-1, keepdims=True)).sum(-1)) + s.max(-1)
+    o_gpu = o.double().cpu().numpy().reshape(B, T, H, hd).transpose(0, 2, 1, 3)
+    assert np.abs(o_gpu - o_ref).max() <= 0.02 * np.abs(o_ref).max()
+    assert np.abs(lse.double().cpu().numpy() - lse_ref).max() <= 2e-2
+
+
+@pytest.mark.parametrize("B,H,T", [(4, 12, 512), (8, 12, 300)])
+def test_attention_forward_many_items(B, H, T):
+    """More (query block, batch, head) work items than SMs: the persistent
+    forward carries its K/V ring and buffer phases across items."""
+    hd = 64
+    d = H * hd
+    qkv = _attn_inputs(B, T, H, hd, 40 + T)
     o = torch.empty((B * T, d), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
     gp.gpt2_op_attention_fwd_bf16(qkv.cuda(), o, lse, B, T, H, hd)
