@@ -64,15 +64,23 @@ DEVI float tanh_fast(float x) {
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Both written to keep the dependent chain short: t = u (K0 + K0 K1 u^2).
 template <bool FAST> DEVI float gelu_f(float u) {
-  float t = GELU_K0 * (u + GELU_K1 * u * u * u);
-  float th = FAST ? tanh_fast(t) : tanhf(t);
-  return 0.5f * u * (1.f + th);
+  const float u2 = u * u;
+  const float t = u * fmaf(u2, GELU_K0 * GELU_K1, GELU_K0);
+  const float th = FAST ? tanh_fast(t) : tanhf(t);
+  const float hu = 0.5f * u;
+  return fmaf(hu, th, hu);
 }
+// d/du of 0.5 u (1 + tanh t) = 0.5 (1 + tanh t) + 0.5 u (1 - tanh^2 t) dt/du,
+// dt/du = K0 (1 + 3 K1 u^2).
 template <bool FAST> DEVI float dgelu_f(float u) {
-  float t = GELU_K0 * (u + GELU_K1 * u * u * u);
-  float th = FAST ? tanh_fast(t) : tanhf(t);
-  return 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * GELU_K0 * (1.f + 3.f * GELU_K1 * u * u);
+  const float u2 = u * u;
+  const float t = u * fmaf(u2, GELU_K0 * GELU_K1, GELU_K0);
+  const float th = FAST ? tanh_fast(t) : tanhf(t);
+  const float dt = fmaf(u2, 3.f * GELU_K0 * GELU_K1, GELU_K0);
+  const float sech2 = fmaf(-th, th, 1.f);
+  return fmaf(0.5f * u * sech2, dt, fmaf(0.5f, th, 0.5f));
 }
 
 // ------------------------------------------------------------ shared mem --

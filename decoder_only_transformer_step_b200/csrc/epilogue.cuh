@@ -69,30 +69,6 @@ DEVI void st_bf16x32(bf16* p, const float (&f)[32]) {
   }
 }
 
-// 32 bf16 values of (row, col0 .. col0+31) of a [M, ld] tensor as four 16-byte
-// words; zeros outside [0, M) x [0, N).
-DEVI void prefetch_bf16x32(const bf16* base, long ld, int M, int N, int row, int col0, uint4 (&u)[4]) {
-  if (row < M && col0 + 32 <= N) {
-    const uint4* p = reinterpret_cast<const uint4*>(base + (long)row * ld + col0);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) u[i] = __ldg(p + i);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t w[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int c = col0 + 8 * i + 2 * k;
-        const bool ok = row < M;
-        const float lo = (ok && c < N) ? to_f(base[(long)row * ld + c]) : 0.f;
-        const float hi = (ok && c + 1 < N) ? to_f(base[(long)row * ld + c + 1]) : 0.f;
-        w[k] = pack_bf16x2(lo, hi);
-      }
-      u[i] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  }
-}
-
 DEVI void unpack8(const uint4& u, float* f) {
   f[0] = bf16lo(u.x); f[1] = bf16hi(u.x); f[2] = bf16lo(u.y); f[3] = bf16hi(u.y);
   f[4] = bf16lo(u.z); f[5] = bf16hi(u.z); f[6] = bf16lo(u.w); f[7] = bf16hi(u.w);
@@ -100,8 +76,8 @@ DEVI void unpack8(const uint4& u, float* f) {
 
 // Epilogue arithmetic for 32 accumulators of one row, without the store (the
 // tensor-core path stages the result in shared memory and stores it with TMA,
-// which clips rows >= M and columns >= N).  `op` holds the prefetched residual
-// (EPI_BIAS_RESID) or GELU' input (EPI_DGELU) chunk.  For EPI_BIAS_GELU v
+// which clips rows >= M and columns >= N).  `op` holds the residual
+// (EPI_BIAS_RESID) or GELU' input (EPI_DGELU) chunk, read from its TMA box.  For EPI_BIAS_GELU v
 // becomes u = acc + bias; the caller derives GELU(u) after storing u.
 DEVI void epi_apply_row32(const EpiArgs& e, int N, int col0, float (&v)[32], const uint4 (&op)[4]) {
   const bool need_bias = e.kind == EPI_BIAS || e.kind == EPI_BIAS_RESID || e.kind == EPI_BIAS_GELU;
@@ -156,24 +132,17 @@ DEVI void stage_bf16_row(uint32_t box, int lane, const float (&v)[32]) {
                  pack_bf16x2(v[8 * j + 2], v[8 * j + 3]), pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
                  pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
 }
-// Write a staged bf16 box to global memory with coalesced 16-byte stores: per
-// instruction the warp covers 8 rows x 64 contiguous bytes (the read-back of
-// the swizzled box is one contiguous, conflict-free 512-byte span).  Rows >= M
-// and 8-column groups >= N are skipped.
-DEVI void unstage_bf16_box(uint32_t box, int lane, bf16* out, long ldo, int M, int N, int row0, int col0) {
-  const int j = lane & 3;
+// Row `lane` of a bf16 32 x 32 box in the 64-byte swizzle (as TMA loads it),
+// as four 16-byte words in column order.
+DEVI void load_bf16_box_row(uint32_t box, int lane, uint4 (&u)[4]) {
+  const uint32_t rb = box + (uint32_t)lane * 64u;
+  const int x = (lane >> 1) & 3;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = 8 * i + (lane >> 2);
-    uint32_t a, b, c, d;
+  for (int j = 0; j < 4; ++j)
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
-                 : "r"(box + (uint32_t)r * 64u + 16u * (uint32_t)(j ^ ((r >> 1) & 3))));
-    const int gr = row0 + r, gc = col0 + 8 * j;
-    if (gr < M && gc < N) *reinterpret_cast<uint4*>(out + (long)gr * ldo + gc) = make_uint4(a, b, c, d);
-  }
+                 : "=r"(u[j].x), "=r"(u[j].y), "=r"(u[j].z), "=r"(u[j].w)
+                 : "r"(rb + 16u * (uint32_t)(j ^ x)));
 }
-
 DEVI void stage_f32_row(uint32_t box, int lane, const float (&v)[32]) {
   const uint32_t rb = box + (uint32_t)lane * 128u;
   const int x = lane & 7;

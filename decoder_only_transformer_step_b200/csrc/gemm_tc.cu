@@ -42,29 +42,38 @@ constexpr int NUM_EPI_WARPS = 8;  // two per TMEM lane quarter, each owning half
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t MN_ATOM_BYTES = 64 * BK * 2;  // one {64 MN x 64 K} TMA box
 
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool BIG_EPI>
 struct TcCfg {
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;   // output rows per work unit
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;   // rows of B this CTA loads per stage
-  static constexpr int STAGES = PAIR ? 6 : (BN == 256 ? 4 : 6);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int NUM_BARS = 2 * STAGES + 5;  // full, empty, acc_full[2], acc_empty[2], drain
+  // Per epilogue warp: two 32 x 32 bf16 staging boxes (TMA stores alternate
+  // between them) or one 4 KB fp32 box; with BIG_EPI 8 KB, adding a second
+  // output's two boxes (GELU) or two boxes for the residual / GELU' operand
+  // (TMA loads run one chunk ahead).  The smaller footprint leaves room for
+  // a deeper operand ring.
+  static constexpr int EPI_WARP_BYTES = BIG_EPI ? 8192 : 4096;
+  static constexpr int EPI_BYTES = NUM_EPI_WARPS * EPI_WARP_BYTES;
+  // full, empty, acc_full[2], acc_empty[2], drain, operand[8 warps][2]
+  static constexpr int NUM_FIXED_BARS = 5 + 2 * NUM_EPI_WARPS;
+  static constexpr int STAGES_FIT = (232448 - EPI_BYTES - 1024 - 512) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static constexpr int NUM_BARS = 2 * STAGES + NUM_FIXED_BARS;
   // accumulator-empty arrivals: one per epilogue warp of every CTA of the unit
   static constexpr uint32_t ACCE_COUNT = (PAIR ? 2 : 1) * NUM_EPI_WARPS;
-  // one 4 KB staging box per epilogue warp (TMA store source)
-  static constexpr int EPI_BYTES = NUM_EPI_WARPS * 4096;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + NUM_BARS * 8 + 16;
+  static_assert(STAGES >= 3, "pipeline depth");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
 // How the epilogue writes its result.
 enum StoreMode : int {
   ST_REG = 0,       // per-thread global stores (general fallback)
-  ST_BF16 = 1,      // one bf16 output, staged and stored coalesced
-  ST_BF16_X2 = 2,   // two bf16 outputs (u and GELU(u)), staged and stored coalesced
+  ST_BF16 = 1,      // one bf16 output, TMA store (residual / GELU' operand by TMA load)
+  ST_BF16_X2 = 2,   // two bf16 outputs (u and GELU(u)), two TMA stores
   ST_F32 = 3,       // fp32 output, TMA store (beta = 0)
   ST_F32_ADD = 4,   // fp32 output, TMA reduce-add (beta = 1)
   ST_F32_PART = 5,  // fp32 split-K partial [split][M][N], 3-D TMA store
@@ -113,12 +122,12 @@ DEVI void decode_unit(const TcParams& p, int u, int& m0, int& nt, int& s, int& k
   kb1 = (int)((long long)(s + 1) * p.kb_total / p.splits);
 }
 
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool BIG_EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
                    const TcParams p) {
-  using C = TcCfg<BN, PAIR>;
+  using C = TcCfg<BN, PAIR, BIG_EPI>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t tiles = (raw + 1023u) & ~1023u;
@@ -134,6 +143,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto accf_bar = [&](int b) { return bars + 8u * (2 * C::STAGES + b); };
   auto acce_bar = [&](int b) { return bars + 8u * (2 * C::STAGES + 2 + b); };
   const uint32_t drain_bar = bars + 8u * (2 * C::STAGES + 4);
+  // operand-load barrier of epilogue warp e, buffer b
+  auto op_bar = [&](int e, int b) { return bars + 8u * (2 * C::STAGES + 5 + 2 * e + b); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -152,6 +163,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(acce_bar(b), C::ACCE_COUNT);
     }
     mbar_init(drain_bar, 1);
+    for (int e = 0; e < NUM_EPI_WARPS; ++e) {
+      mbar_init(op_bar(e, 0), 1);
+      mbar_init(op_bar(e, 1), 1);
+    }
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmA);
@@ -308,14 +323,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ---------------------------------------------------- epilogue ----
+    // Per 32-column chunk: the residual / GELU' operand box arrives by TMA
+    // (issued one chunk ahead), the accumulator comes from TMEM, the result
+    // is staged in a 32 x 32 box and written by a TMA store.  Every global
+    // access of the epilogue is a TMA box; the threads only touch shared
+    // memory and TMEM.
     const int e = warp - 2;
     const int q = warp & 3;              // TMEM lanes [32q, 32q+32) are this warp's
     const int c_begin = (e >> 2) * (BN / 2);
-    const uint32_t box = epi_smem + (uint32_t)e * 4096u;
-    const bool has_operand = p.epi.kind == EPI_BIAS_RESID || p.epi.kind == EPI_DGELU;
-    const bf16* operand = (const bf16*)(p.epi.kind == EPI_DGELU ? p.epi.aux : p.epi.resid);
+    constexpr int NCH = BN / 64;  // 32-column chunks per warp and tile
+    const uint32_t wbox = epi_smem + (uint32_t)e * C::EPI_WARP_BYTES;
+    // (the host selects BIG_EPI whenever there is an operand or a second output)
+    const bool has_operand = BIG_EPI && (p.epi.kind == EPI_BIAS_RESID || p.epi.kind == EPI_DGELU);
+    int chunk = 0;      // chunks stored by this warp: output box chunk & 1
+    int op_issued = 0;  // operand boxes requested: box / barrier k & 1, phase k >> 1
+    int op_used = 0;
+    // box layout inside the warp's region: bf16 outputs at b * 2048 (and the
+    // GELU output at 4096 + b * 2048), operand at 4096 + b * 2048; fp32 at
+    // b * 4096 (BIG_EPI) or 0
+    auto op_box = [&](int k) { return wbox + 4096u + 2048u * (uint32_t)(k & 1); };
+    auto issue_op = [&](int row0_, int col0_) {
+      if (lane == 0) {
+        const uint32_t bar = op_bar(e, op_issued & 1);
+        mbar_arrive_expect_tx(bar, 2048);
+        tma_load_2d(op_box(op_issued), &tmC2, bar, col0_, row0_);
+      }
+      ++op_issued;
+    };
+    bool ok = true;
     int it = 0;
-    for (int u = unit0; u < units; u += unit_step, ++it) {
+    for (int u = unit0; u < units && ok; u += unit_step, ++it) {
       int m0, nt, s, kb0, kb1;
       decode_unit(p, u, m0, nt, s, kb0, kb1);
       const int n0 = nt * BN;
@@ -323,29 +360,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
       const int row0 = m0 + (int)rank * BM + q * 32;
       const int row = row0 + lane;
-      // the first chunk's residual / GELU' operand does not depend on the
-      // accumulator: fetch it while the MMAs run
-      uint4 pre[4];
-      if (has_operand) prefetch_bf16x32(operand, p.epi.ldo, p.M, p.N, row, n0 + c_begin, pre);
-      if (!mbar_wait_bounded(accf_bar(buf), aph, abort_flag, p.err)) break;
+      // the first chunk's operand does not depend on the accumulator: request
+      // it while the MMAs run (every box of the previous tile has been read)
+      if (has_operand && p.store != ST_REG && n0 + c_begin < p.N) issue_op(row0, n0 + c_begin);
+      if (!mbar_wait_bounded(accf_bar(buf), aph, abort_flag, p.err)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      for (int c = c_begin; c < c_begin + BN / 2; c += 32) {
-        const int col0 = n0 + c;
-        if (col0 >= p.N) break;  // warp-uniform
-        uint4 cur[4];
-        if (has_operand) {
+      // chunks of this warp's columns that lie inside N (warp-uniform)
+      const int nch = min(NCH, max(0, (p.N - (n0 + c_begin) + 31) / 32));
+      const uint32_t tm_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c_begin);
+      // With the small layout TMEM loads run one chunk ahead (chunk ci+1 is
+      // requested before chunk ci is processed); the larger epilogues have no
+      // registers to spare for that and load each chunk when they reach it.
+      constexpr bool PREFETCH = !BIG_EPI;
+      uint32_t r[NCH][32];
+      if (PREFETCH && nch > 0) tmem_ld_32x32b_x32(tm_row, r[0]);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) cur[i] = pre[i];
-          if (c + 32 < c_begin + BN / 2 && col0 + 32 < p.N)
-            prefetch_bf16x32(operand, p.epi.ldo, p.M, p.N, row, col0 + 32, pre);
-        }
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c), r);
+      for (int ci = 0; ci < NCH; ++ci) {
+        if (ci >= nch) break;
+        const int c = c_begin + 32 * ci;
+        const int col0 = n0 + c;
+        if (!PREFETCH) tmem_ld_32x32b_x32(tm_row + 32u * (uint32_t)ci, r[ci]);
         tmem_ld_wait();
         float v[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        if (p.store == ST_REG) {
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[ci][j]);
+        if (PREFETCH && ci + 1 < NCH && ci + 1 < nch)
+          tmem_ld_32x32b_x32(tm_row + 32u * (uint32_t)(ci + 1), r[ci + 1]);
+        // (per-element stores are only chosen with the small epilogue layout)
+        if (!BIG_EPI && p.store == ST_REG) {
           if (row < p.M) {
             if (col0 + 32 <= p.N) {
               epi_row32_bf16(p.epi, p.partial, s, p.M, p.N, row, col0, v);
@@ -358,45 +403,69 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           continue;
         }
+        uint4 cur[4];
+        if (has_operand) {
+          // next chunk's box goes to the other buffer, read one chunk ago
+          if (ci + 1 < nch) issue_op(row0, col0 + 32);
+          if (!mbar_wait_bounded(op_bar(e, op_used & 1), (uint32_t)(op_used >> 1) & 1u, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          load_bf16_box_row(op_box(op_used), lane, cur);
+          ++op_used;
+          // these reads precede the TMA load that refills the buffer
+          fence_proxy_async_smem();
+        }
         epi_apply_row32(p.epi, p.N, col0, v, cur);
+        // the store that last used this chunk's box has read it (two chunks
+        // ago; one chunk ago for the single fp32 box of the small layout)
+        const bool f32_single = !BIG_EPI && p.store != ST_BF16;
+        if (lane == 0) {
+          if (f32_single)
+            bulk_wait_read<0>();
+          else
+            bulk_wait_read<1>();
+        }
+        __syncwarp();
+        const uint32_t ob = f32_single ? 0u : (uint32_t)(chunk & 1);
         if (p.store == ST_BF16 || p.store == ST_BF16_X2) {
-          // bf16 outputs: transpose through the box, coalesced direct stores
-          stage_bf16_row(box, lane, v);
-          if (p.store == ST_BF16_X2) {
+          stage_bf16_row(wbox + 2048u * ob, lane, v);
+          if (BIG_EPI && p.store == ST_BF16_X2) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = gelu_f<true>(v[j]);
-            stage_bf16_row(box + 2048u, lane, v);
+            stage_bf16_row(wbox + 4096u + 2048u * ob, lane, v);
           }
-          __syncwarp();
-          unstage_bf16_box(box, lane, (bf16*)p.epi.out, p.epi.ldo, p.M, p.N, row0, col0);
-          if (p.store == ST_BF16_X2)
-            unstage_bf16_box(box + 2048u, lane, (bf16*)p.epi.out2, p.epi.ldo, p.M, p.N, row0, col0);
-          __syncwarp();
-          continue;
+        } else {
+          stage_f32_row(wbox + 4096u * ob, lane, v);
         }
-        // fp32 outputs: TMA store / reduce-add; the previous store from this
-        // box must have read it
-        if (lane == 0) bulk_wait_read<0>();
-        __syncwarp();
-        stage_f32_row(box, lane, v);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           switch (p.store) {
+            case ST_BF16:
+              tma_store_2d(&tmC, wbox + 2048u * ob, col0, row0);
+              break;
+            case ST_BF16_X2:
+              tma_store_2d(&tmC, wbox + 2048u * ob, col0, row0);
+              if (BIG_EPI) tma_store_2d(&tmC2, wbox + 4096u + 2048u * ob, col0, row0);
+              break;
             case ST_F32:
-              tma_store_2d(&tmC, box, col0, row0);
+              tma_store_2d(&tmC, wbox + 4096u * ob, col0, row0);
               break;
             case ST_F32_ADD:
-              tma_reduce_add_2d(&tmC, box, col0, row0);
+              tma_reduce_add_2d(&tmC, wbox + 4096u * ob, col0, row0);
               break;
             case ST_F32_PART:
-              tma_store_3d(&tmC, box, col0, row0, s);
+              tma_store_3d(&tmC, wbox + 4096u * ob, col0, row0, s);
               break;
           }
           bulk_commit();
         }
+        ++chunk;
       }
-      // every lane's TMEM loads have completed (tcgen05.wait::ld above)
+      tmem_ld_wait();  // (a no-op unless the loop left early)
+      if (!ok) break;
+      // every lane's TMEM loads have completed
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -407,7 +476,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mbar_arrive(acce_bar(buf));
       }
     }
-    if (lane == 0) bulk_wait_all();
+    if (lane == 0) {
+      bulk_wait_all();
+      // operand boxes still in flight (abort path) land before the CTA exits
+      for (int k = op_used; k < op_issued; ++k) mbar_drain_bounded(op_bar(e, k & 1), (uint32_t)(k >> 1) & 1u);
+    }
     __syncwarp();
   }
 
@@ -491,8 +564,9 @@ bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer
                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Output [M, N] with pitch ldo, stored in 32 x 32 boxes: bf16 with the 64-byte
-// swizzle, fp32 with the 128-byte swizzle (matching stage_*_row).
+// [M, N] with pitch ldo in 32 x 32 boxes (epilogue stores and operand loads):
+// bf16 with the 64-byte swizzle, fp32 with the 128-byte swizzle (matching
+// stage_*_row and load_bf16_box_row).
 bool make_out_tmap(CUtensorMap* tm, const void* base, int M, int N, long ldo, bool f32) {
   const uint64_t dims[2] = {(uint64_t)N, (uint64_t)M}, strides[1] = {(uint64_t)ldo * (f32 ? 4 : 2)};
   const uint32_t box[2] = {32, 32};
@@ -500,10 +574,10 @@ bool make_out_tmap(CUtensorMap* tm, const void* base, int M, int N, long ldo, bo
                      dims, strides, box, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool BIG_EPI>
 int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tc2,
               const TcParams& p, int units, cudaStream_t st) {
-  using C = TcCfg<BN, PAIR>;
+  using C = TcCfg<BN, PAIR, BIG_EPI>;
   static bool attr_set = false;
   static int max_slots = 0;  // co-resident CTAs (single) or clusters (pairs)
   cudaLaunchConfig_t cfg = {};
@@ -520,12 +594,12 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& t
     cfg.numAttrs = 1;
   }
   if (!attr_set) {
-    CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, PAIR, BIG_EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   C::SMEM_BYTES));
     if (PAIR) {
       cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<BN, PAIR>, &cfg) != cudaSuccess || n <= 0) {
+      if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<BN, PAIR, BIG_EPI>, &cfg) != cudaSuccess || n <= 0) {
         cudaGetLastError();
         n = num_sms() / 2;
       }
@@ -537,7 +611,7 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& t
   }
   const int slots = units < max_slots ? units : max_slots;
   cfg.gridDim = dim3((PAIR ? 2 : 1) * slots, 1, 1);
-  CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, PAIR>, ta, tb, tc, tc2, p));
+  CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, PAIR, BIG_EPI>, ta, tb, tc, tc2, p));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -630,12 +704,24 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   switch (p.epi.kind) {
     case EPI_STORE:
     case EPI_BIAS:
-    case EPI_BIAS_RESID:
-    case EPI_DGELU:
       p.store = ST_BF16;
+      ok_c = make_out_tmap(&tc, g.epi.out, g.M, g.N, g.epi.ldo, false);
       break;
+    case EPI_BIAS_RESID:
+    case EPI_DGELU: {
+      // tmC2: the operand read per chunk (same [M, ldo] layout as the output)
+      const void* opnd = p.epi.kind == EPI_DGELU ? g.epi.aux : g.epi.resid;
+      if ((uintptr_t)opnd & 15) return GPT2_ERR_INVALID_ARG;
+      p.store = ST_BF16;
+      ok_c = make_out_tmap(&tc, g.epi.out, g.M, g.N, g.epi.ldo, false) &&
+             make_out_tmap(&tc2, opnd, g.M, g.N, g.epi.ldo, false);
+      break;
+    }
     case EPI_BIAS_GELU:
+      if ((uintptr_t)g.epi.out2 & 15) return GPT2_ERR_INVALID_ARG;
       p.store = ST_BF16_X2;
+      ok_c = make_out_tmap(&tc, g.epi.out, g.M, g.N, g.epi.ldo, false) &&
+             make_out_tmap(&tc2, g.epi.out2, g.M, g.N, g.epi.ldo, false);
       break;
     case EPI_F32:
       if (g.epi.beta == 0.f || g.epi.beta == 1.f) {
@@ -658,12 +744,20 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
       p.store = ST_REG;
   }
   if (!ok_c) return GPT2_ERR_CUDA;
-  if (p.store == ST_BF16_X2 && ((uintptr_t)g.epi.out2 & 15)) return GPT2_ERR_INVALID_ARG;
 
   const int units = p.m_tiles * p.n_tiles * splits;
-  int rc = pair        ? launch_tc<256, true>(ta, tb, tc, tc2, p, units, st)
-           : bn == 256 ? launch_tc<256, false>(ta, tb, tc, tc2, p, units, st)
-                       : launch_tc<128, false>(ta, tb, tc, tc2, p, units, st);
+  // the second output or the operand boxes need the larger epilogue region
+  const bool big = p.store == ST_BF16_X2 || p.epi.kind == EPI_BIAS_RESID || p.epi.kind == EPI_DGELU;
+  int rc;
+  if (pair)
+    rc = big ? launch_tc<256, true, true>(ta, tb, tc, tc2, p, units, st)
+             : launch_tc<256, true, false>(ta, tb, tc, tc2, p, units, st);
+  else if (bn == 256)
+    rc = big ? launch_tc<256, false, true>(ta, tb, tc, tc2, p, units, st)
+             : launch_tc<256, false, false>(ta, tb, tc, tc2, p, units, st);
+  else
+    rc = big ? launch_tc<128, false, true>(ta, tb, tc, tc2, p, units, st)
+             : launch_tc<128, false, false>(ta, tb, tc, tc2, p, units, st);
   if (rc) return rc;
   if (splits > 1) {
     long mn = (long)g.M * g.N;
