@@ -27,7 +27,8 @@
 namespace {
 
 // 3-D bf16 tensor map, 128-byte swizzle, box {64, 128, 1}.
-bool tmap_3d(CUtensorMap* tm, const void* base, const uint64_t* dims, const uint64_t* strides) {
+bool tmap_3d(CUtensorMap* tm, const void* base, const uint64_t* dims, const uint64_t* strides,
+             CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, uint32_t box0 = 64, uint32_t box1 = 128) {
   static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   if (!enc) {
     void* p = nullptr;
@@ -39,9 +40,9 @@ bool tmap_3d(CUtensorMap* tm, const void* base, const uint64_t* dims, const uint
     enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   }
   cuuint64_t d[3] = {dims[0], dims[1], dims[2]}, s[2] = {strides[0], strides[1]};
-  cuuint32_t box[3] = {64, 128, 1}, e[3] = {1, 1, 1};
-  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), d, s, box, e,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  cuuint32_t box[3] = {box0, box1, 1}, e[3] = {1, 1, 1};
+  return enc(tm, dt, 3, const_cast<void*>(base), d, s, box, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -401,7 +402,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 //   P^T = exp(scale S^T - LSE), dS^T = P^T (dP^T - D)   (elementwise warps)
 //   dV += P^T dO, dK += dS^T Q              (M128 N64 K128, TMEM accumulators)
 //   dQ  = dS K                              (A = the dS^T buffer read MN-major)
-// and dQ is reduced into an fp32 buffer.  Eight elementwise warps (two per TMEM
+// and dQ is added into an fp32 buffer by TMA reductions (staged through the
+// block's spent Q/dO ring slot).  Eight elementwise warps (two per TMEM
 // lane quarter, 64 of the 128 query columns each) need no row reductions here,
 // so they split the columns with no communication; the next block's S^T/dP^T
 // MMAs run while they work.
@@ -422,14 +424,10 @@ constexpr uint32_t C_ST = 0, C_DPT = 128, C_DV = 256, C_DK = 320, C_DQ = 384;
 constexpr uint32_t IDESC_DQ =
     (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
 
-DEVI void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
 __global__ void __launch_bounds__(B_NUM_THREADS, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
-                       const float* __restrict__ lse, const float* __restrict__ dvec, float* __restrict__ dq_acc,
+                       const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse,
+                       const float* __restrict__ dvec,
                        bf16* __restrict__ dqkv, int T, int H, float scale, float scale_log2, int* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -458,7 +456,9 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
     mbar_init(kv_full, 1);
     for (int s = 0; s < QS; ++s) {
       mbar_init(qdo_full(s), 1);
-      mbar_init(qdo_empty(s), 1);
+      // released by the MMAs of the block and by the eight elementwise warps
+      // once their dQ reduction has read the slot
+      mbar_init(qdo_empty(s), 1 + 8);
     }
     mbar_init(st_full, 1);
     mbar_init(st_free, 256);
@@ -567,18 +567,33 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
     const int tid = threadIdx.x - 64;
     bool ok = true;
     auto drain_dq = [&](int t) {
-      // dQ rows are queries of block t; this warp takes 32 of the 64 columns
+      // dQ rows are queries of block t; this warp takes 32 of the 64 columns.
+      // Block t's Q/dO ring slot (its MMAs are complete) holds the fp32 dQ
+      // tile as two 128-row x 32-column boxes in the 128-byte swizzle; each
+      // warp stages its 32 x 32 part and adds it to dq_acc with one TMA
+      // reduce, then releases the slot to the loads.
+      const int sl = t % QS;
       uint32_t r[32];
       tmem_ld_32x32b_x32(tmem + lane_off + C_DQ + 64 * (t & 1) + 32 * half, r);
       tmem_ld_wait();
-      const int gq = (kvb + t) * BQ + row;
-      if (gq < T) {
-        float* dst = dq_acc + ((long)b * T + gq) * d + h * HD + 32 * half;
+      const uint32_t box = base + (half ? BS_DO : BS_Q) + sl * TILE + (uint32_t)(q * 32) * 128u;
+      const uint32_t rb = box + (uint32_t)lane * 128u;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          red_add_v4(dst + 4 * j, __uint_as_float(r[4 * j]) * scale, __uint_as_float(r[4 * j + 1]) * scale,
-                     __uint_as_float(r[4 * j + 2]) * scale, __uint_as_float(r[4 * j + 3]) * scale);
+      for (int j = 0; j < 8; ++j)
+        st_shared_v4(rb + 16u * (uint32_t)(j ^ (lane & 7)), __float_as_uint(__uint_as_float(r[4 * j]) * scale),
+                     __float_as_uint(__uint_as_float(r[4 * j + 1]) * scale),
+                     __float_as_uint(__uint_as_float(r[4 * j + 2]) * scale),
+                     __float_as_uint(__uint_as_float(r[4 * j + 3]) * scale));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        // rows past T are clipped by the tensor map
+        tma_reduce_add_3d(&tmDQ, box, h * HD + 32 * half, (kvb + t) * BQ + q * 32, b);
+        bulk_commit();
+        bulk_wait_read<0>();
+        mbar_arrive(qdo_empty(sl));
       }
+      __syncwarp();
     };
     // LSE (log2 domain) and D of every query block this CTA visits, once:
     // [block][LSE x128 | D x128]; queries past T get LSE = +inf (P = 0).
@@ -661,6 +676,7 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
     if (ok && mbar_wait_bounded(mma2_done, (nblk - 1) & 1, abort_flag, err)) {
       tc_fence_after();
       drain_dq(nblk - 1);
+      if (lane == 0) bulk_wait_all();
       uint32_t rk[32], rv[32];
       tmem_ld_32x32b_x32(tmem + lane_off + C_DK + 32 * half, rk);
       tmem_ld_32x32b_x32(tmem + lane_off + C_DV + 32 * half, rv);
@@ -705,14 +721,18 @@ int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float
   const uint64_t sq[2] = {3 * d * 2, (uint64_t)T * 3 * d * 2};
   const uint64_t dd[3] = {d, (uint64_t)T, (uint64_t)B};
   const uint64_t sd[2] = {d * 2, (uint64_t)T * d * 2};
-  if (!tmap_3d(&tq, qkv, dq, sq) || !tmap_3d(&tdo, dout, dd, sd)) return GPT2_ERR_CUDA;
+  CUtensorMap tdq;
+  const uint64_t sdq[2] = {d * 4, (uint64_t)T * d * 4};
+  if (!tmap_3d(&tq, qkv, dq, sq) || !tmap_3d(&tdo, dout, dd, sd) ||
+      !tmap_3d(&tdq, dq_acc, dd, sdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 32))
+    return GPT2_ERR_CUDA;
   static bool attr = false;
   if (!attr) {
     CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B_SMEM_BYTES));
     attr = true;
   }
   dim3 grid((T + BKV - 1) / BKV, B * H);
-  attn_bwd_tc_kernel<<<grid, B_NUM_THREADS, B_SMEM_BYTES, st>>>(tq, tdo, lse, dvec, dq_acc, (bf16*)dqkv, T, H,
+  attn_bwd_tc_kernel<<<grid, B_NUM_THREADS, B_SMEM_BYTES, st>>>(tq, tdo, tdq, lse, dvec, (bf16*)dqkv, T, H,
                                                                  0.125f, LOG2E_F / 8.f, nullptr);
   LAUNCH_CHECK();
   return GPT2_OK;

@@ -189,6 +189,13 @@ DEVI void tma_reduce_add_2d(const void* tmap, uint32_t src, int c0, int c1) {
                "r"(src), "r"(c0), "r"(c1)
                : "memory");
 }
+DEVI void tma_reduce_add_3d(const void* tmap, uint32_t src, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 DEVI void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 template <int N>
 DEVI void bulk_wait_read() {
