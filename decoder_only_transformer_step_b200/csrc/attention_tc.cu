@@ -99,11 +99,16 @@ DEVI float ex2(float x) {
   return y;
 }
 
-// Persistent: each CTA takes work items (query block, batch, head) w =
-// blockIdx.x, blockIdx.x + gridDim.x, ...; items are numbered longest causal
-// row first.  Key/value blocks are counted globally across a CTA's items (g),
-// so the K/V ring, the S / P / O double buffers and their barrier phases run
-// on without a break between items.
+// Work item of round k for CTA c of G: rounds alternate direction (snake), so
+// the long causal items of early rounds and the short ones of late rounds
+// even out across CTAs.
+DEVI int snake_item(int k, int c, int G) { return k * G + ((k & 1) ? G - 1 - c : c); }
+
+// Persistent: each CTA takes work items (query block, batch, head) in snake
+// order over rounds; items are numbered longest causal row first.  Key/value
+// blocks are counted globally across a CTA's items (g), so the K/V ring, the
+// S / P / O double buffers and their barrier phases run on without a break
+// between items.
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmO,
                        float* __restrict__ lse, int T, int H, int n_items, float scale_log2, int* err) {
@@ -172,7 +177,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       int g = 0, it = 0;
       int q_issued = 0, kv_issued = 0;
-      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+      for (int k = 0; ok; ++k, ++it) {
+        const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
+        if (w >= n_items) break;
         int qb, b, h;
         item(w, qb, b, h);
         const int qs = it & 1;
@@ -225,7 +232,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         return true;
       };
       int g = 0, it = 0;
-      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+      for (int k = 0; ok; ++k, ++it) {
+        const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
+        if (w >= n_items) break;
         int qb, b, h;
         item(w, qb, b, h);
         const int qs = it & 1;
@@ -271,7 +280,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float* xsum = xchg + 2 * 256;                                 // [half][128 rows] sums
     bool ok = true;
     int g = 0, it = 0;
-    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+    for (int k = 0; ok; ++k, ++it) {
+      const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
+      if (w >= n_items) break;
       int qb, b, h;
       item(w, qb, b, h);
       const int q0 = qb * BQ, grow = q0 + row;

@@ -161,6 +161,31 @@ def test_attention_forward_many_items(B, H, T):
     assert np.abs(lse.double().cpu().numpy() - lse_ref).max() <= 2e-2
 
 
+@pytest.mark.parametrize("B,H,T", [(4, 12, 512), (8, 12, 300)])
+def test_attention_backward_many_items(B, H, T):
+    """More (key block, batch, head) work items than SMs: the persistent
+    backward carries its ring phases and dQ buffers across items."""
+    hd = 64
+    d = H * hd
+    qkv = _attn_inputs(B, T, H, hd, 50 + T)
+    dout = bf16_rand((B * T, d), 60 + T)
+    o = torch.empty((B * T, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, T), dtype=torch.float32, device="cuda")
+    gp.gpt2_op_attention_fwd_bf16(qkv.cuda(), o, lse, B, T, H, hd)
+    dqkv = torch.empty((B * T, 3 * d), dtype=torch.bfloat16, device="cuda")
+    scratch = torch.empty(B * T * d + B * H * T, dtype=torch.float32, device="cuda")
+    gp.gpt2_op_attention_bwd_bf16(qkv.cuda(), o, lse, dout.cuda(), dqkv, scratch, B, T, H, hd)
+    q, k, v = _split(qkv, B, T, H, hd)
+    _, p = G.attention_fwd(q, k, v, None)
+    do = dout.double().numpy().reshape(B, T, H, hd).transpose(0, 2, 1, 3)
+    dq, dk, dv = G.attention_bwd(do, q, k, v, p, None)
+    got = _split(dqkv.cpu(), B, T, H, hd)
+    for name, g, r in zip("qkv", got, (dq, dk, dv)):
+        cos = (g * r).sum() / (np.linalg.norm(g) * np.linalg.norm(r))
+        rel = np.abs(g - r).max() / np.abs(r).max()
+        assert cos >= 0.999 and rel <= 2e-2, (name, cos, rel)
+
+
 @pytest.mark.parametrize("hd,T", [(64, 200), (64, 1024), (16, 64), (16, 77)])
 def test_attention_backward(hd, T):
     B, H = 2, 3
