@@ -623,16 +623,34 @@ int resolve_bn(int bn, int N) {
   return bn;
 }
 
+// Split-K factor for an fp32 (weight-gradient) product with fewer output
+// tiles than co-resident CTAs (pairs): the s minimising an estimate of
+//   waves(tiles * s) * (k-blocks per unit) * (time of one k-block of a tile)
+//   + s * M * N * 8 bytes (partials written and read back) / HBM bandwidth,
+// which weighs wave quantisation against the partial-sum traffic.
 int auto_splits(int M, int N, int K, int bn) {
   const bool pair = bn == 512;
   const int tile_m = pair ? 2 * BM : BM, tile_n = pair ? 256 : bn;
-  const int tiles = ((M + tile_m - 1) / tile_m) * ((N + tile_n - 1) / tile_n);
+  const long tiles = (long)((M + tile_m - 1) / tile_m) * ((N + tile_n - 1) / tile_n);
   const int kb = K / BK;
   const int slots = pair ? num_sms() / 2 : num_sms();
-  if (tiles >= slots) return 1;
-  int s = (2 * slots + tiles - 1) / tiles;
-  if (s > kb / 4) s = kb / 4;
-  return s < 1 ? 1 : s;
+  if (tiles >= slots || kb < 8) return 1;
+  // one k-block (64 deep) of one tile at ~11 TFLOP/s per SM, in microseconds
+  const double kblock_us = 2.0 * 128 * tile_n * BK / 11e6;
+  const double bytes_per_us = 6.5e6;  // HBM, bytes per microsecond
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= 16 && s <= kb / 4; ++s) {
+    const long units = tiles * s;
+    const long waves = (units + slots - 1) / slots;
+    const double cost = (double)waves * ((double)kb / s) * kblock_us +
+                        (s > 1 ? (double)s * M * N * 8.0 / bytes_per_us : 0.0);
+    if (cost < best_cost * 0.999) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
 }
 
 }  // namespace
