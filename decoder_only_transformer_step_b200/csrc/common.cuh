@@ -54,6 +54,13 @@ DEVI float warp_max(float v) {
   return v;
 }
 
+// 2^x on the MUFU unit (approximate; subnormal results flush to zero).
+DEVI float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ------------------------------------------------------------------ GELU --
 // tanh form: 0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))).
 #define GELU_K0 0.7978845608028654f

@@ -338,38 +338,65 @@ __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const i
                                                  float* __restrict__ loss_rows, int V, int vocab_real,
                                                  int* err) {
   constexpr int VN = Vec<T>::N;
-  __shared__ float sm_m[256], sm_s[256];
+  constexpr int U = 4;  // 16-byte vectors in flight per thread and trip
+  constexpr float L2E = 1.4426950408889634f;
+  __shared__ float sm_m[8], sm_s[8];
   const int m = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   T* z = logits + (long)m * V;
+  const int step = 256 * VN;
+  // pass 1: running maximum and sum of exp(z - max), U vectors per trip so the
+  // loads of a trip overlap (V is a multiple of 128, so vectors never straddle it)
   float mx = -INFINITY, sum = 0.f;
-  for (int c = threadIdx.x * VN; c < V; c += 256 * VN) {
-    float f[VN];
-    Vec<T>::load(z + c, f);
-    float lm = f[0];
+  for (int c0 = threadIdx.x * VN; c0 < V; c0 += U * step) {
+    float f[U][VN];
 #pragma unroll
-    for (int j = 1; j < VN; ++j) lm = fmaxf(lm, f[j]);
-    if (lm > mx) {
-      sum *= exp2f((mx - lm) * 1.4426950408889634f);
-      mx = lm;
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + u * step;
+      if (c < V) {
+        Vec<T>::load(z + c, f[u]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < VN; ++j) f[u][j] = -INFINITY;
+      }
     }
+    float lm = mx;
 #pragma unroll
-    for (int j = 0; j < VN; ++j) sum += exp2f((f[j] - mx) * 1.4426950408889634f);
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int j = 0; j < VN; ++j) lm = fmaxf(lm, f[u][j]);
+    // the first trip always holds a finite element, so lm is finite here
+    sum *= ex2_approx((mx - lm) * L2E);
+    mx = lm;
+    const float ml = mx * L2E;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int j = 0; j < VN; ++j) sum += ex2_approx(fmaf(f[u][j], L2E, -ml));
   }
-  sm_m[threadIdx.x] = mx;
-  sm_s[threadIdx.x] = sum;
+  // combine (max, sum) pairs: within the warp, then across the eight warps
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, mx, o), s2 = __shfl_xor_sync(0xffffffffu, sum, o);
+    const float mm = fmaxf(mx, m2);
+    // (a thread that saw no element, possible only for V < 2048, holds -inf, 0)
+    sum = (mx == -INFINITY ? 0.f : sum * ex2_approx((mx - mm) * L2E)) +
+          (m2 == -INFINITY ? 0.f : s2 * ex2_approx((m2 - mm) * L2E));
+    mx = mm;
+  }
+  if (lane == 0) {
+    sm_m[warp] = mx;
+    sm_s[warp] = sum;
+  }
   __syncthreads();
-  for (int o = 128; o > 0; o >>= 1) {
-    if (threadIdx.x < o) {
-      float m1 = sm_m[threadIdx.x], m2 = sm_m[threadIdx.x + o];
-      float s1 = sm_s[threadIdx.x], s2 = sm_s[threadIdx.x + o];
-      float mm = fmaxf(m1, m2);
-      float ss = (m1 == -INFINITY ? 0.f : s1 * expf(m1 - mm)) + (m2 == -INFINITY ? 0.f : s2 * expf(m2 - mm));
-      sm_m[threadIdx.x] = mm;
-      sm_s[threadIdx.x] = ss;
-    }
-    __syncthreads();
-  }
-  const float lse = sm_m[0] + logf(sm_s[0]);
+  float M0 = sm_m[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) M0 = fmaxf(M0, sm_m[w]);
+  float S0 = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w)
+    if (sm_m[w] != -INFINITY) S0 += sm_s[w] * ex2_approx((sm_m[w] - M0) * L2E);
+  const float lse = M0 + logf(S0);
   int y = tgt[m];
   if (y < 0 || y >= vocab_real) {
     if (threadIdx.x == 0) atomicOr(err, DEV_ERR_TOKEN);
@@ -378,12 +405,22 @@ __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const i
   const float zy = to_f(z[y]);
   __syncthreads();  // every thread has read z[y] before it is overwritten
   if (threadIdx.x == 0) loss_rows[m] = lse - zy;
-  for (int c = threadIdx.x * VN; c < V; c += 256 * VN) {
-    float f[VN];
-    Vec<T>::load(z + c, f);
+  // pass 2: dz = softmax(z) - onehot(y), in place
+  const float ll = lse * L2E;
+  for (int c0 = threadIdx.x * VN; c0 < V; c0 += U * step) {
+    float f[U][VN];
 #pragma unroll
-    for (int j = 0; j < VN; ++j) f[j] = __expf(f[j] - lse) - (c + j == y ? 1.f : 0.f);
-    Vec<T>::store(z + c, f);
+    for (int u = 0; u < U; ++u)
+      if (c0 + u * step < V) Vec<T>::load(z + c0 + u * step, f[u]);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + u * step;
+      if (c < V) {
+#pragma unroll
+        for (int j = 0; j < VN; ++j) f[u][j] = ex2_approx(fmaf(f[u][j], L2E, -ll)) - (c + j == y ? 1.f : 0.f);
+        Vec<T>::store(z + c, f[u]);
+      }
+    }
   }
 }
 
