@@ -260,11 +260,11 @@ def lm_head_roofline(gp, model, M, V, d, stream):
     C = torch.empty(M, V, dtype=torch.bfloat16, device="cuda")
     reps = 10
     for _ in range(3):
-        gp.gpt2_op_gemm_bf16(A, 0, d, wte, 0, d, C, 0, V, M, V, d)
+        gp.gpt2_op_gemm_bf16(A, 0, d, wte, 0, d, C, 0, V, M, V, d, stream=stream)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(reps):
-        gp.gpt2_op_gemm_bf16(A, 0, d, wte, 0, d, C, 0, V, M, V, d)
+        gp.gpt2_op_gemm_bf16(A, 0, d, wte, 0, d, C, 0, V, M, V, d, stream=stream)
     e1.record(stream)
     torch.cuda.synchronize()
     sec = e0.elapsed_time(e1) / 1e3 / reps
@@ -272,7 +272,7 @@ def lm_head_roofline(gp, model, M, V, d, stream):
     achieved = flop / sec / 1e12
     peak = peaks["bf16_tflops"]
     del A, C
-    return {"kernel": "gemm_tc_kernel<256> (tied LM head, forward: logits = LN_f(x) wte^T)",
+    return {"kernel": "gemm_tc_kernel<256, pair> (tied LM head, forward: logits = LN_f(x) wte^T)",
             "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4), "peak_source": f"{kind} bf16_tflops (burst)",
             "launch_ms": round(sec * 1e3, 4), "flop_per_launch": flop,
@@ -281,18 +281,20 @@ def lm_head_roofline(gp, model, M, V, d, stream):
 
 def recorded_traffic(key):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+    the current kernel sources (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     rec = json.load(open(p)).get(key)
     if not rec:
         return None
-    src = os.path.join(ROOT, rec["source"])
-    if not os.path.exists(src):
-        return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec["bytes_per_launch"] if sha == rec["source_sha256_16"] else None
+    h = hashlib.sha256()
+    for src in rec["sources"]:
+        path = os.path.join(ROOT, src)
+        if not os.path.exists(path):
+            return None
+        h.update(open(path, "rb").read())
+    return rec["bytes_per_launch"] if h.hexdigest()[:16] == rec["sources_sha256_16"] else None
 
 
 # ------------------------------------------------------ CPU oracle timing --
