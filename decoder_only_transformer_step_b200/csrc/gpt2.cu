@@ -104,7 +104,12 @@ struct Work {
   void *x_final, *yf, *logits;
   float *meanf, *rstdf, *loss_rows;
   void *dres, *dy, *du, *dqkv, *dout;
-  float *dq_acc, *dvec, *ln_part, *cs_part;
+  float *dq_acc, *dvec;
+  // block partials of every bias / LayerNorm parameter gradient of one
+  // backward, each in its own slot, all reduced by one launch at its end
+  float* part_arena;
+  size_t part_floats, part_used;
+  std::vector<ReduceJob> jobs;
   void* split_ws;
   size_t split_bytes;
   long long* emb_acc;
@@ -165,8 +170,12 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
   w->dout = c.take<void>(M * d * act);
   w->dq_acc = c.take<float>(M * d * 4);
   w->dvec = c.take<float>(M * s.H * 4);
-  w->ln_part = c.take<float>(layernorm_bwd_part_floats((int)M, (int)d) * 4);
-  w->cs_part = c.take<float>(colsum_part_floats((int)M, (int)(4 * d)) * 4);
+  w->part_floats = (size_t)s.L * (2 * colsum_part_floats((int)M, (int)d) + colsum_part_floats((int)M, (int)(4 * d)) +
+                                   colsum_part_floats((int)M, (int)(3 * d)) +
+                                   2 * layernorm_bwd_part_floats((int)M, (int)d)) +
+                   layernorm_bwd_part_floats((int)M, (int)d);
+  w->part_arena = c.take<float>(w->part_floats * 4);
+  w->part_used = 0;
   w->split_bytes = split_ws_need(s, M);
   w->split_ws = c.take<void>(w->split_bytes);
   w->emb_acc = c.take<long long>((size_t)s.V * d * 8);
@@ -225,14 +234,23 @@ GemmArgs make_gemm(int M, int N, int K, const void* A, int a_mn, long lda, const
     if (rc_) return rc_;    \
   } while (0)
 
-// param grads of one (gamma, beta) pair / bias from block partials
-int ln_param_grads(gpt2_ctx* c, int nblk, size_t goff, float beta, cudaStream_t st) {
-  return reduce_rows_f32(c->w.ln_part, nblk, (int)(2 * c->s.d), c->buf.grad + goff, beta, st);
+// A slot of the partials arena (sized in carve for every slot of a backward).
+float* part_slot(gpt2_ctx* c, size_t floats) {
+  float* p = c->w.part_arena + c->w.part_used;
+  c->w.part_used += floats;
+  return p;
 }
-int bias_grad(gpt2_ctx* c, const void* x, int M, int N, size_t goff, float beta, cudaStream_t st) {
+// param grads of one (gamma, beta) pair / bias: block partials now, the
+// reduction queued for the batched launch that ends the backward
+void ln_param_grads(gpt2_ctx* c, const float* part, int nblk, size_t goff) {
+  c->w.jobs.push_back(ReduceJob{part, c->buf.grad + goff, nblk, (int)(2 * c->s.d)});
+}
+int bias_grad(gpt2_ctx* c, const void* x, int M, int N, size_t goff, cudaStream_t st) {
   int nblk = 0;
-  TRY(colsum_partial(c->s.mode, x, M, N, c->w.cs_part, &nblk, st));
-  return reduce_rows_f32(c->w.cs_part, nblk, N, c->buf.grad + goff, beta, st);
+  float* part = part_slot(c, colsum_part_floats(M, N));
+  TRY(colsum_partial(c->s.mode, x, M, N, part, &nblk, st));
+  c->w.jobs.push_back(ReduceJob{part, c->buf.grad + goff, nblk, N});
+  return GPT2_OK;
 }
 
 }  // namespace
@@ -420,10 +438,13 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
   g.epi.alpha = sc;
   g.epi.beta = beta;
   TRY(run_gemm(c, g, st));
+  w.part_used = 0;
+  w.jobs.clear();
+  const size_t lnp = layernorm_bwd_part_floats(M, d);
   int nblk = 0;
-  TRY(layernorm_bwd(f32, w.dy, w.x_final, w.meanf, w.rstdf, Wp(c, o.lnf_g()), w.dres, 1, w.ln_part, &nblk, M, d,
-                    st));
-  TRY(ln_param_grads(c, nblk, o.lnf_g(), beta, st));
+  float* part = part_slot(c, lnp);
+  TRY(layernorm_bwd(f32, w.dy, w.x_final, w.meanf, w.rstdf, Wp(c, o.lnf_g()), w.dres, 1, part, &nblk, M, d, st));
+  ln_param_grads(c, part, nblk, o.lnf_g());
 
   for (int l = (int)s.L - 1; l >= 0; --l) {
     LayerActs& a = w.layers[l];
@@ -434,24 +455,25 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
     g = make_gemm(d, 4 * d, M, w.dres, 1, d, a.g, 1, 4 * d, EPI_F32, G + o.layer(l, W_MP), 4 * d);
     g.epi.beta = beta;
     TRY(run_gemm(c, g, st));
-    TRY(bias_grad(c, w.dres, M, d, o.layer(l, B_MP), beta, st));
+    TRY(bias_grad(c, w.dres, M, d, o.layer(l, B_MP), st));
     // MLP fc: u = y2 W_fc^T + b_fc
     g = make_gemm(M, d, 4 * d, w.du, 0, 4 * d, Wp(c, o.layer(l, W_FC)), 1, d, EPI_STORE, w.dy, d);
     TRY(run_gemm(c, g, st));
     g = make_gemm(4 * d, d, M, w.du, 1, 4 * d, a.y2, 1, d, EPI_F32, G + o.layer(l, W_FC), d);
     g.epi.beta = beta;
     TRY(run_gemm(c, g, st));
-    TRY(bias_grad(c, w.du, M, 4 * d, o.layer(l, B_FC), beta, st));
-    TRY(layernorm_bwd(f32, w.dy, a.x_mid, a.mean2, a.rstd2, Wp(c, o.layer(l, LN2_G)), w.dres, 0, w.ln_part, &nblk,
-                      M, d, st));
-    TRY(ln_param_grads(c, nblk, o.layer(l, LN2_G), beta, st));
+    TRY(bias_grad(c, w.du, M, 4 * d, o.layer(l, B_FC), st));
+    part = part_slot(c, lnp);
+    TRY(layernorm_bwd(f32, w.dy, a.x_mid, a.mean2, a.rstd2, Wp(c, o.layer(l, LN2_G)), w.dres, 0, part, &nblk, M, d,
+                      st));
+    ln_param_grads(c, part, nblk, o.layer(l, LN2_G));
     // attention projection: x_mid = x_in + o W_o^T + b_o
     g = make_gemm(M, d, d, w.dres, 0, d, Wp(c, o.layer(l, W_O)), 1, d, EPI_STORE, w.dout, d);
     TRY(run_gemm(c, g, st));
     g = make_gemm(d, d, M, w.dres, 1, d, a.o, 1, d, EPI_F32, G + o.layer(l, W_O), d);
     g.epi.beta = beta;
     TRY(run_gemm(c, g, st));
-    TRY(bias_grad(c, w.dres, M, d, o.layer(l, B_O), beta, st));
+    TRY(bias_grad(c, w.dres, M, d, o.layer(l, B_O), st));
     // attention
     if (f32)
       TRY(attn_bwd_f32((const float*)a.qkv, (const float*)a.o, a.lse, (const float*)w.dout, (float*)w.dqkv, w.dvec,
@@ -465,11 +487,14 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
     g = make_gemm(3 * d, d, M, w.dqkv, 1, 3 * d, a.y1, 1, d, EPI_F32, G + o.layer(l, W_QKV), d);
     g.epi.beta = beta;
     TRY(run_gemm(c, g, st));
-    TRY(bias_grad(c, w.dqkv, M, 3 * d, o.layer(l, B_QKV), beta, st));
-    TRY(layernorm_bwd(f32, w.dy, a.x_in, a.mean1, a.rstd1, Wp(c, o.layer(l, LN1_G)), w.dres, 0, w.ln_part, &nblk,
-                      M, d, st));
-    TRY(ln_param_grads(c, nblk, o.layer(l, LN1_G), beta, st));
+    TRY(bias_grad(c, w.dqkv, M, 3 * d, o.layer(l, B_QKV), st));
+    part = part_slot(c, lnp);
+    TRY(layernorm_bwd(f32, w.dy, a.x_in, a.mean1, a.rstd1, Wp(c, o.layer(l, LN1_G)), w.dres, 0, part, &nblk, M, d,
+                      st));
+    ln_param_grads(c, part, nblk, o.layer(l, LN1_G));
   }
+  // every bias and LayerNorm parameter gradient, in one launch
+  TRY(reduce_rows_batch(w.jobs.data(), (int)w.jobs.size(), beta, st));
   // x_0 = wte[tok] + wpe[t]
   TRY(embed_bwd(f32, w.tok, w.dres, G + o.wte(), G + o.wpe(), w.emb_acc, w.touched, M, (int)s.T, d, V, accumulate,
                 st));

@@ -82,6 +82,14 @@ int layernorm_bwd(int f32, const void* dy, const void* x, const float* mean, con
 size_t layernorm_bwd_part_floats(int M, int d);
 // grad[j] = beta*grad[j] + sum_b part[b, j]  for j < n  (part row pitch n)
 int reduce_rows_f32(const float* part, int nrows, int n, float* grad, float beta, cudaStream_t st);
+// Many such reductions in one launch (same per-column summation order).
+struct ReduceJob {
+  const float* part;
+  float* grad;
+  int nrows, n;
+};
+constexpr int MAX_REDUCE_JOBS = 96;
+int reduce_rows_batch(const ReduceJob* jobs, int njobs, float beta, cudaStream_t st);
 // per-block column sums of x [M, N] (act) into part [nblk, N]
 int colsum_partial(int f32, const void* x, int M, int N, float* part, int* nblk, cudaStream_t st);
 size_t colsum_part_floats(int M, int N);

@@ -294,6 +294,36 @@ __global__ void reduce_rows_kernel(const float* __restrict__ part, int nrows, in
   }
 }
 
+// The same reduction for up to MAX_REDUCE_JOBS (part, grad) pairs in one
+// launch: block b takes 32 columns of the job whose column blocks contain b.
+struct ReduceBatchArgs {
+  ReduceJob job[MAX_REDUCE_JOBS];
+  int start[MAX_REDUCE_JOBS + 1];  // first column block of each job
+  int njobs;
+  float beta;
+};
+
+__global__ void reduce_rows_batch_kernel(const __grid_constant__ ReduceBatchArgs a) {
+  __shared__ float sm[8][33];
+  int jb = 0;
+  while (jb + 1 < a.njobs && a.start[jb + 1] <= (int)blockIdx.x) ++jb;
+  const float* part = a.job[jb].part;
+  float* grad = a.job[jb].grad;
+  const int nrows = a.job[jb].nrows, n = a.job[jb].n;
+  const int cx = threadIdx.x & 31, ry = threadIdx.x >> 5;
+  const int j = ((int)blockIdx.x - a.start[jb]) * 32 + cx;
+  float s = 0.f;
+  if (j < n)
+    for (int r = ry; r < nrows; r += 8) s += part[(long)r * n + j];
+  sm[ry][cx] = s;
+  __syncthreads();
+  if (ry == 0 && j < n) {
+    float t = sm[0][cx];
+    for (int k = 1; k < 8; ++k) t += sm[k][cx];
+    grad[j] = (a.beta != 0.f ? a.beta * grad[j] : 0.f) + t;
+  }
+}
+
 // Column sums of x[M, N] over blocks of 128 rows -> part[rowblock, N].
 constexpr int CS_ROWS = 128;
 
@@ -661,6 +691,25 @@ int layernorm_bwd(int f32, const void* dy, const void* x, const float* mean, con
 int reduce_rows_f32(const float* part, int nrows, int n, float* grad, float beta, cudaStream_t st) {
   reduce_rows_kernel<<<(n + 31) / 32, 256, 0, st>>>(part, nrows, n, grad, beta);
   LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int reduce_rows_batch(const ReduceJob* jobs, int njobs, float beta, cudaStream_t st) {
+  for (int j0 = 0; j0 < njobs; j0 += MAX_REDUCE_JOBS) {
+    ReduceBatchArgs a;
+    a.njobs = njobs - j0 < MAX_REDUCE_JOBS ? njobs - j0 : MAX_REDUCE_JOBS;
+    a.beta = beta;
+    int blocks = 0;
+    for (int k = 0; k < a.njobs; ++k) {
+      a.job[k] = jobs[j0 + k];
+      a.start[k] = blocks;
+      blocks += (jobs[j0 + k].n + 31) / 32;
+    }
+    a.start[a.njobs] = blocks;
+    if (blocks == 0) continue;
+    reduce_rows_batch_kernel<<<blocks, 256, 0, st>>>(a);
+    LAUNCH_CHECK();
+  }
   return GPT2_OK;
 }
 
