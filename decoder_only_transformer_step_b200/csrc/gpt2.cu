@@ -170,10 +170,13 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
   w->dout = c.take<void>(M * d * act);
   w->dq_acc = c.take<float>(M * d * 4);
   w->dvec = c.take<float>(M * s.H * 4);
-  w->part_floats = (size_t)s.L * (2 * colsum_part_floats((int)M, (int)d) + colsum_part_floats((int)M, (int)(4 * d)) +
-                                   colsum_part_floats((int)M, (int)(3 * d)) +
-                                   2 * layernorm_bwd_part_floats((int)M, (int)d)) +
-                   layernorm_bwd_part_floats((int)M, (int)d);
+  // per layer: two LayerNorms (gamma/beta partials + the column sums of their
+  // output, the b_o / b_mp gradients) and the b_fc, b_qkv column sums; plus
+  // the final LayerNorm
+  const size_t ln_rows = layernorm_bwd_part_rows((int)M);
+  w->part_floats = (size_t)s.L * (2 * ln_rows * 3 * d + colsum_part_floats((int)M, (int)(4 * d)) +
+                                   colsum_part_floats((int)M, (int)(3 * d))) +
+                   ln_rows * 3 * d;
   w->part_arena = c.take<float>(w->part_floats * 4);
   w->part_used = 0;
   w->split_bytes = split_ws_need(s, M);
@@ -244,6 +247,22 @@ float* part_slot(gpt2_ctx* c, size_t floats) {
 // reduction queued for the batched launch that ends the backward
 void ln_param_grads(gpt2_ctx* c, const float* part, int nblk, size_t goff) {
   c->w.jobs.push_back(ReduceJob{part, c->buf.grad + goff, nblk, (int)(2 * c->s.d)});
+}
+// LayerNorm backward writing the new residual-stream gradient into w.dres,
+// its (gamma, beta) gradient at goff and, when res_goff is not ~0, the column
+// sums of that new gradient (a bias gradient) at res_goff
+int ln_backward(gpt2_ctx* c, const void* x, const float* mean, const float* rstd, size_t g_off, int init,
+                size_t goff, size_t res_goff, int M, cudaStream_t st) {
+  const int d = (int)c->s.d;
+  const size_t rows = layernorm_bwd_part_rows(M);
+  float* part = part_slot(c, rows * 2 * d);
+  float* pres = res_goff != ~(size_t)0 ? part_slot(c, rows * d) : nullptr;
+  int nblk = 0;
+  TRY(layernorm_bwd(c->s.mode, c->w.dy, x, mean, rstd, Wp(c, g_off), c->w.dres, init, part, pres, &nblk, M, d,
+                    st));
+  ln_param_grads(c, part, nblk, goff);
+  if (pres) c->w.jobs.push_back(ReduceJob{pres, c->buf.grad + res_goff, nblk, d});
+  return GPT2_OK;
 }
 int bias_grad(gpt2_ctx* c, const void* x, int M, int N, size_t goff, cudaStream_t st) {
   int nblk = 0;
@@ -440,11 +459,8 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
   TRY(run_gemm(c, g, st));
   w.part_used = 0;
   w.jobs.clear();
-  const size_t lnp = layernorm_bwd_part_floats(M, d);
-  int nblk = 0;
-  float* part = part_slot(c, lnp);
-  TRY(layernorm_bwd(f32, w.dy, w.x_final, w.meanf, w.rstdf, Wp(c, o.lnf_g()), w.dres, 1, part, &nblk, M, d, st));
-  ln_param_grads(c, part, nblk, o.lnf_g());
+  // the new residual gradient's column sums are the last MLP projection's b_mp gradient
+  TRY(ln_backward(c, w.x_final, w.meanf, w.rstdf, o.lnf_g(), 1, o.lnf_g(), o.layer(s.L - 1, B_MP), M, st));
 
   for (int l = (int)s.L - 1; l >= 0; --l) {
     LayerActs& a = w.layers[l];
@@ -455,7 +471,6 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
     g = make_gemm(d, 4 * d, M, w.dres, 1, d, a.g, 1, 4 * d, EPI_F32, G + o.layer(l, W_MP), 4 * d);
     g.epi.beta = beta;
     TRY(run_gemm(c, g, st));
-    TRY(bias_grad(c, w.dres, M, d, o.layer(l, B_MP), st));
     // MLP fc: u = y2 W_fc^T + b_fc
     g = make_gemm(M, d, 4 * d, w.du, 0, 4 * d, Wp(c, o.layer(l, W_FC)), 1, d, EPI_STORE, w.dy, d);
     TRY(run_gemm(c, g, st));
@@ -463,17 +478,14 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
     g.epi.beta = beta;
     TRY(run_gemm(c, g, st));
     TRY(bias_grad(c, w.du, M, 4 * d, o.layer(l, B_FC), st));
-    part = part_slot(c, lnp);
-    TRY(layernorm_bwd(f32, w.dy, a.x_mid, a.mean2, a.rstd2, Wp(c, o.layer(l, LN2_G)), w.dres, 0, part, &nblk, M, d,
-                      st));
-    ln_param_grads(c, part, nblk, o.layer(l, LN2_G));
+    // column sums of the new residual gradient: the attention projection's b_o gradient
+    TRY(ln_backward(c, a.x_mid, a.mean2, a.rstd2, o.layer(l, LN2_G), 0, o.layer(l, LN2_G), o.layer(l, B_O), M, st));
     // attention projection: x_mid = x_in + o W_o^T + b_o
     g = make_gemm(M, d, d, w.dres, 0, d, Wp(c, o.layer(l, W_O)), 1, d, EPI_STORE, w.dout, d);
     TRY(run_gemm(c, g, st));
     g = make_gemm(d, d, M, w.dres, 1, d, a.o, 1, d, EPI_F32, G + o.layer(l, W_O), d);
     g.epi.beta = beta;
     TRY(run_gemm(c, g, st));
-    TRY(bias_grad(c, w.dres, M, d, o.layer(l, B_O), st));
     // attention
     if (f32)
       TRY(attn_bwd_f32((const float*)a.qkv, (const float*)a.o, a.lse, (const float*)w.dout, (float*)w.dqkv, w.dvec,
@@ -488,10 +500,9 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
     g.epi.beta = beta;
     TRY(run_gemm(c, g, st));
     TRY(bias_grad(c, w.dqkv, M, 3 * d, o.layer(l, B_QKV), st));
-    part = part_slot(c, lnp);
-    TRY(layernorm_bwd(f32, w.dy, a.x_in, a.mean1, a.rstd1, Wp(c, o.layer(l, LN1_G)), w.dres, 0, part, &nblk, M, d,
-                      st));
-    ln_param_grads(c, part, nblk, o.layer(l, LN1_G));
+    // column sums of the new residual gradient: the previous layer's b_mp gradient
+    TRY(ln_backward(c, a.x_in, a.mean1, a.rstd1, o.layer(l, LN1_G), 0, o.layer(l, LN1_G),
+                    l > 0 ? o.layer(l - 1, B_MP) : ~(size_t)0, M, st));
   }
   // every bias and LayerNorm parameter gradient, in one launch
   TRY(reduce_rows_batch(w.jobs.data(), (int)w.jobs.size(), beta, st));

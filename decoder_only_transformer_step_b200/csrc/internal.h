@@ -75,10 +75,13 @@ int embed_fwd(int f32, const int32_t* tok, const void* wte, const void* wpe, voi
 int layernorm_fwd(int f32, const void* x, const void* g, const void* b, void* y, float* mean,
                   float* rstd, int M, int d, cudaStream_t st);
 // dres = (dres_init ? 0 : dres) + LN'(dy); writes per-block partials of
-// dgamma, dbeta into part [nblk, 2, d]; returns nblk via *nblk.
+// dgamma, dbeta into part [nblk, 2, d] and, if part_res is not NULL, the
+// column sums of the new dres into part_res [nblk, d]; returns nblk.
 int layernorm_bwd(int f32, const void* dy, const void* x, const float* mean, const float* rstd,
-                  const void* g, void* dres, int dres_init, float* part, int* nblk, int M, int d,
-                  cudaStream_t st);
+                  const void* g, void* dres, int dres_init, float* part, float* part_res, int* nblk, int M,
+                  int d, cudaStream_t st);
+// rows of those partial buffers (floats: rows * 2d and rows * d)
+size_t layernorm_bwd_part_rows(int M);
 size_t layernorm_bwd_part_floats(int M, int d);
 // grad[j] = beta*grad[j] + sum_b part[b, j]  for j < n  (part row pitch n)
 int reduce_rows_f32(const float* part, int nrows, int n, float* grad, float beta, cudaStream_t st);

@@ -41,6 +41,20 @@ struct Vec<float> {
   }
 };
 
+// One 16-byte word as VN floats (the register form of Vec<T>::load).
+template <typename T>
+DEVI void unpack16(const uint4& u, float (&f)[Vec<T>::N]);
+template <>
+DEVI void unpack16<bf16>(const uint4& u, float (&f)[8]) {
+  f[0] = bf16lo(u.x); f[1] = bf16hi(u.x); f[2] = bf16lo(u.y); f[3] = bf16hi(u.y);
+  f[4] = bf16lo(u.z); f[5] = bf16hi(u.z); f[6] = bf16lo(u.w); f[7] = bf16hi(u.w);
+}
+template <>
+DEVI void unpack16<float>(const uint4& u, float (&f)[4]) {
+  f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y); f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+
 // ------------------------------------------------------------- embedding --
 
 // x[m] = wte[tok[m]] + wpe[m mod T]; one warp per row.
@@ -272,6 +286,133 @@ __global__ void __launch_bounds__(256) ln_param_colsum_kernel(const T* __restric
       for (int w = 1; w < 8; ++w) t += red[w][which][k];
       part[(long)blockIdx.y * 2 * d + which * d + col] = t;
     }
+  }
+}
+
+// LayerNorm backward in one pass over dy and x: per row (one warp, the row in
+// registers) dres = (init ? 0 : dres) + dx as in ln_bwd_dx_kernel, and per
+// lane column accumulators of dgamma = sum dy * xhat, dbeta = sum dy and (for
+// RES) sum of the new dres, which is the bias gradient of the linear layer
+// that produced this residual-stream gradient.  Rows are dealt to the
+// grid's warps round-robin; each block writes its column sums (fixed warp
+// order) to part_ln[block][0:d | d:2d] and part_res[block][0:d].
+constexpr int LNF_WARPS = 4;
+constexpr int LNF_BLOCKS_PER_SM = 3;
+
+template <typename T, int NC, bool RES>
+__global__ void __launch_bounds__(32 * LNF_WARPS, LNF_BLOCKS_PER_SM)
+    ln_bwd_fused_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __restrict__ mean,
+                        const float* __restrict__ rstd, const T* __restrict__ g, T* __restrict__ dres,
+                        int dres_init, int M, int d, float* __restrict__ part_ln, float* __restrict__ part_res) {
+  constexpr int VN = Vec<T>::N;
+  extern __shared__ float red[];  // [LNF_WARPS][3][d]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float sg[NC][VN], sb[NC][VN], sr[NC][VN];
+#pragma unroll
+  for (int k = 0; k < NC; ++k)
+#pragma unroll
+    for (int j = 0; j < VN; ++j) sg[k][j] = sb[k][j] = sr[k][j] = 0.f;
+  // the rows stay packed (16-byte words) in registers and are unpacked on
+  // each use, which leaves room to prefetch the next row while this one is
+  // processed: two rows of loads in flight per warp
+  const int stride = gridDim.x * LNF_WARPS;
+  int m = blockIdx.x * LNF_WARPS + warp;
+  uint4 cx[NC], cd[NC];
+  auto load_row = [&](int r, uint4 (&ux)[NC], uint4 (&ud)[NC]) {
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = (lane + 32 * k) * VN;
+      if (r < M && c < d) {
+        ux[k] = *reinterpret_cast<const uint4*>(x + (long)r * d + c);
+        ud[k] = *reinterpret_cast<const uint4*>(dy + (long)r * d + c);
+      }
+    }
+  };
+  load_row(m, cx, cd);
+  for (; m < M; m += stride) {
+    uint4 nx[NC], nd[NC];
+    load_row(m + stride, nx, nd);
+    uint4 cr[NC];
+    if (!dres_init) {
+#pragma unroll
+      for (int k = 0; k < NC; ++k) {
+        const int c = (lane + 32 * k) * VN;
+        if (c < d) cr[k] = *reinterpret_cast<const uint4*>(dres + (long)m * d + c);
+      }
+    }
+    const float mu = mean[m], rs = rstd[m];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = (lane + 32 * k) * VN;
+      if (c < d) {
+        float xv[VN], dv[VN], gv[VN];
+        unpack16<T>(cx[k], xv);
+        unpack16<T>(cd[k], dv);
+        Vec<T>::load(g + c, gv);
+#pragma unroll
+        for (int j = 0; j < VN; ++j) {
+          const float xh = (xv[j] - mu) * rs, gd = dv[j] * gv[j];
+          s1 += gd;
+          s2 += gd * xh;
+          sg[k][j] += dv[j] * xh;
+          sb[k][j] += dv[j];
+        }
+      }
+    }
+    s1 = warp_sum(s1) / d;
+    s2 = warp_sum(s2) / d;
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = (lane + 32 * k) * VN;
+      if (c < d) {
+        float xv[VN], dv[VN], gv[VN], o[VN];
+        unpack16<T>(cx[k], xv);
+        unpack16<T>(cd[k], dv);
+        Vec<T>::load(g + c, gv);
+        if (!dres_init) {
+          unpack16<T>(cr[k], o);
+        } else {
+#pragma unroll
+          for (int j = 0; j < VN; ++j) o[j] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < VN; ++j) {
+          const float xh = (xv[j] - mu) * rs, gd = dv[j] * gv[j];
+          o[j] += rs * (gd - s1 - xh * s2);
+          if (RES) sr[k][j] += o[j];
+        }
+        Vec<T>::store(dres + (long)m * d + c, o);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      cx[k] = nx[k];
+      cd[k] = nd[k];
+    }
+  }
+  constexpr int NQ = RES ? 3 : 2;
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    const int c = (lane + 32 * k) * VN;
+    if (c < d) {
+#pragma unroll
+      for (int j = 0; j < VN; ++j) {
+        red[(warp * NQ + 0) * d + c + j] = sg[k][j];
+        red[(warp * NQ + 1) * d + c + j] = sb[k][j];
+        if (RES) red[(warp * NQ + 2) * d + c + j] = sr[k][j];
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < NQ * d; i += 32 * LNF_WARPS) {
+    float t = red[i];
+#pragma unroll
+    for (int w = 1; w < LNF_WARPS; ++w) t += red[w * NQ * d + i];
+    if (i < 2 * d)
+      part_ln[(long)blockIdx.x * 2 * d + i] = t;
+    else
+      part_res[(long)blockIdx.x * d + (i - 2 * d)] = t;
   }
 }
 
@@ -626,30 +767,61 @@ int ln_fwd_dispatch(const void* x, const void* g, const void* b, void* y, float*
   return GPT2_OK;
 }
 
+int ln_fused_blocks(int M) {
+  const int b = LNF_BLOCKS_PER_SM * num_sms();
+  const int need = (M + LNF_WARPS - 1) / LNF_WARPS;
+  return b < need ? b : need;
+}
+
+// The fused one-pass kernel keeps 2-3 column accumulators per element a lane
+// owns, so it is used while a lane owns at most 24 columns of the row (d 768
+// in bf16 or fp32); wider rows take the row kernel plus the column-sum
+// kernels.
 template <typename T, int NC>
 void ln_bwd_launch(const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
-                   void* dres, int init, float* part, int M, int d, cudaStream_t st) {
+                   void* dres, int init, float* part, float* part_res, int* nblk, int M, int d, cudaStream_t st) {
+  constexpr int VN = Vec<T>::N;
+  if constexpr (NC * VN <= 24) {
+    const int blocks = ln_fused_blocks(M);
+    *nblk = blocks;
+    if (part_res) {
+      const size_t smem = (size_t)LNF_WARPS * 3 * d * sizeof(float);
+      ln_bwd_fused_kernel<T, NC, true><<<blocks, 32 * LNF_WARPS, smem, st>>>(
+          (const T*)dy, (const T*)x, mean, rstd, (const T*)g, (T*)dres, init, M, d, part, part_res);
+    } else {
+      const size_t smem = (size_t)LNF_WARPS * 2 * d * sizeof(float);
+      ln_bwd_fused_kernel<T, NC, false><<<blocks, 32 * LNF_WARPS, smem, st>>>(
+          (const T*)dy, (const T*)x, mean, rstd, (const T*)g, (T*)dres, init, M, d, part, nullptr);
+    }
+    return;
+  }
+  *nblk = (M + LNP_ROWS - 1) / LNP_ROWS;
   ln_bwd_dx_kernel<T, NC><<<(M + 7) / 8, 256, 0, st>>>((const T*)dy, (const T*)x, mean, rstd, (const T*)g,
                                                        (T*)dres, init, M, d);
   gpt2_count_launch();
-  constexpr int VN = Vec<T>::N;
   dim3 grid((d + 32 * VN - 1) / (32 * VN), (M + LNP_ROWS - 1) / LNP_ROWS);
   ln_param_colsum_kernel<T><<<grid, 256, 0, st>>>((const T*)dy, (const T*)x, mean, rstd, M, d, part);
+  if (part_res) {
+    gpt2_count_launch();
+    // column sums of the new dres in the same row blocks (CS_ROWS == LNP_ROWS)
+    dim3 g2((d + 32 * VN - 1) / (32 * VN), (M + CS_ROWS - 1) / CS_ROWS);
+    colsum_kernel<T><<<g2, 256, 0, st>>>((const T*)dres, M, d, part_res);
+  }
 }
 
 template <typename T>
 int ln_bwd_dispatch(const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
-                    void* dres, int init, float* part, int M, int d, cudaStream_t st) {
+                    void* dres, int init, float* part, float* part_res, int* nblk, int M, int d, cudaStream_t st) {
   const int nc = (d / Vec<T>::N + 31) / 32;
   switch (nc) {
-    case 1: ln_bwd_launch<T, 1>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
-    case 2: ln_bwd_launch<T, 2>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
-    case 3: ln_bwd_launch<T, 3>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
-    case 4: ln_bwd_launch<T, 4>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
-    case 5: ln_bwd_launch<T, 5>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
-    case 6: ln_bwd_launch<T, 6>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
-    case 7: ln_bwd_launch<T, 7>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
-    case 8: ln_bwd_launch<T, 8>(dy, x, mean, rstd, g, dres, init, part, M, d, st); break;
+    case 1: ln_bwd_launch<T, 1>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 2: ln_bwd_launch<T, 2>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 3: ln_bwd_launch<T, 3>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 4: ln_bwd_launch<T, 4>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 5: ln_bwd_launch<T, 5>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 6: ln_bwd_launch<T, 6>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 7: ln_bwd_launch<T, 7>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 8: ln_bwd_launch<T, 8>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
     default: return GPT2_ERR_UNSUPPORTED_SHAPE;
   }
   LAUNCH_CHECK();
@@ -679,13 +851,17 @@ int layernorm_fwd(int f32, const void* x, const void* g, const void* b, void* y,
              : ln_fwd_dispatch<bf16>(x, g, b, y, mean, rstd, M, d, st);
 }
 
-size_t layernorm_bwd_part_floats(int M, int d) { return (size_t)((M + LNP_ROWS - 1) / LNP_ROWS) * 2 * d; }
+size_t layernorm_bwd_part_rows(int M) {
+  const int a = ln_fused_blocks(M), b = (M + LNP_ROWS - 1) / LNP_ROWS;
+  return (size_t)(a > b ? a : b);
+}
+size_t layernorm_bwd_part_floats(int M, int d) { return layernorm_bwd_part_rows(M) * 2 * d; }
 
 int layernorm_bwd(int f32, const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
-                  void* dres, int dres_init, float* part, int* nblk, int M, int d, cudaStream_t st) {
-  *nblk = (M + LNP_ROWS - 1) / LNP_ROWS;
-  return f32 ? ln_bwd_dispatch<float>(dy, x, mean, rstd, g, dres, dres_init, part, M, d, st)
-             : ln_bwd_dispatch<bf16>(dy, x, mean, rstd, g, dres, dres_init, part, M, d, st);
+                  void* dres, int dres_init, float* part, float* part_res, int* nblk, int M, int d,
+                  cudaStream_t st) {
+  return f32 ? ln_bwd_dispatch<float>(dy, x, mean, rstd, g, dres, dres_init, part, part_res, nblk, M, d, st)
+             : ln_bwd_dispatch<bf16>(dy, x, mean, rstd, g, dres, dres_init, part, part_res, nblk, M, d, st);
 }
 
 int reduce_rows_f32(const float* part, int nrows, int n, float* grad, float beta, cudaStream_t st) {
