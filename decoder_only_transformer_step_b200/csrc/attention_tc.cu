@@ -59,8 +59,9 @@ constexpr int SM_P = SM_V + KVS * TILE;
 constexpr int SM_XCHG = SM_P + 4 * TILE;  // [2][2][128] row maxima + [2][128] row sums (floats)
 constexpr int SM_TILES = SM_XCHG + 3 * 2 * 128 * 4;
 // q_full[2], q_empty[2], kv_full[KVS], kv_empty[KVS], s_full[2], s_free[2], p_full[2], o_full[2], drain,
-// xch[2] (row-max exchange), row_sync (per-item exchanges of the softmax warps)
-constexpr int NUM_BARS = 2 * KVS + 16;
+// xch[4 lane quarters][2] (row-max exchange between the two warps of a quarter),
+// row_sync (per-item exchanges of all softmax warps)
+constexpr int NUM_BARS = 2 * KVS + 22;
 constexpr int SMEM_BYTES = SM_TILES + 1024 + NUM_BARS * 8 + 16;
 static_assert(SMEM_BYTES <= 232448, "forward shared memory");
 constexpr uint32_t TMEM_COLS = 512;
@@ -128,8 +129,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto p_full = [&](int s) { return bars + 8u * (8 + 2 * KVS + s); };
   auto o_full = [&](int s) { return bars + 8u * (10 + 2 * KVS + s); };
   const uint32_t drain_bar = bars + 8u * (12 + 2 * KVS);
-  auto xch_bar = [&](int s) { return bars + 8u * (13 + 2 * KVS + s); };
-  const uint32_t row_sync = bars + 8u * (15 + 2 * KVS);
+  auto xch_bar = [&](int q, int s) { return bars + 8u * (13 + 2 * KVS + 2 * q + s); };
+  const uint32_t row_sync = bars + 8u * (21 + 2 * KVS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = (T + BQ - 1) / BQ;
@@ -157,8 +158,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(kv_empty(s), 1);
     }
     mbar_init(drain_bar, 1);
-    mbar_init(xch_bar(0), 256);
-    mbar_init(xch_bar(1), 256);
+    for (int qq = 0; qq < 4; ++qq) {
+      mbar_init(xch_bar(qq, 0), 64);
+      mbar_init(xch_bar(qq, 1), 64);
+    }
     mbar_init(row_sync, 256);
     *abort_flag = 0;
     mbar_fence_init();
@@ -269,8 +272,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // Eight warps: two per TMEM lane quarter, each owning 64 of the 128 key
     // columns of its rows and 32 of the 64 output columns; the two halves of
     // a row exchange partial maxima (per block) and sums (per item) through
-    // shared memory.  The exchanges synchronise the 256 threads on mbarriers
-    // (bounded waits), so an abort in one warp cannot strand the others.
+    // shared memory.  The per-block maxima are exchanged between the two warps
+    // of a lane quarter only (a 64-thread mbarrier per quarter), the per-item
+    // steps across all 256 threads; every wait is bounded, so an abort in one
+    // warp cannot strand the others.
     const int e = warp - 2;
     const int q = warp & 3;  // TMEM lanes [32q, 32q+32)
     const int half = e >> 2;
@@ -327,8 +332,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         float* xp = xchg + sb * 256;
         xp[half * 128 + row] = pmax;
-        mbar_arrive(xch_bar(sb));
-        if (!mbar_wait_bounded(xch_bar(sb), (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        // only the partner warp (same rows, other 64 keys) is waited for
+        mbar_arrive(xch_bar(q, sb));
+        if (!mbar_wait_bounded(xch_bar(q, sb), (g >> 1) & 1, abort_flag, err)) { ok = false; break; }
         const float mx = fmaxf(pmax, xp[(1 - half) * 128 + row]);
         const float alpha = ex2(m - mx);
         m = mx;
