@@ -430,8 +430,8 @@ constexpr int BS_DS = BS_P + 2 * TILE;
 constexpr int BS_MAX_QBLOCKS = 32;  // T <= 4096
 constexpr int BS_LD = BS_DS + 2 * TILE;  // [query block][LSE x128 | D x128] floats
 constexpr int BS_TILES = BS_LD + BS_MAX_QBLOCKS * 256 * 4;
-// kv_full, qdo_full[QS], qdo_empty[QS], st_full, st_free, ps_full, mma2_done, drain
-constexpr int B_NUM_BARS = 2 * QS + 6;
+// kv_full, qdo_full[QS], qdo_empty[QS], st_full, st_free, ps_full, mma2_done, drain, tail
+constexpr int B_NUM_BARS = 2 * QS + 7;
 constexpr int B_SMEM_BYTES = BS_TILES + 1024 + B_NUM_BARS * 8 + 16;
 constexpr int B_NUM_THREADS = 320;
 // dQ is double-buffered (C_DQ + 64 * (t & 1)) so block t's MMAs never wait for
@@ -443,9 +443,9 @@ constexpr uint32_t IDESC_DQ =
 
 __global__ void __launch_bounds__(B_NUM_THREADS, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
-                       const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse,
-                       const float* __restrict__ dvec,
-                       bf16* __restrict__ dqkv, int T, int H, float scale, float scale_log2, int* err) {
+                       const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDQKV,
+                       const float* __restrict__ lse, const float* __restrict__ dvec, int T, int H, float scale,
+                       float scale_log2, int* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -460,6 +460,7 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
   const uint32_t st_full = bars + 8u * (1 + 2 * QS), st_free = bars + 8u * (2 + 2 * QS);
   const uint32_t ps_full = bars + 8u * (3 + 2 * QS);
   const uint32_t mma2_done = bars + 8u * (4 + 2 * QS), drain_bar = bars + 8u * (5 + 2 * QS);
+  const uint32_t tail_bar = bars + 8u * (6 + 2 * QS);  // dK/dV staged by all eight elementwise warps
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nq = (T + BQ - 1) / BQ;
@@ -482,6 +483,7 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
     mbar_init(ps_full, 256);
     mbar_init(mma2_done, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(tail_bar, 256);
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmQKV);
@@ -614,11 +616,20 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
     };
     // LSE (log2 domain) and D of every query block this CTA visits, once:
     // [block][LSE x128 | D x128]; queries past T get LSE = +inf (P = 0).
-    for (int i = tid; i < nblk * 256; i += 256) {
-      const int blk = i >> 8, k = i & 255;
-      const int qq = (kvb + blk) * BQ + (k & 127);
-      const long gi = ((long)b * H + h) * T + qq;
-      sLD[i] = k < 128 ? (qq < T ? lse[gi] * LOG2E_F : INFINITY) : (qq < T ? dvec[gi] : 0.f);
+    // eight blocks' loads in flight at a time: a loop with a runtime trip
+    // count would wait out one global-load latency per block
+    const long bh0 = ((long)b * H + h) * T;
+    for (int blk0 = 0; blk0 < nblk; blk0 += 8) {
+      float vals[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int qq = (kvb + blk0 + u) * BQ + (tid & 127);
+        const bool in = blk0 + u < nblk && qq < T;
+        vals[u] = in ? (tid < 128 ? lse[bh0 + qq] * LOG2E_F : dvec[bh0 + qq]) : (tid < 128 ? INFINITY : 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (blk0 + u < nblk) sLD[(blk0 + u) * 256 + tid] = vals[u];
     }
     asm volatile("bar.sync 1, 256;" ::: "memory");
     for (int t = 0; t < nblk; ++t) {
@@ -698,22 +709,30 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
       tmem_ld_32x32b_x32(tmem + lane_off + C_DK + 32 * half, rk);
       tmem_ld_32x32b_x32(tmem + lane_off + C_DV + 32 * half, rv);
       tmem_ld_wait();
-      if (kv < T) {
-        bf16* dst = dqkv + ((long)b * T + kv) * 3 * d + h * HD + 32 * half;
+      // dK and dV (this thread's row, 32 of the 64 columns) go to the K and V
+      // tiles' shared memory (no MMA reads them any more) in the 128-byte
+      // swizzle, and leave as two TMA stores (rows past T are clipped)
+      const uint32_t krow = base + BS_K + (uint32_t)row * 128u, vrow = base + BS_V + (uint32_t)row * 128u;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int o = 8 * j;
-          *reinterpret_cast<uint4*>(dst + d + o) = make_uint4(
-              pack_bf16x2(__uint_as_float(rk[o]) * scale, __uint_as_float(rk[o + 1]) * scale),
-              pack_bf16x2(__uint_as_float(rk[o + 2]) * scale, __uint_as_float(rk[o + 3]) * scale),
-              pack_bf16x2(__uint_as_float(rk[o + 4]) * scale, __uint_as_float(rk[o + 5]) * scale),
-              pack_bf16x2(__uint_as_float(rk[o + 6]) * scale, __uint_as_float(rk[o + 7]) * scale));
-          *reinterpret_cast<uint4*>(dst + 2 * d + o) = make_uint4(
-              pack_bf16x2(__uint_as_float(rv[o]), __uint_as_float(rv[o + 1])),
-              pack_bf16x2(__uint_as_float(rv[o + 2]), __uint_as_float(rv[o + 3])),
-              pack_bf16x2(__uint_as_float(rv[o + 4]), __uint_as_float(rv[o + 5])),
-              pack_bf16x2(__uint_as_float(rv[o + 6]), __uint_as_float(rv[o + 7])));
-        }
+      for (int c = 0; c < 4; ++c) {
+        const int o = 8 * c;
+        const uint32_t off = 16u * (uint32_t)((4 * half + c) ^ (row & 7));
+        st_shared_v4(krow + off, pack_bf16x2(__uint_as_float(rk[o]) * scale, __uint_as_float(rk[o + 1]) * scale),
+                     pack_bf16x2(__uint_as_float(rk[o + 2]) * scale, __uint_as_float(rk[o + 3]) * scale),
+                     pack_bf16x2(__uint_as_float(rk[o + 4]) * scale, __uint_as_float(rk[o + 5]) * scale),
+                     pack_bf16x2(__uint_as_float(rk[o + 6]) * scale, __uint_as_float(rk[o + 7]) * scale));
+        st_shared_v4(vrow + off, pack_bf16x2(__uint_as_float(rv[o]), __uint_as_float(rv[o + 1])),
+                     pack_bf16x2(__uint_as_float(rv[o + 2]), __uint_as_float(rv[o + 3])),
+                     pack_bf16x2(__uint_as_float(rv[o + 4]), __uint_as_float(rv[o + 5])),
+                     pack_bf16x2(__uint_as_float(rv[o + 6]), __uint_as_float(rv[o + 7])));
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(tail_bar);
+      if (mbar_wait_bounded(tail_bar, 0, abort_flag, err) && warp == 2 && lane == 0) {
+        tma_store_3d(&tmDQKV, base + BS_K, d + h * HD, kv0, b);
+        tma_store_3d(&tmDQKV, base + BS_V, 2 * d + h * HD, kv0, b);
+        bulk_commit();
+        bulk_wait_all();
       }
     }
   }
@@ -738,10 +757,10 @@ int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float
   const uint64_t sq[2] = {3 * d * 2, (uint64_t)T * 3 * d * 2};
   const uint64_t dd[3] = {d, (uint64_t)T, (uint64_t)B};
   const uint64_t sd[2] = {d * 2, (uint64_t)T * d * 2};
-  CUtensorMap tdq;
+  CUtensorMap tdq, tdqkv;
   const uint64_t sdq[2] = {d * 4, (uint64_t)T * d * 4};
   if (!tmap_3d(&tq, qkv, dq, sq) || !tmap_3d(&tdo, dout, dd, sd) ||
-      !tmap_3d(&tdq, dq_acc, dd, sdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 32))
+      !tmap_3d(&tdq, dq_acc, dd, sdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 32) || !tmap_3d(&tdqkv, dqkv, dq, sq))
     return GPT2_ERR_CUDA;
   static bool attr = false;
   if (!attr) {
@@ -749,7 +768,7 @@ int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float
     attr = true;
   }
   dim3 grid((T + BKV - 1) / BKV, B * H);
-  attn_bwd_tc_kernel<<<grid, B_NUM_THREADS, B_SMEM_BYTES, st>>>(tq, tdo, tdq, lse, dvec, (bf16*)dqkv, T, H,
+  attn_bwd_tc_kernel<<<grid, B_NUM_THREADS, B_SMEM_BYTES, st>>>(tq, tdo, tdq, tdqkv, lse, dvec, T, H,
                                                                  0.125f, LOG2E_F / 8.f, nullptr);
   LAUNCH_CHECK();
   return GPT2_OK;
