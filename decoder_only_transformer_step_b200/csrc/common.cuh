@@ -90,6 +90,16 @@ template <bool FAST> DEVI float dgelu_f(float u) {
   return fmaf(0.5f * u * sech2, dt, fmaf(0.5f, th, 0.5f));
 }
 
+// GELU(u) and GELU'(u) from one tanh.
+template <bool FAST> DEVI void gelu_and_grad_f(float u, float& gelu, float& grad) {
+  const float u2 = u * u;
+  const float t = u * fmaf(u2, GELU_K0 * GELU_K1, GELU_K0);
+  const float th = FAST ? tanh_fast(t) : tanhf(t);
+  const float hu = 0.5f * u;
+  gelu = fmaf(hu, th, hu);
+  grad = fmaf(hu * fmaf(-th, th, 1.f), fmaf(u2, 3.f * GELU_K0 * GELU_K1, GELU_K0), fmaf(0.5f, th, 0.5f));
+}
+
 // ------------------------------------------------------------ shared mem --
 
 DEVI uint32_t smem_u32(const void* p) {

@@ -24,13 +24,14 @@ DEVI void epi_one(const EpiArgs& e, float* partial, int split, int M, int N, int
           from_f<T>(v + to_f(((const T*)e.bias)[col]) + to_f(((const T*)e.resid)[idx]));
       break;
     case EPI_BIAS_GELU: {
-      float u = v + to_f(((const T*)e.bias)[col]);
-      ((T*)e.out)[idx] = from_f<T>(u);
-      ((T*)e.out2)[idx] = from_f<T>(gelu_f<FAST>(u));
+      float gl, dg;
+      gelu_and_grad_f<FAST>(v + to_f(((const T*)e.bias)[col]), gl, dg);
+      ((T*)e.out)[idx] = from_f<T>(dg);
+      ((T*)e.out2)[idx] = from_f<T>(gl);
       break;
     }
     case EPI_DGELU:
-      ((T*)e.out)[idx] = from_f<T>(v * dgelu_f<FAST>(to_f(((const T*)e.aux)[idx])));
+      ((T*)e.out)[idx] = from_f<T>(v * to_f(((const T*)e.aux)[idx]));
       break;
     case EPI_F32: {
       float* o = (float*)e.out;
@@ -77,8 +78,8 @@ DEVI void unpack8(const uint4& u, float* f) {
 // Epilogue arithmetic for 32 accumulators of one row, without the store (the
 // tensor-core path stages the result in shared memory and stores it with TMA,
 // which clips rows >= M and columns >= N).  `op` holds the residual
-// (EPI_BIAS_RESID) or GELU' input (EPI_DGELU) chunk, read from its TMA box.  For EPI_BIAS_GELU v
-// becomes u = acc + bias; the caller derives GELU(u) after storing u.
+// (EPI_BIAS_RESID) or saved GELU'(u) (EPI_DGELU) chunk, read from its TMA box.  For EPI_BIAS_GELU
+// v becomes u = acc + bias; the caller derives GELU(u) and GELU'(u) from it.
 DEVI void epi_apply_row32(const EpiArgs& e, int N, int col0, float (&v)[32], const uint4 (&op)[4]) {
   const bool need_bias = e.kind == EPI_BIAS || e.kind == EPI_BIAS_RESID || e.kind == EPI_BIAS_GELU;
   if (need_bias) {
@@ -111,7 +112,7 @@ DEVI void epi_apply_row32(const EpiArgs& e, int N, int col0, float (&v)[32], con
       float t[8];
       unpack8(op[i], t);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[8 * i + j] *= dgelu_f<true>(t[j]);
+      for (int j = 0; j < 8; ++j) v[8 * i + j] *= t[j];
     }
   } else if (e.kind == EPI_STORE || e.kind == EPI_F32) {
 #pragma unroll
@@ -143,6 +144,24 @@ DEVI void load_bf16_box_row(uint32_t box, int lane, uint4 (&u)[4]) {
                  : "=r"(u[j].x), "=r"(u[j].y), "=r"(u[j].z), "=r"(u[j].w)
                  : "r"(rb + 16u * (uint32_t)(j ^ x)));
 }
+// GELU'(u) into `box` and GELU(u) into `box2` (the stage_bf16_row layout),
+// eight columns at a time from one tanh each.
+DEVI void stage_gelu_pair_row(uint32_t box, uint32_t box2, int lane, const float (&u)[32]) {
+  const uint32_t rb = box + (uint32_t)lane * 64u, rb2 = box2 + (uint32_t)lane * 64u;
+  const int x = (lane >> 1) & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float g[8], dg[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) gelu_and_grad_f<true>(u[8 * j + i], g[i], dg[i]);
+    const uint32_t off = 16u * (uint32_t)(j ^ x);
+    st_shared_v4(rb + off, pack_bf16x2(dg[0], dg[1]), pack_bf16x2(dg[2], dg[3]), pack_bf16x2(dg[4], dg[5]),
+                 pack_bf16x2(dg[6], dg[7]));
+    st_shared_v4(rb2 + off, pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]), pack_bf16x2(g[4], g[5]),
+                 pack_bf16x2(g[6], g[7]));
+  }
+}
+
 DEVI void stage_f32_row(uint32_t box, int lane, const float (&v)[32]) {
   const uint32_t rb = box + (uint32_t)lane * 128u;
   const int x = lane & 7;
@@ -181,16 +200,14 @@ DEVI void epi_row32_bf16(const EpiArgs& e, float* partial, int split, int M, int
     case EPI_BIAS_GELU:
       ld_bf16x32((const bf16*)e.bias + col0, t);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] += t[j];
-      st_bf16x32((bf16*)e.out + idx, v);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = gelu_f<true>(v[j]);
-      st_bf16x32((bf16*)e.out2 + idx, v);
+      for (int j = 0; j < 32; ++j) gelu_and_grad_f<true>(v[j] + t[j], t[j], v[j]);
+      st_bf16x32((bf16*)e.out + idx, v);   // GELU'(u)
+      st_bf16x32((bf16*)e.out2 + idx, t);  // GELU(u)
       break;
     case EPI_DGELU:
       ld_bf16x32((const bf16*)e.aux + idx, t);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] *= dgelu_f<true>(t[j]);
+      for (int j = 0; j < 32; ++j) v[j] *= t[j];
       st_bf16x32((bf16*)e.out + idx, v);
       break;
     case EPI_F32: {

@@ -73,7 +73,7 @@ struct TcCfg {
 enum StoreMode : int {
   ST_REG = 0,       // per-thread global stores (general fallback)
   ST_BF16 = 1,      // one bf16 output, TMA store (residual / GELU' operand by TMA load)
-  ST_BF16_X2 = 2,   // two bf16 outputs (u and GELU(u)), two TMA stores
+  ST_BF16_X2 = 2,   // two bf16 outputs (GELU'(u) and GELU(u)), two TMA stores
   ST_F32 = 3,       // fp32 output, TMA store (beta = 0)
   ST_F32_ADD = 4,   // fp32 output, TMA reduce-add (beta = 1)
   ST_F32_PART = 5,  // fp32 split-K partial [split][M][N], 3-D TMA store
@@ -428,13 +428,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         __syncwarp();
         const uint32_t ob = f32_single ? 0u : (uint32_t)(chunk & 1);
-        if (p.store == ST_BF16 || p.store == ST_BF16_X2) {
+        if (BIG_EPI && p.store == ST_BF16_X2) {
+          // v = u: GELU'(u) (saved for the backward) and GELU(u)
+          stage_gelu_pair_row(wbox + 2048u * ob, wbox + 4096u + 2048u * ob, lane, v);
+        } else if (p.store == ST_BF16 || p.store == ST_BF16_X2) {
           stage_bf16_row(wbox + 2048u * ob, lane, v);
-          if (BIG_EPI && p.store == ST_BF16_X2) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = gelu_f<true>(v[j]);
-            stage_bf16_row(wbox + 4096u + 2048u * ob, lane, v);
-          }
         } else {
           stage_f32_row(wbox + 4096u * ob, lane, v);
         }

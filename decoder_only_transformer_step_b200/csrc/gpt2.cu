@@ -92,7 +92,8 @@ struct Carver {
 };
 
 struct LayerActs {
-  void *x_in, *x_mid, *y1, *qkv, *o, *y2, *u, *g;
+  // gp = GELU'(u) of the MLP pre-activation u (all the backward needs of u), g = GELU(u)
+  void *x_in, *x_mid, *y1, *qkv, *o, *y2, *gp, *g;
   float *mean1, *rstd1, *mean2, *rstd2, *lse;
 };
 
@@ -153,7 +154,7 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
     a.y2 = c.take<void>(M * d * act);
     a.mean2 = c.take<float>(M * 4);
     a.rstd2 = c.take<float>(M * 4);
-    a.u = c.take<void>(M * 4 * d * act);
+    a.gp = c.take<void>(M * 4 * d * act);
     a.g = c.take<void>(M * 4 * d * act);
     x_prev = c.take<void>(M * d * act);
   }
@@ -415,7 +416,7 @@ int gpt2_forward_loss(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets
     TRY(run_gemm(c, g, st));
     TRY(layernorm_fwd(f32, a.x_mid, Wp(c, o.layer(l, LN2_G)), Wp(c, o.layer(l, LN2_B)), a.y2, a.mean2, a.rstd2,
                       M, d, st));
-    g = make_gemm(M, 4 * d, d, a.y2, 0, d, Wp(c, o.layer(l, W_FC)), 0, d, EPI_BIAS_GELU, a.u, 4 * d);
+    g = make_gemm(M, 4 * d, d, a.y2, 0, d, Wp(c, o.layer(l, W_FC)), 0, d, EPI_BIAS_GELU, a.gp, 4 * d);
     g.epi.bias = Wp(c, o.layer(l, B_FC));
     g.epi.out2 = a.g;
     TRY(run_gemm(c, g, st));
@@ -466,7 +467,7 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
     LayerActs& a = w.layers[l];
     // MLP projection: x_out = x_mid + g W_mp^T + b_mp
     g = make_gemm(M, 4 * d, d, w.dres, 0, d, Wp(c, o.layer(l, W_MP)), 1, 4 * d, EPI_DGELU, w.du, 4 * d);
-    g.epi.aux = a.u;
+    g.epi.aux = a.gp;
     TRY(run_gemm(c, g, st));
     g = make_gemm(d, 4 * d, M, w.dres, 1, d, a.g, 1, 4 * d, EPI_F32, G + o.layer(l, W_MP), 4 * d);
     g.epi.beta = beta;

@@ -11,8 +11,8 @@ enum EpiKind : int {
   EPI_STORE = 0,    // out(act)  = alpha * acc
   EPI_BIAS,         // out(act)  = acc + bias[n]
   EPI_BIAS_RESID,   // out(act)  = acc + bias[n] + resid[m,n]
-  EPI_BIAS_GELU,    // out(act)  = u = acc + bias[n];  out2(act) = gelu(u)
-  EPI_DGELU,        // out(act)  = acc * gelu'(aux[m,n])
+  EPI_BIAS_GELU,    // u = acc + bias[n]: out(act) = gelu'(u), out2(act) = gelu(u)
+  EPI_DGELU,        // out(act)  = acc * aux[m,n]  (aux = the saved gelu'(u))
   EPI_F32,          // out(fp32) = beta * out + alpha * acc
   EPI_F32_PARTIAL,  // partial[split][m,n] = acc (split-K, internal)
 };
