@@ -65,6 +65,7 @@ template <int HD>
 __global__ void __launch_bounds__(256) attn_fwd_kernel(const bf16* __restrict__ qkv,
                                                        bf16* __restrict__ o, float* __restrict__ lse,
                                                        int T, int H, float scale_log2) {
+  pdl_start();
   constexpr int BQ = 128, BKV = 64, NC = HD / 8;
   constexpr int TILE_KV = BKV * HD * 2;
   extern __shared__ __align__(128) uint8_t sm[];
@@ -225,6 +226,7 @@ template <typename T_>
 __global__ void attn_bwd_prep_kernel(const T_* __restrict__ o, const T_* __restrict__ dout,
                                      float* __restrict__ dvec, float* __restrict__ dq_acc, int B,
                                      int T, int H, int hd) {
+  pdl_start();
   long idx = blockIdx.x * (long)blockDim.x + threadIdx.x;
   if (idx >= (long)B * T * H) return;
   const int h = idx % H;
@@ -246,6 +248,7 @@ template <int HD>
 __global__ void attn_bwd_prep_bf16_kernel(const bf16* __restrict__ o, const bf16* __restrict__ dout,
                                           float* __restrict__ dvec, float* __restrict__ dq_acc, long M, int T,
                                           int H) {
+  pdl_start();
   constexpr int CPH = HD / 8;  // 16-byte chunks per head
   const long m = blockIdx.x * (long)(blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
@@ -278,6 +281,7 @@ __global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ 
                                                        bf16* __restrict__ dqkv,
                                                        float* __restrict__ dq_acc, int T, int H,
                                                        float scale, float scale_log2) {
+  pdl_start();
   constexpr int BKV = 64, BQ = 64, NC = HD / 8;
   constexpr int TILE = 64 * HD * 2;
   extern __shared__ __align__(128) uint8_t sm[];
@@ -480,6 +484,7 @@ __global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ 
 // dqkv[:, 0:d] = bf16(dq_acc)
 __global__ void dq_to_bf16_kernel(const float* __restrict__ dq_acc, bf16* __restrict__ dqkv, long M,
                                   int d) {
+  pdl_start();
   long i = (blockIdx.x * (long)blockDim.x + threadIdx.x) * 4;
   if (i >= M * d) return;
   long m = i / d;
@@ -494,6 +499,7 @@ __global__ void dq_to_bf16_kernel(const float* __restrict__ dq_acc, bf16* __rest
 // One CTA of 64 threads per (query t, batch*head).
 __global__ void attn_fwd_f32_kernel(const float* __restrict__ qkv, float* __restrict__ o,
                                     float* __restrict__ lse, int T, int H, int hd, float scale) {
+  pdl_start();
   extern __shared__ float s[];  // [T] scores, then [64] reduction slots
   float* red = s + T;
   const int t = blockIdx.x, b = blockIdx.y / H, h = blockIdx.y % H;
@@ -548,6 +554,7 @@ __global__ void attn_fwd_f32_kernel(const float* __restrict__ qkv, float* __rest
 __global__ void attn_bwd_q_f32_kernel(const float* __restrict__ qkv, const float* __restrict__ dout,
                                       const float* __restrict__ lse, const float* __restrict__ dvec,
                                       float* __restrict__ dqkv, int T, int H, int hd, float scale) {
+  pdl_start();
   extern __shared__ float s[];
   const int t = blockIdx.x, b = blockIdx.y / H, h = blockIdx.y % H;
   const int d = H * hd;
@@ -581,6 +588,7 @@ __global__ void attn_bwd_q_f32_kernel(const float* __restrict__ qkv, const float
 __global__ void attn_bwd_kv_f32_kernel(const float* __restrict__ qkv, const float* __restrict__ dout,
                                        const float* __restrict__ lse, const float* __restrict__ dvec,
                                        float* __restrict__ dqkv, int T, int H, int hd, float scale) {
+  pdl_start();
   extern __shared__ float s[];  // p[T], ds[T]
   float* ds = s + T;
   const int j = blockIdx.x, b = blockIdx.y / H, h = blockIdx.y % H;
@@ -625,7 +633,7 @@ int launch_fwd(const void* qkv, void* o, float* lse, int B, int T, int H, cudaSt
   }
   dim3 grid((T + 127) / 128, B * H);
   const float scale_log2 = LOG2E_F / sqrtf((float)HD);
-  attn_fwd_kernel<HD><<<grid, 256, smem, st>>>((const bf16*)qkv, (bf16*)o, lse, T, H, scale_log2);
+  CUDA_TRY(launch_k(attn_fwd_kernel<HD>, grid, 256, smem, st, (const bf16*)qkv, (bf16*)o, lse, T, H, scale_log2));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -641,8 +649,8 @@ int launch_bwd(const void* qkv, const void* dout, const float* lse, const float*
   }
   dim3 grid((T + 63) / 64, B * H);
   const float scale = 1.f / sqrtf((float)HD);
-  attn_bwd_kernel<HD><<<grid, 128, smem, st>>>((const bf16*)qkv, (const bf16*)dout, lse, dvec, (bf16*)dqkv,
-                                               dq_acc, T, H, scale, scale * LOG2E_F);
+  CUDA_TRY(launch_k(attn_bwd_kernel<HD>, grid, 128, smem, st,
+      (const bf16*)qkv, (const bf16*)dout, lse, dvec, (bf16*)dqkv, dq_acc, T, H, scale, scale * LOG2E_F));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -682,11 +690,11 @@ int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* 
   if (hd != 64 && hd != 16) return GPT2_ERR_UNSUPPORTED_SHAPE;
   const long M = (long)B * T;
   if (hd == 64)
-    attn_bwd_prep_bf16_kernel<64><<<(unsigned)((M + 7) / 8), 256, 0, st>>>((const bf16*)o, (const bf16*)dout,
-                                                                           dvec, dq_acc, M, T, H);
+    CUDA_TRY(launch_k(attn_bwd_prep_bf16_kernel<64>, (unsigned)((M + 7) / 8), 256, 0, st,
+        (const bf16*)o, (const bf16*)dout, dvec, dq_acc, M, T, H));
   else
-    attn_bwd_prep_bf16_kernel<16><<<(unsigned)((M + 7) / 8), 256, 0, st>>>((const bf16*)o, (const bf16*)dout,
-                                                                           dvec, dq_acc, M, T, H);
+    CUDA_TRY(launch_k(attn_bwd_prep_bf16_kernel<16>, (unsigned)((M + 7) / 8), 256, 0, st,
+        (const bf16*)o, (const bf16*)dout, dvec, dq_acc, M, T, H));
   LAUNCH_CHECK();
   int rc = (hd == 64 && !use_mma_bwd() && T <= 4096)
                ? attn_bwd_tc(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st)
@@ -695,7 +703,7 @@ int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* 
   if (rc) return rc;
   const int d = H * hd;
   long n4 = (M * d) / 4;
-  dq_to_bf16_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dq_acc, (bf16*)dqkv, M, d);
+  CUDA_TRY(launch_k(dq_to_bf16_kernel, (unsigned)((n4 + 255) / 256), 256, 0, st, dq_acc, (bf16*)dqkv, M, d));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -704,7 +712,8 @@ int attn_fwd_f32(const float* qkv, float* o, float* lse, int B, int T, int H, in
   if (B <= 0 || T <= 0) return GPT2_OK;
   size_t smem = (size_t)(T + 64) * sizeof(float);
   if (smem > 48 * 1024) return GPT2_ERR_UNSUPPORTED_SHAPE;
-  attn_fwd_f32_kernel<<<dim3(T, B * H), 64, smem, st>>>(qkv, o, lse, T, H, hd, 1.f / sqrtf((float)hd));
+  CUDA_TRY(launch_k(attn_fwd_f32_kernel, dim3(T, B * H), 64, smem, st,
+      qkv, o, lse, T, H, hd, 1.f / sqrtf((float)hd)));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -715,14 +724,15 @@ int attn_bwd_f32(const float* qkv, const float* o, const float* lse, const float
   size_t smem = (size_t)2 * T * sizeof(float);
   if (smem > 48 * 1024) return GPT2_ERR_UNSUPPORTED_SHAPE;
   long rows = (long)B * T * H;
-  attn_bwd_prep_kernel<float><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(o, dout, dvec, nullptr, B, T,
-                                                                               H, hd);
+  CUDA_TRY(launch_k(attn_bwd_prep_kernel<float>, (unsigned)((rows + 255) / 256), 256, 0, st,
+      o, dout, dvec, nullptr, B, T, H, hd));
   LAUNCH_CHECK();
   const float scale = 1.f / sqrtf((float)hd);
-  attn_bwd_q_f32_kernel<<<dim3(T, B * H), 64, (size_t)T * sizeof(float), st>>>(qkv, dout, lse, dvec, dqkv,
-                                                                              T, H, hd, scale);
+  CUDA_TRY(launch_k(attn_bwd_q_f32_kernel, dim3(T, B * H), 64, (size_t)T * sizeof(float), st,
+      qkv, dout, lse, dvec, dqkv, T, H, hd, scale));
   LAUNCH_CHECK();
-  attn_bwd_kv_f32_kernel<<<dim3(T, B * H), 64, smem, st>>>(qkv, dout, lse, dvec, dqkv, T, H, hd, scale);
+  CUDA_TRY(launch_k(attn_bwd_kv_f32_kernel, dim3(T, B * H), 64, smem, st,
+      qkv, dout, lse, dvec, dqkv, T, H, hd, scale));
   LAUNCH_CHECK();
   return GPT2_OK;
 }

@@ -173,6 +173,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // shared memory and TMEM are set up: wait here for the previous kernel
+  pdl_start();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -494,6 +496,8 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // shared memory and TMEM are set up: wait here for the previous kernel
+  pdl_start();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -768,8 +772,8 @@ int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float
     attr = true;
   }
   dim3 grid((T + BKV - 1) / BKV, B * H);
-  attn_bwd_tc_kernel<<<grid, B_NUM_THREADS, B_SMEM_BYTES, st>>>(tq, tdo, tdq, tdqkv, lse, dvec, T, H,
-                                                                 0.125f, LOG2E_F / 8.f, nullptr);
+  CUDA_TRY(launch_k(attn_bwd_tc_kernel, grid, B_NUM_THREADS, B_SMEM_BYTES, st, tq, tdo, tdq, tdqkv, lse, dvec, T, H,
+                                                                 0.125f, LOG2E_F / 8.f, nullptr));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -790,7 +794,8 @@ int attn_fwd_tc(const void* qkv, void* o, float* lse, int B, int T, int H, cudaS
   }
   const int n_items = ((T + BQ - 1) / BQ) * B * H;
   const int grid = n_items < num_sms() ? n_items : num_sms();
-  attn_fwd_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tq, to, lse, T, H, n_items, LOG2E_F / 8.f, nullptr);
+  CUDA_TRY(launch_k(attn_fwd_tc_kernel, grid, NUM_THREADS, SMEM_BYTES, st,
+      tq, to, lse, T, H, n_items, LOG2E_F / 8.f, nullptr));
   LAUNCH_CHECK();
   return GPT2_OK;
 }

@@ -371,6 +371,37 @@ DEVI void tc_commit_pair(uint32_t bar) {
                : "memory");
 }
 
+// ------------------------------------------------ programmatic dependent launch --
+// Every kernel of the library is launched with programmatic stream
+// serialisation.  A kernel lets the next one launch as soon as all of its own
+// blocks have started (so a dependent grid never takes SM room from blocks of
+// its predecessor that are still waiting to start), and waits for its
+// predecessor to complete, with memory visible, before its first global
+// access.  The next kernel's launch and shared-memory / TMEM set-up then
+// overlap this one's tail.
+DEVI void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+DEVI void pdl_start() {
+  pdl_trigger();
+  pdl_wait();
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ------------------------------------------------------------ host checks --
 
 #define CUDA_TRY(expr)                                   \

@@ -11,6 +11,7 @@ namespace {
 constexpr int TM = 64, TN = 64, TK = 16;
 
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const GemmArgs g) {
+  pdl_start();
   __shared__ float As[TK][TM + 4];
   __shared__ float Bs[TK][TN + 4];
   const float* A = (const float*)g.A;
@@ -65,7 +66,7 @@ int gemm_simt_f32(const GemmArgs& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0) return GPT2_OK;
   if (g.epi.kind == EPI_F32_PARTIAL) return GPT2_ERR_INVALID_ARG;
   dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM);
-  gemm_simt_kernel<<<grid, 256, 0, st>>>(g);
+  CUDA_TRY(launch_k(gemm_simt_kernel, grid, 256, 0, st, g));
   LAUNCH_CHECK();
   return GPT2_OK;
 }

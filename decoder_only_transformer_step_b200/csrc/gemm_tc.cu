@@ -184,6 +184,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if constexpr (PAIR) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // shared memory and TMEM are set up: wait here for the previous kernel
+  pdl_start();
 
   const int units = p.m_tiles * p.n_tiles * p.splits;
 
@@ -498,6 +500,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // out = beta*out + alpha * sum_s part[s]   (fixed order over s)
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, long mn,
                                      float* __restrict__ out, float alpha, float beta) {
+  pdl_start();
   long i = (blockIdx.x * (long)blockDim.x + threadIdx.x) * 4;
   if (i >= mn) return;
   if (i + 4 <= mn) {
@@ -579,17 +582,20 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& t
   static bool attr_set = false;
   static int max_slots = 0;  // co-resident CTAs (single) or clusters (pairs)
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (PAIR) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
   }
   if (!attr_set) {
     CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, PAIR, BIG_EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -778,8 +784,8 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   if (splits > 1) {
     long mn = (long)g.M * g.N;
     long threads = (mn + 3) / 4;
-    splitk_reduce_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-        (const float*)ws, splits, mn, (float*)g.epi.out, g.epi.alpha, g.epi.beta);
+    CUDA_TRY(launch_k(splitk_reduce_kernel, (unsigned)((threads + 255) / 256), 256, 0, st, 
+        (const float*)ws, splits, mn, (float*)g.epi.out, g.epi.alpha, g.epi.beta));
     LAUNCH_CHECK();
   }
   return GPT2_OK;

@@ -62,6 +62,7 @@ template <typename T>
 __global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const T* __restrict__ wte,
                                  const T* __restrict__ wpe, T* __restrict__ x, int M, int Tn, int d,
                                  int vocab_real, int* err) {
+  pdl_start();
   constexpr int VN = Vec<T>::N;
   const int m = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
@@ -94,6 +95,7 @@ template <typename T>
 __global__ void embed_scatter_kernel(const int32_t* __restrict__ tok, const T* __restrict__ dx,
                                      unsigned long long* __restrict__ acc, uint8_t* __restrict__ touched,
                                      int M, int d, int V) {
+  pdl_start();
   long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
   if (i >= (long)M * d) return;
   const int m = (int)(i / d), c = (int)(i % d);
@@ -107,6 +109,7 @@ __global__ void embed_scatter_kernel(const int32_t* __restrict__ tok, const T* _
 
 __global__ void embed_convert_kernel(unsigned long long* __restrict__ acc, uint8_t* __restrict__ touched,
                                      float* __restrict__ dwte, int V, int d) {
+  pdl_start();
   const int v = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
   if (v >= V || !touched[v]) return;
@@ -125,6 +128,7 @@ __global__ void embed_convert_kernel(unsigned long long* __restrict__ acc, uint8
 template <typename T>
 __global__ void wpe_grad_kernel(const T* __restrict__ dx, float* __restrict__ dwpe, int B, int Tn, int d,
                                 int accumulate) {
+  pdl_start();
   long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
   if (i >= (long)Tn * d) return;
   float s = 0.f;
@@ -140,6 +144,7 @@ template <typename T, int NC>
 __global__ void ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ g, const T* __restrict__ b,
                               T* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd, int M,
                               int d) {
+  pdl_start();
   constexpr int VN = Vec<T>::N;
   const int m = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
@@ -198,6 +203,7 @@ __global__ void __launch_bounds__(256) ln_bwd_dx_kernel(const T* __restrict__ dy
                                                         const float* __restrict__ rstd,
                                                         const T* __restrict__ g, T* __restrict__ dres,
                                                         int dres_init, int M, int d) {
+  pdl_start();
   constexpr int VN = Vec<T>::N;
   const int m = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
@@ -251,6 +257,7 @@ __global__ void __launch_bounds__(256) ln_param_colsum_kernel(const T* __restric
                                                               const float* __restrict__ mean,
                                                               const float* __restrict__ rstd, int M, int d,
                                                               float* __restrict__ part) {
+  pdl_start();
   constexpr int VN = Vec<T>::N;
   __shared__ float red[8][2][32 * VN];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -304,6 +311,7 @@ __global__ void __launch_bounds__(32 * LNF_WARPS, LNF_BLOCKS_PER_SM)
     ln_bwd_fused_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __restrict__ mean,
                         const float* __restrict__ rstd, const T* __restrict__ g, T* __restrict__ dres,
                         int dres_init, int M, int d, float* __restrict__ part_ln, float* __restrict__ part_res) {
+  pdl_start();
   constexpr int VN = Vec<T>::N;
   extern __shared__ float red[];  // [LNF_WARPS][3][d]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -420,6 +428,7 @@ __global__ void __launch_bounds__(32 * LNF_WARPS, LNF_BLOCKS_PER_SM)
 // column reduced in a fixed order.
 __global__ void reduce_rows_kernel(const float* __restrict__ part, int nrows, int n, float* __restrict__ grad,
                                    float beta) {
+  pdl_start();
   __shared__ float sm[8][33];
   const int cx = threadIdx.x & 31, ry = threadIdx.x >> 5;
   const int j = blockIdx.x * 32 + cx;
@@ -445,6 +454,7 @@ struct ReduceBatchArgs {
 };
 
 __global__ void reduce_rows_batch_kernel(const __grid_constant__ ReduceBatchArgs a) {
+  pdl_start();
   __shared__ float sm[8][33];
   int jb = 0;
   while (jb + 1 < a.njobs && a.start[jb + 1] <= (int)blockIdx.x) ++jb;
@@ -471,6 +481,7 @@ constexpr int CS_ROWS = 128;
 template <typename T>
 __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ x, int M, int N,
                                                      float* __restrict__ part) {
+  pdl_start();
   constexpr int VN = Vec<T>::N;
   __shared__ float red[8][32 * VN];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -508,6 +519,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const int32_t* __restrict__ tgt,
                                                  float* __restrict__ loss_rows, int V, int vocab_real,
                                                  int* err) {
+  pdl_start();
   constexpr int VN = Vec<T>::N;
   constexpr int U = 4;  // 16-byte vectors in flight per thread and trip
   constexpr float L2E = 1.4426950408889634f;
@@ -597,6 +609,7 @@ __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const i
 
 // loss = mean(loss_rows), fixed-order tree; flags a non-finite result.
 __global__ void loss_mean_kernel(const float* __restrict__ rows, int M, float* __restrict__ loss, int* err) {
+  pdl_start();
   __shared__ float sm[1024];
   float s = 0.f;
   for (int i = threadIdx.x; i < M; i += 1024) s += rows[i];
@@ -659,6 +672,7 @@ DEVI int tensor_kind(long i, const LayoutDims& L, int* one) {
 __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
                              float* __restrict__ v, uint16_t* __restrict__ shadow, long n4, LayoutDims L,
                              AdamArgs a) {
+  pdl_start();
   for (long i4 = blockIdx.x * (long)blockDim.x + threadIdx.x; i4 < n4; i4 += (long)gridDim.x * blockDim.x) {
     const long i = i4 * 4;
     int one;
@@ -707,6 +721,7 @@ DEVI void philox4x32_10(uint32_t (&c)[4], uint32_t k0, uint32_t k1) {
 }
 
 __global__ void init_kernel(float* __restrict__ p, long n, LayoutDims L, uint64_t seed) {
+  pdl_start();
   const float std_w = 0.02f;
   const float std_proj = 0.02f / sqrtf(2.f * (float)L.L);
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
@@ -729,6 +744,7 @@ __global__ void init_kernel(float* __restrict__ p, long n, LayoutDims L, uint64_
 }
 
 __global__ void cast_shadow_kernel(const float* __restrict__ p, uint16_t* __restrict__ s, long n4) {
+  pdl_start();
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
     float4 v = reinterpret_cast<const float4*>(p)[i];
     reinterpret_cast<uint2*>(s)[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
@@ -742,27 +758,30 @@ int grid_for(long n, int threads) {
 }
 
 template <typename T, int NC>
-void ln_fwd_launch(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int M,
+int ln_fwd_launch(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int M,
                    int d, cudaStream_t st) {
-  ln_fwd_kernel<T, NC><<<(M + 7) / 8, 256, 0, st>>>((const T*)x, (const T*)g, (const T*)b, (T*)y, mean, rstd,
-                                                    M, d);
+  CUDA_TRY(launch_k(ln_fwd_kernel<T, NC>, (M + 7) / 8, 256, 0, st,
+      (const T*)x, (const T*)g, (const T*)b, (T*)y, mean, rstd, M, d));
+  return GPT2_OK;
 }
 
 template <typename T>
 int ln_fwd_dispatch(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int M,
                     int d, cudaStream_t st) {
   const int nc = (d / Vec<T>::N + 31) / 32;
+  int rc = GPT2_OK;
   switch (nc) {
-    case 1: ln_fwd_launch<T, 1>(x, g, b, y, mean, rstd, M, d, st); break;
-    case 2: ln_fwd_launch<T, 2>(x, g, b, y, mean, rstd, M, d, st); break;
-    case 3: ln_fwd_launch<T, 3>(x, g, b, y, mean, rstd, M, d, st); break;
-    case 4: ln_fwd_launch<T, 4>(x, g, b, y, mean, rstd, M, d, st); break;
-    case 5: ln_fwd_launch<T, 5>(x, g, b, y, mean, rstd, M, d, st); break;
-    case 6: ln_fwd_launch<T, 6>(x, g, b, y, mean, rstd, M, d, st); break;
-    case 7: ln_fwd_launch<T, 7>(x, g, b, y, mean, rstd, M, d, st); break;
-    case 8: ln_fwd_launch<T, 8>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 1: rc = ln_fwd_launch<T, 1>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 2: rc = ln_fwd_launch<T, 2>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 3: rc = ln_fwd_launch<T, 3>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 4: rc = ln_fwd_launch<T, 4>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 5: rc = ln_fwd_launch<T, 5>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 6: rc = ln_fwd_launch<T, 6>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 7: rc = ln_fwd_launch<T, 7>(x, g, b, y, mean, rstd, M, d, st); break;
+    case 8: rc = ln_fwd_launch<T, 8>(x, g, b, y, mean, rstd, M, d, st); break;
     default: return GPT2_ERR_UNSUPPORTED_SHAPE;
   }
+  if (rc) return rc;
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -778,7 +797,7 @@ int ln_fused_blocks(int M) {
 // in bf16 or fp32); wider rows take the row kernel plus the column-sum
 // kernels.
 template <typename T, int NC>
-void ln_bwd_launch(const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
+int ln_bwd_launch(const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
                    void* dres, int init, float* part, float* part_res, int* nblk, int M, int d, cudaStream_t st) {
   constexpr int VN = Vec<T>::N;
   if constexpr (NC * VN <= 24) {
@@ -786,44 +805,47 @@ void ln_bwd_launch(const void* dy, const void* x, const float* mean, const float
     *nblk = blocks;
     if (part_res) {
       const size_t smem = (size_t)LNF_WARPS * 3 * d * sizeof(float);
-      ln_bwd_fused_kernel<T, NC, true><<<blocks, 32 * LNF_WARPS, smem, st>>>(
-          (const T*)dy, (const T*)x, mean, rstd, (const T*)g, (T*)dres, init, M, d, part, part_res);
+      CUDA_TRY(launch_k(ln_bwd_fused_kernel<T, NC, true>, blocks, 32 * LNF_WARPS, smem, st, 
+          (const T*)dy, (const T*)x, mean, rstd, (const T*)g, (T*)dres, init, M, d, part, part_res));
     } else {
       const size_t smem = (size_t)LNF_WARPS * 2 * d * sizeof(float);
-      ln_bwd_fused_kernel<T, NC, false><<<blocks, 32 * LNF_WARPS, smem, st>>>(
-          (const T*)dy, (const T*)x, mean, rstd, (const T*)g, (T*)dres, init, M, d, part, nullptr);
+      CUDA_TRY(launch_k(ln_bwd_fused_kernel<T, NC, false>, blocks, 32 * LNF_WARPS, smem, st, 
+          (const T*)dy, (const T*)x, mean, rstd, (const T*)g, (T*)dres, init, M, d, part, nullptr));
     }
-    return;
+    return GPT2_OK;
   }
   *nblk = (M + LNP_ROWS - 1) / LNP_ROWS;
-  ln_bwd_dx_kernel<T, NC><<<(M + 7) / 8, 256, 0, st>>>((const T*)dy, (const T*)x, mean, rstd, (const T*)g,
-                                                       (T*)dres, init, M, d);
+  CUDA_TRY(launch_k(ln_bwd_dx_kernel<T, NC>, (M + 7) / 8, 256, 0, st,
+      (const T*)dy, (const T*)x, mean, rstd, (const T*)g, (T*)dres, init, M, d));
   gpt2_count_launch();
   dim3 grid((d + 32 * VN - 1) / (32 * VN), (M + LNP_ROWS - 1) / LNP_ROWS);
-  ln_param_colsum_kernel<T><<<grid, 256, 0, st>>>((const T*)dy, (const T*)x, mean, rstd, M, d, part);
+  CUDA_TRY(launch_k(ln_param_colsum_kernel<T>, grid, 256, 0, st, (const T*)dy, (const T*)x, mean, rstd, M, d, part));
   if (part_res) {
     gpt2_count_launch();
     // column sums of the new dres in the same row blocks (CS_ROWS == LNP_ROWS)
     dim3 g2((d + 32 * VN - 1) / (32 * VN), (M + CS_ROWS - 1) / CS_ROWS);
-    colsum_kernel<T><<<g2, 256, 0, st>>>((const T*)dres, M, d, part_res);
+    CUDA_TRY(launch_k(colsum_kernel<T>, g2, 256, 0, st, (const T*)dres, M, d, part_res));
   }
+  return GPT2_OK;
 }
 
 template <typename T>
 int ln_bwd_dispatch(const void* dy, const void* x, const float* mean, const float* rstd, const void* g,
                     void* dres, int init, float* part, float* part_res, int* nblk, int M, int d, cudaStream_t st) {
   const int nc = (d / Vec<T>::N + 31) / 32;
+  int rc = GPT2_OK;
   switch (nc) {
-    case 1: ln_bwd_launch<T, 1>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
-    case 2: ln_bwd_launch<T, 2>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
-    case 3: ln_bwd_launch<T, 3>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
-    case 4: ln_bwd_launch<T, 4>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
-    case 5: ln_bwd_launch<T, 5>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
-    case 6: ln_bwd_launch<T, 6>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
-    case 7: ln_bwd_launch<T, 7>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
-    case 8: ln_bwd_launch<T, 8>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 1: rc = ln_bwd_launch<T, 1>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 2: rc = ln_bwd_launch<T, 2>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 3: rc = ln_bwd_launch<T, 3>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 4: rc = ln_bwd_launch<T, 4>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 5: rc = ln_bwd_launch<T, 5>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 6: rc = ln_bwd_launch<T, 6>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 7: rc = ln_bwd_launch<T, 7>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
+    case 8: rc = ln_bwd_launch<T, 8>(dy, x, mean, rstd, g, dres, init, part, part_res, nblk, M, d, st); break;
     default: return GPT2_ERR_UNSUPPORTED_SHAPE;
   }
+  if (rc) return rc;
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -836,11 +858,11 @@ int embed_fwd(int f32, const int32_t* tok, const void* wte, const void* wpe, voi
               int vocab_real, int* err, cudaStream_t st) {
   const int blocks = (M + 7) / 8;
   if (f32)
-    embed_fwd_kernel<float><<<blocks, 256, 0, st>>>(tok, (const float*)wte, (const float*)wpe, (float*)x, M, T,
-                                                    d, vocab_real, err);
+    CUDA_TRY(launch_k(embed_fwd_kernel<float>, blocks, 256, 0, st,
+        tok, (const float*)wte, (const float*)wpe, (float*)x, M, T, d, vocab_real, err));
   else
-    embed_fwd_kernel<bf16><<<blocks, 256, 0, st>>>(tok, (const bf16*)wte, (const bf16*)wpe, (bf16*)x, M, T, d,
-                                                   vocab_real, err);
+    CUDA_TRY(launch_k(embed_fwd_kernel<bf16>, blocks, 256, 0, st,
+        tok, (const bf16*)wte, (const bf16*)wpe, (bf16*)x, M, T, d, vocab_real, err));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -865,7 +887,7 @@ int layernorm_bwd(int f32, const void* dy, const void* x, const float* mean, con
 }
 
 int reduce_rows_f32(const float* part, int nrows, int n, float* grad, float beta, cudaStream_t st) {
-  reduce_rows_kernel<<<(n + 31) / 32, 256, 0, st>>>(part, nrows, n, grad, beta);
+  CUDA_TRY(launch_k(reduce_rows_kernel, (n + 31) / 32, 256, 0, st, part, nrows, n, grad, beta));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -883,7 +905,7 @@ int reduce_rows_batch(const ReduceJob* jobs, int njobs, float beta, cudaStream_t
     }
     a.start[a.njobs] = blocks;
     if (blocks == 0) continue;
-    reduce_rows_batch_kernel<<<blocks, 256, 0, st>>>(a);
+    CUDA_TRY(launch_k(reduce_rows_batch_kernel, blocks, 256, 0, st, a));
     LAUNCH_CHECK();
   }
   return GPT2_OK;
@@ -896,9 +918,9 @@ int colsum_partial(int f32, const void* x, int M, int N, float* part, int* nblk,
   const int vn = f32 ? 4 : 8;
   dim3 grid((N + 32 * vn - 1) / (32 * vn), *nblk);
   if (f32)
-    colsum_kernel<float><<<grid, 256, 0, st>>>((const float*)x, M, N, part);
+    CUDA_TRY(launch_k(colsum_kernel<float>, grid, 256, 0, st, (const float*)x, M, N, part));
   else
-    colsum_kernel<bf16><<<grid, 256, 0, st>>>((const bf16*)x, M, N, part);
+    CUDA_TRY(launch_k(colsum_kernel<bf16>, grid, 256, 0, st, (const bf16*)x, M, N, part));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -906,15 +928,15 @@ int colsum_partial(int f32, const void* x, int M, int N, float* part, int* nblk,
 int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, int V, int vocab_real, int* err,
            cudaStream_t st) {
   if (f32)
-    ce_kernel<float><<<M, 256, 0, st>>>((float*)logits, tgt, loss_rows, V, vocab_real, err);
+    CUDA_TRY(launch_k(ce_kernel<float>, M, 256, 0, st, (float*)logits, tgt, loss_rows, V, vocab_real, err));
   else
-    ce_kernel<bf16><<<M, 256, 0, st>>>((bf16*)logits, tgt, loss_rows, V, vocab_real, err);
+    CUDA_TRY(launch_k(ce_kernel<bf16>, M, 256, 0, st, (bf16*)logits, tgt, loss_rows, V, vocab_real, err));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
 
 int loss_mean(const float* loss_rows, int M, float* loss, int* err, cudaStream_t st) {
-  loss_mean_kernel<<<1, 1024, 0, st>>>(loss_rows, M, loss, err);
+  CUDA_TRY(launch_k(loss_mean_kernel, 1, 1024, 0, st, loss_rows, M, loss, err));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -924,22 +946,22 @@ int embed_bwd(int f32, const int32_t* tok, const void* dx, float* dwte, float* d
   const long n = (long)M * d;
   unsigned long long* a = reinterpret_cast<unsigned long long*>(acc);
   if (f32)
-    embed_scatter_kernel<float><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(tok, (const float*)dx, a, touched,
-                                                                             M, d, V);
+    CUDA_TRY(launch_k(embed_scatter_kernel<float>, (unsigned)((n + 255) / 256), 256, 0, st,
+        tok, (const float*)dx, a, touched, M, d, V));
   else
-    embed_scatter_kernel<bf16><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(tok, (const bf16*)dx, a, touched, M,
-                                                                            d, V);
+    CUDA_TRY(launch_k(embed_scatter_kernel<bf16>, (unsigned)((n + 255) / 256), 256, 0, st,
+        tok, (const bf16*)dx, a, touched, M, d, V));
   LAUNCH_CHECK();
-  embed_convert_kernel<<<(V + 7) / 8, 256, 0, st>>>(a, touched, dwte, V, d);
+  CUDA_TRY(launch_k(embed_convert_kernel, (V + 7) / 8, 256, 0, st, a, touched, dwte, V, d));
   LAUNCH_CHECK();
   const long tn = (long)T * d;
   const int B = M / T;
   if (f32)
-    wpe_grad_kernel<float><<<(unsigned)((tn + 255) / 256), 256, 0, st>>>((const float*)dx, dwpe, B, T, d,
-                                                                         wpe_accumulate);
+    CUDA_TRY(launch_k(wpe_grad_kernel<float>, (unsigned)((tn + 255) / 256), 256, 0, st,
+        (const float*)dx, dwpe, B, T, d, wpe_accumulate));
   else
-    wpe_grad_kernel<bf16><<<(unsigned)((tn + 255) / 256), 256, 0, st>>>((const bf16*)dx, dwpe, B, T, d,
-                                                                        wpe_accumulate);
+    CUDA_TRY(launch_k(wpe_grad_kernel<bf16>, (unsigned)((tn + 255) / 256), 256, 0, st, (const bf16*)dx, dwpe, B, T, d,
+                                                                        wpe_accumulate));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
@@ -947,20 +969,20 @@ int embed_bwd(int f32, const int32_t* tok, const void* dx, float* dwte, float* d
 int adamw(float* p, const float* g, float* m, float* v, uint16_t* shadow, size_t n, const LayoutDims& ld,
           const AdamArgs& a, cudaStream_t st) {
   const long n4 = (long)(n / 4);
-  adamw_kernel<<<grid_for(n4, 256), 256, 0, st>>>(p, g, m, v, shadow, n4, ld, a);
+  CUDA_TRY(launch_k(adamw_kernel, grid_for(n4, 256), 256, 0, st, p, g, m, v, shadow, n4, ld, a));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
 
 int init_params(float* p, size_t n, const LayoutDims& ld, uint64_t seed, cudaStream_t st) {
-  init_kernel<<<grid_for((long)n, 256), 256, 0, st>>>(p, (long)n, ld, seed);
+  CUDA_TRY(launch_k(init_kernel, grid_for((long)n, 256), 256, 0, st, p, (long)n, ld, seed));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
 
 int cast_shadow(const float* p, uint16_t* shadow, size_t n, cudaStream_t st) {
   const long n4 = (long)(n / 4);
-  cast_shadow_kernel<<<grid_for(n4, 256), 256, 0, st>>>(p, shadow, n4);
+  CUDA_TRY(launch_k(cast_shadow_kernel, grid_for(n4, 256), 256, 0, st, p, shadow, n4));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
