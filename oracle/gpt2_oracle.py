@@ -31,7 +31,9 @@ the task states it.  Where the pages are silent this oracle takes the plainest
 GPT-2 reading: tanh-form GELU, LayerNorm eps 1e-5 with biased variance,
 biases on every linear layer except the tied head, no dropout, softmax scale
 1/sqrt(head_dim), loss averaged over all B*T positions, weight decay on 2-D
-tensors only, AdamW with bias correction and eps 1e-8, no gradient clipping.
+tensors only, AdamW with bias correction and eps 1e-8, no gradient clipping
+(an optional global-norm clip is provided for the training loop around the
+step; it is off unless asked for).
 
 Pins (tests/test_oracle_*.py): central finite differences in fp64 for every
 parameter tensor, an independent PyTorch autograd witness built from library
@@ -327,15 +329,31 @@ def backward(params: dict, cfg: Config, cache: dict, grad_scale: float = 1.0, co
     return grads
 
 
+def clip_grad_norm(grads: dict, max_norm: float):
+    """Global-norm gradient clipping.  The pages do not use it; this is the
+    common form: total = sqrt(sum over every tensor of sum g^2), and when
+    max_norm / (total + 1e-6) < 1 every gradient is multiplied by that ratio.
+    Returns (clipped grads, total)."""
+    total = float(np.sqrt(sum(float(np.sum(np.square(g, dtype=np.float64))) for g in grads.values())))
+    coef = max_norm / (total + 1e-6)
+    if coef >= 1.0:
+        return {n: g.copy() for n, g in grads.items()}, total
+    return {n: g * coef for n, g in grads.items()}, total
+
+
 def adamw_step(params: dict, grads: dict, m: dict, v: dict, step: int, cfg: Config,
-               lr=6e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1):
+               lr=6e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, max_norm=0.0):
     """Decoupled-weight-decay Adam (AdamW), step counter starting at 1.
 
     p <- p * (1 - lr*wd)             (2-D tensors only)
     m <- b1 m + (1-b1) g ;  v <- b2 v + (1-b2) g^2
     p <- p - lr * m_hat / (sqrt(v_hat) + eps),  m_hat = m/(1-b1^t), v_hat = v/(1-b2^t)
-    Returns new (params, m, v) dicts; the inputs are left untouched.
+    With max_norm > 0 the gradients are first clipped to that global norm
+    (clip_grad_norm).  Returns new (params, m, v) dicts; the inputs are left
+    untouched.
     """
+    if max_norm > 0.0:
+        grads, _ = clip_grad_norm(grads, max_norm)
     decay = decay_mask(cfg)
     bc1 = 1.0 - beta1 ** step
     bc2 = 1.0 - beta2 ** step

@@ -230,3 +230,60 @@ def test_zipf_inputs():
     p0 = inputs.zipf_cdf(50257)[0]
     assert abs(p0 - 0.139) < 0.001
     assert abs((tok == 0).mean() - p0) < 0.01
+
+
+# ------------------------------------ optimizer-side steps around the path ---
+
+def test_clip_grad_norm_matches_torch():
+    """The oracle's global-norm clip against torch.nn.utils.clip_grad_norm_
+    (a library routine) on the same tensors, clipping and not clipping."""
+    import torch
+    rng = np.random.default_rng(3)
+    grads = {"a": rng.standard_normal((7, 5)), "b": rng.standard_normal(11), "c": rng.standard_normal((2, 3, 4))}
+    for max_norm in (0.5, 1e6):
+        ts = [torch.from_numpy(g.copy()) for g in grads.values()]
+        for t in ts:
+            t.grad = t.clone()
+        total_t = torch.nn.utils.clip_grad_norm_(ts, max_norm)
+        clipped, total = G.clip_grad_norm(grads, max_norm)
+        assert abs(total - float(total_t)) <= 1e-12 * total
+        for t, (n, g) in zip(ts, clipped.items()):
+            np.testing.assert_allclose(g, t.grad.numpy(), rtol=1e-14, atol=0)
+
+
+def test_clipped_adamw_equals_adamw_on_scaled_grads():
+    """Clipping only rescales the gradients: AdamW with max_norm equals AdamW
+    on gradients multiplied by max_norm / (norm + 1e-6) by hand."""
+    cfg = TINY
+    params = params_for(cfg, 5)
+    rng = np.random.default_rng(6)
+    grads = {n: rng.standard_normal(s) for n, s in param_shapes(cfg)}
+    zeros = {n: np.zeros(s) for n, s in param_shapes(cfg)}
+    norm = math.sqrt(sum(float(np.sum(g * g)) for g in grads.values()))
+    coef = 0.25 / (norm + 1e-6)
+    assert coef < 1.0
+    P1, M1, V1 = adamw_step(params, grads, zeros, zeros, 1, cfg, max_norm=0.25)
+    P2, M2, V2 = adamw_step(params, {n: g * coef for n, g in grads.items()}, zeros, zeros, 1, cfg)
+    for n, _ in param_shapes(cfg):
+        np.testing.assert_allclose(M1[n], M2[n], rtol=1e-15, atol=0)
+        np.testing.assert_allclose(P1[n], P2[n], rtol=1e-15, atol=0)
+
+
+def test_lr_schedule_closed_forms():
+    from decoder_only_transformer_step_b200.schedule import lr_at, steps_for_budget
+    max_lr, min_lr = 6e-4, 6e-5
+    # the page's step: 16 x 1024 tokens with 32-fold accumulation
+    assert steps_for_budget(16 * 1024 * 32 * 1000, 16, 1024, 32) == 1000
+    total, warm = 1000, 100
+    assert lr_at(0, max_lr, total, warm, min_lr) == pytest.approx(max_lr / warm)
+    assert lr_at(warm - 1, max_lr, total, warm, min_lr) == pytest.approx(max_lr)
+    assert lr_at(warm, max_lr, total, warm, min_lr) == pytest.approx(max_lr)        # cos 0
+    mid = warm + (total - warm) // 2
+    assert lr_at(mid, max_lr, total, warm, min_lr) == pytest.approx((max_lr + min_lr) / 2)  # cos(pi/2)
+    assert lr_at(total, max_lr, total, warm, min_lr) == min_lr
+    # plain cosine (no warm-up) decays to zero at the budget and is monotone
+    lrs = [lr_at(s, max_lr, total) for s in range(total + 1)]
+    assert lrs[0] == pytest.approx(max_lr) and lrs[-1] == 0.0
+    assert all(a >= b for a, b in zip(lrs, lrs[1:]))
+    with pytest.raises(ValueError):
+        lr_at(0, max_lr, 10, 10)
