@@ -46,7 +46,7 @@ class gpt2_buffers(ctypes.Structure):
 EXPORTS = [
     "gpt2_param_count", "gpt2_workspace_bytes", "gpt2_tensor_info", "gpt2_create", "gpt2_destroy",
     "gpt2_init_params", "gpt2_refresh_shadow", "gpt2_forward_loss", "gpt2_backward",
-    "gpt2_adamw_step", "gpt2_zero_grad", "gpt2_get_status", "gpt2_step_host", "gpt2_strerror",
+    "gpt2_adamw_step", "gpt2_adamw_step_clip", "gpt2_grad_norm", "gpt2_zero_grad", "gpt2_get_status", "gpt2_step_host", "gpt2_strerror",
     "gpt2_kernel_launches",
     "gpt2_op_gemm_bf16", "gpt2_op_attention_fwd_bf16", "gpt2_op_attention_bwd_bf16",
     "gpt2_op_attention_bwd_bf16_noalloc",
@@ -77,6 +77,8 @@ def _lib():
         "gpt2_forward_loss": (I, [P, P, P, I, P, P]),
         "gpt2_backward": (I, [P, F, I, P]),
         "gpt2_adamw_step": (I, [P, F, F, F, F, F, I, P]),
+        "gpt2_adamw_step_clip": (I, [P, F, F, F, F, F, I, F, P]),
+        "gpt2_grad_norm": (I, [P, P, P]),
         "gpt2_zero_grad": (I, [P, P]),
         "gpt2_get_status": (I, [P, P]),
         "gpt2_step_host": (I, [P, P, P, I, P, F, F, F, F, F, I, P]),
@@ -178,6 +180,15 @@ def gpt2_backward(ctx, grad_scale: float = 1.0, accumulate: int = 0, stream=None
 def gpt2_adamw_step(ctx, lr, beta1, beta2, eps, weight_decay, step, stream=None):
     _check(_lib().gpt2_adamw_step(ctx, lr, beta1, beta2, eps, weight_decay, step, _stream(stream)),
            "gpt2_adamw_step")
+
+
+def gpt2_adamw_step_clip(ctx, lr, beta1, beta2, eps, weight_decay, step, max_norm, stream=None):
+    _check(_lib().gpt2_adamw_step_clip(ctx, lr, beta1, beta2, eps, weight_decay, step, max_norm,
+                                       _stream(stream)), "gpt2_adamw_step_clip")
+
+
+def gpt2_grad_norm(ctx, norm_dev=None, stream=None):
+    _check(_lib().gpt2_grad_norm(ctx, _ptr(norm_dev), _stream(stream)), "gpt2_grad_norm")
 
 
 def gpt2_zero_grad(ctx, stream=None):
@@ -307,8 +318,20 @@ class GPT2:
     def backward(self, grad_scale=1.0, accumulate=0):
         gpt2_backward(self.ctx, grad_scale, accumulate)
 
-    def adamw_step(self, step, lr=6e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1):
-        gpt2_adamw_step(self.ctx, lr, beta1, beta2, eps, weight_decay, step)
+    def adamw_step(self, step, lr=6e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, max_norm=0.0):
+        """AdamW over the flat buffer; max_norm > 0 clips the gradient to that
+        global norm first (on the device)."""
+        if max_norm > 0.0:
+            gpt2_adamw_step_clip(self.ctx, lr, beta1, beta2, eps, weight_decay, step, max_norm)
+        else:
+            gpt2_adamw_step(self.ctx, lr, beta1, beta2, eps, weight_decay, step)
+
+    def grad_norm(self):
+        """Global L2 norm of the gradient buffer as a device fp32 scalar tensor."""
+        import torch
+        out = torch.empty(1, dtype=torch.float32, device=self.grad.device)
+        gpt2_grad_norm(self.ctx, out)
+        return out
 
     def zero_grad(self):
         gpt2_zero_grad(self.ctx)

@@ -106,6 +106,7 @@ struct Work {
   float *meanf, *rstdf, *loss_rows;
   void *dres, *dy, *du, *dqkv, *dout;
   float *dq_acc, *dvec;
+  float *norm_part, *gnorm;  // global gradient norm: block partials and the result
   // block partials of every bias / LayerNorm parameter gradient of one
   // backward, each in its own slot, all reduced by one launch at its end
   float* part_arena;
@@ -179,6 +180,8 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
                                    colsum_part_floats((int)M, (int)(3 * d))) +
                    ln_rows * 3 * d;
   w->part_arena = c.take<float>(w->part_floats * 4);
+  w->norm_part = c.take<float>((size_t)GRAD_NORM_PARTS * 4);
+  w->gnorm = c.take<float>(4);
   w->part_used = 0;
   w->split_bytes = split_ws_need(s, M);
   w->split_ws = c.take<void>(w->split_bytes);
@@ -522,7 +525,28 @@ int gpt2_adamw_step(gpt2_ctx* c, float lr, float beta1, float beta2, float eps, 
   a.bc2 = (float)(1.0 - pow((double)beta2, (double)step));
   LayoutDims ld{c->s.V, c->s.T, c->s.d, c->s.L};
   return adamw(c->buf.master, c->buf.grad, c->buf.m, c->buf.v, c->s.mode ? nullptr : c->buf.shadow,
-               c->off.total(), ld, a, S(stream));
+               c->off.total(), ld, a, nullptr, 0.f, S(stream));
+}
+
+int gpt2_grad_norm(gpt2_ctx* c, float* norm_dev, void* stream) {
+  if (!c) return GPT2_ERR_INVALID_ARG;
+  if (norm_dev && ((uintptr_t)norm_dev & 3)) return GPT2_ERR_INVALID_ARG;
+  return grad_norm(c->buf.grad, c->off.total(), c->w.norm_part, norm_dev ? norm_dev : c->w.gnorm, S(stream));
+}
+
+int gpt2_adamw_step_clip(gpt2_ctx* c, float lr, float beta1, float beta2, float eps, float weight_decay, int step,
+                         float max_norm, void* stream) {
+  if (!c || step < 1 || !(max_norm >= 0.f)) return GPT2_ERR_INVALID_ARG;
+  if (max_norm == 0.f) return gpt2_adamw_step(c, lr, beta1, beta2, eps, weight_decay, step, stream);
+  int rc = grad_norm(c->buf.grad, c->off.total(), c->w.norm_part, c->w.gnorm, S(stream));
+  if (rc) return rc;
+  AdamArgs a;
+  a.lr = lr; a.beta1 = beta1; a.beta2 = beta2; a.eps = eps; a.wd = weight_decay;
+  a.bc1 = (float)(1.0 - pow((double)beta1, (double)step));
+  a.bc2 = (float)(1.0 - pow((double)beta2, (double)step));
+  LayoutDims ld{c->s.V, c->s.T, c->s.d, c->s.L};
+  return adamw(c->buf.master, c->buf.grad, c->buf.m, c->buf.v, c->s.mode ? nullptr : c->buf.shadow,
+               c->off.total(), ld, a, c->w.gnorm, max_norm, S(stream));
 }
 
 int gpt2_get_status(gpt2_ctx* c, void* stream) {

@@ -111,8 +111,12 @@ struct AdamArgs {
 struct LayoutDims {
   long V, T, d, L;
 };
+// gnorm (device scalar, may be NULL): clip the gradient to global norm max_norm.
 int adamw(float* p, const float* g, float* m, float* v, uint16_t* shadow, size_t n,
-          const LayoutDims& ld, const AdamArgs& a, cudaStream_t st);
+          const LayoutDims& ld, const AdamArgs& a, const float* gnorm, float max_norm, cudaStream_t st);
+// ||g||_2 of n floats (n % 4 == 0) into *norm; part holds GRAD_NORM_PARTS floats.
+constexpr int GRAD_NORM_PARTS = 592;
+int grad_norm(const float* g, size_t n, float* part, float* norm, cudaStream_t st);
 int init_params(float* p, size_t n, const LayoutDims& ld, uint64_t seed, cudaStream_t st);
 int cast_shadow(const float* p, uint16_t* shadow, size_t n, cudaStream_t st);
 int fill_zero(void* p, size_t bytes, cudaStream_t st);

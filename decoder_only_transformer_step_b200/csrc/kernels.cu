@@ -669,16 +669,61 @@ DEVI int tensor_kind(long i, const LayoutDims& L, int* one) {
   return 0;                           // b_mp
 }
 
+// Global L2 norm of the flat gradient in two fixed-order passes: per-block
+// sums of squares over a grid of GRAD_NORM_PARTS blocks (fixed, so the result
+// does not depend on the device), then one block adds them and takes the root.
+__global__ void __launch_bounds__(256) sumsq_kernel(const float* __restrict__ g, long n4, float* __restrict__ part) {
+  pdl_start();
+  __shared__ float red[8];
+  float s = 0.f;
+  for (long i4 = blockIdx.x * (long)blockDim.x + threadIdx.x; i4 < n4; i4 += (long)gridDim.x * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(g)[i4];
+    s += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = red[0];
+    for (int w = 1; w < 8; ++w) t += red[w];
+    part[blockIdx.x] = t;
+  }
+}
+
+__global__ void __launch_bounds__(256) norm_final_kernel(const float* __restrict__ part, int nparts,
+                                                         float* __restrict__ norm) {
+  pdl_start();
+  __shared__ float red[8];
+  float s = 0.f;
+  for (int i = threadIdx.x; i < nparts; i += 256) s += part[i];
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = red[0];
+    for (int w = 1; w < 8; ++w) t += red[w];
+    *norm = sqrtf(t);
+  }
+}
+
+// With gnorm != NULL the gradient is first scaled by min(1, max_norm / (gnorm + 1e-6))
+// (global-norm clipping).
 __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
                              float* __restrict__ v, uint16_t* __restrict__ shadow, long n4, LayoutDims L,
-                             AdamArgs a) {
+                             AdamArgs a, const float* __restrict__ gnorm, float max_norm) {
   pdl_start();
+  float clip = 1.f;
+  if (gnorm) {
+    const float c = max_norm / (*gnorm + 1e-6f);
+    clip = c < 1.f ? c : 1.f;
+  }
   for (long i4 = blockIdx.x * (long)blockDim.x + threadIdx.x; i4 < n4; i4 += (long)gridDim.x * blockDim.x) {
     const long i = i4 * 4;
     int one;
     const bool decay = tensor_kind(i, L, &one) != 0;
     float4 pp = reinterpret_cast<float4*>(p)[i4];
-    const float4 gg = reinterpret_cast<const float4*>(g)[i4];
+    float4 gg = reinterpret_cast<const float4*>(g)[i4];
+    gg.x *= clip; gg.y *= clip; gg.z *= clip; gg.w *= clip;
     float4 mm = reinterpret_cast<float4*>(m)[i4];
     float4 vv = reinterpret_cast<float4*>(v)[i4];
     const float dec = decay ? 1.f - a.lr * a.wd : 1.f;
@@ -966,10 +1011,19 @@ int embed_bwd(int f32, const int32_t* tok, const void* dx, float* dwte, float* d
   return GPT2_OK;
 }
 
+int grad_norm(const float* g, size_t n, float* part, float* norm, cudaStream_t st) {
+  if (n % 4) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  CUDA_TRY(launch_k(sumsq_kernel, GRAD_NORM_PARTS, 256, 0, st, g, (long)(n / 4), part));
+  LAUNCH_CHECK();
+  CUDA_TRY(launch_k(norm_final_kernel, 1, 256, 0, st, (const float*)part, GRAD_NORM_PARTS, norm));
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
 int adamw(float* p, const float* g, float* m, float* v, uint16_t* shadow, size_t n, const LayoutDims& ld,
-          const AdamArgs& a, cudaStream_t st) {
+          const AdamArgs& a, const float* gnorm, float max_norm, cudaStream_t st) {
   const long n4 = (long)(n / 4);
-  CUDA_TRY(launch_k(adamw_kernel, grid_for(n4, 256), 256, 0, st, p, g, m, v, shadow, n4, ld, a));
+  CUDA_TRY(launch_k(adamw_kernel, grid_for(n4, 256), 256, 0, st, p, g, m, v, shadow, n4, ld, a, gnorm, max_norm));
   LAUNCH_CHECK();
   return GPT2_OK;
 }

@@ -143,6 +143,21 @@ int gpt2_backward(gpt2_ctx* ctx, float grad_scale, int accumulate, void* stream)
 int gpt2_adamw_step(gpt2_ctx* ctx, float lr, float beta1, float beta2, float eps,
                     float weight_decay, int step, void* stream);
 
+/* Global L2 norm of the flat gradient buffer, sqrt(sum g^2), into the device
+ * fp32 scalar *norm_dev (4-byte aligned; NULL keeps it in the workspace).
+ * Two fixed-order reduction passes over a fixed grid, so the value is
+ * bitwise repeatable.  The pages do not clip gradients; this and
+ * gpt2_adamw_step_clip serve a training loop that does. */
+int gpt2_grad_norm(gpt2_ctx* ctx, float* norm_dev, void* stream);
+
+/* gpt2_adamw_step with global-norm gradient clipping first: every gradient is
+ * scaled by min(1, max_norm / (||g|| + 1e-6)), ||g|| computed on the device as
+ * in gpt2_grad_norm (no host synchronisation).  max_norm = 0 is exactly
+ * gpt2_adamw_step; a negative or NaN max_norm is GPT2_ERR_INVALID_ARG.  The
+ * gradient buffer itself is left unscaled. */
+int gpt2_adamw_step_clip(gpt2_ctx* ctx, float lr, float beta1, float beta2, float eps,
+                         float weight_decay, int step, float max_norm, void* stream);
+
 /* grad <- 0. */
 int gpt2_zero_grad(gpt2_ctx* ctx, void* stream);
 

@@ -223,3 +223,58 @@ def test_step_host_matches_device_path():
     assert abs(lh.item() - loss_a) <= 1e-6 * abs(loss_a)
     torch.cuda.synchronize()
     assert (a.master - b.master).abs().max().item() <= 1e-6
+
+
+def test_grad_norm_matches_torch_and_repeats():
+    """gpt2_grad_norm against a plain PyTorch fp64 norm of the same buffer,
+    against the oracle's norm of its own gradients, and bitwise repeatable."""
+    params = params_for(TINY, seed=41)
+    tok, tgt = inputs.uniform_tokens(4, 64, TINY.vocab, seed=42)
+    model = make_model(TINY, TINY.vocab, 4, 0)
+    p32 = load_params(model, params, TINY)
+    run_step(model, tok, tgt)
+    n1 = model.grad_norm()
+    n2 = model.grad_norm()
+    torch.cuda.synchronize()
+    ref = torch.linalg.vector_norm(model.grad.double()).item()
+    assert abs(n1.item() - ref) <= 1e-5 * ref, (n1.item(), ref)
+    assert torch.equal(n1, n2)
+    _, cache = forward(p32, TINY, tok, tgt)
+    _, total = oracle.gpt2_oracle.clip_grad_norm(backward(p32, TINY, cache), 1.0)
+    assert abs(n1.item() - total) <= 1e-2 * total, (n1.item(), total)
+
+
+def test_tiny_clipped_adamw_steps():
+    """Five steps with global-norm clipping active (max_norm below every
+    step's gradient norm): parameters against the oracle's clipped AdamW."""
+    params = params_for(TINY, seed=51)
+    model = make_model(TINY, TINY.vocab, 4, 0)
+    p = load_params(model, params, TINY)
+    m = {n: np.zeros(s) for n, s in param_shapes(TINY)}
+    v = {n: np.zeros(s) for n, s in param_shapes(TINY)}
+    max_norm = None
+    for step in range(1, 6):
+        tok, tgt = inputs.uniform_tokens(4, 64, TINY.vocab, seed=500 + step)
+        run_step(model, tok, tgt)
+        ref_loss, cache = forward(p, TINY, tok, tgt)
+        g = backward(p, TINY, cache)
+        if max_norm is None:
+            max_norm = 0.3 * oracle.gpt2_oracle.clip_grad_norm(g, 1.0)[1]
+        assert oracle.gpt2_oracle.clip_grad_norm(g, max_norm)[1] > max_norm  # clipping is active
+        model.adamw_step(step, max_norm=max_norm)
+        p, m, v = adamw_step(p, g, m, v, step, TINY, max_norm=max_norm)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    got = oracle.unflatten(model.master.double().cpu().numpy(), TINY)
+    d = TINY.d_model
+    for n in p:
+        a, r = got[n], p[n]
+        if n.endswith("b_qkv"):
+            # zero true gradient for the key bias: Adam's per-step bound (see
+            # test_tiny_ten_adamw_steps)
+            kb = slice(d, 2 * d)
+            assert np.abs(a[kb] - r[kb]).max() <= 2 * 5 * 6e-4 / np.sqrt(1 - 0.95)
+            a = np.concatenate([a[:d], a[2 * d:]])
+            r = np.concatenate([r[:d], r[2 * d:]])
+        rel = np.linalg.norm(a - r) / np.linalg.norm(r)
+        assert rel <= 1e-2, (n, rel)
