@@ -210,6 +210,41 @@ def run_ours(args, rank, world, local_rank):
         e2e_s = float(t.item())
     e2e_tps = world * M * e_steps / e2e_s
 
+    # the pages' optimizer step: the same micro-batch with 32-fold gradient
+    # accumulation (grad_scale 1/k, accumulate after the first), then AdamW
+    accum = None
+    if args.accum > 1:
+        k = args.accum
+
+        def accum_step(i):
+            for j in range(k):
+                tok, tgt = pool[(i * k + j) % len(pool)]
+                model.forward_loss(tok, tgt)
+                model.backward(1.0 / k, 1 if j else 0)
+            if world > 1:
+                average_gradients(model.grad)
+            model.adamw_step(args.warmup + args.steps + e_steps + 2 + i)
+
+        a_steps = 2
+        accum_step(0)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(a_steps):
+            accum_step(1 + i)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        a_ms = a0.elapsed_time(a1)
+        if world > 1:
+            t = torch.tensor([a_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            a_ms = float(t.item())
+        accum = {"accumulation": k, "value": round(world * M * k * a_steps / (a_ms / 1e3), 1), "unit": "tokens/s",
+                 "ms_per_optimizer_step": round(a_ms / a_steps, 2),
+                 "tokens_per_optimizer_step": world * M * k}
+
     # dominant kernel: the tied LM-head GEMM [M x V x d], timed alone
     roof = lm_head_roofline(gp, model, M, V, d, stream)
 
@@ -233,7 +268,10 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2: the step's working set (>5 GB) exceeds the 126 MB L2"},
         "mfu": round(flops.mfu(tokens_per_s / world, fpt, peaks["bf16_tflops"] * 1e12), 4),
         "mfu_vs_sustained": round(flops.mfu(tokens_per_s / world, fpt, peaks["bf16_tflops_sustained"] * 1e12), 4),
+        "mfu_vs_datasheet": round(flops.mfu(tokens_per_s / world, fpt, 2250e12), 4),
         "flops_per_token": fpt,
+        "flops_per_token_matmul": flops.matmul_flops_per_token(L, d, V, T),
+        "max_memory_gb": round(torch.cuda.max_memory_allocated() / 1e9, 2),
         "peak_source": peak_kind,
         "final_loss": round(loss, 4),
         "device_status": status,
@@ -243,6 +281,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roof,
         "clocks": clocks.summary(),
     }
+    if accum:
+        result["accum"] = accum
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args.config)
     if world > 1:
@@ -424,6 +464,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="124m", choices=sorted(CONFIGS))
+    ap.add_argument("--accum", type=int, default=32,
+                    help="also time optimizer steps with this many accumulated micro-batches (0 or 1: skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -22,6 +22,13 @@ def train_flops_per_token(n_layer: int, d: int, vocab: int, n_ctx: int, T: int) 
     return 6 * param_count(n_layer, d, vocab, n_ctx) + 12 * n_layer * T * d
 
 
+def matmul_flops_per_token(n_layer: int, d: int, vocab: int, T: int) -> int:
+    """6 N_matmul + 12 L T d with N_matmul the parameters that enter a matmul
+    (the twelve d^2 per block and the tied head; not wpe, biases or LayerNorm
+    gains): what a FLOP counter sees, with the attention products unmasked."""
+    return 6 * (n_layer * 12 * d * d + vocab * d) + 12 * n_layer * T * d
+
+
 def executed_matmul_flops_per_token(n_layer: int, d: int, vocab: int, T: int) -> float:
     """FLOPs the kernels actually execute per token: every weight matmul three
     times (forward, input gradient, weight gradient) and the attention products

@@ -225,18 +225,27 @@ def attention_bwd(do, q, k, v, p, counter):
     return dq, dk, dv
 
 
+IGNORE = -1  # target id of a position that takes no part in the loss
+
+
 def cross_entropy_fwd(z, targets):
-    """Per-position loss LSE(z) - z[target] with an explicit max-shifted LSE."""
+    """Per-position loss LSE(z) - z[target] with an explicit max-shifted LSE;
+    positions whose target is IGNORE get loss 0.  That is the masked loss of
+    instruction tuning: "Criei GPT-2 do zero com uma RTX 4090", section "Usei
+    SFT para fazê-lo conversar", trains only the assistant's answer and its
+    end marker while the question is only read."""
     zmax = z.max(axis=-1, keepdims=True)
     lse = zmax[..., 0] + np.log(np.exp(z - zmax).sum(axis=-1))
-    z_t = np.take_along_axis(z, targets[..., None], axis=-1)[..., 0]
-    return lse - z_t, lse
+    valid = targets != IGNORE
+    z_t = np.take_along_axis(z, np.where(valid, targets, 0)[..., None], axis=-1)[..., 0]
+    return np.where(valid, lse - z_t, 0.0), lse
 
 
 # ------------------------------------------------------------- the model ---
 
 def forward(params: dict, cfg: Config, tokens, targets, counter=None, head=None):
-    """Mean next-token cross-entropy over all B*T positions, plus a cache.
+    """Mean next-token cross-entropy over the positions that have a target
+    (all B*T of them unless some targets are IGNORE), plus a cache.
 
     ``head`` (optional) replaces the tied LM-head matrix by a separate copy;
     it exists only for the tied-embedding decomposition test.
@@ -271,7 +280,9 @@ def forward(params: dict, cfg: Config, tokens, targets, counter=None, head=None)
     w_head = params["wte"] if head is None else head
     z = linear_fwd(yf, w_head, None, counter)
     loss_pos, lse = cross_entropy_fwd(z, targets)
-    loss = float(loss_pos.mean())
+    # mean over the positions that have a target (all of them unless masked)
+    n_valid = max(1, int(np.sum(targets != IGNORE)))
+    loss = float(loss_pos.sum() / n_valid)
     cache = dict(tokens=tokens, targets=targets, layers=layers, yf=yf, lnf=lnf,
                  z=z, lse=lse, loss_pos=loss_pos, head=head)
     return loss, cache
@@ -291,12 +302,15 @@ def backward(params: dict, cfg: Config, cache: dict, grad_scale: float = 1.0, co
     H = cfg.n_head
     grads = {n: np.zeros(s) for n, s in param_shapes(cfg)}
 
-    # d loss / d z = (softmax(z) - onehot(target)) / M
+    # d loss / d z = (softmax(z) - onehot(target)) / n_valid on positions with
+    # a target, 0 on masked ones (n_valid = M without masking)
     z = cache["z"]
+    valid = targets != IGNORE
+    n_valid = max(1, int(np.sum(valid)))
+    safe_t = np.where(valid, targets, 0)
     dz = np.exp(z - cache["lse"][..., None])
-    np.put_along_axis(dz, targets[..., None],
-                      np.take_along_axis(dz, targets[..., None], axis=-1) - 1.0, axis=-1)
-    dz *= grad_scale / M
+    np.put_along_axis(dz, safe_t[..., None], np.take_along_axis(dz, safe_t[..., None], axis=-1) - 1.0, axis=-1)
+    dz *= np.where(valid, grad_scale / n_valid, 0.0)[..., None]
     w_head = params["wte"] if cache["head"] is None else cache["head"]
     dyf, dw_head, _ = linear_bwd(dz, cache["yf"], w_head, counter)
     if cache["head"] is None:

@@ -287,3 +287,46 @@ def test_lr_schedule_closed_forms():
     assert all(a >= b for a, b in zip(lrs, lrs[1:]))
     with pytest.raises(ValueError):
         lr_at(0, max_lr, 10, 10)
+
+
+def test_masked_cross_entropy_matches_torch():
+    """Targets equal to IGNORE (-1) take no part: loss and dloss/dz against
+    torch.nn.functional.cross_entropy(ignore_index=-1) and its autograd."""
+    import torch
+    rng = np.random.default_rng(8)
+    z = rng.standard_normal((2, 5, 13)) * 2.0
+    t = rng.integers(0, 13, size=(2, 5))
+    t[0, 1] = t[1, 3] = t[1, 4] = G.IGNORE
+    loss_pos, lse = G.cross_entropy_fwd(z, t)
+    assert (loss_pos[t == G.IGNORE] == 0).all()
+    zt = torch.from_numpy(z.reshape(-1, 13)).requires_grad_(True)
+    ref = torch.nn.functional.cross_entropy(zt, torch.from_numpy(t.reshape(-1)), ignore_index=-1)
+    ref.backward()
+    n_valid = int((t != G.IGNORE).sum())
+    assert abs(loss_pos.sum() / n_valid - ref.item()) <= 1e-13
+    # the oracle's dz (as backward forms it) against autograd
+    dz = np.exp(z - lse[..., None])
+    valid = t != G.IGNORE
+    safe = np.where(valid, t, 0)
+    np.put_along_axis(dz, safe[..., None], np.take_along_axis(dz, safe[..., None], axis=-1) - 1.0, axis=-1)
+    dz *= np.where(valid, 1.0 / n_valid, 0.0)[..., None]
+    np.testing.assert_allclose(dz.reshape(-1, 13), zt.grad.numpy(), rtol=1e-12, atol=1e-15)
+
+
+def test_masked_forward_backward_reduces_to_subset():
+    """Masking positions equals dropping them from the mean: with only the
+    first sequence's targets kept, loss and gradients equal the unmasked
+    model run on that sequence alone (the other sequence still shares
+    nothing with it: attention is per sequence)."""
+    cfg = TINY
+    params = params_for(cfg, 9)
+    tok, tgt = inputs.uniform_tokens(2, cfg.n_ctx, cfg.vocab, seed=10)
+    masked = tgt.copy()
+    masked[1, :] = G.IGNORE
+    loss_m, cache_m = forward(params, cfg, tok, masked)
+    g_m = backward(params, cfg, cache_m)
+    loss_1, cache_1 = forward(params, cfg, tok[:1], tgt[:1])
+    g_1 = backward(params, cfg, cache_1)
+    assert abs(loss_m - loss_1) <= 1e-12 * abs(loss_1)
+    for n in g_1:
+        np.testing.assert_allclose(g_m[n], g_1[n], rtol=1e-9, atol=1e-14)
