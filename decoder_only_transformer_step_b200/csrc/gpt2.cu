@@ -107,6 +107,7 @@ struct Work {
   void *dres, *dy, *du, *dqkv, *dout;
   float *dq_acc, *dvec;
   float *norm_part, *gnorm;  // global gradient norm: block partials and the result
+  int* n_valid;              // positions with a target in the last forward
   // block partials of every bias / LayerNorm parameter gradient of one
   // backward, each in its own slot, all reduced by one launch at its end
   float* part_arena;
@@ -182,6 +183,7 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
   w->part_arena = c.take<float>(w->part_floats * 4);
   w->norm_part = c.take<float>((size_t)GRAD_NORM_PARTS * 4);
   w->gnorm = c.take<float>(4);
+  w->n_valid = c.take<int>(4);
   w->part_used = 0;
   w->split_bytes = split_ws_need(s, M);
   w->split_ws = c.take<void>(w->split_bytes);
@@ -432,8 +434,9 @@ int gpt2_forward_loss(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets
   TRY(layernorm_fwd(f32, w.x_final, Wp(c, o.lnf_g()), Wp(c, o.lnf_b()), w.yf, w.meanf, w.rstdf, M, d, st));
   GemmArgs g = make_gemm(M, V, d, w.yf, 0, d, Wp(c, o.wte()), 0, d, EPI_STORE, w.logits, V);
   TRY(run_gemm(c, g, st));
-  TRY(ce_fwd(f32, w.logits, w.tgt, w.loss_rows, M, V, (int)s.Vr, w.err, st));
-  TRY(loss_mean(w.loss_rows, M, loss_dev ? loss_dev : w.loss, w.err, st));
+  TRY(count_targets(w.tgt, M, (int)s.Vr, w.n_valid, w.err, st));
+  TRY(ce_fwd(f32, w.logits, w.tgt, w.loss_rows, M, V, (int)s.Vr, w.n_valid, w.err, st));
+  TRY(loss_mean(w.loss_rows, M, w.n_valid, loss_dev ? loss_dev : w.loss, w.err, st));
   c->have_fwd = 1;
   c->fwd_batch = batch;
   return GPT2_OK;

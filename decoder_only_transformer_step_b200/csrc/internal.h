@@ -96,10 +96,13 @@ int reduce_rows_batch(const ReduceJob* jobs, int njobs, float beta, cudaStream_t
 // per-block column sums of x [M, N] (act) into part [nblk, N]
 int colsum_partial(int f32, const void* x, int M, int N, float* part, int* nblk, cudaStream_t st);
 size_t colsum_part_floats(int M, int N);
-// cross-entropy: logits [M, V] (act) -> in place dz = softmax - onehot; loss_rows [M]
+// targets with an id (not -1) -> *n_valid; other out-of-range ids raise the token bit
+int count_targets(const int32_t* tgt, int M, int vocab_real, int* n_valid, int* err, cudaStream_t st);
+// cross-entropy: logits [M, V] (act) -> in place dz = (softmax - onehot) M / n_valid
+// (zero rows where the target is -1); loss_rows [M] (0 where masked)
 int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, int V,
-           int vocab_real, int* err, cudaStream_t st);
-int loss_mean(const float* loss_rows, int M, float* loss, int* err, cudaStream_t st);
+           int vocab_real, const int* n_valid, int* err, cudaStream_t st);
+int loss_mean(const float* loss_rows, int M, const int* n_valid, float* loss, int* err, cudaStream_t st);
 // dwte[tok[m]] += dx[m] (deterministic fixed-point scatter), dwpe (=/+=) sum_b dx
 int embed_bwd(int f32, const int32_t* tok, const void* dx, float* dwte, float* dwpe,
               long long* acc, uint8_t* touched, int M, int T, int d, int V, int wpe_accumulate,

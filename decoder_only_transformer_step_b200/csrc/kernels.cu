@@ -512,13 +512,38 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ x, in
 }
 
 // ---------------------------------------------------------- cross-entropy --
+// Number of positions with a target (target -1 = masked); any other id outside
+// [0, vocab_real) raises the token-range bit and counts as masked.
+__global__ void __launch_bounds__(1024) count_targets_kernel(const int32_t* __restrict__ tgt, int M,
+                                                             int vocab_real, int* __restrict__ n_valid, int* err) {
+  pdl_start();
+  __shared__ int red[32];
+  int c = 0;
+  for (int i = threadIdx.x; i < M; i += blockDim.x) {
+    const int t = tgt[i];
+    if (t >= 0 && t < vocab_real)
+      ++c;
+    else if (t != -1)
+      atomicOr(err, DEV_ERR_TOKEN);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+    *n_valid = t;
+  }
+}
+
 // Row m: lse = log sum_v exp(z_v) over all V (padded) ids; loss = lse - z[y];
 // then, in place, dz_v = exp(z_v - lse) - [v == y] (unscaled; the backward
 // GEMMs apply grad_scale / M).
 template <typename T>
 __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const int32_t* __restrict__ tgt,
                                                  float* __restrict__ loss_rows, int V, int vocab_real,
-                                                 int* err) {
+                                                 const int* __restrict__ n_valid, int* err) {
   pdl_start();
   constexpr int VN = Vec<T>::N;
   constexpr int U = 4;  // 16-byte vectors in flight per thread and trip
@@ -528,6 +553,15 @@ __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const i
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   T* z = logits + (long)m * V;
   const int step = 256 * VN;
+  if (tgt[m] == -1) {
+    // masked position: no loss, and its dlogits row is zero
+    if (threadIdx.x == 0) loss_rows[m] = 0.f;
+    float zero[VN];
+#pragma unroll
+    for (int j = 0; j < VN; ++j) zero[j] = 0.f;
+    for (int c = threadIdx.x * VN; c < V; c += step) Vec<T>::store(z + c, zero);
+    return;
+  }
   // pass 1: running maximum and sum of exp(z - max), U vectors per trip so the
   // loads of a trip overlap (V is a multiple of 128, so vectors never straddle it)
   float mx = -INFINITY, sum = 0.f;
@@ -588,8 +622,12 @@ __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const i
   const float zy = to_f(z[y]);
   __syncthreads();  // every thread has read z[y] before it is overwritten
   if (threadIdx.x == 0) loss_rows[m] = lse - zy;
-  // pass 2: dz = softmax(z) - onehot(y), in place
+  // pass 2: dz = (softmax(z) - onehot(y)) * M / n_valid, in place: the backward
+  // GEMMs scale by grad_scale / M, so the loss is the mean over the positions
+  // that have a target (the factor is exactly 1 without masking)
   const float ll = lse * L2E;
+  const int nv = *n_valid;
+  const float rs = (float)gridDim.x / (float)(nv > 0 ? nv : 1);
   for (int c0 = threadIdx.x * VN; c0 < V; c0 += U * step) {
     float f[U][VN];
 #pragma unroll
@@ -600,15 +638,18 @@ __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const i
       const int c = c0 + u * step;
       if (c < V) {
 #pragma unroll
-        for (int j = 0; j < VN; ++j) f[u][j] = ex2_approx(fmaf(f[u][j], L2E, -ll)) - (c + j == y ? 1.f : 0.f);
+        for (int j = 0; j < VN; ++j)
+          f[u][j] = (ex2_approx(fmaf(f[u][j], L2E, -ll)) - (c + j == y ? 1.f : 0.f)) * rs;
         Vec<T>::store(z + c, f[u]);
       }
     }
   }
 }
 
-// loss = mean(loss_rows), fixed-order tree; flags a non-finite result.
-__global__ void loss_mean_kernel(const float* __restrict__ rows, int M, float* __restrict__ loss, int* err) {
+// loss = sum(loss_rows) / n_valid (masked rows hold 0), fixed-order tree;
+// flags a non-finite result.
+__global__ void loss_mean_kernel(const float* __restrict__ rows, int M, const int* __restrict__ n_valid,
+                                 float* __restrict__ loss, int* err) {
   pdl_start();
   __shared__ float sm[1024];
   float s = 0.f;
@@ -620,7 +661,8 @@ __global__ void loss_mean_kernel(const float* __restrict__ rows, int M, float* _
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    float v = sm[0] / M;
+    const int nv = *n_valid;
+    float v = sm[0] / (float)(nv > 0 ? nv : 1);
     *loss = v;
     if (!isfinite(v)) atomicOr(err, DEV_ERR_NONFINITE);
   }
@@ -970,18 +1012,26 @@ int colsum_partial(int f32, const void* x, int M, int N, float* part, int* nblk,
   return GPT2_OK;
 }
 
-int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, int V, int vocab_real, int* err,
-           cudaStream_t st) {
-  if (f32)
-    CUDA_TRY(launch_k(ce_kernel<float>, M, 256, 0, st, (float*)logits, tgt, loss_rows, V, vocab_real, err));
-  else
-    CUDA_TRY(launch_k(ce_kernel<bf16>, M, 256, 0, st, (bf16*)logits, tgt, loss_rows, V, vocab_real, err));
+int count_targets(const int32_t* tgt, int M, int vocab_real, int* n_valid, int* err, cudaStream_t st) {
+  CUDA_TRY(launch_k(count_targets_kernel, 1, 1024, 0, st, tgt, M, vocab_real, n_valid, err));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
 
-int loss_mean(const float* loss_rows, int M, float* loss, int* err, cudaStream_t st) {
-  CUDA_TRY(launch_k(loss_mean_kernel, 1, 1024, 0, st, loss_rows, M, loss, err));
+int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, int V, int vocab_real,
+           const int* n_valid, int* err, cudaStream_t st) {
+  if (f32)
+    CUDA_TRY(launch_k(ce_kernel<float>, M, 256, 0, st, (float*)logits, tgt, loss_rows, V, vocab_real, n_valid,
+                      err));
+  else
+    CUDA_TRY(launch_k(ce_kernel<bf16>, M, 256, 0, st, (bf16*)logits, tgt, loss_rows, V, vocab_real, n_valid,
+                      err));
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+int loss_mean(const float* loss_rows, int M, const int* n_valid, float* loss, int* err, cudaStream_t st) {
+  CUDA_TRY(launch_k(loss_mean_kernel, 1, 1024, 0, st, loss_rows, M, n_valid, loss, err));
   LAUNCH_CHECK();
   return GPT2_OK;
 }

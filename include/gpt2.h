@@ -121,8 +121,11 @@ int gpt2_init_params(gpt2_ctx* ctx, uint64_t seed, void* stream);
 int gpt2_refresh_shadow(gpt2_ctx* ctx, void* stream);
 
 /* Forward pass and loss.  tokens, targets: device int32 [batch, n_ctx]
- * (targets[b,t] is the id at t+1 of the stream).  Writes the mean
- * cross-entropy over batch*n_ctx positions to *loss_dev (device fp32) and
+ * (targets[b,t] is the id at t+1 of the stream, or -1 for a position that
+ * takes no part in the loss: the masked loss of instruction tuning, "Criei
+ * GPT-2 do zero com uma RTX 4090", section "Usei SFT para fazê-lo
+ * conversar").  Writes the mean cross-entropy over the positions with a
+ * target (batch*n_ctx of them without -1s) to *loss_dev (device fp32) and
  * keeps the activations (and the dlogits of this batch) in the workspace for
  * gpt2_backward.  The ids are copied into the workspace, so the caller's
  * arrays may be reused as soon as this call's work has run. */

@@ -278,3 +278,40 @@ def test_tiny_clipped_adamw_steps():
             r = np.concatenate([r[:d], r[2 * d:]])
         rel = np.linalg.norm(a - r) / np.linalg.norm(r)
         assert rel <= 1e-2, (n, rel)
+
+
+@pytest.mark.parametrize("mode", [1, 0])
+def test_tiny_masked_loss_and_grads(mode):
+    """Targets of -1 take no part (instruction-tuning loss): loss and every
+    gradient against the oracle, with about a third of the positions masked,
+    including one fully masked sequence."""
+    params = params_for(TINY, seed=61)
+    tok, tgt = inputs.uniform_tokens(4, 64, TINY.vocab, seed=62)
+    rng = np.random.default_rng(63)
+    tgt = tgt.copy()
+    tgt[rng.random(tgt.shape) < 0.3] = -1
+    tgt[2, :] = -1
+    model = make_model(TINY, TINY.vocab, 4, mode)
+    p32 = load_params(model, params, TINY)
+    loss = run_step(model, tok, tgt)
+    ref_loss, cache = forward(p32, TINY, tok, tgt)
+    ref_g = backward(p32, TINY, cache)
+    tol_loss = 1e-4 if mode == 1 else 1e-2
+    assert abs(loss - ref_loss) <= tol_loss * abs(ref_loss), (loss, ref_loss)
+    if mode == 1:
+        compare_grads(gpu_grads(model, TINY), ref_g, 0.99999, 1e-3)
+    else:
+        compare_grads(gpu_grads(model, TINY), ref_g, 0.999, 2e-2)
+
+
+def test_target_minus_one_is_masked_other_negatives_flagged():
+    model = make_model(TINY, 500, 4, 0)
+    model.init_params(seed=2)
+    tok, tgt = inputs.uniform_tokens(4, 64, 500, seed=64)
+    tgt[0, :10] = -1                      # masked: no error
+    model.forward_loss(torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda())
+    assert model.status() == 0
+    tgt[0, 3] = -2                        # neither an id nor the mask value
+    model.forward_loss(torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda())
+    assert model.status() == -5
+    assert model.status() == 0
