@@ -7,6 +7,7 @@ its Python binding) never imports it and shares no code with it.
 from .gpt2_oracle import (  # noqa: F401
     Config, param_shapes, param_count, flatten, unflatten, decay_mask,
     forward, backward, adamw_step, train_step, MatmulCounter,
+    kv_cache_empty, decode_step, prefill, greedy_next,
 )
 from .flops import (  # noqa: F401
     n_params_total, n_params_matmul, flops_per_token, flops_per_token_matmul_only,

@@ -388,3 +388,74 @@ def train_step(params, m, v, step, cfg, tokens, targets, **hp):
     grads = backward(params, cfg, cache)
     P, Mo, Vo = adamw_step(params, grads, m, v, step, cfg, **hp)
     return loss, grads, P, Mo, Vo
+
+
+# ------------------------------------------------ incremental decoding ---
+#
+# "Criei GPT-2 do zero com uma RTX 4090", sections "Vendo o modelo ficar mais
+# inteligente aos poucos" and "Conversando de verdade com ele": the trained
+# model continues a prompt one token at a time.  The distribution of the next
+# token after positions 0..p is the forward's output at position p, and by
+# causality that output depends on the keys and values of positions 0..p only.
+# A decoder therefore keeps every layer's K and V of the positions seen so far
+# (the key/value cache) and, per new token, computes one query row against
+# them.  The pages fix no sampling rule; greedy (the most probable id) is the
+# plainest.
+
+def kv_cache_empty(cfg: Config, batch: int, max_len: int) -> list:
+    """Per layer {"k", "v"}: [batch, H, max_len, hd] zeros."""
+    shape = (batch, cfg.n_head, max_len, cfg.head_dim)
+    return [dict(k=np.zeros(shape), v=np.zeros(shape)) for _ in range(cfg.n_layer)]
+
+
+def decode_step(params: dict, cfg: Config, cache: list, tokens, pos):
+    """Row b feeds token ``tokens[b]`` at position ``pos[b]``: its K and V are
+    written into the cache at that position, its query attends to positions
+    0..pos[b] of the row's cache, and the logits of the next token
+    ([batch, vocab]) are returned."""
+    tokens = np.asarray(tokens)
+    pos = np.asarray(pos)
+    B = tokens.shape[0]
+    H, hd, d = cfg.n_head, cfg.head_dim, cfg.d_model
+    x = params["wte"][tokens] + params["wpe"][pos]                      # [B, d]
+    for l in range(cfg.n_layer):
+        P = lambda t: params[f"h{l}.{t}"]  # noqa: E731
+        y1, _ = layernorm_fwd(x, P("ln1_g"), P("ln1_b"))
+        qkv = linear_fwd(y1, P("w_qkv"), P("b_qkv"), None)               # [B, 3d]
+        q, k, v = (qkv[:, i * d:(i + 1) * d].reshape(B, H, hd) for i in range(3))
+        a = np.zeros((B, H, hd))
+        for b in range(B):
+            p = int(pos[b])
+            cache[l]["k"][b, :, p, :] = k[b]
+            cache[l]["v"][b, :, p, :] = v[b]
+            keys = cache[l]["k"][b, :, :p + 1, :]                         # [H, p+1, hd]
+            vals = cache[l]["v"][b, :, :p + 1, :]
+            s = np.einsum("hd,hjd->hj", q[b], keys) / math.sqrt(hd)
+            e = np.exp(s - s.max(axis=-1, keepdims=True))
+            prob = e / e.sum(axis=-1, keepdims=True)
+            a[b] = np.einsum("hj,hjd->hd", prob, vals)
+        x = x + linear_fwd(a.reshape(B, d), P("w_o"), P("b_o"), None)
+        y2, _ = layernorm_fwd(x, P("ln2_g"), P("ln2_b"))
+        x = x + linear_fwd(gelu_fwd(linear_fwd(y2, P("w_fc"), P("b_fc"), None)), P("w_mp"), P("b_mp"), None)
+    yf, _ = layernorm_fwd(x, params["lnf_g"], params["lnf_b"])
+    return linear_fwd(yf, params["wte"], None, None)
+
+
+def prefill(params: dict, cfg: Config, cache: list, tokens, prompt_len):
+    """Feeds row b's prompt ``tokens[b, :prompt_len[b]]`` through the cache one
+    position at a time; returns each row's logits after its last prompt token
+    ([batch, vocab])."""
+    tokens = np.asarray(tokens)
+    B = tokens.shape[0]
+    out = np.zeros((B, cfg.vocab))
+    for b in range(B):
+        row = [dict(k=c["k"][b:b + 1], v=c["v"][b:b + 1]) for c in cache]  # views: writes land in cache
+        for p in range(int(prompt_len[b])):
+            out[b] = decode_step(params, cfg, row, tokens[b, p:p + 1], np.array([p]))[0]
+    return out
+
+
+def greedy_next(logits, vocab_real: int):
+    """Most probable real id per row (padded ids never chosen); the lowest id
+    among equal maxima, and the first NaN if a row holds one."""
+    return np.argmax(np.asarray(logits)[:, :vocab_real], axis=-1).astype(np.int32)
