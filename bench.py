@@ -247,6 +247,8 @@ def run_ours(args, rank, world, local_rank):
 
     # dominant kernel: the tied LM-head GEMM [M x V x d], timed alone
     roof = lm_head_roofline(gp, model, M, V, d, stream)
+    dec = decode_bench(gp, model, L, d, H, T, Vr, V, args.decode_steps) if rank == 0 and args.decode_steps > 0 \
+        else None
 
     peaks, peak_kind = load_peaks()
     fpt = flops.train_flops_per_token(L, d, V, T, T)
@@ -283,6 +285,8 @@ def run_ours(args, rank, world, local_rank):
     }
     if accum:
         result["accum"] = accum
+    if dec:
+        result["decode"] = dec
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args.config)
     if world > 1:
@@ -290,6 +294,62 @@ def run_ours(args, rank, world, local_rank):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def decode_bench(gp, model, L, d, H, T, Vr, V, steps, batch=8, prompt=128):
+    """Greedy incremental decoding with the key/value cache on the same model:
+    prefill of `batch` prompts of `prompt` tokens, then one CUDA graph per
+    decode step (the step's kernels plus the greedy choice, tokens and
+    positions on the device), `steps` replays timed with CUDA events after 3
+    warm-up replays.  Algorithmic HBM bytes per step: every bf16 weight once
+    (the tied LM head reads all of wte), each row's cached K and V of the
+    positions it attends to, its new K and V, and the fp32 logits."""
+    import torch
+    from decoder_only_transformer_step_b200 import inputs
+    warm = 3
+    steps = min(steps, T - prompt - warm)
+    tok = torch.from_numpy(inputs.zipf_tokens(batch, T, n_ids=Vr, seed=777)[0]).cuda()
+    plen = torch.full((batch,), prompt, dtype=torch.int32, device="cuda")
+    cache = gp.KVCache(model, batch, T)
+    cache.prefill(tok, plen)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):   # first launches (kernel attributes) outside the capture
+        cache.step()
+        cache.greedy_advance()
+    torch.cuda.current_stream().wait_stream(side)
+    cache.prefill(tok, plen)
+    graph = torch.cuda.CUDAGraph()
+    l0 = gp.gpt2_kernel_launches()
+    with torch.cuda.graph(graph):
+        cache.step()
+        cache.greedy_advance()
+    launches = gp.gpt2_kernel_launches() - l0
+    for _ in range(warm):
+        graph.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    status = model.status()
+    del graph
+    weights = L * (12 * d * d + 13 * d) + 2 * d + V * d             # elements read per step
+    keys = prompt + warm + (steps - 1) / 2 + 1                       # mean positions attended
+    kv = L * 2 * batch * d * (keys + 1)                              # elements read + written
+    nbytes = 2 * (weights + kv) + 4 * batch * V
+    peaks, _ = load_peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": f"greedy decode with KV cache, batch {batch}, prompt {prompt}, {steps} new tokens per "
+                        "row, one CUDA graph per step", "tokens_per_s": round(batch / (ms / 1e3), 1),
+            "ms_per_token_step": round(ms, 4), "gpu_launches_per_step": int(launches),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_step": int(nbytes)},
+            "device_status": status}
 
 
 def lm_head_roofline(gp, model, M, V, d, stream):
@@ -419,7 +479,19 @@ def run_kernel(args):
     M = args.tokens
     g = torch.Generator(device="cuda").manual_seed(0)
     torch.cuda.synchronize()
-    if args.kernel == "lm_head":
+    if args.kernel == "decode":
+        # eager decode steps of the 124M model at batch 8 after a 128-token prompt
+        model = gp.GPT2(gp.ModelConfig(L, d, H, T, Vr, V, 8, 0))
+        model.init_params(seed=0)
+        cache = gp.KVCache(model, 8, T)
+        tok = torch.randint(0, Vr, (8, T), dtype=torch.int32, device="cuda", generator=g)
+        cache.prefill(tok, torch.full((8,), 128, dtype=torch.int32, device="cuda"))
+
+        def fn():
+            cache.step()
+            cache.greedy_advance()
+        flop = 2.0 * 8 * (L * 12 * d * d + V * d)
+    elif args.kernel == "lm_head":
         A = torch.randn(M, d, device="cuda", generator=g).to(torch.bfloat16)
         W = (0.02 * torch.randn(V, d, device="cuda", generator=g)).to(torch.bfloat16)
         C = torch.empty(M, V, dtype=torch.bfloat16, device="cuda")
@@ -455,7 +527,7 @@ def run_kernel(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", choices=["lm_head", "attn_fwd", "attn_bwd"], default=None,
+    ap.add_argument("--kernel", choices=["lm_head", "attn_fwd", "attn_bwd", "decode"], default=None,
                     help="time one kernel alone instead of the step (profiler captures)")
     ap.add_argument("--tokens", type=int, default=4096)
     ap.add_argument("--reps", type=int, default=3)
@@ -466,6 +538,8 @@ def main():
     ap.add_argument("--config", default="124m", choices=sorted(CONFIGS))
     ap.add_argument("--accum", type=int, default=32,
                     help="also time optimizer steps with this many accumulated micro-batches (0 or 1: skip)")
+    ap.add_argument("--decode-steps", type=int, default=64,
+                    help="also time this many greedy KV-cache decode steps at batch 8 (0: skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

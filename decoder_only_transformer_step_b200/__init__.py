@@ -22,7 +22,9 @@ ERRORS = {
     -1: "GPT2_ERR_INVALID_ARG", -2: "GPT2_ERR_UNSUPPORTED_SHAPE", -3: "GPT2_ERR_CUDA",
     -4: "GPT2_ERR_BAD_STATE", -5: "GPT2_ERR_TOKEN_RANGE", -6: "GPT2_ERR_NONFINITE",
     -7: "GPT2_ERR_TIMEOUT", -8: "GPT2_ERR_WORKSPACE", -9: "GPT2_ERR_TOO_LARGE",
+    -10: "GPT2_ERR_POSITION_RANGE",
 }
+ERRORS_BY_NAME = {v: k for k, v in ERRORS.items()}
 
 
 class Gpt2Error(RuntimeError):
@@ -48,6 +50,7 @@ EXPORTS = [
     "gpt2_init_params", "gpt2_refresh_shadow", "gpt2_forward_loss", "gpt2_backward",
     "gpt2_adamw_step", "gpt2_adamw_step_clip", "gpt2_grad_norm", "gpt2_zero_grad", "gpt2_get_status", "gpt2_step_host", "gpt2_strerror",
     "gpt2_kernel_launches",
+    "gpt2_kv_cache_bytes", "gpt2_prefill", "gpt2_decode_step", "gpt2_greedy_next",
     "gpt2_op_gemm_bf16", "gpt2_op_attention_fwd_bf16", "gpt2_op_attention_bwd_bf16",
     "gpt2_op_attention_bwd_bf16_noalloc",
 ]
@@ -84,6 +87,10 @@ def _lib():
         "gpt2_step_host": (I, [P, P, P, I, P, F, F, F, F, F, I, P]),
         "gpt2_strerror": (ctypes.c_char_p, [I]),
         "gpt2_kernel_launches": (ctypes.c_uint64, []),
+        "gpt2_kv_cache_bytes": (S, [cfgp, I, I]),
+        "gpt2_prefill": (I, [P, P, S, I, I, P, P, P, P]),
+        "gpt2_decode_step": (I, [P, P, S, I, I, P, P, P, P]),
+        "gpt2_greedy_next": (I, [P, P, I, P, P, P]),
         "gpt2_op_gemm_bf16": (I, [P, I, I, P, I, I, P, I, I, I, I, I, F, F, P, S, I, I, P]),
         "gpt2_op_attention_fwd_bf16": (I, [P, P, P, I, I, I, I, P]),
         "gpt2_op_attention_bwd_bf16": (I, [P, P, P, P, P, P, I, I, I, I, P]),
@@ -209,6 +216,31 @@ def gpt2_step_host(ctx, tokens_host, targets_host, batch, loss_host, lr, beta1, 
 
 def gpt2_kernel_launches() -> int:
     return int(_lib().gpt2_kernel_launches())
+
+
+def gpt2_kv_cache_bytes(cfg: gpt2_config, batch: int, max_len: int) -> int:
+    return int(_lib().gpt2_kv_cache_bytes(ctypes.byref(cfg), batch, max_len))
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def gpt2_prefill(ctx, cache, batch, max_len, tokens, prompt_len, logits, stream=None):
+    """cache: a device tensor of at least gpt2_kv_cache_bytes(cfg, batch, max_len) bytes."""
+    _check(_lib().gpt2_prefill(ctx, _ptr(cache), _nbytes(cache), batch, max_len, _ptr(tokens), _ptr(prompt_len),
+                               _ptr(logits), _stream(stream)), "gpt2_prefill")
+
+
+def gpt2_decode_step(ctx, cache, batch, max_len, tokens, pos, logits, stream=None):
+    """cache: a device tensor of at least gpt2_kv_cache_bytes(cfg, batch, max_len) bytes."""
+    _check(_lib().gpt2_decode_step(ctx, _ptr(cache), _nbytes(cache), batch, max_len, _ptr(tokens), _ptr(pos),
+                                   _ptr(logits), _stream(stream)), "gpt2_decode_step")
+
+
+def gpt2_greedy_next(ctx, logits, batch, next_tokens, pos=None, stream=None):
+    _check(_lib().gpt2_greedy_next(ctx, _ptr(logits), batch, _ptr(next_tokens), _ptr(pos), _stream(stream)),
+           "gpt2_greedy_next")
 
 
 def gpt2_op_gemm_bf16(A, a_mn_major, lda, B, b_mn_major, ldb, C, c_fp32, ldc, M, N, K,
@@ -343,3 +375,42 @@ class GPT2:
                   eps=1e-8, weight_decay=0.1):
         gpt2_step_host(self.ctx, tokens_host, targets_host, tokens_host.shape[0], loss_host, lr, beta1,
                        beta2, eps, weight_decay, step)
+
+
+class KVCache:
+    """Key/value cache of one GPT2 context for ``batch`` sequences of up to
+    ``max_len`` positions, with the device-side token, position and logits
+    buffers a decode loop runs on (so the loop can be captured in a CUDA
+    graph)."""
+
+    def __init__(self, model: "GPT2", batch: int, max_len: int):
+        import torch
+        nbytes = gpt2_kv_cache_bytes(model.cfg, batch, max_len)
+        if nbytes == 0:
+            raise ValueError(f"invalid cache size batch={batch} max_len={max_len}")
+        dev = model.master.device
+        self.model, self.batch, self.max_len = model, batch, max_len
+        self.buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.tokens = torch.zeros(batch, dtype=torch.int32, device=dev)
+        self.pos = torch.zeros(batch, dtype=torch.int32, device=dev)
+        self.logits = torch.zeros(batch, model.cfg.vocab_padded, dtype=torch.float32, device=dev)
+
+    def prefill(self, tokens, prompt_len):
+        """tokens: int32 [batch, n_ctx] (device); prompt_len: int32 [batch]
+        (device).  Leaves the logits after each prompt in self.logits, the
+        greedy next id in self.tokens and self.pos = prompt_len."""
+        gpt2_prefill(self.model.ctx, self.buf, self.batch, self.max_len, tokens, prompt_len, self.logits)
+        self.pos.copy_(prompt_len)
+        gpt2_greedy_next(self.model.ctx, self.logits, self.batch, self.tokens)
+        return self.logits
+
+    def step(self, tokens=None, pos=None):
+        """One decode step on self.tokens / self.pos (or the given device
+        tensors); returns the logits [batch, vocab_padded]."""
+        gpt2_decode_step(self.model.ctx, self.buf, self.batch, self.max_len,
+                         self.tokens if tokens is None else tokens, self.pos if pos is None else pos, self.logits)
+        return self.logits
+
+    def greedy_advance(self):
+        """self.tokens = greedy choice from self.logits; self.pos += 1."""
+        gpt2_greedy_next(self.model.ctx, self.logits, self.batch, self.tokens, self.pos)

@@ -14,7 +14,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libgpt2.so")
 SOURCES = ["gemm_tc.cu", "gemm_simt.cu", "attention.cu", "attention_tc.cu", "attention_noalloc.cu", "kernels.cu",
-           "gpt2.cu"]
+           "decode.cu", "gpt2.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr"]

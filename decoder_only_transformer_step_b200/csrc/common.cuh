@@ -16,6 +16,7 @@ enum : int {
   DEV_ERR_TOKEN = 1,
   DEV_ERR_NONFINITE = 2,
   DEV_ERR_TIMEOUT = 4,
+  DEV_ERR_POSITION = 8,
 };
 
 // A pipeline wait that has not completed after this long is treated as a

@@ -387,19 +387,17 @@ int gpt2_zero_grad(gpt2_ctx* c, void* stream) {
   return fill_zero(c->buf.grad, c->off.total() * 4, S(stream));
 }
 
-int gpt2_forward_loss(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets, int batch, float* loss_dev,
-                      void* stream) {
-  if (!c || !tokens || !targets) return GPT2_ERR_INVALID_ARG;
-  if (batch < 1 || batch > c->cfg.max_batch) return GPT2_ERR_INVALID_ARG;
+namespace {
+
+// The forward up to the logits [batch * T, V] in w.logits; every layer's
+// activations stay in the workspace.
+int forward_logits(gpt2_ctx* c, const int32_t* tokens, int batch, cudaStream_t st) {
   const Shape& s = c->s;
   const int M = batch * (int)s.T, d = (int)s.d, V = (int)s.V;
-  if (s.mode == 0 && M % 64) return GPT2_ERR_UNSUPPORTED_SHAPE;
-  cudaStream_t st = S(stream);
   Work& w = c->w;
   const Offsets& o = c->off;
   const int f32 = s.mode;
   CUDA_TRY(cudaMemcpyAsync(w.tok, tokens, (size_t)M * 4, cudaMemcpyDeviceToDevice, st));
-  CUDA_TRY(cudaMemcpyAsync(w.tgt, targets, (size_t)M * 4, cudaMemcpyDeviceToDevice, st));
   c->have_fwd = 0;
 
   TRY(embed_fwd(f32, w.tok, Wp(c, o.wte()), Wp(c, o.wpe()), w.layers[0].x_in, M, (int)s.T, d, (int)s.Vr, w.err,
@@ -434,6 +432,23 @@ int gpt2_forward_loss(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets
   TRY(layernorm_fwd(f32, w.x_final, Wp(c, o.lnf_g()), Wp(c, o.lnf_b()), w.yf, w.meanf, w.rstdf, M, d, st));
   GemmArgs g = make_gemm(M, V, d, w.yf, 0, d, Wp(c, o.wte()), 0, d, EPI_STORE, w.logits, V);
   TRY(run_gemm(c, g, st));
+  return GPT2_OK;
+}
+
+}  // namespace
+
+int gpt2_forward_loss(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets, int batch, float* loss_dev,
+                      void* stream) {
+  if (!c || !tokens || !targets) return GPT2_ERR_INVALID_ARG;
+  if (batch < 1 || batch > c->cfg.max_batch) return GPT2_ERR_INVALID_ARG;
+  const Shape& s = c->s;
+  const int M = batch * (int)s.T, V = (int)s.V;
+  if (s.mode == 0 && M % 64) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = S(stream);
+  Work& w = c->w;
+  const int f32 = s.mode;
+  CUDA_TRY(cudaMemcpyAsync(w.tgt, targets, (size_t)M * 4, cudaMemcpyDeviceToDevice, st));
+  TRY(forward_logits(c, tokens, batch, st));
   TRY(count_targets(w.tgt, M, (int)s.Vr, w.n_valid, w.err, st));
   TRY(ce_fwd(f32, w.logits, w.tgt, w.loss_rows, M, V, (int)s.Vr, w.n_valid, w.err, st));
   TRY(loss_mean(w.loss_rows, M, w.n_valid, loss_dev ? loss_dev : w.loss, w.err, st));
@@ -561,7 +576,130 @@ int gpt2_get_status(gpt2_ctx* c, void* stream) {
   if (h & DEV_ERR_TIMEOUT) return GPT2_ERR_TIMEOUT;
   if (h & DEV_ERR_NONFINITE) return GPT2_ERR_NONFINITE;
   if (h & DEV_ERR_TOKEN) return GPT2_ERR_TOKEN_RANGE;
+  if (h & DEV_ERR_POSITION) return GPT2_ERR_POSITION_RANGE;
   return GPT2_OK;
+}
+
+// ------------------------------------------------ incremental decoding ----
+
+namespace {
+
+// The cache: K and V planes [batch][H][max_len][hd] (compute dtype) of every
+// layer, layer-major (K of layer l, then V of layer l), then the decode
+// step's fp32 rows x (residual stream), q, o [batch, d] and g [batch, 4d].
+struct DecodeLayout {
+  uint8_t* base = nullptr;
+  size_t plane_bytes = 0;
+  float *x = nullptr, *q = nullptr, *o = nullptr, *g = nullptr;
+  size_t total = 0;
+  void* k(int l) const { return base + (size_t)(2 * l) * plane_bytes; }
+  void* v(int l) const { return base + (size_t)(2 * l + 1) * plane_bytes; }
+};
+
+constexpr int DECODE_MAX_BATCH = 16;
+
+bool decode_layout(const Shape& s, int batch, int max_len, void* cache, DecodeLayout* dl) {
+  if (batch < 1 || batch > DECODE_MAX_BATCH || max_len < 1 || max_len > s.T) return false;
+  const size_t es = s.mode ? 4 : 2;
+  dl->base = reinterpret_cast<uint8_t*>(cache);
+  dl->plane_bytes = ((size_t)batch * s.H * max_len * s.hd * es + 255) & ~(size_t)255;
+  size_t off = (size_t)(2 * s.L) * dl->plane_bytes;
+  auto take = [&](size_t floats) {
+    float* p = cache ? reinterpret_cast<float*>(dl->base + off) : nullptr;
+    off += (floats * 4 + 255) & ~(size_t)255;
+    return p;
+  };
+  dl->x = take((size_t)batch * s.d);
+  dl->q = take((size_t)batch * s.d);
+  dl->o = take((size_t)batch * s.d);
+  dl->g = take((size_t)batch * 4 * s.d);
+  dl->total = off;
+  return true;
+}
+
+int decode_check(gpt2_ctx* c, void* cache, size_t cache_bytes, int batch, int max_len, DecodeLayout* dl) {
+  if (!c || !cache || ((uintptr_t)cache & 255)) return GPT2_ERR_INVALID_ARG;
+  if (!decode_layout(c->s, batch, max_len, cache, dl)) return GPT2_ERR_INVALID_ARG;
+  if (dl->total > cache_bytes) return GPT2_ERR_INVALID_ARG;  // sized for another (batch, max_len)
+  if (decode_gemv_smem(c->s.mode, batch, (int)(4 * c->s.d)) > 227 * 1024) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  return GPT2_OK;
+}
+
+}  // namespace
+
+size_t gpt2_kv_cache_bytes(const gpt2_config* cfg, int batch, int max_len) {
+  Shape s;
+  DecodeLayout dl;
+  if (!shape_from_cfg(cfg, &s) || !decode_layout(s, batch, max_len, nullptr, &dl)) return 0;
+  return dl.total;
+}
+
+int gpt2_decode_step(gpt2_ctx* c, void* cache, size_t cache_bytes, int batch, int max_len, const int32_t* tokens,
+                     const int32_t* pos, float* logits, void* stream) {
+  DecodeLayout dl;
+  TRY(decode_check(c, cache, cache_bytes, batch, max_len, &dl));
+  if (!tokens || !pos || !logits) return GPT2_ERR_INVALID_ARG;
+  const Shape& s = c->s;
+  const Offsets& o = c->off;
+  const int f32 = s.mode, d = (int)s.d;
+  cudaStream_t st = S(stream);
+  TRY(decode_embed(f32, tokens, pos, Wp(c, o.wte()), Wp(c, o.wpe()), dl.x, batch, d, (int)s.Vr, max_len, c->w.err,
+                   st));
+  DecodeGemv g;
+  memset(&g, 0, sizeof(g));
+  g.rows = batch;
+  g.pos = pos;
+  g.d = d; g.H = (int)s.H; g.hd = (int)s.hd; g.max_len = max_len;
+  for (int l = 0; l < (int)s.L; ++l) {
+    // LN1 -> QKV (+ bias): q to dl.q, k and v into the cache at pos
+    g.in = dl.x; g.in_t = 0; g.W = Wp(c, o.layer(l, W_QKV)); g.bias = Wp(c, o.layer(l, B_QKV));
+    g.ln = 1; g.ln_g = Wp(c, o.layer(l, LN1_G)); g.ln_b = Wp(c, o.layer(l, LN1_B));
+    g.epi = DECODE_QKV; g.out = dl.q; g.ldo = d; g.N = 3 * d; g.K = d;
+    g.kc = dl.k(l); g.vc = dl.v(l);
+    TRY(decode_gemv(f32, g, st));
+    TRY(decode_attention(f32, dl.k(l), dl.v(l), dl.q, dl.o, pos, batch, (int)s.H, (int)s.hd, max_len, st));
+    // x += o W_o^T + b_o
+    g.in = dl.o; g.in_t = 0; g.W = Wp(c, o.layer(l, W_O)); g.bias = Wp(c, o.layer(l, B_O));
+    g.ln = 0; g.epi = DECODE_RESID; g.out = dl.x; g.ldo = d; g.N = d; g.K = d;
+    TRY(decode_gemv(f32, g, st));
+    // LN2 -> fc (+ bias) -> GELU
+    g.in = dl.x; g.in_t = 0; g.W = Wp(c, o.layer(l, W_FC)); g.bias = Wp(c, o.layer(l, B_FC));
+    g.ln = 1; g.ln_g = Wp(c, o.layer(l, LN2_G)); g.ln_b = Wp(c, o.layer(l, LN2_B));
+    g.epi = DECODE_GELU; g.out = dl.g; g.ldo = 4 * d; g.N = 4 * d; g.K = d;  // GELU(u) in the compute dtype
+    TRY(decode_gemv(f32, g, st));
+    // x += g W_mp^T + b_mp
+    g.in = dl.g; g.in_t = 1; g.W = Wp(c, o.layer(l, W_MP)); g.bias = Wp(c, o.layer(l, B_MP));
+    g.ln = 0; g.epi = DECODE_RESID; g.out = dl.x; g.ldo = d; g.N = d; g.K = 4 * d;
+    TRY(decode_gemv(f32, g, st));
+  }
+  // final LN -> tied LM head
+  g.in = dl.x; g.in_t = 0; g.W = Wp(c, o.wte()); g.bias = nullptr;
+  g.ln = 1; g.ln_g = Wp(c, o.lnf_g()); g.ln_b = Wp(c, o.lnf_b());
+  g.epi = DECODE_LOGITS; g.out = logits; g.ldo = s.V; g.N = (int)s.V; g.K = d;
+  return decode_gemv(f32, g, st);
+}
+
+int gpt2_prefill(gpt2_ctx* c, void* cache, size_t cache_bytes, int batch, int max_len, const int32_t* tokens,
+                 const int32_t* prompt_len, float* logits, void* stream) {
+  DecodeLayout dl;
+  TRY(decode_check(c, cache, cache_bytes, batch, max_len, &dl));
+  if (!tokens || !prompt_len || !logits) return GPT2_ERR_INVALID_ARG;
+  if (batch > c->cfg.max_batch) return GPT2_ERR_INVALID_ARG;
+  const Shape& s = c->s;
+  if (s.mode == 0 && (batch * s.T) % 64) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = S(stream);
+  const int f32 = s.mode;
+  TRY(forward_logits(c, tokens, batch, st));
+  for (int l = 0; l < (int)s.L; ++l)
+    TRY(prefill_kv(f32, c->w.layers[l].qkv, dl.k(l), dl.v(l), prompt_len, batch, (int)s.T, (int)s.H, (int)s.hd,
+                   max_len, max_len, c->w.err, st));
+  return prefill_logits(f32, c->w.logits, prompt_len, logits, batch, (int)s.T, (int)s.V, max_len, st);
+}
+
+int gpt2_greedy_next(gpt2_ctx* c, const float* logits, int batch, int32_t* next_tokens, int32_t* pos,
+                     void* stream) {
+  if (!c || !logits || !next_tokens || batch < 1) return GPT2_ERR_INVALID_ARG;
+  return decode_greedy(logits, c->s.V, batch, (int)c->s.Vr, next_tokens, pos, S(stream));
 }
 
 int gpt2_step_host(gpt2_ctx* c, const int32_t* tokens_host, const int32_t* targets_host, int batch,
@@ -595,6 +733,7 @@ const char* gpt2_strerror(int code) {
     case GPT2_ERR_TIMEOUT: return "device pipeline wait timed out";
     case GPT2_ERR_WORKSPACE: return "workspace too small";
     case GPT2_ERR_TOO_LARGE: return "problem exceeds the built-in scratch of the allocation-free entry point";
+    case GPT2_ERR_POSITION_RANGE: return "decode position or prompt length out of range";
     default: return "unknown error";
   }
 }

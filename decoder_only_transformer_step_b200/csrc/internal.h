@@ -124,3 +124,36 @@ int init_params(float* p, size_t n, const LayoutDims& ld, uint64_t seed, cudaStr
 int cast_shadow(const float* p, uint16_t* shadow, size_t n, cudaStream_t st);
 int fill_zero(void* p, size_t bytes, cudaStream_t st);
 int f32_to_act(int f32, const float* src, void* dst, long n, float scale, cudaStream_t st);
+
+// ---- incremental decoding (key/value cache) -----------------------------
+// One fused GEMV of the decode step: out[r, n] = epi(sum_k in'[r, k] W[n, k])
+// for r < rows (<= 16), in' = the input row, LayerNorm'd first if ln.
+enum DecodeEpiKind : int { DECODE_QKV = 0, DECODE_RESID = 1, DECODE_GELU = 2, DECODE_LOGITS = 3 };
+struct DecodeGemv {
+  const void* in;  // fp32 rows, or compute-dtype rows when in_t
+  int in_t;
+  const void* W;
+  const void* bias;
+  const void* ln_g;
+  const void* ln_b;
+  void* out;  // compute dtype for DECODE_GELU, else fp32
+  long ldo;
+  int rows, N, K;
+  int ln, epi;
+  void* kc;  // DECODE_QKV: this layer's K and V cache planes
+  void* vc;
+  const int32_t* pos;
+  int d, H, hd, max_len;
+};
+size_t decode_gemv_smem(int f32, int rows, int K);
+int decode_gemv(int f32, const DecodeGemv& g, cudaStream_t st);
+int decode_embed(int f32, const int32_t* tok, const int32_t* pos, const void* wte, const void* wpe, float* x,
+                 int rows, int d, int vocab_real, int limit, int* err, cudaStream_t st);
+int decode_attention(int f32, const void* kc, const void* vc, const float* q, float* o, const int32_t* pos,
+                     int rows, int H, int hd, int max_len, cudaStream_t st);
+int decode_greedy(const float* logits, long ld, int rows, int vocab_real, int32_t* next, int32_t* pos,
+                  cudaStream_t st);
+int prefill_kv(int f32, const void* qkv, void* kc, void* vc, const int32_t* plen, int rows, int T, int H, int hd,
+               int max_len, int limit, int* err, cudaStream_t st);
+int prefill_logits(int f32, const void* logits, const int32_t* plen, float* out, int rows, int T, int V, int limit,
+                   cudaStream_t st);

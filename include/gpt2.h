@@ -63,7 +63,8 @@ enum {
   GPT2_ERR_NONFINITE = -6,        /* device: loss is NaN or Inf */
   GPT2_ERR_TIMEOUT = -7,          /* device: a bounded pipeline wait ran out */
   GPT2_ERR_WORKSPACE = -8,        /* workspace smaller than gpt2_workspace_bytes */
-  GPT2_ERR_TOO_LARGE = -9         /* problem exceeds the built-in scratch of an allocation-free entry point */
+  GPT2_ERR_TOO_LARGE = -9,        /* problem exceeds the built-in scratch of an allocation-free entry point */
+  GPT2_ERR_POSITION_RANGE = -10   /* device: a decode position or prompt length out of range (row 0 / skipped) */
 };
 
 typedef struct {
@@ -165,7 +166,8 @@ int gpt2_adamw_step_clip(gpt2_ctx* ctx, float lr, float beta1, float beta2, floa
 int gpt2_zero_grad(gpt2_ctx* ctx, void* stream);
 
 /* Synchronises `stream`, returns and clears the latched device status
- * (GPT2_OK, GPT2_ERR_TOKEN_RANGE, GPT2_ERR_NONFINITE or GPT2_ERR_TIMEOUT),
+ * (GPT2_OK, GPT2_ERR_TOKEN_RANGE, GPT2_ERR_NONFINITE, GPT2_ERR_TIMEOUT or
+ * GPT2_ERR_POSITION_RANGE),
  * or GPT2_ERR_CUDA if the stream reports an error. */
 int gpt2_get_status(gpt2_ctx* ctx, void* stream);
 
@@ -183,6 +185,63 @@ const char* gpt2_strerror(int code);
 /* Number of CUDA kernels this library has launched in this process so far
  * (all contexts and entry points); a diagnostic for launch accounting. */
 uint64_t gpt2_kernel_launches(void);
+
+/* ------------------------------------------------------------------------
+ * Incremental decoding with a key/value cache: the inference forward of the
+ * sampling loop ("Criei GPT-2 do zero com uma RTX 4090", sections "Vendo o
+ * modelo ficar mais inteligente aos poucos" and "Conversando de verdade com
+ * ele": the model continues a prompt one token at a time).  The logits a
+ * decode step returns for a row whose token sits at position p are the
+ * forward's logits at position p for that row's tokens 0..p; the cache holds
+ * every layer's K and V of positions 0..p-1 so that only the new position is
+ * computed.  Weights are the ones the forward uses (bf16 shadow in mode 0,
+ * fp32 master in mode 1); the cache holds K and V in that dtype, and the
+ * residual stream of a step stays fp32.
+ *
+ * A cache is sized for (batch, max_len): 1 <= batch <= 16, 1 <= max_len <=
+ * n_ctx.  Every call on it passes the same batch and max_len, and the
+ * buffer's size in bytes (cache_bytes): a call whose (batch, max_len) needs
+ * more than cache_bytes is GPT2_ERR_INVALID_ARG before anything is enqueued.
+ * It is one caller-owned device buffer of at least gpt2_kv_cache_bytes bytes,
+ * 256-byte aligned;
+ * layout: per layer l the K plane then the V plane, each [batch][n_head]
+ * [max_len][head_dim] (padded to 256 bytes), then the step's fp32 scratch.
+ * Positions are per row (device int32 [batch]), so rows may sit at different
+ * positions.  A position outside [0, max_len), a prompt length outside
+ * [1, max_len] or an id outside [0, vocab_real) latches
+ * GPT2_ERR_POSITION_RANGE / GPT2_ERR_TOKEN_RANGE for gpt2_get_status (the
+ * row then reads id 0 / position 0 and its cache write is skipped).
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of a cache for (batch, max_len); 0 if the configuration or the
+ * sizes are invalid. */
+size_t gpt2_kv_cache_bytes(const gpt2_config* cfg, int batch, int max_len);
+
+/* Prompt processing: runs the training forward over tokens (device int32
+ * [batch, n_ctx]; batch <= max_batch; ids past a row's prompt are any valid
+ * id, causality keeps them out of the prompt's results), copies K and V of
+ * positions < prompt_len[b] (device int32 [batch]) into the cache, and writes
+ * the logits after each row's last prompt token to logits (device fp32
+ * [batch, vocab_padded]).  Overwrites the forward's activations (a following
+ * gpt2_backward returns GPT2_ERR_BAD_STATE). */
+int gpt2_prefill(gpt2_ctx* ctx, void* cache, size_t cache_bytes, int batch, int max_len,
+                 const int32_t* tokens, const int32_t* prompt_len, float* logits, void* stream);
+
+/* One decode step: row b feeds tokens[b] (device int32 [batch]) at position
+ * pos[b] (device int32 [batch]), writes its K and V into the cache at pos[b],
+ * attends to positions 0..pos[b] and writes the next-token logits to logits
+ * (device fp32 [batch, vocab_padded]).  tokens and pos are read on the device,
+ * so a loop of steps can be captured in one CUDA graph. */
+int gpt2_decode_step(gpt2_ctx* ctx, void* cache, size_t cache_bytes, int batch, int max_len,
+                     const int32_t* tokens, const int32_t* pos, float* logits, void* stream);
+
+/* Greedy choice: next_tokens[b] = the id v < vocab_real with the largest
+ * logits[b, v] (device fp32 [batch, vocab_padded]); the lowest id among equal
+ * maxima, the first NaN if a row holds one.  If pos (device int32 [batch]) is
+ * not NULL, pos[b] += 1, so next_tokens and pos feed the next decode step.
+ * The pages give no sampling rule; greedy is the plainest. */
+int gpt2_greedy_next(gpt2_ctx* ctx, const float* logits, int batch, int32_t* next_tokens, int32_t* pos,
+                     void* stream);
 
 /* ------------------------------------------------------------------------
  * Single-operation entry points used by the kernel unit tests.  They run the

@@ -96,3 +96,16 @@ def test_invalid_configs_are_rejected_on_host():
     assert lib.gpt2_create(ctypes.byref(cfg), ctypes.byref(fake), ctypes.byref(ctx)) == -8
     assert lib.gpt2_backward(None, ctypes.c_float(1.0), 0, None) == -1
     assert lib.gpt2_strerror(-5) == b"token or target id out of range"
+
+
+def test_kv_cache_bytes_layout():
+    # K and V planes [batch][H][max_len][hd] of every layer (bf16 in mode 0,
+    # fp32 in mode 1, each padded to 256 bytes) plus four fp32 row buffers
+    c = gp.GPT2_124M.c()
+    planes = 2 * 12 * 8 * 12 * 1024 * 64 * 2
+    scratch = 3 * 8 * 768 * 4 + 8 * 3072 * 4
+    assert gp.gpt2_kv_cache_bytes(c, 8, 1024) == planes + scratch
+    c1 = gp.GPT2_TINY.c()
+    assert gp.gpt2_kv_cache_bytes(c1, 1, 5) == 2 * 2 * (4 * 5 * 16 * 4) + 3 * 64 * 4 + 256 * 4
+    for b, n in [(0, 8), (17, 8), (4, 0), (4, 1025)]:
+        assert gp.gpt2_kv_cache_bytes(c, b, n) == 0
