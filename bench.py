@@ -116,7 +116,7 @@ def run_ours(args, rank, world, local_rank):
 
     import decoder_only_transformer_step_b200 as gp
     from decoder_only_transformer_step_b200 import inputs, flops
-    from decoder_only_transformer_step_b200.dp import average_gradients
+    from decoder_only_transformer_step_b200.dp import average_gradients, zero1_step
 
     torch.cuda.set_device(local_rank)
     if world > 1:
@@ -135,13 +135,23 @@ def run_ours(args, rank, world, local_rank):
         pool.append((torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda()))
     stream = torch.cuda.current_stream()
 
+    def optimizer_step(step_no):
+        # gradient exchange + AdamW: one all-reduce and the full update, or with
+        # --zero1 a reduce-scatter, the update of this rank's shard and an
+        # all-gather of the weights
+        if world > 1 and args.zero1:
+            zero1_step(model.grad, model.master, lambda off, cnt: model.adamw_step_range(step_no, off, cnt),
+                       model.refresh_shadow)
+            return
+        if world > 1:
+            average_gradients(model.grad)
+        model.adamw_step(step_no)
+
     def step(i):
         tok, tgt = pool[i % len(pool)]
         model.forward_loss(tok, tgt)
         model.backward(1.0, 0)
-        if world > 1:
-            average_gradients(model.grad)
-        model.adamw_step(i + 1)
+        optimizer_step(i + 1)
 
     for i in range(args.warmup):
         step(i)
@@ -190,8 +200,7 @@ def run_ours(args, rank, world, local_rank):
             tgt = tgt_h[i % 2].cuda(non_blocking=True)
             model.forward_loss(tok, tgt)
             model.backward(1.0, 0)
-            average_gradients(model.grad)
-            model.adamw_step(args.warmup + args.steps + i + 1)
+            optimizer_step(args.warmup + args.steps + i + 1)
             loss_h.copy_(model.loss)
             torch.cuda.synchronize()
 
@@ -221,9 +230,7 @@ def run_ours(args, rank, world, local_rank):
                 tok, tgt = pool[(i * k + j) % len(pool)]
                 model.forward_loss(tok, tgt)
                 model.backward(1.0 / k, 1 if j else 0)
-            if world > 1:
-                average_gradients(model.grad)
-            model.adamw_step(args.warmup + args.steps + e_steps + 2 + i)
+            optimizer_step(args.warmup + args.steps + e_steps + 2 + i)
 
         a_steps = 2
         accum_step(0)
@@ -266,7 +273,7 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic Zipf(1.1) token ids over [0, 50257), random-init GPT-2 weights",
         "config": {"workload": workload_name(args.config, CONFIGS[args.config]), "batch_per_gpu": B,
-                   "seq_len": T, "parallelism": f"dp{world}",
+                   "seq_len": T, "parallelism": f"dp{world}" + ("-zero1" if world > 1 and args.zero1 else ""),
                    "l2": "inputs larger than L2: the step's working set (>5 GB) exceeds the 126 MB L2"},
         "mfu": round(flops.mfu(tokens_per_s / world, fpt, peaks["bf16_tflops"] * 1e12), 4),
         "mfu_vs_sustained": round(flops.mfu(tokens_per_s / world, fpt, peaks["bf16_tflops_sustained"] * 1e12), 4),
@@ -540,6 +547,9 @@ def main():
                     help="also time optimizer steps with this many accumulated micro-batches (0 or 1: skip)")
     ap.add_argument("--decode-steps", type=int, default=64,
                     help="also time this many greedy KV-cache decode steps at batch 8 (0: skip)")
+    ap.add_argument("--zero1", action="store_true",
+                    help="N>1: shard the AdamW state (reduce-scatter, own-shard update, all-gather) instead of "
+                         "an all-reduce and the full update")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

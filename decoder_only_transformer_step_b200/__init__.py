@@ -48,7 +48,7 @@ class gpt2_buffers(ctypes.Structure):
 EXPORTS = [
     "gpt2_param_count", "gpt2_workspace_bytes", "gpt2_tensor_info", "gpt2_create", "gpt2_destroy",
     "gpt2_init_params", "gpt2_refresh_shadow", "gpt2_forward_loss", "gpt2_backward",
-    "gpt2_adamw_step", "gpt2_adamw_step_clip", "gpt2_grad_norm", "gpt2_zero_grad", "gpt2_get_status", "gpt2_step_host", "gpt2_strerror",
+    "gpt2_adamw_step", "gpt2_adamw_step_clip", "gpt2_adamw_step_range", "gpt2_grad_norm", "gpt2_zero_grad", "gpt2_get_status", "gpt2_step_host", "gpt2_strerror",
     "gpt2_kernel_launches",
     "gpt2_kv_cache_bytes", "gpt2_prefill", "gpt2_decode_step", "gpt2_greedy_next",
     "gpt2_op_gemm_bf16", "gpt2_op_attention_fwd_bf16", "gpt2_op_attention_bwd_bf16",
@@ -81,6 +81,7 @@ def _lib():
         "gpt2_backward": (I, [P, F, I, P]),
         "gpt2_adamw_step": (I, [P, F, F, F, F, F, I, P]),
         "gpt2_adamw_step_clip": (I, [P, F, F, F, F, F, I, F, P]),
+        "gpt2_adamw_step_range": (I, [P, F, F, F, F, F, I, S, S, P]),
         "gpt2_grad_norm": (I, [P, P, P]),
         "gpt2_zero_grad": (I, [P, P]),
         "gpt2_get_status": (I, [P, P]),
@@ -192,6 +193,11 @@ def gpt2_adamw_step(ctx, lr, beta1, beta2, eps, weight_decay, step, stream=None)
 def gpt2_adamw_step_clip(ctx, lr, beta1, beta2, eps, weight_decay, step, max_norm, stream=None):
     _check(_lib().gpt2_adamw_step_clip(ctx, lr, beta1, beta2, eps, weight_decay, step, max_norm,
                                        _stream(stream)), "gpt2_adamw_step_clip")
+
+
+def gpt2_adamw_step_range(ctx, lr, beta1, beta2, eps, weight_decay, step, offset, count, stream=None):
+    _check(_lib().gpt2_adamw_step_range(ctx, lr, beta1, beta2, eps, weight_decay, step, offset, count,
+                                        _stream(stream)), "gpt2_adamw_step_range")
 
 
 def gpt2_grad_norm(ctx, norm_dev=None, stream=None):
@@ -357,6 +363,11 @@ class GPT2:
             gpt2_adamw_step_clip(self.ctx, lr, beta1, beta2, eps, weight_decay, step, max_norm)
         else:
             gpt2_adamw_step(self.ctx, lr, beta1, beta2, eps, weight_decay, step)
+
+    def adamw_step_range(self, step, offset, count, lr=6e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1):
+        """AdamW on elements [offset, offset + count) only (one shard of the
+        optimizer state)."""
+        gpt2_adamw_step_range(self.ctx, lr, beta1, beta2, eps, weight_decay, step, offset, count)
 
     def grad_norm(self):
         """Global L2 norm of the gradient buffer as a device fp32 scalar tensor."""

@@ -546,6 +546,19 @@ int gpt2_adamw_step(gpt2_ctx* c, float lr, float beta1, float beta2, float eps, 
                c->off.total(), ld, a, nullptr, 0.f, S(stream));
 }
 
+int gpt2_adamw_step_range(gpt2_ctx* c, float lr, float beta1, float beta2, float eps, float weight_decay,
+                          int step, size_t offset, size_t count, void* stream) {
+  if (!c || step < 1 || offset % 4 || count % 4 || offset > c->off.total() || count > c->off.total() - offset)
+    return GPT2_ERR_INVALID_ARG;
+  AdamArgs a;
+  a.lr = lr; a.beta1 = beta1; a.beta2 = beta2; a.eps = eps; a.wd = weight_decay;
+  a.bc1 = (float)(1.0 - pow((double)beta1, (double)step));
+  a.bc2 = (float)(1.0 - pow((double)beta2, (double)step));
+  LayoutDims ld{c->s.V, c->s.T, c->s.d, c->s.L};
+  return adamw(c->buf.master, c->buf.grad, c->buf.m, c->buf.v, c->s.mode ? nullptr : c->buf.shadow, count, ld, a,
+               nullptr, 0.f, S(stream), offset);
+}
+
 int gpt2_grad_norm(gpt2_ctx* c, float* norm_dev, void* stream) {
   if (!c) return GPT2_ERR_INVALID_ARG;
   if (norm_dev && ((uintptr_t)norm_dev & 3)) return GPT2_ERR_INVALID_ARG;

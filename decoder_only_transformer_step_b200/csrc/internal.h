@@ -115,8 +115,10 @@ struct LayoutDims {
   long V, T, d, L;
 };
 // gnorm (device scalar, may be NULL): clip the gradient to global norm max_norm.
+// Updates elements [base, base + n) of the flat buffers (base, n multiples of 4).
 int adamw(float* p, const float* g, float* m, float* v, uint16_t* shadow, size_t n,
-          const LayoutDims& ld, const AdamArgs& a, const float* gnorm, float max_norm, cudaStream_t st);
+          const LayoutDims& ld, const AdamArgs& a, const float* gnorm, float max_norm, cudaStream_t st,
+          size_t base = 0);
 // ||g||_2 of n floats (n % 4 == 0) into *norm; part holds GRAD_NORM_PARTS floats.
 constexpr int GRAD_NORM_PARTS = 592;
 int grad_norm(const float* g, size_t n, float* part, float* norm, cudaStream_t st);

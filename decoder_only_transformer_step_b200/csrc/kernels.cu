@@ -750,9 +750,11 @@ __global__ void __launch_bounds__(256) norm_final_kernel(const float* __restrict
 
 // With gnorm != NULL the gradient is first scaled by min(1, max_norm / (gnorm + 1e-6))
 // (global-norm clipping).
+// Elements [base, base + 4 n4) of the flat buffers; the pointers point at
+// element base, whose layout position decides the weight-decay mask.
 __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
-                             float* __restrict__ v, uint16_t* __restrict__ shadow, long n4, LayoutDims L,
-                             AdamArgs a, const float* __restrict__ gnorm, float max_norm) {
+                             float* __restrict__ v, uint16_t* __restrict__ shadow, long n4, long base,
+                             LayoutDims L, AdamArgs a, const float* __restrict__ gnorm, float max_norm) {
   pdl_start();
   float clip = 1.f;
   if (gnorm) {
@@ -760,7 +762,7 @@ __global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
     clip = c < 1.f ? c : 1.f;
   }
   for (long i4 = blockIdx.x * (long)blockDim.x + threadIdx.x; i4 < n4; i4 += (long)gridDim.x * blockDim.x) {
-    const long i = i4 * 4;
+    const long i = base + i4 * 4;
     int one;
     const bool decay = tensor_kind(i, L, &one) != 0;
     float4 pp = reinterpret_cast<float4*>(p)[i4];
@@ -1071,9 +1073,11 @@ int grad_norm(const float* g, size_t n, float* part, float* norm, cudaStream_t s
 }
 
 int adamw(float* p, const float* g, float* m, float* v, uint16_t* shadow, size_t n, const LayoutDims& ld,
-          const AdamArgs& a, const float* gnorm, float max_norm, cudaStream_t st) {
+          const AdamArgs& a, const float* gnorm, float max_norm, cudaStream_t st, size_t base) {
   const long n4 = (long)(n / 4);
-  CUDA_TRY(launch_k(adamw_kernel, grid_for(n4, 256), 256, 0, st, p, g, m, v, shadow, n4, ld, a, gnorm, max_norm));
+  if (n4 == 0) return GPT2_OK;
+  CUDA_TRY(launch_k(adamw_kernel, grid_for(n4, 256), 256, 0, st, p + base, g + base, m + base, v + base,
+                    shadow ? shadow + base : nullptr, n4, (long)base, ld, a, gnorm, max_norm));
   LAUNCH_CHECK();
   return GPT2_OK;
 }

@@ -162,6 +162,17 @@ int gpt2_grad_norm(gpt2_ctx* ctx, float* norm_dev, void* stream);
 int gpt2_adamw_step_clip(gpt2_ctx* ctx, float lr, float beta1, float beta2, float eps,
                          float weight_decay, int step, float max_norm, void* stream);
 
+/* gpt2_adamw_step restricted to elements [offset, offset + count) of the flat
+ * buffers (master, m, v, the bf16 shadow; grad read there); offset and count
+ * are multiples of 4 and the range lies inside the layout, else
+ * GPT2_ERR_INVALID_ARG.  Each element gets exactly the update the full call
+ * gives it (the weight-decay mask follows the element's tensor).  This is the
+ * optimizer step of a rank that owns one shard of the optimizer state
+ * (data parallelism with sharded AdamW state: reduce-scatter the gradient,
+ * update the own shard, all-gather the weights). */
+int gpt2_adamw_step_range(gpt2_ctx* ctx, float lr, float beta1, float beta2, float eps,
+                          float weight_decay, int step, size_t offset, size_t count, void* stream);
+
 /* grad <- 0. */
 int gpt2_zero_grad(gpt2_ctx* ctx, void* stream);
 

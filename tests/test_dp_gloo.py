@@ -55,3 +55,74 @@ def test_two_rank_gradient_average():
     for r in range(world):
         np.testing.assert_allclose(out[r][0], full, rtol=1e-12, atol=1e-15)
     np.testing.assert_array_equal(out[0][1], out[1][1])
+
+
+# ----------------------------------------- sharded optimizer state (ZeRO-1) ---
+
+def _zero1_worker(rank, world, port, out):
+    import sys
+    sys.path.insert(0, os.path.dirname(__file__))
+    from oracle_fixtures import TINY, params_for
+    from decoder_only_transformer_step_b200.dp import zero1_step
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    params = params_for(TINY, seed=92)
+    tok, tgt = inputs.uniform_tokens(2 * world, 32, TINY.vocab, seed=93)
+    mine = slice(2 * rank, 2 * rank + 2)
+    _, cache = forward(params, TINY, tok[mine], tgt[mine])
+    g_local = flatten(backward(params, TINY, cache), TINY)
+    master = torch.from_numpy(flatten(params, TINY))
+    m = np.zeros(master.numel())
+    v = np.zeros(master.numel())
+    refreshed = []
+    for step in (1, 2):
+        grad = torch.from_numpy(g_local.copy())
+
+        def local_update(off, cnt, step=step, grad=grad):
+            # stand-in for the library's range update: the oracle's AdamW over
+            # the whole buffer, of which only this rank's shard is kept
+            P, Mo, Vo = adamw_step(unflatten(master.numpy(), TINY), unflatten(grad.numpy(), TINY),
+                                   unflatten(m, TINY), unflatten(v, TINY), step, TINY)
+            sl = slice(off, off + cnt)
+            master[sl] = torch.from_numpy(flatten(P, TINY)[sl])
+            m[sl] = flatten(Mo, TINY)[sl]
+            v[sl] = flatten(Vo, TINY)[sl]
+
+        zero1_step(grad, master, local_update, lambda: refreshed.append(step))
+    out[rank] = (master.numpy().copy(), refreshed)
+    dist.destroy_process_group()
+
+
+def test_two_rank_sharded_adamw_equals_full_step():
+    world = 2
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_zero1_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+    import sys
+    sys.path.insert(0, os.path.dirname(__file__))
+    from oracle_fixtures import TINY, params_for
+    params = params_for(TINY, seed=92)
+    tok, tgt = inputs.uniform_tokens(2 * world, 32, TINY.vocab, seed=93)
+    _, cache = forward(params, TINY, tok, tgt)
+    g = backward(params, TINY, cache)
+    zeros = {n: np.zeros(s) for n, s in param_shapes(TINY)}
+    P, Mo, Vo = adamw_step(params, g, zeros, zeros, 1, TINY)
+    P, _, _ = adamw_step(P, g, Mo, Vo, 2, TINY)
+    want = flatten(P, TINY)
+    for r in range(world):
+        np.testing.assert_allclose(out[r][0], want, rtol=1e-12, atol=1e-15)
+        assert list(out[r][1]) == [1, 2]
+
+
+def test_shard_ranges_partition_the_buffer():
+    from decoder_only_transformer_step_b200.dp import shard_range
+    import pytest
+    n = 124475904  # GPT-2 124M flat layout
+    for world in (1, 2, 4, 8):
+        rs = [shard_range(n, world, r) for r in range(world)]
+        assert rs[0][0] == 0 and sum(c for _, c in rs) == n
+        assert all(o % 4 == 0 and c % 4 == 0 for o, c in rs)
+        assert all(rs[i][0] + rs[i][1] == rs[i + 1][0] for i in range(world - 1))
+    with pytest.raises(ValueError):
+        shard_range(4 * 3 * 5 + 4, 3, 0)
