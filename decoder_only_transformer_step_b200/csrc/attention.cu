@@ -482,8 +482,8 @@ __global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ 
 }
 
 // dqkv[:, 0:d] = bf16(dq_acc)
-__global__ void dq_to_bf16_kernel(const float* __restrict__ dq_acc, bf16* __restrict__ dqkv, long M,
-                                  int d) {
+__global__ void dq_to_bf16_kernel(float* __restrict__ dq_acc, bf16* __restrict__ dqkv, long M, int d,
+                                  int zero_after) {
   pdl_start();
   long i = (blockIdx.x * (long)blockDim.x + threadIdx.x) * 4;
   if (i >= M * d) return;
@@ -492,6 +492,8 @@ __global__ void dq_to_bf16_kernel(const float* __restrict__ dq_acc, bf16* __rest
   float4 v = *reinterpret_cast<const float4*>(dq_acc + i);
   uint2 u = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
   *reinterpret_cast<uint2*>(dqkv + m * 3 * d + c) = u;
+  // the next layer's reduce-adds start from zero
+  if (zero_after) *reinterpret_cast<float4*>(dq_acc + i) = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // ------------------------------------------------------- fp32 (mode 1) ----
@@ -685,17 +687,19 @@ int attn_fwd_bf16(const void* qkv, void* o, float* lse, int B, int T, int H, int
 }
 
 int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* dout, void* dqkv,
-                  float* dq_acc, float* dvec, int B, int T, int H, int hd, cudaStream_t st) {
+                  float* dq_acc, float* dvec, int B, int T, int H, int hd, cudaStream_t st, int dvec_ready) {
   if (B <= 0 || T <= 0) return GPT2_OK;
   if (hd != 64 && hd != 16) return GPT2_ERR_UNSUPPORTED_SHAPE;
   const long M = (long)B * T;
-  if (hd == 64)
-    CUDA_TRY(launch_k(attn_bwd_prep_bf16_kernel<64>, (unsigned)((M + 7) / 8), 256, 0, st,
-        (const bf16*)o, (const bf16*)dout, dvec, dq_acc, M, T, H));
-  else
-    CUDA_TRY(launch_k(attn_bwd_prep_bf16_kernel<16>, (unsigned)((M + 7) / 8), 256, 0, st,
-        (const bf16*)o, (const bf16*)dout, dvec, dq_acc, M, T, H));
-  LAUNCH_CHECK();
+  if (!dvec_ready) {
+    if (hd == 64)
+      CUDA_TRY(launch_k(attn_bwd_prep_bf16_kernel<64>, (unsigned)((M + 7) / 8), 256, 0, st,
+          (const bf16*)o, (const bf16*)dout, dvec, dq_acc, M, T, H));
+    else
+      CUDA_TRY(launch_k(attn_bwd_prep_bf16_kernel<16>, (unsigned)((M + 7) / 8), 256, 0, st,
+          (const bf16*)o, (const bf16*)dout, dvec, dq_acc, M, T, H));
+    LAUNCH_CHECK();
+  }
   int rc = (hd == 64 && !use_mma_bwd() && T <= 4096)
                ? attn_bwd_tc(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st)
                : (hd == 64 ? launch_bwd<64>(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st)
@@ -703,7 +707,8 @@ int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* 
   if (rc) return rc;
   const int d = H * hd;
   long n4 = (M * d) / 4;
-  CUDA_TRY(launch_k(dq_to_bf16_kernel, (unsigned)((n4 + 255) / 256), 256, 0, st, dq_acc, (bf16*)dqkv, M, d));
+  CUDA_TRY(launch_k(dq_to_bf16_kernel, (unsigned)((n4 + 255) / 256), 256, 0, st, dq_acc, (bf16*)dqkv, M, d,
+                    dvec_ready));
   LAUNCH_CHECK();
   return GPT2_OK;
 }

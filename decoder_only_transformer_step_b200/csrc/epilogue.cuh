@@ -14,6 +14,7 @@ DEVI void epi_one(const EpiArgs& e, float* partial, int split, int M, int N, int
   const long idx = (long)row * e.ldo + col;
   switch (e.kind) {
     case EPI_STORE:
+    case EPI_ROWDOT:  // (the row sums need the tensor-core epilogue; here only the store)
       ((T*)e.out)[idx] = from_f<T>(e.alpha * v);
       break;
     case EPI_BIAS:
@@ -114,7 +115,7 @@ DEVI void epi_apply_row32(const EpiArgs& e, int N, int col0, float (&v)[32], con
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[8 * i + j] *= t[j];
     }
-  } else if (e.kind == EPI_STORE || e.kind == EPI_F32) {
+  } else if (e.kind == EPI_STORE || e.kind == EPI_F32 || e.kind == EPI_ROWDOT) {
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] *= e.alpha;
   }

@@ -336,7 +336,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     constexpr int NCH = BN / 64;  // 32-column chunks per warp and tile
     const uint32_t wbox = epi_smem + (uint32_t)e * C::EPI_WARP_BYTES;
     // (the host selects BIG_EPI whenever there is an operand or a second output)
-    const bool has_operand = BIG_EPI && (p.epi.kind == EPI_BIAS_RESID || p.epi.kind == EPI_DGELU);
+    const bool has_operand =
+        BIG_EPI && (p.epi.kind == EPI_BIAS_RESID || p.epi.kind == EPI_DGELU || p.epi.kind == EPI_ROWDOT);
+    const bool rowdot = BIG_EPI && p.epi.kind == EPI_ROWDOT;
     int chunk = 0;      // chunks stored by this warp: output box chunk & 1
     int op_issued = 0;  // operand boxes requested: box / barrier k & 1, phase k >> 1
     int op_used = 0;
@@ -378,6 +380,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // registers to spare for that and load each chunk when they reach it.
       constexpr bool PREFETCH = !BIG_EPI;
       uint32_t r[NCH][32];
+      float dsum = 0.f;  // EPI_ROWDOT: this row's sum over the current head's 64 columns
       if (PREFETCH && nch > 0) tmem_ld_32x32b_x32(tm_row, r[0]);
 #pragma unroll
       for (int ci = 0; ci < NCH; ++ci) {
@@ -419,6 +422,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           fence_proxy_async_smem();
         }
         epi_apply_row32(p.epi, p.N, col0, v, cur);
+        if (rowdot) {
+          // the stored (bf16) value times the operand; a head is two chunks
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float t[8];
+            unpack8(cur[i], t);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) dsum = fmaf(__bfloat162float(__float2bfloat16_rn(v[8 * i + j])), t[j], dsum);
+          }
+          if (ci & 1) {
+            if (row < p.M) {
+              const int sq = p.epi.seq;
+              reinterpret_cast<float*>(p.epi.out2)[((long)(row / sq) * (p.N / 64) + col0 / 64) * sq + row % sq] =
+                  dsum;
+            }
+            dsum = 0.f;
+          }
+        }
         // the store that last used this chunk's box has read it (two chunks
         // ago; one chunk ago for the single fp32 box of the small layout)
         const bool f32_single = !BIG_EPI && p.store != ST_BF16;
@@ -729,10 +750,14 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
       p.store = ST_BF16;
       ok_c = make_out_tmap(&tc, g.epi.out, g.M, g.N, g.epi.ldo, false);
       break;
+    case EPI_ROWDOT:
+      if (g.N % 64 || g.epi.seq <= 0 || g.M % g.epi.seq || !g.epi.out2 || ((uintptr_t)g.epi.out2 & 3))
+        return GPT2_ERR_INVALID_ARG;
+      [[fallthrough]];
     case EPI_BIAS_RESID:
     case EPI_DGELU: {
       // tmC2: the operand read per chunk (same [M, ldo] layout as the output)
-      const void* opnd = p.epi.kind == EPI_DGELU ? g.epi.aux : g.epi.resid;
+      const void* opnd = p.epi.kind == EPI_BIAS_RESID ? g.epi.resid : g.epi.aux;
       if ((uintptr_t)opnd & 15) return GPT2_ERR_INVALID_ARG;
       p.store = ST_BF16;
       ok_c = make_out_tmap(&tc, g.epi.out, g.M, g.N, g.epi.ldo, false) &&
@@ -769,7 +794,8 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
 
   const int units = p.m_tiles * p.n_tiles * splits;
   // the second output or the operand boxes need the larger epilogue region
-  const bool big = p.store == ST_BF16_X2 || p.epi.kind == EPI_BIAS_RESID || p.epi.kind == EPI_DGELU;
+  const bool big = p.store == ST_BF16_X2 || p.epi.kind == EPI_BIAS_RESID || p.epi.kind == EPI_DGELU ||
+                   p.epi.kind == EPI_ROWDOT;
   int rc;
   if (pair)
     rc = big ? launch_tc<256, true, true>(ta, tb, tc, tc2, p, units, st)

@@ -470,6 +470,11 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
   const float beta = accumulate ? 1.f : 0.f;
   const float sc = grad_scale / (float)M;
   float* G = c->buf.grad;
+  // D = rowsum(dO * O) fused into the attention projection's input-gradient
+  // GEMM (tensor-core path, head_dim 64); dq_acc then starts zeroed here and
+  // every attention backward leaves it zeroed
+  const int fuse_d = (!f32 && s.hd == 64) ? 1 : 0;
+  if (fuse_d) TRY(fill_zero(w.dq_acc, (size_t)M * d * sizeof(float), st));
 
   // LM head (tied): dX_f = s * dz wte ; dwte (=/+=) s * dz^T X_f
   GemmArgs g = make_gemm(M, d, V, w.logits, 0, V, Wp(c, o.wte()), 1, d, EPI_STORE, w.dy, d);
@@ -503,7 +508,14 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
     // column sums of the new residual gradient: the attention projection's b_o gradient
     TRY(ln_backward(c, a.x_mid, a.mean2, a.rstd2, o.layer(l, LN2_G), 0, o.layer(l, LN2_G), o.layer(l, B_O), M, st));
     // attention projection: x_mid = x_in + o W_o^T + b_o
-    g = make_gemm(M, d, d, w.dres, 0, d, Wp(c, o.layer(l, W_O)), 1, d, EPI_STORE, w.dout, d);
+    // (bf16, head_dim 64: the epilogue also writes D = rowsum(dO * O) per head,
+    // the attention backward's first input)
+    g = make_gemm(M, d, d, w.dres, 0, d, Wp(c, o.layer(l, W_O)), 1, d, fuse_d ? EPI_ROWDOT : EPI_STORE, w.dout, d);
+    if (fuse_d) {
+      g.epi.aux = a.o;
+      g.epi.out2 = w.dvec;
+      g.epi.seq = (int)s.T;
+    }
     TRY(run_gemm(c, g, st));
     g = make_gemm(d, d, M, w.dres, 1, d, a.o, 1, d, EPI_F32, G + o.layer(l, W_O), d);
     g.epi.beta = beta;
@@ -514,7 +526,7 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
                        batch, (int)s.T, (int)s.H, (int)s.hd, st));
     else
       TRY(attn_bwd_bf16(a.qkv, a.o, a.lse, w.dout, w.dqkv, w.dq_acc, w.dvec, batch, (int)s.T, (int)s.H, (int)s.hd,
-                        st));
+                        st, fuse_d));
     // QKV: qkv = y1 W_qkv^T + b_qkv
     g = make_gemm(M, d, 3 * d, w.dqkv, 0, 3 * d, Wp(c, o.layer(l, W_QKV)), 1, d, EPI_STORE, w.dy, d);
     TRY(run_gemm(c, g, st));

@@ -15,6 +15,8 @@ enum EpiKind : int {
   EPI_DGELU,        // out(act)  = acc * aux[m,n]  (aux = the saved gelu'(u))
   EPI_F32,          // out(fp32) = beta * out + alpha * acc
   EPI_F32_PARTIAL,  // partial[split][m,n] = acc (split-K, internal)
+  EPI_ROWDOT,       // out(bf16) = acc; out2(fp32)[(m / seq * N/64 + n/64) * seq + m % seq] =
+                    //   sum over the 64 columns of head n/64 of bf16(acc) * aux[m,n]
 };
 
 struct EpiArgs {
@@ -26,6 +28,7 @@ struct EpiArgs {
   const void* aux;    // [M, ldo] act
   long ldo;
   float alpha, beta;
+  int seq;            // EPI_ROWDOT: rows per sequence
 };
 
 // C[m,n] = sum_k A(m,k) B(n,k), then the epilogue.
@@ -63,9 +66,12 @@ int attn_fwd_bf16(const void* qkv, void* o, float* lse, int B, int T, int H, int
                   cudaStream_t st);
 int attn_fwd_f32(const float* qkv, float* o, float* lse, int B, int T, int H, int hd,
                  cudaStream_t st);
-// dq_acc: fp32 [B*T, H*hd] scratch; dvec: fp32 [B,H,T] scratch.
+// dq_acc: fp32 [B*T, H*hd] scratch; dvec: fp32 [B,H,T] scratch.  With
+// dvec_ready the caller has already written dvec = rowsum(dO * O) (head_dim 64:
+// the EPI_ROWDOT epilogue of the GEMM that produced dO) and zeroed dq_acc; the
+// call leaves dq_acc zeroed again for the next layer.
 int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* dout, void* dqkv,
-                  float* dq_acc, float* dvec, int B, int T, int H, int hd, cudaStream_t st);
+                  float* dq_acc, float* dvec, int B, int T, int H, int hd, cudaStream_t st, int dvec_ready = 0);
 int attn_bwd_f32(const float* qkv, const float* o, const float* lse, const float* dout,
                  float* dqkv, float* dvec, int B, int T, int H, int hd, cudaStream_t st);
 
