@@ -150,7 +150,10 @@ DEVI void ln_store4(T* dst, float4 x, float4 g, float4 b, float mu, float rs) {
 // the input row (LN = true: its LayerNorm with eps 1e-5 and biased variance)
 // rounded to T.  Each warp takes GV_COLS consecutive columns per pass; lane l
 // reads 16-byte pieces l, l + 32, ... of each weight row.
-template <typename T, int ROWS, bool LN, int EPI>
+// KS > 1 splits each column group's k-iterations over KS warps (iterations
+// i = slice, slice + KS, ...); their totals meet in shared memory and the
+// slice-0 warp applies the epilogue, summing the slices in a fixed order.
+template <typename T, int ROWS, bool LN, int EPI, int KS>
 __global__ void __launch_bounds__(GV_WARPS * 32) decode_gemv_kernel(const __grid_constant__ GemvArgs a) {
   extern __shared__ __align__(16) uint8_t dec_smem[];
   T* xs = reinterpret_cast<T*>(dec_smem);  // [ROWS][K]
@@ -159,26 +162,32 @@ __global__ void __launch_bounds__(GV_WARPS * 32) decode_gemv_kernel(const __grid
   const int K = a.K;
   constexpr int VN = V16<T>::N;
   constexpr int P = GV_COLS * ROWS;
+  constexpr int HELD = P >= 32 ? P / 32 : 1;  // totals a lane holds after the reduction
   const T* W = reinterpret_cast<const T*>(a.W);
   const int groups = a.N / GV_COLS;
-  int grp = blockIdx.x * nw + warp;
-  // GV_CHUNK k-iterations of weight loads are issued together, before the
-  // first FMA that uses them; the first chunk of a warp's next column group
-  // is loaded ahead (here: before the input staging, whose memory round trip
-  // it overlaps; later: before the reduction of the previous group)
+  const int gpc = nw / KS;                    // column groups per block and pass
+  const int gi = warp / KS, si = warp % KS;   // this warp's group and k slice
+  const int NI = (K + 32 * VN - 1) / (32 * VN);  // k-iterations of 32 x VN elements
+  // (KS > 1) the slices' totals: [warp][HELD][lane], after the staged rows
+  float* red = reinterpret_cast<float*>(dec_smem + (size_t)ROWS * K * sizeof(T));
+  // GV_CHUNK of this slice's k-iterations of weight loads are issued together,
+  // before the first FMA that uses them; the first chunk of a warp's next
+  // column group is loaded ahead (here: before the input staging, whose
+  // memory round trip it overlaps; later: before the reduction of the
+  // previous group)
   uint4 wv[GV_CHUNK][GV_COLS];
-  auto load_chunk = [&](int g, int k0) {
+  auto load_chunk = [&](int g, int it0) {
     const T* w0 = W + (size_t)g * GV_COLS * K;
 #pragma unroll
     for (int u = 0; u < GV_CHUNK; ++u) {
-      const int k = k0 + u * 32 * VN;
+      const int k = lane * VN + (it0 + u * KS) * 32 * VN;
 #pragma unroll
       for (int c = 0; c < GV_COLS; ++c)
         wv[u][c] = k < K ? ld_stream16(w0 + (size_t)c * K + k) : make_uint4(0u, 0u, 0u, 0u);
     }
   };
   pdl_start();
-  if (grp < groups) load_chunk(grp, lane * VN);
+  if (blockIdx.x * gpc + gi < groups) load_chunk(blockIdx.x * gpc + gi, si);
 
   // Input rows -> shared memory as T.  Every load of a row is issued before
   // the first use (one memory round trip per row): 16-byte loads, the
@@ -272,8 +281,11 @@ __global__ void __launch_bounds__(GV_WARPS * 32) decode_gemv_kernel(const __grid
   }
   __syncthreads();
 
-  constexpr int HELD = P >= 32 ? P / 32 : 1;  // totals a lane holds after the reduction
-  for (; grp < groups; grp += gridDim.x * nw) {
+  // passes over the column groups, uniform across the block (the slices of a
+  // group synchronise through shared memory once per pass)
+  for (int pass_base = blockIdx.x * gpc; pass_base < groups; pass_base += gridDim.x * gpc) {
+    const int grp = pass_base + gi;
+    const bool active = grp < groups;
     const int n0 = grp * GV_COLS;
     // the epilogue's operands (bias, old residual, cache position) are loaded
     // now, so that their latency hides behind the weight stream
@@ -284,7 +296,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) decode_gemv_kernel(const __grid
       bool owner;
       const int idx = rs_index<P>(lane, j, &owner);
       const int c = idx / ROWS, r = idx % ROWS;
-      const bool live = owner && r < a.rows;
+      const bool live = active && si == 0 && owner && r < a.rows;
       pre_b[j] = 0.f;
       pre_x[j] = 0.f;
       pre_p[j] = 0;
@@ -297,57 +309,77 @@ __global__ void __launch_bounds__(GV_WARPS * 32) decode_gemv_kernel(const __grid
     float acc[P];
 #pragma unroll
     for (int i = 0; i < P; ++i) acc[i] = 0.f;
-    for (int k0 = lane * VN; k0 < K; k0 += GV_CHUNK * 32 * VN) {
-      if (k0 != lane * VN) load_chunk(grp, k0);
+    if (active) {
+      for (int it0 = si; it0 < NI; it0 += GV_CHUNK * KS) {
+        if (it0 != si) load_chunk(grp, it0);
 #pragma unroll
-      for (int u = 0; u < GV_CHUNK; ++u) {
-        const int k = k0 + u * 32 * VN;
-        if (k >= K) break;
-        float wf[GV_COLS][VN];
+        for (int u = 0; u < GV_CHUNK; ++u) {
+          const int k = lane * VN + (it0 + u * KS) * 32 * VN;
+          if (k >= K) break;
+          float wf[GV_COLS][VN];
 #pragma unroll
-        for (int c = 0; c < GV_COLS; ++c) V16<T>::unpack(wv[u][c], wf[c]);
+          for (int c = 0; c < GV_COLS; ++c) V16<T>::unpack(wv[u][c], wf[c]);
 #pragma unroll
-        for (int r = 0; r < ROWS; ++r) {
-          float xf[VN];
-          V16<T>::unpack(*reinterpret_cast<const uint4*>(xs + (size_t)r * K + k), xf);
+          for (int r = 0; r < ROWS; ++r) {
+            float xf[VN];
+            V16<T>::unpack(*reinterpret_cast<const uint4*>(xs + (size_t)r * K + k), xf);
 #pragma unroll
-          for (int c = 0; c < GV_COLS; ++c)
+            for (int c = 0; c < GV_COLS; ++c)
 #pragma unroll
-            for (int e = 0; e < VN; ++e) acc[c * ROWS + r] = fmaf(wf[c][e], xf[e], acc[c * ROWS + r]);
-        }
-      }
-    }
-    if (grp + (int)gridDim.x * nw < groups) load_chunk(grp + gridDim.x * nw, lane * VN);
-    ReduceScatter<P, 16>::run(acc, lane);
-#pragma unroll
-    for (int j = 0; j < HELD; ++j) {
-      bool owner;
-      const int idx = rs_index<P>(lane, j, &owner);
-      const int c = idx / ROWS, r = idx % ROWS;
-      if (!owner || r >= a.rows) continue;
-      const int n = n0 + c;
-      const float v = acc[j] + pre_b[j];
-      float* outf = reinterpret_cast<float*>(a.out);
-      if constexpr (EPI == DEC_QKV) {
-        if (n < a.d) {
-          outf[(size_t)r * a.ldo + n] = v;
-        } else {
-          const int kind = n >= 2 * a.d;
-          const int nn = n - a.d - kind * a.d;
-          const int p = pre_p[j];
-          if (p >= 0 && p < a.max_len) {
-            T* plane = reinterpret_cast<T*>(kind ? a.vc : a.kc);
-            plane[(((size_t)r * a.H + nn / a.hd) * a.max_len + p) * a.hd + nn % a.hd] = from_f<T>(v);
+              for (int e = 0; e < VN; ++e) acc[c * ROWS + r] = fmaf(wf[c][e], xf[e], acc[c * ROWS + r]);
           }
         }
-      } else if constexpr (EPI == DEC_RESID) {
-        outf[(size_t)r * a.ldo + n] = pre_x[j] + v;
-      } else if constexpr (EPI == DEC_GELU) {
-        reinterpret_cast<T*>(a.out)[(size_t)r * a.ldo + n] = from_f<T>(gelu_f<false>(v));
-      } else {
-        outf[(size_t)r * a.ldo + n] = v;
+      }
+      if (grp + (int)gridDim.x * gpc < groups) load_chunk(grp + gridDim.x * gpc, si);
+    }
+    ReduceScatter<P, 16>::run(acc, lane);
+    if constexpr (KS > 1) {
+#pragma unroll
+      for (int j = 0; j < HELD; ++j) red[(warp * HELD + j) * 32 + lane] = acc[j];
+      __syncthreads();
+      if (si == 0) {
+#pragma unroll
+        for (int j = 0; j < HELD; ++j) {
+          float t = acc[j];
+#pragma unroll
+          for (int x = 1; x < KS; ++x) t += red[((warp + x) * HELD + j) * 32 + lane];
+          acc[j] = t;
+        }
       }
     }
+    if (active && si == 0) {
+#pragma unroll
+      for (int j = 0; j < HELD; ++j) {
+        bool owner;
+        const int idx = rs_index<P>(lane, j, &owner);
+        const int c = idx / ROWS, r = idx % ROWS;
+        if (!owner || r >= a.rows) continue;
+        const int n = n0 + c;
+        const float v = acc[j] + pre_b[j];
+        float* outf = reinterpret_cast<float*>(a.out);
+        if constexpr (EPI == DEC_QKV) {
+          if (n < a.d) {
+            outf[(size_t)r * a.ldo + n] = v;
+          } else {
+            const int kind = n >= 2 * a.d;
+            const int nn = n - a.d - kind * a.d;
+            const int p = pre_p[j];
+            if (p >= 0 && p < a.max_len) {
+              T* plane = reinterpret_cast<T*>(kind ? a.vc : a.kc);
+              plane[(((size_t)r * a.H + nn / a.hd) * a.max_len + p) * a.hd + nn % a.hd] = from_f<T>(v);
+            }
+          }
+        } else if constexpr (EPI == DEC_RESID) {
+          outf[(size_t)r * a.ldo + n] = pre_x[j] + v;
+        } else if constexpr (EPI == DEC_GELU) {
+          reinterpret_cast<T*>(a.out)[(size_t)r * a.ldo + n] = from_f<T>(gelu_f<false>(v));
+        } else {
+          outf[(size_t)r * a.ldo + n] = v;
+        }
+      }
+    }
+    // the next pass overwrites red only after every slice-0 warp has read it
+    if constexpr (KS > 1) __syncthreads();
   }
 }
 
@@ -581,39 +613,45 @@ __global__ void prefill_logits_kernel(const T* __restrict__ logits, const int32_
     out[(size_t)r * V + v] = to_f(src[v]);
 }
 
-template <typename T, int ROWS, bool LN, int EPI>
+template <typename T, int ROWS, bool LN, int EPI, int KS>
 int gemv_launch(const GemvArgs& a, cudaStream_t st) {
-  const size_t smem = (size_t)ROWS * a.K * sizeof(T);
+  constexpr int HELD = GV_COLS * ROWS >= 32 ? GV_COLS * ROWS / 32 : 1;
+  const size_t smem = (size_t)ROWS * a.K * sizeof(T) + (KS > 1 ? (size_t)GV_WARPS * HELD * 32 * 4 : 0);
   static bool attr = false;
   if (!attr) {
-    CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<T, ROWS, LN, EPI>,
+    CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<T, ROWS, LN, EPI, KS>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
     attr = true;
   }
-  // narrow outputs: 4-warp blocks, so that twice as many SMs stream weights
   const int groups = a.N / GV_COLS;
-  const int nw = (LN || groups >= GV_WARPS * num_sms()) ? GV_WARPS : 4;
-  int grid = (groups + nw - 1) / nw;
+  // narrow outputs: 4-warp blocks (or, with a k split, 8 warps on 2 groups),
+  // so that more SMs stream weights
+  const int nw = (KS > 1 || LN || groups >= GV_WARPS * num_sms()) ? GV_WARPS : 4;
+  const int gpc = nw / KS;
+  int grid = (groups + gpc - 1) / gpc;
   const int cap = 2 * num_sms();
   if (grid > cap) grid = cap;
-  CUDA_TRY(launch_k(decode_gemv_kernel<T, ROWS, LN, EPI>, grid, nw * 32, smem, st, a));
+  CUDA_TRY(launch_k(decode_gemv_kernel<T, ROWS, LN, EPI, KS>, grid, nw * 32, smem, st, a));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
 
-template <typename T, bool LN, int EPI>
+template <typename T, bool LN, int EPI, int KS>
 int gemv_rows(const GemvArgs& a, cudaStream_t st) {
-  if (a.rows <= 4) return gemv_launch<T, 4, LN, EPI>(a, st);
-  if (a.rows <= 8) return gemv_launch<T, 8, LN, EPI>(a, st);
-  return gemv_launch<T, 16, LN, EPI>(a, st);
+  if (a.rows <= 4) return gemv_launch<T, 4, LN, EPI, KS>(a, st);
+  if (a.rows <= 8) return gemv_launch<T, 8, LN, EPI, KS>(a, st);
+  return gemv_launch<T, 16, LN, EPI, KS>(a, st);
 }
 
 template <typename T>
 int gemv_dispatch(const GemvArgs& a, bool ln, int epi, cudaStream_t st) {
-  if (epi == DEC_QKV && ln) return gemv_rows<T, true, DEC_QKV>(a, st);
-  if (epi == DEC_RESID && !ln) return gemv_rows<T, false, DEC_RESID>(a, st);
-  if (epi == DEC_GELU && ln) return gemv_rows<T, true, DEC_GELU>(a, st);
-  if (epi == DEC_LOGITS && ln) return gemv_rows<T, true, DEC_LOGITS>(a, st);
+  // the residual products have narrow outputs (d columns): k split four ways
+  // (for the LayerNorm'd products a split measured slower: every extra block
+  // repeats the LayerNorm of the staged rows)
+  if (epi == DEC_QKV && ln) return gemv_rows<T, true, DEC_QKV, 1>(a, st);
+  if (epi == DEC_RESID && !ln) return gemv_rows<T, false, DEC_RESID, 4>(a, st);
+  if (epi == DEC_GELU && ln) return gemv_rows<T, true, DEC_GELU, 1>(a, st);
+  if (epi == DEC_LOGITS && ln) return gemv_rows<T, true, DEC_LOGITS, 1>(a, st);
   return GPT2_ERR_INVALID_ARG;
 }
 
@@ -621,7 +659,7 @@ int gemv_dispatch(const GemvArgs& a, bool ln, int epi, cudaStream_t st) {
 
 size_t decode_gemv_smem(int f32, int rows, int K) {
   const int R = rows <= 4 ? 4 : (rows <= 8 ? 8 : 16);
-  return (size_t)R * K * (f32 ? 4 : 2);
+  return (size_t)R * K * (f32 ? 4 : 2) + (size_t)GV_WARPS * (R / 8 > 1 ? R / 8 : 1) * 32 * 4;
 }
 
 int decode_embed(int f32, const int32_t* tok, const int32_t* pos, const void* wte, const void* wpe, float* x,
