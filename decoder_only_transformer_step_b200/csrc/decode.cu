@@ -575,6 +575,83 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
+// The greedy choice over many blocks (rows <= GREEDY_SPLIT_MAX_ROWS): block
+// (s, r) scans slice s of row r's real vocabulary and leaves its best
+// (value, id); one warp per row then picks the best of the GREEDY_SLICES.
+constexpr int GREEDY_SLICES = 16;
+__global__ void __launch_bounds__(256)
+    greedy_part_kernel(const float* __restrict__ logits, long ld, int vocab_real, float* __restrict__ pv,
+                       int* __restrict__ pi) {
+  __shared__ float sv[8];
+  __shared__ int si[8];
+  pdl_start();
+  const int s = blockIdx.x, r = blockIdx.y;
+  const int per = (vocab_real + GREEDY_SLICES - 1) / GREEDY_SLICES;
+  const int v0 = s * per, v1 = min(vocab_real, v0 + per);
+  const float* z = logits + (size_t)r * ld;
+  float bv = -INFINITY;
+  int bi = 0x7fffffff;
+  constexpr int U = 8;
+  for (int b0 = v0 + (int)threadIdx.x; b0 < v1; b0 += U * 256) {
+    float x[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) x[u] = b0 + u * 256 < v1 ? z[b0 + u * 256] : -INFINITY;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = b0 + u * 256;
+      if (v < v1 && greedy_better(x[u], v, bv, bi)) {
+        bv = x[u];
+        bi = v;
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+    if (greedy_better(ov, oi, bv, bi)) {
+      bv = ov;
+      bi = oi;
+    }
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    sv[warp] = bv;
+    si[warp] = bi;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < 8; ++w)
+      if (greedy_better(sv[w], si[w], bv, bi)) {
+        bv = sv[w];
+        bi = si[w];
+      }
+    pv[r * GREEDY_SLICES + s] = bv;
+    pi[r * GREEDY_SLICES + s] = bi;
+  }
+}
+
+__global__ void greedy_final_kernel(const float* __restrict__ pv, const int* __restrict__ pi, int vocab_real,
+                                    int32_t* __restrict__ next, int32_t* __restrict__ pos) {
+  pdl_start();
+  const int r = blockIdx.x, lane = threadIdx.x;
+  float bv = lane < GREEDY_SLICES ? pv[r * GREEDY_SLICES + lane] : -INFINITY;
+  int bi = lane < GREEDY_SLICES ? pi[r * GREEDY_SLICES + lane] : 0x7fffffff;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+    if (greedy_better(ov, oi, bv, bi)) {
+      bv = ov;
+      bi = oi;
+    }
+  }
+  if (lane == 0) {
+    next[r] = bi < vocab_real ? bi : 0;
+    if (pos) pos[r] += 1;
+  }
+}
+
 // Prefill: K and V of positions < plen[r] from a layer's qkv activation
 // [rows * T, 3d] into the cache planes; plen outside [1, limit] raises the
 // position bit and copies nothing for that row.
@@ -629,7 +706,14 @@ int gemv_launch(const GemvArgs& a, cudaStream_t st) {
   const int nw = (KS > 1 || LN || groups >= GV_WARPS * num_sms()) ? GV_WARPS : 4;
   const int gpc = nw / KS;
   int grid = (groups + gpc - 1) / gpc;
-  const int cap = 2 * num_sms();
+  // at most one wave of resident blocks (the registers allow one 8-warp block
+  // per SM): a second wave would repeat the input staging and add a tail
+  static int per_sm[2] = {0, 0};
+  int& occ = per_sm[nw == GV_WARPS];
+  if (occ == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_gemv_kernel<T, ROWS, LN, EPI, KS>,
+                                                                   nw * 32, smem) != cudaSuccess || occ < 1))
+    occ = 1;
+  const int cap = occ * num_sms();
   if (grid > cap) grid = cap;
   CUDA_TRY(launch_k(decode_gemv_kernel<T, ROWS, LN, EPI, KS>, grid, nw * 32, smem, st, a));
   LAUNCH_CHECK();
@@ -710,8 +794,16 @@ int decode_attention(int f32, const void* kc, const void* vc, const float* q, fl
 }
 
 int decode_greedy(const float* logits, long ld, int rows, int vocab_real, int32_t* next, int32_t* pos,
-                  cudaStream_t st) {
-  CUDA_TRY(launch_k(greedy_kernel, rows, 1024, 0, st, logits, ld, vocab_real, next, pos));
+                  float* part_v, int* part_i, cudaStream_t st) {
+  if (part_v && part_i && rows <= GREEDY_SPLIT_MAX_ROWS) {
+    CUDA_TRY(launch_k(greedy_part_kernel, dim3(GREEDY_SLICES, rows), 256, 0, st, logits, ld, vocab_real, part_v,
+                      part_i));
+    LAUNCH_CHECK();
+    CUDA_TRY(launch_k(greedy_final_kernel, rows, 32, 0, st, (const float*)part_v, (const int*)part_i, vocab_real,
+                      next, pos));
+  } else {
+    CUDA_TRY(launch_k(greedy_kernel, rows, 1024, 0, st, logits, ld, vocab_real, next, pos));
+  }
   LAUNCH_CHECK();
   return GPT2_OK;
 }

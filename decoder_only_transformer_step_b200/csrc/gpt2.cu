@@ -108,6 +108,8 @@ struct Work {
   float *dq_acc, *dvec;
   float *norm_part, *gnorm;  // global gradient norm: block partials and the result
   int* n_valid;              // positions with a target in the last forward
+  float* greedy_v;           // per-slice best (value, id) of the greedy choice
+  int* greedy_i;
   // block partials of every bias / LayerNorm parameter gradient of one
   // backward, each in its own slot, all reduced by one launch at its end
   float* part_arena;
@@ -184,6 +186,8 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
   w->norm_part = c.take<float>((size_t)GRAD_NORM_PARTS * 4);
   w->gnorm = c.take<float>(4);
   w->n_valid = c.take<int>(4);
+  w->greedy_v = c.take<float>((size_t)GREEDY_SPLIT_MAX_ROWS * 16 * 4);
+  w->greedy_i = c.take<int>((size_t)GREEDY_SPLIT_MAX_ROWS * 16 * 4);
   w->part_used = 0;
   w->split_bytes = split_ws_need(s, M);
   w->split_ws = c.take<void>(w->split_bytes);
@@ -724,7 +728,8 @@ int gpt2_prefill(gpt2_ctx* c, void* cache, size_t cache_bytes, int batch, int ma
 int gpt2_greedy_next(gpt2_ctx* c, const float* logits, int batch, int32_t* next_tokens, int32_t* pos,
                      void* stream) {
   if (!c || !logits || !next_tokens || batch < 1) return GPT2_ERR_INVALID_ARG;
-  return decode_greedy(logits, c->s.V, batch, (int)c->s.Vr, next_tokens, pos, S(stream));
+  return decode_greedy(logits, c->s.V, batch, (int)c->s.Vr, next_tokens, pos, c->w.greedy_v, c->w.greedy_i,
+                       S(stream));
 }
 
 int gpt2_step_host(gpt2_ctx* c, const int32_t* tokens_host, const int32_t* targets_host, int batch,

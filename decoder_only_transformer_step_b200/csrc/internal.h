@@ -159,8 +159,10 @@ int decode_embed(int f32, const int32_t* tok, const int32_t* pos, const void* wt
                  int rows, int d, int vocab_real, int limit, int* err, cudaStream_t st);
 int decode_attention(int f32, const void* kc, const void* vc, const float* q, float* o, const int32_t* pos,
                      int rows, int H, int hd, int max_len, cudaStream_t st);
+// part_v / part_i: GREEDY_SPLIT_MAX_ROWS x 16 scratch (may be NULL: one block per row)
+constexpr int GREEDY_SPLIT_MAX_ROWS = 16;
 int decode_greedy(const float* logits, long ld, int rows, int vocab_real, int32_t* next, int32_t* pos,
-                  cudaStream_t st);
+                  float* part_v, int* part_i, cudaStream_t st);
 int prefill_kv(int f32, const void* qkv, void* kc, void* vc, const int32_t* plen, int rows, int T, int H, int hd,
                int max_len, int limit, int* err, cudaStream_t st);
 int prefill_logits(int f32, const void* logits, const int32_t* plen, float* out, int rows, int T, int V, int limit,
