@@ -183,3 +183,26 @@ def test_invalid_cache_arguments():
         gp.gpt2_decode_step(model.ctx, cache.buf[256:], 2, 8, cache.tokens, cache.pos, cache.logits)
     with pytest.raises(gp.Gpt2Error):
         gp.gpt2_decode_step(model.ctx, cache.buf[1:], 2, 8, cache.tokens, cache.pos, cache.logits)
+
+
+def test_full_size_decode_in_bench_configuration():
+    # GPT-2 124M, batch 8 after 128-token prompts (the bench's decode workload
+    # and kernel variants), two teacher-forced steps: every row's logits
+    # against the oracle forward over the same prefix
+    from oracle_fixtures import GPT2_124M
+    mc = gp.ModelConfig(12, 768, 12, 1024, 50257, 50304, 8, 0)
+    model = gp.GPT2(mc)
+    model.init_params(seed=0)
+    p32 = oracle.unflatten(model.master.double().cpu().numpy(), GPT2_124M)
+    B, P = 8, 128
+    tok = inputs.zipf_tokens(B, 1024, n_ids=50257, seed=777)[0]
+    cache = gp.KVCache(model, B, 1024)
+    cache.prefill(i32(tok), i32(np.full(B, P)))
+    for t in (P, P + 1):
+        z = cache.step(i32(tok[:, t]), i32(np.full(B, t))).cpu().numpy().astype(np.float64)
+    n = P + 2  # the logits after positions 0 .. n-1
+    ref = forward(p32, GPT2_124M, tok[:, :n], np.full((B, n), G.IGNORE))[1]["z"][:, n - 1]
+    for b in range(B):
+        assert rel_err(z[b], ref[b]) <= 2e-2, b
+    torch.cuda.synchronize()
+    assert model.status() == 0
