@@ -219,7 +219,6 @@ cudaStream_t S(void* st) { return reinterpret_cast<cudaStream_t>(st); }
 const void* Wp(const gpt2_ctx* c, size_t off) {
   return c->s.mode ? (const void*)(c->buf.master + off) : (const void*)(c->buf.shadow + off);
 }
-size_t act_bytes(const gpt2_ctx* c) { return c->s.mode ? 4 : 2; }
 
 int run_gemm(gpt2_ctx* c, const GemmArgs& g, cudaStream_t st) {
   if (c->s.mode) return gemm_simt_f32(g, st);
