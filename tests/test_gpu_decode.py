@@ -206,3 +206,26 @@ def test_full_size_decode_in_bench_configuration():
         assert rel_err(z[b], ref[b]) <= 2e-2, b
     torch.cuda.synchronize()
     assert model.status() == 0
+
+
+def test_full_size_training_forward_sampled_logits():
+    # the training forward in the bench's launch configuration (GPT-2 124M,
+    # 16 x 1024 tokens, all 12 layers) read through prefill: each row's logits
+    # at one position against the oracle forward over that row's prefix
+    # (causality: positions <= p depend on tokens 0..p only)
+    from oracle_fixtures import GPT2_124M
+    mc = gp.ModelConfig(12, 768, 12, 1024, 50257, 50304, 16, 0)
+    model = gp.GPT2(mc)
+    model.init_params(seed=3)
+    p32 = oracle.unflatten(model.master.double().cpu().numpy(), GPT2_124M)
+    B = 16
+    tok = inputs.zipf_tokens(B, 1024, n_ids=50257, seed=1000)[0]
+    plen = (np.arange(B, dtype=np.int32) * 3 + 5) % 48 + 1
+    cache = gp.KVCache(model, B, 1024)
+    z = cache.prefill(i32(tok), i32(plen)).cpu().numpy().astype(np.float64)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    for b in range(B):
+        n = int(plen[b])
+        ref = forward(p32, GPT2_124M, tok[b:b + 1, :n], np.full((1, n), G.IGNORE))[1]["z"][0, n - 1]
+        assert rel_err(z[b], ref) <= 2e-2, b
