@@ -315,3 +315,26 @@ def test_target_minus_one_is_masked_other_negatives_flagged():
     model.forward_loss(torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda())
     assert model.status() == -5
     assert model.status() == 0
+
+
+def test_full_size_step_gradients_through_masked_targets():
+    # the step in the bench's launch configuration (GPT-2 124M, 16 x 1024
+    # tokens, 12 layers, bf16): with targets only at positions < n_b of row b
+    # (-1 elsewhere) the loss and every gradient depend on the rows' first
+    # n_b tokens alone (causality), which the oracle computes in full
+    from oracle_fixtures import GPT2_124M
+    B, T = 16, 1024
+    model = make_model(GPT2_124M, 50257, B, 0)
+    model.init_params(seed=5)
+    p32 = oracle.unflatten(model.master.double().cpu().numpy(), GPT2_124M)
+    tok, tgt = inputs.zipf_tokens(B, T, n_ids=50257, seed=1001)
+    nb = (np.arange(B) * 7 + 9) % 40 + 8
+    tgt = tgt.copy()
+    for b in range(B):
+        tgt[b, nb[b]:] = -1
+    loss = run_step(model, tok, tgt)
+    n = int(nb.max())
+    ref_loss, cache = forward(p32, GPT2_124M, tok[:, :n], tgt[:, :n])
+    ref_g = backward(p32, GPT2_124M, cache)
+    assert abs(loss - ref_loss) <= 1e-2 * abs(ref_loss), (loss, ref_loss)
+    compare_grads(gpu_grads(model, GPT2_124M), ref_g, 0.999, 2e-2)
