@@ -321,34 +321,34 @@ __global__ void __launch_bounds__(32 * LNF_WARPS, LNF_BLOCKS_PER_SM)
 #pragma unroll
     for (int j = 0; j < VN; ++j) sg[k][j] = sb[k][j] = sr[k][j] = 0.f;
   // the rows stay packed (16-byte words) in registers and are unpacked on
-  // each use, which leaves room to prefetch the next row while this one is
-  // processed: two rows of loads in flight per warp
+  // each use, which leaves room to prefetch the next row (x, dy, the incoming
+  // residual gradient, its mean and rstd) while this one is processed: two
+  // rows of loads in flight per warp
   const int stride = gridDim.x * LNF_WARPS;
   int m = blockIdx.x * LNF_WARPS + warp;
-  uint4 cx[NC], cd[NC];
-  auto load_row = [&](int r, uint4 (&ux)[NC], uint4 (&ud)[NC]) {
+  uint4 cx[NC], cd[NC], cr[NC];
+  float cmu = 0.f, crs = 0.f;
+  auto load_row = [&](int r, uint4 (&ux)[NC], uint4 (&ud)[NC], uint4 (&ur)[NC], float& mu_, float& rs_) {
 #pragma unroll
     for (int k = 0; k < NC; ++k) {
       const int c = (lane + 32 * k) * VN;
       if (r < M && c < d) {
         ux[k] = *reinterpret_cast<const uint4*>(x + (long)r * d + c);
         ud[k] = *reinterpret_cast<const uint4*>(dy + (long)r * d + c);
+        if (!dres_init) ur[k] = *reinterpret_cast<const uint4*>(dres + (long)r * d + c);
       }
+    }
+    if (r < M) {
+      mu_ = mean[r];
+      rs_ = rstd[r];
     }
   };
-  load_row(m, cx, cd);
+  load_row(m, cx, cd, cr, cmu, crs);
   for (; m < M; m += stride) {
-    uint4 nx[NC], nd[NC];
-    load_row(m + stride, nx, nd);
-    uint4 cr[NC];
-    if (!dres_init) {
-#pragma unroll
-      for (int k = 0; k < NC; ++k) {
-        const int c = (lane + 32 * k) * VN;
-        if (c < d) cr[k] = *reinterpret_cast<const uint4*>(dres + (long)m * d + c);
-      }
-    }
-    const float mu = mean[m], rs = rstd[m];
+    uint4 nx[NC], nd[NC], nr[NC];
+    float nmu = 0.f, nrs = 0.f;
+    load_row(m + stride, nx, nd, nr, nmu, nrs);
+    const float mu = cmu, rs = crs;
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
     for (int k = 0; k < NC; ++k) {
@@ -397,7 +397,10 @@ __global__ void __launch_bounds__(32 * LNF_WARPS, LNF_BLOCKS_PER_SM)
     for (int k = 0; k < NC; ++k) {
       cx[k] = nx[k];
       cd[k] = nd[k];
+      cr[k] = nr[k];
     }
+    cmu = nmu;
+    crs = nrs;
   }
   constexpr int NQ = RES ? 3 : 2;
 #pragma unroll
