@@ -338,3 +338,25 @@ def test_full_size_step_gradients_through_masked_targets():
     ref_g = backward(p32, GPT2_124M, cache)
     assert abs(loss - ref_loss) <= 1e-2 * abs(ref_loss), (loss, ref_loss)
     compare_grads(gpu_grads(model, GPT2_124M), ref_g, 0.999, 2e-2)
+
+
+@pytest.mark.parametrize("d,H,T", [(1024, 16, 256), (1600, 25, 256), (768, 12, 4096)],
+                         ids=["350m-shaped", "1.5b-shaped", "t4096-shaped"])
+def test_other_config_shapes_one_layer(d, H, T):
+    """The widths and the context of the other configurations (GPT-2 medium
+    d 1024 / 16 heads, XL d 1600 / 25 heads, long context T 4096): one layer,
+    vocabulary 50304, bf16, Zipf ids; loss and every gradient against the
+    oracle.  d 1024 and 1600 take the two-kernel LayerNorm backward and (1600)
+    ragged GEMM tiles; T 4096 fills the attention backward's 32 query-block
+    slots."""
+    oc = Config(n_layer=1, d_model=d, n_head=H, n_ctx=T, vocab=50304)
+    params = params_for(oc, seed=43)
+    B = 1
+    tok, tgt = inputs.zipf_tokens(B, T, seed=44)
+    model = make_model(oc, 50257, B, 0)
+    p32 = load_params(model, params, oc)
+    loss = run_step(model, tok, tgt)
+    ref_loss, cache = forward(p32, oc, tok, tgt)
+    ref_g = backward(p32, oc, cache)
+    assert abs(loss - ref_loss) <= 1e-2 * abs(ref_loss), (loss, ref_loss)
+    compare_grads(gpu_grads(model, oc), ref_g, 0.999, 2e-2)
