@@ -229,3 +229,28 @@ def test_full_size_training_forward_sampled_logits():
         n = int(plen[b])
         ref = forward(p32, GPT2_124M, tok[b:b + 1, :n], np.full((1, n), G.IGNORE))[1]["z"][0, n - 1]
         assert rel_err(z[b], ref) <= 2e-2, b
+
+
+@pytest.mark.parametrize("batch", [5, 16])
+def test_decode_wide_model_matches_oracle(batch):
+    # d 1600 / 25 heads (the XL width): the LayerNorm staging's wide-row path
+    # (rows over 1024 wide) and a 6400-deep k split in the MLP projection
+    oc = Config(n_layer=1, d_model=1600, n_head=25, n_ctx=64, vocab=1024)
+    params = params_for(oc, seed=51)
+    model = make_model(oc, 1000, batch, 0)
+    p32 = load_params(model, params, oc)
+    max_len = 48
+    plen = (np.arange(batch, dtype=np.int32) * 5) % 20 + 1
+    tok, _ = inputs.uniform_tokens(batch, oc.n_ctx, 1000, seed=52)
+    cache = gp.KVCache(model, batch, max_len)
+    z = cache.prefill(i32(tok), i32(plen)).cpu().numpy().astype(np.float64)
+    ref_cache = kv_cache_empty(oc, batch, max_len)
+    assert rel_err(z, prefill(p32, oc, ref_cache, tok, plen)) <= 2e-2
+    pos = plen.copy()
+    for step in range(3):
+        t_step = inputs.uniform_tokens(batch, 1, 1000, seed=200 + step)[0][:, 0]
+        z = cache.step(i32(t_step), i32(pos)).cpu().numpy().astype(np.float64)
+        assert rel_err(z, decode_step(p32, oc, ref_cache, t_step, pos)) <= 2e-2, step
+        pos = pos + 1
+    torch.cuda.synchronize()
+    assert model.status() == 0
