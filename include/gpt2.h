@@ -9,8 +9,12 @@
  * forward 2N, backward two matmul-sized gradients per layer; memory section:
  * fp32 weight, gradient, m and v).  Model: pre-LayerNorm decoder blocks with
  * learned positions, causal multi-head attention, GELU(tanh) MLP, LM head
- * tied to the token embedding; mean cross-entropy over all B*T positions;
- * decoupled-weight-decay AdamW with fp32 master weights.
+ * tied to the token embedding; mean cross-entropy over the B*T positions
+ * (those with a target, when some are masked); decoupled-weight-decay AdamW
+ * with fp32 master weights.  Around the step: gradient-norm clipping, AdamW
+ * over one shard of the flat buffers (data parallelism with sharded optimizer
+ * state), and incremental decoding with a key/value cache (prefill, decode
+ * step, greedy choice) on the same model.
  *
  * Conventions for every function below
  * - Ownership: the caller allocates and owns every device buffer (the
