@@ -30,10 +30,13 @@ attention, GELU MLP, LM head tied to the token embedding) is the GPT-2 step as
 the task states it.  Where the pages are silent this oracle takes the plainest
 GPT-2 reading: tanh-form GELU, LayerNorm eps 1e-5 with biased variance,
 biases on every linear layer except the tied head, no dropout, softmax scale
-1/sqrt(head_dim), loss averaged over all B*T positions, weight decay on 2-D
+1/sqrt(head_dim), loss averaged over all B*T positions (over those with a
+target when some targets are -1, the masked loss below), weight decay on 2-D
 tensors only, AdamW with bias correction and eps 1e-8, no gradient clipping
 (an optional global-norm clip is provided for the training loop around the
-step; it is off unless asked for).
+step; it is off unless asked for).  The end of the module holds the
+incremental decoder with a key/value cache (decode step, prefill, greedy
+choice), pinned to the full forward.
 
 Pins (tests/test_oracle_*.py): central finite differences in fp64 for every
 parameter tensor, an independent PyTorch autograd witness built from library
