@@ -109,3 +109,21 @@ def test_kv_cache_bytes_layout():
     assert gp.gpt2_kv_cache_bytes(c1, 1, 5) == 2 * 2 * (4 * 5 * 16 * 4) + 3 * 64 * 4 + 256 * 4
     for b, n in [(0, 8), (17, 8), (4, 0), (4, 1025)]:
         assert gp.gpt2_kv_cache_bytes(c, b, n) == 0
+
+
+def test_null_context_calls_are_rejected_on_host():
+    # every entry point validates its context and pointers before touching the
+    # device, so these return GPT2_ERR_INVALID_ARG without a GPU
+    L = gp._lib()
+    bad = gp.ERRORS_BY_NAME["GPT2_ERR_INVALID_ARG"]
+    assert L.gpt2_forward_loss(None, None, None, 1, None, None) == bad
+    assert L.gpt2_backward(None, 1.0, 0, None) == bad
+    assert L.gpt2_adamw_step(None, 6e-4, 0.9, 0.95, 1e-8, 0.1, 1, None) == bad
+    assert L.gpt2_adamw_step_clip(None, 6e-4, 0.9, 0.95, 1e-8, 0.1, 1, 1.0, None) == bad
+    assert L.gpt2_adamw_step_range(None, 6e-4, 0.9, 0.95, 1e-8, 0.1, 1, 0, 4, None) == bad
+    assert L.gpt2_grad_norm(None, None, None) == bad
+    assert L.gpt2_zero_grad(None, None) == bad
+    assert L.gpt2_get_status(None, None) == bad
+    assert L.gpt2_prefill(None, None, 0, 1, 1, None, None, None, None) == bad
+    assert L.gpt2_decode_step(None, None, 0, 1, 1, None, None, None, None) == bad
+    assert L.gpt2_greedy_next(None, None, 1, None, None, None) == bad
