@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "train tokens/s, GPT-2 124M T=1024 bf16 on 1 B200; MFU (6N+attn FLOPs)"
+HBM_KERNELS = ("ln_fwd", "ln_bwd", "colsum", "adamw")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 CONFIGS = {
@@ -483,10 +484,56 @@ def run_kernel(args):
     import torch
     import decoder_only_transformer_step_b200 as gp
     L, d, H, T, Vr, V, B = CONFIGS[args.config]
-    M = args.tokens
+    hbm = args.kernel in HBM_KERNELS
+    # HBM-bound kernels: inputs larger than the 126 MB L2 by default, so the
+    # DRAM counters of a capture measure HBM traffic
+    M = args.tokens or (131072 if args.kernel in ("ln_fwd", "ln_bwd") else 32768 if args.kernel == "colsum"
+                        else 4096)
     g = torch.Generator(device="cuda").manual_seed(0)
     torch.cuda.synchronize()
-    if args.kernel == "decode":
+    nbytes = 0
+    if args.kernel in ("ln_fwd", "ln_bwd"):
+        x = torch.randn(M, d, device="cuda", generator=g).to(torch.bfloat16)
+        gam = (1 + 0.1 * torch.randn(d, device="cuda", generator=g)).to(torch.bfloat16)
+        bet = (0.1 * torch.randn(d, device="cuda", generator=g)).to(torch.bfloat16)
+        y = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+        mean, rstd = torch.empty(M, device="cuda"), torch.empty(M, device="cuda")
+        gp.gpt2_op_layernorm_fwd_bf16(x, gam, bet, y, mean, rstd, M, d)
+        if args.kernel == "ln_fwd":
+            fn = lambda: gp.gpt2_op_layernorm_fwd_bf16(x, gam, bet, y, mean, rstd, M, d)  # noqa: E731
+            nbytes = M * (4 * d + 8)                       # x in, y out (bf16), mean + rstd out
+        else:
+            dy = torch.randn(M, d, device="cuda", generator=g).to(torch.bfloat16)
+            dx = torch.zeros(M, d, dtype=torch.bfloat16, device="cuda")
+            dgb = torch.empty(2 * d, device="cuda")
+            scr = torch.empty(gp.gpt2_op_layernorm_bwd_scratch_floats(M, d), device="cuda")
+            # accumulate into dx, as the step adds into the residual-stream gradient
+            fn = lambda: gp.gpt2_op_layernorm_bwd_bf16(dy, x, mean, rstd, gam, dx, 1, dgb, scr, M, d)  # noqa: E731
+            nbytes = M * (8 * d + 8)                       # dy, x, dx in; dx out (bf16); mean + rstd in
+        flop = 0.0
+    elif args.kernel == "colsum":
+        N = 4 * d
+        x = torch.randn(M, N, device="cuda", generator=g).to(torch.bfloat16)
+        out = torch.empty(N, device="cuda")
+        scr = torch.empty(gp.gpt2_op_colsum_scratch_floats(M, N), device="cuda")
+        fn = lambda: gp.gpt2_op_colsum_bf16(x, M, N, out, scr)  # noqa: E731
+        nbytes = M * N * 2                                 # the bias gradient's input, read once
+        flop = 0.0
+    elif args.kernel == "adamw":
+        # the optimizer pass over every parameter of the model (batch 1: the
+        # workspace is not used by this kernel)
+        model = gp.GPT2(gp.ModelConfig(L, d, H, T, Vr, V, 1, 0))
+        model.init_params(seed=0)
+        model.grad.normal_(0.0, 1e-3, generator=g)
+        M = model.n_params
+        stepno = [0]
+
+        def fn():
+            stepno[0] += 1
+            model.adamw_step(stepno[0])
+        nbytes = 30 * M                                    # p, g, m, v in; p, m, v out (fp32); bf16 shadow out
+        flop = 0.0
+    elif args.kernel == "decode":
         # eager decode steps of the 124M model at batch 8 after a 128-token prompt
         model = gp.GPT2(gp.ModelConfig(L, d, H, T, Vr, V, 8, 0))
         model.init_params(seed=0)
@@ -528,15 +575,35 @@ def run_kernel(args):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.reps
-    print(json.dumps({"kernel": args.kernel, "tokens": M, "ms": round(ms, 4),
-                      "tflops": round(flop / ms / 1e9, 1)}))
+    rec = {"kernel": args.kernel, "tokens" if args.kernel != "adamw" else "params": M, "ms": round(ms, 4)}
+    if hbm:
+        peaks, kind = load_peaks()
+        gbs = nbytes / (ms / 1e3) / 1e9
+        rec.update({"algorithmic_bytes": int(nbytes), "gbs": round(gbs, 1),
+                    "frac": round(gbs / peaks["hbm_gbs"], 4), "peak": peaks["hbm_gbs"], "peak_source": kind})
+    else:
+        rec["tflops"] = round(flop / ms / 1e9, 1)
+    print(json.dumps(rec))
+
+
+def relaunch_per_gpu(n):
+    """`bench.py --gpus N` started as a plain process: run the same command as
+    N ranks on this node (torchrun, rendezvous on 127.0.0.1), each rank taking
+    its own GPU, and return the launcher's exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
 
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", choices=["lm_head", "attn_fwd", "attn_bwd", "decode"], default=None,
-                    help="time one kernel alone instead of the step (profiler captures)")
-    ap.add_argument("--tokens", type=int, default=4096)
+    ap.add_argument("--kernel", choices=["lm_head", "attn_fwd", "attn_bwd", "decode"] + list(HBM_KERNELS),
+                    default=None, help="time one kernel alone instead of the step (profiler captures)")
+    ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -554,6 +621,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: relaunch this command under torchrun
+        sys.exit(relaunch_per_gpu(args.gpus))
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

@@ -53,6 +53,8 @@ EXPORTS = [
     "gpt2_kv_cache_bytes", "gpt2_prefill", "gpt2_decode_step", "gpt2_greedy_next",
     "gpt2_op_gemm_bf16", "gpt2_op_attention_fwd_bf16", "gpt2_op_attention_bwd_bf16",
     "gpt2_op_attention_bwd_bf16_noalloc",
+    "gpt2_op_layernorm_fwd_bf16", "gpt2_op_layernorm_bwd_scratch_floats", "gpt2_op_layernorm_bwd_bf16",
+    "gpt2_op_colsum_scratch_floats", "gpt2_op_colsum_bf16",
 ]
 
 _LIB = None
@@ -96,6 +98,11 @@ def _lib():
         "gpt2_op_attention_fwd_bf16": (I, [P, P, P, I, I, I, I, P]),
         "gpt2_op_attention_bwd_bf16": (I, [P, P, P, P, P, P, I, I, I, I, P]),
         "gpt2_op_attention_bwd_bf16_noalloc": (I, [P, P, P, P, P, I, I, I, I, P]),
+        "gpt2_op_layernorm_fwd_bf16": (I, [P, P, P, P, P, P, I, I, P]),
+        "gpt2_op_layernorm_bwd_scratch_floats": (S, [I, I]),
+        "gpt2_op_layernorm_bwd_bf16": (I, [P, P, P, P, P, P, I, P, P, S, I, I, P]),
+        "gpt2_op_colsum_scratch_floats": (S, [I, I]),
+        "gpt2_op_colsum_bf16": (I, [P, I, I, P, P, S, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -274,6 +281,30 @@ def gpt2_op_attention_bwd_bf16_noalloc(qkv, o, lse, dout, dqkv, B, T, H, hd, str
     _check(_lib().gpt2_op_attention_bwd_bf16_noalloc(_ptr(qkv), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dqkv),
                                                      B, T, H, hd, _stream(stream)),
            "gpt2_op_attention_bwd_bf16_noalloc")
+
+
+def gpt2_op_layernorm_fwd_bf16(x, gamma, beta, y, mean, rstd, M, d, stream=None):
+    _check(_lib().gpt2_op_layernorm_fwd_bf16(_ptr(x), _ptr(gamma), _ptr(beta), _ptr(y), _ptr(mean), _ptr(rstd),
+                                             M, d, _stream(stream)), "gpt2_op_layernorm_fwd_bf16")
+
+
+def gpt2_op_layernorm_bwd_scratch_floats(M, d) -> int:
+    return int(_lib().gpt2_op_layernorm_bwd_scratch_floats(M, d))
+
+
+def gpt2_op_layernorm_bwd_bf16(dy, x, mean, rstd, gamma, dx, accumulate, dgamma_dbeta, scratch, M, d, stream=None):
+    _check(_lib().gpt2_op_layernorm_bwd_bf16(_ptr(dy), _ptr(x), _ptr(mean), _ptr(rstd), _ptr(gamma), _ptr(dx),
+                                             accumulate, _ptr(dgamma_dbeta), _ptr(scratch), scratch.numel(), M, d,
+                                             _stream(stream)), "gpt2_op_layernorm_bwd_bf16")
+
+
+def gpt2_op_colsum_scratch_floats(M, N) -> int:
+    return int(_lib().gpt2_op_colsum_scratch_floats(M, N))
+
+
+def gpt2_op_colsum_bf16(x, M, N, out, scratch, stream=None):
+    _check(_lib().gpt2_op_colsum_bf16(_ptr(x), M, N, _ptr(out), _ptr(scratch), scratch.numel(), _stream(stream)),
+           "gpt2_op_colsum_bf16")
 
 
 # ------------------------------------------------------------ convenience ---

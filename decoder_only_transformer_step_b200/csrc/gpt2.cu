@@ -792,4 +792,51 @@ int gpt2_op_attention_bwd_bf16(const uint16_t* qkv, const uint16_t* o, const flo
   return attn_bwd_bf16(qkv, o, lse, dout, dqkv, dq_acc, dvec, B, T, H, hd, S(stream));
 }
 
+// ---- single HBM-bound steps of the path (kernel tests and profiling) ----
+
+int gpt2_op_layernorm_fwd_bf16(const uint16_t* x, const uint16_t* gamma, const uint16_t* beta, uint16_t* y,
+                               float* mean, float* rstd, int M, int d, void* stream) {
+  if (!x || !gamma || !beta || !y || !mean || !rstd || M < 0 || d < 1) return GPT2_ERR_INVALID_ARG;
+  if (d % 64 || d > 2048) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (((uintptr_t)x | (uintptr_t)y | (uintptr_t)gamma | (uintptr_t)beta) & 15) return GPT2_ERR_INVALID_ARG;
+  if (M == 0) return GPT2_OK;
+  return layernorm_fwd(0, x, gamma, beta, y, mean, rstd, M, d, S(stream));
+}
+
+size_t gpt2_op_layernorm_bwd_scratch_floats(int M, int d) {
+  if (M < 1 || d < 1) return 0;
+  return layernorm_bwd_part_floats(M, d);
+}
+
+int gpt2_op_layernorm_bwd_bf16(const uint16_t* dy, const uint16_t* x, const float* mean, const float* rstd,
+                               const uint16_t* gamma, uint16_t* dx, int accumulate, float* dgamma_dbeta,
+                               float* scratch, size_t scratch_floats, int M, int d, void* stream) {
+  if (!dy || !x || !mean || !rstd || !gamma || !dx || !dgamma_dbeta || !scratch || M < 1 || d < 1)
+    return GPT2_ERR_INVALID_ARG;
+  if (d % 64 || d > 2048) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (((uintptr_t)dy | (uintptr_t)x | (uintptr_t)dx | (uintptr_t)gamma | (uintptr_t)scratch) & 15)
+    return GPT2_ERR_INVALID_ARG;
+  if (scratch_floats < layernorm_bwd_part_floats(M, d)) return GPT2_ERR_WORKSPACE;
+  const cudaStream_t st = S(stream);
+  int nblk = 0;
+  TRY(layernorm_bwd(0, dy, x, mean, rstd, gamma, dx, accumulate ? 0 : 1, scratch, nullptr, &nblk, M, d, st));
+  return reduce_rows_f32(scratch, nblk, 2 * d, dgamma_dbeta, 0.f, st);
+}
+
+size_t gpt2_op_colsum_scratch_floats(int M, int N) {
+  if (M < 1 || N < 1) return 0;
+  return colsum_part_floats(M, N);
+}
+
+int gpt2_op_colsum_bf16(const uint16_t* x, int M, int N, float* out, float* scratch, size_t scratch_floats,
+                        void* stream) {
+  if (!x || !out || !scratch || M < 1 || N < 1) return GPT2_ERR_INVALID_ARG;
+  if (N % 8 || ((uintptr_t)x & 15)) return GPT2_ERR_INVALID_ARG;
+  if (scratch_floats < colsum_part_floats(M, N)) return GPT2_ERR_WORKSPACE;
+  const cudaStream_t st = S(stream);
+  int nblk = 0;
+  TRY(colsum_partial(0, x, M, N, scratch, &nblk, st));
+  return reduce_rows_f32(scratch, nblk, N, out, 0.f, st);
+}
+
 }  // extern "C"

@@ -299,14 +299,56 @@ int gpt2_op_attention_bwd_bf16(const uint16_t* qkv, const uint16_t* o, const flo
  * cudaMalloc's device synchronisation.  Its scratch (fp32 dQ accumulator and
  * D vector, B*T*H*hd + B*H*T floats) lives in a 16 MiB array compiled into the
  * library, which every GPU that loads the library holds until the process
- * exits.  Larger problems return GPT2_ERR_TOO_LARGE.  The first call on a
- * device looks up that device's address of the array (cudaGetSymbolAddress);
- * make that first call before any stream capture.  All calls share the one
- * array: calls that may overlap on the GPU (unordered streams) race and must
- * not be issued.  It calls no allocator. */
+ * exits.  hd < 1 returns GPT2_ERR_INVALID_ARG and an hd other than 16 or 64
+ * GPT2_ERR_UNSUPPORTED_SHAPE, as for the scratch-taking call; a supported
+ * shape whose scratch exceeds the array returns GPT2_ERR_TOO_LARGE.  Every
+ * call made outside a stream capture looks up the array's address in the
+ * current context (cudaGetSymbolAddress), so a cudaDeviceReset or another
+ * context being current is picked up; inside a capture the address recorded
+ * by the last uncaptured call on that device is used, and a capture with no
+ * such earlier call returns GPT2_ERR_BAD_STATE.  Make the first call on a
+ * device before any stream capture, and call it again (uncaptured) after a
+ * cudaDeviceReset before capturing.  All calls share the one array: calls
+ * that may overlap on the GPU (unordered streams) race and must not be
+ * issued.  It calls no allocator. */
 int gpt2_op_attention_bwd_bf16_noalloc(const uint16_t* qkv, const uint16_t* o, const float* lse,
                                        const uint16_t* dout, uint16_t* dqkv,
                                        int B, int T, int H, int hd, void* stream);
+
+/* ---- single HBM-bound steps of the path, for kernel tests and profiling --
+ * bf16 activations, row-major, 16-byte aligned; d a multiple of 64 up to
+ * 2048 (GPT2_ERR_UNSUPPORTED_SHAPE otherwise).  Asynchronous on `stream`. */
+
+/* LayerNorm forward over M rows of width d ("Pré-treinar um LLM" and the
+ * pre-LayerNorm block of GPT-2): per row mean and biased variance, eps 1e-5,
+ * y = (x - mean) * rstd * gamma + beta.  x, y bf16 [M, d]; gamma, beta bf16
+ * [d]; mean, rstd fp32 [M] (saved for the backward). */
+int gpt2_op_layernorm_fwd_bf16(const uint16_t* x, const uint16_t* gamma, const uint16_t* beta, uint16_t* y,
+                               float* mean, float* rstd, int M, int d, void* stream);
+
+/* Floats of scratch gpt2_op_layernorm_bwd_bf16 needs (0 for M or d < 1). */
+size_t gpt2_op_layernorm_bwd_scratch_floats(int M, int d);
+
+/* Its backward (the chain rule of the forward above): dx (=, or += with
+ * accumulate) the input gradient, bf16 [M, d]; dgamma_dbeta fp32 [2d] =
+ * (sum over rows of dy * xhat, sum over rows of dy), written.  mean, rstd as
+ * the forward saved them.  scratch: device fp32 of at least
+ * gpt2_op_layernorm_bwd_scratch_floats(M, d) (GPT2_ERR_WORKSPACE if smaller);
+ * the row-block partial sums, added in a fixed order. */
+int gpt2_op_layernorm_bwd_bf16(const uint16_t* dy, const uint16_t* x, const float* mean, const float* rstd,
+                               const uint16_t* gamma, uint16_t* dx, int accumulate, float* dgamma_dbeta,
+                               float* scratch, size_t scratch_floats, int M, int d, void* stream);
+
+/* Floats of scratch gpt2_op_colsum_bf16 needs (0 for M or N < 1). */
+size_t gpt2_op_colsum_scratch_floats(int M, int N);
+
+/* Column sums of x (bf16 [M, N], N a multiple of 8): out[n] = sum_m x[m, n]
+ * (fp32 [N], written), the bias gradient of a linear layer ("Pré-treinar um
+ * LLM", compute section: the backward's gradients of each layer).  Row-block
+ * partials in scratch (at least gpt2_op_colsum_scratch_floats(M, N) floats),
+ * added in a fixed order. */
+int gpt2_op_colsum_bf16(const uint16_t* x, int M, int N, float* out, float* scratch, size_t scratch_floats,
+                        void* stream);
 
 #ifdef __cplusplus
 }

@@ -127,3 +127,22 @@ def test_null_context_calls_are_rejected_on_host():
     assert L.gpt2_prefill(None, None, 0, 1, 1, None, None, None, None) == bad
     assert L.gpt2_decode_step(None, None, 0, 1, 1, None, None, None, None) == bad
     assert L.gpt2_greedy_next(None, None, 1, None, None, None) == bad
+
+
+def test_noalloc_attention_backward_validates_shape_before_scratch_size():
+    # a head size below 1 is an invalid argument and an unsupported head size
+    # an unsupported shape, as for the scratch-taking call, even where the
+    # problem would also exceed the built-in scratch; all decided on the host
+    # before any CUDA call (dummy, never-dereferenced pointers)
+    L = gp._lib()
+    p = ctypes.c_void_p(256)
+    inv = gp.ERRORS_BY_NAME["GPT2_ERR_INVALID_ARG"]
+    uns = gp.ERRORS_BY_NAME["GPT2_ERR_UNSUPPORTED_SHAPE"]
+    assert L.gpt2_op_attention_bwd_bf16_noalloc(p, p, p, p, p, 64, 1024, 12, -1, None) == inv
+    assert L.gpt2_op_attention_bwd_bf16_noalloc(p, p, p, p, p, 64, 1024, 12, 0, None) == inv
+    assert L.gpt2_op_attention_bwd_bf16_noalloc(p, p, p, p, p, 64, 1024, 12, 32, None) == uns
+    assert L.gpt2_op_attention_bwd_bf16_noalloc(p, p, p, p, p, 1, 64, 2, 128, None) == uns
+    assert L.gpt2_op_attention_bwd_bf16_noalloc(None, p, p, p, p, 1, 64, 2, 64, None) == inv
+    # a supported shape just past the 4 Mi-float array
+    assert L.gpt2_op_attention_bwd_bf16_noalloc(p, p, p, p, p, 1, 4096, 16, 64, None) == \
+        gp.ERRORS_BY_NAME["GPT2_ERR_TOO_LARGE"]

@@ -207,3 +207,50 @@ def test_attention_backward(hd, T):
         cos = (g * r).sum() / (np.linalg.norm(g) * np.linalg.norm(r))
         rel = np.abs(g - r).max() / np.abs(r).max()
         assert cos >= 0.999 and rel <= 2e-2, (name, cos, rel)
+
+
+@pytest.mark.parametrize("M,d", [(1000, 768), (77, 1600), (4096, 1024)])
+def test_layernorm_ops_against_oracle(M, d):
+    """The LayerNorm forward and backward kernels alone, on ragged row counts
+    and the three model widths, against the oracle's LayerNorm on the same
+    bf16 inputs: y and dx element-wise within 1e-2 of their largest entry,
+    mean / rstd and the fp32 gamma / beta gradients within 1e-4."""
+    x = bf16_rand((M, d), 70 + M, scale=2.0) + 0.5
+    gamma = bf16_rand((d,), 71, scale=0.1) + 1.0
+    beta = bf16_rand((d,), 72, scale=0.1)
+    dy = bf16_rand((M, d), 73 + M)
+    y = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
+    mean = torch.empty(M, device="cuda")
+    rstd = torch.empty(M, device="cuda")
+    gp.gpt2_op_layernorm_fwd_bf16(x.cuda(), gamma.cuda(), beta.cuda(), y, mean, rstd, M, d)
+    X, Gm, Bt, DY = (t.double().numpy() for t in (x, gamma, beta, dy))
+    y_ref, saved = G.layernorm_fwd(X, Gm, Bt)
+    assert np.abs(y.double().cpu().numpy() - y_ref).max() <= 1e-2 * np.abs(y_ref).max()
+    assert np.abs(mean.double().cpu().numpy() - X.mean(-1)).max() <= 1e-4 * np.abs(X).max()
+    assert np.abs(rstd.double().cpu().numpy() / saved[1][:, 0] - 1).max() <= 1e-4
+    dx_ref, dg_ref, db_ref = G.layernorm_bwd(DY, Gm, saved)
+    scratch = torch.empty(gp.gpt2_op_layernorm_bwd_scratch_floats(M, d), device="cuda")
+    dgb = torch.empty(2 * d, device="cuda")
+    prev = bf16_rand((M, d), 74 + M)
+    for accumulate in (0, 1):
+        dx = prev.cuda().clone()
+        gp.gpt2_op_layernorm_bwd_bf16(dy.cuda(), x.cuda(), mean, rstd, gamma.cuda(), dx, accumulate, dgb, scratch,
+                                      M, d)
+        want = dx_ref + (prev.double().numpy() if accumulate else 0.0)
+        assert np.abs(dx.double().cpu().numpy() - want).max() <= 1e-2 * np.abs(want).max(), accumulate
+        got = dgb.double().cpu().numpy()
+        assert np.abs(got[:d] - dg_ref).max() <= 1e-4 * np.abs(dg_ref).max()
+        assert np.abs(got[d:] - db_ref).max() <= 1e-4 * np.abs(db_ref).max()
+
+
+@pytest.mark.parametrize("M,N", [(16384, 3072), (1000, 2304), (77, 64)])
+def test_colsum_op_exact_sums(M, N):
+    """Bias gradients: the column sums of a bf16 matrix against the exact
+    (fp64) sums of the same values; fp32 accumulation keeps the error far
+    below 1e-5 of the sum of magnitudes."""
+    x = bf16_rand((M, N), 80 + M)
+    out = torch.empty(N, device="cuda")
+    scratch = torch.empty(gp.gpt2_op_colsum_scratch_floats(M, N), device="cuda")
+    gp.gpt2_op_colsum_bf16(x.cuda(), M, N, out, scratch)
+    X = x.double().numpy()
+    assert np.abs(out.double().cpu().numpy() - X.sum(0)).max() <= 1e-5 * np.abs(X).sum(0).max()
