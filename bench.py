@@ -488,7 +488,7 @@ def run_kernel(args):
     # HBM-bound kernels: inputs larger than the 126 MB L2 by default, so the
     # DRAM counters of a capture measure HBM traffic
     M = args.tokens or (131072 if args.kernel in ("ln_fwd", "ln_bwd") else 32768 if args.kernel == "colsum"
-                        else 4096)
+                        else 16384 if args.kernel.startswith("lm_head_ce") else 4096)
     g = torch.Generator(device="cuda").manual_seed(0)
     torch.cuda.synchronize()
     nbytes = 0
@@ -545,6 +545,24 @@ def run_kernel(args):
             cache.step()
             cache.greedy_advance()
         flop = 2.0 * 8 * (L * 12 * d * d + V * d)
+    elif args.kernel in ("lm_head_ce", "lm_head_ce_bwd"):
+        # the tied LM head with the fused cross-entropy (op entry points): the
+        # forward GEMM with the log-sum-exp epilogue, target count, merge and
+        # mean; or the two backward GEMMs with the softmax in their operand staging
+        A = torch.randn(M, d, device="cuda", generator=g).to(torch.bfloat16)
+        W = (0.02 * torch.randn(V, d, device="cuda", generator=g)).to(torch.bfloat16)
+        tgt = torch.randint(0, Vr, (M,), device="cuda", generator=g, dtype=torch.int32)
+        scr = torch.empty(gp.gpt2_op_lm_head_ce_scratch_bytes(M, V), dtype=torch.uint8, device="cuda")
+        loss, rows = torch.empty(1, device="cuda"), torch.empty(M, device="cuda")
+        gp.gpt2_op_lm_head_ce_fwd_bf16(A, W, tgt, M, V, d, Vr, loss, rows, scr)
+        if args.kernel == "lm_head_ce":
+            fn = lambda: gp.gpt2_op_lm_head_ce_fwd_bf16(A, W, tgt, M, V, d, Vr, loss, rows, scr)  # noqa: E731
+            flop = 2.0 * M * V * d
+        else:
+            dx = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+            dw = torch.empty(V, d, device="cuda")
+            fn = lambda: gp.gpt2_op_lm_head_ce_bwd_bf16(A, W, M, V, d, 1.0, dx, dw, 0, scr)  # noqa: E731
+            flop = 4.0 * M * V * d
     elif args.kernel == "lm_head":
         A = torch.randn(M, d, device="cuda", generator=g).to(torch.bfloat16)
         W = (0.02 * torch.randn(V, d, device="cuda", generator=g)).to(torch.bfloat16)
@@ -601,7 +619,8 @@ def relaunch_per_gpu(n):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", choices=["lm_head", "attn_fwd", "attn_bwd", "decode"] + list(HBM_KERNELS),
+    ap.add_argument("--kernel", choices=["lm_head", "lm_head_ce", "lm_head_ce_bwd", "attn_fwd", "attn_bwd",
+                                         "decode"] + list(HBM_KERNELS),
                     default=None, help="time one kernel alone instead of the step (profiler captures)")
     ap.add_argument("--tokens", type=int, default=None)
     ap.add_argument("--reps", type=int, default=3)

@@ -55,6 +55,7 @@ EXPORTS = [
     "gpt2_op_attention_bwd_bf16_noalloc",
     "gpt2_op_layernorm_fwd_bf16", "gpt2_op_layernorm_bwd_scratch_floats", "gpt2_op_layernorm_bwd_bf16",
     "gpt2_op_colsum_scratch_floats", "gpt2_op_colsum_bf16",
+    "gpt2_op_lm_head_ce_scratch_bytes", "gpt2_op_lm_head_ce_fwd_bf16", "gpt2_op_lm_head_ce_bwd_bf16",
 ]
 
 _LIB = None
@@ -103,6 +104,9 @@ def _lib():
         "gpt2_op_layernorm_bwd_bf16": (I, [P, P, P, P, P, P, I, P, P, S, I, I, P]),
         "gpt2_op_colsum_scratch_floats": (S, [I, I]),
         "gpt2_op_colsum_bf16": (I, [P, I, I, P, P, S, P]),
+        "gpt2_op_lm_head_ce_scratch_bytes": (S, [I, I]),
+        "gpt2_op_lm_head_ce_fwd_bf16": (I, [P, P, P, I, I, I, I, P, P, P, S, P]),
+        "gpt2_op_lm_head_ce_bwd_bf16": (I, [P, P, I, I, I, F, P, P, I, P, S, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -305,6 +309,22 @@ def gpt2_op_colsum_scratch_floats(M, N) -> int:
 def gpt2_op_colsum_bf16(x, M, N, out, scratch, stream=None):
     _check(_lib().gpt2_op_colsum_bf16(_ptr(x), M, N, _ptr(out), _ptr(scratch), scratch.numel(), _stream(stream)),
            "gpt2_op_colsum_bf16")
+
+
+def gpt2_op_lm_head_ce_scratch_bytes(M, V) -> int:
+    return int(_lib().gpt2_op_lm_head_ce_scratch_bytes(M, V))
+
+
+def gpt2_op_lm_head_ce_fwd_bf16(x, w, targets, M, V, d, vocab_real, loss, loss_rows, scratch, stream=None):
+    _check(_lib().gpt2_op_lm_head_ce_fwd_bf16(_ptr(x), _ptr(w), _ptr(targets), M, V, d, vocab_real, _ptr(loss),
+                                              _ptr(loss_rows), _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                              _stream(stream)), "gpt2_op_lm_head_ce_fwd_bf16")
+
+
+def gpt2_op_lm_head_ce_bwd_bf16(x, w, M, V, d, grad_scale, dx, dw, accumulate, scratch, stream=None):
+    _check(_lib().gpt2_op_lm_head_ce_bwd_bf16(_ptr(x), _ptr(w), M, V, d, grad_scale, _ptr(dx), _ptr(dw), accumulate,
+                                              _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                              _stream(stream)), "gpt2_op_lm_head_ce_bwd_bf16")
 
 
 # ------------------------------------------------------------ convenience ---

@@ -19,6 +19,7 @@
 // so S(j+1) is computed while the softmax of tile j runs.  Every mbarrier wait
 // is bounded; a timeout sets the device status and the CTA drains and exits.
 #include <cuda.h>
+#include <stdlib.h>
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -414,6 +415,352 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// ---------------------------------------------- forward, two query tiles --
+// Persistent; a work item is two consecutive 128-query blocks (2i, 2i+1) of one
+// (batch, head), so the K/V tiles are loaded once for both.  Each of the two
+// query tiles has its own softmax warpgroup (four warps, one thread per query
+// row, so a row's maximum needs no exchange) and its own tensor-memory
+// region: S (128 fp32 columns), O (64) and P (64 columns of bf16 pairs).  O is
+// accumulated by the tensor cores (P V with P read from tensor memory); a row
+// rescales it only when its running maximum grows by more than 2^8, otherwise
+// the probabilities are formed against the stale maximum (at most 256, exact
+// in the final O / l).  The MMA warp issues S of a tile's next key block right
+// after that tile's P V, so one warpgroup's exponentials overlap the other's
+// and the tensor-core work of both.
+//   warp 0      TMA: both tiles' Q (two item slots), K/V ring
+//   warp 1      TMEM allocation, MMA issue
+//   warps 2..5  softmax + output of tile 0, warps 6..9 of tile 1
+constexpr int F2_KVS = 4;
+constexpr int F2_Q = 0;                          // [slot 2][tile 2] Q / O staging
+constexpr int F2_K = F2_Q + 4 * TILE;
+constexpr int F2_V = F2_K + F2_KVS * TILE;
+constexpr int F2_TILES = F2_V + F2_KVS * TILE;
+// q_full[2], q_empty[2], kv_full[KVS], kv_empty[KVS], then per tile s_full,
+// s_free, p_full, pv_done, o_free, o_staged, and drain
+constexpr int F2_NUM_BARS = 4 + 2 * F2_KVS + 12 + 1;
+constexpr int F2_SMEM = F2_TILES + 1024 + F2_NUM_BARS * 8 + 16;
+static_assert(F2_SMEM <= 232448, "forward shared memory");
+constexpr float F2_RESCALE = 8.f;  // log2 of the largest un-rescaled probability
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmO,
+                        float* __restrict__ lse, int T, int H, int n_items, float scale_log2, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t bars = base + F2_TILES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + F2_TILES + F2_NUM_BARS * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto q_full = [&](int s) { return bars + 8u * s; };
+  auto q_empty = [&](int s) { return bars + 8u * (2 + s); };
+  auto kv_full = [&](int s) { return bars + 8u * (4 + s); };
+  auto kv_empty = [&](int s) { return bars + 8u * (4 + F2_KVS + s); };
+  // per-tile barriers: k = 0 s_full, 1 s_free, 2 p_full, 3 pv_done, 4 o_free, 5 o_staged
+  auto tbar = [&](int t, int k) { return bars + 8u * (4 + 2 * F2_KVS + 6 * t + k); };
+  const uint32_t drain_bar = bars + 8u * (4 + 2 * F2_KVS + 12);
+  auto qbuf = [&](int slot, int t) { return base + F2_Q + (uint32_t)(2 * slot + t) * TILE; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = (T + BQ - 1) / BQ;
+  const int npairs = (nqb + 1) / 2;
+  const int BH = n_items / npairs;
+  const int d = H * HD;
+  // work item -> (first query block, batch, head); longest items first
+  auto item = [&](int w, int& qa, int& b, int& h) {
+    qa = 2 * (npairs - 1 - w / BH);
+    const int bh = w % BH;
+    b = bh / H;
+    h = bh % H;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(q_full(s), 1);
+      mbar_init(q_empty(s), 2);  // one arrival per softmax warpgroup
+    }
+    for (int s = 0; s < F2_KVS; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(tbar(t, 0), 1);
+      mbar_init(tbar(t, 1), 4);
+      mbar_init(tbar(t, 2), 4);
+      mbar_init(tbar(t, 3), 1);
+      mbar_init(tbar(t, 4), 4);
+      mbar_init(tbar(t, 5), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tmQKV);
+    tma_prefetch_desc(&tmO);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_start();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- TMA ----
+      bool ok = true;
+      int g = 0, it = 0, q_issued = 0, kv_issued = 0;
+      for (int k = 0; ok; ++k, ++it) {
+        const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
+        if (w >= n_items) break;
+        int qa, b, h;
+        item(w, qa, b, h);
+        const bool hasb = qa + 1 < nqb;
+        const int nkb = hasb ? qa + 2 : qa + 1;
+        const int slot = it & 1;
+        // both Q buffers of the slot were last used by item it-2, whose O
+        // stores have read them
+        if (it >= 2 && !mbar_wait_bounded(q_empty(slot), ((it - 2) >> 1) & 1, abort_flag, err)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(q_full(slot), (hasb ? 2 : 1) * TILE);
+        tma_load_3d(qbuf(slot, 0), &tmQKV, q_full(slot), h * HD, qa * BQ, b);
+        if (hasb) tma_load_3d(qbuf(slot, 1), &tmQKV, q_full(slot), h * HD, (qa + 1) * BQ, b);
+        ++q_issued;
+        for (int j = 0; j < nkb; ++j, ++g) {
+          const int st = g % F2_KVS;
+          if (g >= F2_KVS && !mbar_wait_bounded(kv_empty(st), ((g - F2_KVS) / F2_KVS) & 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(kv_full(st), 2 * TILE);
+          tma_load_3d(base + F2_K + st * TILE, &tmQKV, kv_full(st), d + h * HD, j * BKV, b);
+          tma_load_3d(base + F2_V + st * TILE, &tmQKV, kv_full(st), 2 * d + h * HD, j * BKV, b);
+          ++kv_issued;
+        }
+      }
+      if (!ok) {
+        for (int i = q_issued - 2 < 0 ? 0 : q_issued - 2; i < q_issued; ++i)
+          mbar_drain_bounded(q_full(i & 1), (i >> 1) & 1);
+        for (int i = kv_issued - F2_KVS < 0 ? 0 : kv_issued - F2_KVS; i < kv_issued; ++i)
+          mbar_drain_bounded(kv_full(i % F2_KVS), (i / F2_KVS) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- MMA ----
+      bool ok = true, issued_any = false;
+      int nS[2] = {0, 0}, nP[2] = {0, 0}, nI[2] = {0, 0};
+      int g0 = 0, it = 0, kv_ready = 0;  // K/V blocks (counted over items) known to have landed
+      for (int k = 0; ok; ++k, ++it) {
+        const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
+        if (w >= n_items) break;
+        int qa, b, h;
+        item(w, qa, b, h);
+        const bool hasb = qa + 1 < nqb;
+        const int nkb = hasb ? qa + 2 : qa + 1;
+        const int slot = it & 1;
+        if (!mbar_wait_bounded(q_full(slot), (it >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        auto issue_s = [&](int t, int j) -> bool {
+          const int gg = g0 + j;
+          while (kv_ready <= gg) {
+            if (!mbar_wait_bounded(kv_full(kv_ready % F2_KVS), (kv_ready / F2_KVS) & 1, abort_flag, err))
+              return false;
+            ++kv_ready;
+          }
+          // the softmax has loaded this tile's previous S
+          if (nS[t] >= 1 && !mbar_wait_bounded(tbar(t, 1), (nS[t] - 1) & 1, abort_flag, err)) return false;
+          tc_fence_after();
+          const uint32_t qb = qbuf(slot, t), kb = base + F2_K + (gg % F2_KVS) * TILE;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk)
+            tc_mma_bf16(tmem + 256u * t, sdesc(qb + kk * 32, 16, 1024), sdesc(kb + kk * 32, 16, 1024), IDESC_S,
+                        kk > 0 ? 1u : 0u);
+          tc_commit(tbar(t, 0));
+          ++nS[t];
+          issued_any = true;
+          return true;
+        };
+        auto issue_pv = [&](int t, int j) -> bool {
+          if (!mbar_wait_bounded(tbar(t, 2), nP[t] & 1, abort_flag, err)) return false;
+          // the first block of an item overwrites O: the previous item's
+          // output must have been read out of tensor memory
+          if (j == 0 && nI[t] >= 1 && !mbar_wait_bounded(tbar(t, 4), (nI[t] - 1) & 1, abort_flag, err))
+            return false;
+          tc_fence_after();
+          const uint32_t vb = base + F2_V + ((g0 + j) % F2_KVS) * TILE;
+#pragma unroll
+          for (int kk = 0; kk < BKV / 16; ++kk)
+            tc_mma_bf16_ts(tmem + 256u * t + 128u, tmem + 256u * t + 192u + 8u * kk, sdesc(vb + kk * 2048, 8192, 1024),
+                           IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(tbar(t, 3));
+          ++nP[t];
+          return true;
+        };
+        ok = issue_s(0, 0) && (!hasb || issue_s(1, 0));
+        for (int j = 0; j < nkb && ok; ++j) {
+          if (j <= qa) {
+            if (!issue_pv(0, j) || (j + 1 <= qa && !issue_s(0, j + 1))) { ok = false; break; }
+          }
+          if (hasb) {
+            if (!issue_pv(1, j) || (j + 1 < nkb && !issue_s(1, j + 1))) { ok = false; break; }
+          }
+          // every MMA reading this K/V slot has been issued
+          tc_commit(kv_empty((g0 + j) % F2_KVS));
+        }
+        ++nI[0];
+        if (hasb) ++nI[1];
+        g0 += nkb;
+      }
+      if (!ok && issued_any) {
+        tc_commit(drain_bar);
+        mbar_drain_bounded(drain_bar, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------- softmax, output ----
+    const int t = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int q = warp & 3;         // TMEM lanes [32q, 32q+32)
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t tS = tmem + lane_off + 256u * t, tO = tS + 128u, tP = tS + 192u;
+    const bool leader = (warp & 3) == 2 && lane == 0;  // first warp of the warpgroup
+    bool ok = true;
+    int ns = 0, np = 0, nit = 0;
+    for (int k = 0; ok; ++k) {
+      const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
+      if (w >= n_items) break;
+      int qa, b, h;
+      item(w, qa, b, h);
+      const int slot = k & 1;
+      const int qt = qa + t;  // this tile's query block
+      if (qt >= nqb) {
+        // tile 1 absent (an odd number of query blocks): nothing to compute
+        if (leader) mbar_arrive(q_empty(slot));
+        continue;
+      }
+      const int grow = qt * BQ + row;
+      float m_use = -INFINITY, l = 0.f;
+      for (int j = 0; j <= qt; ++j) {
+        if (!mbar_wait_bounded(tbar(t, 0), ns & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t v[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + 32u * c, v[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tbar(t, 1));
+        ++ns;
+        // raw scores; keys past the query masked on the diagonal block
+        float mx = -INFINITY;
+        if (j == qt) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float x = (32 * c + i > row) ? -INFINITY : __uint_as_float(v[c][i]);
+              v[c][i] = __float_as_uint(x);
+              mx = fmaxf(mx, x);
+            }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(v[c][i]));
+        }
+        const float m_new = fmaxf(m_use, mx * scale_log2);
+        float alpha = 1.f;
+        bool resc = false;
+        if (j == 0) {
+          m_use = m_new;
+        } else if (m_new > m_use + F2_RESCALE) {
+          alpha = ex2(m_use - m_new);
+          m_use = m_new;
+          resc = true;
+        }
+        // P V of the previous block has finished reading P and writing O
+        if (np >= 1 && !mbar_wait_bounded(tbar(t, 3), (np - 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2(fmaf(__uint_as_float(v[c][2 * i]), scale_log2, -m_use));
+            const float p1 = ex2(fmaf(__uint_as_float(v[c][2 * i + 1]), scale_log2, -m_use));
+            sum += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_32x32b_x16(tP + 16u * c, pk);
+        }
+        l = l * alpha + sum;
+        if (__any_sync(0xffffffffu, resc)) {
+          // rare: this warp's rows whose maximum grew rescale their O
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(tO + 32u * hh, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st_32x32b_x32(tO + 32u * hh, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tbar(t, 2));
+        ++np;
+      }
+      if (!ok) break;
+      // ---- output: O / l in bf16 through this tile's Q buffer, one TMA store
+      if (!mbar_wait_bounded(tbar(t, 3), (np - 1) & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t o[2][32];
+      tmem_ld_32x32b_x32(tO, o[0]);
+      tmem_ld_32x32b_x32(tO + 32u, o[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tbar(t, 4));
+      const float inv = 1.f / l;
+      const uint32_t ob = qbuf(slot, t) + (uint32_t)row * 128u;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t* oc = &o[c >> 2][(c & 3) * 8];
+        st_shared_v4(ob + 16u * (uint32_t)(c ^ (row & 7)),
+                     pack_bf16x2(__uint_as_float(oc[0]) * inv, __uint_as_float(oc[1]) * inv),
+                     pack_bf16x2(__uint_as_float(oc[2]) * inv, __uint_as_float(oc[3]) * inv),
+                     pack_bf16x2(__uint_as_float(oc[4]) * inv, __uint_as_float(oc[5]) * inv),
+                     pack_bf16x2(__uint_as_float(oc[6]) * inv, __uint_as_float(oc[7]) * inv));
+      }
+      if (grow < T) lse[((long)b * H + h) * T + grow] = (m_use + __log2f(l)) * LN2_F;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tbar(t, 5));
+      if (!mbar_wait_bounded(tbar(t, 5), nit & 1, abort_flag, err)) { ok = false; break; }
+      ++nit;
+      if (leader) {
+        tma_store_3d(&tmO, qbuf(slot, t), h * HD, qt * BQ, b);
+        bulk_commit();
+        bulk_wait_read<0>();
+        mbar_arrive(q_empty(slot));
+      }
+      __syncwarp();
+    }
+    if (leader) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 // ----------------------------------------------------------------- backward --
 // One CTA per (batch, head, 128-key block), looping over the query blocks at or
 // below the diagonal.  Per query block t:
@@ -787,6 +1134,25 @@ int attn_fwd_tc(const void* qkv, void* o, float* lse, int B, int T, int H, cudaS
   const uint64_t dout[3] = {d, (uint64_t)T, (uint64_t)B};
   const uint64_t sout[2] = {d * 2, (uint64_t)T * d * 2};
   if (!tmap_3d(&tq, qkv, dq, sq) || !tmap_3d(&to, o, dout, sout)) return GPT2_ERR_CUDA;
+  static int v2 = -1;
+  if (v2 < 0) {
+    const char* e = getenv("GPT2_ATTN_FWD_TC");
+    v2 = (e && e[0] == '1') ? 0 : 1;  // "1": the one-tile kernel, for comparison
+  }
+  if (v2) {
+    static bool attr2 = false;
+    if (!attr2) {
+      CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F2_SMEM));
+      attr2 = true;
+    }
+    const int nqb = (T + BQ - 1) / BQ;
+    const int n_items = ((nqb + 1) / 2) * B * H;
+    const int grid = n_items < num_sms() ? n_items : num_sms();
+    CUDA_TRY(launch_k(attn_fwd_tc2_kernel, grid, NUM_THREADS, F2_SMEM, st, tq, to, lse, T, H, n_items,
+                      LOG2E_F / 8.f, nullptr));
+    LAUNCH_CHECK();
+    return GPT2_OK;
+  }
   static bool attr = false;
   if (!attr) {
     CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));

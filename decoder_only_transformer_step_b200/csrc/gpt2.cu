@@ -104,6 +104,10 @@ struct Work {
   std::vector<LayerActs> layers;
   void *x_final, *yf, *logits;
   float *meanf, *rstdf, *loss_rows;
+  // fused cross-entropy (bf16): per-part maxima (then the backward scales)
+  // and sums [V/128][M], target logits, effective targets, M / n_valid
+  float *ce_pm, *ce_ps, *ce_zt, *ce_onehot;
+  int32_t* tgt_eff;
   void *dres, *dy, *du, *dqkv, *dout;
   float *dq_acc, *dvec;
   float *norm_part, *gnorm;  // global gradient norm: block partials and the result
@@ -168,6 +172,12 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
   w->rstdf = c.take<float>(M * 4);
   w->logits = c.take<void>(M * s.V * act);
   w->loss_rows = c.take<float>(M * 4);
+  const long parts = s.V / 128;
+  w->ce_pm = c.take<float>((size_t)parts * M * 4);
+  w->ce_ps = c.take<float>((size_t)parts * M * 4);
+  w->ce_zt = c.take<float>(M * 4);
+  w->tgt_eff = c.take<int32_t>(M * 4);
+  w->ce_onehot = c.take<float>(4);
   w->dres = c.take<void>(M * d * act);
   w->dy = c.take<void>(M * d * act);
   w->du = c.take<void>(M * 4 * d * act);
@@ -392,9 +402,12 @@ int gpt2_zero_grad(gpt2_ctx* c, void* stream) {
 
 namespace {
 
-// The forward up to the logits [batch * T, V] in w.logits; every layer's
-// activations stay in the workspace.
-int forward_logits(gpt2_ctx* c, const int32_t* tokens, int batch, cudaStream_t st) {
+// The forward up to the LM head; every layer's activations stay in the
+// workspace.  Plain: the logits [batch * T, V] in w.logits.  ce_fused (bf16):
+// the LM-head GEMM computes the cross-entropy's per-part maxima and sums of
+// exp(z - max) in its epilogue and stores those exponentials (bf16) in
+// w.logits instead of z, plus the target logits (w.tgt must hold the targets).
+int forward_logits(gpt2_ctx* c, const int32_t* tokens, int batch, cudaStream_t st, bool ce_fused = false) {
   const Shape& s = c->s;
   const int M = batch * (int)s.T, d = (int)s.d, V = (int)s.V;
   Work& w = c->w;
@@ -433,7 +446,13 @@ int forward_logits(gpt2_ctx* c, const int32_t* tokens, int batch, cudaStream_t s
     TRY(run_gemm(c, g, st));
   }
   TRY(layernorm_fwd(f32, w.x_final, Wp(c, o.lnf_g()), Wp(c, o.lnf_b()), w.yf, w.meanf, w.rstdf, M, d, st));
-  GemmArgs g = make_gemm(M, V, d, w.yf, 0, d, Wp(c, o.wte()), 0, d, EPI_STORE, w.logits, V);
+  GemmArgs g = make_gemm(M, V, d, w.yf, 0, d, Wp(c, o.wte()), 0, d, ce_fused ? EPI_CE_FWD : EPI_STORE, w.logits, V);
+  if (ce_fused) {
+    g.epi.ce_max = w.ce_pm;
+    g.epi.ce_sum = w.ce_ps;
+    g.epi.ce_zt = w.ce_zt;
+    g.epi.ce_tgt = w.tgt;
+  }
   TRY(run_gemm(c, g, st));
   return GPT2_OK;
 }
@@ -451,9 +470,13 @@ int gpt2_forward_loss(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets
   Work& w = c->w;
   const int f32 = s.mode;
   CUDA_TRY(cudaMemcpyAsync(w.tgt, targets, (size_t)M * 4, cudaMemcpyDeviceToDevice, st));
-  TRY(forward_logits(c, tokens, batch, st));
+  TRY(forward_logits(c, tokens, batch, st, !f32));
   TRY(count_targets(w.tgt, M, (int)s.Vr, w.n_valid, w.err, st));
-  TRY(ce_fwd(f32, w.logits, w.tgt, w.loss_rows, M, V, (int)s.Vr, w.n_valid, w.err, st));
+  if (f32)
+    TRY(ce_fwd(f32, w.logits, w.tgt, w.loss_rows, M, V, (int)s.Vr, w.n_valid, w.err, st));
+  else
+    TRY(ce_merge(w.ce_pm, w.ce_ps, w.ce_zt, w.tgt, M, V, (int)s.Vr, w.n_valid, w.loss_rows, w.tgt_eff, w.ce_onehot,
+                 st));
   TRY(loss_mean(w.loss_rows, M, w.n_valid, loss_dev ? loss_dev : w.loss, w.err, st));
   c->have_fwd = 1;
   c->fwd_batch = batch;
@@ -479,14 +502,28 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
   const int fuse_d = (!f32 && s.hd == 64) ? 1 : 0;
   if (fuse_d) TRY(fill_zero(w.dq_acc, (size_t)M * d * sizeof(float), st));
 
-  // LM head (tied): dX_f = s * dz wte ; dwte (=/+=) s * dz^T X_f
+  // LM head (tied): dX_f = s * dz wte ; dwte (=/+=) s * dz^T X_f.  bf16: dz =
+  // softmax - onehot is formed in the operand staging of both products from
+  // the stored exponentials, the forward's per-part scales and the targets.
+  AScale as;
+  memset(&as, 0, sizeof(as));
+  if (!f32) {
+    as.r = w.ce_pm;
+    as.tgt = w.tgt_eff;
+    as.onehot = w.ce_onehot;
+    as.ld = M;
+    as.parts = V / 128;
+  }
   GemmArgs g = make_gemm(M, d, V, w.logits, 0, V, Wp(c, o.wte()), 1, d, EPI_STORE, w.dy, d);
   g.epi.alpha = sc;
+  g.ascale = as;
   TRY(run_gemm(c, g, st));
   g = make_gemm(V, d, M, w.logits, 1, V, w.yf, 1, d, EPI_F32, G + o.wte(), d);
   g.epi.alpha = sc;
   g.epi.beta = beta;
+  g.ascale = as;
   TRY(run_gemm(c, g, st));
+  g.ascale = AScale{};
   w.part_used = 0;
   w.jobs.clear();
   // the new residual gradient's column sums are the last MLP projection's b_mp gradient
@@ -545,7 +582,7 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
   TRY(reduce_rows_batch(w.jobs.data(), (int)w.jobs.size(), beta, st));
   // x_0 = wte[tok] + wpe[t]
   TRY(embed_bwd(f32, w.tok, w.dres, G + o.wte(), G + o.wpe(), w.emb_acc, w.touched, M, (int)s.T, d, V, accumulate,
-                st));
+                grad_scale, st));
   return GPT2_OK;
 }
 
@@ -837,6 +874,90 @@ int gpt2_op_colsum_bf16(const uint16_t* x, int M, int N, float* out, float* scra
   int nblk = 0;
   TRY(colsum_partial(0, x, M, N, scratch, &nblk, st));
   return reduce_rows_f32(scratch, nblk, N, out, 0.f, st);
+}
+
+// ---- the LM head with its fused softmax cross-entropy, alone --------------
+
+namespace {
+// Scratch of the LM-head cross-entropy ops: status word, n_valid, M / n_valid,
+// then the stored exponentials [M, V] (bf16), the per-part maxima (backward
+// scales) and sums [V/128][M], the target logits and effective targets [M].
+struct CeScratch {
+  int* err;
+  int* n_valid;
+  float* onehot;
+  void* e;
+  float *pm, *ps, *zt;
+  int32_t* tgt_eff;
+  size_t bytes;
+};
+CeScratch ce_scratch(void* base, int M, int V) {
+  Carver c{(uint8_t*)base};
+  CeScratch s;
+  s.err = c.take<int>(4);
+  s.n_valid = c.take<int>(4);
+  s.onehot = c.take<float>(4);
+  s.e = c.take<void>((size_t)M * V * 2);
+  s.pm = c.take<float>((size_t)(V / 128) * M * 4);
+  s.ps = c.take<float>((size_t)(V / 128) * M * 4);
+  s.zt = c.take<float>((size_t)M * 4);
+  s.tgt_eff = c.take<int32_t>((size_t)M * 4);
+  s.bytes = (c.off + 255) & ~(size_t)255;
+  return s;
+}
+}  // namespace
+
+size_t gpt2_op_lm_head_ce_scratch_bytes(int M, int V) {
+  if (M < 1 || V < 128 || V % 128) return 0;
+  return ce_scratch(nullptr, M, V).bytes;
+}
+
+int gpt2_op_lm_head_ce_fwd_bf16(const uint16_t* x, const uint16_t* w, const int32_t* targets, int M, int V, int d,
+                                int vocab_real, float* loss, float* loss_rows, void* scratch, size_t scratch_bytes,
+                                void* stream) {
+  if (!x || !w || !targets || !loss || !loss_rows || !scratch || M < 1 || d < 1) return GPT2_ERR_INVALID_ARG;
+  if (V < 128 || V % 128 || d % 64 || vocab_real < 1 || vocab_real > V) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (((uintptr_t)x | (uintptr_t)w | (uintptr_t)scratch) & 255) return GPT2_ERR_INVALID_ARG;
+  const CeScratch cs = ce_scratch(scratch, M, V);
+  if (scratch_bytes < cs.bytes) return GPT2_ERR_WORKSPACE;
+  const cudaStream_t st = S(stream);
+  CUDA_TRY(cudaMemsetAsync(cs.err, 0, sizeof(int), st));
+  GemmArgs g = make_gemm(M, V, d, x, 0, d, w, 0, d, EPI_CE_FWD, cs.e, V);
+  g.epi.ce_max = cs.pm;
+  g.epi.ce_sum = cs.ps;
+  g.epi.ce_zt = cs.zt;
+  g.epi.ce_tgt = targets;
+  TRY(gemm_tc_bf16(g, nullptr, 0, 0, 1, cs.err, st));
+  TRY(count_targets(targets, M, vocab_real, cs.n_valid, cs.err, st));
+  TRY(ce_merge(cs.pm, cs.ps, cs.zt, targets, M, V, vocab_real, cs.n_valid, loss_rows, cs.tgt_eff, cs.onehot, st));
+  return loss_mean(loss_rows, M, cs.n_valid, loss, cs.err, st);
+}
+
+int gpt2_op_lm_head_ce_bwd_bf16(const uint16_t* x, const uint16_t* w, int M, int V, int d, float grad_scale,
+                                uint16_t* dx, float* dw, int accumulate, void* scratch, size_t scratch_bytes,
+                                void* stream) {
+  if (!x || !w || !dx || !dw || !scratch || M < 1 || d < 1) return GPT2_ERR_INVALID_ARG;
+  if (V < 128 || V % 128 || d % 64) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (((uintptr_t)x | (uintptr_t)w | (uintptr_t)dx | (uintptr_t)dw | (uintptr_t)scratch) & 255)
+    return GPT2_ERR_INVALID_ARG;
+  const CeScratch cs = ce_scratch(scratch, M, V);
+  if (scratch_bytes < cs.bytes) return GPT2_ERR_WORKSPACE;
+  const cudaStream_t st = S(stream);
+  AScale as;
+  as.r = cs.pm;
+  as.tgt = cs.tgt_eff;
+  as.onehot = cs.onehot;
+  as.ld = M;
+  as.parts = V / 128;
+  GemmArgs g = make_gemm(M, d, V, cs.e, 0, V, w, 1, d, EPI_STORE, dx, d);
+  g.epi.alpha = grad_scale / (float)M;
+  g.ascale = as;
+  TRY(gemm_tc_bf16(g, nullptr, 0, 0, 1, cs.err, st));
+  g = make_gemm(V, d, M, cs.e, 1, V, x, 1, d, EPI_F32, dw, d);
+  g.epi.alpha = grad_scale / (float)M;
+  g.epi.beta = accumulate ? 1.f : 0.f;
+  g.ascale = as;
+  return gemm_tc_bf16(g, nullptr, 0, 0, 1, cs.err, st);
 }
 
 }  // extern "C"

@@ -17,6 +17,10 @@ enum EpiKind : int {
   EPI_F32_PARTIAL,  // partial[split][m,n] = acc (split-K, internal)
   EPI_ROWDOT,       // out(bf16) = acc; out2(fp32)[(m / seq * N/64 + n/64) * seq + m % seq] =
                     //   sum over the 64 columns of head n/64 of bf16(acc) * aux[m,n]
+  EPI_CE_FWD,       // LM head with the cross-entropy's online log-sum-exp: per row m and
+                    //   128-column part p (N % 128 == 0): ce_max[p*M+m] = max_n acc,
+                    //   out(bf16)[m,n] = exp(acc - ce_max), ce_sum[p*M+m] = sum of those
+                    //   (fp32), ce_zt[m] = acc[m, ce_tgt[m]] (fp32) when 0 <= ce_tgt[m] < N
 };
 
 struct EpiArgs {
@@ -29,6 +33,25 @@ struct EpiArgs {
   long ldo;
   float alpha, beta;
   int seq;            // EPI_ROWDOT: rows per sequence
+  // EPI_CE_FWD
+  float* ce_max;
+  float* ce_sum;
+  float* ce_zt;
+  const int32_t* ce_tgt;
+};
+
+// Softmax cross-entropy folded into the operand staging of the LM head's two
+// backward products (A = the stored exp(z - part max) in bf16): before the
+// MMA reads a k-block of A, each token row's run of 64 vocabulary entries is
+// multiplied by r[p*ld + t] (p = 128-column part of the vocabulary, t = token)
+// and the target column t's entry, if it lies in the run, is reduced by
+// *onehot.  K-major A: rows are tokens, k the vocabulary; MN-major A: rows
+// are the vocabulary, k the tokens.
+struct AScale {
+  const float* r;         // [parts][ld] fp32; NULL = no scaling
+  const int32_t* tgt;     // [ld] target id per token, -1 = none
+  const float* onehot;    // device scalar
+  int ld, parts;
 };
 
 // C[m,n] = sum_k A(m,k) B(n,k), then the epilogue.
@@ -39,6 +62,7 @@ struct GemmArgs {
   const void* A; int a_mn; long lda;
   const void* B; int b_mn; long ldb;
   EpiArgs epi;
+  AScale ascale;
 };
 
 // tcgen05 bf16 GEMM (sm_100a).  ws (may be NULL) holds split-K partials for
@@ -109,10 +133,15 @@ int count_targets(const int32_t* tgt, int M, int vocab_real, int* n_valid, int* 
 int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, int V,
            int vocab_real, const int* n_valid, int* err, cudaStream_t st);
 int loss_mean(const float* loss_rows, int M, const int* n_valid, float* loss, int* err, cudaStream_t st);
-// dwte[tok[m]] += dx[m] (deterministic fixed-point scatter), dwpe (=/+=) sum_b dx
+// Log-sum-exp, loss rows and backward scales from the LM head's EPI_CE_FWD
+// partials (part_max [V/128][M] becomes the scales r in place; see AScale).
+int ce_merge(float* part_max, const float* part_sum, const float* zt, const int32_t* tgt, int M, int V,
+             int vocab_real, const int* n_valid, float* loss_rows, int32_t* tgt_eff, float* onehot, cudaStream_t st);
+// dwte[tok[m]] += dx[m] (deterministic fixed-point scatter at a resolution of
+// 2^-32 |grad_scale|), dwpe (=/+=) sum_b dx
 int embed_bwd(int f32, const int32_t* tok, const void* dx, float* dwte, float* dwpe,
               long long* acc, uint8_t* touched, int M, int T, int d, int V, int wpe_accumulate,
-              cudaStream_t st);
+              float grad_scale, cudaStream_t st);
 // AdamW over the flat buffer with the decay mask derived from the layout.
 struct AdamArgs {
   float lr, beta1, beta2, eps, wd, bc1, bc2;

@@ -91,24 +91,27 @@ __global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const T* __res
 // converted back and added to dwte (and the accumulator is re-zeroed).
 #define FIX_SCALE 4294967296.0
 
+// The fixed point is relative to the backward's grad_scale (fix = 2^32 /
+// |grad_scale|): dx is proportional to grad_scale, so the resolution relative
+// to the gradient does not shrink under k-fold accumulation (grad_scale 1/k).
 template <typename T>
 __global__ void embed_scatter_kernel(const int32_t* __restrict__ tok, const T* __restrict__ dx,
                                      unsigned long long* __restrict__ acc, uint8_t* __restrict__ touched,
-                                     int M, int d, int V) {
+                                     int M, int d, int V, double fix) {
   pdl_start();
   long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
   if (i >= (long)M * d) return;
   const int m = (int)(i / d), c = (int)(i % d);
   int id = tok[m];
   if (id < 0 || id >= V) id = 0;
-  double v = (double)to_f(dx[i]) * FIX_SCALE;
+  double v = (double)to_f(dx[i]) * fix;
   v = fmin(fmax(v, -9.2e18), 9.2e18);
   atomicAdd(acc + (long)id * d + c, (unsigned long long)__double2ll_rn(v));
   if (c == 0) touched[id] = 1;
 }
 
 __global__ void embed_convert_kernel(unsigned long long* __restrict__ acc, uint8_t* __restrict__ touched,
-                                     float* __restrict__ dwte, int V, int d) {
+                                     float* __restrict__ dwte, int V, int d, double inv_fix) {
   pdl_start();
   const int v = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
@@ -117,7 +120,7 @@ __global__ void embed_convert_kernel(unsigned long long* __restrict__ acc, uint8
   float* g = dwte + (long)v * d;
   for (int c = lane; c < d; c += 32) {
     long long q = (long long)a[c];
-    g[c] += (float)((double)q / FIX_SCALE);
+    g[c] += (float)((double)q * inv_fix);
     a[c] = 0ull;
   }
   __syncwarp();
@@ -671,6 +674,65 @@ __global__ void loss_mean_kernel(const float* __restrict__ rows, int M, const in
   }
 }
 
+// Cross-entropy from the LM head's partials (the EPI_CE_FWD epilogue of the
+// tied LM-head GEMM): for row m, part p of 128 vocabulary columns, pm[p*M+m]
+// = max_v z and ps[p*M+m] = sum_v exp(z - pm); zt[m] = z[m, target].
+//   lse_m = max_p pm + log sum_p ps exp(pm - max)       (the row's log-sum-exp)
+//   loss_m = lse_m - zt[m] (0 where masked)
+//   r[p*M+m] = exp(pm - lse_m) * M / n_valid (0 where masked), in place of pm,
+// so softmax(z)[m, v] * M / n_valid = e[m, v] * r[part(v)*M + m] with e the
+// stored exp(z - pm); tgt_eff[m] = target or -1; *onehot = M / n_valid.
+// 32 rows per block; the eight warps take every eighth part and their
+// partial results meet in shared memory in a fixed order.
+__global__ void __launch_bounds__(256) ce_merge_kernel(float* __restrict__ pm, const float* __restrict__ ps,
+                                                       const float* __restrict__ zt, const int32_t* __restrict__ tgt,
+                                                       int M, int P, int vocab_real, const int* __restrict__ n_valid,
+                                                       float* __restrict__ loss_rows, int32_t* __restrict__ tgt_eff,
+                                                       float* __restrict__ onehot) {
+  pdl_start();
+  constexpr float L2E = 1.4426950408889634f;
+  __shared__ float red[8][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = blockIdx.x * 32 + lane;
+  const bool in = m < M;
+  float mx = -INFINITY;
+  if (in)
+    for (int p = warp; p < P; p += 8) mx = fmaxf(mx, pm[(long)p * M + m]);
+  red[warp][lane] = mx;
+  __syncthreads();
+  float gm = red[0][lane];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) gm = fmaxf(gm, red[w][lane]);
+  __syncthreads();
+  float sum = 0.f;
+  if (in)
+    for (int p = warp; p < P; p += 8) {
+      const long i = (long)p * M + m;
+      sum += ps[i] * ex2_approx((pm[i] - gm) * L2E);
+    }
+  red[warp][lane] = sum;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += red[w][lane];
+  const float lse = gm + logf(tot);
+  const int y = in ? tgt[m] : -1;
+  const bool valid = y >= 0 && y < vocab_real;
+  const int nv = *n_valid;
+  const float full = (float)M / (float)(nv > 0 ? nv : 1);
+  const float scale = valid ? full : 0.f;
+  if (in)
+    for (int p = warp; p < P; p += 8) {
+      const long i = (long)p * M + m;
+      pm[i] = ex2_approx((pm[i] - lse) * L2E) * scale;
+    }
+  if (warp == 0 && in) {
+    loss_rows[m] = valid ? lse - zt[m] : 0.f;
+    tgt_eff[m] = valid ? y : -1;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *onehot = full;
+}
+
 // ---------------------------------------------------------------- AdamW --
 
 // Which flat-layout elements are 2-D weights (wte, wpe, w_qkv, w_o, w_fc,
@@ -1035,6 +1097,15 @@ int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, i
   return GPT2_OK;
 }
 
+int ce_merge(float* part_max, const float* part_sum, const float* zt, const int32_t* tgt, int M, int V,
+             int vocab_real, const int* n_valid, float* loss_rows, int32_t* tgt_eff, float* onehot, cudaStream_t st) {
+  if (V % 128) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  CUDA_TRY(launch_k(ce_merge_kernel, (M + 31) / 32, 256, 0, st, part_max, part_sum, zt, tgt, M, V / 128, vocab_real,
+                    n_valid, loss_rows, tgt_eff, onehot));
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
 int loss_mean(const float* loss_rows, int M, const int* n_valid, float* loss, int* err, cudaStream_t st) {
   CUDA_TRY(launch_k(loss_mean_kernel, 1, 1024, 0, st, loss_rows, M, n_valid, loss, err));
   LAUNCH_CHECK();
@@ -1042,17 +1113,19 @@ int loss_mean(const float* loss_rows, int M, const int* n_valid, float* loss, in
 }
 
 int embed_bwd(int f32, const int32_t* tok, const void* dx, float* dwte, float* dwpe, long long* acc,
-              uint8_t* touched, int M, int T, int d, int V, int wpe_accumulate, cudaStream_t st) {
+              uint8_t* touched, int M, int T, int d, int V, int wpe_accumulate, float grad_scale, cudaStream_t st) {
   const long n = (long)M * d;
   unsigned long long* a = reinterpret_cast<unsigned long long*>(acc);
+  const double gs = fabs((double)grad_scale);
+  const double fix = FIX_SCALE / (gs > 0.0 && gs < 1e30 ? gs : 1.0);
   if (f32)
     CUDA_TRY(launch_k(embed_scatter_kernel<float>, (unsigned)((n + 255) / 256), 256, 0, st,
-        tok, (const float*)dx, a, touched, M, d, V));
+        tok, (const float*)dx, a, touched, M, d, V, fix));
   else
     CUDA_TRY(launch_k(embed_scatter_kernel<bf16>, (unsigned)((n + 255) / 256), 256, 0, st,
-        tok, (const bf16*)dx, a, touched, M, d, V));
+        tok, (const bf16*)dx, a, touched, M, d, V, fix));
   LAUNCH_CHECK();
-  CUDA_TRY(launch_k(embed_convert_kernel, (V + 7) / 8, 256, 0, st, a, touched, dwte, V, d));
+  CUDA_TRY(launch_k(embed_convert_kernel, (V + 7) / 8, 256, 0, st, a, touched, dwte, V, d, 1.0 / fix));
   LAUNCH_CHECK();
   const long tn = (long)T * d;
   const int B = M / T;

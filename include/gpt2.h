@@ -350,6 +350,31 @@ size_t gpt2_op_colsum_scratch_floats(int M, int N);
 int gpt2_op_colsum_bf16(const uint16_t* x, int M, int N, float* out, float* scratch, size_t scratch_floats,
                         void* stream);
 
+/* ---- the tied LM head with its fused softmax cross-entropy, alone --------
+ * "Pré-treinar um LLM", memory section: the logits are one vocabulary-sized
+ * vector per token; here they never reach HBM in fp32.  The forward GEMM
+ * z = x w^T computes, in its epilogue, each row's maximum and sum of exp(z -
+ * max) per 128-column part of the vocabulary, stores those exponentials
+ * (bf16, [M, V]) in the scratch, and keeps the target logits; a merge kernel
+ * forms each row's log-sum-exp, loss_rows[m] = LSE - z[m, target] (0 for
+ * target -1) and *loss = their mean over the rows with a target.  The
+ * backward forms dz = softmax(z) - onehot(target) from the stored
+ * exponentials inside the operand staging of its two GEMMs:
+ * dx = (grad_scale / n_valid) dz w (bf16 [M, d], written) and
+ * dw (=, or += with accumulate) (grad_scale / n_valid) dz^T x (fp32 [V, d]).
+ * x bf16 [M, d], w bf16 [V, d] (256-byte aligned), targets int32 [M] in
+ * [0, vocab_real) or -1; V a multiple of 128, d of 64.  The backward reads
+ * the scratch the forward wrote (same M, V, targets unchanged).  Device
+ * status: the int at scratch offset 0 (bit 1 = a target id out of range,
+ * counted as masked; bit 2 = non-finite loss), cleared by each forward. */
+size_t gpt2_op_lm_head_ce_scratch_bytes(int M, int V);
+int gpt2_op_lm_head_ce_fwd_bf16(const uint16_t* x, const uint16_t* w, const int32_t* targets, int M, int V, int d,
+                                int vocab_real, float* loss, float* loss_rows, void* scratch, size_t scratch_bytes,
+                                void* stream);
+int gpt2_op_lm_head_ce_bwd_bf16(const uint16_t* x, const uint16_t* w, int M, int V, int d, float grad_scale,
+                                uint16_t* dx, float* dw, int accumulate, void* scratch, size_t scratch_bytes,
+                                void* stream);
+
 #ifdef __cplusplus
 }
 #endif

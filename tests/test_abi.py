@@ -146,3 +146,21 @@ def test_noalloc_attention_backward_validates_shape_before_scratch_size():
     # a supported shape just past the 4 Mi-float array
     assert L.gpt2_op_attention_bwd_bf16_noalloc(p, p, p, p, p, 1, 4096, 16, 64, None) == \
         gp.ERRORS_BY_NAME["GPT2_ERR_TOO_LARGE"]
+
+
+def test_lm_head_cross_entropy_ops_validate_on_host():
+    # scratch sizing and shape rules of the fused LM-head cross-entropy ops,
+    # decided on the host before any CUDA call
+    L = gp._lib()
+    assert gp.gpt2_op_lm_head_ce_scratch_bytes(1024, 1000) == 0           # V not a multiple of 128
+    n = gp.gpt2_op_lm_head_ce_scratch_bytes(1024, 1024)
+    # status words, bf16 exponentials, two [V/128, M] fp32 part arrays, two [M] arrays
+    assert n >= 1024 * 1024 * 2 + 2 * 8 * 1024 * 4 + 2 * 1024 * 4
+    p = ctypes.c_void_p(4096)
+    uns = gp.ERRORS_BY_NAME["GPT2_ERR_UNSUPPORTED_SHAPE"]
+    assert L.gpt2_op_lm_head_ce_fwd_bf16(p, p, p, 64, 1000, 64, 1000, p, p, p, 1 << 30, None) == uns
+    assert L.gpt2_op_lm_head_ce_fwd_bf16(p, p, p, 64, 1024, 96, 1000, p, p, p, 1 << 30, None) == uns
+    assert L.gpt2_op_lm_head_ce_fwd_bf16(p, p, p, 64, 1024, 64, 1000, p, p, p, 16, None) == \
+        gp.ERRORS_BY_NAME["GPT2_ERR_WORKSPACE"]
+    assert L.gpt2_op_lm_head_ce_bwd_bf16(None, p, 64, 1024, 64, 1.0, p, p, 0, p, 1 << 30, None) == \
+        gp.ERRORS_BY_NAME["GPT2_ERR_INVALID_ARG"]

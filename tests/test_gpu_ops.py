@@ -254,3 +254,46 @@ def test_colsum_op_exact_sums(M, N):
     gp.gpt2_op_colsum_bf16(x.cuda(), M, N, out, scratch)
     X = x.double().numpy()
     assert np.abs(out.double().cpu().numpy() - X.sum(0)).max() <= 1e-5 * np.abs(X).sum(0).max()
+
+
+@pytest.mark.parametrize("M,V,d,vocab_real", [(960, 1408, 128, 1400), (1024, 50304, 768, 50257)])
+def test_lm_head_cross_entropy_ops_against_oracle(M, V, d, vocab_real):
+    """The tied LM head with the fused softmax cross-entropy, alone: the
+    forward's per-row losses and mean against the oracle's cross-entropy of
+    z = x w^T (fp64, same bf16 x and w), and the backward's dx and dw against
+    the chain rule of that loss, (softmax - onehot) / n_valid; every tenth
+    target masked (-1).  The rows are not a multiple of the 256-row tile and
+    the first vocabulary is not a multiple of the 256-column tile."""
+    g = torch.Generator().manual_seed(90 + M)
+    x = bf16_rand((M, d), 91 + M)
+    w = bf16_rand((V, d), 92 + V, scale=0.1)
+    tgt = torch.randint(0, vocab_real, (M,), generator=g, dtype=torch.int32)
+    tgt[::10] = -1
+    scratch = torch.empty(gp.gpt2_op_lm_head_ce_scratch_bytes(M, V), dtype=torch.uint8, device="cuda")
+    loss = torch.empty(1, device="cuda")
+    rows = torch.empty(M, device="cuda")
+    xd, wd, td = x.cuda(), w.cuda(), tgt.cuda()
+    gp.gpt2_op_lm_head_ce_fwd_bf16(xd, wd, td, M, V, d, vocab_real, loss, rows, scratch)
+    dx = torch.empty((M, d), dtype=torch.bfloat16, device="cuda")
+    dw = torch.full((V, d), float("nan"), device="cuda")
+    gp.gpt2_op_lm_head_ce_bwd_bf16(xd, wd, M, V, d, 0.5, dx, dw, 0, scratch)
+    torch.cuda.synchronize()
+    assert int(scratch[:4].view(torch.int32).item()) == 0
+    X, W, Y = x.double().numpy(), w.double().numpy(), tgt.numpy().astype(np.int64)
+    z = X @ W.T
+    ref_rows, _ = G.cross_entropy_fwd(z, Y)
+    valid = Y != G.IGNORE
+    n_valid = int(valid.sum())
+    ref_loss = ref_rows.sum() / n_valid
+    assert abs(loss.item() - ref_loss) <= 1e-4 * abs(ref_loss), (loss.item(), ref_loss)
+    assert np.abs(rows.double().cpu().numpy() - ref_rows).max() <= 1e-3 * np.abs(ref_rows).max()
+    p = np.exp(z - z.max(-1, keepdims=True))
+    p /= p.sum(-1, keepdims=True)
+    p[np.arange(M)[valid], Y[valid]] -= 1.0
+    dz = np.where(valid[:, None], p, 0.0) * (0.5 / n_valid)
+    for name, got, ref in (("dx", dx, dz @ W), ("dw", dw, dz.T @ X)):
+        a = got.double().cpu().numpy().ravel()
+        r = ref.ravel()
+        cos = float(a @ r / (np.linalg.norm(a) * np.linalg.norm(r)))
+        rel = float(np.abs(a - r).max() / np.abs(r).max())
+        assert cos >= 0.999 and rel <= 2e-2, (name, cos, rel)
