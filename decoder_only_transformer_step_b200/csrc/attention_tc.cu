@@ -597,14 +597,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ++nP[t];
           return true;
         };
+        // S of a tile's next key block needs only that the softmax has
+        // loaded the current S (P lives in other columns), so it is issued
+        // ahead of the current block's P V: the softmax finds the next S
+        // ready as soon as it has released the current P
         ok = issue_s(0, 0) && (!hasb || issue_s(1, 0));
         for (int j = 0; j < nkb && ok; ++j) {
-          if (j <= qa) {
-            if (!issue_pv(0, j) || (j + 1 <= qa && !issue_s(0, j + 1))) { ok = false; break; }
-          }
-          if (hasb) {
-            if (!issue_pv(1, j) || (j + 1 < nkb && !issue_s(1, j + 1))) { ok = false; break; }
-          }
+          if (j + 1 <= qa && !issue_s(0, j + 1)) { ok = false; break; }
+          if (hasb && j + 1 < nkb && !issue_s(1, j + 1)) { ok = false; break; }
+          if (j <= qa && !issue_pv(0, j)) { ok = false; break; }
+          if (hasb && !issue_pv(1, j)) { ok = false; break; }
           // every MMA reading this K/V slot has been issued
           tc_commit(kv_empty((g0 + j) % F2_KVS));
         }
@@ -635,8 +637,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int slot = k & 1;
       const int qt = qa + t;  // this tile's query block
       if (qt >= nqb) {
-        // tile 1 absent (an odd number of query blocks): nothing to compute
-        if (leader) mbar_arrive(q_empty(slot));
+        // tile 1 absent (an odd number of query blocks): nothing to compute.
+        // Its release of the Q slot must not run ahead into a later phase of
+        // the slot's barrier, so it waits until this item's Q has landed
+        // (which the producer issues only after the slot's previous phase).
+        if (leader) {
+          if (!mbar_wait_bounded(q_full(slot), (k >> 1) & 1, abort_flag, err)) ok = false;
+          mbar_arrive(q_empty(slot));
+        }
+        __syncwarp();
         continue;
       }
       const int grow = qt * BQ + row;
@@ -652,8 +661,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(tbar(t, 1));
         ++ns;
-        // raw scores; keys past the query masked on the diagonal block
-        float mx = -INFINITY;
+        // raw scores; keys past the query masked on the diagonal block.  The
+        // row maximum runs as eight independent chains (one dependent chain
+        // of 128 would cost its latency 128 times).
+        float mxs[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mxs[i] = -INFINITY;
         if (j == qt) {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
@@ -661,14 +674,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int i = 0; i < 32; ++i) {
               const float x = (32 * c + i > row) ? -INFINITY : __uint_as_float(v[c][i]);
               v[c][i] = __float_as_uint(x);
-              mx = fmaxf(mx, x);
+              mxs[i & 7] = fmaxf(mxs[i & 7], x);
             }
         } else {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(v[c][i]));
+            for (int i = 0; i < 32; ++i) mxs[i & 7] = fmaxf(mxs[i & 7], __uint_as_float(v[c][i]));
         }
+        const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
+                               fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
         const float m_new = fmaxf(m_use, mx * scale_log2);
         float alpha = 1.f;
         bool resc = false;
@@ -679,23 +694,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           m_use = m_new;
           resc = true;
         }
-        // P V of the previous block has finished reading P and writing O
-        if (np >= 1 && !mbar_wait_bounded(tbar(t, 3), (np - 1) & 1, abort_flag, err)) { ok = false; break; }
-        tc_fence_after();
-        float sum = 0.f;
+        // probabilities (bf16 pairs) in registers first; the previous P V
+        // is waited for only before they are stored over its P
+        float sums[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[4][16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float p0 = ex2(fmaf(__uint_as_float(v[c][2 * i]), scale_log2, -m_use));
             const float p1 = ex2(fmaf(__uint_as_float(v[c][2 * i + 1]), scale_log2, -m_use));
-            sum += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
+            sums[i & 3] += p0 + p1;
+            pk[c][i] = pack_bf16x2(p0, p1);
           }
-          tmem_st_32x32b_x16(tP + 16u * c, pk);
-        }
-        l = l * alpha + sum;
+        l = l * alpha + ((sums[0] + sums[1]) + (sums[2] + sums[3]));
+        // P V of the previous block has finished reading P and writing O
+        if (np >= 1 && !mbar_wait_bounded(tbar(t, 3), (np - 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st_32x32b_x16(tP + 16u * c, pk[c]);
         if (__any_sync(0xffffffffu, resc)) {
           // rare: this warp's rows whose maximum grew rescale their O
 #pragma unroll
@@ -1096,6 +1113,455 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
   }
 }
 
+// ------------------------------------------------ backward, persistent --
+// Persistent over work items (128-key block, batch, head), longest first, in
+// snake order over rounds.  Sixteen warps in four warpgroups with their own
+// register budgets (setmaxnreg):
+//   WG0  warp 0 TMA (K/V per item, double-buffered; Q/dO per query block),
+//        warp 1 TMEM allocation and MMA issue, warps 2-3 idle      (56 regs)
+//   WG1, WG2  elementwise: P^T = exp(S^T - LSE), dS^T = P^T (dP^T - D) for
+//        64 query columns each; P^T goes to tensor memory (the dV product
+//        reads it there), dS^T to a double-buffered shared tile        (176)
+//   WG3  LSE/D staging one query block ahead, the dQ drain (tensor memory
+//        -> shared -> TMA reduce-add into the fp32 dQ accumulator) and the
+//        dK/dV write-out at the end of an item                           (96)
+// The MMA warp issues S^T, dP^T of the next query block as soon as the
+// elementwise warps have loaded the current ones, ahead of the current
+// block's dV, dK, dQ products, so the elementwise work of one block overlaps
+// the tensor-core work of the other.  Tensor memory: S^T 0-127, dP^T
+// 128-255, P^T 256-319 (bf16 pairs), dV 320-383, dK 384-447, dQ 448-511.
+namespace bw {
+constexpr int QS = 2;  // Q/dO (and LSE/D) ring depth
+constexpr int SM_KV = 0;                       // [item slot 2][K, V] tiles
+constexpr int SM_QR = SM_KV + 4 * TILE;        // [QS] Q tiles
+constexpr int SM_DOR = SM_QR + QS * TILE;      // [QS] dO tiles
+constexpr int SM_DS = SM_DOR + QS * TILE;      // [2][2 halves] dS^T tiles
+constexpr int SM_DQ = SM_DS + 4 * TILE;        // [4 warps] 32 x 32 fp32 staging boxes
+constexpr int SM_LD = SM_DQ + 4 * 4096;        // [QS][LSE x128 | D x128] floats
+constexpr int SM_TILES = SM_LD + QS * 256 * 4;
+// kv_full[2], kv_empty[2], qdo_full[QS], qdo_empty[QS], ld_full[QS], ld_empty[QS],
+// st_full, st_free, ps_full, pt_free, ds_free[2], dq_full, dq_free, dkdv_full,
+// dkdv_free, epi_stage, drain
+constexpr int NUM_BARS = 4 + 4 * QS + 12;
+constexpr int SMEM = SM_TILES + 1024 + NUM_BARS * 8 + 16;
+static_assert(SMEM <= 232448, "backward shared memory");
+constexpr int THREADS = 512;
+constexpr uint32_t C_ST = 0, C_DPT = 128, C_PT = 256, C_DV = 320, C_DK = 384, C_DQ = 448;
+// Register budgets per warpgroup after setmaxnreg; with 128 per thread at
+// launch the block owns 512 x 128 = 65536 and the split below uses
+// 128 x 56 + 256 x 176 + 128 x 96 = 64512 of them.
+constexpr int LAUNCH_REGS = 128, REGS_CTRL = 56, REGS_ELEM = 176, REGS_DRAIN = 96;
+static_assert(128 * REGS_CTRL + 256 * REGS_ELEM + 128 * REGS_DRAIN <= THREADS * LAUNCH_REGS, "register split");
+}  // namespace bw
+
+template <int N> DEVI void reg_dealloc() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N> DEVI void reg_alloc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
+__global__ void __launch_bounds__(bw::THREADS, 1)
+    attn_bwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
+                        const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDQKV,
+                        const float* __restrict__ lse, const float* __restrict__ dvec, int T, int H, int n_items,
+                        float scale, float scale_log2, int* err) {
+  // (local names shadow the one-CTA-per-block backward's constants above)
+  constexpr int QS = bw::QS, SM_KV = bw::SM_KV, SM_QR = bw::SM_QR, SM_DOR = bw::SM_DOR, SM_DS = bw::SM_DS;
+  constexpr int SM_DQ = bw::SM_DQ, SM_LD = bw::SM_LD, SM_TILES = bw::SM_TILES, NUM_BARS = bw::NUM_BARS;
+  constexpr uint32_t C_ST = bw::C_ST, C_DPT = bw::C_DPT, C_PT = bw::C_PT, C_DV = bw::C_DV, C_DK = bw::C_DK,
+                     C_DQ = bw::C_DQ;
+  constexpr int REGS_CTRL = bw::REGS_CTRL, REGS_ELEM = bw::REGS_ELEM, REGS_DRAIN = bw::REGS_DRAIN;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  float* sLD = reinterpret_cast<float*>(base_ptr + SM_LD);
+  const uint32_t bars = base + SM_TILES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + SM_TILES + NUM_BARS * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto kv_full = [&](int s) { return bars + 8u * s; };
+  auto kv_empty = [&](int s) { return bars + 8u * (2 + s); };
+  auto qdo_full = [&](int r) { return bars + 8u * (4 + r); };
+  auto qdo_empty = [&](int r) { return bars + 8u * (4 + QS + r); };
+  auto ld_full = [&](int r) { return bars + 8u * (4 + 2 * QS + r); };
+  auto ld_empty = [&](int r) { return bars + 8u * (4 + 3 * QS + r); };
+  const uint32_t b0 = bars + 8u * (4 + 4 * QS);
+  const uint32_t st_full = b0, st_free = b0 + 8, ps_full = b0 + 16, pt_free = b0 + 24;
+  auto ds_free = [&](int i) { return b0 + 32u + 8u * i; };
+  const uint32_t dq_full = b0 + 48, dq_free = b0 + 56, dkdv_full = b0 + 64, dkdv_free = b0 + 72;
+  const uint32_t epi_stage = b0 + 80, drain_bar = b0 + 88;
+  auto kv_tile = [&](int slot) { return base + SM_KV + (uint32_t)(2 * slot) * TILE; };  // K; V follows
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = (T + BQ - 1) / BQ;
+  const int BH = n_items / nqb;
+  const int d = H * HD;
+  // item w -> (key block, batch, head): low key blocks (most query blocks) first
+  auto item = [&](int w, int& kb, int& b, int& h) {
+    kb = w / BH;
+    const int bh = w % BH;
+    b = bh / H;
+    h = bh % H;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 2);  // the item's last MMAs and the dK/dV store
+      mbar_init(ds_free(s), 1);
+    }
+    for (int r = 0; r < QS; ++r) {
+      mbar_init(qdo_full(r), 1);
+      mbar_init(qdo_empty(r), 1);
+      mbar_init(ld_full(r), 4);
+      mbar_init(ld_empty(r), 8);
+    }
+    mbar_init(st_full, 1);
+    mbar_init(st_free, 8);
+    mbar_init(ps_full, 8);
+    mbar_init(pt_free, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 4);
+    mbar_init(dkdv_full, 1);
+    mbar_init(dkdv_free, 4);
+    mbar_init(epi_stage, 4);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&tmQKV);
+    tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmDQ);
+    tma_prefetch_desc(&tmDQKV);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_start();
+  const int wg = warp >> 2;
+
+  if (wg == 0) {
+    reg_dealloc<REGS_CTRL>();
+    if (warp == 0 && lane == 0) {
+      // ----------------------------------------------------------- TMA ----
+      bool ok = true;
+      int it = 0, gq = 0, kv_issued = 0, q_issued = 0;
+      for (int k = 0; ok; ++k, ++it) {
+        const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
+        if (w >= n_items) break;
+        int kb, b, h;
+        item(w, kb, b, h);
+        const int nblk = nqb - kb, slot = it & 1;
+        if (it >= 2 && !mbar_wait_bounded(kv_empty(slot), ((it - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        mbar_arrive_expect_tx(kv_full(slot), 2 * TILE);
+        tma_load_3d(kv_tile(slot), &tmQKV, kv_full(slot), d + h * HD, kb * BKV, b);
+        tma_load_3d(kv_tile(slot) + TILE, &tmQKV, kv_full(slot), 2 * d + h * HD, kb * BKV, b);
+        ++kv_issued;
+        for (int t = 0; t < nblk; ++t) {
+          const int g = gq + t, r = g % QS;
+          if (g >= QS && !mbar_wait_bounded(qdo_empty(r), ((g - QS) / QS) & 1, abort_flag, err)) { ok = false; break; }
+          const int q0 = (kb + t) * BQ;
+          mbar_arrive_expect_tx(qdo_full(r), 2 * TILE);
+          tma_load_3d(base + SM_QR + r * TILE, &tmQKV, qdo_full(r), h * HD, q0, b);
+          tma_load_3d(base + SM_DOR + r * TILE, &tmDO, qdo_full(r), h * HD, q0, b);
+          ++q_issued;
+        }
+        gq += nblk;
+      }
+      if (!ok) {
+        for (int i = kv_issued - 2 < 0 ? 0 : kv_issued - 2; i < kv_issued; ++i)
+          mbar_drain_bounded(kv_full(i & 1), (i >> 1) & 1);
+        for (int i = q_issued - QS < 0 ? 0 : q_issued - QS; i < q_issued; ++i)
+          mbar_drain_bounded(qdo_full(i % QS), (i / QS) & 1);
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ----------------------------------------------------------- MMA ----
+      bool ok = true, issued_any = false;
+      int it = 0, gq = 0;
+      for (int k = 0; ok; ++k, ++it) {
+        const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
+        if (w >= n_items) break;
+        int kb, b, h;
+        item(w, kb, b, h);
+        const int nblk = nqb - kb, slot = it & 1;
+        if (!mbar_wait_bounded(kv_full(slot), (it >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        const uint32_t kt = kv_tile(slot), vt = kt + TILE;
+        // S^T = K Q^T and dP^T = V dO^T of global query block g
+        auto issue_sdp = [&](int g) -> bool {
+          const int r = g % QS;
+          if (!mbar_wait_bounded(qdo_full(r), (g / QS) & 1, abort_flag, err)) return false;
+          if (g >= 1 && !mbar_wait_bounded(st_free, (g - 1) & 1, abort_flag, err)) return false;
+          tc_fence_after();
+          const uint32_t qt = base + SM_QR + r * TILE, ot = base + SM_DOR + r * TILE;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk)
+            tc_mma_bf16(tmem + C_ST, sdesc(kt + kk * 32, 16, 1024), sdesc(qt + kk * 32, 16, 1024), IDESC_S,
+                        kk > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk)
+            tc_mma_bf16(tmem + C_DPT, sdesc(vt + kk * 32, 16, 1024), sdesc(ot + kk * 32, 16, 1024), IDESC_S,
+                        kk > 0 ? 1u : 0u);
+          tc_commit(st_full);
+          issued_any = true;
+          return true;
+        };
+        if (!issue_sdp(gq)) { ok = false; break; }
+        for (int t = 0; t < nblk; ++t) {
+          const int g = gq + t, r = g % QS;
+          if (t + 1 < nblk && !issue_sdp(g + 1)) { ok = false; break; }
+          if (!mbar_wait_bounded(ps_full, g & 1, abort_flag, err)) { ok = false; break; }
+          // the previous item's dK / dV have been read out of tensor memory
+          if (t == 0 && it >= 1 && !mbar_wait_bounded(dkdv_free, (it - 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t qt = base + SM_QR + r * TILE, ot = base + SM_DOR + r * TILE;
+          const uint32_t ds = base + SM_DS + (uint32_t)(g & 1) * 2 * TILE;
+          // dV += P^T dO (P^T from tensor memory)
+#pragma unroll
+          for (int kk = 0; kk < BQ / 16; ++kk)
+            tc_mma_bf16_ts(tmem + C_DV, tmem + C_PT + 8u * kk, sdesc(ot + kk * 2048, 8192, 1024), IDESC_O,
+                           (t > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(pt_free);
+          // dK += dS^T Q
+#pragma unroll
+          for (int kk = 0; kk < BQ / 16; ++kk)
+            tc_mma_bf16(tmem + C_DK, sdesc(ds + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024),
+                        sdesc(qt + kk * 2048, 8192, 1024), IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
+          // dQ = dS K into the single dQ buffer, once its previous block is drained
+          if (g >= 1 && !mbar_wait_bounded(dq_free, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BKV / 16; ++kk)
+            tc_mma_bf16(tmem + C_DQ, sdesc(ds + kk * 2048, TILE, 1024), sdesc(kt + kk * 2048, 8192, 1024), IDESC_DQ,
+                        kk > 0 ? 1u : 0u);
+          tc_commit(dq_full);
+          tc_commit(ds_free(g & 1));
+          tc_commit(qdo_empty(r));
+        }
+        if (!ok) break;
+        tc_commit(dkdv_full);
+        tc_commit(kv_empty(slot));
+        gq += nblk;
+      }
+      if (!ok && issued_any) {
+        tc_commit(drain_bar);
+        mbar_drain_bounded(drain_bar, 0);
+      }
+    }
+  } else if (wg <= 2) {
+    reg_alloc<REGS_ELEM>();
+    // --------------------------------------------------------- elementwise ----
+    const int q = warp & 3;          // TMEM lanes [32q, 32q+32): key rows
+    const int half = wg - 1;         // query columns [64 half, 64 half + 64)
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    bool ok = true;
+    int gq = 0;
+    for (int k = 0; ok; ++k) {
+      const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
+      if (w >= n_items) break;
+      int kb, b, h;
+      item(w, kb, b, h);
+      const int nblk = nqb - kb;
+      const int kv = kb * BKV + row;
+      for (int t = 0; t < nblk; ++t) {
+        const int g = gq + t, r = g % QS;
+        const int q0 = (kb + t) * BQ;
+        if (!mbar_wait_bounded(ld_full(r), (g / QS) & 1, abort_flag, err)) { ok = false; break; }
+        if (!mbar_wait_bounded(st_full, g & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sv[2][32], dp[2][32];
+        tmem_ld_32x32b_x32(tmem + lane_off + C_ST + 64 * half, sv[0]);
+        tmem_ld_32x32b_x32(tmem + lane_off + C_ST + 64 * half + 32, sv[1]);
+        tmem_ld_32x32b_x32(tmem + lane_off + C_DPT + 64 * half, dp[0]);
+        tmem_ld_32x32b_x32(tmem + lane_off + C_DPT + 64 * half + 32, dp[1]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(st_free);
+        // masking only on the diagonal block, past T, or for keys past T
+        const bool need_mask = (t == 0) || (q0 + BQ > T) || (kv >= T);
+        const float* ld = sLD + r * 256;
+        uint32_t pp[32], pd[32];
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+          const int c0 = 64 * half + 32 * sub;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            // broadcast reads: every lane needs the same four columns
+            const float4 l4 = *reinterpret_cast<const float4*>(ld + c0 + i);
+            const float4 d4 = *reinterpret_cast<const float4*>(ld + 128 + c0 + i);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pv[4], dv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              float p = ex2(fmaf(__uint_as_float(sv[sub][i + u]), scale_log2, -lv[u]));
+              if (need_mask) {
+                const int qq = q0 + c0 + i + u;
+                if (qq < kv || qq >= T || kv >= T) p = 0.f;
+              }
+              pv[u] = p;
+              dv[u] = p * (__uint_as_float(dp[sub][i + u]) - dd[u]);
+            }
+            pp[sub * 16 + i / 2] = pack_bf16x2(pv[0], pv[1]);
+            pp[sub * 16 + i / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+            pd[sub * 16 + i / 2] = pack_bf16x2(dv[0], dv[1]);
+            pd[sub * 16 + i / 2 + 1] = pack_bf16x2(dv[2], dv[3]);
+          }
+        }
+        // every lane has read this block's LSE / D
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ld_empty(r));
+        // dV of the previous block has read P^T; dK, dQ of block g-2 have
+        // read this dS^T buffer
+        if (g >= 1 && !mbar_wait_bounded(pt_free, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (g >= 2 && !mbar_wait_bounded(ds_free(g & 1), ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st_32x32b_x32(tmem + lane_off + C_PT + 32 * half, pp);
+        const uint32_t drow = base + SM_DS + (uint32_t)(g & 1) * 2 * TILE + half * TILE + (uint32_t)row * 128u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(drow + 16u * (uint32_t)(c ^ (row & 7)), pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ps_full);
+      }
+      gq += nblk;
+    }
+  } else {
+    reg_dealloc<REGS_DRAIN>();
+    // ---------------------------------------- LSE/D staging, dQ, dK / dV ----
+    const int q = warp & 3;  // TMEM lanes [32q, 32q+32): query rows of dQ, key rows of dK / dV
+    const int tid = threadIdx.x - 384;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t box = base + SM_DQ + (uint32_t)q * 4096u;
+    bool ok = true;
+    // LSE (log2 domain) and D of query block t of item (kb, b, h) into ring
+    // slot r (queries past T: LSE = +inf, D = 0)
+    auto stage_ld = [&](int g, int kb, int b, int h, int t) -> bool {
+      const int r = g % QS;
+      if (g >= QS && !mbar_wait_bounded(ld_empty(r), ((g - QS) / QS) & 1, abort_flag, err)) return false;
+      const int qq = (kb + t) * BQ + tid;
+      const long bh0 = ((long)b * H + h) * T;
+      sLD[r * 256 + tid] = qq < T ? lse[bh0 + qq] * LOG2E_F : INFINITY;
+      sLD[r * 256 + 128 + tid] = qq < T ? dvec[bh0 + qq] : 0.f;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ld_full(r));
+      return true;
+    };
+    int gq = 0, it = 0;
+    {
+      const int w = snake_item(0, (int)blockIdx.x, (int)gridDim.x);
+      if (w < n_items) {
+        int kb, b, h;
+        item(w, kb, b, h);
+        ok = stage_ld(0, kb, b, h, 0);
+      }
+    }
+    for (int k = 0; ok; ++k, ++it) {
+      const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
+      if (w >= n_items) break;
+      int kb, b, h;
+      item(w, kb, b, h);
+      const int nblk = nqb - kb, slot = it & 1;
+      const int wn = snake_item(k + 1, (int)blockIdx.x, (int)gridDim.x);
+      for (int t = 0; t < nblk; ++t) {
+        const int g = gq + t;
+        // the next query block's LSE / D (of this item, or the next item's first)
+        if (t + 1 < nblk) {
+          if (!stage_ld(g + 1, kb, b, h, t + 1)) { ok = false; break; }
+        } else if (wn < n_items) {
+          int kb2, b2, h2;
+          item(wn, kb2, b2, h2);
+          if (!stage_ld(g + 1, kb2, b2, h2, 0)) { ok = false; break; }
+        }
+        // dQ of block g: tensor memory -> registers (the buffer is then free
+        // for the next block's dQ) -> two 32 x 32 fp32 boxes -> TMA reduce-add
+        if (!mbar_wait_bounded(dq_full, g & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t dq[2][32];
+        tmem_ld_32x32b_x32(tmem + lane_off + C_DQ, dq[0]);
+        tmem_ld_32x32b_x32(tmem + lane_off + C_DQ + 32, dq[1]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_free);
+        const int q0 = (kb + t) * BQ;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          // this warp's box was last read by the previous reduce
+          if (lane == 0) bulk_wait_read<0>();
+          __syncwarp();
+          const uint32_t rb = box + (uint32_t)lane * 128u;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(rb + 16u * (uint32_t)(j ^ (lane & 7)), __float_as_uint(__uint_as_float(dq[c][4 * j]) * scale),
+                         __float_as_uint(__uint_as_float(dq[c][4 * j + 1]) * scale),
+                         __float_as_uint(__uint_as_float(dq[c][4 * j + 2]) * scale),
+                         __float_as_uint(__uint_as_float(dq[c][4 * j + 3]) * scale));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            // rows past T are clipped by the tensor map
+            tma_reduce_add_3d(&tmDQ, box, h * HD + 32 * c, q0 + q * 32, b);
+            bulk_commit();
+          }
+        }
+      }
+      if (!ok) break;
+      // ---- dK (scaled) and dV of the item, bf16, through its K / V tiles
+      if (!mbar_wait_bounded(dkdv_full, it & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after();
+      const int row = q * 32 + lane;
+      const uint32_t kt = kv_tile(slot), vt = kt + TILE;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        uint32_t o[2][32];
+        tmem_ld_32x32b_x32(tmem + lane_off + (which ? C_DV : C_DK), o[0]);
+        tmem_ld_32x32b_x32(tmem + lane_off + (which ? C_DV : C_DK) + 32, o[1]);
+        tmem_ld_wait();
+        if (which == 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dkdv_free);
+        }
+        const float sc = which ? 1.f : scale;
+        const uint32_t orow = (which ? vt : kt) + (uint32_t)row * 128u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t* oc = &o[c >> 2][(c & 3) * 8];
+          st_shared_v4(orow + 16u * (uint32_t)(c ^ (row & 7)),
+                       pack_bf16x2(__uint_as_float(oc[0]) * sc, __uint_as_float(oc[1]) * sc),
+                       pack_bf16x2(__uint_as_float(oc[2]) * sc, __uint_as_float(oc[3]) * sc),
+                       pack_bf16x2(__uint_as_float(oc[4]) * sc, __uint_as_float(oc[5]) * sc),
+                       pack_bf16x2(__uint_as_float(oc[6]) * sc, __uint_as_float(oc[7]) * sc));
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_stage);
+      if (!mbar_wait_bounded(epi_stage, it & 1, abort_flag, err)) { ok = false; break; }
+      if (warp == 12 && lane == 0) {
+        // rows past T are clipped by the tensor map
+        tma_store_3d(&tmDQKV, kt, d + h * HD, kb * BKV, b);
+        tma_store_3d(&tmDQKV, vt, 2 * d + h * HD, kb * BKV, b);
+        bulk_commit();
+        bulk_wait_read<0>();
+        mbar_arrive(kv_empty(slot));
+      }
+      __syncwarp();
+      gq += nblk;
+    }
+    if (lane == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 }  // namespace
 
 int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float* dvec, void* dqkv, float* dq_acc,
@@ -1113,6 +1579,27 @@ int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float
   if (!tmap_3d(&tq, qkv, dq, sq) || !tmap_3d(&tdo, dout, dd, sd) ||
       !tmap_3d(&tdq, dq_acc, dd, sdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 32) || !tmap_3d(&tdqkv, dqkv, dq, sq))
     return GPT2_ERR_CUDA;
+  // The persistent kernel, if its launch register count is the one its
+  // register split is computed for (otherwise a setmaxnreg.inc could wait for
+  // registers the block does not own): checked once on the host.
+  static int v2 = -1;
+  if (v2 < 0) {
+    const char* e = getenv("GPT2_ATTN_BWD_TC");
+    cudaFuncAttributes fa;
+    v2 = (e && e[0] == '1') ? 0
+         : (cudaFuncGetAttributes(&fa, attn_bwd_tc2_kernel) == cudaSuccess && fa.numRegs == bw::LAUNCH_REGS) ? 1
+                                                                                                             : 0;
+    cudaGetLastError();
+    if (v2) CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bw::SMEM));
+  }
+  if (v2) {
+    const int n_items = ((T + BKV - 1) / BKV) * B * H;
+    const int grid = n_items < num_sms() ? n_items : num_sms();
+    CUDA_TRY(launch_k(attn_bwd_tc2_kernel, grid, bw::THREADS, bw::SMEM, st, tq, tdo, tdq, tdqkv, lse, dvec, T, H,
+                      n_items, 0.125f, LOG2E_F / 8.f, nullptr));
+    LAUNCH_CHECK();
+    return GPT2_OK;
+  }
   static bool attr = false;
   if (!attr) {
     CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B_SMEM_BYTES));

@@ -57,12 +57,11 @@ struct TcCfg {
   // a deeper operand ring.
   static constexpr int EPI_WARP_BYTES = BIG_EPI ? 8192 : 4096;
   static constexpr int EPI_BYTES = NUM_EPI_WARPS * EPI_WARP_BYTES;
-  // full, empty, acc_full[2], acc_empty[2], drain, operand[8 warps][2], and
-  // for the A-scaling stage a_full, a_ready per ring slot
+  // full, empty, acc_full[2], acc_empty[2], drain, operand[8 warps][2]
   static constexpr int NUM_FIXED_BARS = 5 + 2 * NUM_EPI_WARPS;
   static constexpr int STAGES_FIT = (232448 - EPI_BYTES - 1024 - 512) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-  static constexpr int NUM_BARS = 4 * STAGES + NUM_FIXED_BARS;
+  static constexpr int NUM_BARS = 2 * STAGES + NUM_FIXED_BARS;
   static_assert(NUM_BARS * 8 + 16 <= 512, "barrier region");
   // accumulator-empty arrivals: one per epilogue warp of every CTA of the unit
   static constexpr uint32_t ACCE_COUNT = (PAIR ? 2 : 1) * NUM_EPI_WARPS;
@@ -89,7 +88,6 @@ struct TcParams {
   uint32_t idesc;
   int store;
   EpiArgs epi;
-  AScale as;
   float* partial;
   int* err;
 };
@@ -113,56 +111,6 @@ DEVI uint64_t operand_desc(uint32_t tile, int mn_major, int k) {
   return mn_major ? sdesc(tile + k * 2048, MN_ATOM_BYTES, 1024) : sdesc(tile + k * 32, 16, 1024);
 }
 
-// Softmax cross-entropy in the operand staging (AScale): one k-block of A,
-// 128 rows of 128 bytes (64 bf16) in the 128-byte swizzle, is rewritten in
-// place by the eight epilogue warps, 16 rows each, two lanes per row.  Every
-// 128-byte row is one token's run of 64 consecutive vocabulary entries (K-major
-// A: row = token, k = vocabulary; MN-major A: the {64 vocabulary x 64 token}
-// boxes hold one token per row), so a row takes one scale r (its token and
-// 128-column part); the swizzle only permutes 16-byte chunks within the row,
-// which matters only for locating the target column.
-struct AsRow {
-  float r;
-  int y;
-};
-DEVI AsRow ascale_row(const AScale& as, int a_mn, int ma, int kb, int R) {
-  int t, part;
-  if (!a_mn) {
-    t = ma + R;          // token row of the tile
-    part = kb >> 1;      // 64-wide k-block inside a 128-wide part
-  } else {
-    t = kb * 64 + (R & 63);
-    part = ma >> 7;      // ma is a multiple of 128
-  }
-  AsRow o{0.f, -1};
-  if (t < as.ld && part < as.parts) {
-    o.r = __ldg(as.r + (long)part * as.ld + t);
-    o.y = __ldg(as.tgt + t);
-  }
-  return o;
-}
-DEVI void ascale_apply(uint32_t sa, int a_mn, int ma, int kb, int R, int h, AsRow a, float onehot) {
-  const int vbase = !a_mn ? kb * 64 : ma + 64 * (R >> 6);
-  const uint32_t rowa = sa + (uint32_t)R * 128u;
-  const int x = R & 7;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int pc = 4 * h + i;     // physical 16-byte chunk of the row
-    const int v0 = vbase + 8 * (pc ^ x);
-    uint32_t u0, u1, u2, u3;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(u0), "=r"(u1), "=r"(u2), "=r"(u3)
-                 : "r"(rowa + 16u * (uint32_t)pc));
-    float f[8] = {bf16lo(u0), bf16hi(u0), bf16lo(u1), bf16hi(u1),
-                  bf16lo(u2), bf16hi(u2), bf16lo(u3), bf16hi(u3)};
-    const int dy = a.y - v0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) f[j] = f[j] * a.r - (dy == j ? onehot : 0.f);
-    st_shared_v4(rowa + 16u * (uint32_t)pc, pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                 pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-  }
-}
-
 // Work unit u -> (m tile origin, n tile index, split index, k-block range).
 // m varies fastest, so consecutive CTAs share the B tile (weights) in L2.
 DEVI void decode_unit(const TcParams& p, int u, int& m0, int& nt, int& s, int& kb0, int& kb1) {
@@ -175,18 +123,17 @@ DEVI void decode_unit(const TcParams& p, int u, int& m0, int& nt, int& s, int& k
   kb1 = (int)((long long)(s + 1) * p.kb_total / p.splits);
 }
 
-enum : int { MODE_PLAIN = 0, MODE_ASCALE = 1, MODE_CE = 2 };
+enum : int { MODE_PLAIN = 0, MODE_CE = 1 };
 
-// MODE: MODE_PLAIN, MODE_ASCALE (the A operand is rewritten in shared memory
-// before the MMAs read it) or MODE_CE (the EPI_CE_FWD epilogue); separate
-// instantiations keep the extra state out of the other variants' registers.
+// MODE: MODE_PLAIN or MODE_CE (the EPI_CE_FWD epilogue); a separate
+// instantiation keeps the cross-entropy state out of the other variants'
+// registers.
 template <int BN, bool PAIR, bool BIG_EPI, int MODE = MODE_PLAIN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
                    const TcParams p) {
   using C = TcCfg<BN, PAIR, BIG_EPI>;
-  constexpr bool ASCALE = MODE == MODE_ASCALE;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t tiles = (raw + 1023u) & ~1023u;
@@ -204,10 +151,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t drain_bar = bars + 8u * (2 * C::STAGES + 4);
   // operand-load barrier of epilogue warp e, buffer b
   auto op_bar = [&](int e, int b) { return bars + 8u * (2 * C::STAGES + 5 + 2 * e + b); };
-  // A-scaling stage: this CTA's A tile landed (local), and every CTA's A
-  // tile of the slot scaled (on the CTA that issues the MMAs)
-  auto afull_bar = [&](int s) { return bars + 8u * (C::NUM_FIXED_BARS + 2 * C::STAGES + s); };
-  auto aready_bar = [&](int s) { return bars + 8u * (C::NUM_FIXED_BARS + 3 * C::STAGES + s); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -229,10 +172,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int e = 0; e < NUM_EPI_WARPS; ++e) {
       mbar_init(op_bar(e, 0), 1);
       mbar_init(op_bar(e, 1), 1);
-    }
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(afull_bar(s), 1);
-      mbar_init(aready_bar(s), C::ACCE_COUNT);  // one arrival per epilogue warp of the unit
     }
     *abort_flag = 0;
     mbar_fence_init();
@@ -275,29 +214,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           const uint32_t sa = tiles + stage * C::STAGE_BYTES;
           const uint32_t sb = sa + C::A_BYTES;
-          if constexpr (ASCALE) {
-            // A lands on this CTA's own barrier (the epilogue warps rewrite it
-            // before the MMA may read it); B as below, counted alone
-            mbar_arrive_expect_tx(afull_bar(stage), C::A_BYTES);
-            if (!p.a_mn) {
-              tma_load_2d(sa, &tmA, afull_bar(stage), kb * BK, ma);
-            } else {
-              tma_load_2d(sa, &tmA, afull_bar(stage), ma, kb * BK);
-              tma_load_2d(sa + MN_ATOM_BYTES, &tmA, afull_bar(stage), ma + 64, kb * BK);
-            }
-            const uint32_t fb = PAIR ? mapa_shared(full_bar(stage), 0) : full_bar(stage);
-            if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), (PAIR ? 2 : 1) * C::B_BYTES);
-            if (!p.b_mn) {
-              if constexpr (PAIR) tma_load_2d_pair(sb, &tmB, fb, kb * BK, nb);
-              else tma_load_2d(sb, &tmB, fb, kb * BK, nb);
-            } else {
-#pragma unroll
-              for (int j = 0; j < C::B_ROWS / 64; ++j) {
-                if constexpr (PAIR) tma_load_2d_pair(sb + j * MN_ATOM_BYTES, &tmB, fb, nb + 64 * j, kb * BK);
-                else tma_load_2d(sb + j * MN_ATOM_BYTES, &tmB, fb, nb + 64 * j, kb * BK);
-              }
-            }
-          } else if constexpr (PAIR) {
+          if constexpr (PAIR) {
             // both CTAs' bytes are counted on the even CTA's full barrier
             const uint32_t fb = mapa_shared(full_bar(stage), 0);
             if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
@@ -340,14 +257,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok) {
         // Let the copies already in flight land before the CTA exits (for a
-        // pair, the even CTA's full barriers count both CTAs' copies of B, and
-        // of A unless A lands on each CTA's own barrier).
+        // pair, the even CTA's full barriers count both CTAs' copies).
         int n = issued < C::STAGES ? issued : C::STAGES;
         for (int i = 1; i <= n; ++i) {
           int s2 = (stage - i + C::STAGES) % C::STAGES;
           uint32_t par = s2 < stage ? phase : (phase ^ 1u);
           if (rank == 0) mbar_drain_bounded(full_bar(s2), par);
-          if (ASCALE) mbar_drain_bounded(afull_bar(s2), par);
         }
       }
     }
@@ -376,14 +291,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.err)) {
             ok = false;
             break;
-          }
-          if constexpr (ASCALE) {
-            const bool ready = PAIR ? mbar_wait_bounded_cluster(aready_bar(stage), phase, abort_flag, p.err)
-                                    : mbar_wait_bounded(aready_bar(stage), phase, abort_flag, p.err);
-            if (!ready) {
-              ok = false;
-              break;
-            }
           }
           tc_fence_after();
           const uint32_t sa = tiles + stage * C::STAGE_BYTES;
@@ -455,50 +362,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     };
     bool ok = true;
     int it = 0;
-    // A-scaling stage: ring position of the next k-block (mirrors the producer)
-    int ts = 0;
-    uint32_t tph = 0;
-    const float onehot = ASCALE ? *p.as.onehot : 0.f;
     constexpr bool ce = MODE == MODE_CE;
     for (int u = unit0; u < units && ok; u += unit_step, ++it) {
       int m0, nt, s, kb0, kb1;
       decode_unit(p, u, m0, nt, s, kb0, kb1);
-      if constexpr (ASCALE) {
-        // rewrite this unit's k-blocks of A as they land, ahead of the MMAs;
-        // each row's scale and target are fetched four k-blocks ahead
-        const int ma = m0 + (int)rank * BM;
-        const int R = e * 16 + (lane >> 1), hh = lane & 1;
-        const AsRow none{0.f, -1};
-        AsRow q0 = ascale_row(p.as, p.a_mn, ma, kb0, R);
-        AsRow q1 = kb0 + 1 < kb1 ? ascale_row(p.as, p.a_mn, ma, kb0 + 1, R) : none;
-        AsRow q2 = kb0 + 2 < kb1 ? ascale_row(p.as, p.a_mn, ma, kb0 + 2, R) : none;
-        AsRow q3 = kb0 + 3 < kb1 ? ascale_row(p.as, p.a_mn, ma, kb0 + 3, R) : none;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          const AsRow q4 = kb + 4 < kb1 ? ascale_row(p.as, p.a_mn, ma, kb + 4, R) : none;
-          if (!mbar_wait_bounded(afull_bar(ts), tph, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
-          ascale_apply(tiles + ts * C::STAGE_BYTES, p.a_mn, ma, kb, R, hh, q0, onehot);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if constexpr (PAIR)
-              mbar_arrive_cluster(mapa_shared(aready_bar(ts), 0));
-            else
-              mbar_arrive(aready_bar(ts));
-          }
-          q0 = q1;
-          q1 = q2;
-          q2 = q3;
-          q3 = q4;
-          if (++ts == C::STAGES) {
-            ts = 0;
-            tph ^= 1u;
-          }
-        }
-        if (!ok) break;
-      }
       const int n0 = nt * BN;
       const int buf = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
@@ -878,11 +745,6 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   if (((uintptr_t)g.A | (uintptr_t)g.B | (uintptr_t)g.epi.out) & 15) return GPT2_ERR_INVALID_ARG;
   bn = resolve_bn(bn, g.N);
   if (bn != 128 && bn != 256 && bn != 512) return GPT2_ERR_INVALID_ARG;
-  const bool ascale = g.ascale.r != nullptr;
-  if (ascale) {
-    if (!g.ascale.tgt || !g.ascale.onehot || g.ascale.ld < 1 || g.ascale.parts < 1) return GPT2_ERR_INVALID_ARG;
-    if (g.epi.kind != EPI_STORE && g.epi.kind != EPI_F32) return GPT2_ERR_INVALID_ARG;
-  }
   if (g.epi.kind == EPI_CE_FWD) {
     // 128-column parts: each epilogue warp owns 128 columns of a 256-wide tile
     if (g.N % 128 || !g.epi.ce_max || !g.epi.ce_sum || !g.epi.ce_zt || !g.epi.ce_tgt) return GPT2_ERR_INVALID_ARG;
@@ -920,7 +782,6 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   p.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)g.a_mn << 15) | ((uint32_t)g.b_mn << 16) |
             ((uint32_t)(n_mma >> 3) << 17) | ((uint32_t)(p.tile_m >> 4) << 24);
   p.epi = g.epi;
-  p.as = g.ascale;
   p.partial = (float*)ws;
   p.err = err;
   if (splits > 1) p.epi.kind = EPI_F32_PARTIAL;
@@ -984,15 +845,7 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   const bool big = p.store == ST_BF16_X2 || p.epi.kind == EPI_BIAS_RESID || p.epi.kind == EPI_DGELU ||
                    p.epi.kind == EPI_ROWDOT;
   int rc;
-  if (ascale) {
-    if (big || p.store == ST_REG) return GPT2_ERR_INVALID_ARG;
-    if (pair)
-      rc = launch_tc<256, true, false, MODE_ASCALE>(ta, tb, tc, tc2, p, units, st);
-    else if (bn == 256)
-      rc = launch_tc<256, false, false, MODE_ASCALE>(ta, tb, tc, tc2, p, units, st);
-    else
-      rc = launch_tc<128, false, false, MODE_ASCALE>(ta, tb, tc, tc2, p, units, st);
-  } else if (p.epi.kind == EPI_CE_FWD) {
+  if (p.epi.kind == EPI_CE_FWD) {
     rc = pair ? launch_tc<256, true, false, MODE_CE>(ta, tb, tc, tc2, p, units, st)
               : launch_tc<256, false, false, MODE_CE>(ta, tb, tc, tc2, p, units, st);
   } else if (pair)

@@ -104,10 +104,8 @@ struct Work {
   std::vector<LayerActs> layers;
   void *x_final, *yf, *logits;
   float *meanf, *rstdf, *loss_rows;
-  // fused cross-entropy (bf16): per-part maxima (then the backward scales)
-  // and sums [V/128][M], target logits, effective targets, M / n_valid
-  float *ce_pm, *ce_ps, *ce_zt, *ce_onehot;
-  int32_t* tgt_eff;
+  // fused cross-entropy (bf16): per-part maxima and sums [V/128][M], target logits
+  float *ce_pm, *ce_ps, *ce_zt;
   void *dres, *dy, *du, *dqkv, *dout;
   float *dq_acc, *dvec;
   float *norm_part, *gnorm;  // global gradient norm: block partials and the result
@@ -176,8 +174,6 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
   w->ce_pm = c.take<float>((size_t)parts * M * 4);
   w->ce_ps = c.take<float>((size_t)parts * M * 4);
   w->ce_zt = c.take<float>(M * 4);
-  w->tgt_eff = c.take<int32_t>(M * 4);
-  w->ce_onehot = c.take<float>(4);
   w->dres = c.take<void>(M * d * act);
   w->dy = c.take<void>(M * d * act);
   w->du = c.take<void>(M * 4 * d * act);
@@ -475,8 +471,7 @@ int gpt2_forward_loss(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets
   if (f32)
     TRY(ce_fwd(f32, w.logits, w.tgt, w.loss_rows, M, V, (int)s.Vr, w.n_valid, w.err, st));
   else
-    TRY(ce_merge(w.ce_pm, w.ce_ps, w.ce_zt, w.tgt, M, V, (int)s.Vr, w.n_valid, w.loss_rows, w.tgt_eff, w.ce_onehot,
-                 st));
+    TRY(ce_merge_dz(w.ce_pm, w.ce_ps, w.ce_zt, w.tgt, w.logits, M, V, (int)s.Vr, w.n_valid, w.loss_rows, st));
   TRY(loss_mean(w.loss_rows, M, w.n_valid, loss_dev ? loss_dev : w.loss, w.err, st));
   c->have_fwd = 1;
   c->fwd_batch = batch;
@@ -502,28 +497,15 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
   const int fuse_d = (!f32 && s.hd == 64) ? 1 : 0;
   if (fuse_d) TRY(fill_zero(w.dq_acc, (size_t)M * d * sizeof(float), st));
 
-  // LM head (tied): dX_f = s * dz wte ; dwte (=/+=) s * dz^T X_f.  bf16: dz =
-  // softmax - onehot is formed in the operand staging of both products from
-  // the stored exponentials, the forward's per-part scales and the targets.
-  AScale as;
-  memset(&as, 0, sizeof(as));
-  if (!f32) {
-    as.r = w.ce_pm;
-    as.tgt = w.tgt_eff;
-    as.onehot = w.ce_onehot;
-    as.ld = M;
-    as.parts = V / 128;
-  }
+  // LM head (tied): dX_f = s * dz wte ; dwte (=/+=) s * dz^T X_f, with dz =
+  // (softmax - onehot) M / n_valid left in w.logits by the forward
   GemmArgs g = make_gemm(M, d, V, w.logits, 0, V, Wp(c, o.wte()), 1, d, EPI_STORE, w.dy, d);
   g.epi.alpha = sc;
-  g.ascale = as;
   TRY(run_gemm(c, g, st));
   g = make_gemm(V, d, M, w.logits, 1, V, w.yf, 1, d, EPI_F32, G + o.wte(), d);
   g.epi.alpha = sc;
   g.epi.beta = beta;
-  g.ascale = as;
   TRY(run_gemm(c, g, st));
-  g.ascale = AScale{};
   w.part_used = 0;
   w.jobs.clear();
   // the new residual gradient's column sums are the last MLP projection's b_mp gradient
@@ -879,16 +861,14 @@ int gpt2_op_colsum_bf16(const uint16_t* x, int M, int N, float* out, float* scra
 // ---- the LM head with its fused softmax cross-entropy, alone --------------
 
 namespace {
-// Scratch of the LM-head cross-entropy ops: status word, n_valid, M / n_valid,
-// then the stored exponentials [M, V] (bf16), the per-part maxima (backward
-// scales) and sums [V/128][M], the target logits and effective targets [M].
+// Scratch of the LM-head cross-entropy ops: status word, n_valid, then the
+// bf16 [M, V] buffer (the forward's exponentials, rewritten as dz), the
+// per-part maxima and sums [V/128][M] and the target logits [M].
 struct CeScratch {
   int* err;
   int* n_valid;
-  float* onehot;
   void* e;
   float *pm, *ps, *zt;
-  int32_t* tgt_eff;
   size_t bytes;
 };
 CeScratch ce_scratch(void* base, int M, int V) {
@@ -896,12 +876,10 @@ CeScratch ce_scratch(void* base, int M, int V) {
   CeScratch s;
   s.err = c.take<int>(4);
   s.n_valid = c.take<int>(4);
-  s.onehot = c.take<float>(4);
   s.e = c.take<void>((size_t)M * V * 2);
   s.pm = c.take<float>((size_t)(V / 128) * M * 4);
   s.ps = c.take<float>((size_t)(V / 128) * M * 4);
   s.zt = c.take<float>((size_t)M * 4);
-  s.tgt_eff = c.take<int32_t>((size_t)M * 4);
   s.bytes = (c.off + 255) & ~(size_t)255;
   return s;
 }
@@ -929,7 +907,7 @@ int gpt2_op_lm_head_ce_fwd_bf16(const uint16_t* x, const uint16_t* w, const int3
   g.epi.ce_tgt = targets;
   TRY(gemm_tc_bf16(g, nullptr, 0, 0, 1, cs.err, st));
   TRY(count_targets(targets, M, vocab_real, cs.n_valid, cs.err, st));
-  TRY(ce_merge(cs.pm, cs.ps, cs.zt, targets, M, V, vocab_real, cs.n_valid, loss_rows, cs.tgt_eff, cs.onehot, st));
+  TRY(ce_merge_dz(cs.pm, cs.ps, cs.zt, targets, cs.e, M, V, vocab_real, cs.n_valid, loss_rows, st));
   return loss_mean(loss_rows, M, cs.n_valid, loss, cs.err, st);
 }
 
@@ -943,20 +921,12 @@ int gpt2_op_lm_head_ce_bwd_bf16(const uint16_t* x, const uint16_t* w, int M, int
   const CeScratch cs = ce_scratch(scratch, M, V);
   if (scratch_bytes < cs.bytes) return GPT2_ERR_WORKSPACE;
   const cudaStream_t st = S(stream);
-  AScale as;
-  as.r = cs.pm;
-  as.tgt = cs.tgt_eff;
-  as.onehot = cs.onehot;
-  as.ld = M;
-  as.parts = V / 128;
   GemmArgs g = make_gemm(M, d, V, cs.e, 0, V, w, 1, d, EPI_STORE, dx, d);
   g.epi.alpha = grad_scale / (float)M;
-  g.ascale = as;
   TRY(gemm_tc_bf16(g, nullptr, 0, 0, 1, cs.err, st));
   g = make_gemm(V, d, M, cs.e, 1, V, x, 1, d, EPI_F32, dw, d);
   g.epi.alpha = grad_scale / (float)M;
   g.epi.beta = accumulate ? 1.f : 0.f;
-  g.ascale = as;
   return gemm_tc_bf16(g, nullptr, 0, 0, 1, cs.err, st);
 }
 

@@ -40,29 +40,11 @@ struct EpiArgs {
   const int32_t* ce_tgt;
 };
 
-// Softmax cross-entropy folded into the operand staging of the LM head's two
-// backward products (A = the stored exp(z - part max) in bf16): before the
-// MMA reads a k-block of A, each token row's run of 64 vocabulary entries is
-// multiplied by r[p*ld + t] (p = 128-column part of the vocabulary, t = token)
-// and the target column t's entry, if it lies in the run, is reduced by
-// *onehot.  K-major A: rows are tokens, k the vocabulary; MN-major A: rows
-// are the vocabulary, k the tokens.
-struct AScale {
-  const float* r;         // [parts][ld] fp32; NULL = no scaling
-  const int32_t* tgt;     // [ld] target id per token, -1 = none
-  const float* onehot;    // device scalar
-  int ld, parts;
-};
-
-// C[m,n] = sum_k A(m,k) B(n,k), then the epilogue.
-// a_mn = 0: A(m,k) = A[m*lda + k]; a_mn = 1: A(m,k) = A[k*lda + m].
-// b_mn = 0: B(n,k) = B[n*ldb + k]; b_mn = 1: B(n,k) = B[k*ldb + n].
 struct GemmArgs {
   int M, N, K;
   const void* A; int a_mn; long lda;
   const void* B; int b_mn; long ldb;
   EpiArgs epi;
-  AScale ascale;
 };
 
 // tcgen05 bf16 GEMM (sm_100a).  ws (may be NULL) holds split-K partials for
@@ -133,10 +115,13 @@ int count_targets(const int32_t* tgt, int M, int vocab_real, int* n_valid, int* 
 int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, int V,
            int vocab_real, const int* n_valid, int* err, cudaStream_t st);
 int loss_mean(const float* loss_rows, int M, const int* n_valid, float* loss, int* err, cudaStream_t st);
-// Log-sum-exp, loss rows and backward scales from the LM head's EPI_CE_FWD
-// partials (part_max [V/128][M] becomes the scales r in place; see AScale).
-int ce_merge(float* part_max, const float* part_sum, const float* zt, const int32_t* tgt, int M, int V,
-             int vocab_real, const int* n_valid, float* loss_rows, int32_t* tgt_eff, float* onehot, cudaStream_t st);
+// The cross-entropy from the LM head's EPI_CE_FWD outputs: per row the
+// log-sum-exp from the per-part maxima / sums [V/128][M], the loss row
+// (LSE - z[target], 0 where masked), and, in place over the stored bf16
+// exp(z - part max) [M, V], dz = (softmax - onehot(target)) * M / n_valid
+// (zero rows where masked), the operand of the two backward GEMMs.
+int ce_merge_dz(const float* part_max, const float* part_sum, const float* zt, const int32_t* tgt, void* e, int M,
+                int V, int vocab_real, const int* n_valid, float* loss_rows, cudaStream_t st);
 // dwte[tok[m]] += dx[m] (deterministic fixed-point scatter at a resolution of
 // 2^-32 |grad_scale|), dwpe (=/+=) sum_b dx
 int embed_bwd(int f32, const int32_t* tok, const void* dx, float* dwte, float* dwpe,

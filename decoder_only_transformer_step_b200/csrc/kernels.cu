@@ -675,25 +675,33 @@ __global__ void loss_mean_kernel(const float* __restrict__ rows, int M, const in
 }
 
 // Cross-entropy from the LM head's partials (the EPI_CE_FWD epilogue of the
-// tied LM-head GEMM): for row m, part p of 128 vocabulary columns, pm[p*M+m]
-// = max_v z and ps[p*M+m] = sum_v exp(z - pm); zt[m] = z[m, target].
+// tied LM-head GEMM): for row m and part p of 128 vocabulary columns,
+// pm[p*M+m] = max_v z and ps[p*M+m] = sum_v exp(z - pm); zt[m] = z[m, target];
+// e[m, v] = bf16 exp(z - pm) for v in part p.  Per row:
 //   lse_m = max_p pm + log sum_p ps exp(pm - max)       (the row's log-sum-exp)
 //   loss_m = lse_m - zt[m] (0 where masked)
-//   r[p*M+m] = exp(pm - lse_m) * M / n_valid (0 where masked), in place of pm,
-// so softmax(z)[m, v] * M / n_valid = e[m, v] * r[part(v)*M + m] with e the
-// stored exp(z - pm); tgt_eff[m] = target or -1; *onehot = M / n_valid.
-// 32 rows per block; the eight warps take every eighth part and their
-// partial results meet in shared memory in a fixed order.
-__global__ void __launch_bounds__(256) ce_merge_kernel(float* __restrict__ pm, const float* __restrict__ ps,
-                                                       const float* __restrict__ zt, const int32_t* __restrict__ tgt,
-                                                       int M, int P, int vocab_real, const int* __restrict__ n_valid,
-                                                       float* __restrict__ loss_rows, int32_t* __restrict__ tgt_eff,
-                                                       float* __restrict__ onehot) {
+//   e[m, v] <- e[m, v] exp(pm - lse_m) M / n_valid - [v == target] M / n_valid,
+// i.e. dz = (softmax - onehot) scaled so the backward GEMMs' alpha =
+// grad_scale / M gives the mean over the positions with a target.  32 rows per
+// block: the eight warps take every eighth part for the log-sum-exp (partials
+// meet in shared memory in a fixed order), then every thread rewrites 16-byte
+// pieces of the block's rows with the row's part scales from shared memory.
+constexpr int CEM_ROWS = 32;
+__global__ void __launch_bounds__(256) ce_merge_dz_kernel(const float* __restrict__ pm, const float* __restrict__ ps,
+                                                          const float* __restrict__ zt,
+                                                          const int32_t* __restrict__ tgt, bf16* __restrict__ e,
+                                                          int M, int V, int vocab_real,
+                                                          const int* __restrict__ n_valid,
+                                                          float* __restrict__ loss_rows) {
   pdl_start();
   constexpr float L2E = 1.4426950408889634f;
-  __shared__ float red[8][32];
+  extern __shared__ float sc[];          // [CEM_ROWS][P] scales
+  __shared__ float red[8][CEM_ROWS];
+  __shared__ int ytgt[CEM_ROWS];
+  const int P = V / 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m = blockIdx.x * 32 + lane;
+  const int m0 = blockIdx.x * CEM_ROWS;
+  const int m = m0 + lane;
   const bool in = m < M;
   float mx = -INFINITY;
   if (in)
@@ -722,15 +730,31 @@ __global__ void __launch_bounds__(256) ce_merge_kernel(float* __restrict__ pm, c
   const float full = (float)M / (float)(nv > 0 ? nv : 1);
   const float scale = valid ? full : 0.f;
   if (in)
-    for (int p = warp; p < P; p += 8) {
-      const long i = (long)p * M + m;
-      pm[i] = ex2_approx((pm[i] - lse) * L2E) * scale;
-    }
-  if (warp == 0 && in) {
-    loss_rows[m] = valid ? lse - zt[m] : 0.f;
-    tgt_eff[m] = valid ? y : -1;
+    for (int p = warp; p < P; p += 8) sc[lane * P + p] = ex2_approx((pm[(long)p * M + m] - lse) * L2E) * scale;
+  if (warp == 0) {
+    if (in) loss_rows[m] = valid ? lse - zt[m] : 0.f;
+    ytgt[lane] = valid ? y : -1;
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) *onehot = full;
+  __syncthreads();
+  // the rewrite: 8 bf16 (16 bytes) per step, a row's V / 8 pieces in order
+  const int nrows = min(CEM_ROWS, M - m0);
+  const int per_row = V / 8;
+  for (int i = threadIdx.x; i < nrows * per_row; i += blockDim.x) {
+    const int r = i / per_row, c = (i % per_row) * 8;
+    uint4* ptr = reinterpret_cast<uint4*>(e + (long)(m0 + r) * V + c);
+    uint4 u = *ptr;
+    const float s = sc[r * P + (c >> 7)];
+    const int dy = ytgt[r] - c;
+    float f[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
+                  bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = f[j] * s - (dy == j ? full : 0.f);
+    u.x = pack_bf16x2(f[0], f[1]);
+    u.y = pack_bf16x2(f[2], f[3]);
+    u.z = pack_bf16x2(f[4], f[5]);
+    u.w = pack_bf16x2(f[6], f[7]);
+    *ptr = u;
+  }
 }
 
 // ---------------------------------------------------------------- AdamW --
@@ -1097,11 +1121,17 @@ int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, i
   return GPT2_OK;
 }
 
-int ce_merge(float* part_max, const float* part_sum, const float* zt, const int32_t* tgt, int M, int V,
-             int vocab_real, const int* n_valid, float* loss_rows, int32_t* tgt_eff, float* onehot, cudaStream_t st) {
-  if (V % 128) return GPT2_ERR_UNSUPPORTED_SHAPE;
-  CUDA_TRY(launch_k(ce_merge_kernel, (M + 31) / 32, 256, 0, st, part_max, part_sum, zt, tgt, M, V / 128, vocab_real,
-                    n_valid, loss_rows, tgt_eff, onehot));
+int ce_merge_dz(const float* part_max, const float* part_sum, const float* zt, const int32_t* tgt, void* e, int M,
+                int V, int vocab_real, const int* n_valid, float* loss_rows, cudaStream_t st) {
+  if (V % 128 || V > 65536) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  const size_t smem = (size_t)CEM_ROWS * (V / 128) * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    CUDA_TRY(cudaFuncSetAttribute(ce_merge_dz_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536));
+    attr = true;
+  }
+  CUDA_TRY(launch_k(ce_merge_dz_kernel, (M + CEM_ROWS - 1) / CEM_ROWS, 256, smem, st, part_max, part_sum, zt, tgt,
+                    (bf16*)e, M, V, vocab_real, n_valid, loss_rows));
   LAUNCH_CHECK();
   return GPT2_OK;
 }

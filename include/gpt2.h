@@ -357,9 +357,9 @@ int gpt2_op_colsum_bf16(const uint16_t* x, int M, int N, float* out, float* scra
  * max) per 128-column part of the vocabulary, stores those exponentials
  * (bf16, [M, V]) in the scratch, and keeps the target logits; a merge kernel
  * forms each row's log-sum-exp, loss_rows[m] = LSE - z[m, target] (0 for
- * target -1) and *loss = their mean over the rows with a target.  The
- * backward forms dz = softmax(z) - onehot(target) from the stored
- * exponentials inside the operand staging of its two GEMMs:
+ * target -1) and *loss = their mean over the rows with a target, and
+ * rewrites the stored exponentials in place as dz = softmax(z) -
+ * onehot(target) (bf16).  The backward's two GEMMs read that dz:
  * dx = (grad_scale / n_valid) dz w (bf16 [M, d], written) and
  * dw (=, or += with accumulate) (grad_scale / n_valid) dz^T x (fp32 [V, d]).
  * x bf16 [M, d], w bf16 [V, d] (256-byte aligned), targets int32 [M] in
