@@ -56,6 +56,7 @@ EXPORTS = [
     "gpt2_op_layernorm_fwd_bf16", "gpt2_op_layernorm_bwd_scratch_floats", "gpt2_op_layernorm_bwd_bf16",
     "gpt2_op_colsum_scratch_floats", "gpt2_op_colsum_bf16",
     "gpt2_op_lm_head_ce_scratch_bytes", "gpt2_op_lm_head_ce_fwd_bf16", "gpt2_op_lm_head_ce_bwd_bf16",
+    "gpt2_set_wait_timeout_ns", "gpt2_op_gemm_bf16_status",
 ]
 
 _LIB = None
@@ -107,6 +108,8 @@ def _lib():
         "gpt2_op_lm_head_ce_scratch_bytes": (S, [I, I]),
         "gpt2_op_lm_head_ce_fwd_bf16": (I, [P, P, P, I, I, I, I, P, P, P, S, P]),
         "gpt2_op_lm_head_ce_bwd_bf16": (I, [P, P, I, I, I, F, P, P, I, P, S, P]),
+        "gpt2_set_wait_timeout_ns": (I, [U64]),
+        "gpt2_op_gemm_bf16_status": (I, [P, I, I, P, I, I, P, I, I, I, I, I, F, F, P, S, I, I, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -325,6 +328,18 @@ def gpt2_op_lm_head_ce_bwd_bf16(x, w, M, V, d, grad_scale, dx, dw, accumulate, s
     _check(_lib().gpt2_op_lm_head_ce_bwd_bf16(_ptr(x), _ptr(w), M, V, d, grad_scale, _ptr(dx), _ptr(dw), accumulate,
                                               _ptr(scratch), scratch.numel() * scratch.element_size(),
                                               _stream(stream)), "gpt2_op_lm_head_ce_bwd_bf16")
+
+
+def gpt2_set_wait_timeout_ns(ns: int):
+    _check(_lib().gpt2_set_wait_timeout_ns(ns), "gpt2_set_wait_timeout_ns")
+
+
+def gpt2_op_gemm_bf16_status(A, a_mn, lda, B, b_mn, ldb, C, c_fp32, ldc, M, N, K, alpha=1.0, beta=0.0,
+                             workspace=None, bn=0, splits=0, status=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib().gpt2_op_gemm_bf16_status(_ptr(A), a_mn, lda, _ptr(B), b_mn, ldb, _ptr(C), c_fp32, ldc, M, N, K,
+                                           alpha, beta, _ptr(workspace), ws_bytes, bn, splits, _ptr(status),
+                                           _stream(stream)), "gpt2_op_gemm_bf16_status")
 
 
 # ------------------------------------------------------------ convenience ---

@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // and the tensor-core work of both.
 //   warp 0      TMA: both tiles' Q (two item slots), K/V ring
 //   warp 1      TMEM allocation, MMA issue
-//   warps 2..5  softmax + output of tile 0, warps 6..9 of tile 1
+//   warps 4..7  softmax + output of tile 0, warps 8..11 of tile 1
 constexpr int F2_KVS = 4;
 constexpr int F2_Q = 0;                          // [slot 2][tile 2] Q / O staging
 constexpr int F2_K = F2_Q + 4 * TILE;
@@ -441,8 +441,18 @@ constexpr int F2_NUM_BARS = 4 + 2 * F2_KVS + 12 + 1;
 constexpr int F2_SMEM = F2_TILES + 1024 + F2_NUM_BARS * 8 + 16;
 static_assert(F2_SMEM <= 232448, "forward shared memory");
 constexpr float F2_RESCALE = 8.f;  // log2 of the largest un-rescaled probability
+// Twelve warps in three warpgroups: WG0 = TMA (warp 0), MMA (warp 1), two idle
+// warps; WG1 / WG2 = the softmax of query tile 0 / 1.  Register budgets after
+// setmaxnreg: with 168 per thread at launch the block owns 384 x 168 = 64512,
+// split as 128 x 80 + 256 x 208 = 63488.
+constexpr int F2_THREADS = 384;
+constexpr int F2_LAUNCH_REGS = 168, F2_REGS_CTRL = 80, F2_REGS_SOFT = 208;
+static_assert(128 * F2_REGS_CTRL + 256 * F2_REGS_SOFT <= F2_THREADS * F2_LAUNCH_REGS, "register split");
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <int N> DEVI void reg_dealloc() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N> DEVI void reg_alloc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
+__global__ void __launch_bounds__(F2_THREADS, 1)
     attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmO,
                         float* __restrict__ lse, int T, int H, int n_items, float scale_log2, int* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -504,7 +514,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   pdl_start();
 
-  if (warp == 0) {
+  if (warp < 4) {
+   reg_dealloc<F2_REGS_CTRL>();
+   if (warp == 0) {
     if (lane == 0) {
       // ----------------------------------------------------------- TMA ----
       bool ok = true;
@@ -619,14 +631,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_drain_bounded(drain_bar, 0);
       }
     }
+   }
   } else {
+    reg_alloc<F2_REGS_SOFT>();
     // ------------------------------------------------- softmax, output ----
-    const int t = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int t = (warp - 4) >> 2;  // query tile of this warpgroup
     const int q = warp & 3;         // TMEM lanes [32q, 32q+32)
     const int row = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t tS = tmem + lane_off + 256u * t, tO = tS + 128u, tP = tS + 192u;
-    const bool leader = (warp & 3) == 2 && lane == 0;  // first warp of the warpgroup
+    const bool leader = (warp & 3) == 0 && lane == 0;  // first warp of the warpgroup
     bool ok = true;
     int ns = 0, np = 0, nit = 0;
     for (int k = 0; ok; ++k) {
@@ -696,18 +710,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         // probabilities (bf16 pairs) in registers first; the previous P V
         // is waited for only before they are stored over its P
-        float sums[4] = {0.f, 0.f, 0.f, 0.f};
+        // two columns per packed fp32x2 multiply-add and add
+        float2 sums[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_use, -m_use);
         uint32_t pk[4][16];
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(__uint_as_float(v[c][2 * i]), scale_log2, -m_use));
-            const float p1 = ex2(fmaf(__uint_as_float(v[c][2 * i + 1]), scale_log2, -m_use));
-            sums[i & 3] += p0 + p1;
-            pk[c][i] = pack_bf16x2(p0, p1);
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[c][2 * i]), __uint_as_float(v[c][2 * i + 1])),
+                                        sc2, nm2);
+            const float2 pr = make_float2(ex2(x.x), ex2(x.y));
+            sums[i & 1] = __fadd2_rn(sums[i & 1], pr);
+            pk[c][i] = pack_bf16x2(pr.x, pr.y);
           }
-        l = l * alpha + ((sums[0] + sums[1]) + (sums[2] + sums[3]));
+        l = l * alpha + ((sums[0].x + sums[0].y) + (sums[1].x + sums[1].y));
         // P V of the previous block has finished reading P and writing O
         if (np >= 1 && !mbar_wait_bounded(tbar(t, 3), (np - 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
@@ -1118,30 +1135,30 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
 // snake order over rounds.  Sixteen warps in four warpgroups with their own
 // register budgets (setmaxnreg):
 //   WG0  warp 0 TMA (K/V per item, double-buffered; Q/dO per query block),
-//        warp 1 TMEM allocation and MMA issue, warps 2-3 idle      (56 regs)
+//        warp 1 TMEM allocation and MMA issue, warps 2-3 idle      (80 regs)
 //   WG1, WG2  elementwise: P^T = exp(S^T - LSE), dS^T = P^T (dP^T - D) for
 //        64 query columns each; P^T goes to tensor memory (the dV product
-//        reads it there), dS^T to a double-buffered shared tile        (176)
+//        reads it there), dS^T to a shared tile                          (160)
 //   WG3  LSE/D staging one query block ahead, the dQ drain (tensor memory
 //        -> shared -> TMA reduce-add into the fp32 dQ accumulator) and the
-//        dK/dV write-out at the end of an item                           (96)
+//        dK/dV write-out at the end of an item                          (112)
 // The MMA warp issues S^T, dP^T of the next query block as soon as the
 // elementwise warps have loaded the current ones, ahead of the current
 // block's dV, dK, dQ products, so the elementwise work of one block overlaps
 // the tensor-core work of the other.  Tensor memory: S^T 0-127, dP^T
 // 128-255, P^T 256-319 (bf16 pairs), dV 320-383, dK 384-447, dQ 448-511.
 namespace bw {
-constexpr int QS = 2;  // Q/dO (and LSE/D) ring depth
+constexpr int QS = 3;  // Q/dO (and LSE/D) ring depth: loads run two query blocks ahead
 constexpr int SM_KV = 0;                       // [item slot 2][K, V] tiles
 constexpr int SM_QR = SM_KV + 4 * TILE;        // [QS] Q tiles
 constexpr int SM_DOR = SM_QR + QS * TILE;      // [QS] dO tiles
-constexpr int SM_DS = SM_DOR + QS * TILE;      // [2][2 halves] dS^T tiles
-constexpr int SM_DQ = SM_DS + 4 * TILE;        // [4 warps] 32 x 32 fp32 staging boxes
-constexpr int SM_LD = SM_DQ + 4 * 4096;        // [QS][LSE x128 | D x128] floats
+constexpr int SM_DS = SM_DOR + QS * TILE;      // [2 halves] dS^T tile
+constexpr int SM_DQ = SM_DS + 2 * TILE;        // [4 warps] 32 x 32 fp32 staging boxes
+constexpr int SM_LD = SM_DQ + 4 * 4096;        // [QS][-LSE x128 | -D x128] floats
 constexpr int SM_TILES = SM_LD + QS * 256 * 4;
 // kv_full[2], kv_empty[2], qdo_full[QS], qdo_empty[QS], ld_full[QS], ld_empty[QS],
-// st_full, st_free, ps_full, pt_free, ds_free[2], dq_full, dq_free, dkdv_full,
-// dkdv_free, epi_stage, drain
+// st_full, st_free, ps_full, pt_free, ds_free, (spare), dq_full, dq_free,
+// dkdv_full, dkdv_free, epi_stage, drain
 constexpr int NUM_BARS = 4 + 4 * QS + 12;
 constexpr int SMEM = SM_TILES + 1024 + NUM_BARS * 8 + 16;
 static_assert(SMEM <= 232448, "backward shared memory");
@@ -1149,13 +1166,10 @@ constexpr int THREADS = 512;
 constexpr uint32_t C_ST = 0, C_DPT = 128, C_PT = 256, C_DV = 320, C_DK = 384, C_DQ = 448;
 // Register budgets per warpgroup after setmaxnreg; with 128 per thread at
 // launch the block owns 512 x 128 = 65536 and the split below uses
-// 128 x 56 + 256 x 176 + 128 x 96 = 64512 of them.
-constexpr int LAUNCH_REGS = 128, REGS_CTRL = 56, REGS_ELEM = 176, REGS_DRAIN = 96;
+// 128 x 80 + 256 x 160 + 128 x 112 = 65536 of them.
+constexpr int LAUNCH_REGS = 128, REGS_CTRL = 80, REGS_ELEM = 160, REGS_DRAIN = 112;
 static_assert(128 * REGS_CTRL + 256 * REGS_ELEM + 128 * REGS_DRAIN <= THREADS * LAUNCH_REGS, "register split");
 }  // namespace bw
-
-template <int N> DEVI void reg_dealloc() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
-template <int N> DEVI void reg_alloc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 
 __global__ void __launch_bounds__(bw::THREADS, 1)
     attn_bwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
@@ -1205,8 +1219,8 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 2);  // the item's last MMAs and the dK/dV store
-      mbar_init(ds_free(s), 1);
     }
+    mbar_init(ds_free(0), 1);
     for (int r = 0; r < QS; ++r) {
       mbar_init(qdo_full(r), 1);
       mbar_init(qdo_empty(r), 1);
@@ -1312,7 +1326,7 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
           if (t == 0 && it >= 1 && !mbar_wait_bounded(dkdv_free, (it - 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t qt = base + SM_QR + r * TILE, ot = base + SM_DOR + r * TILE;
-          const uint32_t ds = base + SM_DS + (uint32_t)(g & 1) * 2 * TILE;
+          const uint32_t ds = base + SM_DS;
           // dV += P^T dO (P^T from tensor memory)
 #pragma unroll
           for (int kk = 0; kk < BQ / 16; ++kk)
@@ -1332,7 +1346,7 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
             tc_mma_bf16(tmem + C_DQ, sdesc(ds + kk * 2048, TILE, 1024), sdesc(kt + kk * 2048, 8192, 1024), IDESC_DQ,
                         kk > 0 ? 1u : 0u);
           tc_commit(dq_full);
-          tc_commit(ds_free(g & 1));
+          tc_commit(ds_free(0));
           tc_commit(qdo_empty(r));
         }
         if (!ok) break;
@@ -1367,55 +1381,68 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
         if (!mbar_wait_bounded(ld_full(r), (g / QS) & 1, abort_flag, err)) { ok = false; break; }
         if (!mbar_wait_bounded(st_full, g & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sv[2][32], dp[2][32];
-        tmem_ld_32x32b_x32(tmem + lane_off + C_ST + 64 * half, sv[0]);
-        tmem_ld_32x32b_x32(tmem + lane_off + C_ST + 64 * half + 32, sv[1]);
-        tmem_ld_32x32b_x32(tmem + lane_off + C_DPT + 64 * half, dp[0]);
-        tmem_ld_32x32b_x32(tmem + lane_off + C_DPT + 64 * half + 32, dp[1]);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(st_free);
         // masking only on the diagonal block, past T, or for keys past T
         const bool need_mask = (t == 0) || (q0 + BQ > T) || (kv >= T);
-        const float* ld = sLD + r * 256;
+        const float* ld = sLD + r * 256;  // -LSE, -D
         uint32_t pp[32], pd[32];
+        const float2 sc2 = make_float2(scale_log2, scale_log2);
+        // the two 32-column halves one after the other (fewer live
+        // registers); S^T / dP^T are released once both halves are loaded
 #pragma unroll
         for (int sub = 0; sub < 2; ++sub) {
+          uint32_t sv[1][32], dp[1][32];
+          tmem_ld_32x32b_x32(tmem + lane_off + C_ST + 64 * half + 32 * sub, sv[0]);
+          tmem_ld_32x32b_x32(tmem + lane_off + C_DPT + 64 * half + 32 * sub, dp[0]);
+          tmem_ld_wait();
+          if (sub == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(st_free);
+          }
           const int c0 = 64 * half + 32 * sub;
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
             // broadcast reads: every lane needs the same four columns
             const float4 l4 = *reinterpret_cast<const float4*>(ld + c0 + i);
             const float4 d4 = *reinterpret_cast<const float4*>(ld + 128 + c0 + i);
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
-            float pv[4], dv[4];
+            // two columns per packed fp32x2 operation
+            const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sv[0][i]), __uint_as_float(sv[0][i + 1])),
+                                          sc2, make_float2(l4.x, l4.y));
+            const float2 x23 = __ffma2_rn(
+                make_float2(__uint_as_float(sv[0][i + 2]), __uint_as_float(sv[0][i + 3])), sc2,
+                make_float2(l4.z, l4.w));
+            float pv[4] = {ex2(x01.x), ex2(x01.y), ex2(x23.x), ex2(x23.y)};
+            if (need_mask) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              float p = ex2(fmaf(__uint_as_float(sv[sub][i + u]), scale_log2, -lv[u]));
-              if (need_mask) {
+              for (int u = 0; u < 4; ++u) {
                 const int qq = q0 + c0 + i + u;
-                if (qq < kv || qq >= T || kv >= T) p = 0.f;
+                if (qq < kv || qq >= T || kv >= T) pv[u] = 0.f;
               }
-              pv[u] = p;
-              dv[u] = p * (__uint_as_float(dp[sub][i + u]) - dd[u]);
             }
+            const float2 e01 = __fadd2_rn(make_float2(__uint_as_float(dp[0][i]), __uint_as_float(dp[0][i + 1])),
+                                          make_float2(d4.x, d4.y));
+            const float2 e23 = __fadd2_rn(
+                make_float2(__uint_as_float(dp[0][i + 2]), __uint_as_float(dp[0][i + 3])),
+                make_float2(d4.z, d4.w));
+            const float2 g01 = __fmul2_rn(make_float2(pv[0], pv[1]), e01);
+            const float2 g23 = __fmul2_rn(make_float2(pv[2], pv[3]), e23);
             pp[sub * 16 + i / 2] = pack_bf16x2(pv[0], pv[1]);
             pp[sub * 16 + i / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-            pd[sub * 16 + i / 2] = pack_bf16x2(dv[0], dv[1]);
-            pd[sub * 16 + i / 2 + 1] = pack_bf16x2(dv[2], dv[3]);
+            pd[sub * 16 + i / 2] = pack_bf16x2(g01.x, g01.y);
+            pd[sub * 16 + i / 2 + 1] = pack_bf16x2(g23.x, g23.y);
           }
         }
         // every lane has read this block's LSE / D
         __syncwarp();
         if (lane == 0) mbar_arrive(ld_empty(r));
-        // dV of the previous block has read P^T; dK, dQ of block g-2 have
-        // read this dS^T buffer
+        // dV of the previous block has read P^T, its dK and dQ have read dS^T
+        // (they are issued right after this warp's previous release, and this
+        // block's arithmetic above is longer than they take)
         if (g >= 1 && !mbar_wait_bounded(pt_free, (g - 1) & 1, abort_flag, err)) { ok = false; break; }
-        if (g >= 2 && !mbar_wait_bounded(ds_free(g & 1), ((g - 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        if (g >= 1 && !mbar_wait_bounded(ds_free(0), (g - 1) & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         tmem_st_32x32b_x32(tmem + lane_off + C_PT + 32 * half, pp);
-        const uint32_t drow = base + SM_DS + (uint32_t)(g & 1) * 2 * TILE + half * TILE + (uint32_t)row * 128u;
+        const uint32_t drow = base + SM_DS + half * TILE + (uint32_t)row * 128u;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           st_shared_v4(drow + 16u * (uint32_t)(c ^ (row & 7)), pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
@@ -1435,15 +1462,16 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t box = base + SM_DQ + (uint32_t)q * 4096u;
     bool ok = true;
-    // LSE (log2 domain) and D of query block t of item (kb, b, h) into ring
-    // slot r (queries past T: LSE = +inf, D = 0)
+    // -LSE (log2 domain) and -D of query block t of item (kb, b, h) into
+    // ring slot r (queries past T: -LSE = -inf, -D = 0), negated so the
+    // elementwise warps need one fused multiply-add and one add per pair
     auto stage_ld = [&](int g, int kb, int b, int h, int t) -> bool {
       const int r = g % QS;
       if (g >= QS && !mbar_wait_bounded(ld_empty(r), ((g - QS) / QS) & 1, abort_flag, err)) return false;
       const int qq = (kb + t) * BQ + tid;
       const long bh0 = ((long)b * H + h) * T;
-      sLD[r * 256 + tid] = qq < T ? lse[bh0 + qq] * LOG2E_F : INFINITY;
-      sLD[r * 256 + 128 + tid] = qq < T ? dvec[bh0 + qq] : 0.f;
+      sLD[r * 256 + tid] = qq < T ? -lse[bh0 + qq] * LOG2E_F : -INFINITY;
+      sLD[r * 256 + 128 + tid] = qq < T ? -dvec[bh0 + qq] : 0.f;
       __syncwarp();
       if (lane == 0) mbar_arrive(ld_full(r));
       return true;
@@ -1476,6 +1504,7 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
         }
         // dQ of block g: tensor memory -> registers (the buffer is then free
         // for the next block's dQ) -> two 32 x 32 fp32 boxes -> TMA reduce-add
+        // (bulk reductions into L2; per-lane vector reductions measured slower)
         if (!mbar_wait_bounded(dq_full, g & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         uint32_t dq[2][32];
@@ -1564,6 +1593,8 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
 
 }  // namespace
 
+int attn_tc_set_wait_limit(unsigned long long ns) { return set_unit_wait_limit(ns); }
+
 int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float* dvec, void* dqkv, float* dq_acc,
                 int B, int T, int H, cudaStream_t st) {
   if (B <= 0 || T <= 0) return GPT2_OK;
@@ -1621,21 +1652,24 @@ int attn_fwd_tc(const void* qkv, void* o, float* lse, int B, int T, int H, cudaS
   const uint64_t dout[3] = {d, (uint64_t)T, (uint64_t)B};
   const uint64_t sout[2] = {d * 2, (uint64_t)T * d * 2};
   if (!tmap_3d(&tq, qkv, dq, sq) || !tmap_3d(&to, o, dout, sout)) return GPT2_ERR_CUDA;
+  // The two-tile kernel, if its launch register count is the one its
+  // register split is computed for (checked once on the host; "1" in
+  // GPT2_ATTN_FWD_TC selects the one-tile kernel, for comparison).
   static int v2 = -1;
   if (v2 < 0) {
     const char* e = getenv("GPT2_ATTN_FWD_TC");
-    v2 = (e && e[0] == '1') ? 0 : 1;  // "1": the one-tile kernel, for comparison
+    cudaFuncAttributes fa;
+    v2 = (e && e[0] == '1') ? 0
+         : (cudaFuncGetAttributes(&fa, attn_fwd_tc2_kernel) == cudaSuccess && fa.numRegs == F2_LAUNCH_REGS) ? 1
+                                                                                                           : 0;
+    cudaGetLastError();
+    if (v2) CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F2_SMEM));
   }
   if (v2) {
-    static bool attr2 = false;
-    if (!attr2) {
-      CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F2_SMEM));
-      attr2 = true;
-    }
     const int nqb = (T + BQ - 1) / BQ;
     const int n_items = ((nqb + 1) / 2) * B * H;
     const int grid = n_items < num_sms() ? n_items : num_sms();
-    CUDA_TRY(launch_k(attn_fwd_tc2_kernel, grid, NUM_THREADS, F2_SMEM, st, tq, to, lse, T, H, n_items,
+    CUDA_TRY(launch_k(attn_fwd_tc2_kernel, grid, F2_THREADS, F2_SMEM, st, tq, to, lse, T, H, n_items,
                       LOG2E_F / 8.f, nullptr));
     LAUNCH_CHECK();
     return GPT2_OK;

@@ -20,8 +20,15 @@ enum : int {
 };
 
 // A pipeline wait that has not completed after this long is treated as a
-// hang: the kernel records DEV_ERR_TIMEOUT and leaves the wait.
+// hang: the kernel records DEV_ERR_TIMEOUT and leaves the wait.  The limit of
+// the pipeline waits can be changed per device (gpt2_set_wait_timeout_ns; one
+// copy per compilation unit that has such waits); the waits that drain copies
+// already in flight before a kernel exits keep WAIT_TIMEOUT_NS.
 #define WAIT_TIMEOUT_NS 2000000000ull
+static __device__ unsigned long long g_wait_limit_ns = WAIT_TIMEOUT_NS;
+static inline int set_unit_wait_limit(unsigned long long ns) {
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns)) == cudaSuccess ? 0 : -3;
+}
 
 #define DEVI __device__ __forceinline__
 
@@ -150,12 +157,12 @@ DEVI bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 DEVI bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                             int* err) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer();
+  const uint64_t t0 = globaltimer(), lim = g_wait_limit_ns;
   uint32_t spins = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if ((++spins & 63u) == 0 && globaltimer() - t0 > WAIT_TIMEOUT_NS) {
+    if ((++spins & 63u) == 0 && globaltimer() - t0 > lim) {
       *abort_flag = 1;
       if (err) atomicOr(err, DEV_ERR_TIMEOUT);
       return false;
@@ -213,6 +220,11 @@ DEVI void tma_reduce_add_3d(const void* tmap, uint32_t src, int c0, int c1, int 
           reinterpret_cast<uint64_t>(tmap)),
       "r"(src), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+// Four consecutive floats added to global memory as one vector reduction
+// (16-byte aligned address).
+DEVI void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 DEVI void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 template <int N>
@@ -349,12 +361,12 @@ DEVI bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
 // mbar_wait_bounded for a barrier that threads of the peer CTA arrive on.
 DEVI bool mbar_wait_bounded_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
-  uint64_t t0 = globaltimer();
+  const uint64_t t0 = globaltimer(), lim = g_wait_limit_ns;
   uint32_t spins = 0;
   while (true) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if (*abort_flag) return false;
-    if ((++spins & 63u) == 0 && globaltimer() - t0 > WAIT_TIMEOUT_NS) {
+    if ((++spins & 63u) == 0 && globaltimer() - t0 > lim) {
       *abort_flag = 1;
       if (err) atomicOr(err, DEV_ERR_TIMEOUT);
       return false;

@@ -393,16 +393,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // pass over TMEM), then exp(acc - max) and its sum in the store pass
       float cmax = -INFINITY, csum = 0.f;
       int ytgt = -1;
-      if (ce) {
+      if (ce && nch > 0) {
+        // N is a multiple of 128, so a warp's 128 columns are all inside N or
+        // all outside: the maximum pass takes two chunks per TMEM wait
         if (row < p.M) ytgt = __ldg(p.epi.ce_tgt + row);
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int ci = 0; ci < NCH; ++ci) {
-          if (ci >= nch) break;
+        for (int ci = 0; ci < NCH; ci += 2) {
           tmem_ld_32x32b_x32(tm_row + 32u * (uint32_t)ci, r[0]);
+          tmem_ld_32x32b_x32(tm_row + 32u * (uint32_t)(ci + 1), r[1]);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) cmax = fmaxf(cmax, __uint_as_float(r[0][j]));
+          for (int j = 0; j < 32; ++j) {
+            mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(r[0][j]));
+            mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(r[1][j]));
+          }
         }
+        cmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       }
       if (PREFETCH && nch > 0) tmem_ld_32x32b_x32(tm_row, r[0]);
 #pragma unroll
@@ -547,6 +554,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   tc_fence_before();
+  // After an abort a pair's CTAs cannot observe each other's copies in flight
+  // (the odd CTA's loads complete on the even CTA's barriers, which the even
+  // CTA drains only for the stages it armed itself): on that error path both
+  // wait out a copy's latency many times over before leaving.
+  if (PAIR && *abort_flag && (warp == 0 && lane == 0)) {
+    const uint64_t t0 = globaltimer();
+    while (globaltimer() - t0 < 100000ull) {
+    }
+  }
   __syncthreads();
   // neither CTA of a pair leaves while the other may still signal its barriers
   if constexpr (PAIR) cluster_sync_all();
@@ -731,6 +747,8 @@ int num_sms() {
   }
   return n;
 }
+
+int gemm_tc_set_wait_limit(unsigned long long ns) { return set_unit_wait_limit(ns); }
 
 size_t gemm_tc_split_bytes(int M, int N, int K) {
   int s = auto_splits(M, N, K, resolve_bn(0, N));

@@ -104,8 +104,9 @@ struct Work {
   std::vector<LayerActs> layers;
   void *x_final, *yf, *logits;
   float *meanf, *rstdf, *loss_rows;
-  // fused cross-entropy (bf16): per-part maxima and sums [V/128][M], target logits
-  float *ce_pm, *ce_ps, *ce_zt;
+  // fused cross-entropy (bf16): per-part maxima and sums [V/128][M], target
+  // logits, row log-sum-exps
+  float *ce_pm, *ce_ps, *ce_zt, *ce_lse;
   void *dres, *dy, *du, *dqkv, *dout;
   float *dq_acc, *dvec;
   float *norm_part, *gnorm;  // global gradient norm: block partials and the result
@@ -174,6 +175,7 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
   w->ce_pm = c.take<float>((size_t)parts * M * 4);
   w->ce_ps = c.take<float>((size_t)parts * M * 4);
   w->ce_zt = c.take<float>(M * 4);
+  w->ce_lse = c.take<float>(M * 4);
   w->dres = c.take<void>(M * d * act);
   w->dy = c.take<void>(M * d * act);
   w->du = c.take<void>(M * 4 * d * act);
@@ -471,7 +473,8 @@ int gpt2_forward_loss(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets
   if (f32)
     TRY(ce_fwd(f32, w.logits, w.tgt, w.loss_rows, M, V, (int)s.Vr, w.n_valid, w.err, st));
   else
-    TRY(ce_merge_dz(w.ce_pm, w.ce_ps, w.ce_zt, w.tgt, w.logits, M, V, (int)s.Vr, w.n_valid, w.loss_rows, st));
+    TRY(ce_merge_dz(w.ce_pm, w.ce_ps, w.ce_zt, w.tgt, w.logits, w.ce_lse, M, V, (int)s.Vr, w.n_valid, w.loss_rows,
+                    st));
   TRY(loss_mean(w.loss_rows, M, w.n_valid, loss_dev ? loss_dev : w.loss, w.err, st));
   c->have_fwd = 1;
   c->fwd_batch = batch;
@@ -797,6 +800,25 @@ int gpt2_op_gemm_bf16(const uint16_t* A, int a_mn_major, int lda, const uint16_t
   return gemm_tc_bf16(g, workspace, workspace_bytes, bn, splits, nullptr, S(stream));
 }
 
+int gpt2_set_wait_timeout_ns(uint64_t ns) {
+  const unsigned long long v = ns ? (unsigned long long)ns : WAIT_TIMEOUT_NS;
+  TRY(gemm_tc_set_wait_limit(v));
+  return attn_tc_set_wait_limit(v);
+}
+
+int gpt2_op_gemm_bf16_status(const uint16_t* A, int a_mn_major, int lda, const uint16_t* B, int b_mn_major, int ldb,
+                             void* C, int c_fp32, int ldc, int M, int N, int K, float alpha, float beta,
+                             void* workspace, size_t workspace_bytes, int bn, int splits, int* status,
+                             void* stream) {
+  if (!A || !B || !C || !status || M < 0 || N < 0 || K < 0) return GPT2_ERR_INVALID_ARG;
+  if ((uintptr_t)status & 3) return GPT2_ERR_INVALID_ARG;
+  GemmArgs g = make_gemm(M, N, K, A, a_mn_major ? 1 : 0, lda, B, b_mn_major ? 1 : 0, ldb,
+                         c_fp32 ? EPI_F32 : EPI_STORE, C, ldc);
+  g.epi.alpha = alpha;
+  g.epi.beta = c_fp32 ? beta : 0.f;
+  return gemm_tc_bf16(g, workspace, workspace_bytes, bn, splits, status, S(stream));
+}
+
 int gpt2_op_attention_fwd_bf16(const uint16_t* qkv, uint16_t* o, float* lse, int B, int T, int H, int hd,
                                void* stream) {
   if (!qkv || !o || !lse || B < 0 || T < 0 || H < 1) return GPT2_ERR_INVALID_ARG;
@@ -863,12 +885,13 @@ int gpt2_op_colsum_bf16(const uint16_t* x, int M, int N, float* out, float* scra
 namespace {
 // Scratch of the LM-head cross-entropy ops: status word, n_valid, then the
 // bf16 [M, V] buffer (the forward's exponentials, rewritten as dz), the
-// per-part maxima and sums [V/128][M] and the target logits [M].
+// per-part maxima and sums [V/128][M], the target logits and the row
+// log-sum-exps [M].
 struct CeScratch {
   int* err;
   int* n_valid;
   void* e;
-  float *pm, *ps, *zt;
+  float *pm, *ps, *zt, *lse;
   size_t bytes;
 };
 CeScratch ce_scratch(void* base, int M, int V) {
@@ -880,6 +903,7 @@ CeScratch ce_scratch(void* base, int M, int V) {
   s.pm = c.take<float>((size_t)(V / 128) * M * 4);
   s.ps = c.take<float>((size_t)(V / 128) * M * 4);
   s.zt = c.take<float>((size_t)M * 4);
+  s.lse = c.take<float>((size_t)M * 4);
   s.bytes = (c.off + 255) & ~(size_t)255;
   return s;
 }
@@ -907,7 +931,7 @@ int gpt2_op_lm_head_ce_fwd_bf16(const uint16_t* x, const uint16_t* w, const int3
   g.epi.ce_tgt = targets;
   TRY(gemm_tc_bf16(g, nullptr, 0, 0, 1, cs.err, st));
   TRY(count_targets(targets, M, vocab_real, cs.n_valid, cs.err, st));
-  TRY(ce_merge_dz(cs.pm, cs.ps, cs.zt, targets, cs.e, M, V, vocab_real, cs.n_valid, loss_rows, st));
+  TRY(ce_merge_dz(cs.pm, cs.ps, cs.zt, targets, cs.e, cs.lse, M, V, vocab_real, cs.n_valid, loss_rows, st));
   return loss_mean(loss_rows, M, cs.n_valid, loss, cs.err, st);
 }
 

@@ -59,6 +59,11 @@ int gemm_simt_f32(const GemmArgs& g, cudaStream_t st);
 
 int num_sms();
 
+// Limit (ns) of the pipeline waits of the tcgen05 GEMM / attention kernels on
+// the current device.
+int gemm_tc_set_wait_limit(unsigned long long ns);
+int attn_tc_set_wait_limit(unsigned long long ns);
+
 // tcgen05 causal attention forward / backward, head_dim 64 (bf16).  The
 // backward expects dvec = rowsum(dO * O) and a zeroed fp32 dq_acc; it writes dK,
 // dV into dqkv and reduces scale * dQ into dq_acc.
@@ -116,12 +121,12 @@ int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, i
            int vocab_real, const int* n_valid, int* err, cudaStream_t st);
 int loss_mean(const float* loss_rows, int M, const int* n_valid, float* loss, int* err, cudaStream_t st);
 // The cross-entropy from the LM head's EPI_CE_FWD outputs: per row the
-// log-sum-exp from the per-part maxima / sums [V/128][M], the loss row
+// log-sum-exp (lse [M]) from the per-part maxima / sums [V/128][M], the loss row
 // (LSE - z[target], 0 where masked), and, in place over the stored bf16
 // exp(z - part max) [M, V], dz = (softmax - onehot(target)) * M / n_valid
 // (zero rows where masked), the operand of the two backward GEMMs.
-int ce_merge_dz(const float* part_max, const float* part_sum, const float* zt, const int32_t* tgt, void* e, int M,
-                int V, int vocab_real, const int* n_valid, float* loss_rows, cudaStream_t st);
+int ce_merge_dz(const float* part_max, const float* part_sum, const float* zt, const int32_t* tgt, void* e,
+                float* lse, int M, int V, int vocab_real, const int* n_valid, float* loss_rows, cudaStream_t st);
 // dwte[tok[m]] += dx[m] (deterministic fixed-point scatter at a resolution of
 // 2^-32 |grad_scale|), dwpe (=/+=) sum_b dx
 int embed_bwd(int f32, const int32_t* tok, const void* dx, float* dwte, float* dwpe,

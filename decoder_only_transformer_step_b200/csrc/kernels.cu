@@ -677,31 +677,26 @@ __global__ void loss_mean_kernel(const float* __restrict__ rows, int M, const in
 // Cross-entropy from the LM head's partials (the EPI_CE_FWD epilogue of the
 // tied LM-head GEMM): for row m and part p of 128 vocabulary columns,
 // pm[p*M+m] = max_v z and ps[p*M+m] = sum_v exp(z - pm); zt[m] = z[m, target];
-// e[m, v] = bf16 exp(z - pm) for v in part p.  Per row:
+// e[m, v] = bf16 exp(z - pm) for v in part p.
+// ce_merge_kernel, per row:
 //   lse_m = max_p pm + log sum_p ps exp(pm - max)       (the row's log-sum-exp)
 //   loss_m = lse_m - zt[m] (0 where masked)
-//   e[m, v] <- e[m, v] exp(pm - lse_m) M / n_valid - [v == target] M / n_valid,
-// i.e. dz = (softmax - onehot) scaled so the backward GEMMs' alpha =
-// grad_scale / M gives the mean over the positions with a target.  32 rows per
-// block: the eight warps take every eighth part for the log-sum-exp (partials
-// meet in shared memory in a fixed order), then every thread rewrites 16-byte
-// pieces of the block's rows with the row's part scales from shared memory.
-constexpr int CEM_ROWS = 32;
-__global__ void __launch_bounds__(256) ce_merge_dz_kernel(const float* __restrict__ pm, const float* __restrict__ ps,
-                                                          const float* __restrict__ zt,
-                                                          const int32_t* __restrict__ tgt, bf16* __restrict__ e,
-                                                          int M, int V, int vocab_real,
-                                                          const int* __restrict__ n_valid,
-                                                          float* __restrict__ loss_rows) {
+// 32 rows per block; the eight warps take every eighth part and their partial
+// results meet in shared memory in a fixed order.
+// ce_dz_kernel, in place over e:
+//   e[m, v] <- (e[m, v] exp(pm - lse_m) - [v == target]) M / n_valid
+// (0 where masked), i.e. dz = (softmax - onehot) scaled so that the backward
+// GEMMs' alpha = grad_scale / M gives the mean over the positions with a
+// target.  One block per token row, four 16-byte loads in flight per thread.
+__global__ void __launch_bounds__(256) ce_merge_kernel(const float* __restrict__ pm, const float* __restrict__ ps,
+                                                       const float* __restrict__ zt, const int32_t* __restrict__ tgt,
+                                                       int M, int P, int vocab_real, float* __restrict__ lse_out,
+                                                       float* __restrict__ loss_rows) {
   pdl_start();
   constexpr float L2E = 1.4426950408889634f;
-  extern __shared__ float sc[];          // [CEM_ROWS][P] scales
-  __shared__ float red[8][CEM_ROWS];
-  __shared__ int ytgt[CEM_ROWS];
-  const int P = V / 128;
+  __shared__ float red[8][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * CEM_ROWS;
-  const int m = m0 + lane;
+  const int m = blockIdx.x * 32 + lane;
   const bool in = m < M;
   float mx = -INFINITY;
   if (in)
@@ -720,40 +715,62 @@ __global__ void __launch_bounds__(256) ce_merge_dz_kernel(const float* __restric
     }
   red[warp][lane] = sum;
   __syncthreads();
-  float tot = 0.f;
+  if (warp == 0 && in) {
+    float tot = 0.f;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) tot += red[w][lane];
-  const float lse = gm + logf(tot);
-  const int y = in ? tgt[m] : -1;
+    for (int w = 0; w < 8; ++w) tot += red[w][lane];
+    const float lse = gm + logf(tot);
+    const int y = tgt[m];
+    const bool valid = y >= 0 && y < vocab_real;
+    lse_out[m] = lse;
+    loss_rows[m] = valid ? lse - zt[m] : 0.f;
+  }
+}
+
+__global__ void __launch_bounds__(256) ce_dz_kernel(bf16* __restrict__ e, const float* __restrict__ pm,
+                                                    const float* __restrict__ lse, const int32_t* __restrict__ tgt,
+                                                    int M, int V, int vocab_real, const int* __restrict__ n_valid) {
+  pdl_start();
+  constexpr float L2E = 1.4426950408889634f;
+  constexpr int U = 4;
+  const int m = blockIdx.x;
+  const int y = tgt[m];
   const bool valid = y >= 0 && y < vocab_real;
   const int nv = *n_valid;
   const float full = (float)M / (float)(nv > 0 ? nv : 1);
   const float scale = valid ? full : 0.f;
-  if (in)
-    for (int p = warp; p < P; p += 8) sc[lane * P + p] = ex2_approx((pm[(long)p * M + m] - lse) * L2E) * scale;
-  if (warp == 0) {
-    if (in) loss_rows[m] = valid ? lse - zt[m] : 0.f;
-    ytgt[lane] = valid ? y : -1;
-  }
-  __syncthreads();
-  // the rewrite: 8 bf16 (16 bytes) per step, a row's V / 8 pieces in order
-  const int nrows = min(CEM_ROWS, M - m0);
-  const int per_row = V / 8;
-  for (int i = threadIdx.x; i < nrows * per_row; i += blockDim.x) {
-    const int r = i / per_row, c = (i % per_row) * 8;
-    uint4* ptr = reinterpret_cast<uint4*>(e + (long)(m0 + r) * V + c);
-    uint4 u = *ptr;
-    const float s = sc[r * P + (c >> 7)];
-    const int dy = ytgt[r] - c;
-    float f[8] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y),
-                  bf16lo(u.z), bf16hi(u.z), bf16lo(u.w), bf16hi(u.w)};
+  const float l2 = lse[m] * L2E;
+  const int yv = valid ? y : -1;
+  bf16* row = e + (long)m * V;
+  const int pieces = V / 8;
+  // the whole row, 16-byte pieces 4 KB apart, four loads in flight per thread
+  for (int p0 = threadIdx.x; p0 < pieces; p0 += 256 * U) {
+    uint4 u[U];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) f[j] = f[j] * s - (dy == j ? full : 0.f);
-    u.x = pack_bf16x2(f[0], f[1]);
-    u.y = pack_bf16x2(f[2], f[3]);
-    u.z = pack_bf16x2(f[4], f[5]);
-    u.w = pack_bf16x2(f[6], f[7]);
-    *ptr = u;
+    for (int k = 0; k < U; ++k) {
+      const int pi = p0 + 256 * k;
+      if (pi < pieces) u[k] = *reinterpret_cast<const uint4*>(row + 8 * pi);
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int pi = p0 + 256 * k;
+      if (pi < pieces) {
+        const int c = 8 * pi;
+        // one part's scale exp(pm - lse) per 16-byte piece (V is a multiple of 128)
+        const float s = ex2_approx(fmaf(pm[(long)(c >> 7) * M + m], L2E, -l2)) * scale;
+        const int dy = yv - c;
+        float f[8] = {bf16lo(u[k].x), bf16hi(u[k].x), bf16lo(u[k].y), bf16hi(u[k].y),
+                      bf16lo(u[k].z), bf16hi(u[k].z), bf16lo(u[k].w), bf16hi(u[k].w)};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] = f[j] * s - (dy == j ? full : 0.f);
+        uint4 o;
+        o.x = pack_bf16x2(f[0], f[1]);
+        o.y = pack_bf16x2(f[2], f[3]);
+        o.z = pack_bf16x2(f[4], f[5]);
+        o.w = pack_bf16x2(f[6], f[7]);
+        *reinterpret_cast<uint4*>(row + c) = o;
+      }
+    }
   }
 }
 
@@ -1121,17 +1138,14 @@ int ce_fwd(int f32, void* logits, const int32_t* tgt, float* loss_rows, int M, i
   return GPT2_OK;
 }
 
-int ce_merge_dz(const float* part_max, const float* part_sum, const float* zt, const int32_t* tgt, void* e, int M,
-                int V, int vocab_real, const int* n_valid, float* loss_rows, cudaStream_t st) {
-  if (V % 128 || V > 65536) return GPT2_ERR_UNSUPPORTED_SHAPE;
-  const size_t smem = (size_t)CEM_ROWS * (V / 128) * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    CUDA_TRY(cudaFuncSetAttribute(ce_merge_dz_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536));
-    attr = true;
-  }
-  CUDA_TRY(launch_k(ce_merge_dz_kernel, (M + CEM_ROWS - 1) / CEM_ROWS, 256, smem, st, part_max, part_sum, zt, tgt,
-                    (bf16*)e, M, V, vocab_real, n_valid, loss_rows));
+int ce_merge_dz(const float* part_max, const float* part_sum, const float* zt, const int32_t* tgt, void* e,
+                float* lse, int M, int V, int vocab_real, const int* n_valid, float* loss_rows, cudaStream_t st) {
+  if (V % 128) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  CUDA_TRY(launch_k(ce_merge_kernel, (M + 31) / 32, 256, 0, st, part_max, part_sum, zt, tgt, M, V / 128, vocab_real,
+                    lse, loss_rows));
+  LAUNCH_CHECK();
+  CUDA_TRY(launch_k(ce_dz_kernel, M, 256, 0, st, (bf16*)e, part_max, (const float*)lse, tgt, M, V, vocab_real,
+                    n_valid));
   LAUNCH_CHECK();
   return GPT2_OK;
 }

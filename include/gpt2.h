@@ -291,6 +291,26 @@ int gpt2_op_attention_bwd_bf16(const uint16_t* qkv, const uint16_t* o, const flo
                                const uint16_t* dout, uint16_t* dqkv, float* scratch,
                                int B, int T, int H, int hd, void* stream);
 
+/* Hang detection.  Every pipeline wait inside the tcgen05 GEMM and attention
+ * kernels (a TMA copy, an MMA, a hand-off between warps) gives up after a
+ * limit, records GPT2_ERR_TIMEOUT in the device status word (what
+ * gpt2_get_status reads, or the status argument of gpt2_op_gemm_bf16_status),
+ * lets the copies and MMAs already in flight finish, frees its tensor memory
+ * and returns, so the context stays usable.  This sets the limit in
+ * nanoseconds on the current device (0 restores the default of 2 s).  The
+ * survey's failure-detection item: a hung pipeline becomes an error the host
+ * reads instead of a hung GPU.  Not stream-ordered: call it with no kernel of
+ * the library in flight. */
+int gpt2_set_wait_timeout_ns(uint64_t ns);
+
+/* gpt2_op_gemm_bf16 with a device status word: status (device int, 4-byte
+ * aligned) is OR-ed with GPT2's device error bits (4 = a pipeline wait timed
+ * out). */
+int gpt2_op_gemm_bf16_status(const uint16_t* A, int a_mn_major, int lda, const uint16_t* B, int b_mn_major, int ldb,
+                             void* C, int c_fp32, int ldc, int M, int N, int K, float alpha, float beta,
+                             void* workspace, size_t workspace_bytes, int bn, int splits, int* status,
+                             void* stream);
+
 /* Allocation-free variant of gpt2_op_attention_bwd_bf16 (same inputs, same
  * output dqkv, no scratch argument).  The paper has no counterpart: this entry
  * point exists for callers that cannot call cudaMalloc -- a host that gives a

@@ -164,3 +164,15 @@ def test_lm_head_cross_entropy_ops_validate_on_host():
         gp.ERRORS_BY_NAME["GPT2_ERR_WORKSPACE"]
     assert L.gpt2_op_lm_head_ce_bwd_bf16(None, p, 64, 1024, 64, 1.0, p, p, 0, p, 1 << 30, None) == \
         gp.ERRORS_BY_NAME["GPT2_ERR_INVALID_ARG"]
+
+
+def test_status_gemm_validates_on_host():
+    # the status-word GEMM rejects a missing or misaligned status pointer
+    # before any CUDA call
+    L = gp._lib()
+    p = ctypes.c_void_p(4096)
+    inv = gp.ERRORS_BY_NAME["GPT2_ERR_INVALID_ARG"]
+    assert L.gpt2_op_gemm_bf16_status(p, 0, 64, p, 0, 64, p, 0, 64, 64, 64, 64, 1.0, 0.0, None, 0, 0, 0, None,
+                                      None) == inv
+    assert L.gpt2_op_gemm_bf16_status(p, 0, 64, p, 0, 64, p, 0, 64, 64, 64, 64, 1.0, 0.0, None, 0, 0, 0,
+                                      ctypes.c_void_p(4098), None) == inv
