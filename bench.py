@@ -117,7 +117,7 @@ def run_ours(args, rank, world, local_rank):
 
     import decoder_only_transformer_step_b200 as gp
     from decoder_only_transformer_step_b200 import inputs, flops
-    from decoder_only_transformer_step_b200.dp import average_gradients, zero1_step
+    from decoder_only_transformer_step_b200 import dp
 
     torch.cuda.set_device(local_rank)
     if world > 1:
@@ -136,22 +136,41 @@ def run_ours(args, rank, world, local_rank):
         pool.append((torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda()))
     stream = torch.cuda.current_stream()
 
-    def optimizer_step(step_no):
-        # gradient exchange + AdamW: one all-reduce and the full update, or with
-        # --zero1 a reduce-scatter, the update of this rank's shard and an
-        # all-gather of the weights
-        if world > 1 and args.zero1:
-            zero1_step(model.grad, model.master, lambda off, cnt: model.adamw_step_range(step_no, off, cnt),
-                       model.refresh_shadow)
+    # data parallel (N > 1): the gradient exchange per bucket (a decoder block,
+    # the final LayerNorm, the embeddings) on a side stream, each bucket's
+    # collective started by the event the backward records when the bucket's
+    # gradients are final, overlapped with the rest of the backward; all-reduce
+    # and the full AdamW, or with --zero1 reduce-scatter, the update of this
+    # rank's part of every bucket and an all-gather of the weights
+    exchange = None
+    if world > 1:
+        buckets = dp.gradient_buckets(gp.gpt2_tensors(mc.c()), L)
+        events = [torch.cuda.Event() for _ in buckets]
+        for ev in events:
+            ev.record()
+        exchange = dp.BucketedExchange(buckets, zero1=args.zero1, events=events, stream=torch.cuda.Stream())
+
+    def backward(grad_scale, accumulate, last):
+        # the exchange runs with the last micro-batch's backward only
+        if exchange is None or not last:
+            model.backward(grad_scale, accumulate)
             return
-        if world > 1:
-            average_gradients(model.grad)
-        model.adamw_step(step_no)
+        model.backward_bucketed(exchange.events, grad_scale, accumulate)
+        for b in dp.completion_order(L):
+            exchange.bucket_ready(model.grad, b)
+        exchange.finish()
+
+    def optimizer_step(step_no):
+        if exchange is None:
+            model.adamw_step(step_no)
+            return
+        exchange.optimizer_step(model.master, lambda off, cnt: model.adamw_step_range(step_no, off, cnt),
+                                model.refresh_shadow)
 
     def step(i):
         tok, tgt = pool[i % len(pool)]
         model.forward_loss(tok, tgt)
-        model.backward(1.0, 0)
+        backward(1.0, 0, True)
         optimizer_step(i + 1)
 
     for i in range(args.warmup):
@@ -200,7 +219,7 @@ def run_ours(args, rank, world, local_rank):
             tok = tok_h[i % 2].cuda(non_blocking=True)
             tgt = tgt_h[i % 2].cuda(non_blocking=True)
             model.forward_loss(tok, tgt)
-            model.backward(1.0, 0)
+            backward(1.0, 0, True)
             optimizer_step(args.warmup + args.steps + i + 1)
             loss_h.copy_(model.loss)
             torch.cuda.synchronize()
@@ -230,7 +249,7 @@ def run_ours(args, rank, world, local_rank):
             for j in range(k):
                 tok, tgt = pool[(i * k + j) % len(pool)]
                 model.forward_loss(tok, tgt)
-                model.backward(1.0 / k, 1 if j else 0)
+                backward(1.0 / k, 1 if j else 0, j == k - 1)
             optimizer_step(args.warmup + args.steps + e_steps + 2 + i)
 
         a_steps = 2

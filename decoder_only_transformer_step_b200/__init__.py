@@ -56,7 +56,7 @@ EXPORTS = [
     "gpt2_op_layernorm_fwd_bf16", "gpt2_op_layernorm_bwd_scratch_floats", "gpt2_op_layernorm_bwd_bf16",
     "gpt2_op_colsum_scratch_floats", "gpt2_op_colsum_bf16",
     "gpt2_op_lm_head_ce_scratch_bytes", "gpt2_op_lm_head_ce_fwd_bf16", "gpt2_op_lm_head_ce_bwd_bf16",
-    "gpt2_set_wait_timeout_ns", "gpt2_op_gemm_bf16_status",
+    "gpt2_set_wait_timeout_ns", "gpt2_op_gemm_bf16_status", "gpt2_backward_bucketed",
 ]
 
 _LIB = None
@@ -109,6 +109,7 @@ def _lib():
         "gpt2_op_lm_head_ce_fwd_bf16": (I, [P, P, P, I, I, I, I, P, P, P, S, P]),
         "gpt2_op_lm_head_ce_bwd_bf16": (I, [P, P, I, I, I, F, P, P, I, P, S, P]),
         "gpt2_set_wait_timeout_ns": (I, [U64]),
+        "gpt2_backward_bucketed": (I, [P, F, I, P, I, P]),
         "gpt2_op_gemm_bf16_status": (I, [P, I, I, P, I, I, P, I, I, I, I, I, F, F, P, S, I, I, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -197,6 +198,14 @@ def gpt2_forward_loss(ctx, tokens, targets, batch: int, loss_dev, stream=None):
 
 def gpt2_backward(ctx, grad_scale: float = 1.0, accumulate: int = 0, stream=None):
     _check(_lib().gpt2_backward(ctx, grad_scale, accumulate, _stream(stream)), "gpt2_backward")
+
+
+def gpt2_backward_bucketed(ctx, grad_scale, accumulate, events, stream=None):
+    """events: torch.cuda.Event objects (already created, e.g. recorded once),
+    n_layer + 2 of them."""
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(_lib().gpt2_backward_bucketed(ctx, grad_scale, accumulate, arr, len(events), _stream(stream)),
+           "gpt2_backward_bucketed")
 
 
 def gpt2_adamw_step(ctx, lr, beta1, beta2, eps, weight_decay, step, stream=None):
@@ -353,7 +362,7 @@ class ModelConfig:
     vocab_real: int
     vocab_padded: int
     max_batch: int
-    mode: int = 0  # 0 bf16 tensor cores, 1 fp32 correctness mode
+    mode: int = 0  # 0 bf16 tensor cores, 1 fp32 correctness mode, 2 bf16 bitwise repeatable
 
     def c(self) -> gpt2_config:
         return make_config(self.n_layer, self.d_model, self.n_head, self.n_ctx, self.vocab_real,
@@ -421,6 +430,11 @@ class GPT2:
 
     def backward(self, grad_scale=1.0, accumulate=0):
         gpt2_backward(self.ctx, grad_scale, accumulate)
+
+    def backward_bucketed(self, events, grad_scale=1.0, accumulate=0):
+        """The backward recording events[i] when bucket i's gradients are
+        final (see gpt2_backward_bucketed; n_layer + 2 events)."""
+        gpt2_backward_bucketed(self.ctx, grad_scale, accumulate, events)
 
     def adamw_step(self, step, lr=6e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, max_norm=0.0):
         """AdamW over the flat buffer; max_norm > 0 clips the gradient to that

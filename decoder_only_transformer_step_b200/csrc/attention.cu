@@ -481,6 +481,23 @@ __global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ 
   }
 }
 
+// dqkv[m, 0:d] = bf16(sum over key blocks kb <= query block of part[kb][m])
+// in key-block order (the deterministic mode of the attention backward)
+__global__ void dq_sum_bf16_kernel(const float* __restrict__ part, bf16* __restrict__ dqkv, long M, int T, int d) {
+  pdl_start();
+  long i = (blockIdx.x * (long)blockDim.x + threadIdx.x) * 4;
+  if (i >= M * d) return;
+  const long m = i / d;
+  const int c = (int)(i % d);
+  const int qb = (int)(m % T) / 128;
+  float4 acc = *reinterpret_cast<const float4*>(part + i);
+  for (int kb = 1; kb <= qb; ++kb) {
+    const float4 v = *reinterpret_cast<const float4*>(part + (long)kb * M * d + i);
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  *reinterpret_cast<uint2*>(dqkv + m * 3 * d + c) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+}
+
 // dqkv[:, 0:d] = bf16(dq_acc)
 __global__ void dq_to_bf16_kernel(float* __restrict__ dq_acc, bf16* __restrict__ dqkv, long M, int d,
                                   int zero_after) {
@@ -687,9 +704,11 @@ int attn_fwd_bf16(const void* qkv, void* o, float* lse, int B, int T, int H, int
 }
 
 int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* dout, void* dqkv,
-                  float* dq_acc, float* dvec, int B, int T, int H, int hd, cudaStream_t st, int dvec_ready) {
+                  float* dq_acc, float* dvec, int B, int T, int H, int hd, cudaStream_t st, int dvec_ready,
+                  float* dq_part) {
   if (B <= 0 || T <= 0) return GPT2_OK;
   if (hd != 64 && hd != 16) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (dq_part && (hd != 64 || T > 4096)) return GPT2_ERR_UNSUPPORTED_SHAPE;
   const long M = (long)B * T;
   if (!dvec_ready) {
     if (hd == 64)
@@ -700,13 +719,19 @@ int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* 
           (const bf16*)o, (const bf16*)dout, dvec, dq_acc, M, T, H));
     LAUNCH_CHECK();
   }
-  int rc = (hd == 64 && !use_mma_bwd() && T <= 4096)
-               ? attn_bwd_tc(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st)
+  int rc = (hd == 64 && (dq_part || !use_mma_bwd()) && T <= 4096)
+               ? attn_bwd_tc(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st, dq_part)
                : (hd == 64 ? launch_bwd<64>(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st)
                            : launch_bwd<16>(qkv, dout, lse, dvec, dqkv, dq_acc, B, T, H, st));
   if (rc) return rc;
   const int d = H * hd;
   long n4 = (M * d) / 4;
+  if (dq_part) {
+    CUDA_TRY(launch_k(dq_sum_bf16_kernel, (unsigned)((n4 + 255) / 256), 256, 0, st, (const float*)dq_part,
+                      (bf16*)dqkv, M, T, d));
+    LAUNCH_CHECK();
+    return GPT2_OK;
+  }
   CUDA_TRY(launch_k(dq_to_bf16_kernel, (unsigned)((n4 + 255) / 256), 256, 0, st, dq_acc, (bf16*)dqkv, M, d,
                     dvec_ready));
   LAUNCH_CHECK();

@@ -1175,7 +1175,7 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
     attn_bwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
                         const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDQKV,
                         const float* __restrict__ lse, const float* __restrict__ dvec, int T, int H, int n_items,
-                        float scale, float scale_log2, int* err) {
+                        float scale, float scale_log2, int det, int* err) {
   // (local names shadow the one-CTA-per-block backward's constants above)
   constexpr int QS = bw::QS, SM_KV = bw::SM_KV, SM_QR = bw::SM_QR, SM_DOR = bw::SM_DOR, SM_DS = bw::SM_DS;
   constexpr int SM_DQ = bw::SM_DQ, SM_LD = bw::SM_LD, SM_TILES = bw::SM_TILES, NUM_BARS = bw::NUM_BARS;
@@ -1530,8 +1530,13 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            // rows past T are clipped by the tensor map
-            tma_reduce_add_3d(&tmDQ, box, h * HD + 32 * c, q0 + q * 32, b);
+            // rows past T are clipped by the tensor map.  Deterministic mode:
+            // the tile goes to the key block's own slice of the partial buffer
+            // (z = key block * batch + batch index), summed later in order
+            if (det)
+              tma_store_3d(&tmDQ, box, h * HD + 32 * c, q0 + q * 32, kb * (BH / H) + b);
+            else
+              tma_reduce_add_3d(&tmDQ, box, h * HD + 32 * c, q0 + q * 32, b);
             bulk_commit();
           }
         }
@@ -1596,10 +1601,11 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
 int attn_tc_set_wait_limit(unsigned long long ns) { return set_unit_wait_limit(ns); }
 
 int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float* dvec, void* dqkv, float* dq_acc,
-                int B, int T, int H, cudaStream_t st) {
+                int B, int T, int H, cudaStream_t st, float* dq_part) {
   if (B <= 0 || T <= 0) return GPT2_OK;
   if ((T + BQ - 1) / BQ > BS_MAX_QBLOCKS) return GPT2_ERR_UNSUPPORTED_SHAPE;
   const uint64_t d = (uint64_t)H * HD;
+  const uint64_t nqb = (uint64_t)((T + BQ - 1) / BQ);
   CUtensorMap tq, tdo;
   const uint64_t dq[3] = {3 * d, (uint64_t)T, (uint64_t)B};
   const uint64_t sq[2] = {3 * d * 2, (uint64_t)T * 3 * d * 2};
@@ -1607,8 +1613,12 @@ int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float
   const uint64_t sd[2] = {d * 2, (uint64_t)T * d * 2};
   CUtensorMap tdq, tdqkv;
   const uint64_t sdq[2] = {d * 4, (uint64_t)T * d * 4};
+  // deterministic mode: [key block][batch] slices of [T, d] fp32
+  const uint64_t dpart[3] = {d, (uint64_t)T, nqb * (uint64_t)B};
   if (!tmap_3d(&tq, qkv, dq, sq) || !tmap_3d(&tdo, dout, dd, sd) ||
-      !tmap_3d(&tdq, dq_acc, dd, sdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 32) || !tmap_3d(&tdqkv, dqkv, dq, sq))
+      !tmap_3d(&tdq, dq_part ? dq_part : dq_acc, dq_part ? dpart : dd, sdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32,
+               32) ||
+      !tmap_3d(&tdqkv, dqkv, dq, sq))
     return GPT2_ERR_CUDA;
   // The persistent kernel, if its launch register count is the one its
   // register split is computed for (otherwise a setmaxnreg.inc could wait for
@@ -1627,10 +1637,11 @@ int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float
     const int n_items = ((T + BKV - 1) / BKV) * B * H;
     const int grid = n_items < num_sms() ? n_items : num_sms();
     CUDA_TRY(launch_k(attn_bwd_tc2_kernel, grid, bw::THREADS, bw::SMEM, st, tq, tdo, tdq, tdqkv, lse, dvec, T, H,
-                      n_items, 0.125f, LOG2E_F / 8.f, nullptr));
+                      n_items, 0.125f, LOG2E_F / 8.f, dq_part ? 1 : 0, nullptr));
     LAUNCH_CHECK();
     return GPT2_OK;
   }
+  if (dq_part) return GPT2_ERR_UNSUPPORTED_SHAPE;  // (a mode of the persistent kernel only)
   static bool attr = false;
   if (!attr) {
     CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B_SMEM_BYTES));

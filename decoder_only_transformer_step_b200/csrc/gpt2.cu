@@ -20,7 +20,8 @@ const char* const kLayerNames[N_LT] = {"ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o"
 
 struct Shape {
   long L, d, H, T, V, Vr, hd;
-  int mode;
+  int mode;  // 0 bf16, 1 fp32 (the configuration's mode 2 is bf16 with det set)
+  bool det;  // bf16 with the attention backward's dQ summed in a fixed order
 };
 
 void lt_dims(long d, int t, long* rows, long* cols) {
@@ -60,11 +61,13 @@ struct Offsets {
 bool shape_from_cfg(const gpt2_config* c, Shape* s) {
   if (!c) return false;
   if (c->n_layer < 1 || c->d_model < 1 || c->n_head < 1 || c->n_ctx < 1 || c->vocab_real < 1 ||
-      c->vocab_padded < c->vocab_real || c->max_batch < 1 || (c->mode != 0 && c->mode != 1))
+      c->vocab_padded < c->vocab_real || c->max_batch < 1 || c->mode < 0 || c->mode > 2)
     return false;
   if (c->d_model % c->n_head) return false;
   s->L = c->n_layer; s->d = c->d_model; s->H = c->n_head; s->T = c->n_ctx;
-  s->V = c->vocab_padded; s->Vr = c->vocab_real; s->hd = c->d_model / c->n_head; s->mode = c->mode;
+  s->V = c->vocab_padded; s->Vr = c->vocab_real; s->hd = c->d_model / c->n_head;
+  s->mode = c->mode == 1 ? 1 : 0;
+  s->det = c->mode == 2;
   return true;
 }
 
@@ -74,6 +77,8 @@ int check_supported(const Shape& s, int max_batch) {
   if (s.hd != 16 && s.hd != 64) return GPT2_ERR_UNSUPPORTED_SHAPE;
   if (s.d > 2048) return GPT2_ERR_UNSUPPORTED_SHAPE;
   if (s.mode == 1 && s.T > 4096) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  // the fixed-order dQ sum is a mode of the tensor-core attention backward
+  if (s.det && (s.hd != 64 || s.T > 4096)) return GPT2_ERR_UNSUPPORTED_SHAPE;
   if ((long)max_batch * s.T > (1L << 30)) return GPT2_ERR_UNSUPPORTED_SHAPE;
   return GPT2_OK;
 }
@@ -109,6 +114,7 @@ struct Work {
   float *ce_pm, *ce_ps, *ce_zt, *ce_lse;
   void *dres, *dy, *du, *dqkv, *dout;
   float *dq_acc, *dvec;
+  float* dq_part;  // deterministic mode: per-key-block dQ tiles [T/128][M][d]
   float *norm_part, *gnorm;  // global gradient norm: block partials and the result
   int* n_valid;              // positions with a target in the last forward
   float* greedy_v;           // per-slice best (value, id) of the greedy choice
@@ -182,6 +188,7 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
   w->dqkv = c.take<void>(M * 3 * d * act);
   w->dout = c.take<void>(M * d * act);
   w->dq_acc = c.take<float>(M * d * 4);
+  w->dq_part = s.det ? c.take<float>((size_t)((s.T + 127) / 128) * M * d * 4) : nullptr;
   w->dvec = c.take<float>(M * s.H * 4);
   // per layer: two LayerNorms (gamma/beta partials + the column sums of their
   // output, the b_o / b_mp gradients) and the b_fc, b_qkv column sums; plus
@@ -481,7 +488,18 @@ int gpt2_forward_loss(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets
   return GPT2_OK;
 }
 
-int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The backward.  With events (L + 2 of them) the gradients are finished in
+// buckets and each bucket's event is recorded on the stream as soon as its
+// gradients are final: events[l] for layer l's block, events[L] for the final
+// LayerNorm, events[L + 1] for the token and position embeddings (the tied
+// wte gradient takes the embedding scatter last).  The block partials of the
+// bias and LayerNorm gradients are then reduced per bucket instead of in one
+// launch at the end.
+int backward_impl(gpt2_ctx* c, float grad_scale, int accumulate, void* const* events, void* stream) {
   if (!c) return GPT2_ERR_INVALID_ARG;
   if (!c->have_fwd) return GPT2_ERR_BAD_STATE;
   const Shape& s = c->s;
@@ -513,6 +531,17 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
   w.jobs.clear();
   // the new residual gradient's column sums are the last MLP projection's b_mp gradient
   TRY(ln_backward(c, w.x_final, w.meanf, w.rstdf, o.lnf_g(), 1, o.lnf_g(), o.layer(s.L - 1, B_MP), M, st));
+  // bucketed: reduce every pending job except the last (it belongs to the next
+  // bucket, the block below), then mark the bucket
+  size_t flushed = 0;
+  auto flush_bucket = [&](size_t keep, void* ev) -> int {
+    const size_t upto = w.jobs.size() - keep;
+    if (upto > flushed) TRY(reduce_rows_batch(w.jobs.data() + flushed, (int)(upto - flushed), beta, st));
+    flushed = upto;
+    if (ev) CUDA_TRY(cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev), st));
+    return GPT2_OK;
+  };
+  if (events) TRY(flush_bucket(1, events[s.L]));
 
   for (int l = (int)s.L - 1; l >= 0; --l) {
     LayerActs& a = w.layers[l];
@@ -551,7 +580,7 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
                        batch, (int)s.T, (int)s.H, (int)s.hd, st));
     else
       TRY(attn_bwd_bf16(a.qkv, a.o, a.lse, w.dout, w.dqkv, w.dq_acc, w.dvec, batch, (int)s.T, (int)s.H, (int)s.hd,
-                        st, fuse_d));
+                        st, fuse_d, w.dq_part));
     // QKV: qkv = y1 W_qkv^T + b_qkv
     g = make_gemm(M, d, 3 * d, w.dqkv, 0, 3 * d, Wp(c, o.layer(l, W_QKV)), 1, d, EPI_STORE, w.dy, d);
     TRY(run_gemm(c, g, st));
@@ -562,13 +591,35 @@ int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
     // column sums of the new residual gradient: the previous layer's b_mp gradient
     TRY(ln_backward(c, a.x_in, a.mean1, a.rstd1, o.layer(l, LN1_G), 0, o.layer(l, LN1_G),
                     l > 0 ? o.layer(l - 1, B_MP) : ~(size_t)0, M, st));
+    // layer l's gradients are final once its partials are reduced (the last
+    // job is layer l-1's b_mp)
+    if (events) TRY(flush_bucket(l > 0 ? 1 : 0, events[l]));
   }
-  // every bias and LayerNorm parameter gradient, in one launch
-  TRY(reduce_rows_batch(w.jobs.data(), (int)w.jobs.size(), beta, st));
+  // every (remaining) bias and LayerNorm parameter gradient, in one launch
+  if (w.jobs.size() > flushed)
+    TRY(reduce_rows_batch(w.jobs.data() + flushed, (int)(w.jobs.size() - flushed), beta, st));
   // x_0 = wte[tok] + wpe[t]
   TRY(embed_bwd(f32, w.tok, w.dres, G + o.wte(), G + o.wpe(), w.emb_acc, w.touched, M, (int)s.T, d, V, accumulate,
                 grad_scale, st));
+  if (events) CUDA_TRY(cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[s.L + 1]), st));
   return GPT2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gpt2_backward(gpt2_ctx* c, float grad_scale, int accumulate, void* stream) {
+  return backward_impl(c, grad_scale, accumulate, nullptr, stream);
+}
+
+int gpt2_backward_bucketed(gpt2_ctx* c, float grad_scale, int accumulate, void* const* events, int n_events,
+                           void* stream) {
+  if (!c || !events) return GPT2_ERR_INVALID_ARG;
+  if (n_events != (int)c->s.L + 2) return GPT2_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return GPT2_ERR_INVALID_ARG;
+  return backward_impl(c, grad_scale, accumulate, events, stream);
 }
 
 int gpt2_adamw_step(gpt2_ctx* c, float lr, float beta1, float beta2, float eps, float weight_decay, int step,

@@ -69,7 +69,7 @@ int attn_tc_set_wait_limit(unsigned long long ns);
 // dV into dqkv and reduces scale * dQ into dq_acc.
 int attn_fwd_tc(const void* qkv, void* o, float* lse, int B, int T, int H, cudaStream_t st);
 int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float* dvec, void* dqkv, float* dq_acc,
-                int B, int T, int H, cudaStream_t st);
+                int B, int T, int H, cudaStream_t st, float* dq_part = nullptr);
 
 // ---- attention ----------------------------------------------------------
 // qkv [B*T, 3*H*hd] (act), o [B*T, H*hd] (act), lse [B,H,T] fp32.
@@ -81,8 +81,12 @@ int attn_fwd_f32(const float* qkv, float* o, float* lse, int B, int T, int H, in
 // dvec_ready the caller has already written dvec = rowsum(dO * O) (head_dim 64:
 // the EPI_ROWDOT epilogue of the GEMM that produced dO) and zeroed dq_acc; the
 // call leaves dq_acc zeroed again for the next layer.
+// With dq_part (fp32 [ceil(T/128)][B*T][H*hd], head_dim 64, T <= 4096) every
+// key block's dQ tile is stored in its own slice and the slices are added in
+// key-block order: bitwise repeatable (dq_acc is then not used).
 int attn_bwd_bf16(const void* qkv, const void* o, const float* lse, const void* dout, void* dqkv,
-                  float* dq_acc, float* dvec, int B, int T, int H, int hd, cudaStream_t st, int dvec_ready = 0);
+                  float* dq_acc, float* dvec, int B, int T, int H, int hd, cudaStream_t st, int dvec_ready = 0,
+                  float* dq_part = nullptr);
 int attn_bwd_f32(const float* qkv, const float* o, const float* lse, const float* dout,
                  float* dqkv, float* dvec, int B, int T, int H, int hd, cudaStream_t st);
 

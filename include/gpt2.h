@@ -33,7 +33,13 @@
  *   asserts.
  * - Precision: mode 0 computes in bf16 on tensor cores with fp32 accumulation
  *   (activations bf16; master weights, gradients and AdamW state fp32); mode 1
- *   is a correctness mode that computes everything in fp32 on CUDA cores.
+ *   is a correctness mode that computes everything in fp32 on CUDA cores;
+ *   mode 2 is mode 0 made bitwise repeatable: the one reduction of mode 0
+ *   whose order varies from run to run (the attention backward's fp32 dQ sum
+ *   over key blocks) is done in key-block order from per-block partial tiles
+ *   (head_dim 64, n_ctx <= 4096; ceil(n_ctx/128) * max_batch * n_ctx * d more
+ *   fp32 of workspace; every other reduction of the step is already in a
+ *   fixed order).
  *
  * Flat parameter layout (fp32 master, fp32 grad, m, v and the bf16 shadow all
  * share it; offsets in elements):
@@ -79,7 +85,7 @@ typedef struct {
   int vocab_real;   /* ids must lie in [0, vocab_real) (50257 for GPT-2) */
   int vocab_padded; /* V >= vocab_real, a multiple of 128 (50304); the softmax spans all V */
   int max_batch;    /* largest batch any call will pass */
-  int mode;         /* 0 = bf16 tensor-core compute, 1 = fp32 correctness mode */
+  int mode;         /* 0 = bf16 tensor-core compute, 1 = fp32 correctness mode, 2 = mode 0, bitwise repeatable */
 } gpt2_config;
 
 typedef struct {
@@ -142,6 +148,21 @@ int gpt2_forward_loss(gpt2_ctx* ctx, const int32_t* tokens, const int32_t* targe
  * grad_scale = 1/k and accumulate = 0 on the first micro-batch, 1 after.
  * GPT2_ERR_BAD_STATE if no forward preceded it. */
 int gpt2_backward(gpt2_ctx* ctx, float grad_scale, int accumulate, void* stream);
+
+/* gpt2_backward that finishes the gradients in buckets, for a data-parallel
+ * exchange overlapped with the backward ("Pré-treinar um LLM", parallelism
+ * paragraph: the gradients are averaged over the data-parallel copies).
+ * events: n_events = n_layer + 2 CUDA events (cudaEvent_t) owned by the
+ * caller; each is recorded on `stream` as soon as its bucket's gradients are
+ * final: events[l] for decoder block l (its weights, biases and LayerNorm
+ * parameters, one contiguous range of the flat layout), events[n_layer] for
+ * the final LayerNorm, events[n_layer + 1] for wte and wpe (recorded last:
+ * the tied wte gradient takes the embedding scatter at the end).  The order
+ * of recording is n_layer, n_layer - 1, ..., 0, n_layer + 1.  The gradients
+ * equal gpt2_backward's.  GPT2_ERR_INVALID_ARG for a wrong event count or a
+ * NULL event. */
+int gpt2_backward_bucketed(gpt2_ctx* ctx, float grad_scale, int accumulate, void* const* events, int n_events,
+                           void* stream);
 
 /* One AdamW step over the whole flat buffer (decoupled weight decay on the
  * 2-D tensors only; bias-corrected with step counter `step` >= 1):

@@ -435,3 +435,43 @@ def test_other_config_shapes_one_layer(d, H, T):
     ref_g = backward(p32, oc, cache)
     assert abs(loss - ref_loss) <= 1e-2 * abs(ref_loss), (loss, ref_loss)
     compare_grads(gpu_grads(model, oc), ref_g, 0.999, 2e-2)
+
+
+def test_deterministic_mode_repeats_bitwise_and_matches_oracle():
+    """Mode 2 (bf16, attention dQ summed in key-block order): the same step
+    twice gives bitwise the same loss and gradients, and they match the
+    oracle within the bf16 tolerances."""
+    oc = HD64_L2
+    params = params_for(oc, seed=61)
+    tok, tgt = inputs.uniform_tokens(4, oc.n_ctx, oc.vocab, seed=62)
+    model = make_model(oc, oc.vocab, 4, 2)
+    p32 = load_params(model, params, oc)
+    losses, grads = [], []
+    for _ in range(2):
+        losses.append(run_step(model, tok, tgt))
+        grads.append(model.grad.clone())
+    assert losses[0] == losses[1]
+    assert torch.equal(grads[0], grads[1])
+    ref_loss, cache = forward(p32, oc, tok, tgt)
+    assert abs(losses[0] - ref_loss) <= 1e-2 * abs(ref_loss)
+    compare_grads(gpu_grads(model, oc), backward(p32, oc, cache), 0.999, 2e-2)
+
+
+@pytest.mark.slow
+def test_deterministic_mode_full_size_step_repeats_bitwise():
+    """The bench's workload (GPT-2 124M, 16 x 1024 Zipf tokens) in mode 2:
+    two identical steps give bitwise the same loss and every gradient."""
+    mc = gp.ModelConfig(12, 768, 12, 1024, 50257, 50304, 16, 2)
+    model = gp.GPT2(mc)
+    model.init_params(seed=0)
+    tok, tgt = inputs.zipf_tokens(16, 1024, seed=63)
+    tok_d, tgt_d = torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda()
+    out = []
+    for _ in range(2):
+        loss = model.forward_loss(tok_d, tgt_d)
+        model.backward(1.0, 0)
+        torch.cuda.synchronize()
+        assert model.status() == 0
+        out.append((float(loss.item()), model.grad.clone()))
+    assert out[0][0] == out[1][0]
+    assert torch.equal(out[0][1], out[1][1])

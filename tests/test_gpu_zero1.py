@@ -60,3 +60,44 @@ def test_range_arguments_are_checked():
         with pytest.raises(gp.Gpt2Error):
             model.adamw_step_range(1, off, cnt)
     model.adamw_step_range(1, n, 0)  # empty range at the end: nothing to do
+
+
+@pytest.mark.parametrize("accumulate", [0, 1])
+def test_bucketed_backward_equals_backward_and_orders_its_events(accumulate):
+    """gpt2_backward_bucketed: the same gradients as gpt2_backward (each bias
+    / LayerNorm reduction is the same fixed-order sum, only launched per
+    bucket; the attention backward's fp32 dQ reductions arrive in no fixed
+    order in either, hence a tolerance rather than bitwise equality), and each
+    bucket's event recorded in the stated order (final LayerNorm, blocks
+    L-1 .. 0, embeddings)."""
+    from decoder_only_transformer_step_b200 import dp, inputs
+    L = 3
+    mc = gp.ModelConfig(L, 128, 2, 128, 1000, 1024, 2, 0)
+    model = gp.GPT2(mc)
+    model.init_params(seed=8)
+    tok, tgt = inputs.uniform_tokens(2, 128, 1000, seed=9)
+    tok, tgt = torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda()
+    g0 = torch.randn(model.n_params, device="cuda") * 1e-3
+    model.grad.copy_(g0)
+    model.forward_loss(tok, tgt)
+    model.backward(1.0, accumulate)
+    want = model.grad.clone()
+    model.grad.copy_(g0)
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(L + 2)]
+    for ev in events:
+        ev.record()
+    start = torch.cuda.Event(enable_timing=True)
+    model.forward_loss(tok, tgt)
+    start.record()
+    model.backward_bucketed(events, 1.0, accumulate)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    diff = (model.grad - want).double()
+    assert diff.norm().item() <= 1e-4 * want.double().norm().item()
+    times = [start.elapsed_time(events[b]) for b in dp.completion_order(L)]
+    assert all(t >= 0 for t in times)
+    assert all(times[i] <= times[i + 1] for i in range(len(times) - 1)), times
+    # the buckets tile the flat layout
+    buckets = sorted(dp.gradient_buckets(gp.gpt2_tensors(mc.c()), L))
+    assert buckets[0][0] == 0 and buckets[-1][0] + buckets[-1][1] == model.n_params
+    assert all(buckets[i][0] + buckets[i][1] == buckets[i + 1][0] for i in range(len(buckets) - 1))
