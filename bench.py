@@ -20,6 +20,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -31,6 +32,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "train tokens/s, GPT-2 124M T=1024 bf16 on 1 B200; MFU (6N+attn FLOPs)"
 HBM_KERNELS = ("ln_fwd", "ln_bwd", "colsum", "adamw")
+# linear layers of a decoder block with their fused epilogues (gpt2_op_linear_bf16)
+LINEAR_KERNELS = ("qkv", "attn_proj", "fc", "mlp_proj")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 CONFIGS = {
@@ -507,7 +510,8 @@ def run_kernel(args):
     # HBM-bound kernels: inputs larger than the 126 MB L2 by default, so the
     # DRAM counters of a capture measure HBM traffic
     M = args.tokens or (131072 if args.kernel in ("ln_fwd", "ln_bwd") else 32768 if args.kernel == "colsum"
-                        else 16384 if args.kernel.startswith("lm_head_ce") else 4096)
+                        else 16384 if args.kernel.startswith("lm_head_ce") or args.kernel in LINEAR_KERNELS
+                        else 4096)
     g = torch.Generator(device="cuda").manual_seed(0)
     torch.cuda.synchronize()
     nbytes = 0
@@ -582,6 +586,18 @@ def run_kernel(args):
             dw = torch.empty(V, d, device="cuda")
             fn = lambda: gp.gpt2_op_lm_head_ce_bwd_bf16(A, W, M, V, d, 1.0, dx, dw, 0, scr)  # noqa: E731
             flop = 4.0 * M * V * d
+    elif args.kernel in LINEAR_KERNELS:
+        # one linear layer of a decoder block with its fused epilogue
+        N, K, act = {"qkv": (3 * d, d, 0), "attn_proj": (d, d, 1), "fc": (4 * d, d, 2),
+                     "mlp_proj": (d, 4 * d, 1)}[args.kernel]
+        A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+        W = (torch.randn(N, K, device="cuda", generator=g) / math.sqrt(K)).to(torch.bfloat16)
+        bias = (0.1 * torch.randn(N, device="cuda", generator=g)).to(torch.bfloat16)
+        R = torch.randn(M, N, device="cuda", generator=g).to(torch.bfloat16) if act == 1 else None
+        C = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        C2 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda") if act == 2 else None
+        fn = lambda: gp.gpt2_op_linear_bf16(A, W, bias, R, C, C2, M, N, K, act)  # noqa: E731
+        flop = 2.0 * M * N * K
     elif args.kernel == "lm_head":
         A = torch.randn(M, d, device="cuda", generator=g).to(torch.bfloat16)
         W = (0.02 * torch.randn(V, d, device="cuda", generator=g)).to(torch.bfloat16)
@@ -639,6 +655,7 @@ def relaunch_per_gpu(n):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", choices=["lm_head", "lm_head_ce", "lm_head_ce_bwd", "attn_fwd", "attn_bwd",
+                                         *LINEAR_KERNELS,
                                          "decode"] + list(HBM_KERNELS),
                     default=None, help="time one kernel alone instead of the step (profiler captures)")
     ap.add_argument("--tokens", type=int, default=None)

@@ -57,6 +57,7 @@ EXPORTS = [
     "gpt2_op_colsum_scratch_floats", "gpt2_op_colsum_bf16",
     "gpt2_op_lm_head_ce_scratch_bytes", "gpt2_op_lm_head_ce_fwd_bf16", "gpt2_op_lm_head_ce_bwd_bf16",
     "gpt2_set_wait_timeout_ns", "gpt2_op_gemm_bf16_status", "gpt2_backward_bucketed",
+    "gpt2_op_linear_bf16",
 ]
 
 _LIB = None
@@ -111,6 +112,7 @@ def _lib():
         "gpt2_set_wait_timeout_ns": (I, [U64]),
         "gpt2_backward_bucketed": (I, [P, F, I, P, I, P]),
         "gpt2_op_gemm_bf16_status": (I, [P, I, I, P, I, I, P, I, I, I, I, I, F, F, P, S, I, I, P, P]),
+        "gpt2_op_linear_bf16": (I, [P, P, P, P, P, P, I, I, I, I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -302,6 +304,12 @@ def gpt2_op_attention_bwd_bf16_noalloc(qkv, o, lse, dout, dqkv, B, T, H, hd, str
 def gpt2_op_layernorm_fwd_bf16(x, gamma, beta, y, mean, rstd, M, d, stream=None):
     _check(_lib().gpt2_op_layernorm_fwd_bf16(_ptr(x), _ptr(gamma), _ptr(beta), _ptr(y), _ptr(mean), _ptr(rstd),
                                              M, d, _stream(stream)), "gpt2_op_layernorm_fwd_bf16")
+
+
+def gpt2_op_linear_bf16(x, w, bias, resid, out, out2, M, N, K, act, stream=None):
+    """act 0: out = x w^T + bias; 1: + resid; 2: out = GELU(u), out2 = GELU'(u)."""
+    _check(_lib().gpt2_op_linear_bf16(_ptr(x), _ptr(w), _ptr(bias), _ptr(resid), _ptr(out), _ptr(out2), M, N, K,
+                                      act, _stream(stream)), "gpt2_op_linear_bf16")
 
 
 def gpt2_op_layernorm_bwd_scratch_floats(M, d) -> int:

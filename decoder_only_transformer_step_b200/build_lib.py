@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libgpt2.so")
-SOURCES = ["gemm_tc.cu", "gemm_simt.cu", "attention.cu", "attention_tc.cu", "attention_noalloc.cu", "kernels.cu",
+SOURCES = ["gemm_tc.cu", "gemm_tc_pair.cu", "gemm_tc_single.cu", "gemm_simt.cu", "attention.cu", "attention_tc.cu", "attention_noalloc.cu", "kernels.cu",
            "decode.cu", "gpt2.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

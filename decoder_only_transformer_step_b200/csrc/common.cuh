@@ -221,11 +221,6 @@ DEVI void tma_reduce_add_3d(const void* tmap, uint32_t src, int c0, int c1, int 
       "r"(src), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
-// Four consecutive floats added to global memory as one vector reduction
-// (16-byte aligned address).
-DEVI void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
-}
 DEVI void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 template <int N>
 DEVI void bulk_wait_read() {

@@ -851,6 +851,24 @@ int gpt2_op_gemm_bf16(const uint16_t* A, int a_mn_major, int lda, const uint16_t
   return gemm_tc_bf16(g, workspace, workspace_bytes, bn, splits, nullptr, S(stream));
 }
 
+int gpt2_op_linear_bf16(const uint16_t* x, const uint16_t* w, const uint16_t* bias, const uint16_t* resid,
+                        uint16_t* out, uint16_t* out2, int M, int N, int K, int act, void* stream) {
+  if (!x || !w || !bias || !out || M < 0 || N < 0 || K < 0 || act < 0 || act > 2) return GPT2_ERR_INVALID_ARG;
+  if ((act == 1 && !resid) || (act == 2 && !out2)) return GPT2_ERR_INVALID_ARG;
+  const uintptr_t al = (uintptr_t)x | (uintptr_t)w | (uintptr_t)bias | (uintptr_t)out |
+                       (act == 1 ? (uintptr_t)resid : 0) | (act == 2 ? (uintptr_t)out2 : 0);
+  if (al & 15) return GPT2_ERR_INVALID_ARG;
+  if (K % 64 || N % 8) return GPT2_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return GPT2_OK;
+  static const int kinds[3] = {EPI_BIAS, EPI_BIAS_RESID, EPI_BIAS_GELU};
+  // the GELU epilogue writes GELU'(u) to epi.out and GELU(u) to epi.out2
+  GemmArgs g = make_gemm(M, N, K, x, 0, K, w, 0, K, kinds[act], act == 2 ? (void*)out2 : (void*)out, N);
+  g.epi.bias = bias;
+  if (act == 1) g.epi.resid = resid;
+  if (act == 2) g.epi.out2 = out;
+  return gemm_tc_bf16(g, nullptr, 0, 0, 1, nullptr, S(stream));
+}
+
 int gpt2_set_wait_timeout_ns(uint64_t ns) {
   const unsigned long long v = ns ? (unsigned long long)ns : WAIT_TIMEOUT_NS;
   TRY(gemm_tc_set_wait_limit(v));

@@ -416,6 +416,25 @@ int gpt2_op_lm_head_ce_bwd_bf16(const uint16_t* x, const uint16_t* w, int M, int
                                 uint16_t* dx, float* dw, int accumulate, void* scratch, size_t scratch_bytes,
                                 void* stream);
 
+/* One linear layer of a decoder block with the epilogue the step fuses into
+ * its GEMM ("Criei GPT-2 do zero", model section: the QKV and attention
+ * output projections, the GELU(tanh) MLP and the residual stream;
+ * "Pré-treinar um LLM", compute section: one matmul of the forward):
+ *   act 0: out = x w^T + bias                       (QKV projection)
+ *   act 1: out = x w^T + bias + resid                (attention output / MLP proj)
+ *   act 2: u = x w^T + bias; out = GELU(u), out2 = GELU'(u)   (MLP fc; GELU'
+ *          is what the backward multiplies the incoming gradient by)
+ * GELU(u) = u/2 (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))).  Accumulation in
+ * fp32, every output rounded once to bf16.
+ * x bf16 [M, K] row-major, w bf16 [N, K] row-major (the layer's weight as
+ * stored), bias bf16 [N], resid / out / out2 bf16 [M, N] row-major; all
+ * 16-byte aligned.  resid is read only for act 1 and out2 written only for
+ * act 2 (both may be NULL otherwise).  K a multiple of 64, N of 8.  Errors:
+ * INVALID_ARG for NULL or misaligned buffers, a negative size or an act
+ * outside 0..2; UNSUPPORTED_SHAPE for K or N off those multiples. */
+int gpt2_op_linear_bf16(const uint16_t* x, const uint16_t* w, const uint16_t* bias, const uint16_t* resid,
+                        uint16_t* out, uint16_t* out2, int M, int N, int K, int act, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -176,3 +176,20 @@ def test_status_gemm_validates_on_host():
                                       None) == inv
     assert L.gpt2_op_gemm_bf16_status(p, 0, 64, p, 0, 64, p, 0, 64, 64, 64, 64, 1.0, 0.0, None, 0, 0, 0,
                                       ctypes.c_void_p(4098), None) == inv
+
+
+def test_linear_op_validates_on_host():
+    # argument and shape rules of the fused linear-layer op, decided on the
+    # host before any CUDA call
+    L = gp._lib()
+    p = ctypes.c_void_p(4096)
+    inv = gp.ERRORS_BY_NAME["GPT2_ERR_INVALID_ARG"]
+    uns = gp.ERRORS_BY_NAME["GPT2_ERR_UNSUPPORTED_SHAPE"]
+    assert L.gpt2_op_linear_bf16(p, p, p, None, p, None, 64, 64, 64, 3, None) == inv    # act out of range
+    assert L.gpt2_op_linear_bf16(p, p, p, None, p, None, 64, 64, 64, 1, None) == inv    # act 1 needs resid
+    assert L.gpt2_op_linear_bf16(p, p, p, None, p, None, 64, 64, 64, 2, None) == inv    # act 2 needs out2
+    assert L.gpt2_op_linear_bf16(p, p, p, None, ctypes.c_void_p(4104), None, 64, 64, 64, 0, None) == inv
+    assert L.gpt2_op_linear_bf16(p, p, None, None, p, None, 64, 64, 64, 0, None) == inv
+    assert L.gpt2_op_linear_bf16(p, p, p, None, p, None, 64, 64, 96, 0, None) == uns    # K % 64
+    assert L.gpt2_op_linear_bf16(p, p, p, None, p, None, 64, 60, 64, 0, None) == uns    # N % 8
+    assert L.gpt2_op_linear_bf16(p, p, p, None, p, None, 0, 64, 64, 0, None) == 0       # empty: nothing to do

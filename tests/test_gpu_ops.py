@@ -297,3 +297,35 @@ def test_lm_head_cross_entropy_ops_against_oracle(M, V, d, vocab_real):
         cos = float(a @ r / (np.linalg.norm(a) * np.linalg.norm(r)))
         rel = float(np.abs(a - r).max() / np.abs(r).max())
         assert cos >= 0.999 and rel <= 2e-2, (name, cos, rel)
+
+
+@pytest.mark.parametrize("act", [0, 1, 2])
+@pytest.mark.parametrize("M,N,K", [(300, 520, 192), (2048, 3072, 768)])
+def test_linear_op_fused_epilogues_against_oracle(act, M, N, K):
+    """One linear layer with the epilogue the forward fuses into its GEMM
+    (bias; bias + residual; bias + GELU with the saved GELU') against the
+    oracle's linear layer and GELU on the same bf16 inputs.  Ragged M and N
+    against the 256 x 256 tile in the small case; the MLP fc shape of GPT-2
+    small in the large one.  Each output is rounded once to bf16 from an fp32
+    accumulator: element-wise within 2^-7 of the value plus 4e-3 absolute
+    (the tanh of the GELU is the hardware approximation)."""
+    x = bf16_rand((M, K), 90 + M)
+    w = bf16_rand((N, K), 91 + N, scale=2.0 / math.sqrt(K))
+    bias = bf16_rand((N,), 92, scale=0.5)
+    resid = bf16_rand((M, N), 93 + M)
+    X, W, Bv, R = (t.double().numpy() for t in (x, w, bias, resid))
+    u = G.linear_fwd(X, W, Bv, None)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    out2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda") if act == 2 else None
+    gp.gpt2_op_linear_bf16(x.cuda(), w.cuda(), bias.cuda(), resid.cuda() if act == 1 else None, out, out2,
+                           M, N, K, act)
+    torch.cuda.synchronize()
+    if act == 0:
+        wants = [(out, u)]
+    elif act == 1:
+        wants = [(out, u + R)]
+    else:
+        wants = [(out, G.gelu_fwd(u)), (out2, G.gelu_bwd(np.ones_like(u), u))]
+    for got, want in wants:
+        err = np.abs(got.double().cpu().numpy() - want)
+        assert (err <= np.abs(want) / 128 + 4e-3).all(), (act, err.max())
