@@ -230,6 +230,9 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
       [[fallthrough]];
     case EPI_BIAS_RESID:
     case EPI_DGELU: {
+      // the optional column-sum partials are written as fp32 pairs
+      if (p.epi.kind == EPI_DGELU && g.epi.colsum && (((uintptr_t)g.epi.colsum & 7) || (g.N & 1)))
+        return GPT2_ERR_INVALID_ARG;
       // tmC2: the operand read per 64-column half (same [M, ldo] layout as the output)
       const void* opnd = p.epi.kind == EPI_BIAS_RESID ? g.epi.resid : g.epi.aux;
       if ((uintptr_t)opnd & 15) return GPT2_ERR_INVALID_ARG;

@@ -600,6 +600,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 dacc.x + dacc.y;
           }
         }
+        if constexpr (EK == EPI_DGELU) {
+          // bias gradient partials: lane l sums columns col0 + 2l, 2l + 1 of
+          // the staged (bf16) rows, the values the store writes
+          if (p.epi.colsum && row0 < p.M) {
+            __syncwarp();
+            float2 cs = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int rr = 0; rr < 32; ++rr) {
+              uint32_t wv;
+              asm volatile("ld.shared.b32 %0, [%1];"
+                           : "=r"(wv)
+                           : "r"(box + (uint32_t)rr * 128u + 16u * (uint32_t)((lane >> 2) ^ (rr & 7)) +
+                                 4u * (uint32_t)(lane & 3)));
+              cs = __fadd2_rn(cs, bf2(wv));
+            }
+            if (col0 + 2 * lane < p.N)
+              *reinterpret_cast<float2*>(p.epi.colsum + (long)(row0 >> 5) * p.N + col0 + 2 * lane) = cs;
+          }
+        }
         if (EK == EPI_F32 && p.store == ST_REG) continue;
         fence_proxy_async_smem();
         __syncwarp();

@@ -6,6 +6,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <vector>
 
@@ -194,8 +195,10 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
   // output, the b_o / b_mp gradients) and the b_fc, b_qkv column sums; plus
   // the final LayerNorm
   const size_t ln_rows = layernorm_bwd_part_rows((int)M);
-  w->part_floats = (size_t)s.L * (2 * ln_rows * 3 * d + colsum_part_floats((int)M, (int)(4 * d)) +
-                                   colsum_part_floats((int)M, (int)(3 * d))) +
+  // (the b_fc sums come from the GELU' GEMM's epilogue, one row per 32 tokens,
+  // on the tensor-core path)
+  const size_t fc_part = std::max(colsum_part_floats((int)M, (int)(4 * d)), (size_t)((M + 31) / 32) * 4 * d);
+  w->part_floats = (size_t)s.L * (2 * ln_rows * 3 * d + fc_part + colsum_part_floats((int)M, (int)(3 * d))) +
                    ln_rows * 3 * d;
   w->part_arena = c.take<float>(w->part_floats * 4);
   w->norm_part = c.take<float>((size_t)GRAD_NORM_PARTS * 4);
@@ -548,6 +551,9 @@ int backward_impl(gpt2_ctx* c, float grad_scale, int accumulate, void* const* ev
     // MLP projection: x_out = x_mid + g W_mp^T + b_mp
     g = make_gemm(M, 4 * d, d, w.dres, 0, d, Wp(c, o.layer(l, W_MP)), 1, 4 * d, EPI_DGELU, w.du, 4 * d);
     g.epi.aux = a.gp;
+    // b_fc gradient partials (column sums of du per 32 rows) from the same epilogue
+    float* fc_part = f32 ? nullptr : part_slot(c, (size_t)((M + 31) / 32) * 4 * d);
+    g.epi.colsum = fc_part;
     TRY(run_gemm(c, g, st));
     g = make_gemm(d, 4 * d, M, w.dres, 1, d, a.g, 1, 4 * d, EPI_F32, G + o.layer(l, W_MP), 4 * d);
     g.epi.beta = beta;
@@ -558,7 +564,10 @@ int backward_impl(gpt2_ctx* c, float grad_scale, int accumulate, void* const* ev
     g = make_gemm(4 * d, d, M, w.du, 1, 4 * d, a.y2, 1, d, EPI_F32, G + o.layer(l, W_FC), d);
     g.epi.beta = beta;
     TRY(run_gemm(c, g, st));
-    TRY(bias_grad(c, w.du, M, 4 * d, o.layer(l, B_FC), st));
+    if (fc_part)
+      w.jobs.push_back(ReduceJob{fc_part, G + o.layer(l, B_FC), (M + 31) / 32, 4 * d});
+    else
+      TRY(bias_grad(c, w.du, M, 4 * d, o.layer(l, B_FC), st));
     // column sums of the new residual gradient: the attention projection's b_o gradient
     TRY(ln_backward(c, a.x_mid, a.mean2, a.rstd2, o.layer(l, LN2_G), 0, o.layer(l, LN2_G), o.layer(l, B_O), M, st));
     // attention projection: x_mid = x_in + o W_o^T + b_o

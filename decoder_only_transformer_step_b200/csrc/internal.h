@@ -12,7 +12,8 @@ enum EpiKind : int {
   EPI_BIAS,         // out(act)  = acc + bias[n]
   EPI_BIAS_RESID,   // out(act)  = acc + bias[n] + resid[m,n]
   EPI_BIAS_GELU,    // u = acc + bias[n]: out(act) = gelu'(u), out2(act) = gelu(u)
-  EPI_DGELU,        // out(act)  = acc * aux[m,n]  (aux = the saved gelu'(u))
+  EPI_DGELU,        // out(act)  = acc * aux[m,n]  (aux = the saved gelu'(u)); optionally
+                    //   colsum[m/32][n] = sum of out over rows 32 (m/32) .. 32 (m/32) + 31
   EPI_F32,          // out(fp32) = beta * out + alpha * acc
   EPI_F32_PARTIAL,  // partial[split][m,n] = acc (split-K, internal)
   EPI_ROWDOT,       // out(bf16) = acc; out2(fp32)[(m / seq * N/64 + n/64) * seq + m % seq] =
@@ -33,6 +34,8 @@ struct EpiArgs {
   long ldo;
   float alpha, beta;
   int seq;            // EPI_ROWDOT: rows per sequence
+  float* colsum;      // EPI_DGELU, optional: [ceil(M/32), N] fp32 sums of the stored (bf16)
+                      //   output over each 32-row group (the bias gradient's partials)
   // EPI_CE_FWD
   float* ce_max;
   float* ce_sum;
