@@ -48,6 +48,23 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
   }
 }
 
+// bf16 out = alpha * sum_s part[s]   (fixed order over s; mn a multiple of 4)
+__global__ void splitk_reduce_bf16_kernel(const float* __restrict__ part, int splits, long mn,
+                                          bf16* __restrict__ out, float alpha) {
+  pdl_start();
+  const long i = (blockIdx.x * (long)blockDim.x + threadIdx.x) * 4;
+  if (i >= mn) return;
+  float4 acc = reinterpret_cast<const float4*>(part + i)[0];
+  for (int s = 1; s < splits; ++s) {
+    const float4 t = reinterpret_cast<const float4*>(part + (long)s * mn + i)[0];
+    acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
+  }
+  uint2 o;
+  o.x = pack_bf16x2(alpha * acc.x, alpha * acc.y);
+  o.y = pack_bf16x2(alpha * acc.z, alpha * acc.w);
+  *reinterpret_cast<uint2*>(out + i) = o;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -178,7 +195,10 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   if (splits == 0) splits = g.epi.kind == EPI_F32 ? auto_splits(g.M, g.N, g.K, bn) : 1;
   if (splits > kb_total) splits = kb_total;
   if (splits > 1) {
-    if (g.epi.kind != EPI_F32 || g.N % 4 || g.epi.ldo != g.N) return GPT2_ERR_INVALID_ARG;
+    // fp32 (weight-gradient) outputs, or a plain bf16 store: partial sums in
+    // the workspace, then a fixed-order reduction
+    if ((g.epi.kind != EPI_F32 && g.epi.kind != EPI_STORE) || g.N % 4 || g.epi.ldo != g.N)
+      return GPT2_ERR_INVALID_ARG;
     size_t need = (size_t)splits * g.M * g.N * sizeof(float);
     if (!ws || ws_bytes < need) splits = 1;
   }
@@ -197,6 +217,8 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   p.m_tiles = (g.M + p.tile_m - 1) / p.tile_m;
   p.n_tiles = (g.N + n_mma - 1) / n_mma;
   p.splits = splits;
+  // the larger operand's tiles are the ones the concurrent units share
+  p.n_fast = g.M > g.N ? 1 : 0;
   p.kb_total = kb_total;
   // instruction descriptor, kind::f16: D fp32 (bit 4), A and B bf16 (bits 7, 10),
   // operand majorness (bits 15, 16), N >> 3 at bit 17, M >> 4 at bit 24 (M = 256
@@ -296,8 +318,12 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   if (splits > 1) {
     long mn = (long)g.M * g.N;
     long threads = (mn + 3) / 4;
-    CUDA_TRY(launch_k(splitk_reduce_kernel, (unsigned)((threads + 255) / 256), 256, 0, st, 
-        (const float*)ws, splits, mn, (float*)g.epi.out, g.epi.alpha, g.epi.beta));
+    if (g.epi.kind == EPI_STORE)
+      CUDA_TRY(launch_k(splitk_reduce_bf16_kernel, (unsigned)((threads + 255) / 256), 256, 0, st,
+                        (const float*)ws, splits, mn, (bf16*)g.epi.out, g.epi.alpha));
+    else
+      CUDA_TRY(launch_k(splitk_reduce_kernel, (unsigned)((threads + 255) / 256), 256, 0, st,
+                        (const float*)ws, splits, mn, (float*)g.epi.out, g.epi.alpha, g.epi.beta));
     LAUNCH_CHECK();
   }
   return GPT2_OK;

@@ -97,6 +97,7 @@ struct TcParams {
   int a_mn, b_mn;
   int m_tiles, n_tiles, splits, kb_total;
   int tile_m;  // output rows per work unit (128, or 256 for a CTA pair)
+  int n_fast;  // unit order: n varies fastest (1) or m (0)
   uint32_t idesc;
   int store;
   EpiArgs epi;
@@ -124,12 +125,16 @@ DEVI uint64_t operand_desc(uint32_t tile, int mn_major, int k) {
 }
 
 // Work unit u -> (m tile origin, n tile index, split index, k-block range).
-// m varies fastest, so consecutive CTAs share the B tile (weights) in L2.
+// The units running at one time share the tiles of the larger operand: with
+// m fastest, consecutive CTAs load the same B tile and the smaller A is
+// re-read from L2; with n fastest the roles swap.  The split index varies
+// slowest.
 DEVI void decode_unit(const TcParams& p, int u, int& m0, int& nt, int& s, int& kb0, int& kb1) {
-  const int mt = u % p.m_tiles;
-  const int rest = u / p.m_tiles;
-  nt = rest % p.n_tiles;
-  s = rest / p.n_tiles;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int t = u % tiles;
+  s = u / tiles;
+  const int mt = p.n_fast ? t / p.n_tiles : t % p.m_tiles;
+  nt = p.n_fast ? t % p.n_tiles : t / p.m_tiles;
   m0 = mt * p.tile_m;
   kb0 = (int)((long long)s * p.kb_total / p.splits);
   kb1 = (int)((long long)(s + 1) * p.kb_total / p.splits);
@@ -341,6 +346,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int it = 0;
       bool ok = true;
       bool issued_any = false;
+      // Descriptors of stage 0, k-slice 0; the start-address field (bits
+      // 0..13, address >> 4) of the others is an add away: every shared-memory
+      // address is below 2^18, so the field never carries into the next one.
+      const uint64_t a_desc0 = operand_desc(tiles, p.a_mn, 0);
+      const uint64_t b_desc0 = operand_desc(tiles + C::A_BYTES, p.b_mn, 0);
+      const uint32_t a_kstep = p.a_mn ? 2048u >> 4 : 32u >> 4;
+      const uint32_t b_kstep = p.b_mn ? 2048u >> 4 : 32u >> 4;
       for (int u = unit0; u < units && ok; u += unit_step, ++it) {
         int m0, nt, s, kb0, kb1;
         decode_unit(p, u, m0, nt, s, kb0, kb1);
@@ -360,11 +372,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = tiles + stage * C::STAGE_BYTES;
-          const uint32_t sb = sa + C::A_BYTES;
+          const uint32_t soff = (uint32_t)stage * (C::STAGE_BYTES >> 4);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = operand_desc(sa, p.a_mn, k), bd = operand_desc(sb, p.b_mn, k);
+            const uint64_t ad = a_desc0 + (soff + k * a_kstep), bd = b_desc0 + (soff + k * b_kstep);
             const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
             if constexpr (PAIR)
               tc_mma_bf16_pair(d_tmem, ad, bd, p.idesc, acc);

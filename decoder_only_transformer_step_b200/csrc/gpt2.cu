@@ -131,6 +131,11 @@ struct Work {
   uint8_t* touched;
 };
 
+// The LM head's input-gradient GEMM (M x d, K = V) has only M/256 * d/256
+// output tiles (192 at the 124M shape) for 74 SM pairs, 2.6 waves; three
+// K splits make 7.8 waves of a third of the work each.
+constexpr int LM_DGRAD_SPLITS = 3;
+
 size_t split_ws_need(const Shape& s, long M) {
   if (s.mode != 0) return 0;
   size_t need = 0;
@@ -140,7 +145,9 @@ size_t split_ws_need(const Shape& s, long M) {
     size_t b = gemm_tc_split_bytes((int)sh[0], (int)sh[1], (int)M);
     if (b > need) need = b;
   }
-  return need;
+  // the LM head's input gradient, split along the vocabulary
+  const size_t lm = (size_t)LM_DGRAD_SPLITS * M * d * sizeof(float);
+  return need > lm ? need : lm;
 }
 
 size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
@@ -525,7 +532,10 @@ int backward_impl(gpt2_ctx* c, float grad_scale, int accumulate, void* const* ev
   // (softmax - onehot) M / n_valid left in w.logits by the forward
   GemmArgs g = make_gemm(M, d, V, w.logits, 0, V, Wp(c, o.wte()), 1, d, EPI_STORE, w.dy, d);
   g.epi.alpha = sc;
-  TRY(run_gemm(c, g, st));
+  if (f32)
+    TRY(run_gemm(c, g, st));
+  else
+    TRY(gemm_tc_bf16(g, w.split_ws, w.split_bytes, 0, LM_DGRAD_SPLITS, w.err, st));
   g = make_gemm(V, d, M, w.logits, 1, V, w.yf, 1, d, EPI_F32, G + o.wte(), d);
   g.epi.alpha = sc;
   g.epi.beta = beta;
