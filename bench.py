@@ -170,12 +170,30 @@ def run_ours(args, rank, world, local_rank):
         exchange.optimizer_step(model.master, lambda off, cnt: model.adamw_step_range(step_no, off, cnt),
                                 model.refresh_shadow)
 
+    # one GPU: forward + loss + backward replayed as one CUDA graph per step
+    # (gpt2_graph_capture / gpt2_graph_step: the same kernels without the gaps
+    # between ~300 separate launches); the ids are copied into the graph's
+    # input buffers each step and AdamW runs after it with the step's number.
+    # Several GPUs: the eager backward, which records the per-bucket events the
+    # overlapped exchange waits on.
+    use_graph = world == 1 and not args.eager
+
     def step(i):
         tok, tgt = pool[i % len(pool)]
-        model.forward_loss(tok, tgt)
-        backward(1.0, 0, True)
+        if use_graph:
+            model.graph_step(tok, tgt)
+        else:
+            model.forward_loss(tok, tgt)
+            backward(1.0, 0, True)
         optimizer_step(i + 1)
 
+    if use_graph:
+        # one eager step sets every kernel up, then the capture
+        tok, tgt = pool[0]
+        model.forward_loss(tok, tgt)
+        model.backward(1.0, 0)
+        torch.cuda.synchronize()
+        model.graph_capture(B)
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -248,11 +266,21 @@ def run_ours(args, rank, world, local_rank):
     if args.accum > 1:
         k = args.accum
 
+        if use_graph:
+            # the accumulating micro-step as the graph: gradients zeroed once per
+            # optimizer step, then k micro-steps that add into them
+            model.graph_capture(B, grad_scale=1.0 / k, accumulate=1)
+
         def accum_step(i):
+            if use_graph:
+                model.zero_grad()
             for j in range(k):
                 tok, tgt = pool[(i * k + j) % len(pool)]
-                model.forward_loss(tok, tgt)
-                backward(1.0 / k, 1 if j else 0, j == k - 1)
+                if use_graph:
+                    model.graph_step(tok, tgt)
+                else:
+                    model.forward_loss(tok, tgt)
+                    backward(1.0 / k, 1 if j else 0, j == k - 1)
             optimizer_step(args.warmup + args.steps + e_steps + 2 + i)
 
         a_steps = 2
@@ -297,7 +325,9 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic Zipf(1.1) token ids over [0, 50257), random-init GPT-2 weights",
         "config": {"workload": workload_name(args.config, CONFIGS[args.config]), "batch_per_gpu": B,
                    "seq_len": T, "parallelism": f"dp{world}" + ("-zero1" if world > 1 and args.zero1 else ""),
-                   "l2": "inputs larger than L2: the step's working set (>5 GB) exceeds the 126 MB L2"},
+                   "l2": "inputs larger than L2: the step's working set (>5 GB) exceeds the 126 MB L2",
+                   "launch": "one CUDA graph per step (forward, loss, backward) + AdamW" if use_graph
+                   else "eager launches"},
         "mfu": round(flops.mfu(tokens_per_s / world, fpt, peaks["bf16_tflops"] * 1e12), 4),
         "mfu_vs_sustained": round(flops.mfu(tokens_per_s / world, fpt, peaks["bf16_tflops_sustained"] * 1e12), 4),
         "mfu_vs_datasheet": round(flops.mfu(tokens_per_s / world, fpt, 2250e12), 4),
@@ -665,6 +695,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="124m", choices=sorted(CONFIGS))
+    ap.add_argument("--eager", action="store_true",
+                    help="issue the step's kernels one by one instead of replaying the captured CUDA graph")
     ap.add_argument("--accum", type=int, default=32,
                     help="also time optimizer steps with this many accumulated micro-batches (0 or 1: skip)")
     ap.add_argument("--decode-steps", type=int, default=64,

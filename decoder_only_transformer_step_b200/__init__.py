@@ -57,7 +57,7 @@ EXPORTS = [
     "gpt2_op_colsum_scratch_floats", "gpt2_op_colsum_bf16",
     "gpt2_op_lm_head_ce_scratch_bytes", "gpt2_op_lm_head_ce_fwd_bf16", "gpt2_op_lm_head_ce_bwd_bf16",
     "gpt2_set_wait_timeout_ns", "gpt2_op_gemm_bf16_status", "gpt2_backward_bucketed",
-    "gpt2_op_linear_bf16",
+    "gpt2_op_linear_bf16", "gpt2_graph_capture", "gpt2_graph_step", "gpt2_graph_release",
 ]
 
 _LIB = None
@@ -113,6 +113,9 @@ def _lib():
         "gpt2_backward_bucketed": (I, [P, F, I, P, I, P]),
         "gpt2_op_gemm_bf16_status": (I, [P, I, I, P, I, I, P, I, I, I, I, I, F, F, P, S, I, I, P, P]),
         "gpt2_op_linear_bf16": (I, [P, P, P, P, P, P, I, I, I, I, P]),
+        "gpt2_graph_capture": (I, [P, I, F, I, P, P]),
+        "gpt2_graph_step": (I, [P, P, P, P]),
+        "gpt2_graph_release": (I, [P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -208,6 +211,21 @@ def gpt2_backward_bucketed(ctx, grad_scale, accumulate, events, stream=None):
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _check(_lib().gpt2_backward_bucketed(ctx, grad_scale, accumulate, arr, len(events), _stream(stream)),
            "gpt2_backward_bucketed")
+
+
+def gpt2_graph_capture(ctx, batch, grad_scale, accumulate, loss_dev, stream):
+    """Records forward + loss + backward into the context's graph; `stream` is
+    a torch.cuda.Stream the caller created (not the default stream)."""
+    _check(_lib().gpt2_graph_capture(ctx, batch, grad_scale, accumulate, _ptr(loss_dev), _stream(stream)),
+           "gpt2_graph_capture")
+
+
+def gpt2_graph_step(ctx, tokens, targets, stream=None):
+    _check(_lib().gpt2_graph_step(ctx, _ptr(tokens), _ptr(targets), _stream(stream)), "gpt2_graph_step")
+
+
+def gpt2_graph_release(ctx):
+    _check(_lib().gpt2_graph_release(ctx), "gpt2_graph_release")
 
 
 def gpt2_adamw_step(ctx, lr, beta1, beta2, eps, weight_decay, step, stream=None):
@@ -438,6 +456,21 @@ class GPT2:
 
     def backward(self, grad_scale=1.0, accumulate=0):
         gpt2_backward(self.ctx, grad_scale, accumulate)
+
+    def graph_capture(self, batch, grad_scale=1.0, accumulate=0, stream=None):
+        """Record forward + loss + backward of one micro-batch into the
+        context's CUDA graph (after at least one eager step).  The capture runs
+        on a side stream of its own unless one is given."""
+        import torch
+        s = stream if stream is not None else torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        gpt2_graph_capture(self.ctx, batch, grad_scale, accumulate, self.loss, s)
+        torch.cuda.current_stream().wait_stream(s)
+
+    def graph_step(self, tokens, targets):
+        """One captured micro-step on the current stream: the ids are copied in,
+        then the graph runs (as forward_loss + backward)."""
+        gpt2_graph_step(self.ctx, tokens, targets)
 
     def backward_bucketed(self, events, grad_scale=1.0, accumulate=0):
         """The backward recording events[i] when bucket i's gradients are

@@ -107,6 +107,7 @@ struct Work {
   int* err;
   float* loss;
   int32_t *tok, *tgt, *tok_stage, *tgt_stage;
+  int32_t *gtok, *gtgt;  // inputs of the captured step
   std::vector<LayerActs> layers;
   void *x_final, *yf, *logits;
   float *meanf, *rstdf, *loss_rows;
@@ -158,6 +159,9 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
   w->loss = c.take<float>(sizeof(float));
   w->tok = c.take<int32_t>(M * 4);
   w->tgt = c.take<int32_t>(M * 4);
+  // the captured step's inputs (copied in by gpt2_graph_step)
+  w->gtok = c.take<int32_t>(M * 4);
+  w->gtgt = c.take<int32_t>(M * 4);
   w->tok_stage = c.take<int32_t>(M * 4);
   w->tgt_stage = c.take<int32_t>(M * 4);
   w->layers.assign(s.L, LayerActs{});
@@ -234,6 +238,15 @@ struct gpt2_ctx {
   Work w;
   int have_fwd = 0;
   int fwd_batch = 0;
+  // the captured micro-step (gpt2_graph_capture)
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t graph_exec = nullptr;
+  int graph_batch = 0;
+  unsigned long long graph_launches = 0;  // kernels in one launch of the graph
+  ~gpt2_ctx() {
+    if (graph_exec) cudaGraphExecDestroy(graph_exec);
+    if (graph) cudaGraphDestroy(graph);
+  }
 };
 
 namespace {
@@ -841,6 +854,66 @@ int gpt2_step_host(gpt2_ctx* c, const int32_t* tokens_host, const int32_t* targe
 }
 
 uint64_t gpt2_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int gpt2_graph_release(gpt2_ctx* c) {
+  if (!c) return GPT2_ERR_INVALID_ARG;
+  if (c->graph_exec) CUDA_TRY(cudaGraphExecDestroy(c->graph_exec));
+  if (c->graph) CUDA_TRY(cudaGraphDestroy(c->graph));
+  c->graph_exec = nullptr;
+  c->graph = nullptr;
+  c->graph_batch = 0;
+  c->graph_launches = 0;
+  return GPT2_OK;
+}
+
+int gpt2_graph_capture(gpt2_ctx* c, int batch, float grad_scale, int accumulate, float* loss_dev, void* stream) {
+  if (!c || !stream) return GPT2_ERR_INVALID_ARG;
+  if (batch < 1 || batch > c->cfg.max_batch) return GPT2_ERR_INVALID_ARG;
+  TRY(gpt2_graph_release(c));
+  cudaStream_t st = S(stream);
+  const unsigned long long l0 = g_launches.load(std::memory_order_relaxed);
+  CUDA_TRY(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+  // the recorded forward reads the graph's own input buffers
+  int rc = gpt2_forward_loss(c, c->w.gtok, c->w.gtgt, batch, loss_dev, stream);
+  if (rc == GPT2_OK) rc = backward_impl(c, grad_scale, accumulate, nullptr, stream);
+  cudaGraph_t g = nullptr;
+  const cudaError_t ec = cudaStreamEndCapture(st, &g);
+  const unsigned long long n = g_launches.load(std::memory_order_relaxed) - l0;
+  // the capture launched nothing: take its kernels back out of the count
+  g_launches.fetch_sub(n, std::memory_order_relaxed);
+  c->have_fwd = 0;
+  if (rc != GPT2_OK || ec != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+    return rc != GPT2_OK ? rc : GPT2_ERR_CUDA;
+  }
+  cudaGraphExec_t ex = nullptr;
+  if (cudaGraphInstantiate(&ex, g, 0) != cudaSuccess) {
+    cudaGraphDestroy(g);
+    cudaGetLastError();
+    return GPT2_ERR_CUDA;
+  }
+  c->graph = g;
+  c->graph_exec = ex;
+  c->graph_batch = batch;
+  c->graph_launches = n;
+  return GPT2_OK;
+}
+
+int gpt2_graph_step(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets, void* stream) {
+  if (!c || !tokens || !targets) return GPT2_ERR_INVALID_ARG;
+  if (!c->graph_exec) return GPT2_ERR_BAD_STATE;
+  cudaStream_t st = S(stream);
+  const size_t bytes = (size_t)c->graph_batch * c->s.T * 4;
+  CUDA_TRY(cudaMemcpyAsync(c->w.gtok, tokens, bytes, cudaMemcpyDeviceToDevice, st));
+  CUDA_TRY(cudaMemcpyAsync(c->w.gtgt, targets, bytes, cudaMemcpyDeviceToDevice, st));
+  CUDA_TRY(cudaGraphLaunch(c->graph_exec, st));
+  g_launches.fetch_add(c->graph_launches, std::memory_order_relaxed);
+  // as after gpt2_forward_loss + gpt2_backward
+  c->have_fwd = 1;
+  c->fwd_batch = c->graph_batch;
+  return GPT2_OK;
+}
 
 const char* gpt2_strerror(int code) {
   switch (code) {

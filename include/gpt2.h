@@ -416,6 +416,30 @@ int gpt2_op_lm_head_ce_bwd_bf16(const uint16_t* x, const uint16_t* w, int M, int
                                 uint16_t* dx, float* dw, int accumulate, void* scratch, size_t scratch_bytes,
                                 void* stream);
 
+/* ------------------------------------------------------------------------
+ * The micro-step as a CUDA graph.  A step launches about 300 kernels; issued
+ * one by one, the gaps between them cost about 3 % of the step.
+ * gpt2_graph_capture records the forward, the loss and the backward of one
+ * micro-batch of `batch` rows (grad_scale and accumulate as in gpt2_backward,
+ * fixed by the capture; the loss written to loss_dev, a device float, or to
+ * the context's own loss word when NULL) into a graph the context owns,
+ * replacing an earlier one.  It computes nothing: the kernels are recorded on
+ * `stream`, which must be a stream the caller created (not the legacy default
+ * stream), and every kernel must have been run once on the device before (one
+ * eager step), since their one-time set-up cannot happen inside a capture.
+ * gpt2_graph_step copies the step's token and target ids (device int32
+ * [batch, n_ctx]) into the graph's own input buffers and launches the graph on
+ * `stream`: the same kernels and the same results as gpt2_forward_loss and
+ * gpt2_backward with those arguments.  gpt2_adamw_step (or its variants)
+ * follows as usual.  The graph's kernels count in gpt2_kernel_launches at each
+ * launch.  Errors: INVALID_ARG for a NULL context or stream, or a batch outside
+ * [1, max_batch]; BAD_STATE for gpt2_graph_step without a graph; CUDA if the
+ * capture fails (no graph is kept).  gpt2_graph_release frees the graph
+ * (gpt2_destroy does too). */
+int gpt2_graph_capture(gpt2_ctx* ctx, int batch, float grad_scale, int accumulate, float* loss_dev, void* stream);
+int gpt2_graph_step(gpt2_ctx* ctx, const int32_t* tokens, const int32_t* targets, void* stream);
+int gpt2_graph_release(gpt2_ctx* ctx);
+
 /* One linear layer of a decoder block with the epilogue the step fuses into
  * its GEMM ("Criei GPT-2 do zero", model section: the QKV and attention
  * output projections, the GELU(tanh) MLP and the residual stream;
