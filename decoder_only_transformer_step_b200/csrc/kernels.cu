@@ -7,6 +7,8 @@
 // reductions use warp shuffles; every cross-row reduction is a fixed-order
 // two-level sum (per-block partials, then a column reduction), so repeated
 // runs give bitwise-identical results.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -194,6 +196,96 @@ __global__ void ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ g, 
   if (lane == 0) {
     mean[m] = mu;
     rstd[m] = rs;
+  }
+}
+
+// bf16 rows: the same normalisation with the arithmetic on fp32 pairs
+// (mean, the centred sum of squares, y = (x rstd - mean rstd) g + b as two
+// packed multiply-adds), ROWS rows per warp so gamma and beta are unpacked
+// once, and the next row's load in flight while one is normalised.
+DEVI float2 bf2w(uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); }
+
+template <int NC, int ROWS>
+__global__ void __launch_bounds__(256) ln_fwd_bf16_kernel(const bf16* __restrict__ x, const bf16* __restrict__ g,
+                                                          const bf16* __restrict__ b, bf16* __restrict__ y,
+                                                          float* __restrict__ mean, float* __restrict__ rstd,
+                                                          int M, int d) {
+  pdl_start();
+  const int lane = threadIdx.x & 31;
+  const int m0 = (blockIdx.x * 8 + (threadIdx.x >> 5)) * ROWS;
+  if (m0 >= M) return;
+  float2 gg[NC][4], bb[NC][4];
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    const int c = (lane + 32 * k) * 8;
+    uint4 ug = make_uint4(0, 0, 0, 0), ub = make_uint4(0, 0, 0, 0);
+    if (c < d) {
+      ug = __ldg(reinterpret_cast<const uint4*>(g + c));
+      ub = __ldg(reinterpret_cast<const uint4*>(b + c));
+    }
+    gg[k][0] = bf2w(ug.x); gg[k][1] = bf2w(ug.y); gg[k][2] = bf2w(ug.z); gg[k][3] = bf2w(ug.w);
+    bb[k][0] = bf2w(ub.x); bb[k][1] = bf2w(ub.y); bb[k][2] = bf2w(ub.z); bb[k][3] = bf2w(ub.w);
+  }
+  const float inv_d = 1.f / (float)d;
+  auto load = [&](int m, uint4 (&u)[NC]) {
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = (lane + 32 * k) * 8;
+      u[k] = c < d ? *reinterpret_cast<const uint4*>(x + (long)m * d + c) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  uint4 cur[NC];
+  load(m0, cur);
+#pragma unroll 1
+  for (int r = 0; r < ROWS; ++r) {
+    const int m = m0 + r;
+    if (m >= M) break;
+    uint4 nxt[NC];
+    if (r + 1 < ROWS && m + 1 < M) load(m + 1, nxt);
+    float2 v[NC][4];
+    float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      v[k][0] = bf2w(cur[k].x); v[k][1] = bf2w(cur[k].y); v[k][2] = bf2w(cur[k].z); v[k][3] = bf2w(cur[k].w);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s2 = __fadd2_rn(s2, v[k][j]);
+    }
+    const float mu = warp_sum(s2.x + s2.y) * inv_d;
+    const float2 nmu2 = make_float2(-mu, -mu);
+    float2 q2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = (lane + 32 * k) * 8;
+      if (c < d) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 t = __fadd2_rn(v[k][j], nmu2);
+          q2 = __ffma2_rn(t, t, q2);
+        }
+      }
+    }
+    const float rs = rsqrtf(warp_sum(q2.x + q2.y) * inv_d + 1e-5f);
+    const float2 rs2 = make_float2(rs, rs), c2 = make_float2(-mu * rs, -mu * rs);
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = (lane + 32 * k) * 8;
+      if (c < d) {
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 xh = __ffma2_rn(v[k][j], rs2, c2);
+          const float2 o = __ffma2_rn(xh, gg[k][j], bb[k][j]);
+          w[j] = pack_bf16x2(o.x, o.y);
+        }
+        *reinterpret_cast<uint4*>(y + (long)m * d + c) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    if (lane == 0) {
+      mean[m] = mu;
+      rstd[m] = rs;
+    }
+#pragma unroll
+    for (int k = 0; k < NC; ++k) cur[k] = nxt[k];
   }
 }
 
@@ -415,6 +507,136 @@ __global__ void __launch_bounds__(32 * LNF_WARPS, LNF_BLOCKS_PER_SM)
         red[(warp * NQ + 0) * d + c + j] = sg[k][j];
         red[(warp * NQ + 1) * d + c + j] = sb[k][j];
         if (RES) red[(warp * NQ + 2) * d + c + j] = sr[k][j];
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < NQ * d; i += 32 * LNF_WARPS) {
+    float t = red[i];
+#pragma unroll
+    for (int w = 1; w < LNF_WARPS; ++w) t += red[w * NQ * d + i];
+    if (i < 2 * d)
+      part_ln[(long)blockIdx.x * 2 * d + i] = t;
+    else
+      part_res[(long)blockIdx.x * d + (i - 2 * d)] = t;
+  }
+}
+
+// bf16 rows of ln_bwd_fused_kernel with the arithmetic on fp32 pairs and
+// gamma held in registers across a warp's rows.  Per element, in pairs:
+//   xh = x rstd - mean rstd, gd = dy g, s1 += gd, s2 += gd xh,
+//   dgamma += dy xh, dbeta += dy, then
+//   dres = (init ? 0 : dres) + rstd (gd - s1/d - xh s2/d)   (and its column sum)
+// Two blocks per SM (up to 255 registers a thread): the three column
+// accumulators, gamma and two rows of loads stay in registers without spills.
+constexpr int LNB_BLOCKS_PER_SM = 2;
+
+template <int NC, bool RES>
+__global__ void __launch_bounds__(32 * LNF_WARPS, LNB_BLOCKS_PER_SM)
+    ln_bwd_bf16_kernel(const bf16* __restrict__ dy, const bf16* __restrict__ x, const float* __restrict__ mean,
+                       const float* __restrict__ rstd, const bf16* __restrict__ g, bf16* __restrict__ dres,
+                       int dres_init, int M, int d, float* __restrict__ part_ln, float* __restrict__ part_res) {
+  pdl_start();
+  extern __shared__ float red[];  // [LNF_WARPS][3][d]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float2 gg[NC][4];
+  float2 sg[NC][4], sb[NC][4], sr[NC][4];
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    const int c = (lane + 32 * k) * 8;
+    const uint4 u = c < d ? __ldg(reinterpret_cast<const uint4*>(g + c)) : make_uint4(0, 0, 0, 0);
+    gg[k][0] = bf2w(u.x); gg[k][1] = bf2w(u.y); gg[k][2] = bf2w(u.z); gg[k][3] = bf2w(u.w);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sg[k][j] = sb[k][j] = sr[k][j] = make_float2(0.f, 0.f);
+  }
+  const float inv_d = 1.f / (float)d;
+  const int stride = gridDim.x * LNF_WARPS;
+  int m = blockIdx.x * LNF_WARPS + warp;
+  uint4 cx[NC], cd[NC], cr[NC];
+  float cmu = 0.f, crs = 0.f;
+  auto load_row = [&](int r, uint4 (&ux)[NC], uint4 (&ud)[NC], uint4 (&ur)[NC], float& mu_, float& rs_) {
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = (lane + 32 * k) * 8;
+      if (r < M && c < d) {
+        ux[k] = *reinterpret_cast<const uint4*>(x + (long)r * d + c);
+        ud[k] = *reinterpret_cast<const uint4*>(dy + (long)r * d + c);
+        ur[k] = dres_init ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(dres + (long)r * d + c);
+      } else {
+        ux[k] = ud[k] = ur[k] = make_uint4(0, 0, 0, 0);
+      }
+    }
+    if (r < M) {
+      mu_ = mean[r];
+      rs_ = rstd[r];
+    }
+  };
+  load_row(m, cx, cd, cr, cmu, crs);
+  for (; m < M; m += stride) {
+    uint4 nx[NC], nd[NC], nr[NC];
+    float nmu = 0.f, nrs = 0.f;
+    load_row(m + stride, nx, nd, nr, nmu, nrs);
+    const float2 rs2 = make_float2(crs, crs), c2 = make_float2(-cmu * crs, -cmu * crs);
+    float2 s1 = make_float2(0.f, 0.f), s2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const uint32_t* xw = &cx[k].x;
+      const uint32_t* dw = &cd[k].x;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 dv = bf2w(dw[j]);
+        const float2 xh = __ffma2_rn(bf2w(xw[j]), rs2, c2);
+        const float2 gd = __fmul2_rn(dv, gg[k][j]);
+        s1 = __fadd2_rn(s1, gd);
+        s2 = __ffma2_rn(gd, xh, s2);
+        sg[k][j] = __ffma2_rn(dv, xh, sg[k][j]);
+        sb[k][j] = __fadd2_rn(sb[k][j], dv);
+      }
+    }
+    const float m1 = warp_sum(s1.x + s1.y) * inv_d, m2 = warp_sum(s2.x + s2.y) * inv_d;
+    const float2 nm1 = make_float2(-m1, -m1), nm2 = make_float2(-m2, -m2);
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      const int c = (lane + 32 * k) * 8;
+      const uint32_t* xw = &cx[k].x;
+      const uint32_t* dw = &cd[k].x;
+      const uint32_t* rw = &cr[k].x;
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 xh = __ffma2_rn(bf2w(xw[j]), rs2, c2);
+        const float2 gd = __fmul2_rn(bf2w(dw[j]), gg[k][j]);
+        const float2 t = __fadd2_rn(__ffma2_rn(xh, nm2, gd), nm1);   // gd - s1/d - xh s2/d
+        const float2 o = __ffma2_rn(t, rs2, bf2w(rw[j]));
+        if (RES) sr[k][j] = __fadd2_rn(sr[k][j], o);
+        w[j] = pack_bf16x2(o.x, o.y);
+      }
+      if (c < d) *reinterpret_cast<uint4*>(dres + (long)m * d + c) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+#pragma unroll
+    for (int k = 0; k < NC; ++k) {
+      cx[k] = nx[k];
+      cd[k] = nd[k];
+      cr[k] = nr[k];
+    }
+    cmu = nmu;
+    crs = nrs;
+  }
+  constexpr int NQ = RES ? 3 : 2;
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    const int c = (lane + 32 * k) * 8;
+    if (c < d) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        red[(warp * NQ + 0) * d + c + 2 * j] = sg[k][j].x;
+        red[(warp * NQ + 0) * d + c + 2 * j + 1] = sg[k][j].y;
+        red[(warp * NQ + 1) * d + c + 2 * j] = sb[k][j].x;
+        red[(warp * NQ + 1) * d + c + 2 * j + 1] = sb[k][j].y;
+        if (RES) {
+          red[(warp * NQ + 2) * d + c + 2 * j] = sr[k][j].x;
+          red[(warp * NQ + 2) * d + c + 2 * j + 1] = sr[k][j].y;
+        }
       }
     }
   }
@@ -955,8 +1177,14 @@ int grid_for(long n, int threads) {
 template <typename T, int NC>
 int ln_fwd_launch(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int M,
                    int d, cudaStream_t st) {
-  CUDA_TRY(launch_k(ln_fwd_kernel<T, NC>, (M + 7) / 8, 256, 0, st,
-      (const T*)x, (const T*)g, (const T*)b, (T*)y, mean, rstd, M, d));
+  if constexpr (std::is_same<T, bf16>::value) {
+    constexpr int ROWS = 4;
+    CUDA_TRY(launch_k(ln_fwd_bf16_kernel<NC, ROWS>, (M + 8 * ROWS - 1) / (8 * ROWS), 256, 0, st,
+        (const bf16*)x, (const bf16*)g, (const bf16*)b, (bf16*)y, mean, rstd, M, d));
+  } else {
+    CUDA_TRY(launch_k(ln_fwd_kernel<T, NC>, (M + 7) / 8, 256, 0, st,
+        (const T*)x, (const T*)g, (const T*)b, (T*)y, mean, rstd, M, d));
+  }
   return GPT2_OK;
 }
 
@@ -981,8 +1209,8 @@ int ln_fwd_dispatch(const void* x, const void* g, const void* b, void* y, float*
   return GPT2_OK;
 }
 
-int ln_fused_blocks(int M) {
-  const int b = LNF_BLOCKS_PER_SM * num_sms();
+int ln_fused_blocks(int M, int per_sm = LNF_BLOCKS_PER_SM) {
+  const int b = per_sm * num_sms();
   const int need = (M + LNF_WARPS - 1) / LNF_WARPS;
   return b < need ? b : need;
 }
@@ -996,8 +1224,21 @@ int ln_bwd_launch(const void* dy, const void* x, const float* mean, const float*
                    void* dres, int init, float* part, float* part_res, int* nblk, int M, int d, cudaStream_t st) {
   constexpr int VN = Vec<T>::N;
   if constexpr (NC * VN <= 24) {
-    const int blocks = ln_fused_blocks(M);
+    const bool pk = std::is_same<T, bf16>::value;
+    const int blocks = ln_fused_blocks(M, pk ? LNB_BLOCKS_PER_SM : LNF_BLOCKS_PER_SM);
     *nblk = blocks;
+    if constexpr (std::is_same<T, bf16>::value) {
+      if (part_res) {
+        const size_t smem = (size_t)LNF_WARPS * 3 * d * sizeof(float);
+        CUDA_TRY(launch_k(ln_bwd_bf16_kernel<NC, true>, blocks, 32 * LNF_WARPS, smem, st, (const bf16*)dy,
+                          (const bf16*)x, mean, rstd, (const bf16*)g, (bf16*)dres, init, M, d, part, part_res));
+      } else {
+        const size_t smem = (size_t)LNF_WARPS * 2 * d * sizeof(float);
+        CUDA_TRY(launch_k(ln_bwd_bf16_kernel<NC, false>, blocks, 32 * LNF_WARPS, smem, st, (const bf16*)dy,
+                          (const bf16*)x, mean, rstd, (const bf16*)g, (bf16*)dres, init, M, d, part, nullptr));
+      }
+      return GPT2_OK;
+    }
     if (part_res) {
       const size_t smem = (size_t)LNF_WARPS * 3 * d * sizeof(float);
       CUDA_TRY(launch_k(ln_bwd_fused_kernel<T, NC, true>, blocks, 32 * LNF_WARPS, smem, st, 
