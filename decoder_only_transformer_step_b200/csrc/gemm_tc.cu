@@ -194,14 +194,23 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   const int kb_total = g.K / BK;
   if (splits == 0) splits = g.epi.kind == EPI_F32 ? auto_splits(g.M, g.N, g.K, bn) : 1;
   if (splits > kb_total) splits = kb_total;
+  // With per-tile counters an fp32 output (beta 0 or 1) is split in order
+  // inside the kernel: S - 1 partial slices, no separate reduction pass.
+  const int tiles = ((g.M + (pair ? 2 * BM : BM) - 1) / (pair ? 2 * BM : BM)) * ((g.N + n_mma - 1) / n_mma);
+  // (The last split reads the earlier partials one after another, so deeper
+  // splits keep the separate reduction.)
+  bool serial = splits > 1 && splits <= 3 && g.epi.kind == EPI_F32 && g.epi.split_cnt &&
+                (g.epi.beta == 0.f || g.epi.beta == 1.f) &&
+                (long)tiles * (pair ? 2 : 1) * NUM_EPI_WARPS <= g.epi.split_cnt_len;
   if (splits > 1) {
     // fp32 (weight-gradient) outputs, or a plain bf16 store: partial sums in
     // the workspace, then a fixed-order reduction
     if ((g.epi.kind != EPI_F32 && g.epi.kind != EPI_STORE) || g.N % 4 || g.epi.ldo != g.N)
       return GPT2_ERR_INVALID_ARG;
-    size_t need = (size_t)splits * g.M * g.N * sizeof(float);
+    size_t need = (size_t)(serial ? splits - 1 : splits) * g.M * g.N * sizeof(float);
     if (!ws || ws_bytes < need) splits = 1;
   }
+  if (splits <= 1) serial = false;
 
   CUtensorMap ta, tb;
   bool ok_a = g.a_mn ? make_tmap(&ta, g.A, g.M, g.K, g.lda, 64, 64)
@@ -228,7 +237,8 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   p.epi = g.epi;
   p.partial = (float*)ws;
   p.err = err;
-  if (splits > 1) {
+  p.serial = serial ? 1 : 0;
+  if (splits > 1 && !serial) {
     // raw partial sums: the reduction applies alpha and beta
     p.epi.kind = EPI_F32_PARTIAL;
     p.epi.alpha = 1.f;
@@ -276,6 +286,14 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
       } else {
         p.store = ST_REG;
       }
+      if (serial) {
+        // tmC2: the partial slices [split][M][N] of splits 0 .. S-2
+        const uint64_t dims[3] = {(uint64_t)g.N, (uint64_t)g.M, (uint64_t)(splits - 1)};
+        const uint64_t strides[2] = {(uint64_t)g.N * 4, (uint64_t)g.M * g.N * 4};
+        const uint32_t box[3] = {32, 32, 1};
+        ok_c = ok_c && encode_tmap(&tc2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ws, 3, dims, strides, box,
+                                   CU_TENSOR_MAP_SWIZZLE_128B);
+      }
       break;
     case EPI_F32_PARTIAL: {
       p.store = ST_F32_PART;
@@ -315,7 +333,7 @@ int gemm_tc_bf16(const GemmArgs& g, void* ws, size_t ws_bytes, int bn, int split
   }
 #undef TCG_CASE
   if (rc) return rc;
-  if (splits > 1) {
+  if (splits > 1 && !serial) {
     long mn = (long)g.M * g.N;
     long threads = (mn + 3) / 4;
     if (g.epi.kind == EPI_STORE)

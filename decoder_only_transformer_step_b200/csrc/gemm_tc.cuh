@@ -98,6 +98,7 @@ struct TcParams {
   int m_tiles, n_tiles, splits, kb_total;
   int tile_m;  // output rows per work unit (128, or 256 for a CTA pair)
   int n_fast;  // unit order: n varies fastest (1) or m (0)
+  int serial;  // EPI_F32 split along K, reduced in the kernel in split order
   uint32_t idesc;
   int store;
   EpiArgs epi;
@@ -457,6 +458,114 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tm_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN + c_begin);
 
+      // Split along K, reduced here in split order: the units of splits
+      // 0 .. S-2 store their raw partial tile in their split's slice of the
+      // workspace (tmC2) and count it done per (tile, CTA, warp); the unit of
+      // the last split, which comes after them in every CTA's unit order,
+      // waits for those counts, adds the partials in split order and its own
+      // accumulator last, and writes beta * out + alpha * sum through tmC.
+      bool serial_done = false;
+      if constexpr (EK == EPI_F32) {
+        if (p.serial) {
+          serial_done = true;
+          int* cnt = p.epi.split_cnt + ((u % (p.m_tiles * p.n_tiles)) * (PAIR ? 2 : 1) + (int)rank) * NUM_EPI_WARPS + e;
+          const bool last = s + 1 == p.splits;
+          if (last) {
+            // the earlier splits' partials of this warp's rows and columns
+            if (lane == 0) {
+              const uint64_t t0 = globaltimer(), lim = g_wait_limit_ns;
+              uint32_t spins = 0;
+              while (ld_acquire(cnt) < p.splits - 1) {
+                if (*abort_flag) {
+                  ok = false;
+                  break;
+                }
+                if ((++spins & 63u) == 0 && globaltimer() - t0 > lim) {
+                  *abort_flag = 1;
+                  if (p.err) atomicOr(p.err, DEV_ERR_TIMEOUT);
+                  ok = false;
+                  break;
+                }
+              }
+              // the TMA loads below come after that acquire
+              fence_proxy_async_global();
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          }
+          // 32 columns at a time, alternating between the warp's two boxes
+          const int nch = min(2 * NH, max(0, (p.N - (n0 + c_begin) + 31) / 32));
+#pragma unroll
+          for (int ci = 0; ci < 2 * NH; ++ci) {
+            if (!ok || ci >= nch) break;
+            const int cc = n0 + c_begin + 32 * ci;
+            const uint32_t box = wbox + BOX_BYTES * (uint32_t)(ci & 1);
+            // the store that last used this box (two chunks ago) has read it
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            float2 v[16];
+            if (last) {
+              for (int sp = 0; sp + 1 < p.splits; ++sp) {
+                if (lane == 0) {
+                  const uint32_t bar = op_bar(e, ci & 1);
+                  mbar_arrive_expect_tx(bar, BOX_BYTES);
+                  tma_load_3d(box, &tmC2, bar, cc, row0, sp);
+                }
+                ++op_issued[ci & 1];
+                if (!mbar_wait_bounded(op_bar(e, ci & 1), (uint32_t)op_used[ci & 1] & 1u, abort_flag, p.err)) {
+                  ok = false;
+                  break;
+                }
+                ++op_used[ci & 1];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const uint4 w4 = ld_slot(box_slot(box, lane, j));
+                  const float2 a0 = f2(w4.x, w4.y), a1 = f2(w4.z, w4.w);
+                  v[2 * j] = sp == 0 ? a0 : __fadd2_rn(v[2 * j], a0);
+                  v[2 * j + 1] = sp == 0 ? a1 : __fadd2_rn(v[2 * j + 1], a1);
+                }
+                // these reads precede the next TMA write of the box
+                fence_proxy_async_smem();
+                __syncwarp();
+              }
+              if (!ok) break;
+            }
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tm_row + 32u * (uint32_t)ci, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 a = f2(r[2 * i], r[2 * i + 1]);
+              v[i] = last ? __fmul2_rn(__fadd2_rn(v[i], a), al2) : a;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              st_shared_v4(box_slot(box, lane, j), __float_as_uint(v[2 * j].x), __float_as_uint(v[2 * j].y),
+                           __float_as_uint(v[2 * j + 1].x), __float_as_uint(v[2 * j + 1].y));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (!last)
+                tma_store_3d(&tmC2, box, cc, row0, s);
+              else if (p.store == ST_F32)
+                tma_store_2d(&tmC, box, cc, row0);
+              else
+                tma_reduce_add_2d(&tmC, box, cc, row0);
+              bulk_commit();
+            }
+          }
+          if (ok && lane == 0) {
+            if (!last) {
+              // the partial is in memory before it is counted
+              bulk_wait_all();
+              fence_proxy_async_global();
+              red_release_add(cnt, 1);
+            } else {
+              *cnt = 0;  // ready for the next launch
+            }
+          }
+        }
+      }
+
       // EPI_CE_FWD: this row's maximum over the warp's 128 columns (one
       // cross-entropy part; N is a multiple of 128, so they are all inside N
       // or all outside), then exp(acc - max) and its sum in the store pass
@@ -487,7 +596,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
-        if (h >= nh) break;
+        if (serial_done || h >= nh) break;
         const int col0 = n0 + c_begin + 64 * h;
         uint32_t r[2][32];
         tmem_ld_32x32b_x32(tm_row + 64u * (uint32_t)h, r[0]);

@@ -128,6 +128,7 @@ struct Work {
   std::vector<ReduceJob> jobs;
   void* split_ws;
   size_t split_bytes;
+  int* split_cnt;  // per-tile split-order counters, zeroed at each backward
   long long* emb_acc;
   uint8_t* touched;
 };
@@ -136,6 +137,9 @@ struct Work {
 // output tiles (192 at the 124M shape) for 74 SM pairs, 2.6 waves; three
 // K splits make 7.8 waves of a third of the work each.
 constexpr int LM_DGRAD_SPLITS = 3;
+// Counters of the in-kernel split-K ordering: one per (tile, CTA, epilogue
+// warp); split-K is chosen only with fewer tiles than SM pairs or SMs.
+constexpr int SPLIT_COUNTERS = 4096;
 
 size_t split_ws_need(const Shape& s, long M) {
   if (s.mode != 0) return 0;
@@ -220,6 +224,7 @@ size_t carve(const Shape& s, int batch, uint8_t* base, Work* w) {
   w->part_used = 0;
   w->split_bytes = split_ws_need(s, M);
   w->split_ws = c.take<void>(w->split_bytes);
+  w->split_cnt = c.take<int>(SPLIT_COUNTERS * sizeof(int));
   w->emb_acc = c.take<long long>((size_t)s.V * d * 8);
   w->touched = c.take<uint8_t>((size_t)s.V);
   return (c.off + 255) & ~(size_t)255;
@@ -260,7 +265,11 @@ const void* Wp(const gpt2_ctx* c, size_t off) {
 
 int run_gemm(gpt2_ctx* c, const GemmArgs& g, cudaStream_t st) {
   if (c->s.mode) return gemm_simt_f32(g, st);
-  return gemm_tc_bf16(g, c->w.split_ws, c->w.split_bytes, 0, 0, c->w.err, st);
+  GemmArgs h = g;
+  // weight gradients split along K are reduced inside the kernel, in order
+  h.epi.split_cnt = c->w.split_cnt;
+  h.epi.split_cnt_len = SPLIT_COUNTERS;
+  return gemm_tc_bf16(h, c->w.split_ws, c->w.split_bytes, 0, 0, c->w.err, st);
 }
 
 GemmArgs make_gemm(int M, int N, int K, const void* A, int a_mn, long lda, const void* B, int b_mn, long ldb,
@@ -540,6 +549,9 @@ int backward_impl(gpt2_ctx* c, float grad_scale, int accumulate, void* const* ev
   // every attention backward leaves it zeroed
   const int fuse_d = (!f32 && s.hd == 64) ? 1 : 0;
   if (fuse_d) TRY(fill_zero(w.dq_acc, (size_t)M * d * sizeof(float), st));
+  // the split-order counters start at zero (each reduction also leaves them
+  // so; this also clears what an aborted launch may have left)
+  if (!f32) TRY(fill_zero(w.split_cnt, SPLIT_COUNTERS * sizeof(int), st));
 
   // LM head (tied): dX_f = s * dz wte ; dwte (=/+=) s * dz^T X_f, with dz =
   // (softmax - onehot) M / n_valid left in w.logits by the forward

@@ -36,6 +36,8 @@ struct EpiArgs {
   int seq;            // EPI_ROWDOT: rows per sequence
   float* colsum;      // EPI_DGELU, optional: [ceil(M/32), N] fp32 sums of the stored (bf16)
                       //   output over each 32-row group (the bias gradient's partials)
+  int* split_cnt;     // EPI_F32 split along K, optional: zeroed per-tile counters that order
+  int split_cnt_len;  //   the splits inside the kernel (no separate reduction pass)
   // EPI_CE_FWD
   float* ce_max;
   float* ce_sum;
