@@ -475,3 +475,31 @@ def test_deterministic_mode_full_size_step_repeats_bitwise():
         out.append((float(loss.item()), model.grad.clone()))
     assert out[0][0] == out[1][0]
     assert torch.equal(out[0][1], out[1][1])
+
+
+@pytest.mark.slow
+def test_full_size_gradient_scale_equivariance_bitwise():
+    """The page's 32-fold accumulation scales each micro-batch's gradients by
+    grad_scale = 1/32.  In mode 2 every reduction is fixed-order and the
+    embedding scatter's fixed-point unit is relative to grad_scale, so at the
+    bench's full size (124M, 16 x 1024 Zipf tokens) the gradient at
+    grad_scale 1/32 is bitwise 1/32 of the gradient at grad_scale 1 — the
+    scale costs no precision anywhere (the grad_scale-1 gradient is itself
+    checked against the oracle at this size by the prefix-masked test)."""
+    mc = gp.ModelConfig(12, 768, 12, 1024, 50257, 50304, 16, 2)
+    model = gp.GPT2(mc)
+    model.init_params(seed=0)
+    tok, tgt = inputs.zipf_tokens(16, 1024, seed=64)
+    tok_d, tgt_d = torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda()
+    grads = []
+    for scale in (1.0, 1.0 / 32):
+        model.forward_loss(tok_d, tgt_d)
+        model.backward(scale, 0)
+        torch.cuda.synchronize()
+        assert model.status() == 0
+        grads.append(model.grad.clone())
+    g1, g32 = grads
+    assert torch.equal(g32 * 32, g1)
+    # the embedding rows of ids that occur, where the fixed point acts
+    wte = g1[: 50304 * 768].view(50304, 768)
+    assert torch.count_nonzero(wte[:1000]) > 0
