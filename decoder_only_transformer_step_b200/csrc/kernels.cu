@@ -199,95 +199,8 @@ __global__ void ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ g, 
   }
 }
 
-// bf16 rows: the same normalisation with the arithmetic on fp32 pairs
-// (mean, the centred sum of squares, y = (x rstd - mean rstd) g + b as two
-// packed multiply-adds), ROWS rows per warp so gamma and beta are unpacked
-// once, and the next row's load in flight while one is normalised.
+// the two bf16 of a packed word as an fp32 pair (low half first)
 DEVI float2 bf2w(uint32_t w) { return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)); }
-
-template <int NC, int ROWS>
-__global__ void __launch_bounds__(256) ln_fwd_bf16_kernel(const bf16* __restrict__ x, const bf16* __restrict__ g,
-                                                          const bf16* __restrict__ b, bf16* __restrict__ y,
-                                                          float* __restrict__ mean, float* __restrict__ rstd,
-                                                          int M, int d) {
-  pdl_start();
-  const int lane = threadIdx.x & 31;
-  const int m0 = (blockIdx.x * 8 + (threadIdx.x >> 5)) * ROWS;
-  if (m0 >= M) return;
-  float2 gg[NC][4], bb[NC][4];
-#pragma unroll
-  for (int k = 0; k < NC; ++k) {
-    const int c = (lane + 32 * k) * 8;
-    uint4 ug = make_uint4(0, 0, 0, 0), ub = make_uint4(0, 0, 0, 0);
-    if (c < d) {
-      ug = __ldg(reinterpret_cast<const uint4*>(g + c));
-      ub = __ldg(reinterpret_cast<const uint4*>(b + c));
-    }
-    gg[k][0] = bf2w(ug.x); gg[k][1] = bf2w(ug.y); gg[k][2] = bf2w(ug.z); gg[k][3] = bf2w(ug.w);
-    bb[k][0] = bf2w(ub.x); bb[k][1] = bf2w(ub.y); bb[k][2] = bf2w(ub.z); bb[k][3] = bf2w(ub.w);
-  }
-  const float inv_d = 1.f / (float)d;
-  auto load = [&](int m, uint4 (&u)[NC]) {
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-      const int c = (lane + 32 * k) * 8;
-      u[k] = c < d ? *reinterpret_cast<const uint4*>(x + (long)m * d + c) : make_uint4(0, 0, 0, 0);
-    }
-  };
-  uint4 cur[NC];
-  load(m0, cur);
-#pragma unroll 1
-  for (int r = 0; r < ROWS; ++r) {
-    const int m = m0 + r;
-    if (m >= M) break;
-    uint4 nxt[NC];
-    if (r + 1 < ROWS && m + 1 < M) load(m + 1, nxt);
-    float2 v[NC][4];
-    float2 s2 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-      v[k][0] = bf2w(cur[k].x); v[k][1] = bf2w(cur[k].y); v[k][2] = bf2w(cur[k].z); v[k][3] = bf2w(cur[k].w);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) s2 = __fadd2_rn(s2, v[k][j]);
-    }
-    const float mu = warp_sum(s2.x + s2.y) * inv_d;
-    const float2 nmu2 = make_float2(-mu, -mu);
-    float2 q2 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-      const int c = (lane + 32 * k) * 8;
-      if (c < d) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 t = __fadd2_rn(v[k][j], nmu2);
-          q2 = __ffma2_rn(t, t, q2);
-        }
-      }
-    }
-    const float rs = rsqrtf(warp_sum(q2.x + q2.y) * inv_d + 1e-5f);
-    const float2 rs2 = make_float2(rs, rs), c2 = make_float2(-mu * rs, -mu * rs);
-#pragma unroll
-    for (int k = 0; k < NC; ++k) {
-      const int c = (lane + 32 * k) * 8;
-      if (c < d) {
-        uint32_t w[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 xh = __ffma2_rn(v[k][j], rs2, c2);
-          const float2 o = __ffma2_rn(xh, gg[k][j], bb[k][j]);
-          w[j] = pack_bf16x2(o.x, o.y);
-        }
-        *reinterpret_cast<uint4*>(y + (long)m * d + c) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
-    if (lane == 0) {
-      mean[m] = mu;
-      rstd[m] = rs;
-    }
-#pragma unroll
-    for (int k = 0; k < NC; ++k) cur[k] = nxt[k];
-  }
-}
 
 // dx = rstd * (dxhat - mean(dxhat) - xhat * mean(dxhat * xhat)), dxhat = dy * g;
 // dres = (init ? 0 : dres) + dx.  One warp per row with the row in registers;
@@ -1177,14 +1090,11 @@ int grid_for(long n, int threads) {
 template <typename T, int NC>
 int ln_fwd_launch(const void* x, const void* g, const void* b, void* y, float* mean, float* rstd, int M,
                    int d, cudaStream_t st) {
-  if constexpr (std::is_same<T, bf16>::value) {
-    constexpr int ROWS = 4;
-    CUDA_TRY(launch_k(ln_fwd_bf16_kernel<NC, ROWS>, (M + 8 * ROWS - 1) / (8 * ROWS), 256, 0, st,
-        (const bf16*)x, (const bf16*)g, (const bf16*)b, (bf16*)y, mean, rstd, M, d));
-  } else {
-    CUDA_TRY(launch_k(ln_fwd_kernel<T, NC>, (M + 7) / 8, 256, 0, st,
-        (const T*)x, (const T*)g, (const T*)b, (T*)y, mean, rstd, M, d));
-  }
+  // (a packed-arithmetic bf16 variant with gamma / beta in registers over
+  // four rows per warp measured the same in the step and 13 % slower at
+  // 131072 rows: this kernel is not issue-bound enough for it to pay)
+  CUDA_TRY(launch_k(ln_fwd_kernel<T, NC>, (M + 7) / 8, 256, 0, st,
+      (const T*)x, (const T*)g, (const T*)b, (T*)y, mean, rstd, M, d));
   return GPT2_OK;
 }
 
