@@ -247,6 +247,8 @@ struct gpt2_ctx {
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t graph_exec = nullptr;
   int graph_batch = 0;
+  int graph_plain = 0;  // captured with grad_scale 1, accumulate 0
+  float* graph_loss = nullptr;  // where the graph writes the loss
   unsigned long long graph_launches = 0;  // kernels in one launch of the graph
   ~gpt2_ctx() {
     if (graph_exec) cudaGraphExecDestroy(graph_exec);
@@ -855,12 +857,23 @@ int gpt2_step_host(gpt2_ctx* c, const int32_t* tokens_host, const int32_t* targe
   if (batch < 1 || batch > c->cfg.max_batch) return GPT2_ERR_INVALID_ARG;
   cudaStream_t st = S(stream);
   const size_t bytes = (size_t)batch * c->s.T * 4;
-  CUDA_TRY(cudaMemcpyAsync(c->w.tok_stage, tokens_host, bytes, cudaMemcpyHostToDevice, st));
-  CUDA_TRY(cudaMemcpyAsync(c->w.tgt_stage, targets_host, bytes, cudaMemcpyHostToDevice, st));
-  TRY(gpt2_forward_loss(c, c->w.tok_stage, c->w.tgt_stage, batch, c->w.loss, stream));
-  TRY(gpt2_backward(c, 1.f, 0, stream));
+  if (c->graph_exec && c->graph_batch == batch && c->graph_plain) {
+    // the captured micro-step of this shape: ids straight into its inputs
+    CUDA_TRY(cudaMemcpyAsync(c->w.gtok, tokens_host, bytes, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaMemcpyAsync(c->w.gtgt, targets_host, bytes, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaGraphLaunch(c->graph_exec, st));
+    g_launches.fetch_add(c->graph_launches, std::memory_order_relaxed);
+    c->have_fwd = 1;
+    c->fwd_batch = batch;
+  } else {
+    CUDA_TRY(cudaMemcpyAsync(c->w.tok_stage, tokens_host, bytes, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaMemcpyAsync(c->w.tgt_stage, targets_host, bytes, cudaMemcpyHostToDevice, st));
+    TRY(gpt2_forward_loss(c, c->w.tok_stage, c->w.tgt_stage, batch, c->w.loss, stream));
+    TRY(gpt2_backward(c, 1.f, 0, stream));
+  }
   TRY(gpt2_adamw_step(c, lr, beta1, beta2, eps, weight_decay, step, stream));
-  CUDA_TRY(cudaMemcpyAsync(loss_host, c->w.loss, sizeof(float), cudaMemcpyDeviceToHost, st));
+  const float* loss_src = (c->graph_exec && c->graph_batch == batch && c->graph_plain) ? c->graph_loss : c->w.loss;
+  CUDA_TRY(cudaMemcpyAsync(loss_host, loss_src, sizeof(float), cudaMemcpyDeviceToHost, st));
   CUDA_TRY(cudaStreamSynchronize(st));
   return GPT2_OK;
 }
@@ -874,6 +887,7 @@ int gpt2_graph_release(gpt2_ctx* c) {
   c->graph_exec = nullptr;
   c->graph = nullptr;
   c->graph_batch = 0;
+  c->graph_plain = 0;
   c->graph_launches = 0;
   return GPT2_OK;
 }
@@ -908,6 +922,8 @@ int gpt2_graph_capture(gpt2_ctx* c, int batch, float grad_scale, int accumulate,
   c->graph = g;
   c->graph_exec = ex;
   c->graph_batch = batch;
+  c->graph_plain = (grad_scale == 1.f && accumulate == 0) ? 1 : 0;
+  c->graph_loss = loss_dev ? loss_dev : c->w.loss;
   c->graph_launches = n;
   return GPT2_OK;
 }

@@ -210,7 +210,11 @@ int gpt2_get_status(gpt2_ctx* ctx, void* stream);
 /* One whole training step from HOST memory: copies tokens/targets (host,
  * int32 [batch, n_ctx], preferably pinned) to the device, runs forward,
  * backward (grad_scale 1, accumulate 0) and AdamW, copies the loss back into
- * *loss_host and synchronises the stream before returning. */
+ * *loss_host and synchronises the stream before returning.  When the context
+ * holds a captured micro-step (gpt2_graph_capture) for the same batch with
+ * grad_scale 1 and accumulate 0, the ids are copied straight into the
+ * graph's inputs and the graph runs instead of the separate launches (same
+ * kernels, same results; the loss is read from where the graph writes it). */
 int gpt2_step_host(gpt2_ctx* ctx, const int32_t* tokens_host, const int32_t* targets_host,
                    int batch, float* loss_host, float lr, float beta1, float beta2,
                    float eps, float weight_decay, int step, void* stream);

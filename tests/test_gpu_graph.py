@@ -80,3 +80,32 @@ def test_graph_launch_count_and_host_checks():
         model.graph_step(tok, tgt)
     assert np.isfinite(float(model.loss.item()))
     assert model.status() == 0
+
+
+def test_step_host_replays_the_graph_bitwise():
+    """gpt2_step_host with a captured micro-step of the same shape (grad_scale
+    1, accumulate 0) takes the graph: parameters and loss after the step are
+    bitwise those of the step without a graph (mode 2), and the graph's
+    kernels are counted."""
+    B, T, Vr, V = 2, 256, 1000, 1024
+    tok, tgt = inputs.zipf_tokens(B, T, n_ids=Vr, seed=91)
+    th, gh = torch.from_numpy(tok).pin_memory(), torch.from_numpy(tgt).pin_memory()
+    out = []
+    for use_graph in (False, True):
+        model = gp.GPT2(gp.ModelConfig(2, 256, 4, T, Vr, V, B, 2))
+        model.init_params(seed=12)
+        model.forward_loss(th.cuda(), gh.cuda())
+        model.backward()
+        torch.cuda.synchronize()
+        model.grad.zero_()
+        if use_graph:
+            model.graph_capture(B)
+        lh = torch.zeros(1).pin_memory()
+        l0 = gp.gpt2_kernel_launches()
+        model.step_host(th, gh, lh, 1)
+        launched = gp.gpt2_kernel_launches() - l0
+        assert model.status() == 0
+        out.append((float(lh.item()), model.master.clone(), launched))
+    assert out[0][0] == out[1][0]
+    assert torch.equal(out[0][1], out[1][1])
+    assert out[0][2] == out[1][2]
