@@ -62,7 +62,7 @@ DEVI uint32_t swz(int r, int c) {
 // ----------------------------------------------------------------- forward --
 
 template <int HD>
-__global__ void __launch_bounds__(256) attn_fwd_kernel(const bf16* __restrict__ qkv,
+__global__ void __launch_bounds__(256) attn_fwd_kernel(const bf16* qkv,
                                                        bf16* __restrict__ o, float* __restrict__ lse,
                                                        int T, int H, float scale_log2) {
   pdl_start();
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(256) attn_fwd_kernel(const bf16* __restrict__ 
 
 // D[b,h,t] = sum_c dO[t,c] O[t,c]; also zeroes the fp32 dQ accumulator.
 template <typename T_>
-__global__ void attn_bwd_prep_kernel(const T_* __restrict__ o, const T_* __restrict__ dout,
+__global__ void attn_bwd_prep_kernel(const T_* o, const T_* dout,
                                      float* __restrict__ dvec, float* __restrict__ dq_acc, int B,
                                      int T, int H, int hd) {
   pdl_start();
@@ -245,7 +245,7 @@ __global__ void attn_bwd_prep_kernel(const T_* __restrict__ o, const T_* __restr
 // bf16 version: one warp per token row, 16-byte loads; the lanes holding one
 // head's chunks reduce with shuffles.  Also zeroes the dQ accumulator row.
 template <int HD>
-__global__ void attn_bwd_prep_bf16_kernel(const bf16* __restrict__ o, const bf16* __restrict__ dout,
+__global__ void attn_bwd_prep_bf16_kernel(const bf16* o, const bf16* dout,
                                           float* __restrict__ dvec, float* __restrict__ dq_acc, long M, int T,
                                           int H) {
   pdl_start();
@@ -274,10 +274,10 @@ __global__ void attn_bwd_prep_bf16_kernel(const bf16* __restrict__ o, const bf16
 }
 
 template <int HD>
-__global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ qkv,
-                                                       const bf16* __restrict__ dout,
-                                                       const float* __restrict__ lse,
-                                                       const float* __restrict__ dvec,
+__global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* qkv,
+                                                       const bf16* dout,
+                                                       const float* lse,
+                                                       const float* dvec,
                                                        bf16* __restrict__ dqkv,
                                                        float* __restrict__ dq_acc, int T, int H,
                                                        float scale, float scale_log2) {
@@ -483,7 +483,7 @@ __global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ 
 
 // dqkv[m, 0:d] = bf16(sum over key blocks kb <= query block of part[kb][m])
 // in key-block order (the deterministic mode of the attention backward)
-__global__ void dq_sum_bf16_kernel(const float* __restrict__ part, bf16* __restrict__ dqkv, long M, int T, int d) {
+__global__ void dq_sum_bf16_kernel(const float* part, bf16* __restrict__ dqkv, long M, int T, int d) {
   pdl_start();
   long i = (blockIdx.x * (long)blockDim.x + threadIdx.x) * 4;
   if (i >= M * d) return;
@@ -516,7 +516,7 @@ __global__ void dq_to_bf16_kernel(float* __restrict__ dq_acc, bf16* __restrict__
 // ------------------------------------------------------- fp32 (mode 1) ----
 
 // One CTA of 64 threads per (query t, batch*head).
-__global__ void attn_fwd_f32_kernel(const float* __restrict__ qkv, float* __restrict__ o,
+__global__ void attn_fwd_f32_kernel(const float* qkv, float* __restrict__ o,
                                     float* __restrict__ lse, int T, int H, int hd, float scale) {
   pdl_start();
   extern __shared__ float s[];  // [T] scores, then [64] reduction slots
@@ -570,8 +570,8 @@ __global__ void attn_fwd_f32_kernel(const float* __restrict__ qkv, float* __rest
 }
 
 // dQ for query t: ds_j = p_j (dO.v_j - D) scale ; dq = sum_j ds_j k_j.
-__global__ void attn_bwd_q_f32_kernel(const float* __restrict__ qkv, const float* __restrict__ dout,
-                                      const float* __restrict__ lse, const float* __restrict__ dvec,
+__global__ void attn_bwd_q_f32_kernel(const float* qkv, const float* dout,
+                                      const float* lse, const float* dvec,
                                       float* __restrict__ dqkv, int T, int H, int hd, float scale) {
   pdl_start();
   extern __shared__ float s[];
@@ -604,8 +604,8 @@ __global__ void attn_bwd_q_f32_kernel(const float* __restrict__ qkv, const float
 }
 
 // dK, dV for key j: over queries i >= j.
-__global__ void attn_bwd_kv_f32_kernel(const float* __restrict__ qkv, const float* __restrict__ dout,
-                                       const float* __restrict__ lse, const float* __restrict__ dvec,
+__global__ void attn_bwd_kv_f32_kernel(const float* qkv, const float* dout,
+                                       const float* lse, const float* dvec,
                                        float* __restrict__ dqkv, int T, int H, int hd, float scale) {
   pdl_start();
   extern __shared__ float s[];  // p[T], ds[T]

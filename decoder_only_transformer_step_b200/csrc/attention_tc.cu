@@ -819,7 +819,7 @@ constexpr uint32_t IDESC_DQ =
 __global__ void __launch_bounds__(B_NUM_THREADS, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
                        const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDQKV,
-                       const float* __restrict__ lse, const float* __restrict__ dvec, int T, int H, float scale,
+                       const float* lse, const float* dvec, int T, int H, float scale,
                        float scale_log2, int* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -1166,7 +1166,7 @@ static_assert(128 * REGS_CTRL + 256 * REGS_ELEM + 128 * REGS_DRAIN <= THREADS * 
 __global__ void __launch_bounds__(bw::THREADS, 1)
     attn_bwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmDO,
                         const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDQKV,
-                        const float* __restrict__ lse, const float* __restrict__ dvec, int T, int H, int n_items,
+                        const float* lse, const float* dvec, int T, int H, int n_items,
                         float scale, float scale_log2, int det, int* err) {
   // (local names shadow the one-CTA-per-block backward's constants above)
   constexpr int QS = bw::QS, SM_KV = bw::SM_KV, SM_QR = bw::SM_QR, SM_DOR = bw::SM_DOR, SM_DS = bw::SM_DS;

@@ -442,6 +442,12 @@ DEVI void tc_commit_pair(uint32_t bar) {
 // predecessor to complete, with memory visible, before its first global
 // access.  The next kernel's launch and shared-memory / TMEM set-up then
 // overlap this one's tail.
+//
+// Kernel inputs are therefore never declared `const T* __restrict__` (nor read
+// with __ldg): a read-only no-alias argument counts as invariant for the whole
+// kernel, so the compiler may issue its loads ahead of griddepcontrol.wait,
+// i.e. before the kernels that write it have finished.  `__restrict__` stays
+// on outputs, which is enough for the no-alias reasoning between the two.
 DEVI void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 DEVI void pdl_start() {

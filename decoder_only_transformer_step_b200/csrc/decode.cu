@@ -386,8 +386,8 @@ __global__ void __launch_bounds__(GV_WARPS * 32) decode_gemv_kernel(const __grid
 // x[r, :] = wte[tok[r]] + wpe[pos[r]] (fp32); an id outside [0, vocab_real)
 // or a position outside [0, limit) raises its status bit and reads row 0.
 template <typename T>
-__global__ void embed_decode_kernel(const int32_t* __restrict__ tok, const int32_t* __restrict__ pos,
-                                    const T* __restrict__ wte, const T* __restrict__ wpe, float* __restrict__ x,
+__global__ void embed_decode_kernel(const int32_t* tok, const int32_t* pos,
+                                    const T* wte, const T* wpe, float* __restrict__ x,
                                     int d, int vocab_real, int limit, int* err) {
   pdl_start();
   const int r = blockIdx.x;
@@ -415,8 +415,8 @@ constexpr int AD_WARPS = 8;
 // warps' results merged through shared memory.
 template <typename T, int HD>
 __global__ void __launch_bounds__(AD_WARPS * 32)
-    attn_decode_kernel(const T* __restrict__ kc, const T* __restrict__ vc, const float* __restrict__ q,
-                       float* __restrict__ o, const int32_t* __restrict__ pos, int H, int max_len,
+    attn_decode_kernel(const T* kc, const T* vc, const float* q,
+                       float* __restrict__ o, const int32_t* pos, int H, int max_len,
                        float scale_log2) {
   __shared__ float sm_m[AD_WARPS], sm_l[AD_WARPS];
   __shared__ float sm_o[AD_WARPS][HD];
@@ -514,7 +514,7 @@ DEVI bool greedy_better(float a, int ia, float b, int ib) {
 
 // next[r] = argmax over v < vocab_real of logits[r, v]; pos[r] += 1 if pos.
 __global__ void __launch_bounds__(1024)
-    greedy_kernel(const float* __restrict__ logits, long ld, int vocab_real, int32_t* __restrict__ next,
+    greedy_kernel(const float* logits, long ld, int vocab_real, int32_t* __restrict__ next,
                   int32_t* __restrict__ pos) {
   __shared__ float sv[32];
   __shared__ int si[32];
@@ -580,7 +580,7 @@ __global__ void __launch_bounds__(1024)
 // (value, id); one warp per row then picks the best of the GREEDY_SLICES.
 constexpr int GREEDY_SLICES = 16;
 __global__ void __launch_bounds__(256)
-    greedy_part_kernel(const float* __restrict__ logits, long ld, int vocab_real, float* __restrict__ pv,
+    greedy_part_kernel(const float* logits, long ld, int vocab_real, float* __restrict__ pv,
                        int* __restrict__ pi) {
   __shared__ float sv[8];
   __shared__ int si[8];
@@ -631,7 +631,7 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-__global__ void greedy_final_kernel(const float* __restrict__ pv, const int* __restrict__ pi, int vocab_real,
+__global__ void greedy_final_kernel(const float* pv, const int* pi, int vocab_real,
                                     int32_t* __restrict__ next, int32_t* __restrict__ pos) {
   pdl_start();
   const int r = blockIdx.x, lane = threadIdx.x;
@@ -656,8 +656,8 @@ __global__ void greedy_final_kernel(const float* __restrict__ pv, const int* __r
 // [rows * T, 3d] into the cache planes; plen outside [1, limit] raises the
 // position bit and copies nothing for that row.
 template <typename T>
-__global__ void prefill_kv_kernel(const T* __restrict__ qkv, T* __restrict__ kc, T* __restrict__ vc,
-                                  const int32_t* __restrict__ plen, int T_ctx, int H, int hd, int max_len,
+__global__ void prefill_kv_kernel(const T* qkv, T* __restrict__ kc, T* __restrict__ vc,
+                                  const int32_t* plen, int T_ctx, int H, int hd, int max_len,
                                   int limit, int* err) {
   pdl_start();
   const int p = blockIdx.x, r = blockIdx.y;
@@ -679,7 +679,7 @@ __global__ void prefill_kv_kernel(const T* __restrict__ qkv, T* __restrict__ kc,
 // logits_out[r, :] = logits[r * T + plen[r] - 1, :] in fp32 (plen clamped to
 // [1, limit]; the position bit is raised by the K/V copy).
 template <typename T>
-__global__ void prefill_logits_kernel(const T* __restrict__ logits, const int32_t* __restrict__ plen,
+__global__ void prefill_logits_kernel(const T* logits, const int32_t* plen,
                                       float* __restrict__ out, int T_ctx, int V, int limit) {
   pdl_start();
   const int r = blockIdx.y;

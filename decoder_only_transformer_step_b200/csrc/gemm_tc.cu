@@ -21,7 +21,7 @@ using namespace tcg;
 namespace {
 
 // out = beta*out + alpha * sum_s part[s]   (fixed order over s)
-__global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, long mn,
+__global__ void splitk_reduce_kernel(const float* part, int splits, long mn,
                                      float* __restrict__ out, float alpha, float beta) {
   pdl_start();
   long i = (blockIdx.x * (long)blockDim.x + threadIdx.x) * 4;
@@ -49,7 +49,7 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
 }
 
 // bf16 out = alpha * sum_s part[s]   (fixed order over s; mn a multiple of 4)
-__global__ void splitk_reduce_bf16_kernel(const float* __restrict__ part, int splits, long mn,
+__global__ void splitk_reduce_bf16_kernel(const float* part, int splits, long mn,
                                           bf16* __restrict__ out, float alpha) {
   pdl_start();
   const long i = (blockIdx.x * (long)blockDim.x + threadIdx.x) * 4;

@@ -177,7 +177,7 @@ namespace tcg {
 // the loads broadcast.
 DEVI void bias8(const bf16* bias, int N, int c, float2 (&b)[4]) {
   if (c + 8 <= N) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(bias + c));
+    const uint4 u = *reinterpret_cast<const uint4*>(bias + c);
     b[0] = bf2(u.x);
     b[1] = bf2(u.y);
     b[2] = bf2(u.z);
@@ -574,7 +574,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int ytgt = -1;
       if constexpr (EK == EPI_CE_FWD) {
         if (nh > 0) {
-          if (row < p.M) ytgt = __ldg(p.epi.ce_tgt + row);
+          if (row < p.M) ytgt = p.epi.ce_tgt[row];
           float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int ci = 0; ci < 2 * NH; ci += 2) {

@@ -61,8 +61,8 @@ DEVI void unpack16<float>(const uint4& u, float (&f)[4]) {
 
 // x[m] = wte[tok[m]] + wpe[m mod T]; one warp per row.
 template <typename T>
-__global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const T* __restrict__ wte,
-                                 const T* __restrict__ wpe, T* __restrict__ x, int M, int Tn, int d,
+__global__ void embed_fwd_kernel(const int32_t* tok, const T* wte,
+                                 const T* wpe, T* __restrict__ x, int M, int Tn, int d,
                                  int vocab_real, int* err) {
   pdl_start();
   constexpr int VN = Vec<T>::N;
@@ -97,7 +97,7 @@ __global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const T* __res
 // |grad_scale|): dx is proportional to grad_scale, so the resolution relative
 // to the gradient does not shrink under k-fold accumulation (grad_scale 1/k).
 template <typename T>
-__global__ void embed_scatter_kernel(const int32_t* __restrict__ tok, const T* __restrict__ dx,
+__global__ void embed_scatter_kernel(const int32_t* tok, const T* dx,
                                      unsigned long long* __restrict__ acc, uint8_t* __restrict__ touched,
                                      int M, int d, int V, double fix) {
   pdl_start();
@@ -131,7 +131,7 @@ __global__ void embed_convert_kernel(unsigned long long* __restrict__ acc, uint8
 
 // dwpe[t] = (accumulate ? dwpe[t] : 0) + sum_b dx[b, t]   (fixed order in b)
 template <typename T>
-__global__ void wpe_grad_kernel(const T* __restrict__ dx, float* __restrict__ dwpe, int B, int Tn, int d,
+__global__ void wpe_grad_kernel(const T* dx, float* __restrict__ dwpe, int B, int Tn, int d,
                                 int accumulate) {
   pdl_start();
   long i = blockIdx.x * (long)blockDim.x + threadIdx.x;
@@ -146,7 +146,7 @@ __global__ void wpe_grad_kernel(const T* __restrict__ dx, float* __restrict__ dw
 // One warp per row; NC = 16-byte chunks per lane (row cached in registers).
 
 template <typename T, int NC>
-__global__ void ln_fwd_kernel(const T* __restrict__ x, const T* __restrict__ g, const T* __restrict__ b,
+__global__ void ln_fwd_kernel(const T* x, const T* g, const T* b,
                               T* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd, int M,
                               int d) {
   pdl_start();
@@ -206,10 +206,10 @@ DEVI float2 bf2w(uint32_t w) { return make_float2(__uint_as_float(w << 16), __ui
 // dres = (init ? 0 : dres) + dx.  One warp per row with the row in registers;
 // no per-thread accumulators, so many warps are resident to cover HBM latency.
 template <typename T, int NC>
-__global__ void __launch_bounds__(256) ln_bwd_dx_kernel(const T* __restrict__ dy, const T* __restrict__ x,
-                                                        const float* __restrict__ mean,
-                                                        const float* __restrict__ rstd,
-                                                        const T* __restrict__ g, T* __restrict__ dres,
+__global__ void __launch_bounds__(256) ln_bwd_dx_kernel(const T* dy, const T* x,
+                                                        const float* mean,
+                                                        const float* rstd,
+                                                        const T* g, T* __restrict__ dres,
                                                         int dres_init, int M, int d) {
   pdl_start();
   constexpr int VN = Vec<T>::N;
@@ -261,9 +261,9 @@ __global__ void __launch_bounds__(256) ln_bwd_dx_kernel(const T* __restrict__ dy
 constexpr int LNP_ROWS = 128;
 
 template <typename T>
-__global__ void __launch_bounds__(256) ln_param_colsum_kernel(const T* __restrict__ dy, const T* __restrict__ x,
-                                                              const float* __restrict__ mean,
-                                                              const float* __restrict__ rstd, int M, int d,
+__global__ void __launch_bounds__(256) ln_param_colsum_kernel(const T* dy, const T* x,
+                                                              const float* mean,
+                                                              const float* rstd, int M, int d,
                                                               float* __restrict__ part) {
   pdl_start();
   constexpr int VN = Vec<T>::N;
@@ -316,8 +316,8 @@ constexpr int LNF_BLOCKS_PER_SM = 3;
 
 template <typename T, int NC, bool RES>
 __global__ void __launch_bounds__(32 * LNF_WARPS, LNF_BLOCKS_PER_SM)
-    ln_bwd_fused_kernel(const T* __restrict__ dy, const T* __restrict__ x, const float* __restrict__ mean,
-                        const float* __restrict__ rstd, const T* __restrict__ g, T* __restrict__ dres,
+    ln_bwd_fused_kernel(const T* dy, const T* x, const float* mean,
+                        const float* rstd, const T* g, T* __restrict__ dres,
                         int dres_init, int M, int d, float* __restrict__ part_ln, float* __restrict__ part_res) {
   pdl_start();
   constexpr int VN = Vec<T>::N;
@@ -446,8 +446,8 @@ constexpr int LNB_BLOCKS_PER_SM = 2;
 
 template <int NC, bool RES>
 __global__ void __launch_bounds__(32 * LNF_WARPS, LNB_BLOCKS_PER_SM)
-    ln_bwd_bf16_kernel(const bf16* __restrict__ dy, const bf16* __restrict__ x, const float* __restrict__ mean,
-                       const float* __restrict__ rstd, const bf16* __restrict__ g, bf16* __restrict__ dres,
+    ln_bwd_bf16_kernel(const bf16* dy, const bf16* x, const float* mean,
+                       const float* rstd, const bf16* g, bf16* __restrict__ dres,
                        int dres_init, int M, int d, float* __restrict__ part_ln, float* __restrict__ part_res) {
   pdl_start();
   extern __shared__ float red[];  // [LNF_WARPS][3][d]
@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(32 * LNF_WARPS, LNB_BLOCKS_PER_SM)
 #pragma unroll
   for (int k = 0; k < NC; ++k) {
     const int c = (lane + 32 * k) * 8;
-    const uint4 u = c < d ? __ldg(reinterpret_cast<const uint4*>(g + c)) : make_uint4(0, 0, 0, 0);
+    const uint4 u = c < d ? *reinterpret_cast<const uint4*>(g + c) : make_uint4(0, 0, 0, 0);
     gg[k][0] = bf2w(u.x); gg[k][1] = bf2w(u.y); gg[k][2] = bf2w(u.z); gg[k][3] = bf2w(u.w);
 #pragma unroll
     for (int j = 0; j < 4; ++j) sg[k][j] = sb[k][j] = sr[k][j] = make_float2(0.f, 0.f);
@@ -567,7 +567,7 @@ __global__ void __launch_bounds__(32 * LNF_WARPS, LNB_BLOCKS_PER_SM)
 
 // grad[j] = beta * grad[j] + sum_r part[r, j] (r ascending); 8 row slices per
 // column reduced in a fixed order.
-__global__ void reduce_rows_kernel(const float* __restrict__ part, int nrows, int n, float* __restrict__ grad,
+__global__ void reduce_rows_kernel(const float* part, int nrows, int n, float* __restrict__ grad,
                                    float beta) {
   pdl_start();
   __shared__ float sm[8][33];
@@ -620,7 +620,7 @@ __global__ void reduce_rows_batch_kernel(const __grid_constant__ ReduceBatchArgs
 constexpr int CS_ROWS = 128;
 
 template <typename T>
-__global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ x, int M, int N,
+__global__ void __launch_bounds__(256) colsum_kernel(const T* x, int M, int N,
                                                      float* __restrict__ part) {
   pdl_start();
   constexpr int VN = Vec<T>::N;
@@ -655,7 +655,7 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ x, in
 // ---------------------------------------------------------- cross-entropy --
 // Number of positions with a target (target -1 = masked); any other id outside
 // [0, vocab_real) raises the token-range bit and counts as masked.
-__global__ void __launch_bounds__(1024) count_targets_kernel(const int32_t* __restrict__ tgt, int M,
+__global__ void __launch_bounds__(1024) count_targets_kernel(const int32_t* tgt, int M,
                                                              int vocab_real, int* __restrict__ n_valid, int* err) {
   pdl_start();
   __shared__ int red[32];
@@ -682,9 +682,9 @@ __global__ void __launch_bounds__(1024) count_targets_kernel(const int32_t* __re
 // then, in place, dz_v = exp(z_v - lse) - [v == y] (unscaled; the backward
 // GEMMs apply grad_scale / M).
 template <typename T>
-__global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const int32_t* __restrict__ tgt,
+__global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const int32_t* tgt,
                                                  float* __restrict__ loss_rows, int V, int vocab_real,
-                                                 const int* __restrict__ n_valid, int* err) {
+                                                 const int* n_valid, int* err) {
   pdl_start();
   constexpr int VN = Vec<T>::N;
   constexpr int U = 4;  // 16-byte vectors in flight per thread and trip
@@ -789,7 +789,7 @@ __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ logits, const i
 
 // loss = sum(loss_rows) / n_valid (masked rows hold 0), fixed-order tree;
 // flags a non-finite result.
-__global__ void loss_mean_kernel(const float* __restrict__ rows, int M, const int* __restrict__ n_valid,
+__global__ void loss_mean_kernel(const float* rows, int M, const int* n_valid,
                                  float* __restrict__ loss, int* err) {
   pdl_start();
   __shared__ float sm[1024];
@@ -823,8 +823,8 @@ __global__ void loss_mean_kernel(const float* __restrict__ rows, int M, const in
 // (0 where masked), i.e. dz = (softmax - onehot) scaled so that the backward
 // GEMMs' alpha = grad_scale / M gives the mean over the positions with a
 // target.  One block per token row, four 16-byte loads in flight per thread.
-__global__ void __launch_bounds__(256) ce_merge_kernel(const float* __restrict__ pm, const float* __restrict__ ps,
-                                                       const float* __restrict__ zt, const int32_t* __restrict__ tgt,
+__global__ void __launch_bounds__(256) ce_merge_kernel(const float* pm, const float* ps,
+                                                       const float* zt, const int32_t* tgt,
                                                        int M, int P, int vocab_real, float* __restrict__ lse_out,
                                                        float* __restrict__ loss_rows) {
   pdl_start();
@@ -862,9 +862,9 @@ __global__ void __launch_bounds__(256) ce_merge_kernel(const float* __restrict__
   }
 }
 
-__global__ void __launch_bounds__(256) ce_dz_kernel(bf16* __restrict__ e, const float* __restrict__ pm,
-                                                    const float* __restrict__ lse, const int32_t* __restrict__ tgt,
-                                                    int M, int V, int vocab_real, const int* __restrict__ n_valid) {
+__global__ void __launch_bounds__(256) ce_dz_kernel(bf16* __restrict__ e, const float* pm,
+                                                    const float* lse, const int32_t* tgt,
+                                                    int M, int V, int vocab_real, const int* n_valid) {
   pdl_start();
   constexpr float L2E = 1.4426950408889634f;
   constexpr int U = 4;
@@ -878,6 +878,11 @@ __global__ void __launch_bounds__(256) ce_dz_kernel(bf16* __restrict__ e, const 
   const int yv = valid ? y : -1;
   bf16* row = e + (long)m * V;
   const int pieces = V / 8;
+  // the row's per-part scales exp(pm - lse) * scale, once, in shared memory
+  extern __shared__ float part_scale[];  // [V / 128]
+  for (int p = threadIdx.x; p < (V >> 7); p += 256)
+    part_scale[p] = ex2_approx(fmaf(pm[(long)p * M + m], L2E, -l2)) * scale;
+  __syncthreads();
   // the whole row, 16-byte pieces 4 KB apart, four loads in flight per thread
   for (int p0 = threadIdx.x; p0 < pieces; p0 += 256 * U) {
     uint4 u[U];
@@ -891,8 +896,8 @@ __global__ void __launch_bounds__(256) ce_dz_kernel(bf16* __restrict__ e, const 
       const int pi = p0 + 256 * k;
       if (pi < pieces) {
         const int c = 8 * pi;
-        // one part's scale exp(pm - lse) per 16-byte piece (V is a multiple of 128)
-        const float s = ex2_approx(fmaf(pm[(long)(c >> 7) * M + m], L2E, -l2)) * scale;
+        // (V is a multiple of 128: a 16-byte piece lies in one part)
+        const float s = part_scale[c >> 7];
         const int dy = yv - c;
         float f[8] = {bf16lo(u[k].x), bf16hi(u[k].x), bf16lo(u[k].y), bf16hi(u[k].y),
                       bf16lo(u[k].z), bf16hi(u[k].z), bf16lo(u[k].w), bf16hi(u[k].w)};
@@ -955,7 +960,7 @@ DEVI int tensor_kind(long i, const LayoutDims& L, int* one) {
 // Global L2 norm of the flat gradient in two fixed-order passes: per-block
 // sums of squares over a grid of GRAD_NORM_PARTS blocks (fixed, so the result
 // does not depend on the device), then one block adds them and takes the root.
-__global__ void __launch_bounds__(256) sumsq_kernel(const float* __restrict__ g, long n4, float* __restrict__ part) {
+__global__ void __launch_bounds__(256) sumsq_kernel(const float* g, long n4, float* __restrict__ part) {
   pdl_start();
   __shared__ float red[8];
   float s = 0.f;
@@ -973,7 +978,7 @@ __global__ void __launch_bounds__(256) sumsq_kernel(const float* __restrict__ g,
   }
 }
 
-__global__ void __launch_bounds__(256) norm_final_kernel(const float* __restrict__ part, int nparts,
+__global__ void __launch_bounds__(256) norm_final_kernel(const float* part, int nparts,
                                                          float* __restrict__ norm) {
   pdl_start();
   __shared__ float red[8];
@@ -993,9 +998,9 @@ __global__ void __launch_bounds__(256) norm_final_kernel(const float* __restrict
 // (global-norm clipping).
 // Elements [base, base + 4 n4) of the flat buffers; the pointers point at
 // element base, whose layout position decides the weight-decay mask.
-__global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
+__global__ void adamw_kernel(float* __restrict__ p, const float* g, float* __restrict__ m,
                              float* __restrict__ v, uint16_t* __restrict__ shadow, long n4, long base,
-                             LayoutDims L, AdamArgs a, const float* __restrict__ gnorm, float max_norm) {
+                             LayoutDims L, AdamArgs a, const float* gnorm, float max_norm) {
   pdl_start();
   float clip = 1.f;
   if (gnorm) {
@@ -1073,7 +1078,7 @@ __global__ void init_kernel(float* __restrict__ p, long n, LayoutDims L, uint64_
   }
 }
 
-__global__ void cast_shadow_kernel(const float* __restrict__ p, uint16_t* __restrict__ s, long n4) {
+__global__ void cast_shadow_kernel(const float* p, uint16_t* __restrict__ s, long n4) {
   pdl_start();
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
     float4 v = reinterpret_cast<const float4*>(p)[i];
@@ -1295,8 +1300,8 @@ int ce_merge_dz(const float* part_max, const float* part_sum, const float* zt, c
   CUDA_TRY(launch_k(ce_merge_kernel, (M + 31) / 32, 256, 0, st, part_max, part_sum, zt, tgt, M, V / 128, vocab_real,
                     lse, loss_rows));
   LAUNCH_CHECK();
-  CUDA_TRY(launch_k(ce_dz_kernel, M, 256, 0, st, (bf16*)e, part_max, (const float*)lse, tgt, M, V, vocab_real,
-                    n_valid));
+  CUDA_TRY(launch_k(ce_dz_kernel, M, 256, (size_t)(V / 128) * sizeof(float), st, (bf16*)e, part_max,
+                    (const float*)lse, tgt, M, V, vocab_real, n_valid));
   LAUNCH_CHECK();
   return GPT2_OK;
 }
