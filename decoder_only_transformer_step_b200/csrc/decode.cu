@@ -46,12 +46,16 @@ DEVI float4 ld4f(const bf16* p) {
 }
 DEVI float4 ld4f(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
-// Weights are read once per step: keep them out of L1.
+// Weights are read once per step: keep them out of L1.  Volatile, with a
+// memory clobber, so that it stays after the kernel's grid-dependency wait
+// (a plain asm is free to move, and an earlier kernel still in flight may be
+// writing the weights).
 DEVI uint4 ld_stream16(const void* p) {
   uint4 r;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-      : "l"(p));
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p)
+               : "memory");
   return r;
 }
 

@@ -254,3 +254,25 @@ def test_decode_wide_model_matches_oracle(batch):
         pos = pos + 1
     torch.cuda.synchronize()
     assert model.status() == 0
+
+
+def test_decode_step_launch_count_and_repeatability():
+    # one decode step = embedding, 5 kernels per layer (LN1 + QKV, attention,
+    # attention projection, LN2 + fc, MLP projection), LN_f + LM head; every
+    # sum in a fixed order, so the same step on the same cache is bitwise the same
+    oc = Config(n_layer=2, d_model=128, n_head=2, n_ctx=64, vocab=1024)
+    params = params_for(oc, seed=71)
+    model = make_model(oc, 1000, 4, 0)
+    load_params(model, params, oc)
+    tok, _ = inputs.uniform_tokens(4, oc.n_ctx, 1000, seed=72)
+    plen = np.array([3, 9, 1, 20], dtype=np.int32)
+    cache = gp.KVCache(model, 4, 48)
+    cache.prefill(i32(tok), i32(plen))
+    t_step = i32(tok[:, 30])
+    l0 = gp.gpt2_kernel_launches()
+    a = cache.step(t_step, i32(plen)).clone()
+    assert gp.gpt2_kernel_launches() - l0 == 2 + 5 * oc.n_layer
+    b = cache.step(t_step, i32(plen)).clone()  # the same cache rows rewritten with the same values
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert model.status() == 0
