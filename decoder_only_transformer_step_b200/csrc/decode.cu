@@ -47,9 +47,8 @@ DEVI float4 ld4f(const bf16* p) {
 DEVI float4 ld4f(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
 // Weights are read once per step: keep them out of L1.  Volatile, with a
-// memory clobber, so that it stays after the kernel's grid-dependency wait
-// (a plain asm is free to move, and an earlier kernel still in flight may be
-// writing the weights).
+// memory clobber, so that each load stays on the side of the kernel's
+// grid-dependency wait where the code puts it (a plain asm is free to move).
 DEVI uint4 ld_stream16(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -190,8 +189,13 @@ __global__ void __launch_bounds__(GV_WARPS * 32) decode_gemv_kernel(const __grid
         wv[u][c] = k < K ? ld_stream16(w0 + (size_t)c * K + k) : make_uint4(0u, 0u, 0u, 0u);
     }
   };
-  pdl_start();
+  // The first weight chunk is loaded before the grid-dependency wait: no
+  // kernel of the decode step writes weights, and the step's first kernel
+  // (the embedding) lets its successors start only after every kernel before
+  // the step has finished.  The loads then overlap the predecessor's tail.
+  pdl_trigger();
   if (blockIdx.x * gpc + gi < groups) load_chunk(blockIdx.x * gpc + gi, si);
+  pdl_wait();
 
   // Input rows -> shared memory as T.  Every load of a row is issued before
   // the first use (one memory round trip per row): 16-byte loads, the
@@ -393,7 +397,10 @@ template <typename T>
 __global__ void embed_decode_kernel(const int32_t* tok, const int32_t* pos,
                                     const T* wte, const T* wpe, float* __restrict__ x,
                                     int d, int vocab_real, int limit, int* err) {
-  pdl_start();
+  // wait before letting the step's kernels start: they load weights before
+  // their own waits, and a kernel before the step may still be writing them
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   int id = tok[r], p = pos[r];
   if (id < 0 || id >= vocab_real) {
@@ -424,32 +431,60 @@ __global__ void __launch_bounds__(AD_WARPS * 32)
                        float scale_log2) {
   __shared__ float sm_m[AD_WARPS], sm_l[AD_WARPS];
   __shared__ float sm_o[AD_WARPS][HD];
-  pdl_start();
+  pdl_trigger();
   const int h = blockIdx.x, r = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = H * HD;
+  // positions come from before the step (the step's first kernel waited for
+  // their writers), and so do the cached rows of positions < p: the warp's
+  // first tile of those is loaded ahead of the grid-dependency wait; row p
+  // (written by the QKV product just before) and q only after it
   int p = pos[r];
   p = p < 0 ? 0 : (p >= max_len ? max_len - 1 : p);  // out of range: flagged by the embedding
   const int n = p + 1;
   constexpr int VN = V16<T>::N;
+  const size_t plane = ((size_t)r * H + h) * max_len * HD;
+  const T* kb = kc + plane;
+  const T* vb = vc + plane;
+  // (bf16 rows: the fp32 rows of the correctness mode do not fit twice in registers)
+  constexpr bool PRE = sizeof(T) == 2;
+  const int j0 = warp * 32 + lane;
+  const bool early = PRE && j0 < p;
+  uint4 kr0[HD / VN], vr0[HD / VN];
+  if (early) {
+#pragma unroll
+    for (int c = 0; c < HD / VN; ++c) kr0[c] = *reinterpret_cast<const uint4*>(kb + (size_t)j0 * HD + c * VN);
+#pragma unroll
+    for (int c = 0; c < HD / VN; ++c) vr0[c] = *reinterpret_cast<const uint4*>(vb + (size_t)j0 * HD + c * VN);
+  }
+  pdl_wait();
   float qf[HD];
 #pragma unroll
   for (int i = 0; i < HD; i += 4) {
     const float4 v = *reinterpret_cast<const float4*>(q + (size_t)r * d + h * HD + i);
     qf[i] = v.x * scale_log2; qf[i + 1] = v.y * scale_log2; qf[i + 2] = v.z * scale_log2; qf[i + 3] = v.w * scale_log2;
   }
-  const size_t plane = ((size_t)r * H + h) * max_len * HD;
-  const T* kb = kc + plane;
-  const T* vb = vc + plane;
   float m = -INFINITY, l = 0.f, acc[HD];
 #pragma unroll
   for (int e = 0; e < HD; ++e) acc[e] = 0.f;
   for (int t = warp; t * 32 < n; t += AD_WARPS) {
     const int j = t * 32 + lane;
     const int jr = j < n ? j : n - 1;  // rows past n are read in bounds and weighted 0
-    uint4 kr[HD / VN];
+    uint4 kr[HD / VN], vr[HD / VN];
+    if (t == warp && early) {
 #pragma unroll
-    for (int c = 0; c < HD / VN; ++c) kr[c] = *reinterpret_cast<const uint4*>(kb + (size_t)jr * HD + c * VN);
+      for (int c = 0; c < HD / VN; ++c) {
+        kr[c] = kr0[c];
+        vr[c] = vr0[c];
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < HD / VN; ++c) kr[c] = *reinterpret_cast<const uint4*>(kb + (size_t)jr * HD + c * VN);
+      if constexpr (PRE) {
+#pragma unroll
+        for (int c = 0; c < HD / VN; ++c) vr[c] = *reinterpret_cast<const uint4*>(vb + (size_t)jr * HD + c * VN);
+      }
+    }
     float s = 0.f;
 #pragma unroll
     for (int c = 0; c < HD / VN; ++c) {
@@ -467,7 +502,7 @@ __global__ void __launch_bounds__(AD_WARPS * 32)
 #pragma unroll
     for (int c = 0; c < HD / VN; ++c) {
       float vf[VN];
-      V16<T>::unpack(*reinterpret_cast<const uint4*>(vb + (size_t)jr * HD + c * VN), vf);
+      V16<T>::unpack(PRE ? vr[c] : *reinterpret_cast<const uint4*>(vb + (size_t)jr * HD + c * VN), vf);
 #pragma unroll
       for (int e = 0; e < VN; ++e) acc[c * VN + e] = fmaf(pj, vf[e], acc[c * VN + e] * alpha);
     }
