@@ -327,14 +327,22 @@ __global__ void __launch_bounds__(GV_WARPS * 32) decode_gemv_kernel(const __grid
           float wf[GV_COLS][VN];
 #pragma unroll
           for (int c = 0; c < GV_COLS; ++c) V16<T>::unpack(wv[u][c], wf[c]);
+          // two rows per packed fp32x2 multiply-add (each lane of the pair
+          // rounds like fmaf, in the same order: the sums are unchanged)
 #pragma unroll
-          for (int r = 0; r < ROWS; ++r) {
-            float xf[VN];
-            V16<T>::unpack(*reinterpret_cast<const uint4*>(xs + (size_t)r * K + k), xf);
+          for (int r = 0; r < ROWS; r += 2) {
+            float xa[VN], xb[VN];
+            V16<T>::unpack(*reinterpret_cast<const uint4*>(xs + (size_t)r * K + k), xa);
+            V16<T>::unpack(*reinterpret_cast<const uint4*>(xs + (size_t)(r + 1) * K + k), xb);
 #pragma unroll
-            for (int c = 0; c < GV_COLS; ++c)
+            for (int c = 0; c < GV_COLS; ++c) {
+              float2 a2 = make_float2(acc[c * ROWS + r], acc[c * ROWS + r + 1]);
 #pragma unroll
-              for (int e = 0; e < VN; ++e) acc[c * ROWS + r] = fmaf(wf[c][e], xf[e], acc[c * ROWS + r]);
+              for (int e = 0; e < VN; ++e)
+                a2 = __ffma2_rn(make_float2(wf[c][e], wf[c][e]), make_float2(xa[e], xb[e]), a2);
+              acc[c * ROWS + r] = a2.x;
+              acc[c * ROWS + r + 1] = a2.y;
+            }
           }
         }
       }
