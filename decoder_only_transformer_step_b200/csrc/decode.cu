@@ -11,6 +11,9 @@
 // all rows held in shared memory, and fuse the LayerNorm in front of them and
 // the bias / GELU / residual / cache write behind them.  Attention of the new
 // query against the cached keys and values runs one block per (head, row).
+#include <stdlib.h>
+#include <string.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -149,6 +152,105 @@ DEVI void ln_store4(T* dst, float4 x, float4 g, float4 b, float mu, float rs) {
   dst[3] = from_f<T>((x.w - mu) * rs * g.w + b.w);
 }
 
+// Input rows -> shared memory as T, row pitch ld elements (rows past a.rows
+// zero).  Every load of a row is issued before the first use (one memory
+// round trip per row): 16-byte loads, the LayerNorm's row held in registers
+// for its two statistics.  nw warps take the rows of the LayerNorm.
+template <typename T, int ROWS, bool LN>
+DEVI void gemv_stage_rows(const GemvArgs& a, T* xs, int ld, int warp, int lane, int nw) {
+  const int K = a.K;
+  constexpr int VN = V16<T>::N;
+  if constexpr (LN) {
+    constexpr int NC = LN_MAX_K / 128;  // float4 pieces per lane (widest row)
+    constexpr int NC_FAST = 8;          // rows up to 1024 wide
+    const T* g = reinterpret_cast<const T*>(a.ln_g);
+    const T* b = reinterpret_cast<const T*>(a.ln_b);
+    const int K4 = K / 4;
+    for (int r = warp; r < ROWS; r += nw) {
+      T* dst = xs + (size_t)r * ld;
+      if (r >= a.rows) {
+        for (int k = lane; k < K; k += 32) dst[k] = from_f<T>(0.f);
+        continue;
+      }
+      const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.in) + (size_t)r * K);
+      if (K4 <= 32 * NC_FAST) {
+        // the row and its gains and shifts in one round trip
+        float4 v[NC_FAST], gv[NC_FAST], bv[NC_FAST];
+#pragma unroll
+        for (int c = 0; c < NC_FAST; ++c) {
+          const int i = lane + 32 * c;
+          const bool in = i < K4;
+          v[c] = in ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+          gv[c] = in ? ld4f(g + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+          bv[c] = in ? ld4f(b + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float mu, rs;
+        ln_stats<NC_FAST>(v, lane, K4, K, &mu, &rs);
+#pragma unroll
+        for (int c = 0; c < NC_FAST; ++c) {
+          const int i = lane + 32 * c;
+          if (i < K4) ln_store4(dst + 4 * i, v[c], gv[c], bv[c], mu, rs);
+        }
+      } else {
+        // wide rows: the row in registers, gains and shifts a few pieces at a time
+        float4 v[NC];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          const int i = lane + 32 * c;
+          v[c] = i < K4 ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float mu, rs;
+        ln_stats<NC>(v, lane, K4, K, &mu, &rs);
+#pragma unroll 4
+        for (int c = 0; c < NC; ++c) {
+          const int i = lane + 32 * c;
+          if (i < K4) ln_store4(dst + 4 * i, v[c], ld4f(g + 4 * i), ld4f(b + 4 * i), mu, rs);
+        }
+      }
+    }
+  } else if (a.in_t) {
+    // rows already in T: 16-byte copies, GV_STAGE of them in flight per thread
+    const int KV = K / VN, n16 = ROWS * KV, nthr = nw * 32;
+    const uint4* src = reinterpret_cast<const uint4*>(a.in);
+    for (int i0 = threadIdx.x; i0 < n16; i0 += GV_STAGE * nthr) {
+      uint4 v[GV_STAGE];
+#pragma unroll
+      for (int u = 0; u < GV_STAGE; ++u) {
+        const int i = i0 + u * nthr;
+        v[u] = (i < n16 && i / KV < a.rows) ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < GV_STAGE; ++u) {
+        const int i = i0 + u * nthr, r = i / KV;
+        if (i < n16) *reinterpret_cast<uint4*>(xs + (size_t)r * ld + (size_t)(i - r * KV) * VN) = v[u];
+      }
+    }
+  } else {
+    const int K4 = K / 4, n4 = ROWS * K4, nthr = nw * 32;
+    const float4* src = reinterpret_cast<const float4*>(a.in);
+    for (int i0 = threadIdx.x; i0 < n4; i0 += GV_STAGE * nthr) {
+      float4 v[GV_STAGE];
+#pragma unroll
+      for (int u = 0; u < GV_STAGE; ++u) {
+        const int i = i0 + u * nthr;
+        v[u] = (i < n4 && i / K4 < a.rows) ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < GV_STAGE; ++u) {
+        const int i = i0 + u * nthr;
+        if (i < n4) {
+          const int r = i / K4;
+          T* d = xs + (size_t)r * ld + 4 * (i - r * K4);
+          d[0] = from_f<T>(v[u].x);
+          d[1] = from_f<T>(v[u].y);
+          d[2] = from_f<T>(v[u].z);
+          d[3] = from_f<T>(v[u].w);
+        }
+      }
+    }
+  }
+}
+
 // out[r, n] = epi(sum_k in'[r, k] W[n, k]) for r < rows, n < N, where in' is
 // the input row (LN = true: its LayerNorm with eps 1e-5 and biased variance)
 // rounded to T.  Each warp takes GV_COLS consecutive columns per pass; lane l
@@ -197,96 +299,7 @@ __global__ void __launch_bounds__(GV_WARPS * 32) decode_gemv_kernel(const __grid
   if (blockIdx.x * gpc + gi < groups) load_chunk(blockIdx.x * gpc + gi, si);
   pdl_wait();
 
-  // Input rows -> shared memory as T.  Every load of a row is issued before
-  // the first use (one memory round trip per row): 16-byte loads, the
-  // LayerNorm's row held in registers for its two statistics.
-  if constexpr (LN) {
-    constexpr int NC = LN_MAX_K / 128;  // float4 pieces per lane (widest row)
-    constexpr int NC_FAST = 8;          // rows up to 1024 wide
-    const T* g = reinterpret_cast<const T*>(a.ln_g);
-    const T* b = reinterpret_cast<const T*>(a.ln_b);
-    const int K4 = K / 4;
-    for (int r = warp; r < ROWS; r += nw) {
-      T* dst = xs + (size_t)r * K;
-      if (r >= a.rows) {
-        for (int k = lane; k < K; k += 32) dst[k] = from_f<T>(0.f);
-        continue;
-      }
-      const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.in) + (size_t)r * K);
-      if (K4 <= 32 * NC_FAST) {
-        // the row and its gains and shifts in one round trip
-        float4 v[NC_FAST], gv[NC_FAST], bv[NC_FAST];
-#pragma unroll
-        for (int c = 0; c < NC_FAST; ++c) {
-          const int i = lane + 32 * c;
-          const bool in = i < K4;
-          v[c] = in ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-          gv[c] = in ? ld4f(g + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
-          bv[c] = in ? ld4f(b + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        float mu, rs;
-        ln_stats<NC_FAST>(v, lane, K4, K, &mu, &rs);
-#pragma unroll
-        for (int c = 0; c < NC_FAST; ++c) {
-          const int i = lane + 32 * c;
-          if (i < K4) ln_store4(dst + 4 * i, v[c], gv[c], bv[c], mu, rs);
-        }
-      } else {
-        // wide rows: the row in registers, gains and shifts a few pieces at a time
-        float4 v[NC];
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-          const int i = lane + 32 * c;
-          v[c] = i < K4 ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        float mu, rs;
-        ln_stats<NC>(v, lane, K4, K, &mu, &rs);
-#pragma unroll 4
-        for (int c = 0; c < NC; ++c) {
-          const int i = lane + 32 * c;
-          if (i < K4) ln_store4(dst + 4 * i, v[c], ld4f(g + 4 * i), ld4f(b + 4 * i), mu, rs);
-        }
-      }
-    }
-  } else if (a.in_t) {
-    // rows already in T: 16-byte copies, GV_STAGE of them in flight per thread
-    const int KV = K / VN, n16 = ROWS * KV, nthr = nw * 32;
-    const uint4* src = reinterpret_cast<const uint4*>(a.in);
-    uint4* dst = reinterpret_cast<uint4*>(xs);
-    for (int i0 = threadIdx.x; i0 < n16; i0 += GV_STAGE * nthr) {
-      uint4 v[GV_STAGE];
-#pragma unroll
-      for (int u = 0; u < GV_STAGE; ++u) {
-        const int i = i0 + u * nthr;
-        v[u] = (i < n16 && i / KV < a.rows) ? src[i] : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int u = 0; u < GV_STAGE; ++u)
-        if (i0 + u * nthr < n16) dst[i0 + u * nthr] = v[u];
-    }
-  } else {
-    const int K4 = K / 4, n4 = ROWS * K4, nthr = nw * 32;
-    const float4* src = reinterpret_cast<const float4*>(a.in);
-    for (int i0 = threadIdx.x; i0 < n4; i0 += GV_STAGE * nthr) {
-      float4 v[GV_STAGE];
-#pragma unroll
-      for (int u = 0; u < GV_STAGE; ++u) {
-        const int i = i0 + u * nthr;
-        v[u] = (i < n4 && i / K4 < a.rows) ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < GV_STAGE; ++u) {
-        const int i = i0 + u * nthr;
-        if (i < n4) {
-          T* d = xs + (size_t)4 * i;
-          d[0] = from_f<T>(v[u].x);
-          d[1] = from_f<T>(v[u].y);
-          d[2] = from_f<T>(v[u].z);
-          d[3] = from_f<T>(v[u].w);
-        }
-      }
-    }
-  }
+  gemv_stage_rows<T, ROWS, LN>(a, xs, K, warp, lane, nw);
   __syncthreads();
 
   // passes over the column groups, uniform across the block (the slices of a
@@ -391,6 +404,173 @@ __global__ void __launch_bounds__(GV_WARPS * 32) decode_gemv_kernel(const __grid
           reinterpret_cast<T*>(a.out)[(size_t)r * a.ldo + n] = from_f<T>(gelu_f<false>(v));
         } else {
           outf[(size_t)r * a.ldo + n] = v;
+        }
+      }
+    }
+    // the next pass overwrites red only after every slice-0 warp has read it
+    if constexpr (KS > 1) __syncthreads();
+  }
+}
+
+// ------------------------------------------------------ tensor-core GEMV --
+// The same products for bf16 and at most 8 rows on mma.sync m16n8k16: the
+// weights are the A operand (16 weight rows, i.e. 16 output columns, per
+// warp), the staged rows the B operand (N 8; rows past a.rows are zero).  Per
+// 32 k-elements a lane loads 16 bytes of each of its two weight rows (g and
+// g + 8 of the warp's 16, g = lane / 4) and the 16 bytes of staged row g at
+// the same k; within those 32 elements both operands take the same
+// permutation of the fragment's k order (lane quad t holds elements 8t ..
+// 8t + 7; the first mma reads 8t .. 8t + 3 of each, the second 8t + 4 ..
+// 8t + 7), so the loads are the fragments as they stand.  Each (column, row)
+// total ends on one lane, with no cross-lane reduction; KS warps split a
+// group's k range and add their parts in shared memory in a fixed order.  At
+// 8 rows a weight element feeds 8 products, so the dot products would
+// otherwise cost as many CUDA-core instructions as the weight stream allows
+// loads; on the tensor core they are a few instructions per 32 elements.
+constexpr int MG_COLS = 16;  // output columns per warp (the mma M)
+constexpr int MG_KC = 32;    // k elements per lane load of a weight row
+constexpr int MG_U = 4;      // k chunks of weight loads in flight per batch
+constexpr int MG_PAD = 32;   // elements (64 bytes) after each staged row: the 8
+                             // rows' 16-byte fragment loads then avoid bank conflicts
+
+DEVI void gemv_mma(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <bool LN, int EPI, int KS>
+__global__ void __launch_bounds__(GV_WARPS * 32) decode_gemv_mma_kernel(const __grid_constant__ GemvArgs a) {
+  extern __shared__ __align__(16) uint8_t dec_smem[];
+  constexpr int GPB = GV_WARPS / KS;  // column groups per block and pass
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int K = a.K, ld = K + MG_PAD;
+  bf16* xs = reinterpret_cast<bf16*>(dec_smem);                              // [8][ld]
+  float* red = reinterpret_cast<float*>(dec_smem + (size_t)8 * ld * sizeof(bf16));  // [warps][32][4]
+  const bf16* W = reinterpret_cast<const bf16*>(a.W);
+  const int groups = a.N / MG_COLS;
+  const int gi = warp / KS, si = warp % KS;
+  const int nch = K / MG_KC;
+  const int c0 = si * nch / KS, c1 = (si + 1) * nch / KS;  // this warp's k chunks
+  const int nb = (c1 - c0 + MG_U - 1) / MG_U;              // batches of them per group
+  uint4 wa[MG_U], wb[MG_U], na[MG_U], nb_[MG_U];
+  // batch b of group grp: chunks c0 + MG_U b + u < c1, rows g and g + 8
+  auto load_batch = [&](uint4 (&x0)[MG_U], uint4 (&x1)[MG_U], int grp, int b) {
+    const bf16* w0 = W + (size_t)(grp * MG_COLS + g) * K + 8 * t;
+    const bf16* w1 = w0 + (size_t)8 * K;
+#pragma unroll
+    for (int u = 0; u < MG_U; ++u) {
+      const int ch = c0 + b * MG_U + u;
+      if (ch < c1) {
+        x0[u] = ld_stream16(w0 + ch * MG_KC);
+        x1[u] = ld_stream16(w1 + ch * MG_KC);
+      }
+    }
+  };
+  // The first batch is requested before the grid-dependency wait, as in
+  // decode_gemv_kernel (no kernel of the decode step writes weights).
+  pdl_trigger();
+  if (blockIdx.x * GPB + gi < groups && nb > 0) load_batch(wa, wb, blockIdx.x * GPB + gi, 0);
+  pdl_wait();
+  gemv_stage_rows<bf16, 8, LN>(a, xs, ld, warp, lane, GV_WARPS);
+  __syncthreads();
+
+  for (int pass_base = blockIdx.x * GPB; pass_base < groups; pass_base += gridDim.x * GPB) {
+    const int grp = pass_base + gi;
+    const bool active = grp < groups;
+    const int n0 = grp * MG_COLS;
+    // the epilogue's operands (bias, old residual, cache positions) of this
+    // lane's outputs (columns n0 + g, n0 + g + 8; rows 2t, 2t + 1), loaded
+    // now so that their latency hides behind the products
+    float pre_b[2] = {0.f, 0.f}, pre_x[4] = {0.f, 0.f, 0.f, 0.f};
+    int pre_p[2] = {0, 0};
+    if (active && si == 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int n = n0 + g + 8 * h;
+        if constexpr (EPI != DEC_LOGITS) pre_b[h] = to_f(reinterpret_cast<const bf16*>(a.bias)[n]);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int r = 2 * t + j;
+          if constexpr (EPI == DEC_RESID)
+            if (r < a.rows) pre_x[2 * h + j] = reinterpret_cast<const float*>(a.out)[(size_t)r * a.ldo + n];
+        }
+      }
+      if constexpr (EPI == DEC_QKV) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) pre_p[j] = 2 * t + j < a.rows ? a.pos[2 * t + j] : 0;
+      }
+    }
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    if (active) {
+      for (int b = 0; b < nb; ++b) {
+        // the next batch (of this group, else the first of this warp's next
+        // group) is requested before this one is used
+        const int ngrp = grp + (int)gridDim.x * GPB;
+        if (b + 1 < nb)
+          load_batch(na, nb_, grp, b + 1);
+        else if (ngrp < groups)
+          load_batch(na, nb_, ngrp, 0);
+#pragma unroll
+        for (int u = 0; u < MG_U; ++u) {
+          const int ch = c0 + b * MG_U + u;
+          if (ch < c1) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(xs + (size_t)g * ld + ch * MG_KC + 8 * t);
+            gemv_mma(c, wa[u].x, wb[u].x, wa[u].y, wb[u].y, xv.x, xv.y);
+            gemv_mma(c, wa[u].z, wb[u].z, wa[u].w, wb[u].w, xv.z, xv.w);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < MG_U; ++u) {
+          wa[u] = na[u];
+          wb[u] = nb_[u];
+        }
+      }
+    }
+    if constexpr (KS > 1) {
+      *reinterpret_cast<float4*>(red + (warp * 32 + lane) * 4) = make_float4(c[0], c[1], c[2], c[3]);
+      __syncthreads();
+      if (si == 0) {
+#pragma unroll
+        for (int x = 1; x < KS; ++x) {
+          const float4 q = *reinterpret_cast<const float4*>(red + ((warp + x) * 32 + lane) * 4);
+          c[0] += q.x;
+          c[1] += q.y;
+          c[2] += q.z;
+          c[3] += q.w;
+        }
+      }
+    }
+    if (active && si == 0) {
+      // c[i]: column n0 + g + 8 (i / 2), row 2t + i % 2
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int h = i >> 1, r = 2 * t + (i & 1);
+        if (r >= a.rows) continue;
+        const int n = n0 + g + 8 * h;
+        const float v = c[i] + pre_b[h];
+        float* outf = reinterpret_cast<float*>(a.out);
+        if constexpr (EPI == DEC_QKV) {
+          if (n < a.d) {
+            outf[(size_t)r * a.ldo + n] = v;
+          } else {
+            const int kind = n >= 2 * a.d;
+            const int nn = n - a.d - kind * a.d;
+            const int p = pre_p[i & 1];
+            if (p >= 0 && p < a.max_len) {
+              bf16* plane = reinterpret_cast<bf16*>(kind ? a.vc : a.kc);
+              plane[(((size_t)r * a.H + nn / a.hd) * a.max_len + p) * a.hd + nn % a.hd] = from_f<bf16>(v);
+            }
+          }
+        } else if constexpr (EPI == DEC_RESID) {
+          outf[(size_t)r * a.ldo + n] = pre_x[i] + v;
+        } else if constexpr (EPI == DEC_GELU) {
+          reinterpret_cast<bf16*>(a.out)[(size_t)r * a.ldo + n] = from_f<bf16>(gelu_f<false>(v));
+        } else {
+          outf[(size_t)r * a.ldo + n] = c[i];
         }
       }
     }
@@ -774,6 +954,34 @@ int gemv_rows(const GemvArgs& a, cudaStream_t st) {
   return gemv_launch<T, 16, LN, EPI, KS>(a, st);
 }
 
+template <bool LN, int EPI, int KS>
+int gemv_mma_launch(const GemvArgs& a, cudaStream_t st) {
+  const size_t smem = (size_t)8 * (a.K + MG_PAD) * sizeof(bf16) + (size_t)GV_WARPS * 32 * 16;
+  CUDA_TRY(cudaFuncSetAttribute(decode_gemv_mma_kernel<LN, EPI, KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                227 * 1024));
+  constexpr int GPB = GV_WARPS / KS;
+  const int groups = a.N / MG_COLS;
+  int grid = (groups + GPB - 1) / GPB;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_gemv_mma_kernel<LN, EPI, KS>, GV_WARPS * 32, smem) !=
+          cudaSuccess || occ < 1)
+    occ = 1;
+  if (grid > occ * num_sms()) grid = occ * num_sms();  // one resident wave
+  CUDA_TRY(launch_k(decode_gemv_mma_kernel<LN, EPI, KS>, grid, GV_WARPS * 32, smem, st, a));
+  LAUNCH_CHECK();
+  return GPT2_OK;
+}
+
+// the k split: all 8 warps of a block on one 16-column group while the
+// groups fit one block per SM, fewer as they grow
+template <bool LN, int EPI>
+int gemv_mma_ks(const GemvArgs& a, cudaStream_t st) {
+  const int groups = a.N / MG_COLS;
+  if (groups <= num_sms()) return gemv_mma_launch<LN, EPI, 8>(a, st);
+  if (groups <= 2 * num_sms()) return gemv_mma_launch<LN, EPI, 4>(a, st);
+  return gemv_mma_launch<LN, EPI, 2>(a, st);
+}
+
 template <typename T>
 int gemv_dispatch(const GemvArgs& a, bool ln, int epi, cudaStream_t st) {
   // the residual products have narrow outputs (d columns): k split four ways
@@ -812,6 +1020,16 @@ int decode_gemv(int f32, const DecodeGemv& g, cudaStream_t st) {
   a.in = g.in; a.in_t = g.in_t; a.W = g.W; a.bias = g.bias; a.ln_g = g.ln_g; a.ln_b = g.ln_b;
   a.out = g.out; a.ldo = g.ldo; a.rows = g.rows; a.N = g.N; a.K = g.K;
   a.kc = g.kc; a.vc = g.vc; a.pos = g.pos; a.d = g.d; a.H = g.H; a.hd = g.hd; a.max_len = g.max_len;
+  // bf16 at up to 8 rows: the tensor-core GEMV ("simt" in GPT2_DECODE_GEMV
+  // selects the CUDA-core kernel, for comparison)
+  const char* e = getenv("GPT2_DECODE_GEMV");
+  if (!f32 && g.rows <= 8 && g.N % MG_COLS == 0 && !(e && !strcmp(e, "simt"))) {
+    if (g.epi == DEC_QKV && g.ln) return gemv_mma_ks<true, DEC_QKV>(a, st);
+    if (g.epi == DEC_RESID && !g.ln) return gemv_mma_ks<false, DEC_RESID>(a, st);
+    if (g.epi == DEC_GELU && g.ln) return gemv_mma_ks<true, DEC_GELU>(a, st);
+    if (g.epi == DEC_LOGITS && g.ln) return gemv_mma_ks<true, DEC_LOGITS>(a, st);
+    return GPT2_ERR_INVALID_ARG;
+  }
   return f32 ? gemv_dispatch<float>(a, g.ln, g.epi, st) : gemv_dispatch<bf16>(a, g.ln, g.epi, st);
 }
 
