@@ -276,3 +276,50 @@ def test_decode_step_launch_count_and_repeatability():
     torch.cuda.synchronize()
     assert torch.equal(a, b)
     assert model.status() == 0
+
+
+@pytest.mark.parametrize("batch", [1, 8])
+def test_tensor_core_gemv_matches_cuda_core_gemv_and_oracle(batch):
+    # bf16 at up to 8 rows the decode GEMVs run on the tensor cores;
+    # GPT2_DECODE_GEMV=simt selects the CUDA-core kernel.  Both against the
+    # oracle's cache decoder and against each other (they differ only in
+    # summation order) over steps with the rows at different positions.
+    import os
+    oc = Config(n_layer=2, d_model=256, n_head=4, n_ctx=128, vocab=2048)
+    vocab_real = 2000
+    params = params_for(oc, seed=61)
+    model = make_model(oc, vocab_real, batch, 0)
+    p32 = load_params(model, params, oc)
+    max_len = 64
+    plen = (np.arange(batch, dtype=np.int32) * 7) % 30 + 1
+    tok, _ = inputs.uniform_tokens(batch, oc.n_ctx, vocab_real, seed=62)
+    out = {}
+    for kind in ("mma", "simt"):
+        old = os.environ.pop("GPT2_DECODE_GEMV", None)
+        if kind == "simt":
+            os.environ["GPT2_DECODE_GEMV"] = "simt"
+        try:
+            cache = gp.KVCache(model, batch, max_len)
+            cache.prefill(i32(tok), i32(plen))
+            pos, zs = plen.copy(), []
+            for step in range(4):
+                t_step = inputs.uniform_tokens(batch, 1, vocab_real, seed=300 + step)[0][:, 0]
+                zs.append(cache.step(i32(t_step), i32(pos)).cpu().numpy().astype(np.float64))
+                pos = pos + 1
+            torch.cuda.synchronize()
+        finally:
+            os.environ.pop("GPT2_DECODE_GEMV", None)
+            if old is not None:
+                os.environ["GPT2_DECODE_GEMV"] = old
+        assert model.status() == 0
+        out[kind] = zs
+    ref_cache = kv_cache_empty(oc, batch, max_len)
+    prefill(p32, oc, ref_cache, tok, plen)
+    pos = plen.copy()
+    for step in range(4):
+        t_step = inputs.uniform_tokens(batch, 1, vocab_real, seed=300 + step)[0][:, 0]
+        z_ref = decode_step(p32, oc, ref_cache, t_step, pos)
+        assert rel_err(out["mma"][step], z_ref) <= 2e-2, step
+        assert rel_err(out["simt"][step], z_ref) <= 2e-2, step
+        assert rel_err(out["mma"][step], out["simt"][step]) <= 5e-3, step
+        pos = pos + 1
