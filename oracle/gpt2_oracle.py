@@ -26,8 +26,8 @@ section):
   the padded ids take part in the softmax.
 
 The block structure (pre-LayerNorm, learned positions, causal multi-head
-attention, GELU MLP, LM head tied to the token embedding) is the GPT-2 step as
-the task states it.  Where the pages are silent this oracle takes the plainest
+attention, GELU MLP, LM head tied to the token embedding) is the GPT-2 model
+the pages train.  Where the pages are silent this oracle takes the plainest
 GPT-2 reading: tanh-form GELU, LayerNorm eps 1e-5 with biased variance,
 biases on every linear layer except the tied head, no dropout, softmax scale
 1/sqrt(head_dim), loss averaged over all B*T positions (over those with a
