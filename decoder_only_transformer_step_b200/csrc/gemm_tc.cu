@@ -124,7 +124,9 @@ int resolve_bn(int bn, int N) {
 // Split-K factor for an fp32 (weight-gradient) product with fewer output
 // tiles than co-resident CTAs (pairs): the s minimising an estimate of
 //   waves(tiles * s) * (k-blocks per unit) * (time of one k-block of a tile)
-//   + s * M * N * 8 bytes (partials written and read back) / HBM bandwidth,
+//   + s * M * N * 8 bytes (partials written and read back) / HBM bandwidth
+//   + (s > 3: the separate reduction launch; up to 3 splits are reduced
+//      inside the kernel),
 // which weighs wave quantisation against the partial-sum traffic.
 int auto_splits(int M, int N, int K, int bn) {
   const bool pair = bn == 512;
@@ -136,13 +138,14 @@ int auto_splits(int M, int N, int K, int bn) {
   // one k-block (64 deep) of one tile at ~11 TFLOP/s per SM, in microseconds
   const double kblock_us = 2.0 * 128 * tile_n * BK / 11e6;
   const double bytes_per_us = 6.5e6;  // HBM, bytes per microsecond
+  const double reduce_us = 4.0;       // a reduction launch: its set-up and tail
   int best = 1;
   double best_cost = 1e30;
   for (int s = 1; s <= 16 && s <= kb / 4; ++s) {
     const long units = tiles * s;
     const long waves = (units + slots - 1) / slots;
     const double cost = (double)waves * ((double)kb / s) * kblock_us +
-                        (s > 1 ? (double)s * M * N * 8.0 / bytes_per_us : 0.0);
+                        (s > 1 ? (double)s * M * N * 8.0 / bytes_per_us : 0.0) + (s > 3 ? reduce_us : 0.0);
     if (cost < best_cost * 0.999) {
       best_cost = cost;
       best = s;
