@@ -645,11 +645,9 @@ __global__ void attn_bwd_kv_f32_kernel(const float* qkv, const float* dout,
 template <int HD>
 int launch_fwd(const void* qkv, void* o, float* lse, int B, int T, int H, cudaStream_t st) {
   constexpr int smem = 128 * HD * 2 + 4 * 64 * HD * 2;
-  static bool attr = false;
-  if (!attr) {
-    CUDA_TRY(cudaFuncSetAttribute(attn_fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    attr = true;
-  }
+  CUDA_TRY(once_per_device((const void*)attn_fwd_kernel<HD>, [](int) {
+    return cudaFuncSetAttribute(attn_fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  }));
   dim3 grid((T + 127) / 128, B * H);
   const float scale_log2 = LOG2E_F / sqrtf((float)HD);
   CUDA_TRY(launch_k(attn_fwd_kernel<HD>, grid, 256, smem, st, (const bf16*)qkv, (bf16*)o, lse, T, H, scale_log2));
@@ -661,11 +659,9 @@ template <int HD>
 int launch_bwd(const void* qkv, const void* dout, const float* lse, const float* dvec, void* dqkv,
                float* dq_acc, int B, int T, int H, cudaStream_t st) {
   constexpr int smem = 6 * 64 * HD * 2 + 64 * 64 * 2 + 4 * 64 * 4;
-  static bool attr = false;
-  if (!attr) {
-    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    attr = true;
-  }
+  CUDA_TRY(once_per_device((const void*)attn_bwd_kernel<HD>, [](int) {
+    return cudaFuncSetAttribute(attn_bwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  }));
   dim3 grid((T + 63) / 64, B * H);
   const float scale = 1.f / sqrtf((float)HD);
   CUDA_TRY(launch_k(attn_bwd_kernel<HD>, grid, 128, smem, st,

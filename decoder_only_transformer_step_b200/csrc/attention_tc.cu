@@ -1623,9 +1623,11 @@ int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float
          : (cudaFuncGetAttributes(&fa, attn_bwd_tc2_kernel) == cudaSuccess && fa.numRegs == bw::LAUNCH_REGS) ? 1
                                                                                                              : 0;
     cudaGetLastError();
-    if (v2) CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bw::SMEM));
   }
   if (v2) {
+    CUDA_TRY(once_per_device((const void*)attn_bwd_tc2_kernel, [](int) {
+      return cudaFuncSetAttribute(attn_bwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bw::SMEM);
+    }));
     const int n_items = ((T + BKV - 1) / BKV) * B * H;
     const int grid = n_items < num_sms() ? n_items : num_sms();
     CUDA_TRY(launch_k(attn_bwd_tc2_kernel, grid, bw::THREADS, bw::SMEM, st, tq, tdo, tdq, tdqkv, lse, dvec, T, H,
@@ -1634,11 +1636,9 @@ int attn_bwd_tc(const void* qkv, const void* dout, const float* lse, const float
     return GPT2_OK;
   }
   if (dq_part) return GPT2_ERR_UNSUPPORTED_SHAPE;  // (a mode of the persistent kernel only)
-  static bool attr = false;
-  if (!attr) {
-    CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B_SMEM_BYTES));
-    attr = true;
-  }
+  CUDA_TRY(once_per_device((const void*)attn_bwd_tc_kernel, [](int) {
+    return cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, B_SMEM_BYTES);
+  }));
   dim3 grid((T + BKV - 1) / BKV, B * H);
   CUDA_TRY(launch_k(attn_bwd_tc_kernel, grid, B_NUM_THREADS, B_SMEM_BYTES, st, tq, tdo, tdq, tdqkv, lse, dvec, T, H,
                                                                  0.125f, LOG2E_F / 8.f, nullptr));
@@ -1666,9 +1666,11 @@ int attn_fwd_tc(const void* qkv, void* o, float* lse, int B, int T, int H, cudaS
          : (cudaFuncGetAttributes(&fa, attn_fwd_tc2_kernel) == cudaSuccess && fa.numRegs == F2_LAUNCH_REGS) ? 1
                                                                                                            : 0;
     cudaGetLastError();
-    if (v2) CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F2_SMEM));
   }
   if (v2) {
+    CUDA_TRY(once_per_device((const void*)attn_fwd_tc2_kernel, [](int) {
+      return cudaFuncSetAttribute(attn_fwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F2_SMEM);
+    }));
     const int nqb = (T + BQ - 1) / BQ;
     const int n_items = ((nqb + 1) / 2) * B * H;
     const int grid = n_items < num_sms() ? n_items : num_sms();
@@ -1677,11 +1679,9 @@ int attn_fwd_tc(const void* qkv, void* o, float* lse, int B, int T, int H, cudaS
     LAUNCH_CHECK();
     return GPT2_OK;
   }
-  static bool attr = false;
-  if (!attr) {
-    CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    attr = true;
-  }
+  CUDA_TRY(once_per_device((const void*)attn_fwd_tc_kernel, [](int) {
+    return cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  }));
   const int n_items = ((T + BQ - 1) / BQ) * B * H;
   const int grid = n_items < num_sms() ? n_items : num_sms();
   CUDA_TRY(launch_k(attn_fwd_tc_kernel, grid, NUM_THREADS, SMEM_BYTES, st,

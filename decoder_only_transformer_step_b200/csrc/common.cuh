@@ -7,6 +7,10 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <utility>
+#include <vector>
+
 #include "../../include/gpt2.h"
 
 typedef __nv_bfloat16 bf16;
@@ -453,6 +457,30 @@ DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 DEVI void pdl_start() {
   pdl_trigger();
   pdl_wait();
+}
+
+// ------------------------------------------------- per-device set-up --
+// Kernel attributes (and what the launchers derive from them, such as
+// occupancy) belong to the device that was current when they were set, and
+// a process may drive several devices: `set` runs once per (kernel, device).
+constexpr int MAX_DEVICES = 64;
+template <typename F>
+inline cudaError_t once_per_device(const void* func, F&& set) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& d : done)
+    if (d.first == func && d.second == dev) return cudaSuccess;
+  e = set(dev);
+  if (e == cudaSuccess) done.emplace_back(func, dev);
+  return e;
+}
+inline int current_device() {
+  int dev = 0;
+  return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < MAX_DEVICES ? dev : 0;
 }
 
 template <typename... KArgs, typename... Args>

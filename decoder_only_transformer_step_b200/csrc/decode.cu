@@ -921,12 +921,10 @@ template <typename T, int ROWS, bool LN, int EPI, int KS>
 int gemv_launch(const GemvArgs& a, cudaStream_t st) {
   constexpr int HELD = GV_COLS * ROWS >= 32 ? GV_COLS * ROWS / 32 : 1;
   const size_t smem = (size_t)ROWS * a.K * sizeof(T) + (KS > 1 ? (size_t)GV_WARPS * HELD * 32 * 4 : 0);
-  static bool attr = false;
-  if (!attr) {
-    CUDA_TRY(cudaFuncSetAttribute(decode_gemv_kernel<T, ROWS, LN, EPI, KS>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-    attr = true;
-  }
+  CUDA_TRY(once_per_device((const void*)decode_gemv_kernel<T, ROWS, LN, EPI, KS>, [](int) {
+    return cudaFuncSetAttribute(decode_gemv_kernel<T, ROWS, LN, EPI, KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                227 * 1024);
+  }));
   const int groups = a.N / GV_COLS;
   // narrow outputs: 4-warp blocks (or, with a k split, 8 warps on 2 groups),
   // so that more SMs stream weights
@@ -935,8 +933,8 @@ int gemv_launch(const GemvArgs& a, cudaStream_t st) {
   int grid = (groups + gpc - 1) / gpc;
   // at most one wave of resident blocks (the registers allow one 8-warp block
   // per SM): a second wave would repeat the input staging and add a tail
-  static int per_sm[2] = {0, 0};
-  int& occ = per_sm[nw == GV_WARPS];
+  static int per_sm[MAX_DEVICES][2] = {};
+  int& occ = per_sm[current_device()][nw == GV_WARPS];
   if (occ == 0 && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_gemv_kernel<T, ROWS, LN, EPI, KS>,
                                                                    nw * 32, smem) != cudaSuccess || occ < 1))
     occ = 1;
@@ -957,8 +955,10 @@ int gemv_rows(const GemvArgs& a, cudaStream_t st) {
 template <bool LN, int EPI, int KS>
 int gemv_mma_launch(const GemvArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)8 * (a.K + MG_PAD) * sizeof(bf16) + (size_t)GV_WARPS * 32 * 16;
-  CUDA_TRY(cudaFuncSetAttribute(decode_gemv_mma_kernel<LN, EPI, KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                227 * 1024));
+  CUDA_TRY(once_per_device((const void*)decode_gemv_mma_kernel<LN, EPI, KS>, [](int) {
+    return cudaFuncSetAttribute(decode_gemv_mma_kernel<LN, EPI, KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                227 * 1024);
+  }));
   constexpr int GPB = GV_WARPS / KS;
   const int groups = a.N / MG_COLS;
   int grid = (groups + GPB - 1) / GPB;

@@ -825,8 +825,7 @@ template <int BN, bool PAIR, int EK>
 int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tc2,
               const TcParams& p, int units, cudaStream_t st) {
   using C = TcCfg<BN, PAIR, EK>;
-  static bool attr_set = false;
-  static int max_slots = 0;  // co-resident CTAs (single) or clusters (pairs)
+  static int max_slots_dev[MAX_DEVICES] = {0};  // co-resident CTAs (single) or clusters (pairs)
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -843,22 +842,22 @@ int launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& t
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
   }
-  if (!attr_set) {
-    CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, PAIR, EK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  C::SMEM_BYTES));
+  CUDA_TRY(once_per_device((const void*)gemm_tc_kernel<BN, PAIR, EK>, [&](int dev) -> cudaError_t {
+    const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, PAIR, EK>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    int n = num_sms();
     if (PAIR) {
       cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
-      int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<BN, PAIR, EK>, &cfg) != cudaSuccess || n <= 0) {
         cudaGetLastError();
         n = num_sms() / 2;
       }
-      max_slots = n;
-    } else {
-      max_slots = num_sms();
     }
-    attr_set = true;
-  }
+    max_slots_dev[dev < MAX_DEVICES ? dev : 0] = n;
+    return cudaSuccess;
+  }));
+  const int max_slots = max_slots_dev[current_device()];
   const int slots = units < max_slots ? units : max_slots;
   cfg.gridDim = dim3((PAIR ? 2 : 1) * slots, 1, 1);
   CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, PAIR, EK>, ta, tb, tc, tc2, p));
