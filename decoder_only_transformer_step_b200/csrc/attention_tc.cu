@@ -444,6 +444,14 @@ static_assert(128 * F2_REGS_CTRL + 256 * F2_REGS_SOFT <= F2_THREADS * F2_LAUNCH_
 template <int N> DEVI void reg_dealloc() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 template <int N> DEVI void reg_alloc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 
+// max(a, b, c): the three-operand form of max.f32 (NaN operands are
+// ignored as by fmaxf), half the instructions of a pairwise row maximum.
+DEVI float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __global__ void __launch_bounds__(F2_THREADS, 1)
     attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmO,
                         float* __restrict__ lse, int T, int H, int n_items, float scale_log2, int* err) {
@@ -680,14 +688,13 @@ __global__ void __launch_bounds__(F2_THREADS, 1)
             for (int i = 0; i < 32; ++i) {
               const float x = (32 * c + i > row) ? -INFINITY : __uint_as_float(v[c][i]);
               v[c][i] = __float_as_uint(x);
-              mxs[i & 7] = fmaxf(mxs[i & 7], x);
             }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; ++i) mxs[i & 7] = fmaxf(mxs[i & 7], __uint_as_float(v[c][i]));
         }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            mxs[(i >> 1) & 7] = fmax3(mxs[(i >> 1) & 7], __uint_as_float(v[c][i]), __uint_as_float(v[c][i + 1]));
         const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
                                fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
         const float m_new = fmaxf(m_use, mx * scale_log2);
