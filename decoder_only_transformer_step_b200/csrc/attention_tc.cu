@@ -1461,46 +1461,66 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t box = base + SM_DQ + (uint32_t)q * 4096u;
     bool ok = true;
-    // -LSE (log2 domain) and -D of query block t of item (kb, b, h) into
-    // ring slot r (queries past T: -LSE = -inf, -D = 0), negated so the
-    // elementwise warps need one fused multiply-add and one add per pair
-    auto stage_ld = [&](int g, int kb, int b, int h, int t) -> bool {
+    // -LSE (log2 domain) and -D of a query block into its ring slot (queries
+    // past T: -LSE = -inf, -D = 0), negated so the elementwise warps need one
+    // fused multiply-add and one add per pair.  Staged two query blocks ahead
+    // along this CTA's sequence of (item, query block): the global loads of
+    // block g + 2 are issued before block g's dQ drain and written to the ring
+    // after it, so their latency overlaps the drain instead of preceding it.
+    int ks = 0, ts = 0, kbs = 0, bs = 0, hs = 0, nbs = 0;  // the staging cursor
+    bool have = false;
+    auto cursor_item = [&](int kk) {
+      const int w = snake_item(kk, (int)blockIdx.x, (int)gridDim.x);
+      have = w < n_items;
+      if (have) {
+        item(w, kbs, bs, hs);
+        nbs = nqb - kbs;
+        ks = kk;
+        ts = 0;
+      }
+    };
+    auto cursor_next = [&]() {
+      if (++ts >= nbs) cursor_item(ks + 1);
+    };
+    auto stage_load = [&](float& lv, float& dv) {
+      const int qq = (kbs + ts) * BQ + tid;
+      const long bh0 = ((long)bs * H + hs) * T;
+      lv = qq < T ? lse[bh0 + qq] : 0.f;
+      dv = qq < T ? dvec[bh0 + qq] : 0.f;
+    };
+    // the cursor's block, number g of the sequence, into ring slot g % QS
+    auto stage_store = [&](int g, float lv, float dv) -> bool {
       const int r = g % QS;
       if (g >= QS && !mbar_wait_bounded(ld_empty(r), ((g - QS) / QS) & 1, abort_flag, err)) return false;
-      const int qq = (kb + t) * BQ + tid;
-      const long bh0 = ((long)b * H + h) * T;
-      sLD[r * 256 + tid] = qq < T ? -lse[bh0 + qq] * LOG2E_F : -INFINITY;
-      sLD[r * 256 + 128 + tid] = qq < T ? -dvec[bh0 + qq] : 0.f;
+      const int qq = (kbs + ts) * BQ + tid;
+      sLD[r * 256 + tid] = qq < T ? -lv * LOG2E_F : -INFINITY;
+      sLD[r * 256 + 128 + tid] = qq < T ? -dv : 0.f;
       __syncwarp();
       if (lane == 0) mbar_arrive(ld_full(r));
       return true;
     };
-    int gq = 0, it = 0;
-    {
-      const int w = snake_item(0, (int)blockIdx.x, (int)gridDim.x);
-      if (w < n_items) {
-        int kb, b, h;
-        item(w, kb, b, h);
-        ok = stage_ld(0, kb, b, h, 0);
-      }
+    int staged = 0;  // query blocks staged so far
+    cursor_item(0);
+    for (int i = 0; i < 2 && have && ok; ++i) {
+      float lv, dv;
+      stage_load(lv, dv);
+      ok = stage_store(staged, lv, dv);
+      ++staged;
+      cursor_next();
     }
+    int gq = 0, it = 0;
     for (int k = 0; ok; ++k, ++it) {
       const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
       if (w >= n_items) break;
       int kb, b, h;
       item(w, kb, b, h);
       const int nblk = nqb - kb, slot = it & 1;
-      const int wn = snake_item(k + 1, (int)blockIdx.x, (int)gridDim.x);
       for (int t = 0; t < nblk; ++t) {
         const int g = gq + t;
-        // the next query block's LSE / D (of this item, or the next item's first)
-        if (t + 1 < nblk) {
-          if (!stage_ld(g + 1, kb, b, h, t + 1)) { ok = false; break; }
-        } else if (wn < n_items) {
-          int kb2, b2, h2;
-          item(wn, kb2, b2, h2);
-          if (!stage_ld(g + 1, kb2, b2, h2, 0)) { ok = false; break; }
-        }
+        // block g + 2's LSE / D: loaded now, written after this block's dQ drain
+        const bool pend = have;
+        float lv = 0.f, dv = 0.f;
+        if (pend) stage_load(lv, dv);
         // dQ of block g: tensor memory -> registers (the buffer is then free
         // for the next block's dQ) -> two 32 x 32 fp32 boxes -> TMA reduce-add
         // (bulk reductions into L2; per-lane vector reductions measured slower)
@@ -1538,6 +1558,11 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
               tma_reduce_add_3d(&tmDQ, box, h * HD + 32 * c, q0 + q * 32, b);
             bulk_commit();
           }
+        }
+        if (pend) {
+          if (!stage_store(staged, lv, dv)) { ok = false; break; }
+          ++staged;
+          cursor_next();
         }
       }
       if (!ok) break;
