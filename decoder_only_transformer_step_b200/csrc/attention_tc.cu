@@ -1288,17 +1288,9 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
     } else if (warp == 1 && lane == 0) {
       // ----------------------------------------------------------- MMA ----
       bool ok = true, issued_any = false;
-      int it = 0, gq = 0;
-      for (int k = 0; ok; ++k, ++it) {
-        const int w = snake_item(k, (int)blockIdx.x, (int)gridDim.x);
-        if (w >= n_items) break;
-        int kb, b, h;
-        item(w, kb, b, h);
-        const int nblk = nqb - kb, slot = it & 1;
-        if (!mbar_wait_bounded(kv_full(slot), (it >> 1) & 1, abort_flag, err)) { ok = false; break; }
-        const uint32_t kt = kv_tile(slot), vt = kt + TILE;
-        // S^T = K Q^T and dP^T = V dO^T of global query block g
-        auto issue_sdp = [&](int g) -> bool {
+      // S^T = K Q^T and dP^T = V dO^T of global query block g with the K / V
+      // tiles at kt, vt
+      auto issue_sdp = [&](int g, uint32_t kt, uint32_t vt) -> bool {
           const int r = g % QS;
           if (!mbar_wait_bounded(qdo_full(r), (g / QS) & 1, abort_flag, err)) return false;
           if (g >= 1 && !mbar_wait_bounded(st_free, (g - 1) & 1, abort_flag, err)) return false;
@@ -1315,11 +1307,31 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
           tc_commit(st_full);
           issued_any = true;
           return true;
-        };
-        if (!issue_sdp(gq)) { ok = false; break; }
+      };
+      int it = 0, gq = 0;
+      int w = snake_item(0, (int)blockIdx.x, (int)gridDim.x);
+      // the first item's K / V, and its first block's S^T, dP^T
+      if (w < n_items) {
+        ok = mbar_wait_bounded(kv_full(0), 0, abort_flag, err) && issue_sdp(0, kv_tile(0), kv_tile(0) + TILE);
+      }
+      for (int k = 0; ok && w < n_items; ++k, ++it) {
+        int kb, b, h;
+        item(w, kb, b, h);
+        const int nblk = nqb - kb, slot = it & 1;
+        const uint32_t kt = kv_tile(slot), vt = kt + TILE;
+        const int wn = snake_item(k + 1, (int)blockIdx.x, (int)gridDim.x);
         for (int t = 0; t < nblk; ++t) {
           const int g = gq + t, r = g % QS;
-          if (t + 1 < nblk && !issue_sdp(g + 1)) { ok = false; break; }
+          // the next block's S^T, dP^T ahead of this block's products; at the
+          // item's last block that is the next item's first block, so the
+          // elementwise warps do not wait out this block's products there
+          if (t + 1 < nblk) {
+            if (!issue_sdp(g + 1, kt, vt)) { ok = false; break; }
+          } else if (wn < n_items) {
+            const uint32_t kn = kv_tile(slot ^ 1);
+            if (!mbar_wait_bounded(kv_full(slot ^ 1), ((it + 1) >> 1) & 1, abort_flag, err) ||
+                !issue_sdp(g + 1, kn, kn + TILE)) { ok = false; break; }
+          }
           if (!mbar_wait_bounded(ps_full, g & 1, abort_flag, err)) { ok = false; break; }
           // the previous item's dK / dV have been read out of tensor memory
           if (t == 0 && it >= 1 && !mbar_wait_bounded(dkdv_free, (it - 1) & 1, abort_flag, err)) { ok = false; break; }
@@ -1352,6 +1364,7 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
         tc_commit(dkdv_full);
         tc_commit(kv_empty(slot));
         gq += nblk;
+        w = wn;
       }
       if (!ok && issued_any) {
         tc_commit(drain_bar);
