@@ -1138,13 +1138,13 @@ __global__ void __launch_bounds__(B_NUM_THREADS, 1)
 //   WG1, WG2  elementwise: P^T = exp(S^T - LSE), dS^T = P^T (dP^T - D) for
 //        64 query columns each; P^T goes to tensor memory (the dV product
 //        reads it there), dS^T to a shared tile                          (160)
-//   WG3  LSE/D staging one query block ahead, the dQ drain (tensor memory
+//   WG3  LSE/D staging two query blocks ahead, the dQ drain (tensor memory
 //        -> shared -> TMA reduce-add into the fp32 dQ accumulator) and the
 //        dK/dV write-out at the end of an item                          (112)
-// The MMA warp issues S^T, dP^T of the next query block as soon as the
-// elementwise warps have loaded the current ones, ahead of the current
-// block's dV, dK, dQ products, so the elementwise work of one block overlaps
-// the tensor-core work of the other.  Tensor memory: S^T 0-127, dP^T
+// The MMA warp issues S^T, dP^T of the next query block (the next item's
+// first at an item's last) as soon as the elementwise warps have loaded the
+// current ones, ahead of the current block's dV, dK, dQ products, so the
+// elementwise work of one block overlaps the tensor-core work of the other.  Tensor memory: S^T 0-127, dP^T
 // 128-255, P^T 256-319 (bf16 pairs), dV 320-383, dK 384-447, dQ 448-511.
 namespace bw {
 constexpr int QS = 3;  // Q/dO (and LSE/D) ring depth: loads run two query blocks ahead
