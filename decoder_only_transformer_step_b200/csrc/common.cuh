@@ -155,6 +155,21 @@ DEVI bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep until the phase completes or
+// hint_ns elapse, instead of polling.
+DEVI bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
+constexpr uint32_t WAIT_SLEEP_NS = 20000;
+
 // Bounded wait on an mbarrier phase.  Returns false (after raising the
 // shared abort flag and the device timeout bit) if the phase did not complete
 // within WAIT_TIMEOUT_NS, or if another role of the CTA already aborted.
@@ -162,11 +177,10 @@ DEVI bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_f
                             int* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer(), lim = g_wait_limit_ns;
-  uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, WAIT_SLEEP_NS)) return true;
     if (*abort_flag) return false;
-    if ((++spins & 63u) == 0 && globaltimer() - t0 > lim) {
+    if (globaltimer() - t0 > lim) {
       *abort_flag = 1;
       if (err) atomicOr(err, DEV_ERR_TIMEOUT);
       return false;
@@ -368,6 +382,17 @@ DEVI void cluster_sync_all() {
 DEVI void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+DEVI bool mbar_try_wait_cluster_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
 DEVI bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
@@ -383,11 +408,10 @@ DEVI bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
 DEVI bool mbar_wait_bounded_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer(), lim = g_wait_limit_ns;
-  uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (mbar_try_wait_cluster_sleep(bar, parity, WAIT_SLEEP_NS)) return true;
     if (*abort_flag) return false;
-    if ((++spins & 63u) == 0 && globaltimer() - t0 > lim) {
+    if (globaltimer() - t0 > lim) {
       *abort_flag = 1;
       if (err) atomicOr(err, DEV_ERR_TIMEOUT);
       return false;
