@@ -586,23 +586,59 @@ __global__ void reduce_rows_kernel(const float* part, int nrows, int n, float* _
 }
 
 // The same reduction for up to MAX_REDUCE_JOBS (part, grad) pairs in one
-// launch: block b takes 32 columns of the job whose column blocks contain b.
+// launch: block b takes a column block of the job whose column blocks
+// contain b, 128 columns as four per thread (float4) when the job's width is
+// a multiple of 4 and both arrays are 16-byte aligned, else 32 columns.
+// Either way a column's sum runs over the same rows in the same order
+// (thread row group ry takes rows ry, ry + 8, ... ascending, then the eight
+// groups in order), so both forms give the same bits.
 struct ReduceBatchArgs {
   ReduceJob job[MAX_REDUCE_JOBS];
   int start[MAX_REDUCE_JOBS + 1];  // first column block of each job
+  int vec[MAX_REDUCE_JOBS];        // 1: float4 column blocks
   int njobs;
   float beta;
 };
 
+DEVI float4 add4(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+
 __global__ void reduce_rows_batch_kernel(const __grid_constant__ ReduceBatchArgs a) {
   pdl_start();
-  __shared__ float sm[8][33];
+  __shared__ float4 sm4[8][32];
+  float (*sm)[33] = reinterpret_cast<float (*)[33]>(&sm4[0][0]);  // the scalar form's [8][33]
   int jb = 0;
   while (jb + 1 < a.njobs && a.start[jb + 1] <= (int)blockIdx.x) ++jb;
   const float* part = a.job[jb].part;
   float* grad = a.job[jb].grad;
   const int nrows = a.job[jb].nrows, n = a.job[jb].n;
   const int cx = threadIdx.x & 31, ry = threadIdx.x >> 5;
+  if (a.vec[jb]) {
+    const int j = ((int)blockIdx.x - a.start[jb]) * 128 + 4 * cx;  // n % 4 == 0: all four inside or none
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < n) {
+      int r = ry;
+      // four rows in flight, added in row order
+      for (; r + 24 < nrows; r += 32) {
+        const float4 v0 = *reinterpret_cast<const float4*>(part + (long)r * n + j);
+        const float4 v1 = *reinterpret_cast<const float4*>(part + (long)(r + 8) * n + j);
+        const float4 v2 = *reinterpret_cast<const float4*>(part + (long)(r + 16) * n + j);
+        const float4 v3 = *reinterpret_cast<const float4*>(part + (long)(r + 24) * n + j);
+        s = add4(add4(add4(add4(s, v0), v1), v2), v3);
+      }
+      for (; r < nrows; r += 8) s = add4(s, *reinterpret_cast<const float4*>(part + (long)r * n + j));
+    }
+    sm4[ry][cx] = s;
+    __syncthreads();
+    if (ry == 0 && j < n) {
+      float4 t = sm4[0][cx];
+      for (int k = 1; k < 8; ++k) t = add4(t, sm4[k][cx]);
+      float4* g4 = reinterpret_cast<float4*>(grad + j);
+      const float4 old = a.beta != 0.f ? *g4 : make_float4(0.f, 0.f, 0.f, 0.f);
+      *g4 = make_float4((a.beta != 0.f ? a.beta * old.x : 0.f) + t.x, (a.beta != 0.f ? a.beta * old.y : 0.f) + t.y,
+                        (a.beta != 0.f ? a.beta * old.z : 0.f) + t.z, (a.beta != 0.f ? a.beta * old.w : 0.f) + t.w);
+    }
+    return;
+  }
   const int j = ((int)blockIdx.x - a.start[jb]) * 32 + cx;
   float s = 0.f;
   if (j < n)
@@ -1250,9 +1286,12 @@ int reduce_rows_batch(const ReduceJob* jobs, int njobs, float beta, cudaStream_t
     a.beta = beta;
     int blocks = 0;
     for (int k = 0; k < a.njobs; ++k) {
-      a.job[k] = jobs[j0 + k];
+      const ReduceJob& jk = jobs[j0 + k];
+      a.job[k] = jk;
       a.start[k] = blocks;
-      blocks += (jobs[j0 + k].n + 31) / 32;
+      a.vec[k] = jk.n % 4 == 0 && reinterpret_cast<uintptr_t>(jk.part) % 16 == 0 &&
+                 reinterpret_cast<uintptr_t>(jk.grad) % 16 == 0;
+      blocks += a.vec[k] ? (jk.n + 127) / 128 : (jk.n + 31) / 32;
     }
     a.start[a.njobs] = blocks;
     if (blocks == 0) continue;
