@@ -141,6 +141,34 @@ __global__ void wpe_grad_kernel(const T* dx, float* __restrict__ dwpe, int B, in
   dwpe[i] = (accumulate ? dwpe[i] : 0.f) + s;
 }
 
+// The same with one 16-byte chunk of dx per thread and four batch rows'
+// loads in flight (the sum still runs over b in order); for T d a multiple of
+// the chunk and 16-byte aligned dx and dwpe.
+template <typename T>
+__global__ void wpe_grad_vec_kernel(const T* dx, float* __restrict__ dwpe, int B, long tn, int accumulate) {
+  pdl_start();
+  constexpr int VN = Vec<T>::N;
+  const long i = (blockIdx.x * (long)blockDim.x + threadIdx.x) * VN;
+  if (i >= tn) return;
+  float s[VN];
+#pragma unroll
+  for (int j = 0; j < VN; ++j) s[j] = 0.f;
+#pragma unroll 4
+  for (int b = 0; b < B; ++b) {
+    float f[VN];
+    Vec<T>::load(dx + (long)b * tn + i, f);
+#pragma unroll
+    for (int j = 0; j < VN; ++j) s[j] += f[j];
+  }
+#pragma unroll
+  for (int j = 0; j < VN; j += 4) {
+    float4* o = reinterpret_cast<float4*>(dwpe + i + j);
+    const float4 old = accumulate ? *o : make_float4(0.f, 0.f, 0.f, 0.f);
+    *o = make_float4((accumulate ? old.x : 0.f) + s[j], (accumulate ? old.y : 0.f) + s[j + 1],
+                     (accumulate ? old.z : 0.f) + s[j + 2], (accumulate ? old.w : 0.f) + s[j + 3]);
+  }
+}
+
 // ------------------------------------------------------------- LayerNorm --
 // y = (x - mean) * rstd * g + b, mean/var over the row, var biased, eps 1e-5.
 // One warp per row; NC = 16-byte chunks per lane (row cached in registers).
@@ -870,7 +898,10 @@ __global__ void __launch_bounds__(256) ce_merge_kernel(const float* pm, const fl
   const int m = blockIdx.x * 32 + lane;
   const bool in = m < M;
   float mx = -INFINITY;
+  // (four parts' loads in flight; the running maximum and, below, the sum
+  // take the parts in the same order as a plain loop)
   if (in)
+#pragma unroll 4
     for (int p = warp; p < P; p += 8) mx = fmaxf(mx, pm[(long)p * M + m]);
   red[warp][lane] = mx;
   __syncthreads();
@@ -880,6 +911,7 @@ __global__ void __launch_bounds__(256) ce_merge_kernel(const float* pm, const fl
   __syncthreads();
   float sum = 0.f;
   if (in)
+#pragma unroll 4
     for (int p = warp; p < P; p += 8) {
       const long i = (long)p * M + m;
       sum += ps[i] * ex2_approx((pm[i] - gm) * L2E);
@@ -1368,7 +1400,16 @@ int embed_bwd(int f32, const int32_t* tok, const void* dx, float* dwte, float* d
   LAUNCH_CHECK();
   const long tn = (long)T * d;
   const int B = M / T;
-  if (f32)
+  const int vn = f32 ? 4 : 8;
+  const bool vec = tn % vn == 0 && reinterpret_cast<uintptr_t>(dx) % 16 == 0 &&
+                   reinterpret_cast<uintptr_t>(dwpe) % 16 == 0;
+  if (vec && f32)
+    CUDA_TRY(launch_k(wpe_grad_vec_kernel<float>, (unsigned)((tn / vn + 255) / 256), 256, 0, st,
+        (const float*)dx, dwpe, B, tn, wpe_accumulate));
+  else if (vec)
+    CUDA_TRY(launch_k(wpe_grad_vec_kernel<bf16>, (unsigned)((tn / vn + 255) / 256), 256, 0, st,
+        (const bf16*)dx, dwpe, B, tn, wpe_accumulate));
+  else if (f32)
     CUDA_TRY(launch_k(wpe_grad_kernel<float>, (unsigned)((tn + 255) / 256), 256, 0, st,
         (const float*)dx, dwpe, B, T, d, wpe_accumulate));
   else
