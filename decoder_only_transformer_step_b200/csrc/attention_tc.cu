@@ -1423,14 +1423,7 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
             const float2 x23 = __ffma2_rn(
                 make_float2(__uint_as_float(sv[0][i + 2]), __uint_as_float(sv[0][i + 3])), sc2,
                 make_float2(l4.z, l4.w));
-            float pv[4] = {ex2(x01.x), ex2(x01.y), ex2(x23.x), ex2(x23.y)};
-            if (need_mask) {
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int qq = q0 + c0 + i + u;
-                if (qq < kv || qq >= T || kv >= T) pv[u] = 0.f;
-              }
-            }
+            const float pv[4] = {ex2(x01.x), ex2(x01.y), ex2(x23.x), ex2(x23.y)};
             const float2 e01 = __fadd2_rn(make_float2(__uint_as_float(dp[0][i]), __uint_as_float(dp[0][i + 1])),
                                           make_float2(d4.x, d4.y));
             const float2 e23 = __fadd2_rn(
@@ -1442,6 +1435,21 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
             pp[sub * 16 + i / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
             pd[sub * 16 + i / 2] = pack_bf16x2(g01.x, g01.y);
             pd[sub * 16 + i / 2 + 1] = pack_bf16x2(g23.x, g23.y);
+          }
+        }
+        if (need_mask) {
+          // the causal and ragged masks: the packed P and dS words of masked
+          // columns (two columns a word) cleared after the fact, so that the
+          // unrolled loop above carries no mask code.  Column c of this
+          // half (query q0 + 64 half + c) stays iff lo <= c < hi.
+          const int lo = kv - (q0 + 64 * half);
+          const int hi = kv < T ? T - (q0 + 64 * half) : lo;
+#pragma unroll
+          for (int w = 0; w < 32; ++w) {
+            const uint32_t m = (2 * w >= lo && 2 * w < hi ? 0x0000ffffu : 0u) |
+                               (2 * w + 1 >= lo && 2 * w + 1 < hi ? 0xffff0000u : 0u);
+            pp[w] &= m;
+            pd[w] &= m;
           }
         }
         // every lane has read this block's LSE / D
