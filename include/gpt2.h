@@ -322,10 +322,10 @@ int gpt2_op_attention_bwd_bf16(const uint16_t* qkv, const uint16_t* o, const flo
  * gpt2_get_status reads, or the status argument of gpt2_op_gemm_bf16_status),
  * lets the copies and MMAs already in flight finish, frees its tensor memory
  * and returns, so the context stays usable.  This sets the limit in
- * nanoseconds on the current device (0 restores the default of 2 s).  The
- * survey's failure-detection item: a hung pipeline becomes an error the host
- * reads instead of a hung GPU.  Not stream-ordered: call it with no kernel of
- * the library in flight. */
+ * nanoseconds on the current device (0 restores the default of 2 s).  This
+ * is the library's failure detection: a hung pipeline becomes an error the
+ * host reads instead of a hung GPU.  Not stream-ordered: call it with no
+ * kernel of the library in flight. */
 int gpt2_set_wait_timeout_ns(uint64_t ns);
 
 /* gpt2_op_gemm_bf16 with a device status word: status (device int, 4-byte
